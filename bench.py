@@ -1,0 +1,415 @@
+"""Throughput of the LIME hot path on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload standard]
+    python bench.py --impl reference ...      # the fp64 CPU oracle on host cores
+
+A step is one pass of the whole hot path over one batch of synthetic input of
+the named workload (default: 64 users x 1,024 history tokens, 32 links, d=128,
+4 heads, 2 LIME-XOR layers, a 1,000,000-item catalogue, 1,024 Zipf(1.1)
+candidates per user): context links, the LIME-XOR layers, the QK-cache build
+over the whole catalogue, and cached scoring of every candidate.  The metric
+is user-candidate pairs scored per second of step time; per-phase throughputs
+(history tokens/s through the XOR layers, items/s of the cache build, pairs/s
+of scoring alone) ride along.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
+device synchronize on both sides.  Before every step a 512 MB buffer is
+written to flush the 126 MB L2 (outside the step's events).  Step and phase
+times come from CUDA events on the launching stream; the job time is the max
+over ranks.  With N > 1 each rank runs an independent replica of the step
+(users and catalogue rows are independent; no collective on the data path),
+so scaling is weak.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+# Per-launch DRAM traffic of the dominant kernel from the committed ncu
+# summaries under profiles/ (bytes read + written per launch); None until a
+# capture of the current kernel exists.
+NCU_TRAFFIC = {}
+
+
+def env_int(name, default):
+    v = os.environ.get(name)
+    return int(v) if v not in (None, "") else default
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                    source="fallback")
+
+
+# --------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Polls NVML for the SM clock and the clock-event reasons while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # no NVML: clocks are reported as null
+            self.ok = False
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "reasons": names}
+
+
+# ------------------------------------------------------- algorithmic work
+
+def work_units(w, total_hist, total_cand):
+    """Algorithmic flops / bytes per phase of one step (see the design notes)."""
+    d, l, f, H = w.d, w.l, w.f, w.H
+    es = 2 if w.dtype == "bf16" else 4
+    n_mid = w.layers - 1
+    flops_tok_mid = 2 * (3 * d * d + d * d + 3 * d * f + 4 * l * d)   # QKV, O, GatedMLP, attention
+    flops_tok_last = 2 * (2 * d * d + 2 * l * d)                       # K,V of history + link branch
+    user_flops = total_hist * (n_mid * flops_tok_mid + flops_tok_last)
+    user_bytes = total_hist * d * es * (2 * n_mid + 1)
+    cache_bytes = w.n_items * (d + H * l) * es
+    cache_flops = w.n_items * 2 * d * H * l
+    score_bytes = total_cand * (H * l * es + 4 + d * es)
+    score_flops = total_cand * 2 * l * d
+    return dict(user=(user_flops, user_bytes), cache=(cache_flops, cache_bytes),
+                score=(score_flops, score_bytes))
+
+
+# --------------------------------------------------------------- oracle
+
+def oracle_step_seconds(w, us, cs, n_users=4, n_items=65536, seed=0):
+    """Time the fp64 oracle on a bounded sample of one step and extrapolate
+    linearly to the whole step (the work is linear in users, items and
+    candidate pairs).  Returns (seconds per full step, sample description)."""
+    import numpy as np
+    from oracle import lime_oracle as O
+    from recsys_decoupled_link_b200 import synth
+    f = synth.to_f64
+    g = torch.Generator().manual_seed(seed)
+    users = sorted(torch.randperm(w.B, generator=g)[:n_users].tolist())
+    layers = [{k: f(v) for k, v in lw.as_dict().items()} for lw in us.layers]
+    offs = us.hist_offsets.numpy()
+    t0 = time.perf_counter()
+    if w.c > 0:
+        Z0 = np.zeros((w.B, w.l, w.d))
+        for u in users:
+            Z0[u] = O.context_links(f(us.L), f(us.ctx[u]), f(us.ctx_w.Wc1), f(us.ctx_w.bc1),
+                                    f(us.ctx_w.Wc2), f(us.ctx_w.bc2))
+    else:
+        Z0 = np.broadcast_to(f(us.L), (w.B, w.l, w.d)).copy()
+    _, LP = O.user_encode(f(us.E), offs, Z0, layers, w.H, users=users)
+    t_user = time.perf_counter() - t0
+    rows = torch.randint(0, w.n_items, (n_items,), generator=g)
+    Trows = f(synth.item_rows(w, rows))
+    t0 = time.perf_counter()
+    O.qk_cache(Trows, f(us.L), f(cs.Wq_c), f(cs.Wk_c), w.H)
+    t_cache = time.perf_counter() - t0
+    co = cs.cand_offsets.numpy()
+    pairs = sum(int(co[u + 1] - co[u]) for u in users)
+    ids = np.concatenate([cs.cand_ids.numpy()[co[u]:co[u + 1]] for u in users])
+    uniq, inv = np.unique(ids, return_inverse=True)
+    small_cache = O.qk_cache(f(synth.item_rows(w, torch.from_numpy(uniq.astype(np.int64)))),
+                             f(us.L), f(cs.Wq_c), f(cs.Wk_c), w.H)
+    sub_offs = [0]
+    for u in users:
+        sub_offs.append(sub_offs[-1] + int(co[u + 1] - co[u]))
+    LP_sub = LP[users]
+    t0 = time.perf_counter()
+    O.score_candidates(small_cache, inv, sub_offs, LP_sub)
+    t_score = time.perf_counter() - t0
+    total_cand = int(co[-1])
+    est = (t_user / len(users) * w.B + t_cache / n_items * w.n_items +
+           (t_score / max(pairs, 1)) * total_cand)
+    sample = (f"{len(users)} of {w.B} users (context links + {w.layers} layers), "
+              f"{n_items} of {w.n_items} catalogue rows, the sampled users' {pairs} candidates; "
+              f"extrapolated linearly to the full step")
+    return est, sample, t_user + t_cache + t_score
+
+
+def blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = [i.get("num_threads") for i in info if i.get("user_api") == "blas"]
+        if n:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    from recsys_decoupled_link_b200 import synth
+    w = synth.workload(args.workload)
+    us = synth.user_side(w)
+    cs = synth.candidate_side(w)
+    total_cand = int(cs.cand_offsets[-1])
+    for _ in range(args.warmup):
+        oracle_step_seconds(w, us, cs, n_users=1, n_items=8192)
+    ests, sample = [], ""
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        est, sample, _ = oracle_step_seconds(w, us, cs, n_users=2, n_items=16384, seed=k)
+        ests.append(est)
+    wall = time.perf_counter() - t0
+    sec = statistics.mean(ests)
+    value = total_cand / sec
+    line = {"impl": "reference", "metric": "user-candidate pairs scored/s (full LIME step)",
+            "value": value, "unit": "pairs/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, total_cand),
+            "cpu_baseline": {"value": value, "unit": "pairs/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample + f"; {args.steps} samples, "
+                             f"{wall:.1f} s of CPU time"},
+            "e2e": {"value": value, "unit": "pairs/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, total_cand, total_hist=None):
+    c = {"workload": f"{w.name}: B={w.B} users, N={w.N} history, l={w.l} links, d={w.d}, "
+                     f"H={w.H}, {w.layers} LIME-XOR layers, context dim {w.c}, "
+                     f"{w.n_items} items, M={w.M} candidates ({w.cand[0]}"
+                     f"{'' if len(w.cand) == 1 else ' ' + str(w.cand[1])})",
+         "pairs_per_step": total_cand, "l2": "flushed before every step (512 MB write)"}
+    if total_hist is not None:
+        c["history_tokens_per_step"] = total_hist
+    return c
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lime", choices=["lime", "reference"])
+    ap.add_argument("--workload", default="standard")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank, world = env_int("RANK", 0), env_int("WORLD_SIZE", 1)
+    local = env_int("LOCAL_RANK", 0)
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    from recsys_decoupled_link_b200 import lime, pipeline, synth
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    w = synth.workload(args.workload)
+    us = synth.user_side(w)
+    cs = synth.candidate_side(w)
+    T = synth.item_table(w)
+    x = pipeline.to_device(w, us, cs, T)
+    buf = pipeline.alloc(x)
+    total_cand, total_hist = x.total_cand, x.total_hist
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step_events():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        pipeline.step(x, buf)
+    torch.cuda.synchronize()
+    if lime.lime_get_status(buf.ws) != 0:
+        raise RuntimeError("device status flags set during warm-up")
+
+    evs = [step_events() for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    launches0 = lime.lime_launch_count()
+    with sampler:
+        for k in range(args.steps):
+            flush.zero_()
+            e = evs[k]
+            e[0].record(stream)
+            LP = pipeline.user_encode(x, buf)
+            e[1].record(stream)
+            pipeline.build_cache(x, buf)
+            e[2].record(stream)
+            pipeline.score(x, buf, LP)
+            e[3].record(stream)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+    t_wall = time.perf_counter() - t_wall
+    launches = lime.lime_launch_count() - launches0
+    ph = {"user": 0.0, "cache": 0.0, "score": 0.0}
+    total_ms = 0.0
+    for e in evs:
+        ph["user"] += e[0].elapsed_time(e[1])
+        ph["cache"] += e[1].elapsed_time(e[2])
+        ph["score"] += e[2].elapsed_time(e[3])
+        total_ms += e[0].elapsed_time(e[3])
+    t_dev = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+    if dist:
+        dist.all_reduce(t_dev, op=dist.ReduceOp.MAX)
+    total_ms = float(t_dev.item())
+    ms_step = total_ms / args.steps
+    value = world * total_cand / (ms_step * 1e-3)
+
+    # end to end through the public API: pinned host inputs in, scores out
+    host = {"E": x.E.cpu().pin_memory(), "ctx": x.ctx.cpu().pin_memory() if x.ctx is not None else None,
+            "hist_offsets": x.hist_offsets.cpu().pin_memory(), "T": x.T.cpu().pin_memory(),
+            "cand_ids": x.cand_ids.cpu().pin_memory(),
+            "cand_offsets": x.cand_offsets.cpu().pin_memory()}
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    O_host = torch.empty(buf.O.shape, dtype=buf.O.dtype).pin_memory()
+    d2h = O_host.numel() * O_host.element_size()
+    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+
+    def e2e_step():
+        for k, t in host.items():
+            if t is not None:
+                getattr(x, k).copy_(t, non_blocking=True)
+        out = pipeline.step(x, buf)
+        O_host.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    for k in range(args.steps):
+        flush.zero_()
+        ee[k][0].record(stream)
+        e2e_step()
+        ee[k][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in ee)], dtype=torch.float64,
+                          device="cuda")
+    if dist:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_step_ms = float(e2e_ms.item()) / args.steps
+    if lime.lime_get_status(buf.ws) != 0:
+        raise RuntimeError("device status flags set during the timed steps")
+
+    if rank == 0:
+        pk = peaks()
+        work = work_units(w, total_hist, total_cand)
+        phase_ms = {k: v / args.steps for k, v in ph.items()}
+        dom = max(phase_ms, key=phase_ms.get)
+        fl, by = work[dom]
+        sec = phase_ms[dom] * 1e-3
+        if dom == "user" and w.dtype == "bf16":
+            roof = {"bound": "tensor", "achieved": fl / sec / 1e12, "peak": pk["bf16_tflops"],
+                    "unit": "TFLOP/s"}
+        else:
+            roof = {"bound": "hbm", "achieved": by / sec / 1e9, "peak": pk["hbm_gbs"],
+                    "unit": "GB/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = NCU_TRAFFIC.get(dom)
+        roof["kernel"] = {"user": "context links + LIME-XOR layers", "cache": "QK-cache build",
+                          "score": "candidate scoring"}[dom]
+        roof["peak_source"] = pk["source"]
+        phases = {
+            "user_encode": {"ms": phase_ms["user"],
+                            "history_tokens_per_s": total_hist / (phase_ms["user"] * 1e-3),
+                            "tflops": work["user"][0] / (phase_ms["user"] * 1e-3) / 1e12},
+            "qk_cache": {"ms": phase_ms["cache"],
+                         "items_per_s": w.n_items / (phase_ms["cache"] * 1e-3),
+                         "gbs": work["cache"][1] / (phase_ms["cache"] * 1e-3) / 1e9},
+            "score": {"ms": phase_ms["score"],
+                      "pairs_per_s": total_cand / (phase_ms["score"] * 1e-3),
+                      "gbs": work["score"][1] / (phase_ms["score"] * 1e-3) / 1e9},
+        }
+        line = {"metric": "user-candidate pairs scored/s (full LIME step)", "value": value,
+                "unit": "pairs/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+                "data": "synthetic (seeded; shapes of the pages' workloads)",
+                "config": config_of(w, total_cand, total_hist),
+                "phases": phases, "roofline": roof,
+                "clocks": sampler.summary(),
+                "e2e": {"value": world * total_cand / (e2e_step_ms * 1e-3), "unit": "pairs/s",
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                        "note": "inputs (history, context, offsets, item table, candidate IDs) "
+                                "copied from pinned host memory and scores copied back inside "
+                                "each timed step; weights stay resident"},
+                "gpu_launches": launches, "wall_s_timed": t_wall}
+        if world == 1 and not args.no_cpu_baseline:
+            est, sample, cpu_s = oracle_step_seconds(w, us, cs, n_users=8, n_items=131072)
+            line["cpu_baseline"] = {"value": total_cand / est, "unit": "pairs/s",
+                                    "cores": blas_threads(), "kind": "oracle",
+                                    "sample": sample + f" ({cpu_s:.1f} s of CPU time)"}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

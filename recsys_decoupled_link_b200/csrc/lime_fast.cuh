@@ -1,0 +1,24 @@
+// Tensor-core (tcgen05) and vectorised bf16 kernels of the LIME hot path.
+#pragma once
+#include "lime_common.cuh"
+
+namespace lime {
+
+size_t fast_ws_bytes(const lime_dims& D, int64_t B, int64_t total_hist);
+
+bool fast_cache_supported(const lime_dims& D);
+int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void* L,
+                        const void* Wq, const void* Wk, void* cache, float* ws,
+                        unsigned* status, cudaStream_t st);
+
+bool fast_score_supported(const lime_dims& D);
+int fast_score(const lime_dims& D, int64_t B, const void* cache, int64_t n_items,
+               const int32_t* ids, const int64_t* off, int64_t total, const void* LP, void* O,
+               float* ws, unsigned* status, cudaStream_t st);
+
+bool fast_layer_supported(const lime_dims& D);
+int fast_xor_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh,
+                   const void* E_in, const void* Z_in, const lime_layer_w& w, void* E_out,
+                   void* Z_out, float* ws, unsigned* status, cudaStream_t st);
+
+}  // namespace lime

@@ -1,0 +1,116 @@
+"""One pass of the LIME hot path through the C ABI, for a synthetic workload.
+
+Plumbing only: it moves the seeded inputs of ``synth`` to the device and calls
+the library in the order the method runs them (LIME note, 整体框架 and
+一个完整示例): context links, the LIME-XOR layer stack (the last layer marked
+by E_out = NULL), the QK-cache build over the catalogue, and cached candidate
+scoring.  All arithmetic happens inside liblime.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional
+
+import torch
+
+from . import lime, synth
+
+
+@dataclasses.dataclass
+class DeviceInputs:
+    w: synth.Workload
+    dims: lime.lime_dims
+    L: torch.Tensor
+    Z0: Optional[torch.Tensor]          # [B, l, d] when there is no context MLP (L^C = L)
+    ctx: Optional[torch.Tensor]
+    ctx_w: Optional[List[torch.Tensor]]
+    layers: List[lime.lime_layer_w]
+    layer_tensors: List[List[torch.Tensor]]
+    E: torch.Tensor
+    hist_offsets: torch.Tensor
+    total_hist: int
+    T: Optional[torch.Tensor]
+    Wq_c: torch.Tensor
+    Wk_c: torch.Tensor
+    cand_ids: torch.Tensor
+    cand_offsets: torch.Tensor
+    total_cand: int
+
+
+@dataclasses.dataclass
+class Buffers:
+    LC: torch.Tensor
+    E_bufs: List[torch.Tensor]
+    Z_bufs: List[torch.Tensor]
+    cache: torch.Tensor
+    O: torch.Tensor
+    ws: lime.Workspace
+
+
+def to_device(w: synth.Workload, us: synth.UserSide, cs: synth.CandidateSide,
+              T: Optional[torch.Tensor], device="cuda") -> DeviceInputs:
+    dev = lambda t: None if t is None else t.to(device).contiguous()
+    dims = lime.make_dims(w.d, w.H, w.l, w.f, w.c, w.dtype)
+    layer_tensors = [[dev(t) for t in lw.as_dict().values()] for lw in us.layers]
+    if w.c > 0:
+        ctx_w = [dev(us.ctx_w.Wc1), dev(us.ctx_w.bc1), dev(us.ctx_w.Wc2), dev(us.ctx_w.bc2)]
+        Z0 = None
+    else:
+        ctx_w = None
+        Z0 = dev(us.L).unsqueeze(0).expand(w.B, w.l, w.d).contiguous()
+    return DeviceInputs(
+        w=w, dims=dims, L=dev(us.L), Z0=Z0, ctx=dev(us.ctx), ctx_w=ctx_w,
+        layers=[lime.layer_struct(ts) for ts in layer_tensors], layer_tensors=layer_tensors,
+        E=dev(us.E), hist_offsets=dev(us.hist_offsets), total_hist=int(us.hist_offsets[-1]),
+        T=dev(T), Wq_c=dev(cs.Wq_c), Wk_c=dev(cs.Wk_c), cand_ids=dev(cs.cand_ids),
+        cand_offsets=dev(cs.cand_offsets), total_cand=int(cs.cand_offsets[-1]))
+
+
+def alloc(x: DeviceInputs, n_items: Optional[int] = None, device="cuda") -> Buffers:
+    w = x.w
+    dt = synth.torch_dtype(w)
+    n_items = w.n_items if n_items is None else n_items
+    nbuf = 2 if w.layers > 1 else 1
+    return Buffers(
+        LC=torch.empty(w.B, w.l, w.d, dtype=dt, device=device),
+        E_bufs=[torch.empty(x.total_hist, w.d, dtype=dt, device=device) for _ in range(nbuf)],
+        Z_bufs=[torch.empty(w.B, w.l, w.d, dtype=dt, device=device) for _ in range(2)],
+        cache=torch.empty(n_items, w.H, w.l, dtype=dt, device=device),
+        O=torch.empty(x.total_cand, w.d, dtype=dt, device=device),
+        ws=lime.Workspace(x.dims, w.B, x.total_hist, device=device))
+
+
+def user_encode(x: DeviceInputs, buf: Buffers, stream=None) -> torch.Tensor:
+    """Context links then the layer stack; returns L^P [B, l, d]."""
+    if x.ctx_w is not None:
+        lime.lime_context_links(x.dims, x.L, x.ctx, *x.ctx_w, buf.LC, stream=stream)
+        Z = buf.LC
+    else:
+        Z = x.Z0
+    E = x.E
+    n = len(x.layers)
+    for i, lw in enumerate(x.layers):
+        last = i == n - 1
+        E_out = None if last else buf.E_bufs[i % len(buf.E_bufs)]
+        Z_out = buf.Z_bufs[i % 2]
+        lime.lime_xor_layer(x.dims, x.hist_offsets, x.total_hist, E, Z, lw, E_out, Z_out,
+                            buf.ws, stream=stream)
+        E, Z = E_out, Z_out
+    return Z
+
+
+def build_cache(x: DeviceInputs, buf: Buffers, stream=None):
+    lime.lime_build_qk_cache(x.dims, x.T, x.L, x.Wq_c, x.Wk_c, buf.cache, buf.ws, stream=stream)
+
+
+def score(x: DeviceInputs, buf: Buffers, LP: torch.Tensor, stream=None):
+    lime.lime_score_candidates(x.dims, buf.cache, x.cand_ids, x.cand_offsets, x.total_cand, LP,
+                               buf.O, buf.ws, stream=stream)
+
+
+def step(x: DeviceInputs, buf: Buffers, stream=None) -> torch.Tensor:
+    """One pass of the whole hot path; returns O [sum M, d]."""
+    LP = user_encode(x, buf, stream)
+    build_cache(x, buf, stream)
+    score(x, buf, LP, stream)
+    return buf.O

@@ -1,0 +1,106 @@
+"""CPU-only checks of the C ABI: the library builds, loads and exports every
+function include/lime.h declares, and host-side argument validation rejects bad
+calls before anything reaches the device (these calls return before any CUDA
+API call, so they run without a GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from recsys_decoupled_link_b200 import build as lime_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lime():
+    lime_build.build()
+    from recsys_decoupled_link_b200 import lime as m
+    return m
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "lime.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|uint64_t)\s+(lime_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    assert declared_functions() == sorted([
+        "lime_workspace_bytes", "lime_workspace_init", "lime_build_qk_cache",
+        "lime_context_links", "lime_xor_layer", "lime_score_candidates", "lime_get_status",
+        "lime_launch_count"])
+
+
+def test_library_exports_every_declared_symbol(lime):
+    out = subprocess.run(["nm", "-D", "--defined-only", lime.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s+(lime_\w+)$", out, re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert name in lime.EXPORTED
+    assert not [s for s in exported if not s.startswith("lime_")]
+
+
+def test_header_compiles_as_c():
+    src = '#include "lime.h"\nint main(void){ lime_dims d = {128,4,32,256,64,LIME_BF16};' \
+          ' return (int)lime_workspace_bytes(&d, 1, 1) == 0; }\n'
+    r = subprocess.run(["gcc", "-std=c99", "-fsyntax-only", "-x", "c", "-",
+                        "-I", os.path.join(ROOT, "include"), "-I", "/usr/local/cuda/include"],
+                       input=src, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
+def test_workspace_bytes(lime):
+    d = lime.make_dims(128, 4, 32, 256, 64, "bf16")
+    small = lime.lime_workspace_bytes(d, 1, 10)
+    big = lime.lime_workspace_bytes(d, 64, 65536)
+    assert 256 < small <= big
+    assert lime.lime_workspace_bytes(lime.make_dims(128, 3, 32, 256, 64, "bf16"), 1, 1) == 0
+    assert lime.lime_workspace_bytes(lime.make_dims(128, 4, 200, 256, 64, "bf16"), 1, 1) == 0
+    assert lime.lime_workspace_bytes(lime.lime_dims(128, 4, 32, 256, 64, 7), 1, 1) == 0
+    assert lime.lime_workspace_bytes(d, -1, 1) == 0
+
+
+def _call_layer(lime, dims, B=2, total=10, E_in=0x10000, Z_in=0x20000, E_out=0x30000,
+                Z_out=0x40000, ws=0x100000, ws_bytes=None, offs=0x50000, weights=0x60000):
+    w = lime.lime_layer_w(*([weights] * 11))
+    if ws_bytes is None:
+        ws_bytes = lime.lime_workspace_bytes(dims, B, total)
+    return lime._lib.lime_xor_layer(ctypes.byref(dims), B, offs, total, E_in, Z_in,
+                                    ctypes.byref(w), E_out, Z_out, ws, ws_bytes, None)
+
+
+def test_host_validation_of_layer_calls(lime):
+    dims = lime.make_dims(128, 4, 32, 256, 64, "bf16")
+    assert _call_layer(lime, dims, Z_in=None) == lime.LIME_ERR_ARG
+    assert _call_layer(lime, dims, weights=0x60008) == lime.LIME_ERR_ARG       # unaligned
+    assert _call_layer(lime, dims, ws=0x100010) == lime.LIME_ERR_ARG           # ws unaligned
+    assert _call_layer(lime, dims, ws_bytes=512) == lime.LIME_ERR_ARG          # ws too small
+    assert _call_layer(lime, dims, E_out=0x10000) == lime.LIME_ERR_ALIAS       # E_out == E_in
+    assert _call_layer(lime, dims, Z_out=0x20000 + 64) == lime.LIME_ERR_ALIAS  # overlap
+    bad = lime.make_dims(128, 4, 129, 256, 64, "bf16")
+    assert _call_layer(lime, bad) == lime.LIME_ERR_SHAPE
+    assert _call_layer(lime, dims, B=-1) == lime.LIME_ERR_ARG
+
+
+def test_host_validation_of_scoring_and_cache(lime):
+    dims = lime.make_dims(128, 4, 32, 256, 64, "bf16")
+    nws = lime.lime_workspace_bytes(dims, 0, 0)
+    f = lime._lib.lime_score_candidates
+    # O_out overlapping the cache
+    assert f(ctypes.byref(dims), 1, 0x100000, 100, 0x200000, 0x300000, 5, 0x400000,
+             0x100000 + 256, 0x1000000, nws, None) == lime.LIME_ERR_ALIAS
+    assert f(ctypes.byref(dims), 1, 0x100000, 100, 0x200000, None, 5, 0x400000,
+             0x500000, 0x1000000, nws, None) == lime.LIME_ERR_ARG
+    g = lime._lib.lime_build_qk_cache
+    assert g(ctypes.byref(dims), 0x100000, 10, 0x200000, 0x300000, 0x400000, 0x100000,
+             0x1000000, nws, None) == lime.LIME_ERR_ALIAS
+    assert g(ctypes.byref(dims), 0x100000, 10, None, 0x300000, 0x400000, 0x500000,
+             0x1000000, nws, None) == lime.LIME_ERR_ARG
+    c = lime._lib.lime_context_links
+    nodims = lime.make_dims(128, 4, 32, 256, 0, "bf16")
+    mlp = lime.lime_ctx_mlp(0x10000, 0x20000, 0x30000, 0x40000)
+    assert c(ctypes.byref(nodims), 2, 0x50000, 0x60000, ctypes.byref(mlp), 0x70000,
+             None) == lime.LIME_ERR_SHAPE

@@ -1,0 +1,268 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Each case runs the library on seeded synthetic inputs and the oracle on the
+same values widened to float64.  Layer outputs are checked both in isolation
+(the oracle's layer fed the GPU's previous-layer output) and end to end;
+scoring is checked in isolation (GPU cache and L^P fed to the oracle) and end
+to end (the oracle's own cache and L^P).  Tolerances: bf16 storage max-abs
+<= 2e-2 and rel-L2 <= 5e-3; fp32 <= 1e-4; candidate gathers bit-exact.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import lime_oracle as O
+from recsys_decoupled_link_b200 import lime, pipeline, synth
+from parity_util import assert_close, f64, oracle_layer_weights, oracle_Z0
+
+pytestmark = pytest.mark.gpu
+
+
+def run_user_side(x, buf):
+    """Context links + layers through the C ABI; returns Z0 and per-layer (E', Z')."""
+    if x.ctx_w is not None:
+        lime.lime_context_links(x.dims, x.L, x.ctx, *x.ctx_w, buf.LC)
+        Z = buf.LC.clone()
+    else:
+        Z = x.Z0
+    Z0 = Z
+    E = x.E
+    outs = []
+    for i, lw in enumerate(x.layers):
+        last = i == len(x.layers) - 1
+        E_out = None if last else torch.empty_like(x.E)
+        Z_out = torch.empty_like(Z)
+        lime.lime_xor_layer(x.dims, x.hist_offsets, x.total_hist, E, Z, lw, E_out, Z_out, buf.ws)
+        outs.append((E_out, Z_out))
+        E, Z = E_out, Z_out
+    torch.cuda.synchronize()
+    return Z0, outs
+
+
+def check_workload(w, n_hist=None, n_cand=None, check_e2e=True):
+    us = synth.user_side(w, n_hist)
+    cs = synth.candidate_side(w, n_cand)
+    T = synth.item_table(w)
+    x = pipeline.to_device(w, us, cs, T)
+    buf = pipeline.alloc(x)
+    Z0_gpu, outs = run_user_side(x, buf)
+    pipeline.build_cache(x, buf)
+    LP_gpu = outs[-1][1]
+    pipeline.score(x, buf, LP_gpu)
+    torch.cuda.synchronize()
+    assert lime.lime_get_status(buf.ws) == 0
+    dt = w.dtype
+    offs = us.hist_offsets.numpy()
+    layers = oracle_layer_weights(us)
+    # context links
+    Z0_ref = oracle_Z0(w, us)
+    assert_close(Z0_gpu, Z0_ref, dt, "context links")
+    # each layer in isolation
+    E_prev, Z_prev = f64(us.E), f64(Z0_gpu)
+    for i, (E_out, Z_out) in enumerate(outs):
+        E_ref, Z_ref = O.xor_layer(E_prev, offs, Z_prev, layers[i], w.H)
+        assert_close(Z_out, Z_ref, dt, f"layer {i} links")
+        if E_out is not None:
+            assert_close(E_out, E_ref, dt, f"layer {i} history")
+            E_prev = f64(E_out)
+        Z_prev = f64(Z_out)
+    # end to end user side: a chain of the context-link and layer stores
+    chain = w.layers + (1 if w.c > 0 else 0)
+    _, LP_ref = O.user_encode(f64(us.E), offs, Z0_ref, layers, w.H)
+    if check_e2e:
+        assert_close(LP_gpu, LP_ref, dt, "L^P end to end", stages=chain)
+    # cache
+    cache_ref = O.qk_cache(f64(T), f64(us.L), f64(cs.Wq_c), f64(cs.Wk_c), w.H)
+    assert_close(buf.cache, cache_ref, dt, "QK cache")
+    # scoring, isolated and end to end
+    O_iso = O.score_candidates(f64(buf.cache), cs.cand_ids.numpy(), cs.cand_offsets.numpy(),
+                               f64(LP_gpu))
+    assert_close(buf.O, O_iso, dt, "scoring (GPU cache and L^P)")
+    if check_e2e:
+        O_e2e = O.score_candidates(cache_ref, cs.cand_ids.numpy(), cs.cand_offsets.numpy(), LP_ref)
+        assert_close(buf.O, O_e2e, dt, "scoring end to end", stages=chain + 2)
+
+
+SMALL = {
+    "tiny": dict(),
+    "standard": dict(B=3, n_items=200_000),
+    "long": dict(B=2, N=4100, n_items=100_000),
+    "large_cand": dict(B=2, n_items=300_000, M=8192),
+    "ragged16": dict(B=5, l=16, n_items=100_000),
+    "ragged32": dict(B=5, l=32, n_items=100_000),
+    "ragged64": dict(B=5, l=64, n_items=100_000),
+}
+
+
+@pytest.mark.parametrize("case", list(SMALL))
+def test_workload_parity(case):
+    base = "ragged" if case.startswith("ragged") else case
+    check_workload(synth.workload(base, **SMALL[case]))
+
+
+@pytest.mark.parametrize("base", ["tiny", "standard"])
+def test_edge_cases(base):
+    # empty histories, one-row history, exact tiles and ragged tails; users with
+    # no candidates; the batch starts and ends with edge users
+    n_hist = [0, 1, 127, 128, 129, 300, 0]
+    n_cand = [5, 0, 1, 130, 7, 0, 3]
+    w = synth.workload(base, B=len(n_hist), n_items=5000,
+                       cand=("uniform",), layers=2)
+    check_workload(w, n_hist=n_hist, n_cand=n_cand)
+
+
+def test_single_user_single_token():
+    w = synth.workload("standard", B=1, n_items=1000, layers=1)
+    check_workload(w, n_hist=[1], n_cand=[1])
+
+
+def test_gather_is_bit_exact():
+    # d_h = l = 32 and every head slice of L^P equal to I_32: O[m, h*32 + c] is
+    # cache[id_m, h, c] times 1 plus zeros, exact in fp32 and in the bf16 store.
+    d, H, l, n_items, B = 128, 4, 32, 50_000, 3
+    dims = lime.make_dims(d, H, l, 2 * d, 64, "bf16")
+    g = torch.Generator().manual_seed(7)
+    cache = torch.rand(n_items, H, l, generator=g).to(torch.bfloat16).cuda()
+    LP = torch.zeros(B, l, d)
+    for h in range(H):
+        LP[:, :, h * 32:(h + 1) * 32] = torch.eye(32)
+    LP = LP.to(torch.bfloat16).cuda()
+    counts = [1000, 0, 2345]
+    ids = torch.randint(0, n_items, (sum(counts),), generator=g, dtype=torch.int32)
+    offs = synth.offsets(counts)
+    O_gpu = torch.empty(sum(counts), d, dtype=torch.bfloat16, device="cuda")
+    ws = lime.Workspace(dims, B, 0)
+    lime.lime_score_candidates(dims, cache, ids.cuda(), offs.cuda(), sum(counts), LP, O_gpu, ws)
+    torch.cuda.synchronize()
+    expect = cache.cpu()[ids.long()].reshape(-1, d)
+    assert torch.equal(O_gpu.cpu().view(torch.int16), expect.view(torch.int16))
+
+
+def test_bad_candidate_ids_give_zero_rows_and_flag():
+    d, H, l, n_items = 128, 4, 32, 1000
+    for dt in ("bf16", "f32"):
+        tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+        dims = lime.make_dims(d, H, l, 2 * d, 64, dt)
+        c = torch.rand(n_items, H, l)
+        cache = (c / c.sum(-1, keepdim=True)).to(tdt).cuda()   # rows are distributions
+        LP = torch.randn(1, l, d).to(tdt).cuda()
+        ids = torch.tensor([3, n_items, -5, 999, 2**31 - 1], dtype=torch.int32)
+        offs = synth.offsets([5])
+        O_gpu = torch.full((5, d), 7.0, dtype=tdt, device="cuda")
+        ws = lime.Workspace(dims, 1, 0)
+        lime.lime_score_candidates(dims, cache, ids.cuda(), offs.cuda(), 5, LP, O_gpu, ws)
+        assert lime.lime_get_status(ws) == lime.LIME_FLAG_BAD_ID
+        assert lime.lime_get_status(ws) == 0  # read clears
+        out = O_gpu.float().cpu()
+        assert (out[1] == 0).all() and (out[2] == 0).all() and (out[4] == 0).all()
+        ref = O.score_candidates(f64(cache.cpu()), ids.numpy(), [0, 5], f64(LP.cpu()))
+        assert_close(O_gpu, ref, dt, "scores with bad IDs")
+
+
+def test_bad_offsets_are_flagged_and_stay_in_bounds():
+    w = synth.workload("standard", B=3, n_items=1000, layers=1)
+    us = synth.user_side(w, [10, 20, 30])
+    cs = synth.candidate_side(w, [4, 4, 4])
+    x = pipeline.to_device(w, us, cs, synth.item_table(w))
+    buf = pipeline.alloc(x)
+    x.hist_offsets.copy_(torch.tensor([0, 40, 5, 60]))   # not monotone
+    pipeline.user_encode(x, buf)
+    torch.cuda.synchronize()
+    assert lime.lime_get_status(buf.ws) & lime.LIME_FLAG_BAD_OFFSETS
+    x.cand_offsets.copy_(torch.tensor([0, 8, 2, 99]))    # ends past total
+    pipeline.build_cache(x, buf)
+    pipeline.score(x, buf, buf.Z_bufs[0])
+    torch.cuda.synchronize()
+    assert lime.lime_get_status(buf.ws) & lime.LIME_FLAG_BAD_OFFSETS
+
+
+def test_argument_errors():
+    d, H, l = 128, 4, 32
+    dims = lime.make_dims(d, H, l, 2 * d, 64, "bf16")
+    B, N = 2, 64
+    ws = lime.Workspace(dims, B, B * N)
+    E = torch.randn(B * N, d, device="cuda").to(torch.bfloat16)
+    Z = torch.randn(B, l, d, device="cuda").to(torch.bfloat16)
+    offs = torch.tensor([0, N, 2 * N], device="cuda")
+    w = synth.layer_weights(synth.workload("standard"), 0)
+    wt = [t.cuda() for t in w.as_dict().values()]
+    Zo = torch.empty_like(Z)
+    with pytest.raises(lime.LimeError) as e:
+        lime.lime_xor_layer(dims, offs, B * N, E, Z, wt, E, Zo, ws)        # E_out aliases E_in
+    assert e.value.rc == lime.LIME_ERR_ALIAS
+    with pytest.raises(lime.LimeError) as e:
+        lime.lime_xor_layer(dims, offs, B * N, E, Z, wt, None, Z, ws)      # Z_out aliases Z_in
+    assert e.value.rc == lime.LIME_ERR_ALIAS
+    small = lime.Workspace(dims, 1, 1)
+    with pytest.raises(lime.LimeError) as e:
+        lime.lime_xor_layer(dims, offs, B * N, E, Z, wt, None, Zo, small)  # workspace too small
+    assert e.value.rc == lime.LIME_ERR_ARG
+    bad = lime.make_dims(d, 3, l, 2 * d, 64, "bf16")
+    with pytest.raises(lime.LimeError) as e:
+        lime.lime_xor_layer(bad, offs, B * N, E, Z, wt, None, Zo, ws)
+    assert e.value.rc == lime.LIME_ERR_SHAPE
+
+
+# ----------------------------------------------------------- full sizes
+
+def sample_users(counts, k, g):
+    nonempty = [u for u, n in enumerate(counts) if n > 0]
+    longest = max(range(len(counts)), key=lambda u: counts[u])
+    pick = set(torch.randperm(len(nonempty), generator=g)[:k - 1].tolist())
+    return sorted({nonempty[i] for i in pick} | {longest})
+
+
+FULL = ["standard", "long", "large_cand", "ragged16", "ragged32", "ragged64", "tiny"]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("case", FULL)
+def test_full_size_sampled(case):
+    """Full-size workloads in the bench's launch configuration; the oracle
+    checks sampled users end to end, 65,536 sampled cache rows and the sampled
+    users' candidates (isolated)."""
+    base, over = case, {}
+    if case.startswith("ragged"):
+        base, over = "ragged", dict(l=int(case[6:]))
+    w = synth.workload(base, **over)
+    us = synth.user_side(w)
+    cs = synth.candidate_side(w)
+    x = pipeline.to_device(w, us, cs, None)
+    # item table straight to the device block by block (keeps host memory low)
+    dt = synth.torch_dtype(w)
+    x.T = torch.empty(w.n_items, w.d, dtype=dt, device="cuda")
+    nb = (w.n_items + synth.BLOCK_ROWS - 1) // synth.BLOCK_ROWS
+    for b in range(nb):
+        r0 = b * synth.BLOCK_ROWS
+        blk = synth.item_block(w, b)
+        x.T[r0:r0 + blk.shape[0]].copy_(blk)
+    buf = pipeline.alloc(x)
+    LP = pipeline.user_encode(x, buf)
+    pipeline.build_cache(x, buf)
+    pipeline.score(x, buf, LP)
+    torch.cuda.synchronize()
+    assert lime.lime_get_status(buf.ws) == 0
+    g = torch.Generator().manual_seed(99)
+    users = sample_users(us.n_hist, 3, g)
+    offs = us.hist_offsets.numpy()
+    layers = oracle_layer_weights(us)
+    Z0 = oracle_Z0(w, us)
+    _, LP_ref = O.user_encode(f64(us.E), offs, Z0, layers, w.H, users=users)
+    LP_cpu = LP.cpu()
+    chain = w.layers + (1 if w.c > 0 else 0)
+    for u in users:
+        assert_close(LP_cpu[u], LP_ref[u], w.dtype, f"L^P user {u}", stages=chain)
+    rows = torch.randint(0, w.n_items, (65536,), generator=g)
+    cache_ref = O.qk_cache(f64(synth.item_rows(w, rows)), f64(us.L), f64(cs.Wq_c),
+                           f64(cs.Wk_c), w.H)
+    assert_close(buf.cache[rows.cuda()], cache_ref, w.dtype, "sampled cache rows")
+    co = cs.cand_offsets.numpy()
+    cache_cpu = None
+    for u in users:
+        a, b = int(co[u]), int(co[u + 1])
+        ids = cs.cand_ids[a:b]
+        rows_u = buf.cache[ids.long().cuda()].cpu()
+        ref = O.score_candidates(f64(rows_u), np.arange(b - a), [0, b - a], f64(LP_cpu[u:u + 1]))
+        assert_close(buf.O[a:b], ref, w.dtype, f"scores user {u}")

@@ -1,0 +1,286 @@
+// QK-cache build on the 5th-generation tensor cores (bf16, d = 128).
+//
+// LIME note, 关键设计 1: the candidate-side weights phi(T L^T) depend only on
+// the item embedding and the global links, so they are computed offline for
+// the whole catalogue.  With per-head scaled-softmax attention,
+//     cache[m, h, :] = softmax_k( T_m · G[:, h*l + k] ),
+//     G[:, h*l + k]  = s * Wq_c[:, h-cols] (L_k Wk_c[:, h-cols])^T,
+// so the build is one catalogue x (H*l) GEMM with a softmax epilogue.
+//
+// k_fold_g_img folds G (d x H*l, fp32 then bf16) and writes it pre-swizzled in
+// the K-major 128-byte-swizzle image the MMA reads, so each CTA loads it with
+// one bulk copy.  k_cache_tc is persistent (one CTA per SM):
+//   warp 0     TMA producer: 128-row tiles of T into a STAGES-deep ring
+//   warp 1     tcgen05.mma issuer (M=128, N=H*l, K=128 as 8 K-steps) into one
+//              of two TMEM accumulators
+//   warps 2-5  epilogue: tcgen05.ld of its row, softmax per head over l
+//              links in fp32, bf16 into a 128-byte-swizzled staging tile,
+//              TMA store of the tile (rows past n_items are clipped by TMA)
+// Every wait is bounded; a timeout sets LIME_FLAG_TIMEOUT and the CTA drains
+// and returns.  The catalogue read is the roofline: 2*(d + H*l) bytes/item.
+#include "lime_fast.cuh"
+#include "sm100.cuh"
+
+namespace lime {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kD = 128;    // model dim handled here
+constexpr int kBM = 128;   // catalogue rows per tile
+
+template <int HL>
+struct CacheCfg {
+  static constexpr int STAGES = HL <= 128 ? 4 : 3;
+  static constexpr int OUTB = HL <= 128 ? 2 : 1;
+  static constexpr int A_BYTES = kBM * kD * 2;      // one T tile
+  static constexpr int B_BYTES = HL * kD * 2;       // the G^T image
+  static constexpr int O_BYTES = kBM * HL * 2;      // one output tile
+  static constexpr int TMEM_COLS = 2 * HL;
+  static constexpr int OFF_B = STAGES * A_BYTES;
+  static constexpr int OFF_O = OFF_B + B_BYTES;
+  static constexpr int OFF_BAR = OFF_O + OUTB * O_BYTES;
+  static constexpr int SMEM = 1024 + OFF_BAR + 256;
+};
+
+// G^T image: block b (K columns [64b, 64b+64)) of HL rows x 128 bytes,
+// element (row j = h*l + k, K index i) at b*HL*128 + sw128_offset(j, i % 64).
+template <class T>
+__global__ void k_fold_g_img(const T* __restrict__ L, const T* __restrict__ Wq,
+                             const T* __restrict__ Wk, int d, int H, int l, float scale,
+                             bf16* __restrict__ img) {
+  __shared__ float kc[64];
+  const int j = blockIdx.x, h = j / l, k = j % l, dh = d / H, HL = H * l;
+  for (int c = threadIdx.x; c < dh; c += blockDim.x) {
+    float acc = 0.f;
+    for (int t = 0; t < d; ++t) acc += to_f(L[(int64_t)k * d + t]) * to_f(Wk[(int64_t)t * d + h * dh + c]);
+    kc[c] = acc;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    float acc = 0.f;
+    for (int c = 0; c < dh; ++c) acc += to_f(Wq[(int64_t)i * d + h * dh + c]) * kc[c];
+    uint8_t* base = reinterpret_cast<uint8_t*>(img) + (size_t)(i >> 6) * HL * 128;
+    *reinterpret_cast<bf16*>(base + sw128_offset(j, i & 63)) = __float2bfloat16_rn(acc * scale);
+  }
+}
+
+template <int HL, int L>
+__global__ void __launch_bounds__(192, 1)
+    k_cache_tc(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmC,
+               const bf16* __restrict__ gimg, int n_tiles, unsigned* status) {
+  using C = CacheCfg<HL>;
+  constexpr int H = HL / L;
+  constexpr uint32_t IDESC = idesc_bf16(kBM, HL);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::OFF_B;
+  uint8_t* sO = smem + C::OFF_O;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* ofull = tempty + 2;
+  uint64_t* ofree = ofull + 2;
+  uint64_t* bready = ofree + 2;
+  uint64_t* mdone = bready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + 1);
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+      mbar_init(&ofull[a], 128);
+      mbar_init(&ofree[a], 1);
+    }
+    mbar_init(bready, 1);
+    mbar_init(mdone, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmT);
+      prefetch_tmap(&tmC);
+      mbar_arrive_expect_tx(bready, C::B_BYTES);
+      bulk_load(sB, gimg, C::B_BYTES, bready);
+      int it = 0;
+      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+        const int s = it % C::STAGES;
+        const uint32_t ph = (it / C::STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, status, &abort_flag)) break;
+        mbar_arrive_expect_tx(&full[s], C::A_BYTES);
+        uint8_t* dst = sA + s * C::A_BYTES;
+        tma_load_2d(dst, &tmT, 0, tile * kBM, &full[s]);
+        tma_load_2d(dst + C::A_BYTES / 2, &tmT, 64, tile * kBM, &full[s]);
+      }
+      // drain: every issued load has landed before the CTA may exit
+      const int issued = it;
+      for (int j = issued > C::STAGES ? issued - C::STAGES : 0; j < issued; ++j)
+        mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1, status, &abort_flag);
+      mbar_wait(bready, 0, status, &abort_flag);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      if (mbar_wait(bready, 0, status, &abort_flag)) {
+        const uint32_t bBase = smem_u32(sB);
+        int it = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          const int acc = it & 1;
+          const uint32_t aph = (it >> 1) & 1;
+          if (!mbar_wait(&tempty[acc], aph ^ 1, status, &abort_flag)) break;
+          if (!mbar_wait(&full[s], ph, status, &abort_flag)) break;
+          tc_fence_after();
+          const uint32_t aBase = smem_u32(sA + s * C::A_BYTES);
+#pragma unroll
+          for (int k = 0; k < kD / 16; ++k) {
+            const uint32_t koff = (k & 3) * 32;
+            const uint64_t ad = sdesc_sw128(aBase + (k >> 2) * (C::A_BYTES / 2) + koff);
+            const uint64_t bd = sdesc_sw128(bBase + (k >> 2) * (C::B_BYTES / 2) + koff);
+            mma_bf16(tmem + acc * HL, ad, bd, IDESC, k > 0);
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&tfull[acc]);
+        }
+      }
+      mma_commit(mdone);
+      mbar_wait(mdone, 0, status, &abort_flag);
+    }
+  } else {
+    // epilogue: 128 threads, thread owns TMEM lane / tile row `row`
+    const int et = threadIdx.x - 64;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      const int ob = C::OUTB == 2 ? (it & 1) : 0;
+      const uint32_t oph = (it / C::OUTB) & 1;
+      if (!mbar_wait(&ofree[ob], oph ^ 1, status, &abort_flag)) break;
+      if (!mbar_wait(&tfull[acc], aph, status, &abort_flag)) break;
+      tc_fence_after();
+      uint8_t* stage = sO + ob * C::O_BYTES;
+#pragma unroll 1
+      for (int h = 0; h < H; ++h) {
+        float z[L];
+#pragma unroll
+        for (int q = 0; q < L / 16; ++q)
+          tmem_ld16(tmem + lane_base + acc * HL + h * L + q * 16, z + q * 16);
+        tmem_ld_wait();
+        float m = z[0];
+#pragma unroll
+        for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
+        float ssum = 0.f;
+#pragma unroll
+        for (int k = 0; k < L; ++k) {
+          z[k] = __expf(z[k] - m);
+          ssum += z[k];
+        }
+        const float inv = 1.0f / ssum;
+#pragma unroll
+        for (int c = 0; c < L / 8; ++c) {
+          const int col = h * L + c * 8;
+          uint4 v;
+          v.x = pack_bf16(z[c * 8 + 0] * inv, z[c * 8 + 1] * inv);
+          v.y = pack_bf16(z[c * 8 + 2] * inv, z[c * 8 + 3] * inv);
+          v.z = pack_bf16(z[c * 8 + 4] * inv, z[c * 8 + 5] * inv);
+          v.w = pack_bf16(z[c * 8 + 6] * inv, z[c * 8 + 7] * inv);
+          *reinterpret_cast<uint4*>(stage + (col >> 6) * (kBM * 128) + sw128_offset(row, col & 63)) = v;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      fence_proxy_async_smem();
+      mbar_arrive(&ofull[ob]);
+      if (et == 0) {
+        if (!mbar_wait(&ofull[ob], oph, status, &abort_flag)) break;
+#pragma unroll
+        for (int b = 0; b < HL / 64; ++b) tma_store_2d(&tmC, stage + b * (kBM * 128), b * 64, tile * kBM);
+        bulk_commit();
+        // the store issued OUTB-1 tiles ago has finished reading its buffer
+        bulk_wait_read<C::OUTB - 1>();
+        if (C::OUTB == 2) {
+          if (it >= 1) mbar_arrive(&ofree[ob ^ 1]);
+        } else {
+          mbar_arrive(&ofree[0]);
+        }
+      }
+    }
+    if (et == 0) bulk_wait<0>();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int HL, int L>
+int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, unsigned* status,
+                 cudaStream_t st) {
+  using C = CacheCfg<HL>;
+  CUtensorMap tmT, tmC;
+  if (!make_tmap_2d_bf16(&tmT, T, kD, (uint64_t)n, kD * 2, 64, kBM)) return LIME_ERR_CUDA;
+  if (!make_tmap_2d_bf16(&tmC, cache, HL, (uint64_t)n, HL * 2, 64, kBM)) return LIME_ERR_CUDA;
+  if (cudaFuncSetAttribute(k_cache_tc<HL, L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM) != cudaSuccess)
+    return LIME_ERR_CUDA;
+  const int n_tiles = (int)((n + kBM - 1) / kBM);
+  const int grid = n_tiles < num_sms() ? n_tiles : num_sms();
+  k_cache_tc<HL, L><<<grid, 192, C::SMEM, st>>>(tmT, tmC, img, n_tiles, status);
+  note_launches(1);
+  return LIME_OK;
+}
+
+}  // namespace
+
+size_t fast_cache_ws_bytes(const lime_dims& D) { return (size_t)D.H * D.l * D.d * 2; }
+
+bool fast_cache_supported(const lime_dims& D) {
+  if (D.dtype != LIME_BF16 || D.d != kD) return false;
+  const int HL = D.H * D.l, dh = D.d / D.H;
+  if (dh != 16 && dh != 32 && dh != 64) return false;
+  if (D.l != 16 && D.l != 32 && D.l != 64) return false;
+  return HL == 64 || HL == 128 || HL == 256;
+}
+
+int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void* L,
+                        const void* Wq, const void* Wk, void* cache, float* ws, unsigned* status,
+                        cudaStream_t st) {
+  const int HL = D.H * D.l;
+  bf16* img = reinterpret_cast<bf16*>(ws);
+  const float scale = 1.0f / sqrtf((float)(D.d / D.H));
+  k_fold_g_img<bf16><<<HL, 128, 0, st>>>((const bf16*)L, (const bf16*)Wq, (const bf16*)Wk, D.d,
+                                         D.H, D.l, scale, img);
+  note_launches(1);
+  if (n == 0) return LIME_OK;
+  switch (HL * 1000 + D.l) {
+    case 64016: return launch_cache<64, 16>(T, n, img, cache, status, st);
+    case 64032: return launch_cache<64, 32>(T, n, img, cache, status, st);
+    case 64064: return launch_cache<64, 64>(T, n, img, cache, status, st);
+    case 128016: return launch_cache<128, 16>(T, n, img, cache, status, st);
+    case 128032: return launch_cache<128, 32>(T, n, img, cache, status, st);
+    case 128064: return launch_cache<128, 64>(T, n, img, cache, status, st);
+    case 256032: return launch_cache<256, 32>(T, n, img, cache, status, st);
+    case 256064: return launch_cache<256, 64>(T, n, img, cache, status, st);
+    default: return LIME_ERR_SHAPE;
+  }
+}
+
+}  // namespace lime

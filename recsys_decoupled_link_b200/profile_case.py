@@ -1,0 +1,65 @@
+"""Runs one phase of the hot path a few times, for profiler captures.
+
+    python -m recsys_decoupled_link_b200.profile_case --phase cache --workload standard --reps 3
+
+Phases: ``cache`` (QK-cache build over the catalogue), ``score`` (cached
+scoring; the cache is built once first), ``layer`` (one LIME-XOR layer, the
+first of the stack, with history outputs), ``last`` (the last-layer variant
+without history outputs), ``step`` (the whole pass).  Inputs are the seeded
+synthetic workloads of ``synth``; ``--items`` and ``--users`` shrink them.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import lime, pipeline, synth
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--phase", default="cache", choices=["cache", "score", "layer", "last", "step"])
+    ap.add_argument("--workload", default="standard")
+    ap.add_argument("--items", type=int, default=None)
+    ap.add_argument("--users", type=int, default=None)
+    ap.add_argument("--reps", type=int, default=3)
+    a = ap.parse_args()
+    over = {}
+    if a.items:
+        over["n_items"] = a.items
+    if a.users:
+        over["B"] = a.users
+    w = synth.workload(a.workload, **over)
+    us, cs = synth.user_side(w), synth.candidate_side(w)
+    x = pipeline.to_device(w, us, cs, synth.item_table(w))
+    buf = pipeline.alloc(x)
+    Z = buf.LC
+    if x.ctx_w is not None:
+        lime.lime_context_links(x.dims, x.L, x.ctx, *x.ctx_w, buf.LC)
+    else:
+        Z = x.Z0
+    if a.phase == "score":
+        pipeline.build_cache(x, buf)
+    for _ in range(a.reps):
+        if a.phase == "cache":
+            pipeline.build_cache(x, buf)
+        elif a.phase == "score":
+            pipeline.score(x, buf, Z)
+        elif a.phase == "layer":
+            lime.lime_xor_layer(x.dims, x.hist_offsets, x.total_hist, x.E, Z, x.layers[0],
+                                buf.E_bufs[0], buf.Z_bufs[0], buf.ws)
+        elif a.phase == "last":
+            lime.lime_xor_layer(x.dims, x.hist_offsets, x.total_hist, x.E, Z, x.layers[-1],
+                                None, buf.Z_bufs[0], buf.ws)
+        else:
+            pipeline.step(x, buf)
+    torch.cuda.synchronize()
+    flags = lime.lime_get_status(buf.ws)
+    if flags:
+        raise SystemExit(f"device status flags {flags}")
+    print(f"ok: {a.phase} x{a.reps} on {w.name}")
+
+
+if __name__ == "__main__":
+    main()

@@ -109,6 +109,30 @@ int lime_build_qk_cache(const lime_dims* dims, const void* T, int64_t n_items,
                         void* cache_out, void* workspace, size_t workspace_bytes,
                         cudaStream_t stream);
 
+/* Allocation-free variant of lime_build_qk_cache.  The paper has no
+ * counterpart: it exists for callers that cannot allocate device memory, such
+ * as a plug-in whose host framework owns the whole device memory pool, or a
+ * latency-critical serving loop that cannot accept cudaMalloc's implicit
+ * device synchronisation.  The caller still owns T, L, Wq_c, Wk_c and
+ * cache_out (same meaning, layout and checks as lime_build_qk_cache); the
+ * scratch lives in a static device array of LIME_NOALLOC_SCRATCH_BYTES bytes
+ * that every GPU loading the library holds until the process exits.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address; make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; each
+ *     call clears the status word it uses.  Calls that overlap on the GPU (on
+ *     different streams, say) race on the array.
+ *   - Sizes whose scratch exceeds the maximum (2*d*H*l bytes on the bf16
+ *     tensor-core path, 4*(l*d + d*H*l) bytes otherwise, plus 256) return
+ *     LIME_ERR_SCRATCH; use lime_build_qk_cache with a workspace instead.
+ *   - Device-side status flags of these calls are not reported.
+ * Calls no cudaMalloc, cudaFree or allocating library routine.            */
+#define LIME_NOALLOC_SCRATCH_BYTES (1u << 20)
+enum { LIME_ERR_SCRATCH = -5 /* scratch need above LIME_NOALLOC_SCRATCH_BYTES */ };
+int lime_build_qk_cache_noalloc(const lime_dims* dims, const void* T, int64_t n_items,
+                                const void* L, const void* Wq_c, const void* Wk_c,
+                                void* cache_out, cudaStream_t stream);
+
 /* Context links: LC[u, k, :] = SiLU([L_k ; ctx_u] Wc1 + bc1) Wc2 + bc2.
  * LIME note 整体框架 (L^C = MLP(L ⊕ E^C)) and 一个完整示例 step 2.
  *   L   device [l, d];  ctx device [B, c];  LC_out device [B, l, d].

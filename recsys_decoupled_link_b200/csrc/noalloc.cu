@@ -1,0 +1,76 @@
+// lime_build_qk_cache_noalloc: the QK-cache build for callers that cannot
+// allocate device memory.
+//
+// Some callers cannot call cudaMalloc: a plug-in hosted by a serving framework
+// that owns the whole device memory pool and forbids its plug-ins to allocate,
+// or a latency-critical serving loop where cudaMalloc's implicit device
+// synchronisation is not acceptable.  They still own their inputs and
+// outputs, but cannot provide the workspace lime_build_qk_cache takes.  This
+// entry point runs the same cache build with its scratch in a file-scope
+// static device array of LIME_NOALLOC_SCRATCH_BYTES bytes instead.
+//
+// The array is part of the library's device image: every GPU that loads the
+// library holds it until the process exits.  Host code cannot use the array's
+// name as a device address (on the host it names a stand-in object), so the
+// first call on each device, with that device current, looks its device
+// address up with cudaGetSymbolAddress and keeps it; that first call should
+// therefore come before any stream capture.  All calls share the one array and
+// it keeps the last call's contents: each call clears the status word at its
+// head before use, and calls that overlap on the GPU (e.g. on two streams) race
+// on it.  Nothing here calls cudaMalloc, cudaFree or an allocating library
+// routine.
+#include <stdio.h>
+
+#include <mutex>
+
+#include "lime.h"
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LIME_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+std::mutex g_scratch_mu;
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device; nullptr if the runtime refuses.
+void* scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) {
+      fprintf(stderr, "liblime: cudaGetSymbolAddress(scratch) failed: %s\n",
+              cudaGetErrorString(e));
+      return nullptr;
+    }
+    g_scratch_ptr[dev] = p;
+  }
+  return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" int lime_build_qk_cache_noalloc(const lime_dims* dims, const void* T,
+                                           int64_t n_items, const void* L, const void* Wq_c,
+                                           const void* Wk_c, void* cache_out,
+                                           cudaStream_t stream) {
+  const size_t need = lime_workspace_bytes(dims, 0, 0);
+  if (need == 0) return dims == nullptr ? LIME_ERR_ARG : LIME_ERR_SHAPE;
+  if (need > (size_t)LIME_NOALLOC_SCRATCH_BYTES) {
+    fprintf(stderr,
+            "liblime: lime_build_qk_cache_noalloc needs %zu bytes of scratch, more than its "
+            "static maximum of %u bytes; use lime_build_qk_cache with a workspace\n",
+            need, (unsigned)LIME_NOALLOC_SCRATCH_BYTES);
+    return LIME_ERR_SCRATCH;
+  }
+  void* scratch = scratch_address();
+  if (!scratch) return LIME_ERR_CUDA;
+  int rc = lime_workspace_init(scratch, LIME_NOALLOC_SCRATCH_BYTES, stream);
+  if (rc != LIME_OK) return rc;
+  return lime_build_qk_cache(dims, T, n_items, L, Wq_c, Wk_c, cache_out, scratch,
+                             LIME_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -18,10 +18,13 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblime.so
 
 LIME_F32, LIME_BF16 = 0, 1
 LIME_OK, LIME_ERR_ARG, LIME_ERR_SHAPE, LIME_ERR_ALIAS, LIME_ERR_CUDA = 0, -1, -2, -3, -4
+LIME_ERR_SCRATCH = -5
+LIME_NOALLOC_SCRATCH_BYTES = 1 << 20
 LIME_FLAG_BAD_ID, LIME_FLAG_BAD_OFFSETS, LIME_FLAG_TIMEOUT = 1, 2, 4
 
 _ERRORS = {LIME_ERR_ARG: "bad argument", LIME_ERR_SHAPE: "unsupported shape",
-           LIME_ERR_ALIAS: "output aliases an input", LIME_ERR_CUDA: "CUDA error"}
+           LIME_ERR_ALIAS: "output aliases an input", LIME_ERR_CUDA: "CUDA error",
+           LIME_ERR_SCRATCH: "scratch above the allocation-free maximum"}
 
 
 class LimeError(RuntimeError):
@@ -61,6 +64,7 @@ def _load() -> ctypes.CDLL:
         "lime_score_candidates": (I32, [D, I64, P, I64, P, P, I64, P, P, P, SZ, P]),
         "lime_get_status": (I32, [P, P, ctypes.POINTER(ctypes.c_int)]),
         "lime_launch_count": (ctypes.c_uint64, []),
+        "lime_build_qk_cache_noalloc": (I32, [D, P, I64, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -71,7 +75,7 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 EXPORTED = ("lime_workspace_bytes", "lime_workspace_init", "lime_build_qk_cache",
             "lime_context_links", "lime_xor_layer", "lime_score_candidates",
-            "lime_get_status", "lime_launch_count")
+            "lime_get_status", "lime_launch_count", "lime_build_qk_cache_noalloc")
 
 
 def library_path() -> str:
@@ -132,6 +136,14 @@ def lime_build_qk_cache(dims, T, L, Wq_c, Wk_c, cache_out, ws: Workspace, stream
     _check("lime_build_qk_cache", _lib.lime_build_qk_cache(
         ctypes.byref(dims), _ptr(T), n_items, _ptr(L), _ptr(Wq_c), _ptr(Wk_c),
         _ptr(cache_out), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def lime_build_qk_cache_noalloc(dims, T, L, Wq_c, Wk_c, cache_out, stream=None):
+    """lime_build_qk_cache without a workspace (scratch in a static device array)."""
+    n_items = 0 if T is None else T.shape[0]
+    _check("lime_build_qk_cache_noalloc", _lib.lime_build_qk_cache_noalloc(
+        ctypes.byref(dims), _ptr(T), n_items, _ptr(L), _ptr(Wq_c), _ptr(Wk_c),
+        _ptr(cache_out), _stream(stream)))
 
 
 def lime_context_links(dims, L, ctx, Wc1, bc1, Wc2, bc2, LC_out, stream=None):

@@ -59,7 +59,8 @@ size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t scratch_bytes(const lime_dims* D, int64_t B, int64_t total_hist) {
   size_t s = simt_cache_ws_bytes(*D);
-  size_t t = simt_layer_ws_bytes(*D, B, total_hist);
+  // the CUDA-core layer path needs fp32 row buffers; the tensor-core path does not
+  size_t t = fast_layer_supported(*D) ? 0 : simt_layer_ws_bytes(*D, B, total_hist);
   if (t > s) s = t;
   size_t u = fast_ws_bytes(*D, B, total_hist);
   if (u > s) s = u;

@@ -6,6 +6,7 @@ namespace lime {
 
 size_t fast_ws_bytes(const lime_dims& D, int64_t B, int64_t total_hist);
 size_t fast_cache_ws_bytes(const lime_dims& D);
+size_t fast_layer_ws_bytes(const lime_dims& D, int64_t B, int64_t total_hist);
 
 bool fast_cache_supported(const lime_dims& D);
 int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void* L,

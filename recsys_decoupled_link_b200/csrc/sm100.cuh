@@ -217,3 +217,80 @@ bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint6
 int num_sms();
 
 }  // namespace lime
+
+namespace lime {
+namespace sm100 {
+
+// tcgen05.st of 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Issues the MMAs of one 128-row tile: D[128 x N] (+)= A[128 x K] * B[N x K]^T.
+// A and B are K-major 128-byte-swizzled operands split into blocks of 64 K
+// columns; a_blk / b_blk are the byte strides between those blocks and
+// a_base / b_base may point into a block at a 32-byte multiple (a K slice).
+__device__ __forceinline__ void mma_tile(uint32_t d_tmem, uint32_t a_base, uint32_t a_blk,
+                                         uint32_t b_base, uint32_t b_blk, int N, int K,
+                                         bool accumulate) {
+  const uint32_t idesc = idesc_bf16(128, N);
+  for (int k = 0; k < K / 16; ++k) {
+    const uint32_t off = (uint32_t)(k & 3) * 32;
+    mma_bf16(d_tmem, sdesc_sw128(a_base + (k >> 2) * a_blk + off),
+             sdesc_sw128(b_base + (k >> 2) * b_blk + off), idesc, accumulate || k > 0);
+  }
+}
+
+// Thread 0 commits the MMAs it issued to `bar`; every thread of the CTA then
+// waits for them (bounded) and flips its phase bit.
+__device__ __forceinline__ void cta_mma_wait(uint64_t* bar, uint32_t& phase, unsigned* status,
+                                             volatile int* abort_flag) {
+  if (threadIdx.x == 0) mma_commit(bar);
+  mbar_wait(bar, phase, status, abort_flag);
+  phase ^= 1u;
+  tc_fence_after();
+}
+
+// Reads 8 bf16 (16 bytes) of row `row`, columns [c8*8, c8*8+8), of a K-major
+// swizzled [rows x (64*nblk)] operand whose blocks are `blk` bytes apart.
+__device__ __forceinline__ uint4 sw_ld16(const uint8_t* base, uint32_t blk, int row, int col) {
+  return *reinterpret_cast<const uint4*>(base + (col >> 6) * blk + sw128_offset(row, col & 63));
+}
+__device__ __forceinline__ void sw_st16(uint8_t* base, uint32_t blk, int row, int col, uint4 v) {
+  *reinterpret_cast<uint4*>(base + (col >> 6) * blk + sw128_offset(row, col & 63)) = v;
+}
+
+__device__ __forceinline__ void unpack8(uint4 v, float* f) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(p[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  uint4 v;
+  v.x = pack_bf16(f[0], f[1]);
+  v.y = pack_bf16(f[2], f[3]);
+  v.z = pack_bf16(f[4], f[5]);
+  v.w = pack_bf16(f[6], f[7]);
+  return v;
+}
+
+}  // namespace sm100
+}  // namespace lime

@@ -1,0 +1,1005 @@
+// One LIME-XOR layer on the 5th-generation tensor cores (bf16 storage,
+// d = 128, 4 heads of 32, l in {16, 32}, GatedMLP width 256).
+//
+// LIME note, 关键设计 2: over X = [E; Z] the XOR mask keeps only history<->link
+// attention, XORA(X,X,X) = MHA(E, Z, Z) ⊕ MHA(Z, E, E), at O(l·N) cost; the
+// layer is pre-LN with residual connections and a gated feed-forward block.
+//
+// Work is split by row kind.  Link rows (B·l of them) carry L^P, so their
+// projections run with split-bf16 activations (x = hi + lo, both bf16; the
+// bf16 weights are exact), i.e. at close to fp32 accuracy for twice the MMA
+// work on a few rows.  History rows (the O(N) part) use bf16 operands with
+// fp32 accumulation, statistics and residual adds.  History rows are cut into
+// per-user tiles of 128 rows (a tile never spans two users; its tail rows are
+// masked).
+//
+//   k_prep_weights   layer weights -> K-major 128B-swizzled images (W^T)
+//   k_schedule       hist_offsets -> tile list (user, first row, valid rows)
+//   k_link_proj      LN1(Z) -> Q_Z, K_Z, V_Z (split precision) -> per-user
+//                    operand images: s·K_Z, V_Z^T, and s·Q_Z laid out
+//                    block-diagonally over heads so that one MMA yields the
+//                    link branch's scores transposed (links on TMEM lanes)
+//   k_hist_proj      LN1(E) -> Q_E, K_E (row-major) and V_E^T (per tile)
+//   k_hist_attn      history branch: softmax over the user's l links, P·V_Z,
+//                    then (P·V_Z)·Wo -> Yd (fp32 attention delta);
+//                    link branch: per tile and (head, link) the partial
+//                    softmax statistics (max, sum) and the weighted V sum
+//   k_link_merge     log-sum-exp merge of a user's tile partials -> b (fp32)
+//   k_hist_ffn       Y = E + Yd, LN2, GatedMLP in 64-wide chunks, E' = Y + ·
+//   k_link_out       Y_Z = Z + b·Wo, LN2, GatedMLP, Z' (split precision)
+// The last layer (E_out = NULL) skips everything only E' needs: Q_E, the
+// history branch, Wo on history rows and k_hist_ffn.
+//
+// CTAs run their phases synchronously: thread 0 issues the MMAs of a phase,
+// all 128 threads wait on an mbarrier (bounded), then each thread works on its
+// TMEM lane (one tile row).  Every wait is bounded and sets LIME_FLAG_TIMEOUT.
+#include "lime_fast.cuh"
+#include "sm100.cuh"
+
+namespace lime {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kD = 128, kH = 4, kDH = 32, kF = 256, kTile = 128;
+constexpr uint32_t kBlk = 128 * 128;  // bytes of one [128 rows x 64 cols] bf16 block
+constexpr float kLnEps = 1e-5f;
+
+struct LayerWs {
+  size_t img_q, img_k, img_v, img_o, img_1, img_3, img_2;
+  size_t sched, tiles, tile_start;
+  size_t qe, ke, vt, yd, uimg, part, bmerge;
+  size_t total;
+  int64_t max_tiles;
+  uint32_t uimg_bytes;
+};
+
+__host__ __device__ constexpr size_t up1k(size_t x) { return (x + 1023) & ~(size_t)1023; }
+
+__host__ __device__ constexpr uint32_t kz_bytes(int l) { return (uint32_t)l * 256; }  // [l x 128] bf16
+__host__ __device__ constexpr uint32_t uimg_bytes(int l) {
+  return (uint32_t)up1k(kz_bytes(l) + kBlk + 2 * kBlk);
+}
+
+LayerWs layer_ws(int l, int64_t B, int64_t nh) {
+  LayerWs w;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o = up1k(o + bytes); return r; };
+  w.img_q = take(2 * kBlk);
+  w.img_k = take(2 * kBlk);
+  w.img_v = take(2 * kBlk);
+  w.img_o = take(2 * kBlk);
+  w.img_1 = take(4 * kBlk);
+  w.img_3 = take(4 * kBlk);
+  w.img_2 = take(4 * kBlk);
+  w.max_tiles = nh / kTile + B + 1;
+  w.sched = take(16);
+  w.tiles = take((size_t)w.max_tiles * 16);
+  w.tile_start = take((size_t)(B + 1) * 4);
+  w.qe = take((size_t)nh * kD * 2);
+  w.ke = take((size_t)nh * kD * 2);
+  w.vt = take((size_t)w.max_tiles * kTile * kD * 2);
+  w.yd = take((size_t)nh * kD * 4);   // fp32 attention delta
+  w.uimg_bytes = uimg_bytes(l);
+  w.uimg = take((size_t)B * w.uimg_bytes);
+  w.part = take((size_t)w.max_tiles * (2 + kDH) * kH * l * 4);
+  w.bmerge = take((size_t)B * l * kD * 4);
+  w.total = o;
+  return w;
+}
+
+// Reads row `row` (128 bf16) of a [128 x 128] swizzled tile into fp32.
+__device__ __forceinline__ void tile_row_ld(const uint8_t* t, int row, float* x) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c) unpack8(sw_ld16(t, kBlk, row, c * 8), x + c * 8);
+}
+__device__ __forceinline__ void tile_row_st(uint8_t* t, int row, const float* x) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c) sw_st16(t, kBlk, row, c * 8, pack8(x + c * 8));
+}
+
+// x <- LayerNorm(x) * g + b over 128 values (biased variance).
+__device__ __forceinline__ void layer_norm_128(float* x, const bf16* g, const bf16* b) {
+  float mu = 0.f;
+#pragma unroll
+  for (int i = 0; i < kD; ++i) mu += x[i];
+  mu *= (1.0f / kD);
+  float var = 0.f;
+#pragma unroll
+  for (int i = 0; i < kD; ++i) { const float t = x[i] - mu; var += t * t; }
+  const float rstd = rsqrtf(var * (1.0f / kD) + kLnEps);
+#pragma unroll
+  for (int i = 0; i < kD; ++i)
+    x[i] = (x[i] - mu) * rstd * __bfloat162float(g[i]) + __bfloat162float(b[i]);
+}
+
+// Loads 128 consecutive fp32 TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_row128(uint32_t taddr, float* x) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) tmem_ld16(taddr + q * 16, x + q * 16);
+  tmem_ld_wait();
+}
+
+__device__ __forceinline__ void gl_row_st(bf16* dst, const float* x) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int c = 0; c < 16; ++c) d[c] = pack8(x + c * 8);
+}
+__device__ __forceinline__ void gl_row_ld(const bf16* src, float* x) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int c = 0; c < 16; ++c) unpack8(s[c], x + c * 8);
+}
+
+// Writes x (fp32) as hi = bf16(x) and lo = bf16(x - hi) rows of two operands.
+__device__ __forceinline__ void split_row_st(uint8_t* hi, uint8_t* lo, uint32_t blk, int row,
+                                             const float* x, int n) {
+  for (int c = 0; c < n / 8; ++c) {
+    float h[8], r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      h[i] = __bfloat162float(__float2bfloat16_rn(x[c * 8 + i]));
+      r[i] = x[c * 8 + i] - h[i];
+    }
+    sw_st16(hi, blk, row, c * 8, pack8(h));
+    sw_st16(lo, blk, row, c * 8, pack8(r));
+  }
+}
+
+__device__ __forceinline__ float silu_fast(float x) { return x / (1.0f + __expf(-x)); }
+
+// Common CTA prologue: barriers, abort flag, TMEM allocation (512 columns).
+struct Cta {
+  uint64_t* bar;      // [0] loads, [1] mma, [2..3] extra loads
+  uint32_t* slot;
+  int* abort_flag;
+  uint32_t tmem;
+};
+
+__device__ __forceinline__ void cta_setup(uint8_t* bar_area, int nbar, Cta& c) {
+  c.bar = reinterpret_cast<uint64_t*>(bar_area);
+  c.slot = reinterpret_cast<uint32_t*>(bar_area + 8 * nbar);
+  c.abort_flag = reinterpret_cast<int*>(bar_area + 8 * nbar + 8);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nbar; ++i) mbar_init(&c.bar[i], 1);
+    *c.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 32) tmem_alloc(c.slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  c.tmem = *c.slot;
+}
+
+__device__ __forceinline__ void cta_teardown(Cta& c) {
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    tc_fence_after();
+    tmem_dealloc(c.tmem, 512);
+  }
+}
+
+__device__ __forceinline__ uint32_t lane_addr(const Cta& c) {
+  return c.tmem + ((uint32_t)(threadIdx.x & ~31) << 16);
+}
+
+__device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// ------------------------------------------------------------ weight images
+// Image of W^T (K-major B operand) for x·W, W row-major [k_in, n_out]:
+//   Wq, Wk, Wv, Wo, W2: element (n, k) at (k/64)*rows*128 + sw128_offset(n, k%64)
+//   W1, W3 (n in [0,256)): chunk n/64 of 16 KB, inside it (k/64)*8192 +
+//   sw128_offset(n%64, k%64), so one 64-wide GatedMLP chunk is contiguous.
+__global__ void k_prep_weights(const bf16* __restrict__ Wq, const bf16* __restrict__ Wk,
+                               const bf16* __restrict__ Wv, const bf16* __restrict__ Wo,
+                               const bf16* __restrict__ W1, const bf16* __restrict__ W3,
+                               const bf16* __restrict__ W2, uint8_t* __restrict__ ws,
+                               LayerWs L) {
+  const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t n_sq = kD * kD, n_ff = kD * kF;
+  if (e < 4 * n_sq) {
+    const int w = (int)(e / n_sq), r = (int)(e % n_sq);
+    const int k = r / kD, n = r % kD;
+    const bf16* src = w == 0 ? Wq : w == 1 ? Wk : w == 2 ? Wv : Wo;
+    const size_t base = w == 0 ? L.img_q : w == 1 ? L.img_k : w == 2 ? L.img_v : L.img_o;
+    *reinterpret_cast<bf16*>(ws + base + (k >> 6) * kBlk + sw128_offset(n, k & 63)) = src[r];
+  } else if (e < 4 * n_sq + 2 * n_ff) {
+    const int64_t r0 = e - 4 * n_sq;
+    const int w = (int)(r0 / n_ff), r = (int)(r0 % n_ff);
+    const int k = r / kF, n = r % kF;
+    const bf16* src = w == 0 ? W1 : W3;
+    const size_t base = w == 0 ? L.img_1 : L.img_3;
+    *reinterpret_cast<bf16*>(ws + base + (n >> 6) * 16384 + (k >> 6) * 8192 +
+                             sw128_offset(n & 63, k & 63)) = src[r];
+  } else if (e < 4 * n_sq + 3 * n_ff) {
+    const int r = (int)(e - 4 * n_sq - 2 * n_ff);
+    const int k = r / kD, n = r % kD;   // W2 is [256, 128]
+    *reinterpret_cast<bf16*>(ws + L.img_2 + (k >> 6) * kBlk + sw128_offset(n, k & 63)) = W2[r];
+  }
+}
+
+// --------------------------------------------------------------- schedule
+// Tiles of 128 history rows per user, in user order.  Writes n_tiles to
+// sched[0], tiles[t] = (u, first row, valid rows, 0) and tile_start[u] (the
+// first tile of user u; tile_start[B] = n_tiles).  Offsets are clamped into
+// [0, nh]; violations set LIME_FLAG_BAD_OFFSETS.
+__global__ void k_schedule(const int64_t* __restrict__ off, int64_t B, int64_t nh,
+                           int max_tiles, int* __restrict__ sched, int4* __restrict__ tiles,
+                           int* __restrict__ tile_start, unsigned* status) {
+  __shared__ int warp_sums[32];
+  __shared__ int s_base;
+  if (threadIdx.x == 0) s_base = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int64_t u0 = 0; u0 < B; u0 += blockDim.x) {
+    const int64_t u = u0 + threadIdx.x;
+    int64_t a = 0, b = 0;
+    int cnt = 0;
+    if (u < B) {
+      user_range(off, u, B, nh, &a, &b, status);
+      cnt = (int)((b - a + kTile - 1) / kTile);
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int v = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+      }
+      warp_sums[lane] = v;
+    }
+    __syncthreads();
+    const int start = s_base + (warp > 0 ? warp_sums[warp - 1] : 0) + incl - cnt;
+    if (u < B) {
+      tile_start[u] = start;
+      for (int i = 0; i < cnt && start + i < max_tiles; ++i) {
+        const int64_t r0 = a + (int64_t)i * kTile;
+        const int64_t nv = b - r0 < kTile ? b - r0 : kTile;
+        tiles[start + i] = make_int4((int)u, (int)r0, (int)nv, 0);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) s_base += warp_sums[(blockDim.x >> 5) - 1];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const int n = s_base < max_tiles ? s_base : max_tiles;
+    sched[0] = n;
+    tile_start[B] = n;
+  }
+}
+
+// ----------------------------------------------------- link projections
+// Per-user operand images (at uimg + u * uimg_bytes, ℓ = L):
+//   KZ   [L rows x 128] bf16, 2 blocks of L*128 bytes:  s·K_Z
+//   VZT  [128 rows (c) x 64 cols (k)] bf16, 1 block:     V_Z^T, k >= L zero
+//   QZBD [128 rows (h,k) x 128] bf16, 2 blocks of 16 KB: row h*L + k holds
+//        s·Q_Z[k] in head h's 32 columns and zeros elsewhere; rows >= 4L zero
+template <int L>
+__global__ void __launch_bounds__(128, 1)
+    k_link_proj(const bf16* __restrict__ Z, int64_t nrows, const bf16* __restrict__ g1,
+                const bf16* __restrict__ b1, const uint8_t* __restrict__ ws_c,
+                uint8_t* __restrict__ ws, LayerWs Lw, float scale, unsigned* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1k(smem_raw);
+  uint8_t* sAh = sm;
+  uint8_t* sAl = sm + 2 * kBlk;
+  uint8_t* sW = sm + 4 * kBlk;  // Wq, Wk, Wv images
+  Cta c;
+  cta_setup(sm + 10 * kBlk, 2, c);
+  uint32_t mph = 0;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&c.bar[0], 6 * kBlk);
+    bulk_load(sW, ws_c + Lw.img_q, 2 * kBlk, &c.bar[0]);
+    bulk_load(sW + 2 * kBlk, ws_c + Lw.img_k, 2 * kBlk, &c.bar[0]);
+    bulk_load(sW + 4 * kBlk, ws_c + Lw.img_v, 2 * kBlk, &c.bar[0]);
+  }
+  const int r = threadIdx.x;
+  const int64_t R = (int64_t)blockIdx.x * kTile + r;
+  float x[kD];
+  if (R < nrows) {
+    gl_row_ld(Z + R * kD, x);
+    layer_norm_128(x, g1, b1);
+  } else {
+#pragma unroll
+    for (int i = 0; i < kD; ++i) x[i] = 0.f;
+  }
+  split_row_st(sAh, sAl, kBlk, r, x, kD);
+  fence_proxy_async_smem();
+  __syncthreads();
+  mbar_wait(&c.bar[0], 0, status, c.abort_flag);
+  if (threadIdx.x == 0) {
+    tc_fence_after();
+    for (int w = 0; w < 3; ++w) {
+      const uint32_t bw = smem_u32(sW + w * 2 * kBlk);
+      mma_tile(c.tmem + w * 128, smem_u32(sAh), kBlk, bw, kBlk, 128, 128, false);
+      mma_tile(c.tmem + w * 128, smem_u32(sAl), kBlk, bw, kBlk, 128, 128, true);
+    }
+  }
+  cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+  // TMEM loads are warp-collective: every thread loads, valid rows store.
+  const uint32_t ta = lane_addr(c);
+  const bool valid = R < nrows;
+  const int64_t u = valid ? R / L : 0;
+  const int k = (int)(R % L);
+  uint8_t* img = ws + Lw.uimg + u * Lw.uimg_bytes;
+  uint8_t* kz = img;
+  uint8_t* vzt = img + kz_bytes(L);
+  uint8_t* qbd = vzt + kBlk;
+  float v[kD];
+  // s·K_Z row k
+  tmem_row128(ta + 128, v);
+  if (valid) {
+#pragma unroll
+    for (int i = 0; i < kD; ++i) v[i] *= scale;
+    for (int cc = 0; cc < 16; ++cc) sw_st16(kz, (uint32_t)L * 128, k, cc * 8, pack8(v + cc * 8));
+  }
+  // V_Z^T column k (and zero padding columns k + L, k + 2L, ... < 64)
+  tmem_row128(ta + 256, v);
+  if (valid) {
+    for (int cc = 0; cc < kD; ++cc) {
+      *reinterpret_cast<bf16*>(vzt + sw128_offset(cc, k)) = __float2bfloat16_rn(v[cc]);
+      for (int kp = k + L; kp < 64; kp += L)
+        *reinterpret_cast<bf16*>(vzt + sw128_offset(cc, kp)) = __float2bfloat16_rn(0.f);
+    }
+  }
+  // block-diagonal s·Q_Z: rows h*L + k; rows >= 4L are zero
+  tmem_row128(ta, v);
+  if (valid) {
+#pragma unroll
+    for (int i = 0; i < kD; ++i) v[i] *= scale;
+    const float zero8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int h = 0; h < kH; ++h) {
+      for (int cc = 0; cc < 16; ++cc) {
+        const bool mine = (cc >> 2) == h;   // 4 chunks of 8 columns per head
+        sw_st16(qbd, kBlk, h * L + k, cc * 8, pack8(mine ? v + cc * 8 : zero8));
+      }
+    }
+    for (int p = kH * L + k; p < kTile; p += L)
+      for (int cc = 0; cc < 16; ++cc) sw_st16(qbd, kBlk, p, cc * 8, pack8(zero8));
+  }
+  cta_teardown(c);
+}
+
+// ----------------------------------------------------- history projections
+// One persistent CTA per SM walks the tile list.  For each tile: TMA the 128
+// history rows, LN1 in place, Q/K/V = X^·W on the tensor cores; writes Q_E and
+// K_E rows (valid rows only) and the tile's V_E^T block [128 c x 128 j] with
+// zero columns for rows past the user's history.  The next tile's rows are
+// loaded while this tile's outputs are written.
+template <bool LAST>
+__global__ void __launch_bounds__(128, 1)
+    k_hist_proj(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ g1,
+                const bf16* __restrict__ b1, uint8_t* __restrict__ ws, LayerWs Lw,
+                unsigned* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1k(smem_raw);
+  uint8_t* sE = sm;
+  uint8_t* sW = sm + 2 * kBlk;   // [Wq,] Wk, Wv images
+  constexpr int NW = LAST ? 2 : 3;
+  Cta c;
+  cta_setup(sm + (2 + 2 * NW) * kBlk, 3, c);
+  const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
+  const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
+  bf16* qe = reinterpret_cast<bf16*>(ws + Lw.qe);
+  bf16* ke = reinterpret_cast<bf16*>(ws + Lw.ke);
+  bf16* vt = reinterpret_cast<bf16*>(ws + Lw.vt);
+  uint32_t eph = 0, mph = 0;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&c.bar[2], NW * 2 * kBlk);
+    int slot = 0;
+    if (!LAST) bulk_load(sW + 2 * kBlk * slot++, ws + Lw.img_q, 2 * kBlk, &c.bar[2]);
+    bulk_load(sW + 2 * kBlk * slot++, ws + Lw.img_k, 2 * kBlk, &c.bar[2]);
+    bulk_load(sW + 2 * kBlk * slot, ws + Lw.img_v, 2 * kBlk, &c.bar[2]);
+    if ((int)blockIdx.x < n_tiles) {
+      const int4 tl = tiles[blockIdx.x];
+      mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
+      tma_load_2d(sE, &tmE, 0, tl.y, &c.bar[0]);
+      tma_load_2d(sE + kBlk, &tmE, 64, tl.y, &c.bar[0]);
+    }
+  }
+  mbar_wait(&c.bar[2], 0, status, c.abort_flag);
+  const int i = threadIdx.x;
+  const uint32_t ta = lane_addr(c);
+  for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const int4 tl = tiles[t];
+    const int r0 = tl.y, nv = tl.z;
+    mbar_wait(&c.bar[0], eph, status, c.abort_flag);
+    eph ^= 1u;
+    {
+      float x[kD];
+      tile_row_ld(sE, i, x);
+      layer_norm_128(x, g1, b1);
+      tile_row_st(sE, i, x);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      for (int w = 0; w < NW; ++w)
+        mma_tile(c.tmem + (LAST ? w + 1 : w) * 128, smem_u32(sE), kBlk,
+                 smem_u32(sW + w * 2 * kBlk), kBlk, 128, 128, false);
+    }
+    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+    const int tn = t + gridDim.x;
+    if (threadIdx.x == 0 && tn < n_tiles) {
+      const int4 tl2 = tiles[tn];
+      mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
+      tma_load_2d(sE, &tmE, 0, tl2.y, &c.bar[0]);
+      tma_load_2d(sE + kBlk, &tmE, 64, tl2.y, &c.bar[0]);
+    }
+    float v[kD];
+    if (!LAST) {
+      tmem_row128(ta, v);
+      if (i < nv) gl_row_st(qe + (int64_t)(r0 + i) * kD, v);
+    }
+    tmem_row128(ta + 128, v);
+    if (i < nv) gl_row_st(ke + (int64_t)(r0 + i) * kD, v);
+    tmem_row128(ta + 256, v);
+    bf16* vtt = vt + (int64_t)t * kTile * kD;
+    for (int cc = 0; cc < kD; ++cc)
+      vtt[cc * kTile + i] = __float2bfloat16_rn(i < nv ? v[cc] : 0.f);
+    tc_fence_before();
+    __syncthreads();
+  }
+  cta_teardown(c);
+}
+
+// --------------------------------------------------------- XOR attention
+template <int L, bool LAST>
+__global__ void __launch_bounds__(128, 1)
+    k_hist_attn(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmVT, uint8_t* __restrict__ ws, LayerWs Lw,
+                unsigned* status) {
+  constexpr int HL = kH * L;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1k(smem_raw);
+  uint8_t* sQ = sm;                 // Q_E -> P -> A_E
+  uint8_t* sK = sm + 2 * kBlk;      // K_E -> P2
+  uint8_t* sVT = sm + 4 * kBlk;     // V_E^T block
+  uint8_t* sWo = sm + 6 * kBlk;     // Wo image (not in the last layer)
+  uint8_t* sU = sm + (LAST ? 6 : 8) * kBlk;  // user images
+  uint8_t* sKZ = sU;
+  uint8_t* sVZT = sU + kz_bytes(L);
+  uint8_t* sQBD = sVZT + kBlk;
+  Cta c;
+  cta_setup(sU + uimg_bytes(L), 3, c);
+  const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
+  const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
+  float* yd = reinterpret_cast<float*>(ws + Lw.yd);
+  float* part = reinterpret_cast<float*>(ws + Lw.part);
+  uint32_t lph = 0, mph = 0;
+  if (!LAST) {
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(&c.bar[2], 2 * kBlk);
+      bulk_load(sWo, ws + Lw.img_o, 2 * kBlk, &c.bar[2]);
+    }
+    mbar_wait(&c.bar[2], 0, status, c.abort_flag);
+  }
+  const int i = threadIdx.x;
+  const uint32_t ta = lane_addr(c);
+  int cur_u = -1;
+  for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const int4 tl = tiles[t];
+    const int u = tl.x, r0 = tl.y, nv = tl.z;
+    if (threadIdx.x == 0) {
+      uint32_t bytes = 4 * kBlk + (LAST ? 0 : 2 * kBlk) + (u != cur_u ? Lw.uimg_bytes : 0);
+      mbar_arrive_expect_tx(&c.bar[0], bytes);
+      if (!LAST) {
+        tma_load_2d(sQ, &tmQ, 0, r0, &c.bar[0]);
+        tma_load_2d(sQ + kBlk, &tmQ, 64, r0, &c.bar[0]);
+      }
+      tma_load_2d(sK, &tmK, 0, r0, &c.bar[0]);
+      tma_load_2d(sK + kBlk, &tmK, 64, r0, &c.bar[0]);
+      tma_load_2d(sVT, &tmVT, 0, t * kTile, &c.bar[0]);
+      tma_load_2d(sVT + kBlk, &tmVT, 64, t * kTile, &c.bar[0]);
+      if (u != cur_u) bulk_load(sU, ws + Lw.uimg + (size_t)u * Lw.uimg_bytes, Lw.uimg_bytes, &c.bar[0]);
+    }
+    cur_u = u;
+    mbar_wait(&c.bar[0], lph, status, c.abort_flag);
+    lph ^= 1u;
+    // phase 1: history scores S_h = Q_E,h (s K_Z,h)^T -> TMEM [0, HL);
+    //          link scores, transposed: S'^T = (s Q_Z)_bd K_E^T -> TMEM [128, 256)
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      if (!LAST)
+        for (int h = 0; h < kH; ++h)
+          mma_tile(c.tmem + h * L, smem_u32(sQ + (h >> 1) * kBlk + (h & 1) * 64), kBlk,
+                   smem_u32(sKZ + (h >> 1) * (L * 128) + (h & 1) * 64), L * 128, L, kDH, false);
+      mma_tile(c.tmem + 128, smem_u32(sQBD), kBlk, smem_u32(sK), kBlk, 128, 128, false);
+    }
+    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+    // history softmax over the user's L links, per head -> P in sQ
+    if (!LAST) {
+      for (int h = 0; h < kH; ++h) {
+        float z[L];
+#pragma unroll
+        for (int q = 0; q < L / 16; ++q) tmem_ld16(ta + h * L + q * 16, z + q * 16);
+        tmem_ld_wait();
+        float m = z[0];
+#pragma unroll
+        for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < L; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
+        const float inv = 1.0f / s;
+#pragma unroll
+        for (int k = 0; k < L; ++k) z[k] *= inv;
+#pragma unroll
+        for (int q = 0; q < L / 8; ++q) sw_st16(sQ, kBlk, i, h * L + q * 8, pack8(z + q * 8));
+      }
+    }
+    // link softmax over this tile's valid history rows, per (head, link) lane
+    float lm = 0.f, ls = 0.f;
+    {
+      float z[kTile];
+      tmem_row128(ta + 128, z);
+      float m = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kTile; ++j) {
+        if (j >= nv) z[j] = -INFINITY;
+        m = fmaxf(m, z[j]);
+      }
+      float s = 0.f;
+#pragma unroll
+      for (int j = 0; j < kTile; ++j) {
+        z[j] = j < nv ? __expf(z[j] - m) : 0.f;
+        s += z[j];
+      }
+      lm = m;
+      ls = s;
+      tile_row_st(sK, i, z);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // phase 2: A_E,h = P_h V_Z,h -> TMEM [256, 384); link P2 V_E -> TMEM [384, 512)
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      if (!LAST)
+        for (int h = 0; h < kH; ++h)
+          mma_tile(c.tmem + 256 + h * kDH,
+                   smem_u32(sQ + ((h * L) >> 6) * kBlk + ((h * L) & 63) * 2), kBlk,
+                   smem_u32(sVZT + h * kDH * 128), kBlk, kDH, L, false);
+      mma_tile(c.tmem + 384, smem_u32(sK), kBlk, smem_u32(sVT), kBlk, 128, 128, false);
+    }
+    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+    if (!LAST) {
+      // A_E enters the Wo GEMM as hi + lo bf16 halves (sQ, sK), so the
+      // attention delta keeps close to fp32 accuracy.
+      float a[kD];
+      tmem_row128(ta + 256, a);
+      split_row_st(sQ, sK, kBlk, i, a, kD);
+    }
+    if (i < HL) {  // warp-uniform: HL is a multiple of 32
+      // A warp's lanes may span two heads (L = 16), and tcgen05.ld takes one
+      // address per warp: load the whole row, then keep this lane's head.
+      const int h = i / L;
+      float row[kD], acc[kDH];
+      tmem_row128(ta + 384, row);
+#pragma unroll
+      for (int hh = 0; hh < kH; ++hh)
+        if (hh == h) {
+#pragma unroll
+          for (int cc = 0; cc < kDH; ++cc) acc[cc] = row[hh * kDH + cc];
+        }
+      float* rec = part + (size_t)t * (2 + kDH) * HL;
+      rec[i] = lm;
+      rec[HL + i] = ls;
+#pragma unroll
+      for (int cc = 0; cc < kDH; ++cc) rec[(2 + cc) * HL + i] = acc[cc];
+    }
+    if (!LAST) {
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      // phase 3: Yd = A_E Wo -> TMEM [0, 128)
+      if (threadIdx.x == 0) {
+        tc_fence_after();
+        mma_tile(c.tmem, smem_u32(sQ), kBlk, smem_u32(sWo), kBlk, 128, 128, false);
+        mma_tile(c.tmem, smem_u32(sK), kBlk, smem_u32(sWo), kBlk, 128, 128, true);
+      }
+      cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+      float y[kD];
+      tmem_row128(ta, y);
+      if (i < nv) {
+        float4* dst = reinterpret_cast<float4*>(yd + (int64_t)(r0 + i) * kD);
+#pragma unroll
+        for (int q = 0; q < kD / 4; ++q) dst[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+  }
+  cta_teardown(c);
+}
+
+// ------------------------------------------------------------ link merge
+// b[u, k, h*32 + c] = merge over the user's tiles of (max, sum, acc) records:
+// the link-branch softmax of link k (head h) over all of the user's history.
+// One warp per (user, head, link); lane c owns output column h*32 + c.
+template <int L>
+__global__ void k_link_merge(const uint8_t* __restrict__ ws, LayerWs Lw, int64_t B,
+                             float* __restrict__ bout) {
+  constexpr int HL = kH * L;
+  const int64_t task = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (task >= B * HL) return;
+  const int64_t u = task / HL;
+  const int p = (int)(task % HL), h = p / L, k = p % L;
+  const int* ts = reinterpret_cast<const int*>(ws + Lw.tile_start);
+  const float* part = reinterpret_cast<const float*>(ws + Lw.part);
+  const int t0 = ts[u], t1 = ts[u + 1];
+  float M = -INFINITY, S = 0.f, acc = 0.f;
+  for (int t = t0; t < t1; ++t) {
+    const float* rec = part + (size_t)t * (2 + kDH) * HL;
+    const float m = rec[p], s = rec[HL + p], a = rec[(2 + lane) * HL + p];
+    const float Mn = fmaxf(M, m);
+    const float so = M == -INFINITY ? 0.f : __expf(M - Mn);
+    const float sn = __expf(m - Mn);
+    S = S * so + s * sn;
+    acc = acc * so + a * sn;
+    M = Mn;
+  }
+  bout[(u * L + k) * kD + h * kDH + lane] = S > 0.f ? acc / S : 0.f;
+}
+
+// ------------------------------------------------------- history GatedMLP
+// Per tile: Y = E + Yd (Yd fp32 from the attention kernel; Y kept in TMEM
+// [0,128)), h2 = LN2(Y) in bf16,
+// then for each 64-wide chunk of the hidden layer: G1 = h2 W1c, G3 = h2 W3c
+// (TMEM [128,256)), hid = SiLU(G1) * G3 in bf16, OUT += hid W2c (TMEM
+// [256,384)); E' = Y + OUT.  Chunk weights stream through two 48 KB slots.
+__global__ void __launch_bounds__(128, 1)
+    k_hist_ffn(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ g2, const bf16* __restrict__ b2,
+               const uint8_t* __restrict__ ws, LayerWs Lw, bf16* __restrict__ E_out,
+               unsigned* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1k(smem_raw);
+  uint8_t* sE = sm;                 // E -> h2
+  uint8_t* sY = sm + 2 * kBlk;      // hid chunk
+  uint8_t* sW = sm + 4 * kBlk;      // 2 slots x (W1c 16K, W3c 16K, W2c 16K)
+  constexpr uint32_t kSlot = 3 * kBlk;
+  Cta c;
+  cta_setup(sm + 4 * kBlk + 2 * kSlot, 4, c);  // bar: 0 rows, 1 mma, 2/3 weight slots
+  const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
+  const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
+  const float* yd = reinterpret_cast<const float*>(ws + Lw.yd);
+  uint32_t lph = 0, mph = 0, wph[2] = {0, 0};
+  const int i = threadIdx.x;
+  const uint32_t ta = lane_addr(c);
+  auto load_chunk = [&](int ch) {
+    uint8_t* dst = sW + (ch & 1) * kSlot;
+    mbar_arrive_expect_tx(&c.bar[2 + (ch & 1)], kSlot);
+    bulk_load(dst, ws + Lw.img_1 + ch * kBlk, kBlk, &c.bar[2 + (ch & 1)]);
+    bulk_load(dst + kBlk, ws + Lw.img_3 + ch * kBlk, kBlk, &c.bar[2 + (ch & 1)]);
+    bulk_load(dst + 2 * kBlk, ws + Lw.img_2 + ch * kBlk, kBlk, &c.bar[2 + (ch & 1)]);
+  };
+  for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const int4 tl = tiles[t];
+    const int r0 = tl.y, nv = tl.z;
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
+      tma_load_2d(sE, &tmE, 0, r0, &c.bar[0]);
+      tma_load_2d(sE + kBlk, &tmE, 64, r0, &c.bar[0]);
+      load_chunk(0);
+      load_chunk(1);
+    }
+    mbar_wait(&c.bar[0], lph, status, c.abort_flag);
+    lph ^= 1u;
+    {
+      float y[kD];
+      tile_row_ld(sE, i, y);
+      if (i < nv) {
+        const float4* src = reinterpret_cast<const float4*>(yd + (int64_t)(r0 + i) * kD);
+#pragma unroll
+        for (int q = 0; q < kD / 4; ++q) {
+          const float4 v = src[q];
+          y[4 * q] += v.x; y[4 * q + 1] += v.y; y[4 * q + 2] += v.z; y[4 * q + 3] += v.w;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) tmem_st16(ta + q * 16, y + q * 16);
+      tmem_st_wait();
+      layer_norm_128(y, g2, b2);
+      tile_row_st(sE, i, y);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    for (int ch = 0; ch < kF / 64; ++ch) {
+      const int s = ch & 1;
+      mbar_wait(&c.bar[2 + s], wph[s], status, c.abort_flag);
+      wph[s] ^= 1u;
+      uint8_t* slot = sW + s * kSlot;
+      if (threadIdx.x == 0) {
+        tc_fence_after();
+        mma_tile(c.tmem + 128, smem_u32(sE), kBlk, smem_u32(slot), 8192, 64, 128, false);
+        mma_tile(c.tmem + 192, smem_u32(sE), kBlk, smem_u32(slot + kBlk), 8192, 64, 128, false);
+      }
+      cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+      {
+        float g[64], gg[64];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld16(ta + 128 + q * 16, g + q * 16);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld16(ta + 192 + q * 16, gg + q * 16);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 64; ++k) g[k] = silu_fast(g[k]) * gg[k];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) sw_st16(sY, kBlk, i, q * 8, pack8(g + q * 8));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        tc_fence_after();
+        mma_tile(c.tmem + 256, smem_u32(sY), kBlk, smem_u32(slot + 2 * kBlk), kBlk, 128, 64,
+                 ch > 0);
+      }
+      cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+      if (threadIdx.x == 0 && ch + 2 < kF / 64) load_chunk(ch + 2);
+    }
+    {
+      float y[kD], o[kD];
+      tmem_row128(ta, y);
+      tmem_row128(ta + 256, o);
+#pragma unroll
+      for (int k = 0; k < kD; ++k) y[k] += o[k];
+      if (i < nv) gl_row_st(E_out + (int64_t)(r0 + i) * kD, y);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+  }
+  cta_teardown(c);
+}
+
+// ---------------------------------------------------------- link outputs
+// Link rows, split precision: Y_Z = Z + b Wo, h2 = LN2(Y_Z),
+// Z' = Y_Z + (SiLU(h2 W1) * (h2 W3)) W2.  One CTA per 128 link rows.
+__global__ void __launch_bounds__(128, 1)
+    k_link_out(const bf16* __restrict__ Z, const float* __restrict__ bm, int64_t nrows,
+               const bf16* __restrict__ g2, const bf16* __restrict__ b2,
+               const uint8_t* __restrict__ ws, LayerWs Lw, bf16* __restrict__ Z_out,
+               unsigned* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1k(smem_raw);
+  uint8_t* sAh = sm;
+  uint8_t* sAl = sm + 2 * kBlk;
+  uint8_t* sHh = sm + 4 * kBlk;
+  uint8_t* sHl = sm + 5 * kBlk;
+  uint8_t* sWo = sm + 6 * kBlk;
+  uint8_t* sW = sm + 8 * kBlk;      // one slot: W1c, W3c, W2c
+  Cta c;
+  cta_setup(sm + 11 * kBlk, 3, c);  // bar: 0 Wo, 1 mma, 2 chunk slot
+  uint32_t mph = 0, wph = 0;
+  auto load_chunk = [&](int ch) {
+    mbar_arrive_expect_tx(&c.bar[2], 3 * kBlk);
+    bulk_load(sW, ws + Lw.img_1 + ch * kBlk, kBlk, &c.bar[2]);
+    bulk_load(sW + kBlk, ws + Lw.img_3 + ch * kBlk, kBlk, &c.bar[2]);
+    bulk_load(sW + 2 * kBlk, ws + Lw.img_2 + ch * kBlk, kBlk, &c.bar[2]);
+  };
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
+    bulk_load(sWo, ws + Lw.img_o, 2 * kBlk, &c.bar[0]);
+    load_chunk(0);
+  }
+  const int r = threadIdx.x;
+  const int64_t R = (int64_t)blockIdx.x * kTile + r;
+  const bool valid = R < nrows;
+  const uint32_t ta = lane_addr(c);
+  {
+    float x[kD];
+    if (valid) {
+      const float4* src = reinterpret_cast<const float4*>(bm + R * kD);
+#pragma unroll
+      for (int q = 0; q < kD / 4; ++q) {
+        const float4 v = src[q];
+        x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < kD; ++k) x[k] = 0.f;
+    }
+    split_row_st(sAh, sAl, kBlk, r, x, kD);
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  mbar_wait(&c.bar[0], 0, status, c.abort_flag);
+  if (threadIdx.x == 0) {
+    tc_fence_after();
+    mma_tile(c.tmem, smem_u32(sAh), kBlk, smem_u32(sWo), kBlk, 128, 128, false);
+    mma_tile(c.tmem, smem_u32(sAl), kBlk, smem_u32(sWo), kBlk, 128, 128, true);
+  }
+  cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+  {
+    float y[kD], z[kD];
+    tmem_row128(ta, y);
+    if (valid) gl_row_ld(Z + R * kD, z);
+    else {
+#pragma unroll
+      for (int k = 0; k < kD; ++k) z[k] = 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kD; ++k) y[k] += z[k];
+    layer_norm_128(y, g2, b2);
+    split_row_st(sAh, sAl, kBlk, r, y, kD);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  for (int ch = 0; ch < kF / 64; ++ch) {
+    mbar_wait(&c.bar[2], wph, status, c.abort_flag);
+    wph ^= 1u;
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      mma_tile(c.tmem + 128, smem_u32(sAh), kBlk, smem_u32(sW), 8192, 64, 128, false);
+      mma_tile(c.tmem + 128, smem_u32(sAl), kBlk, smem_u32(sW), 8192, 64, 128, true);
+      mma_tile(c.tmem + 192, smem_u32(sAh), kBlk, smem_u32(sW + kBlk), 8192, 64, 128, false);
+      mma_tile(c.tmem + 192, smem_u32(sAl), kBlk, smem_u32(sW + kBlk), 8192, 64, 128, true);
+    }
+    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+    {
+      float g[64], gg[64];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld16(ta + 128 + q * 16, g + q * 16);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld16(ta + 192 + q * 16, gg + q * 16);
+      tmem_ld_wait();
+#pragma unroll
+      for (int k = 0; k < 64; ++k) g[k] = silu_fast(g[k]) * gg[k];
+      split_row_st(sHh, sHl, kBlk, r, g, 64);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      mma_tile(c.tmem + 256, smem_u32(sHh), kBlk, smem_u32(sW + 2 * kBlk), kBlk, 128, 64, ch > 0);
+      mma_tile(c.tmem + 256, smem_u32(sHl), kBlk, smem_u32(sW + 2 * kBlk), kBlk, 128, 64, true);
+    }
+    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+    if (threadIdx.x == 0 && ch + 1 < kF / 64) load_chunk(ch + 1);
+  }
+  {
+    float y[kD], o[kD], z[kD];
+    tmem_row128(ta, y);          // warp-collective: every thread loads
+    tmem_row128(ta + 256, o);
+    if (valid) {
+      gl_row_ld(Z + R * kD, z);
+#pragma unroll
+      for (int k = 0; k < kD; ++k) y[k] += z[k] + o[k];
+      gl_row_st(Z_out + R * kD, y);
+    }
+  }
+  cta_teardown(c);
+}
+
+constexpr int kBarBytes = 64;
+
+template <class K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+         cudaSuccess;
+}
+
+template <int L>
+int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, const void* E_in,
+              const void* Z_in, const lime_layer_w& w, void* E_out, void* Z_out, uint8_t* ws,
+              unsigned* status, cudaStream_t st) {
+  const LayerWs Lw = layer_ws(L, B, nh);
+  const bool last = E_out == nullptr;
+  const float scale = 1.0f / sqrtf((float)kDH);
+  const int64_t nz = B * L;
+  const int sms = num_sms();
+  {
+    const int64_t n = 4 * kD * kD + 3 * kD * kF;
+    k_prep_weights<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+        (const bf16*)w.Wq, (const bf16*)w.Wk, (const bf16*)w.Wv, (const bf16*)w.Wo,
+        (const bf16*)w.W1, (const bf16*)w.W3, (const bf16*)w.W2, ws, Lw);
+    note_launches(1);
+  }
+  k_schedule<<<1, 1024, 0, st>>>(off, B, nh, (int)Lw.max_tiles, reinterpret_cast<int*>(ws + Lw.sched),
+                                 reinterpret_cast<int4*>(ws + Lw.tiles),
+                                 reinterpret_cast<int*>(ws + Lw.tile_start), status);
+  note_launches(1);
+  {
+    const int smem = 1024 + 10 * kBlk + kBarBytes;
+    if (!set_smem(k_link_proj<L>, smem)) return LIME_ERR_CUDA;
+    k_link_proj<L><<<(unsigned)((nz + kTile - 1) / kTile), 128, smem, st>>>(
+        (const bf16*)Z_in, nz, (const bf16*)w.g1, (const bf16*)w.b1, ws, ws, Lw, scale, status);
+    note_launches(1);
+  }
+  if (nh > 0) {
+    CUtensorMap tmE, tmQ, tmK, tmVT;
+    if (!make_tmap_2d_bf16(&tmE, E_in, kD, (uint64_t)nh, kD * 2, 64, kTile) ||
+        !make_tmap_2d_bf16(&tmQ, ws + Lw.qe, kD, (uint64_t)nh, kD * 2, 64, kTile) ||
+        !make_tmap_2d_bf16(&tmK, ws + Lw.ke, kD, (uint64_t)nh, kD * 2, 64, kTile) ||
+        !make_tmap_2d_bf16(&tmVT, ws + Lw.vt, kD, (uint64_t)Lw.max_tiles * kTile, kD * 2, 64,
+                           kTile))
+      return LIME_ERR_CUDA;
+    const int64_t tiles_hi = Lw.max_tiles;
+    const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
+    if (last) {
+      const int smem = 1024 + 6 * kBlk + kBarBytes;
+      if (!set_smem(k_hist_proj<true>, smem)) return LIME_ERR_CUDA;
+      k_hist_proj<true><<<grid, 128, smem, st>>>(tmE, (const bf16*)w.g1, (const bf16*)w.b1, ws,
+                                                  Lw, status);
+    } else {
+      const int smem = 1024 + 8 * kBlk + kBarBytes;
+      if (!set_smem(k_hist_proj<false>, smem)) return LIME_ERR_CUDA;
+      k_hist_proj<false><<<grid, 128, smem, st>>>(tmE, (const bf16*)w.g1, (const bf16*)w.b1, ws,
+                                                   Lw, status);
+    }
+    note_launches(1);
+    if (last) {
+      const int smem = 1024 + 6 * kBlk + uimg_bytes(L) + kBarBytes;
+      if (!set_smem(k_hist_attn<L, true>, smem)) return LIME_ERR_CUDA;
+      k_hist_attn<L, true><<<grid, 128, smem, st>>>(tmQ, tmK, tmVT, ws, Lw, status);
+    } else {
+      const int smem = 1024 + 8 * kBlk + uimg_bytes(L) + kBarBytes;
+      if (!set_smem(k_hist_attn<L, false>, smem)) return LIME_ERR_CUDA;
+      k_hist_attn<L, false><<<grid, 128, smem, st>>>(tmQ, tmK, tmVT, ws, Lw, status);
+    }
+    note_launches(1);
+    if (!last) {
+      const int smem = 1024 + 10 * kBlk + kBarBytes;
+      if (!set_smem(k_hist_ffn, smem)) return LIME_ERR_CUDA;
+      k_hist_ffn<<<grid, 128, smem, st>>>(tmE, (const bf16*)w.g2, (const bf16*)w.b2, ws, Lw,
+                                          (bf16*)E_out, status);
+      note_launches(1);
+    }
+  }
+  {
+    const int64_t tasks = B * kH * L;
+    k_link_merge<L><<<(unsigned)((tasks * 32 + 255) / 256), 256, 0, st>>>(
+        ws, Lw, B, reinterpret_cast<float*>(ws + Lw.bmerge));
+    note_launches(1);
+  }
+  {
+    const int smem = 1024 + 11 * kBlk + kBarBytes;
+    if (!set_smem(k_link_out, smem)) return LIME_ERR_CUDA;
+    k_link_out<<<(unsigned)((nz + kTile - 1) / kTile), 128, smem, st>>>(
+        (const bf16*)Z_in, reinterpret_cast<const float*>(ws + Lw.bmerge), nz,
+        (const bf16*)w.g2, (const bf16*)w.b2, ws, Lw, (bf16*)Z_out, status);
+    note_launches(1);
+  }
+  return LIME_OK;
+}
+
+}  // namespace
+
+bool fast_layer_supported(const lime_dims& D) {
+  return D.dtype == LIME_BF16 && D.d == kD && D.H == kH && D.f == kF && (D.l == 16 || D.l == 32);
+}
+
+size_t fast_layer_ws_bytes(const lime_dims& D, int64_t B, int64_t total_hist) {
+  if (!fast_layer_supported(D)) return 0;
+  return layer_ws(D.l, B, total_hist).total;
+}
+
+int fast_xor_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh,
+                   const void* E_in, const void* Z_in, const lime_layer_w& w, void* E_out,
+                   void* Z_out, float* ws, unsigned* status, cudaStream_t st) {
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
+  if (D.l == 16) return run_layer<16>(D, B, off, nh, E_in, Z_in, w, E_out, Z_out, wsb, status, st);
+  return run_layer<32>(D, B, off, nh, E_in, Z_in, w, E_out, Z_out, wsb, status, st);
+}
+
+}  // namespace lime

@@ -47,20 +47,31 @@ struct CacheCfg {
 // G^T image: block b (K columns [64b, 64b+64)) of HL rows x 128 bytes,
 // element (row j = h*l + k, K index i) at b*HL*128 + sw128_offset(j, i % 64).
 template <class T>
-__global__ void k_fold_g_img(const T* __restrict__ L, const T* __restrict__ Wq,
-                             const T* __restrict__ Wk, int d, int H, int l, float scale,
-                             bf16* __restrict__ img) {
+__global__ void __launch_bounds__(128) k_fold_g_img(const T* __restrict__ L, const T* __restrict__ Wq,
+                                                    const T* __restrict__ Wk, int d, int H, int l,
+                                                    float scale, bf16* __restrict__ img) {
+  // block j = h*l + k: kc = L_k Wk_c[:, h-cols] (the head-h slice of the
+  // link's key, split over blockDim/d_h partial sums), then G^T row j.
+  __shared__ float part[8][64];
   __shared__ float kc[64];
   const int j = blockIdx.x, h = j / l, k = j % l, dh = d / H, HL = H * l;
-  for (int c = threadIdx.x; c < dh; c += blockDim.x) {
+  const int c = threadIdx.x % dh, q = threadIdx.x / dh, nq = blockDim.x / dh;
+  {
     float acc = 0.f;
-    for (int t = 0; t < d; ++t) acc += to_f(L[(int64_t)k * d + t]) * to_f(Wk[(int64_t)t * d + h * dh + c]);
-    kc[c] = acc;
+    for (int t = q; t < d; t += nq)
+      acc += to_f(L[(int64_t)k * d + t]) * to_f(Wk[(int64_t)t * d + h * dh + c]);
+    part[q][c] = acc;
+  }
+  __syncthreads();
+  if (threadIdx.x < dh) {
+    float s = 0.f;
+    for (int qq = 0; qq < nq; ++qq) s += part[qq][threadIdx.x];
+    kc[threadIdx.x] = s;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
     float acc = 0.f;
-    for (int c = 0; c < dh; ++c) acc += to_f(Wq[(int64_t)i * d + h * dh + c]) * kc[c];
+    for (int cc = 0; cc < dh; ++cc) acc += to_f(Wq[(int64_t)i * d + h * dh + cc]) * kc[cc];
     uint8_t* base = reinterpret_cast<uint8_t*>(img) + (size_t)(i >> 6) * HL * 128;
     *reinterpret_cast<bf16*>(base + sw128_offset(j, i & 63)) = __float2bfloat16_rn(acc * scale);
   }

@@ -132,6 +132,7 @@ int lime_context_links(const lime_dims* dims, int64_t B, const void* L, const vo
   if (B == 0) return LIME_OK;
   if (!L || !ctx || !w || !LC_out || !w->Wc1 || !w->bc1 || !w->Wc2 || !w->bc2)
     return LIME_ERR_ARG;
+  if (!aligned16(w->Wc1) || !aligned16(w->Wc2)) return LIME_ERR_ARG;
   const size_t es = esize(dims);
   const size_t out_sz = (size_t)B * dims->l * dims->d * es;
   if (overlap(LC_out, out_sz, L, (size_t)dims->l * dims->d * es) ||

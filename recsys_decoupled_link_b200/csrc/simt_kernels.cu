@@ -11,33 +11,79 @@ namespace lime {
 
 // ------------------------------------------------------------ context links
 // LC[u,k,:] = SiLU([L_k ; ctx_u] Wc1 + bc1) Wc2 + bc2
-// (LIME note, 整体框架: L^C = MLP(L ⊕ E^C)).  One block per user, one thread
-// per output column; the link loop is sequential.
+// (LIME note, 整体框架: L^C = MLP(L ⊕ E^C)).  Block (u, g) computes links
+// [g*kCtxLinks, (g+1)*kCtxLinks) of user u; each thread owns one output column
+// for kCtxLinks link rows at a time, so every weight read is reused kCtxLinks
+// times.  With `stage` the weights are first copied to shared memory (when
+// they fit); otherwise they are read from global memory.
+constexpr int kCtxLinks = 8;
+
 template <class T>
-__global__ void k_context_links(int d, int c, int l, const T* __restrict__ L,
-                                const T* __restrict__ ctx, const T* __restrict__ Wc1,
-                                const T* __restrict__ bc1, const T* __restrict__ Wc2,
-                                const T* __restrict__ bc2, T* __restrict__ LC) {
+__global__ void __launch_bounds__(128) k_context_links(int d, int c, int l,
+                                                       const T* __restrict__ L,
+                                                       const T* __restrict__ ctx,
+                                                       const T* __restrict__ Wc1,
+                                                       const T* __restrict__ bc1,
+                                                       const T* __restrict__ Wc2,
+                                                       const T* __restrict__ bc2,
+                                                       T* __restrict__ LC, bool stage) {
   extern __shared__ float sm[];
-  float* x = sm;            // [d + c]
-  float* hid = sm + d + c;  // [d]
+  const int din = d + c;
+  float* x = sm;                                     // [kCtxLinks][din]
+  float* hid = x + kCtxLinks * din;                  // [kCtxLinks][d]
+  // staged weights start on a 16-byte boundary
+  T* ws1 = reinterpret_cast<T*>(
+      (reinterpret_cast<uintptr_t>(hid + kCtxLinks * d) + 15) & ~uintptr_t(15));  // [din][d]
+  T* ws2 = ws1 + (size_t)din * d;                    // [d][d] when staged
+  const T* w1 = stage ? ws1 : Wc1;
+  const T* w2 = stage ? ws2 : Wc2;
   const int64_t u = blockIdx.x;
-  for (int i = threadIdx.x; i < c; i += blockDim.x) x[d + i] = to_f(ctx[u * c + i]);
-  for (int k = 0; k < l; ++k) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < d; i += blockDim.x) x[i] = to_f(L[(int64_t)k * d + i]);
-    __syncthreads();
-    for (int j = threadIdx.x; j < d; j += blockDim.x) {
-      float acc = to_f(bc1[j]);
-      for (int i = 0; i < d + c; ++i) acc += x[i] * to_f(Wc1[(int64_t)i * d + j]);
-      hid[j] = silu_f(acc);
+  const int k0 = blockIdx.y * kCtxLinks;
+  const int nk = l - k0 < kCtxLinks ? l - k0 : kCtxLinks;
+  if (stage) {
+    // 16-byte copies, several in flight per thread (d * sizeof(T) % 16 == 0)
+    const int n1 = din * d * (int)sizeof(T) / 16, n2 = d * d * (int)sizeof(T) / 16;
+    const uint4* g1 = reinterpret_cast<const uint4*>(Wc1);
+    const uint4* g2 = reinterpret_cast<const uint4*>(Wc2);
+    uint4* s1 = reinterpret_cast<uint4*>(ws1);
+    uint4* s2 = reinterpret_cast<uint4*>(ws2);
+#pragma unroll 8
+    for (int e = threadIdx.x; e < n1; e += blockDim.x) s1[e] = g1[e];
+#pragma unroll 8
+    for (int e = threadIdx.x; e < n2; e += blockDim.x) s2[e] = g2[e];
+  }
+  for (int e = threadIdx.x; e < kCtxLinks * din; e += blockDim.x) {
+    const int kk = e / din, i = e % din;
+    float v = 0.f;
+    if (kk < nk) v = i < d ? to_f(L[(int64_t)(k0 + kk) * d + i]) : to_f(ctx[u * c + (i - d)]);
+    x[e] = v;
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    float acc[kCtxLinks];
+    const float b = to_f(bc1[j]);
+#pragma unroll
+    for (int kk = 0; kk < kCtxLinks; ++kk) acc[kk] = b;
+    for (int i = 0; i < din; ++i) {
+      const float wv = to_f(w1[(size_t)i * d + j]);
+#pragma unroll
+      for (int kk = 0; kk < kCtxLinks; ++kk) acc[kk] += x[kk * din + i] * wv;
     }
-    __syncthreads();
-    for (int j = threadIdx.x; j < d; j += blockDim.x) {
-      float acc = to_f(bc2[j]);
-      for (int i = 0; i < d; ++i) acc += hid[i] * to_f(Wc2[(int64_t)i * d + j]);
-      LC[(u * l + k) * d + j] = from_f<T>(acc);
+#pragma unroll
+    for (int kk = 0; kk < kCtxLinks; ++kk) hid[kk * d + j] = silu_f(acc[kk]);
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    float acc[kCtxLinks];
+    const float b = to_f(bc2[j]);
+#pragma unroll
+    for (int kk = 0; kk < kCtxLinks; ++kk) acc[kk] = b;
+    for (int i = 0; i < d; ++i) {
+      const float wv = to_f(w2[(size_t)i * d + j]);
+#pragma unroll
+      for (int kk = 0; kk < kCtxLinks; ++kk) acc[kk] += hid[kk * d + i] * wv;
     }
+    for (int kk = 0; kk < nk; ++kk) LC[(u * l + k0 + kk) * d + j] = from_f<T>(acc[kk]);
   }
 }
 
@@ -373,10 +419,16 @@ static inline int grid_for(int64_t n, int per_block, int cap = 148 * 32) {
 template <class T>
 void simt_context_links(const lime_dims& D, int64_t B, const void* L, const void* ctx,
                         const lime_ctx_mlp& w, void* LC, cudaStream_t st) {
-  size_t smem = (size_t)(2 * D.d + D.c) * sizeof(float);
-  k_context_links<T><<<(unsigned)B, 128, smem, st>>>(
+  const int din = D.d + D.c;
+  const size_t small = (size_t)kCtxLinks * (din + D.d) * sizeof(float);
+  const size_t staged = small + 16 + ((size_t)din * D.d + (size_t)D.d * D.d) * sizeof(T);
+  const bool stage = staged <= 200 * 1024;
+  const size_t smem = stage ? staged : small;
+  cudaFuncSetAttribute(k_context_links<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  dim3 grid((unsigned)B, (unsigned)((D.l + kCtxLinks - 1) / kCtxLinks));
+  k_context_links<T><<<grid, 128, smem, st>>>(
       D.d, D.c, D.l, (const T*)L, (const T*)ctx, (const T*)w.Wc1, (const T*)w.bc1,
-      (const T*)w.Wc2, (const T*)w.bc2, (T*)LC);
+      (const T*)w.Wc2, (const T*)w.bc2, (T*)LC, stage);
   note_launches(1);
 }
 

@@ -26,7 +26,9 @@
 //                    softmax statistics (max, sum) and the weighted V sum
 //   k_link_merge     log-sum-exp merge of a user's tile partials -> b (fp32)
 //   k_hist_ffn       Y = E + Yd, LN2, GatedMLP in 64-wide chunks, E' = Y + ·
-//   k_link_out       Y_Z = Z + b·Wo, LN2, GatedMLP, Z' (split precision)
+//   k_link_out       Y_Z = Z + b·Wo, LN2, one GatedMLP chunk per CTA (split
+//                    precision), fp32 partials; k_link_finish sums them -> Z'
+//   (k_link_proj also runs one CTA per (tile, Q|K|V))
 // The last layer (E_out = NULL) skips everything only E' needs: Q_E, the
 // history branch, Wo on history rows and k_hist_ffn.
 //
@@ -45,11 +47,12 @@ namespace {
 constexpr int kD = 128, kH = 4, kDH = 32, kF = 256, kTile = 128;
 constexpr uint32_t kBlk = 128 * 128;  // bytes of one [128 rows x 64 cols] bf16 block
 constexpr float kLnEps = 1e-5f;
+constexpr int kRec = 36;  // floats per link-branch record: max, sum, 32 weighted sums, 2 pad
 
 struct LayerWs {
   size_t img_q, img_k, img_v, img_o, img_1, img_3, img_2;
   size_t sched, tiles, tile_start;
-  size_t qe, ke, vt, yd, uimg, part, bmerge;
+  size_t qe, ke, vt, yd, uimg, part, bmerge, zpart;
   size_t total;
   int64_t max_tiles;
   uint32_t uimg_bytes;
@@ -83,8 +86,9 @@ LayerWs layer_ws(int l, int64_t B, int64_t nh) {
   w.yd = take((size_t)nh * kD * 4);   // fp32 attention delta
   w.uimg_bytes = uimg_bytes(l);
   w.uimg = take((size_t)B * w.uimg_bytes);
-  w.part = take((size_t)w.max_tiles * (2 + kDH) * kH * l * 4);
+  w.part = take((size_t)w.max_tiles * kH * l * kRec * 4);
   w.bmerge = take((size_t)B * l * kD * 4);
+  w.zpart = take((size_t)5 * B * l * kD * 4);
   w.total = o;
   return w;
 }
@@ -149,15 +153,18 @@ __device__ __forceinline__ void split_row_st(uint8_t* hi, uint8_t* lo, uint32_t 
 
 __device__ __forceinline__ float silu_fast(float x) { return x / (1.0f + __expf(-x)); }
 
-// Common CTA prologue: barriers, abort flag, TMEM allocation (512 columns).
+// Common CTA prologue: barriers, abort flag, TMEM allocation (`ncols` columns).
 struct Cta {
   uint64_t* bar;      // [0] loads, [1] mma, [2..3] extra loads
   uint32_t* slot;
   int* abort_flag;
   uint32_t tmem;
+  uint32_t ncols;
 };
 
-__device__ __forceinline__ void cta_setup(uint8_t* bar_area, int nbar, Cta& c) {
+__device__ __forceinline__ void cta_setup(uint8_t* bar_area, int nbar, Cta& c,
+                                          uint32_t ncols = 512) {
+  c.ncols = ncols;
   c.bar = reinterpret_cast<uint64_t*>(bar_area);
   c.slot = reinterpret_cast<uint32_t*>(bar_area + 8 * nbar);
   c.abort_flag = reinterpret_cast<int*>(bar_area + 8 * nbar + 8);
@@ -166,7 +173,7 @@ __device__ __forceinline__ void cta_setup(uint8_t* bar_area, int nbar, Cta& c) {
     *c.abort_flag = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x < 32) tmem_alloc(c.slot, 512);
+  if (threadIdx.x < 32) tmem_alloc(c.slot, ncols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -178,7 +185,7 @@ __device__ __forceinline__ void cta_teardown(Cta& c) {
   __syncthreads();
   if (threadIdx.x < 32) {
     tc_fence_after();
-    tmem_dealloc(c.tmem, 512);
+    tmem_dealloc(c.tmem, c.ncols);
   }
 }
 
@@ -289,87 +296,80 @@ __global__ void k_schedule(const int64_t* __restrict__ off, int64_t B, int64_t n
 //   QZBD [128 rows (h,k) x 128] bf16, 2 blocks of 16 KB: row h*L + k holds
 //        s·Q_Z[k] in head h's 32 columns and zeros elsewhere; rows >= 4L zero
 template <int L>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128)
     k_link_proj(const bf16* __restrict__ Z, int64_t nrows, const bf16* __restrict__ g1,
                 const bf16* __restrict__ b1, const uint8_t* __restrict__ ws_c,
                 uint8_t* __restrict__ ws, LayerWs Lw, float scale, unsigned* status) {
+  // CTA (tile, which): which = 0 -> Q_Z (block-diagonal image), 1 -> K_Z, 2 -> V_Z^T
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
   uint8_t* sAh = sm;
   uint8_t* sAl = sm + 2 * kBlk;
-  uint8_t* sW = sm + 4 * kBlk;  // Wq, Wk, Wv images
+  uint8_t* sW = sm + 4 * kBlk;
+  const int which = blockIdx.y;
   Cta c;
-  cta_setup(sm + 10 * kBlk, 2, c);
+  cta_setup(sm + 6 * kBlk, 2, c, 128);
   uint32_t mph = 0;
   if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(&c.bar[0], 6 * kBlk);
-    bulk_load(sW, ws_c + Lw.img_q, 2 * kBlk, &c.bar[0]);
-    bulk_load(sW + 2 * kBlk, ws_c + Lw.img_k, 2 * kBlk, &c.bar[0]);
-    bulk_load(sW + 4 * kBlk, ws_c + Lw.img_v, 2 * kBlk, &c.bar[0]);
+    const size_t img = which == 0 ? Lw.img_q : which == 1 ? Lw.img_k : Lw.img_v;
+    mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
+    bulk_load(sW, ws_c + img, 2 * kBlk, &c.bar[0]);
   }
   const int r = threadIdx.x;
   const int64_t R = (int64_t)blockIdx.x * kTile + r;
-  float x[kD];
-  if (R < nrows) {
-    gl_row_ld(Z + R * kD, x);
-    layer_norm_128(x, g1, b1);
-  } else {
+  const bool valid = R < nrows;
+  {
+    float x[kD];
+    if (valid) {
+      gl_row_ld(Z + R * kD, x);
+      layer_norm_128(x, g1, b1);
+    } else {
 #pragma unroll
-    for (int i = 0; i < kD; ++i) x[i] = 0.f;
+      for (int i2 = 0; i2 < kD; ++i2) x[i2] = 0.f;
+    }
+    split_row_st(sAh, sAl, kBlk, r, x, kD);
   }
-  split_row_st(sAh, sAl, kBlk, r, x, kD);
   fence_proxy_async_smem();
   __syncthreads();
   mbar_wait(&c.bar[0], 0, status, c.abort_flag);
   if (threadIdx.x == 0) {
     tc_fence_after();
-    for (int w = 0; w < 3; ++w) {
-      const uint32_t bw = smem_u32(sW + w * 2 * kBlk);
-      mma_tile(c.tmem + w * 128, smem_u32(sAh), kBlk, bw, kBlk, 128, 128, false);
-      mma_tile(c.tmem + w * 128, smem_u32(sAl), kBlk, bw, kBlk, 128, 128, true);
-    }
+    mma_tile(c.tmem, smem_u32(sAh), kBlk, smem_u32(sW), kBlk, 128, 128, false);
+    mma_tile(c.tmem, smem_u32(sAl), kBlk, smem_u32(sW), kBlk, 128, 128, true);
   }
   cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-  // TMEM loads are warp-collective: every thread loads, valid rows store.
-  const uint32_t ta = lane_addr(c);
-  const bool valid = R < nrows;
-  const int64_t u = valid ? R / L : 0;
-  const int k = (int)(R % L);
-  uint8_t* img = ws + Lw.uimg + u * Lw.uimg_bytes;
-  uint8_t* kz = img;
-  uint8_t* vzt = img + kz_bytes(L);
-  uint8_t* qbd = vzt + kBlk;
   float v[kD];
-  // s·K_Z row k
-  tmem_row128(ta + 128, v);
+  tmem_row128(lane_addr(c), v);   // warp-collective: every thread loads
   if (valid) {
+    const int64_t u = R / L;
+    const int k = (int)(R % L);
+    uint8_t* img = ws + Lw.uimg + u * Lw.uimg_bytes;
+    if (which == 1) {           // s·K_Z row k
+      uint8_t* kz = img;
 #pragma unroll
-    for (int i = 0; i < kD; ++i) v[i] *= scale;
-    for (int cc = 0; cc < 16; ++cc) sw_st16(kz, (uint32_t)L * 128, k, cc * 8, pack8(v + cc * 8));
-  }
-  // V_Z^T column k (and zero padding columns k + L, k + 2L, ... < 64)
-  tmem_row128(ta + 256, v);
-  if (valid) {
-    for (int cc = 0; cc < kD; ++cc) {
-      *reinterpret_cast<bf16*>(vzt + sw128_offset(cc, k)) = __float2bfloat16_rn(v[cc]);
-      for (int kp = k + L; kp < 64; kp += L)
-        *reinterpret_cast<bf16*>(vzt + sw128_offset(cc, kp)) = __float2bfloat16_rn(0.f);
-    }
-  }
-  // block-diagonal s·Q_Z: rows h*L + k; rows >= 4L are zero
-  tmem_row128(ta, v);
-  if (valid) {
-#pragma unroll
-    for (int i = 0; i < kD; ++i) v[i] *= scale;
-    const float zero8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int h = 0; h < kH; ++h) {
-      for (int cc = 0; cc < 16; ++cc) {
-        const bool mine = (cc >> 2) == h;   // 4 chunks of 8 columns per head
-        sw_st16(qbd, kBlk, h * L + k, cc * 8, pack8(mine ? v + cc * 8 : zero8));
+      for (int i2 = 0; i2 < kD; ++i2) v[i2] *= scale;
+      for (int cc = 0; cc < 16; ++cc) sw_st16(kz, (uint32_t)L * 128, k, cc * 8, pack8(v + cc * 8));
+    } else if (which == 2) {    // V_Z^T column k, zero padding columns k + L, ... < 64
+      uint8_t* vzt = img + kz_bytes(L);
+      for (int cc = 0; cc < kD; ++cc) {
+        *reinterpret_cast<bf16*>(vzt + sw128_offset(cc, k)) = __float2bfloat16_rn(v[cc]);
+        for (int kp = k + L; kp < 64; kp += L)
+          *reinterpret_cast<bf16*>(vzt + sw128_offset(cc, kp)) = __float2bfloat16_rn(0.f);
       }
+    } else {                    // block-diagonal s·Q_Z rows h*L + k; rows >= 4L zero
+      uint8_t* qbd = img + kz_bytes(L) + kBlk;
+#pragma unroll
+      for (int i2 = 0; i2 < kD; ++i2) v[i2] *= scale;
+      const float zero8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int h = 0; h < kH; ++h) {
+        for (int cc = 0; cc < 16; ++cc) {
+          const bool mine = (cc >> 2) == h;   // 4 chunks of 8 columns per head
+          sw_st16(qbd, kBlk, h * L + k, cc * 8, pack8(mine ? v + cc * 8 : zero8));
+        }
+      }
+      for (int p = kH * L + k; p < kTile; p += L)
+        for (int cc = 0; cc < 16; ++cc) sw_st16(qbd, kBlk, p, cc * 8, pack8(zero8));
     }
-    for (int p = kH * L + k; p < kTile; p += L)
-      for (int cc = 0; cc < 16; ++cc) sw_st16(qbd, kBlk, p, cc * 8, pack8(zero8));
   }
   cta_teardown(c);
 }
@@ -596,11 +596,12 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
           for (int cc = 0; cc < kDH; ++cc) acc[cc] = row[hh * kDH + cc];
         }
-      float* rec = part + (size_t)t * (2 + kDH) * HL;
-      rec[i] = lm;
-      rec[HL + i] = ls;
+      float4* rec = reinterpret_cast<float4*>(part + ((size_t)t * HL + i) * kRec);
+      rec[0] = make_float4(lm, ls, acc[0], acc[1]);
 #pragma unroll
-      for (int cc = 0; cc < kDH; ++cc) rec[(2 + cc) * HL + i] = acc[cc];
+      for (int q = 1; q < 8; ++q)
+        rec[q] = make_float4(acc[4 * q - 2], acc[4 * q - 1], acc[4 * q], acc[4 * q + 1]);
+      rec[8] = make_float4(acc[30], acc[31], 0.f, 0.f);
     }
     if (!LAST) {
       fence_proxy_async_smem();
@@ -646,8 +647,8 @@ __global__ void k_link_merge(const uint8_t* __restrict__ ws, LayerWs Lw, int64_t
   const int t0 = ts[u], t1 = ts[u + 1];
   float M = -INFINITY, S = 0.f, acc = 0.f;
   for (int t = t0; t < t1; ++t) {
-    const float* rec = part + (size_t)t * (2 + kDH) * HL;
-    const float m = rec[p], s = rec[HL + p], a = rec[(2 + lane) * HL + p];
+    const float* rec = part + ((size_t)t * HL + p) * kRec;
+    const float m = rec[0], s = rec[1], a = rec[2 + lane];
     const float Mn = fmaxf(M, m);
     const float so = M == -INFINITY ? 0.f : __expf(M - Mn);
     const float sn = __expf(m - Mn);
@@ -659,35 +660,45 @@ __global__ void k_link_merge(const uint8_t* __restrict__ ws, LayerWs Lw, int64_t
 }
 
 // ------------------------------------------------------- history GatedMLP
-// Per tile: Y = E + Yd (Yd fp32 from the attention kernel; Y kept in TMEM
-// [0,128)), h2 = LN2(Y) in bf16,
-// then for each 64-wide chunk of the hidden layer: G1 = h2 W1c, G3 = h2 W3c
-// (TMEM [128,256)), hid = SiLU(G1) * G3 in bf16, OUT += hid W2c (TMEM
-// [256,384)); E' = Y + OUT.  Chunk weights stream through two 48 KB slots.
-__global__ void __launch_bounds__(128, 1)
-    k_hist_ffn(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ g2, const bf16* __restrict__ b2,
+// Per tile: Y = E + Yd (Yd fp32 from the attention kernel), h2 = LN2(Y) in
+// bf16, then for each 64-wide chunk of the hidden layer: G1 = h2 W1c, G3 =
+// h2 W3c (TMEM [0,128)), hid = SiLU(G1) * G3 in bf16, OUT += hid W2c (TMEM
+// [128,256)); E' = Y + OUT with Y re-read from E and Yd.  256 TMEM columns
+// and ~97 KB of shared memory let two CTAs share an SM, so one CTA's waits
+// overlap the other's work.
+__global__ void __launch_bounds__(128, 2)
+    k_hist_ffn(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ E_in,
+               const bf16* __restrict__ g2, const bf16* __restrict__ b2,
                const uint8_t* __restrict__ ws, LayerWs Lw, bf16* __restrict__ E_out,
                unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
   uint8_t* sE = sm;                 // E -> h2
-  uint8_t* sY = sm + 2 * kBlk;      // hid chunk
-  uint8_t* sW = sm + 4 * kBlk;      // 2 slots x (W1c 16K, W3c 16K, W2c 16K)
-  constexpr uint32_t kSlot = 3 * kBlk;
+  uint8_t* sH = sm + 2 * kBlk;      // hid chunk [128 x 64]
+  uint8_t* sW = sm + 3 * kBlk;      // W1c, W3c, W2c
   Cta c;
-  cta_setup(sm + 4 * kBlk + 2 * kSlot, 4, c);  // bar: 0 rows, 1 mma, 2/3 weight slots
+  cta_setup(sm + 6 * kBlk, 3, c, 256);  // bar: 0 rows, 1 mma, 2 weights
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
   const float* yd = reinterpret_cast<const float*>(ws + Lw.yd);
-  uint32_t lph = 0, mph = 0, wph[2] = {0, 0};
+  uint32_t lph = 0, mph = 0, wph = 0;
   const int i = threadIdx.x;
   const uint32_t ta = lane_addr(c);
   auto load_chunk = [&](int ch) {
-    uint8_t* dst = sW + (ch & 1) * kSlot;
-    mbar_arrive_expect_tx(&c.bar[2 + (ch & 1)], kSlot);
-    bulk_load(dst, ws + Lw.img_1 + ch * kBlk, kBlk, &c.bar[2 + (ch & 1)]);
-    bulk_load(dst + kBlk, ws + Lw.img_3 + ch * kBlk, kBlk, &c.bar[2 + (ch & 1)]);
-    bulk_load(dst + 2 * kBlk, ws + Lw.img_2 + ch * kBlk, kBlk, &c.bar[2 + (ch & 1)]);
+    mbar_arrive_expect_tx(&c.bar[2], 3 * kBlk);
+    bulk_load(sW, ws + Lw.img_1 + ch * kBlk, kBlk, &c.bar[2]);
+    bulk_load(sW + kBlk, ws + Lw.img_3 + ch * kBlk, kBlk, &c.bar[2]);
+    bulk_load(sW + 2 * kBlk, ws + Lw.img_2 + ch * kBlk, kBlk, &c.bar[2]);
+  };
+  auto y_row = [&](int64_t row, float* y, bool from_smem) {
+    if (from_smem) tile_row_ld(sE, i, y);
+    else gl_row_ld(E_in + row * kD, y);
+    const float4* src = reinterpret_cast<const float4*>(yd + row * kD);
+#pragma unroll
+    for (int q = 0; q < kD / 4; ++q) {
+      const float4 v = src[q];
+      y[4 * q] += v.x; y[4 * q + 1] += v.y; y[4 * q + 2] += v.z; y[4 * q + 3] += v.w;
+    }
   };
   for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
     const int4 tl = tiles[t];
@@ -697,24 +708,16 @@ __global__ void __launch_bounds__(128, 1)
       tma_load_2d(sE, &tmE, 0, r0, &c.bar[0]);
       tma_load_2d(sE + kBlk, &tmE, 64, r0, &c.bar[0]);
       load_chunk(0);
-      load_chunk(1);
     }
     mbar_wait(&c.bar[0], lph, status, c.abort_flag);
     lph ^= 1u;
     {
       float y[kD];
-      tile_row_ld(sE, i, y);
-      if (i < nv) {
-        const float4* src = reinterpret_cast<const float4*>(yd + (int64_t)(r0 + i) * kD);
+      if (i < nv) y_row(r0 + i, y, true);
+      else {
 #pragma unroll
-        for (int q = 0; q < kD / 4; ++q) {
-          const float4 v = src[q];
-          y[4 * q] += v.x; y[4 * q + 1] += v.y; y[4 * q + 2] += v.z; y[4 * q + 3] += v.w;
-        }
+        for (int k = 0; k < kD; ++k) y[k] = 0.f;
       }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) tmem_st16(ta + q * 16, y + q * 16);
-      tmem_st_wait();
       layer_norm_128(y, g2, b2);
       tile_row_st(sE, i, y);
     }
@@ -722,46 +725,46 @@ __global__ void __launch_bounds__(128, 1)
     tc_fence_before();
     __syncthreads();
     for (int ch = 0; ch < kF / 64; ++ch) {
-      const int s = ch & 1;
-      mbar_wait(&c.bar[2 + s], wph[s], status, c.abort_flag);
-      wph[s] ^= 1u;
-      uint8_t* slot = sW + s * kSlot;
+      mbar_wait(&c.bar[2], wph, status, c.abort_flag);
+      wph ^= 1u;
       if (threadIdx.x == 0) {
         tc_fence_after();
-        mma_tile(c.tmem + 128, smem_u32(sE), kBlk, smem_u32(slot), 8192, 64, 128, false);
-        mma_tile(c.tmem + 192, smem_u32(sE), kBlk, smem_u32(slot + kBlk), 8192, 64, 128, false);
+        mma_tile(c.tmem, smem_u32(sE), kBlk, smem_u32(sW), 8192, 64, 128, false);
+        mma_tile(c.tmem + 64, smem_u32(sE), kBlk, smem_u32(sW + kBlk), 8192, 64, 128, false);
       }
       cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
       {
         float g[64], gg[64];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld16(ta + 128 + q * 16, g + q * 16);
+        for (int q = 0; q < 4; ++q) tmem_ld16(ta + q * 16, g + q * 16);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld16(ta + 192 + q * 16, gg + q * 16);
+        for (int q = 0; q < 4; ++q) tmem_ld16(ta + 64 + q * 16, gg + q * 16);
         tmem_ld_wait();
 #pragma unroll
         for (int k = 0; k < 64; ++k) g[k] = silu_fast(g[k]) * gg[k];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) sw_st16(sY, kBlk, i, q * 8, pack8(g + q * 8));
+        for (int q = 0; q < 8; ++q) sw_st16(sH, kBlk, i, q * 8, pack8(g + q * 8));
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
       if (threadIdx.x == 0) {
         tc_fence_after();
-        mma_tile(c.tmem + 256, smem_u32(sY), kBlk, smem_u32(slot + 2 * kBlk), kBlk, 128, 64,
-                 ch > 0);
+        mma_tile(c.tmem + 128, smem_u32(sH), kBlk, smem_u32(sW + 2 * kBlk), kBlk, 128, 64, ch > 0);
       }
       cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-      if (threadIdx.x == 0 && ch + 2 < kF / 64) load_chunk(ch + 2);
+      if (threadIdx.x == 0 && ch + 1 < kF / 64) load_chunk(ch + 1);
     }
     {
-      float y[kD], o[kD];
-      tmem_row128(ta, y);
-      tmem_row128(ta + 256, o);
+      float o[kD];
+      tmem_row128(ta + 128, o);   // warp-collective: every thread loads
+      if (i < nv) {
+        float y[kD];
+        y_row(r0 + i, y, false);
 #pragma unroll
-      for (int k = 0; k < kD; ++k) y[k] += o[k];
-      if (i < nv) gl_row_st(E_out + (int64_t)(r0 + i) * kD, y);
+        for (int k = 0; k < kD; ++k) y[k] += o[k];
+        gl_row_st(E_out + (int64_t)(r0 + i) * kD, y);
+      }
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -772,11 +775,14 @@ __global__ void __launch_bounds__(128, 1)
 
 // ---------------------------------------------------------- link outputs
 // Link rows, split precision: Y_Z = Z + b Wo, h2 = LN2(Y_Z),
-// Z' = Y_Z + (SiLU(h2 W1) * (h2 W3)) W2.  One CTA per 128 link rows.
+// Z' = Y_Z + (SiLU(h2 W1) * (h2 W3)) W2.  CTA (tile, ch) computes Y_Z's delta
+// b Wo and LN2 for its 128 rows, then GatedMLP chunk ch only, and writes the
+// chunk's fp32 contribution to zpart[ch] (chunk 0 also writes b Wo to
+// zpart[4]); k_link_finish sums them.  Deterministic, no atomics.
 __global__ void __launch_bounds__(128, 1)
     k_link_out(const bf16* __restrict__ Z, const float* __restrict__ bm, int64_t nrows,
                const bf16* __restrict__ g2, const bf16* __restrict__ b2,
-               const uint8_t* __restrict__ ws, LayerWs Lw, bf16* __restrict__ Z_out,
+               const uint8_t* __restrict__ ws_c, LayerWs Lw, float* __restrict__ zpart,
                unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
@@ -785,20 +791,18 @@ __global__ void __launch_bounds__(128, 1)
   uint8_t* sHh = sm + 4 * kBlk;
   uint8_t* sHl = sm + 5 * kBlk;
   uint8_t* sWo = sm + 6 * kBlk;
-  uint8_t* sW = sm + 8 * kBlk;      // one slot: W1c, W3c, W2c
+  uint8_t* sW = sm + 8 * kBlk;      // W1c, W3c, W2c of chunk ch
+  const int ch = blockIdx.y;
   Cta c;
-  cta_setup(sm + 11 * kBlk, 3, c);  // bar: 0 Wo, 1 mma, 2 chunk slot
-  uint32_t mph = 0, wph = 0;
-  auto load_chunk = [&](int ch) {
-    mbar_arrive_expect_tx(&c.bar[2], 3 * kBlk);
-    bulk_load(sW, ws + Lw.img_1 + ch * kBlk, kBlk, &c.bar[2]);
-    bulk_load(sW + kBlk, ws + Lw.img_3 + ch * kBlk, kBlk, &c.bar[2]);
-    bulk_load(sW + 2 * kBlk, ws + Lw.img_2 + ch * kBlk, kBlk, &c.bar[2]);
-  };
+  cta_setup(sm + 11 * kBlk, 3, c);  // bar: 0 Wo, 1 mma, 2 chunk
+  uint32_t mph = 0;
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
-    bulk_load(sWo, ws + Lw.img_o, 2 * kBlk, &c.bar[0]);
-    load_chunk(0);
+    bulk_load(sWo, ws_c + Lw.img_o, 2 * kBlk, &c.bar[0]);
+    mbar_arrive_expect_tx(&c.bar[2], 3 * kBlk);
+    bulk_load(sW, ws_c + Lw.img_1 + ch * kBlk, kBlk, &c.bar[2]);
+    bulk_load(sW + kBlk, ws_c + Lw.img_3 + ch * kBlk, kBlk, &c.bar[2]);
+    bulk_load(sW + 2 * kBlk, ws_c + Lw.img_2 + ch * kBlk, kBlk, &c.bar[2]);
   }
   const int r = threadIdx.x;
   const int64_t R = (int64_t)blockIdx.x * kTile + r;
@@ -831,6 +835,11 @@ __global__ void __launch_bounds__(128, 1)
   {
     float y[kD], z[kD];
     tmem_row128(ta, y);
+    if (valid && ch == 0) {
+      float4* dst = reinterpret_cast<float4*>(zpart + ((size_t)4 * nrows + R) * kD);
+#pragma unroll
+      for (int q = 0; q < kD / 4; ++q) dst[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+    }
     if (valid) gl_row_ld(Z + R * kD, z);
     else {
 #pragma unroll
@@ -844,51 +853,58 @@ __global__ void __launch_bounds__(128, 1)
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
-  for (int ch = 0; ch < kF / 64; ++ch) {
-    mbar_wait(&c.bar[2], wph, status, c.abort_flag);
-    wph ^= 1u;
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      mma_tile(c.tmem + 128, smem_u32(sAh), kBlk, smem_u32(sW), 8192, 64, 128, false);
-      mma_tile(c.tmem + 128, smem_u32(sAl), kBlk, smem_u32(sW), 8192, 64, 128, true);
-      mma_tile(c.tmem + 192, smem_u32(sAh), kBlk, smem_u32(sW + kBlk), 8192, 64, 128, false);
-      mma_tile(c.tmem + 192, smem_u32(sAl), kBlk, smem_u32(sW + kBlk), 8192, 64, 128, true);
-    }
-    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    {
-      float g[64], gg[64];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld16(ta + 128 + q * 16, g + q * 16);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld16(ta + 192 + q * 16, gg + q * 16);
-      tmem_ld_wait();
-#pragma unroll
-      for (int k = 0; k < 64; ++k) g[k] = silu_fast(g[k]) * gg[k];
-      split_row_st(sHh, sHl, kBlk, r, g, 64);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      mma_tile(c.tmem + 256, smem_u32(sHh), kBlk, smem_u32(sW + 2 * kBlk), kBlk, 128, 64, ch > 0);
-      mma_tile(c.tmem + 256, smem_u32(sHl), kBlk, smem_u32(sW + 2 * kBlk), kBlk, 128, 64, true);
-    }
-    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    if (threadIdx.x == 0 && ch + 1 < kF / 64) load_chunk(ch + 1);
+  mbar_wait(&c.bar[2], 0, status, c.abort_flag);
+  if (threadIdx.x == 0) {
+    tc_fence_after();
+    mma_tile(c.tmem + 128, smem_u32(sAh), kBlk, smem_u32(sW), 8192, 64, 128, false);
+    mma_tile(c.tmem + 128, smem_u32(sAl), kBlk, smem_u32(sW), 8192, 64, 128, true);
+    mma_tile(c.tmem + 192, smem_u32(sAh), kBlk, smem_u32(sW + kBlk), 8192, 64, 128, false);
+    mma_tile(c.tmem + 192, smem_u32(sAl), kBlk, smem_u32(sW + kBlk), 8192, 64, 128, true);
   }
+  cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
   {
-    float y[kD], o[kD], z[kD];
-    tmem_row128(ta, y);          // warp-collective: every thread loads
-    tmem_row128(ta + 256, o);
-    if (valid) {
-      gl_row_ld(Z + R * kD, z);
+    float g[64], gg[64];
 #pragma unroll
-      for (int k = 0; k < kD; ++k) y[k] += z[k] + o[k];
-      gl_row_st(Z_out + R * kD, y);
+    for (int q = 0; q < 4; ++q) tmem_ld16(ta + 128 + q * 16, g + q * 16);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) tmem_ld16(ta + 192 + q * 16, gg + q * 16);
+    tmem_ld_wait();
+#pragma unroll
+    for (int k = 0; k < 64; ++k) g[k] = silu_fast(g[k]) * gg[k];
+    split_row_st(sHh, sHl, kBlk, r, g, 64);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    tc_fence_after();
+    mma_tile(c.tmem + 256, smem_u32(sHh), kBlk, smem_u32(sW + 2 * kBlk), kBlk, 128, 64, false);
+    mma_tile(c.tmem + 256, smem_u32(sHl), kBlk, smem_u32(sW + 2 * kBlk), kBlk, 128, 64, true);
+  }
+  cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+  {
+    float o[kD];
+    tmem_row128(ta + 256, o);    // warp-collective: every thread loads
+    if (valid) {
+      float4* dst = reinterpret_cast<float4*>(zpart + ((size_t)ch * nrows + R) * kD);
+#pragma unroll
+      for (int q = 0; q < kD / 4; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
     }
   }
   cta_teardown(c);
+}
+
+// Z' = Z + (b Wo) + sum of the four GatedMLP chunk contributions, in bf16.
+__global__ void k_link_finish(const bf16* __restrict__ Z, const float* __restrict__ zpart,
+                              int64_t nrows, bf16* __restrict__ Z_out) {
+  const int64_t n = nrows * kD;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    float v = __bfloat162float(Z[e]) + zpart[4 * n + e];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v += zpart[q * n + e];
+    Z_out[e] = __float2bfloat16_rn(v);
+  }
 }
 
 constexpr int kBarBytes = 64;
@@ -920,9 +936,9 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
                                  reinterpret_cast<int*>(ws + Lw.tile_start), status);
   note_launches(1);
   {
-    const int smem = 1024 + 10 * kBlk + kBarBytes;
+    const int smem = 1024 + 6 * kBlk + kBarBytes;
     if (!set_smem(k_link_proj<L>, smem)) return LIME_ERR_CUDA;
-    k_link_proj<L><<<(unsigned)((nz + kTile - 1) / kTile), 128, smem, st>>>(
+    k_link_proj<L><<<dim3((unsigned)((nz + kTile - 1) / kTile), 3), 128, smem, st>>>(
         (const bf16*)Z_in, nz, (const bf16*)w.g1, (const bf16*)w.b1, ws, ws, Lw, scale, status);
     note_launches(1);
   }
@@ -959,10 +975,11 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     }
     note_launches(1);
     if (!last) {
-      const int smem = 1024 + 10 * kBlk + kBarBytes;
+      const int smem = 1024 + 6 * kBlk + kBarBytes;
       if (!set_smem(k_hist_ffn, smem)) return LIME_ERR_CUDA;
-      k_hist_ffn<<<grid, 128, smem, st>>>(tmE, (const bf16*)w.g2, (const bf16*)w.b2, ws, Lw,
-                                          (bf16*)E_out, status);
+      const int g2 = (int)(tiles_hi < 2 * sms ? tiles_hi : 2 * sms);
+      k_hist_ffn<<<g2, 128, smem, st>>>(tmE, (const bf16*)E_in, (const bf16*)w.g2,
+                                        (const bf16*)w.b2, ws, Lw, (bf16*)E_out, status);
       note_launches(1);
     }
   }
@@ -975,9 +992,14 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
   {
     const int smem = 1024 + 11 * kBlk + kBarBytes;
     if (!set_smem(k_link_out, smem)) return LIME_ERR_CUDA;
-    k_link_out<<<(unsigned)((nz + kTile - 1) / kTile), 128, smem, st>>>(
+    float* zpart = reinterpret_cast<float*>(ws + Lw.zpart);
+    k_link_out<<<dim3((unsigned)((nz + kTile - 1) / kTile), kF / 64), 128, smem, st>>>(
         (const bf16*)Z_in, reinterpret_cast<const float*>(ws + Lw.bmerge), nz,
-        (const bf16*)w.g2, (const bf16*)w.b2, ws, Lw, (bf16*)Z_out, status);
+        (const bf16*)w.g2, (const bf16*)w.b2, ws, Lw, zpart, status);
+    note_launches(1);
+    const int64_t n = nz * kD;
+    k_link_finish<<<(unsigned)((n + 255) / 256 < 148 * 8 ? (n + 255) / 256 : 148 * 8), 256, 0, st>>>(
+        (const bf16*)Z_in, zpart, nz, (bf16*)Z_out);
     note_launches(1);
   }
   return LIME_OK;

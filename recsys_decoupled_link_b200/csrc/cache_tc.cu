@@ -13,9 +13,10 @@
 //   warp 0     TMA producer: 128-row tiles of T into a STAGES-deep ring
 //   warp 1     tcgen05.mma issuer (M=128, N=H*l, K=128 as 8 K-steps) into one
 //              of two TMEM accumulators
-//   warps 2-5  epilogue: tcgen05.ld of its row, softmax per head over l
-//              links in fp32, bf16 into a 128-byte-swizzled staging tile,
-//              TMA store of the tile (rows past n_items are clipped by TMA)
+//   warps 2-9  epilogue, two warps per TMEM lane quadrant each taking half of
+//              the heads: tcgen05.ld of its row, softmax per head over l links
+//              in fp32, bf16 into a 128-byte-swizzled staging tile, TMA store
+//              of the tile (rows past n_items are clipped by TMA)
 // Every wait is bounded; a timeout sets LIME_FLAG_TIMEOUT and the CTA drains
 // and returns.  The catalogue read is the roofline: 2*(d + H*l) bytes/item.
 #include "lime_fast.cuh"
@@ -78,7 +79,7 @@ __global__ void __launch_bounds__(128) k_fold_g_img(const T* __restrict__ L, con
 }
 
 template <int HL, int L>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     k_cache_tc(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmC,
                const bf16* __restrict__ gimg, int n_tiles, unsigned* status) {
   using C = CacheCfg<HL>;
@@ -105,8 +106,8 @@ __global__ void __launch_bounds__(192, 1)
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
-      mbar_init(&ofull[a], 128);
+      mbar_init(&tempty[a], 256);
+      mbar_init(&ofull[a], 256);
       mbar_init(&ofree[a], 1);
     }
     mbar_init(bready, 1);
@@ -171,9 +172,11 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(mdone, 0, status, &abort_flag);
     }
   } else {
-    // epilogue: 128 threads, thread owns TMEM lane / tile row `row`
+    // epilogue: 8 warps, two per TMEM lane quadrant; the warp's lane is tile row
+    // `row` and it handles half of the heads (half = 0 for warps 2-5, 1 for 6-9)
     const int et = threadIdx.x - 64;
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     int it = 0;
@@ -187,7 +190,7 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       uint8_t* stage = sO + ob * C::O_BYTES;
 #pragma unroll 1
-      for (int h = 0; h < H; ++h) {
+      for (int h = half * (H / 2); h < (half + 1) * (H / 2); ++h) {
         float z[L];
 #pragma unroll
         for (int q = 0; q < L / 16; ++q)
@@ -254,7 +257,7 @@ int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, unsigne
     return LIME_ERR_CUDA;
   const int n_tiles = (int)((n + kBM - 1) / kBM);
   const int grid = n_tiles < num_sms() ? n_tiles : num_sms();
-  k_cache_tc<HL, L><<<grid, 192, C::SMEM, st>>>(tmT, tmC, img, n_tiles, status);
+  k_cache_tc<HL, L><<<grid, 320, C::SMEM, st>>>(tmT, tmC, img, n_tiles, status);
   note_launches(1);
   return LIME_OK;
 }
@@ -284,7 +287,6 @@ int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void
   switch (HL * 1000 + D.l) {
     case 64016: return launch_cache<64, 16>(T, n, img, cache, status, st);
     case 64032: return launch_cache<64, 32>(T, n, img, cache, status, st);
-    case 64064: return launch_cache<64, 64>(T, n, img, cache, status, st);
     case 128016: return launch_cache<128, 16>(T, n, img, cache, status, st);
     case 128032: return launch_cache<128, 32>(T, n, img, cache, status, st);
     case 128064: return launch_cache<128, 64>(T, n, img, cache, status, st);

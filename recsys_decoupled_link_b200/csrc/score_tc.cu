@@ -13,9 +13,11 @@
 // CTA (u, g) stages L^P_u^T once (a [128 c x 64 k] 128B-swizzled block, k >= l
 // zero) and walks tiles g, g + G, ... of user u's candidates.  Per tile each
 // thread gathers one candidate's row with 16-byte loads into the swizzled A
-// tile (an out-of-range ID gives a zero row and LIME_FLAG_BAD_ID), thread 0
-// issues one MMA group per head into TMEM, and each thread stores its row of
-// O as bf16.  No workspace is used.
+// tile (an out-of-range ID gives a zero row and LIME_FLAG_BAD_ID) — the
+// threads of a warp cover whole rows, so the gather is coalesced — thread 0
+// issues one MMA group per head into TMEM, each thread stages its row of O in
+// bf16, and the tile is written back with coalesced 16-byte stores.  No
+// workspace is used.
 #include "lime_fast.cuh"
 #include "sm100.cuh"
 
@@ -34,7 +36,9 @@ __global__ void __launch_bounds__(128)
                const int64_t* __restrict__ off, int64_t B, int64_t total,
                const bf16* __restrict__ LP, bf16* __restrict__ O, unsigned* status) {
   constexpr int HL = kH * L;
-  constexpr int ABLK = HL / 64;             // A blocks of 64 columns
+  // A tile blocks of 64 columns; at least 2 because the same region later
+  // stages the [128 x 128] output tile
+  constexpr int ABLK = HL / 64 < 2 ? 2 : HL / 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = sm;
@@ -42,6 +46,7 @@ __global__ void __launch_bounds__(128)
   uint64_t* bar = reinterpret_cast<uint64_t*>(sB + kBlk);
   uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 1);
   int* abort_flag = reinterpret_cast<int*>(bar + 2);
+  int64_t* s_ids = reinterpret_cast<int64_t*>(bar + 4);   // [128] candidate IDs of the tile
 
   const int64_t u = blockIdx.x;
   int64_t a, b;
@@ -56,12 +61,26 @@ __global__ void __launch_bounds__(128)
     fence_mbar_init();
   }
   if (i < 32) tmem_alloc(slot, 128);
-  // L^P_u transposed: thread i owns output column c = i
+  // L^P_u transposed into sB: element (c, k) at sw128_offset(c, k), k >= L zero.
+  // Coalesced 16-byte copies of L^P_u into the (still unused) A tile, then each
+  // thread builds its own row c of the transpose with 16-byte swizzled stores.
   {
-    const bf16* lp = LP + (u * L) * kD + i;
-    for (int k = 0; k < 64; ++k)
-      *reinterpret_cast<bf16*>(sB + sw128_offset(i, k)) =
-          k < L ? lp[(int64_t)k * kD] : __float2bfloat16_rn(0.f);
+    const uint4* lp = reinterpret_cast<const uint4*>(LP + (u * L) * kD);
+    uint4* stage = reinterpret_cast<uint4*>(sA);   // [L][128] bf16, plain row-major
+#pragma unroll
+    for (int q = 0; q < L * kD / 8 / 128; ++q) stage[q * 128 + i] = __ldg(lp + q * 128 + i);
+    __syncthreads();
+    const bf16* st = reinterpret_cast<const bf16*>(sA);
+#pragma unroll
+    for (int k8 = 0; k8 < 8; ++k8) {
+      float f[8];
+#pragma unroll
+      for (int z = 0; z < 8; ++z) {
+        const int k = k8 * 8 + z;
+        f[z] = k < L ? __bfloat162float(st[k * kD + i]) : 0.f;
+      }
+      sw_st16(sB, kBlk, i, k8 * 8, pack8(f));
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -81,12 +100,26 @@ __global__ void __launch_bounds__(128)
           id = -1;
         }
       }
-      uint4 v[HL / 8];
-      const uint4* src = reinterpret_cast<const uint4*>(cache + (id < 0 ? 0 : id) * HL);
+      s_ids[i] = id;
+    }
+    __syncthreads();
+    // cooperative gather: 16-byte chunk q*128 + i is chunk (idx % CH) of row idx / CH,
+    // so a warp reads whole cache rows (coalesced) instead of one row per thread
+    {
+      constexpr int CH = HL / 8;               // 16-byte chunks per cache row
+      uint4 v[CH];
 #pragma unroll
-      for (int c = 0; c < HL / 8; ++c) v[c] = id < 0 ? make_uint4(0, 0, 0, 0) : __ldg(src + c);
+      for (int q = 0; q < CH; ++q) {
+        const int idx = q * 128 + i, r = idx / CH, cc = idx % CH;
+        const int64_t id = s_ids[r];
+        v[q] = id < 0 ? make_uint4(0, 0, 0, 0)
+                      : __ldg(reinterpret_cast<const uint4*>(cache + id * HL) + cc);
+      }
 #pragma unroll
-      for (int c = 0; c < HL / 8; ++c) sw_st16(sA, kBlk, i, c * 8, v[c]);
+      for (int q = 0; q < CH; ++q) {
+        const int idx = q * 128 + i, r = idx / CH, cc = idx % CH;
+        sw_st16(sA, kBlk, r, cc * 8, v[q]);
+      }
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -102,17 +135,25 @@ __global__ void __launch_bounds__(128)
     mbar_wait(bar, ph, status, abort_flag);
     ph ^= 1u;
     tc_fence_after();
-    float row[kD];
+    {
+      // thread = row: TMEM -> bf16 -> swizzled staging in sA (the MMA is done with it)
+      float row[kD];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) tmem_ld16(ta + q * 16, row + q * 16);
-    tmem_ld_wait();
-    if (i < nv) {
-      uint4* dst = reinterpret_cast<uint4*>(O + (m0 + i) * kD);
+      for (int q = 0; q < 8; ++q) tmem_ld16(ta + q * 16, row + q * 16);
+      tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < 16; ++c) dst[c] = pack8(row + c * 8);
+      for (int c = 0; c < 16; ++c) sw_st16(sA, kBlk, i, c * 8, pack8(row + c * 8));
     }
     tc_fence_before();
-    __syncthreads();   // TMEM and the A tile are reused by the next tile
+    __syncthreads();
+    // cooperative, coalesced store of the valid rows
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int idx = q * 128 + i, r = idx / 16, cc = idx % 16;
+      if (r < nv)
+        reinterpret_cast<uint4*>(O + (m0 + r) * kD)[cc] = sw_ld16(sA, kBlk, r, cc * 8);
+    }
+    __syncthreads();   // sA, s_ids and TMEM are reused by the next tile
   }
   if (i < 32) {
     tc_fence_after();
@@ -125,7 +166,7 @@ int launch_score(int64_t B, const void* cache, int64_t n_items, const int32_t* i
                  const int64_t* off, int64_t total, const void* LP, void* O, unsigned* status,
                  cudaStream_t st) {
   constexpr int HL = kH * L;
-  const int smem = 1024 + (HL / 64 + 1) * kBlk + 64;
+  const int smem = 1024 + ((HL / 64 < 2 ? 2 : HL / 64) + 1) * kBlk + 64 + 128 * 8;
   if (cudaFuncSetAttribute(k_score_tc<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return LIME_ERR_CUDA;

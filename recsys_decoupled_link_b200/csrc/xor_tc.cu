@@ -19,7 +19,8 @@
 //                    operand images: s·K_Z, V_Z^T, and s·Q_Z laid out
 //                    block-diagonally over heads so that one MMA yields the
 //                    link branch's scores transposed (links on TMEM lanes)
-//   k_hist_proj      LN1(E) -> Q_E, K_E (row-major) and V_E^T (per tile)
+//   k_hist_proj      LN1(E) (split precision) -> Q_E, K_E (row-major) and
+//                    V_E^T (per tile)
 //   k_hist_attn      history branch: softmax over the user's l links, P·V_Z,
 //                    then (P·V_Z)·Wo -> Yd (fp32 attention delta);
 //                    link branch: per tile and (head, link) the partial
@@ -62,7 +63,7 @@ __host__ __device__ constexpr size_t up1k(size_t x) { return (x + 1023) & ~(size
 
 __host__ __device__ constexpr uint32_t kz_bytes(int l) { return (uint32_t)l * 256; }  // [l x 128] bf16
 __host__ __device__ constexpr uint32_t uimg_bytes(int l) {
-  return (uint32_t)up1k(kz_bytes(l) + kBlk + 2 * kBlk);
+  return (uint32_t)up1k(kz_bytes(l) + kBlk + 4 * kBlk);   // KZ, VZT, QBD hi, QBD lo
 }
 
 LayerWs layer_ws(int l, int64_t B, int64_t nh) {
@@ -294,7 +295,9 @@ __global__ void k_schedule(const int64_t* __restrict__ off, int64_t B, int64_t n
 //   KZ   [L rows x 128] bf16, 2 blocks of L*128 bytes:  s·K_Z
 //   VZT  [128 rows (c) x 64 cols (k)] bf16, 1 block:     V_Z^T, k >= L zero
 //   QZBD [128 rows (h,k) x 128] bf16, 2 blocks of 16 KB: row h*L + k holds
-//        s·Q_Z[k] in head h's 32 columns and zeros elsewhere; rows >= 4L zero
+//        s·Q_Z[k] in head h's 32 columns and zeros elsewhere; rows >= 4L zero;
+//        stored twice, as the hi and lo bf16 halves of the fp32 value (the
+//        link query is one vector per link, so its rounding is not averaged)
 template <int L>
 __global__ void __launch_bounds__(128)
     k_link_proj(const bf16* __restrict__ Z, int64_t nrows, const bf16* __restrict__ g1,
@@ -356,19 +359,29 @@ __global__ void __launch_bounds__(128)
         for (int kp = k + L; kp < 64; kp += L)
           *reinterpret_cast<bf16*>(vzt + sw128_offset(cc, kp)) = __float2bfloat16_rn(0.f);
       }
-    } else {                    // block-diagonal s·Q_Z rows h*L + k; rows >= 4L zero
+    } else {                    // block-diagonal s·Q_Z rows h*L + k (hi, lo); rows >= 4L zero
       uint8_t* qbd = img + kz_bytes(L) + kBlk;
+      uint8_t* qbl = qbd + 2 * kBlk;
+      float lo[kD];
 #pragma unroll
-      for (int i2 = 0; i2 < kD; ++i2) v[i2] *= scale;
+      for (int i2 = 0; i2 < kD; ++i2) {
+        const float x = v[i2] * scale;
+        v[i2] = __bfloat162float(__float2bfloat16_rn(x));
+        lo[i2] = x - v[i2];
+      }
       const float zero8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       for (int h = 0; h < kH; ++h) {
         for (int cc = 0; cc < 16; ++cc) {
           const bool mine = (cc >> 2) == h;   // 4 chunks of 8 columns per head
           sw_st16(qbd, kBlk, h * L + k, cc * 8, pack8(mine ? v + cc * 8 : zero8));
+          sw_st16(qbl, kBlk, h * L + k, cc * 8, pack8(mine ? lo + cc * 8 : zero8));
         }
       }
       for (int p = kH * L + k; p < kTile; p += L)
-        for (int cc = 0; cc < 16; ++cc) sw_st16(qbd, kBlk, p, cc * 8, pack8(zero8));
+        for (int cc = 0; cc < 16; ++cc) {
+          sw_st16(qbd, kBlk, p, cc * 8, pack8(zero8));
+          sw_st16(qbl, kBlk, p, cc * 8, pack8(zero8));
+        }
     }
   }
   cta_teardown(c);
@@ -387,11 +400,12 @@ __global__ void __launch_bounds__(128, 1)
                 unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
-  uint8_t* sE = sm;
-  uint8_t* sW = sm + 2 * kBlk;   // [Wq,] Wk, Wv images
+  uint8_t* sE = sm;               // E tile -> LN1 output, hi half
+  uint8_t* sEl = sm + 2 * kBlk;    // LN1 output, lo half
+  uint8_t* sW = sm + 4 * kBlk;     // [Wq,] Wk, Wv images
   constexpr int NW = LAST ? 2 : 3;
   Cta c;
-  cta_setup(sm + (2 + 2 * NW) * kBlk, 3, c);
+  cta_setup(sm + (4 + 2 * NW) * kBlk, 3, c);
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
   bf16* qe = reinterpret_cast<bf16*>(ws + Lw.qe);
@@ -420,18 +434,22 @@ __global__ void __launch_bounds__(128, 1)
     mbar_wait(&c.bar[0], eph, status, c.abort_flag);
     eph ^= 1u;
     {
+      // LN1 output as hi + lo bf16 halves: K_E and V_E feed the link branch,
+      // whose softmax over a short history does not average rounding away
       float x[kD];
       tile_row_ld(sE, i, x);
       layer_norm_128(x, g1, b1);
-      tile_row_st(sE, i, x);
+      split_row_st(sE, sEl, kBlk, i, x, kD);
     }
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {
       tc_fence_after();
-      for (int w = 0; w < NW; ++w)
-        mma_tile(c.tmem + (LAST ? w + 1 : w) * 128, smem_u32(sE), kBlk,
-                 smem_u32(sW + w * 2 * kBlk), kBlk, 128, 128, false);
+      for (int w = 0; w < NW; ++w) {
+        const uint32_t d = c.tmem + (LAST ? w + 1 : w) * 128;
+        mma_tile(d, smem_u32(sE), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128, 128, false);
+        mma_tile(d, smem_u32(sEl), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128, 128, true);
+      }
     }
     cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
     const int tn = t + gridDim.x;
@@ -520,6 +538,7 @@ __global__ void __launch_bounds__(128, 1)
           mma_tile(c.tmem + h * L, smem_u32(sQ + (h >> 1) * kBlk + (h & 1) * 64), kBlk,
                    smem_u32(sKZ + (h >> 1) * (L * 128) + (h & 1) * 64), L * 128, L, kDH, false);
       mma_tile(c.tmem + 128, smem_u32(sQBD), kBlk, smem_u32(sK), kBlk, 128, 128, false);
+      mma_tile(c.tmem + 128, smem_u32(sQBD + 2 * kBlk), kBlk, smem_u32(sK), kBlk, 128, 128, true);
     }
     cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
     // history softmax over the user's L links, per head -> P in sQ
@@ -953,12 +972,12 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     const int64_t tiles_hi = Lw.max_tiles;
     const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
     if (last) {
-      const int smem = 1024 + 6 * kBlk + kBarBytes;
+      const int smem = 1024 + 8 * kBlk + kBarBytes;
       if (!set_smem(k_hist_proj<true>, smem)) return LIME_ERR_CUDA;
       k_hist_proj<true><<<grid, 128, smem, st>>>(tmE, (const bf16*)w.g1, (const bf16*)w.b1, ws,
                                                   Lw, status);
     } else {
-      const int smem = 1024 + 8 * kBlk + kBarBytes;
+      const int smem = 1024 + 10 * kBlk + kBarBytes;
       if (!set_smem(k_hist_proj<false>, smem)) return LIME_ERR_CUDA;
       k_hist_proj<false><<<grid, 128, smem, st>>>(tmE, (const bf16*)w.g1, (const bf16*)w.b1, ws,
                                                    Lw, status);

@@ -113,6 +113,13 @@ def test_edge_cases(base):
     check_workload(w, n_hist=n_hist, n_cand=n_cand)
 
 
+@pytest.mark.parametrize("l", [16, 32, 64])
+def test_scoring_many_tiles_per_user(l):
+    # few users with many candidates: each scoring CTA walks several tiles
+    w = synth.workload("standard", B=2, l=l, n_items=20_000, layers=1, cand=("uniform",))
+    check_workload(w, n_hist=[130, 40], n_cand=[5000, 3333])
+
+
 def test_single_user_single_token():
     w = synth.workload("standard", B=1, n_items=1000, layers=1)
     check_workload(w, n_hist=[1], n_cand=[1])

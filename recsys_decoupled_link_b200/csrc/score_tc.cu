@@ -61,14 +61,21 @@ __global__ void __launch_bounds__(128)
     fence_mbar_init();
   }
   if (i < 32) tmem_alloc(slot, 128);
+  // The first tile's candidate ID is loaded together with L^P_u (one memory
+  // round trip for both).
+  int32_t first_id = -1;
+  if ((int64_t)i < b - (a + (int64_t)blockIdx.y * kTile)) first_id = ids[a + (int64_t)blockIdx.y * kTile + i];
   // L^P_u transposed into sB: element (c, k) at sw128_offset(c, k), k >= L zero.
   // Coalesced 16-byte copies of L^P_u into the (still unused) A tile, then each
   // thread builds its own row c of the transpose with 16-byte swizzled stores.
   {
     const uint4* lp = reinterpret_cast<const uint4*>(LP + (u * L) * kD);
     uint4* stage = reinterpret_cast<uint4*>(sA);   // [L][128] bf16, plain row-major
+    uint4 lv[L * kD / 8 / 128];
 #pragma unroll
-    for (int q = 0; q < L * kD / 8 / 128; ++q) stage[q * 128 + i] = __ldg(lp + q * 128 + i);
+    for (int q = 0; q < L * kD / 8 / 128; ++q) lv[q] = __ldg(lp + q * 128 + i);
+#pragma unroll
+    for (int q = 0; q < L * kD / 8 / 128; ++q) stage[q * 128 + i] = lv[q];
     __syncthreads();
     const bf16* st = reinterpret_cast<const bf16*>(sA);
 #pragma unroll
@@ -94,7 +101,7 @@ __global__ void __launch_bounds__(128)
     {
       int64_t id = -1;
       if (i < nv) {
-        id = ids[m0 + i];
+        id = t == (int)blockIdx.y ? first_id : ids[m0 + i];
         if (id < 0 || id >= n_items) {
           raise_flag(status, LIME_FLAG_BAD_ID);
           id = -1;

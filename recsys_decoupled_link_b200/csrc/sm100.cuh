@@ -294,3 +294,44 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
 
 }  // namespace sm100
 }  // namespace lime
+
+namespace lime {
+namespace sm100 {
+
+// Shared-memory descriptor of an MN-major operand in the 128-byte-swizzled
+// layout: each K row holds 64 MN elements in 128 bytes, 8 K rows form a
+// 1024-byte atom (stride between 8-row groups 1024 bytes), and consecutive
+// 64-wide MN blocks are `lbo` bytes apart.  This is the byte image of a
+// row-major [K x MN] tile stored as [rows x 64] swizzled blocks; a K step of
+// 16 rows advances the start address by 2048 bytes.
+__device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t addr, uint32_t lbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// D[128 x N] (+)= A[128 x K] (K-major) * B where B is stored MN-major as a
+// row-major [K x N] tile (blocks of 64 N columns `b_lbo` bytes apart).
+__device__ __forceinline__ void mma_tile_bmn(uint32_t d_tmem, uint32_t a_base, uint32_t a_blk,
+                                             uint32_t b_base, uint32_t b_lbo, int N, int K,
+                                             bool accumulate) {
+  const uint32_t idesc = idesc_bf16(128, N) | (1u << 16);   // B is MN-major
+  for (int k = 0; k < K / 16; ++k) {
+    const uint32_t off = (uint32_t)(k & 3) * 32;
+    mma_bf16(d_tmem, sdesc_sw128(a_base + (k >> 2) * a_blk + off),
+             sdesc_sw128_mn(b_base + (uint32_t)k * 2048, b_lbo), idesc, accumulate || k > 0);
+  }
+}
+
+// Cooperative, coalesced store of the first `nv` rows of a [128 x 128] bf16
+// tile held in the swizzled layout (2 blocks of [128 x 64]) to row-major
+// global rows (128 threads; a warp writes two whole 256-byte rows per step).
+__device__ __forceinline__ void tile_store_rows(const uint8_t* tile, bf16* dst, int nv) {
+#pragma unroll 4
+  for (int q = 0; q < 16; ++q) {
+    const int idx = q * 128 + (int)threadIdx.x, r = idx >> 4, cc = idx & 15;
+    if (r < nv) reinterpret_cast<uint4*>(dst + (int64_t)r * 128)[cc] = sw_ld16(tile, 128 * 128, r, cc * 8);
+  }
+}
+
+}  // namespace sm100
+}  // namespace lime

@@ -13,18 +13,19 @@
 // per-user tiles of 128 rows (a tile never spans two users; its tail rows are
 // masked).
 //
-//   k_prep_weights   layer weights -> K-major 128B-swizzled images (W^T)
-//   k_schedule       hist_offsets -> tile list (user, first row, valid rows)
+//   k_prep_weights   layer weights -> K-major 128B-swizzled images (W^T); its
+//                    block 0 turns hist_offsets into the tile list (user,
+//                    first row, valid rows)
 //   k_link_proj      LN1(Z) -> Q_Z, K_Z, V_Z (split precision) -> per-user
 //                    operand images: s·K_Z, V_Z^T, and s·Q_Z laid out
 //                    block-diagonally over heads so that one MMA yields the
 //                    link branch's scores transposed (links on TMEM lanes)
-//   k_hist_proj      LN1(E) (split precision) -> Q_E, K_E (row-major) and
-//                    V_E^T (per tile)
+//   k_hist_proj      LN1(E) (split precision) -> Q_E, K_E, V_E (row-major)
 //   k_hist_attn      history branch: softmax over the user's l links, P·V_Z,
 //                    then (P·V_Z)·Wo -> Yd (fp32 attention delta);
 //                    link branch: per tile and (head, link) the partial
 //                    softmax statistics (max, sum) and the weighted V sum
+//                    (V_E read as an MN-major operand, no transpose)
 //   k_link_merge     log-sum-exp merge of a user's tile partials -> b (fp32)
 //   k_hist_ffn       Y = E + Yd, LN2, GatedMLP in 64-wide chunks, E' = Y + ·
 //   k_link_out       Y_Z = Z + b·Wo, LN2, one GatedMLP chunk per CTA (split
@@ -53,7 +54,7 @@ constexpr int kRec = 36;  // floats per link-branch record: max, sum, 32 weighte
 struct LayerWs {
   size_t img_q, img_k, img_v, img_o, img_1, img_3, img_2;
   size_t sched, tiles, tile_start;
-  size_t qe, ke, vt, yd, uimg, part, bmerge, zpart;
+  size_t qe, ke, ve, yd, uimg, part, bmerge, zpart;
   size_t total;
   int64_t max_tiles;
   uint32_t uimg_bytes;
@@ -83,7 +84,7 @@ LayerWs layer_ws(int l, int64_t B, int64_t nh) {
   w.tile_start = take((size_t)(B + 1) * 4);
   w.qe = take((size_t)nh * kD * 2);
   w.ke = take((size_t)nh * kD * 2);
-  w.vt = take((size_t)w.max_tiles * kTile * kD * 2);
+  w.ve = take((size_t)nh * kD * 2);
   w.yd = take((size_t)nh * kD * 4);   // fp32 attention delta
   w.uimg_bytes = uimg_bytes(l);
   w.uimg = take((size_t)B * w.uimg_bytes);
@@ -154,6 +155,24 @@ __device__ __forceinline__ void split_row_st(uint8_t* hi, uint8_t* lo, uint32_t 
 
 __device__ __forceinline__ float silu_fast(float x) { return x / (1.0f + __expf(-x)); }
 
+// fp32 [rows x 128] staging: row r is 512 bytes, its 16-byte chunk c sits at
+// r*512 + ((c ^ (r & 31)) * 16), so row-per-thread and row-per-warp accesses
+// are both free of bank conflicts.
+__device__ __forceinline__ float4* f32_chunk(uint8_t* base, int r, int c) {
+  return reinterpret_cast<float4*>(base + r * 512 + ((c ^ (r & 31)) << 4));
+}
+
+// Cooperatively loads fp32 rows p*32 .. p*32+31 of `src` (128 columns, row 0 =
+// the tile's first row) into staging rows 0..31; rows at or past `nv` are not read.
+__device__ __forceinline__ void f32_stage32(uint8_t* stage, const float* src, int p, int nv) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int idx = q * 128 + (int)threadIdx.x, r = idx >> 5, c = idx & 31;
+    if (p * 32 + r < nv)
+      *f32_chunk(stage, r, c) = reinterpret_cast<const float4*>(src + (int64_t)(p * 32 + r) * kD)[c];
+  }
+}
+
 // Common CTA prologue: barriers, abort flag, TMEM allocation (`ncols` columns).
 struct Cta {
   uint64_t* bar;      // [0] loads, [1] mma, [2..3] extra loads
@@ -203,12 +222,23 @@ __device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
 //   Wq, Wk, Wv, Wo, W2: element (n, k) at (k/64)*rows*128 + sw128_offset(n, k%64)
 //   W1, W3 (n in [0,256)): chunk n/64 of 16 KB, inside it (k/64)*8192 +
 //   sw128_offset(n%64, k%64), so one 64-wide GatedMLP chunk is contiguous.
-__global__ void k_prep_weights(const bf16* __restrict__ Wq, const bf16* __restrict__ Wk,
-                               const bf16* __restrict__ Wv, const bf16* __restrict__ Wo,
-                               const bf16* __restrict__ W1, const bf16* __restrict__ W3,
-                               const bf16* __restrict__ W2, uint8_t* __restrict__ ws,
-                               LayerWs L) {
-  const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+__device__ void schedule_tiles(const int64_t* __restrict__ off, int64_t B, int64_t nh,
+                               int max_tiles, int* __restrict__ sched, int4* __restrict__ tiles,
+                               int* __restrict__ tile_start, unsigned* status);
+
+// Block 0 builds the tile schedule; the other blocks write the weight images.
+__global__ void __launch_bounds__(1024) k_prep_weights(
+    const bf16* __restrict__ Wq, const bf16* __restrict__ Wk, const bf16* __restrict__ Wv,
+    const bf16* __restrict__ Wo, const bf16* __restrict__ W1, const bf16* __restrict__ W3,
+    const bf16* __restrict__ W2, uint8_t* __restrict__ ws, LayerWs L,
+    const int64_t* __restrict__ off, int64_t B, int64_t nh, unsigned* status) {
+  if (blockIdx.x == 0) {
+    schedule_tiles(off, B, nh, (int)L.max_tiles, reinterpret_cast<int*>(ws + L.sched),
+                   reinterpret_cast<int4*>(ws + L.tiles), reinterpret_cast<int*>(ws + L.tile_start),
+                   status);
+    return;
+  }
+  const int64_t e = (blockIdx.x - 1) * (int64_t)blockDim.x + threadIdx.x;
   const int64_t n_sq = kD * kD, n_ff = kD * kF;
   if (e < 4 * n_sq) {
     const int w = (int)(e / n_sq), r = (int)(e % n_sq);
@@ -236,9 +266,9 @@ __global__ void k_prep_weights(const bf16* __restrict__ Wq, const bf16* __restri
 // sched[0], tiles[t] = (u, first row, valid rows, 0) and tile_start[u] (the
 // first tile of user u; tile_start[B] = n_tiles).  Offsets are clamped into
 // [0, nh]; violations set LIME_FLAG_BAD_OFFSETS.
-__global__ void k_schedule(const int64_t* __restrict__ off, int64_t B, int64_t nh,
-                           int max_tiles, int* __restrict__ sched, int4* __restrict__ tiles,
-                           int* __restrict__ tile_start, unsigned* status) {
+__device__ void schedule_tiles(const int64_t* __restrict__ off, int64_t B, int64_t nh,
+                               int max_tiles, int* __restrict__ sched, int4* __restrict__ tiles,
+                               int* __restrict__ tile_start, unsigned* status) {
   __shared__ int warp_sums[32];
   __shared__ int s_base;
   if (threadIdx.x == 0) s_base = 0;
@@ -369,18 +399,21 @@ __global__ void __launch_bounds__(128)
         v[i2] = __bfloat162float(__float2bfloat16_rn(x));
         lo[i2] = x - v[i2];
       }
-      const float zero8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int h = 0; h < kH; ++h) {
-        for (int cc = 0; cc < 16; ++cc) {
+      const uint4 z4 = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int cc = 0; cc < 16; ++cc) {
+        const uint4 hv = pack8(v + cc * 8), lv = pack8(lo + cc * 8);
+#pragma unroll
+        for (int h = 0; h < kH; ++h) {
           const bool mine = (cc >> 2) == h;   // 4 chunks of 8 columns per head
-          sw_st16(qbd, kBlk, h * L + k, cc * 8, pack8(mine ? v + cc * 8 : zero8));
-          sw_st16(qbl, kBlk, h * L + k, cc * 8, pack8(mine ? lo + cc * 8 : zero8));
+          sw_st16(qbd, kBlk, h * L + k, cc * 8, mine ? hv : z4);
+          sw_st16(qbl, kBlk, h * L + k, cc * 8, mine ? lv : z4);
         }
       }
       for (int p = kH * L + k; p < kTile; p += L)
         for (int cc = 0; cc < 16; ++cc) {
-          sw_st16(qbd, kBlk, p, cc * 8, pack8(zero8));
-          sw_st16(qbl, kBlk, p, cc * 8, pack8(zero8));
+          sw_st16(qbd, kBlk, p, cc * 8, z4);
+          sw_st16(qbl, kBlk, p, cc * 8, z4);
         }
     }
   }
@@ -389,9 +422,9 @@ __global__ void __launch_bounds__(128)
 
 // ----------------------------------------------------- history projections
 // One persistent CTA per SM walks the tile list.  For each tile: TMA the 128
-// history rows, LN1 in place, Q/K/V = X^·W on the tensor cores; writes Q_E and
-// K_E rows (valid rows only) and the tile's V_E^T block [128 c x 128 j] with
-// zero columns for rows past the user's history.  The next tile's rows are
+// history rows, LN1, Q/K/V = X^·W on the tensor cores (X^ as hi + lo bf16);
+// writes the valid rows of Q_E, K_E and V_E (row-major bf16) through a
+// swizzled staging tile with coalesced stores.  The next tile's rows are
 // loaded while this tile's outputs are written.
 template <bool LAST>
 __global__ void __launch_bounds__(128, 1)
@@ -410,7 +443,7 @@ __global__ void __launch_bounds__(128, 1)
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
   bf16* qe = reinterpret_cast<bf16*>(ws + Lw.qe);
   bf16* ke = reinterpret_cast<bf16*>(ws + Lw.ke);
-  bf16* vt = reinterpret_cast<bf16*>(ws + Lw.vt);
+  bf16* ve = reinterpret_cast<bf16*>(ws + Lw.ve);
   uint32_t eph = 0, mph = 0;
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(&c.bar[2], NW * 2 * kBlk);
@@ -459,17 +492,20 @@ __global__ void __launch_bounds__(128, 1)
       tma_load_2d(sE, &tmE, 0, tl2.y, &c.bar[0]);
       tma_load_2d(sE + kBlk, &tmE, 64, tl2.y, &c.bar[0]);
     }
-    float v[kD];
-    if (!LAST) {
-      tmem_row128(ta, v);
-      if (i < nv) gl_row_st(qe + (int64_t)(r0 + i) * kD, v);
+    // Q_E, K_E, V_E rows: TMEM -> bf16 -> swizzled staging tile -> coalesced
+    // stores of the valid rows.  The staging alternates between the two halves
+    // of sW's spare space so a store and the next staging overlap safely.
+    const int m0 = LAST ? 1 : 0;
+    for (int mtx = m0; mtx < 3; ++mtx) {
+      uint8_t* stage = sEl;          // the lo half of LN1's output is free now
+      float v[kD];
+      tmem_row128(ta + mtx * 128, v);
+      tile_row_st(stage, i, v);
+      __syncthreads();
+      bf16* dst = (mtx == 0 ? qe : mtx == 1 ? ke : ve) + (int64_t)r0 * kD;
+      tile_store_rows(stage, dst, nv);
+      __syncthreads();
     }
-    tmem_row128(ta + 128, v);
-    if (i < nv) gl_row_st(ke + (int64_t)(r0 + i) * kD, v);
-    tmem_row128(ta + 256, v);
-    bf16* vtt = vt + (int64_t)t * kTile * kD;
-    for (int cc = 0; cc < kD; ++cc)
-      vtt[cc * kTile + i] = __float2bfloat16_rn(i < nv ? v[cc] : 0.f);
     tc_fence_before();
     __syncthreads();
   }
@@ -480,14 +516,14 @@ __global__ void __launch_bounds__(128, 1)
 template <int L, bool LAST>
 __global__ void __launch_bounds__(128, 1)
     k_hist_attn(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmVT, uint8_t* __restrict__ ws, LayerWs Lw,
+                const __grid_constant__ CUtensorMap tmV, uint8_t* __restrict__ ws, LayerWs Lw,
                 unsigned* status) {
   constexpr int HL = kH * L;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
   uint8_t* sQ = sm;                 // Q_E -> P -> A_E
   uint8_t* sK = sm + 2 * kBlk;      // K_E -> P2
-  uint8_t* sVT = sm + 4 * kBlk;     // V_E^T block
+  uint8_t* sV = sm + 4 * kBlk;      // V_E rows (row-major, read as an MN-major operand)
   uint8_t* sWo = sm + 6 * kBlk;     // Wo image (not in the last layer)
   uint8_t* sU = sm + (LAST ? 6 : 8) * kBlk;  // user images
   uint8_t* sKZ = sU;
@@ -522,8 +558,8 @@ __global__ void __launch_bounds__(128, 1)
       }
       tma_load_2d(sK, &tmK, 0, r0, &c.bar[0]);
       tma_load_2d(sK + kBlk, &tmK, 64, r0, &c.bar[0]);
-      tma_load_2d(sVT, &tmVT, 0, t * kTile, &c.bar[0]);
-      tma_load_2d(sVT + kBlk, &tmVT, 64, t * kTile, &c.bar[0]);
+      tma_load_2d(sV, &tmV, 0, r0, &c.bar[0]);
+      tma_load_2d(sV + kBlk, &tmV, 64, r0, &c.bar[0]);
       if (u != cur_u) bulk_load(sU, ws + Lw.uimg + (size_t)u * Lw.uimg_bytes, Lw.uimg_bytes, &c.bar[0]);
     }
     cur_u = u;
@@ -593,7 +629,7 @@ __global__ void __launch_bounds__(128, 1)
           mma_tile(c.tmem + 256 + h * kDH,
                    smem_u32(sQ + ((h * L) >> 6) * kBlk + ((h * L) & 63) * 2), kBlk,
                    smem_u32(sVZT + h * kDH * 128), kBlk, kDH, L, false);
-      mma_tile(c.tmem + 384, smem_u32(sK), kBlk, smem_u32(sVT), kBlk, 128, 128, false);
+      mma_tile_bmn(c.tmem + 384, smem_u32(sK), kBlk, smem_u32(sV), kBlk, 128, 128, false);
     }
     cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
     if (!LAST) {
@@ -633,12 +669,20 @@ __global__ void __launch_bounds__(128, 1)
         mma_tile(c.tmem, smem_u32(sK), kBlk, smem_u32(sWo), kBlk, 128, 128, true);
       }
       cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-      float y[kD];
-      tmem_row128(ta, y);
-      if (i < nv) {
-        float4* dst = reinterpret_cast<float4*>(yd + (int64_t)(r0 + i) * kD);
+      {
+        // fp32 delta rows -> staging in sQ+sK (64 KB, free after the Wo MMA) ->
+        // coalesced stores of the valid rows
+        float y[kD];
+        tmem_row128(ta, y);
 #pragma unroll
-        for (int q = 0; q < kD / 4; ++q) dst[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+        for (int q = 0; q < kD / 4; ++q)
+          *f32_chunk(sQ, i, q) = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int q = 0; q < 32; ++q) {
+        const int idx = q * 128 + i, r = idx >> 5, cc = idx & 31;
+        if (r < nv) reinterpret_cast<float4*>(yd + (int64_t)(r0 + r) * kD)[cc] = *f32_chunk(sQ, r, cc);
       }
     }
     fence_proxy_async_smem();
@@ -945,15 +989,11 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
   const int sms = num_sms();
   {
     const int64_t n = 4 * kD * kD + 3 * kD * kF;
-    k_prep_weights<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+    k_prep_weights<<<(unsigned)(1 + (n + 1023) / 1024), 1024, 0, st>>>(
         (const bf16*)w.Wq, (const bf16*)w.Wk, (const bf16*)w.Wv, (const bf16*)w.Wo,
-        (const bf16*)w.W1, (const bf16*)w.W3, (const bf16*)w.W2, ws, Lw);
+        (const bf16*)w.W1, (const bf16*)w.W3, (const bf16*)w.W2, ws, Lw, off, B, nh, status);
     note_launches(1);
   }
-  k_schedule<<<1, 1024, 0, st>>>(off, B, nh, (int)Lw.max_tiles, reinterpret_cast<int*>(ws + Lw.sched),
-                                 reinterpret_cast<int4*>(ws + Lw.tiles),
-                                 reinterpret_cast<int*>(ws + Lw.tile_start), status);
-  note_launches(1);
   {
     const int smem = 1024 + 6 * kBlk + kBarBytes;
     if (!set_smem(k_link_proj<L>, smem)) return LIME_ERR_CUDA;
@@ -962,12 +1002,11 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     note_launches(1);
   }
   if (nh > 0) {
-    CUtensorMap tmE, tmQ, tmK, tmVT;
+    CUtensorMap tmE, tmQ, tmK, tmV;
     if (!make_tmap_2d_bf16(&tmE, E_in, kD, (uint64_t)nh, kD * 2, 64, kTile) ||
         !make_tmap_2d_bf16(&tmQ, ws + Lw.qe, kD, (uint64_t)nh, kD * 2, 64, kTile) ||
         !make_tmap_2d_bf16(&tmK, ws + Lw.ke, kD, (uint64_t)nh, kD * 2, 64, kTile) ||
-        !make_tmap_2d_bf16(&tmVT, ws + Lw.vt, kD, (uint64_t)Lw.max_tiles * kTile, kD * 2, 64,
-                           kTile))
+        !make_tmap_2d_bf16(&tmV, ws + Lw.ve, kD, (uint64_t)nh, kD * 2, 64, kTile))
       return LIME_ERR_CUDA;
     const int64_t tiles_hi = Lw.max_tiles;
     const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
@@ -986,11 +1025,11 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     if (last) {
       const int smem = 1024 + 6 * kBlk + uimg_bytes(L) + kBarBytes;
       if (!set_smem(k_hist_attn<L, true>, smem)) return LIME_ERR_CUDA;
-      k_hist_attn<L, true><<<grid, 128, smem, st>>>(tmQ, tmK, tmVT, ws, Lw, status);
+      k_hist_attn<L, true><<<grid, 128, smem, st>>>(tmQ, tmK, tmV, ws, Lw, status);
     } else {
       const int smem = 1024 + 8 * kBlk + uimg_bytes(L) + kBarBytes;
       if (!set_smem(k_hist_attn<L, false>, smem)) return LIME_ERR_CUDA;
-      k_hist_attn<L, false><<<grid, 128, smem, st>>>(tmQ, tmK, tmVT, ws, Lw, status);
+      k_hist_attn<L, false><<<grid, 128, smem, st>>>(tmQ, tmK, tmV, ws, Lw, status);
     }
     note_launches(1);
     if (!last) {

@@ -324,11 +324,12 @@ __device__ __forceinline__ void mma_tile_bmn(uint32_t d_tmem, uint32_t a_base, u
 
 // Cooperative, coalesced store of the first `nv` rows of a [128 x 128] bf16
 // tile held in the swizzled layout (2 blocks of [128 x 64]) to row-major
-// global rows (128 threads; a warp writes two whole 256-byte rows per step).
+// global rows (any multiple of 32 threads; a warp writes two whole 256-byte
+// rows per step).
 __device__ __forceinline__ void tile_store_rows(const uint8_t* tile, bf16* dst, int nv) {
 #pragma unroll 4
-  for (int q = 0; q < 16; ++q) {
-    const int idx = q * 128 + (int)threadIdx.x, r = idx >> 4, cc = idx & 15;
+  for (int idx = (int)threadIdx.x; idx < 2048; idx += (int)blockDim.x) {
+    const int r = idx >> 4, cc = idx & 15;
     if (r < nv) reinterpret_cast<uint4*>(dst + (int64_t)r * 128)[cc] = sw_ld16(tile, 128 * 128, r, cc * 8);
   }
 }

@@ -120,6 +120,41 @@ __device__ __forceinline__ void layer_norm_128(float* x, const bf16* g, const bf
     x[i] = (x[i] - mu) * rstd * __bfloat162float(g[i]) + __bfloat162float(b[i]);
 }
 
+// Row reductions over the four column parts of a row (thread = (row, part),
+// 512 threads): every thread gets the total.  `red` holds 512 floats; all
+// threads of the block take part (two block-wide barriers).
+__device__ __forceinline__ float row_sum4(float v, float* red, int part, int row) {
+  red[part * 128 + row] = v;
+  __syncthreads();
+  const float t = red[row] + red[128 + row] + red[256 + row] + red[384 + row];
+  __syncthreads();
+  return t;
+}
+__device__ __forceinline__ float row_max4(float v, float* red, int part, int row) {
+  red[part * 128 + row] = v;
+  __syncthreads();
+  const float t = fmaxf(fmaxf(red[row], red[128 + row]), fmaxf(red[256 + row], red[384 + row]));
+  __syncthreads();
+  return t;
+}
+
+// LayerNorm of one row held as four 32-column parts (x = this thread's part,
+// columns c0..c0+31), affine with g, b.
+__device__ __forceinline__ void layer_norm_part(float* x, int c0, const bf16* g, const bf16* b,
+                                                float* red, int part, int row) {
+  float s1 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) s1 += x[k];
+  const float mu = row_sum4(s1, red, part, row) * (1.0f / kD);
+  float s2 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) { const float d0 = x[k] - mu; s2 += d0 * d0; }
+  const float rstd = rsqrtf(row_sum4(s2, red, part, row) * (1.0f / kD) + kLnEps);
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    x[k] = (x[k] - mu) * rstd * __bfloat162float(g[c0 + k]) + __bfloat162float(b[c0 + k]);
+}
+
 // Loads 128 consecutive fp32 TMEM columns of this thread's lane.
 __device__ __forceinline__ void tmem_row128(uint32_t taddr, float* x) {
 #pragma unroll
@@ -211,6 +246,10 @@ __device__ __forceinline__ void cta_teardown(Cta& c) {
 
 __device__ __forceinline__ uint32_t lane_addr(const Cta& c) {
   return c.tmem + ((uint32_t)(threadIdx.x & ~31) << 16);
+}
+// 512-thread kernels: warp w serves TMEM lane quadrant w % 4.
+__device__ __forceinline__ uint32_t quad_addr(const Cta& c) {
+  return c.tmem + ((uint32_t)(((threadIdx.x >> 5) & 3) * 32) << 16);
 }
 
 __device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
@@ -329,38 +368,55 @@ __device__ void schedule_tiles(const int64_t* __restrict__ off, int64_t B, int64
 //        stored twice, as the hi and lo bf16 halves of the fp32 value (the
 //        link query is one vector per link, so its rounding is not averaged)
 template <int L>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(512)
     k_link_proj(const bf16* __restrict__ Z, int64_t nrows, const bf16* __restrict__ g1,
                 const bf16* __restrict__ b1, const uint8_t* __restrict__ ws_c,
                 uint8_t* __restrict__ ws, LayerWs Lw, float scale, unsigned* status) {
-  // CTA (tile, which): which = 0 -> Q_Z (block-diagonal image), 1 -> K_Z, 2 -> V_Z^T
+  // CTA (tile, which): which = 0 -> Q_Z (block-diagonal image), 1 -> K_Z, 2 -> V_Z^T.
+  // 512 threads: thread (row, part) owns columns part*32 .. part*32+31.
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
   uint8_t* sAh = sm;
   uint8_t* sAl = sm + 2 * kBlk;
   uint8_t* sW = sm + 4 * kBlk;
+  float* red = reinterpret_cast<float*>(sm + 6 * kBlk);
   const int which = blockIdx.y;
   Cta c;
-  cta_setup(sm + 6 * kBlk, 2, c, 128);
+  cta_setup(sm + 6 * kBlk + 2048, 2, c, 128);
   uint32_t mph = 0;
   if (threadIdx.x == 0) {
     const size_t img = which == 0 ? Lw.img_q : which == 1 ? Lw.img_k : Lw.img_v;
     mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
     bulk_load(sW, ws_c + img, 2 * kBlk, &c.bar[0]);
   }
-  const int r = threadIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int part = warp >> 2;
+  const int r = (warp & 3) * 32 + (threadIdx.x & 31);
+  const int c0 = part * 32;
   const int64_t R = (int64_t)blockIdx.x * kTile + r;
   const bool valid = R < nrows;
   {
-    float x[kD];
+    float x[32];
     if (valid) {
-      gl_row_ld(Z + R * kD, x);
-      layer_norm_128(x, g1, b1);
+      const uint4* src = reinterpret_cast<const uint4*>(Z + R * kD + c0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) unpack8(src[q], x + q * 8);
     } else {
 #pragma unroll
-      for (int i2 = 0; i2 < kD; ++i2) x[i2] = 0.f;
+      for (int i2 = 0; i2 < 32; ++i2) x[i2] = 0.f;
     }
-    split_row_st(sAh, sAl, kBlk, r, x, kD);
+    layer_norm_part(x, c0, g1, b1, red, part, r);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float h8[8], l8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        h8[k] = __bfloat162float(__float2bfloat16_rn(x[q * 8 + k]));
+        l8[k] = x[q * 8 + k] - h8[k];
+      }
+      sw_st16(sAh, kBlk, r, c0 + q * 8, pack8(h8));
+      sw_st16(sAl, kBlk, r, c0 + q * 8, pack8(l8));
+    }
   }
   fence_proxy_async_smem();
   __syncthreads();
@@ -371,49 +427,52 @@ __global__ void __launch_bounds__(128)
     mma_tile(c.tmem, smem_u32(sAl), kBlk, smem_u32(sW), kBlk, 128, 128, true);
   }
   cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-  float v[kD];
-  tmem_row128(lane_addr(c), v);   // warp-collective: every thread loads
+  float v[32];
+  tmem_ld16(quad_addr(c) + c0, v);          // warp-collective: every thread loads
+  tmem_ld16(quad_addr(c) + c0 + 16, v + 16);
+  tmem_ld_wait();
   if (valid) {
     const int64_t u = R / L;
     const int k = (int)(R % L);
     uint8_t* img = ws + Lw.uimg + u * Lw.uimg_bytes;
     if (which == 1) {           // s·K_Z row k
-      uint8_t* kz = img;
 #pragma unroll
-      for (int i2 = 0; i2 < kD; ++i2) v[i2] *= scale;
-      for (int cc = 0; cc < 16; ++cc) sw_st16(kz, (uint32_t)L * 128, k, cc * 8, pack8(v + cc * 8));
+      for (int i2 = 0; i2 < 32; ++i2) v[i2] *= scale;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sw_st16(img, (uint32_t)L * 128, k, c0 + q * 8, pack8(v + q * 8));
     } else if (which == 2) {    // V_Z^T column k, zero padding columns k + L, ... < 64
       uint8_t* vzt = img + kz_bytes(L);
-      for (int cc = 0; cc < kD; ++cc) {
-        *reinterpret_cast<bf16*>(vzt + sw128_offset(cc, k)) = __float2bfloat16_rn(v[cc]);
+      for (int cc = 0; cc < 32; ++cc) {
+        *reinterpret_cast<bf16*>(vzt + sw128_offset(c0 + cc, k)) = __float2bfloat16_rn(v[cc]);
         for (int kp = k + L; kp < 64; kp += L)
-          *reinterpret_cast<bf16*>(vzt + sw128_offset(cc, kp)) = __float2bfloat16_rn(0.f);
+          *reinterpret_cast<bf16*>(vzt + sw128_offset(c0 + cc, kp)) = __float2bfloat16_rn(0.f);
       }
     } else {                    // block-diagonal s·Q_Z rows h*L + k (hi, lo); rows >= 4L zero
       uint8_t* qbd = img + kz_bytes(L) + kBlk;
       uint8_t* qbl = qbd + 2 * kBlk;
-      float lo[kD];
+      float lo[32];
 #pragma unroll
-      for (int i2 = 0; i2 < kD; ++i2) {
+      for (int i2 = 0; i2 < 32; ++i2) {
         const float x = v[i2] * scale;
         v[i2] = __bfloat162float(__float2bfloat16_rn(x));
         lo[i2] = x - v[i2];
       }
       const uint4 z4 = make_uint4(0, 0, 0, 0);
+      // this thread's 32 columns belong to head `part`
 #pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        const uint4 hv = pack8(v + cc * 8), lv = pack8(lo + cc * 8);
+      for (int q = 0; q < 4; ++q) {
+        const uint4 hv = pack8(v + q * 8), lv = pack8(lo + q * 8);
 #pragma unroll
         for (int h = 0; h < kH; ++h) {
-          const bool mine = (cc >> 2) == h;   // 4 chunks of 8 columns per head
-          sw_st16(qbd, kBlk, h * L + k, cc * 8, mine ? hv : z4);
-          sw_st16(qbl, kBlk, h * L + k, cc * 8, mine ? lv : z4);
+          sw_st16(qbd, kBlk, h * L + k, c0 + q * 8, h == part ? hv : z4);
+          sw_st16(qbl, kBlk, h * L + k, c0 + q * 8, h == part ? lv : z4);
         }
       }
       for (int p = kH * L + k; p < kTile; p += L)
-        for (int cc = 0; cc < 16; ++cc) {
-          sw_st16(qbd, kBlk, p, cc * 8, z4);
-          sw_st16(qbl, kBlk, p, cc * 8, z4);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          sw_st16(qbd, kBlk, p, c0 + q * 8, z4);
+          sw_st16(qbl, kBlk, p, c0 + q * 8, z4);
         }
     }
   }
@@ -425,20 +484,23 @@ __global__ void __launch_bounds__(128)
 // history rows, LN1, Q/K/V = X^·W on the tensor cores (X^ as hi + lo bf16);
 // writes the valid rows of Q_E, K_E and V_E (row-major bf16) through a
 // swizzled staging tile with coalesced stores.  The next tile's rows are
-// loaded while this tile's outputs are written.
+// loaded while this tile's outputs are written.  512 threads: thread (row,
+// part) handles a quarter of the row's columns; LN1's statistics are reduced
+// across the four parts.
 template <bool LAST>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(512, 1)
     k_hist_proj(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ g1,
                 const bf16* __restrict__ b1, uint8_t* __restrict__ ws, LayerWs Lw,
                 unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
   uint8_t* sE = sm;               // E tile -> LN1 output, hi half
-  uint8_t* sEl = sm + 2 * kBlk;    // LN1 output, lo half
+  uint8_t* sEl = sm + 2 * kBlk;    // LN1 output, lo half -> output staging
   uint8_t* sW = sm + 4 * kBlk;     // [Wq,] Wk, Wv images
   constexpr int NW = LAST ? 2 : 3;
+  float* red = reinterpret_cast<float*>(sm + (4 + 2 * NW) * kBlk);
   Cta c;
-  cta_setup(sm + (4 + 2 * NW) * kBlk, 3, c);
+  cta_setup(sm + (4 + 2 * NW) * kBlk + 2048, 3, c);
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
   bf16* qe = reinterpret_cast<bf16*>(ws + Lw.qe);
@@ -459,8 +521,11 @@ __global__ void __launch_bounds__(128, 1)
     }
   }
   mbar_wait(&c.bar[2], 0, status, c.abort_flag);
-  const int i = threadIdx.x;
-  const uint32_t ta = lane_addr(c);
+  const int warp = threadIdx.x >> 5;
+  const int part = warp >> 2;
+  const int row = (warp & 3) * 32 + (threadIdx.x & 31);
+  const int c0 = part * 32;
+  const uint32_t ta = quad_addr(c);
   for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
     const int4 tl = tiles[t];
     const int r0 = tl.y, nv = tl.z;
@@ -469,10 +534,21 @@ __global__ void __launch_bounds__(128, 1)
     {
       // LN1 output as hi + lo bf16 halves: K_E and V_E feed the link branch,
       // whose softmax over a short history does not average rounding away
-      float x[kD];
-      tile_row_ld(sE, i, x);
-      layer_norm_128(x, g1, b1);
-      split_row_st(sE, sEl, kBlk, i, x, kD);
+      float x[32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sE, kBlk, row, c0 + q * 8), x + q * 8);
+      layer_norm_part(x, c0, g1, b1, red, part, row);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float h8[8], l8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          h8[k] = __bfloat162float(__float2bfloat16_rn(x[q * 8 + k]));
+          l8[k] = x[q * 8 + k] - h8[k];
+        }
+        sw_st16(sE, kBlk, row, c0 + q * 8, pack8(h8));
+        sw_st16(sEl, kBlk, row, c0 + q * 8, pack8(l8));
+      }
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -492,20 +568,21 @@ __global__ void __launch_bounds__(128, 1)
       tma_load_2d(sE, &tmE, 0, tl2.y, &c.bar[0]);
       tma_load_2d(sE + kBlk, &tmE, 64, tl2.y, &c.bar[0]);
     }
-    // Q_E, K_E, V_E rows: TMEM -> bf16 -> swizzled staging tile -> coalesced
-    // stores of the valid rows.  The staging alternates between the two halves
-    // of sW's spare space so a store and the next staging overlap safely.
-    const int m0 = LAST ? 1 : 0;
-    for (int mtx = m0; mtx < 3; ++mtx) {
-      uint8_t* stage = sEl;          // the lo half of LN1's output is free now
-      float v[kD];
-      tmem_row128(ta + mtx * 128, v);
-      tile_row_st(stage, i, v);
+    // Q_E, K_E, V_E rows: TMEM -> bf16 -> swizzled staging tile (the lo half
+    // of LN1's output is free now) -> coalesced stores of the valid rows
+    for (int mtx = LAST ? 1 : 0; mtx < 3; ++mtx) {
+      float v[32];
+      tmem_ld16(ta + mtx * 128 + c0, v);
+      tmem_ld16(ta + mtx * 128 + c0 + 16, v + 16);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sw_st16(sEl, kBlk, row, c0 + q * 8, pack8(v + q * 8));
       __syncthreads();
       bf16* dst = (mtx == 0 ? qe : mtx == 1 ? ke : ve) + (int64_t)r0 * kD;
-      tile_store_rows(stage, dst, nv);
+      tile_store_rows(sEl, dst, nv);
       __syncthreads();
     }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
   }
@@ -513,28 +590,32 @@ __global__ void __launch_bounds__(128, 1)
 }
 
 // --------------------------------------------------------- XOR attention
+// 512 threads: thread (row, part) with row = 32*(warp%4) + lane (a TMEM lane)
+// and part = warp/4, a quarter of the row's columns (or of the tile's tokens
+// for the link branch).  Thread 0 issues the MMAs.
 template <int L, bool LAST>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(512, 1)
     k_hist_attn(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, uint8_t* __restrict__ ws, LayerWs Lw,
                 unsigned* status) {
   constexpr int HL = kH * L;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
-  uint8_t* sQ = sm;                 // Q_E -> P -> A_E
-  uint8_t* sK = sm + 2 * kBlk;      // K_E -> P2
+  uint8_t* sQ = sm;                 // Q_E -> P -> A_E (hi); with sK: fp32 delta staging
+  uint8_t* sK = sm + 2 * kBlk;      // K_E -> P2 -> A_E (lo)
   uint8_t* sV = sm + 4 * kBlk;      // V_E rows (row-major, read as an MN-major operand)
   uint8_t* sWo = sm + 6 * kBlk;     // Wo image (not in the last layer)
   uint8_t* sU = sm + (LAST ? 6 : 8) * kBlk;  // user images
   uint8_t* sKZ = sU;
   uint8_t* sVZT = sU + kz_bytes(L);
   uint8_t* sQBD = sVZT + kBlk;
+  float* red = reinterpret_cast<float*>(sU + uimg_bytes(L));   // [4][128]
   Cta c;
-  cta_setup(sU + uimg_bytes(L), 3, c);
+  cta_setup(sU + uimg_bytes(L) + 2048, 3, c);
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
   float* yd = reinterpret_cast<float*>(ws + Lw.yd);
-  float* part = reinterpret_cast<float*>(ws + Lw.part);
+  float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
   uint32_t lph = 0, mph = 0;
   if (!LAST) {
     if (threadIdx.x == 0) {
@@ -543,8 +624,10 @@ __global__ void __launch_bounds__(128, 1)
     }
     mbar_wait(&c.bar[2], 0, status, c.abort_flag);
   }
-  const int i = threadIdx.x;
-  const uint32_t ta = lane_addr(c);
+  const int warp = threadIdx.x >> 5;
+  const int part = warp >> 2;
+  const int row = (warp & 3) * 32 + (threadIdx.x & 31);
+  const uint32_t ta = quad_addr(c);
   int cur_u = -1;
   for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
     const int4 tl = tiles[t];
@@ -577,46 +660,50 @@ __global__ void __launch_bounds__(128, 1)
       mma_tile(c.tmem + 128, smem_u32(sQBD + 2 * kBlk), kBlk, smem_u32(sK), kBlk, 128, 128, true);
     }
     cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    // history softmax over the user's L links, per head -> P in sQ
+    // history softmax over the user's L links: part = head
     if (!LAST) {
-      for (int h = 0; h < kH; ++h) {
-        float z[L];
+      const int h = part;
+      float z[L];
 #pragma unroll
-        for (int q = 0; q < L / 16; ++q) tmem_ld16(ta + h * L + q * 16, z + q * 16);
-        tmem_ld_wait();
-        float m = z[0];
+      for (int q = 0; q < L / 16; ++q) tmem_ld16(ta + h * L + q * 16, z + q * 16);
+      tmem_ld_wait();
+      float m = z[0];
 #pragma unroll
-        for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
-        float s = 0.f;
-#pragma unroll
-        for (int k = 0; k < L; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
-        const float inv = 1.0f / s;
-#pragma unroll
-        for (int k = 0; k < L; ++k) z[k] *= inv;
-#pragma unroll
-        for (int q = 0; q < L / 8; ++q) sw_st16(sQ, kBlk, i, h * L + q * 8, pack8(z + q * 8));
-      }
-    }
-    // link softmax over this tile's valid history rows, per (head, link) lane
-    float lm = 0.f, ls = 0.f;
-    {
-      float z[kTile];
-      tmem_row128(ta + 128, z);
-      float m = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < kTile; ++j) {
-        if (j >= nv) z[j] = -INFINITY;
-        m = fmaxf(m, z[j]);
-      }
+      for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
       float s = 0.f;
 #pragma unroll
-      for (int j = 0; j < kTile; ++j) {
-        z[j] = j < nv ? __expf(z[j] - m) : 0.f;
+      for (int k = 0; k < L; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
+      const float inv = 1.0f / s;
+#pragma unroll
+      for (int k = 0; k < L; ++k) z[k] *= inv;
+#pragma unroll
+      for (int q = 0; q < L / 8; ++q) sw_st16(sQ, kBlk, row, h * L + q * 8, pack8(z + q * 8));
+    }
+    // link softmax over this tile's valid history rows; row = (head, link)
+    // lane, part = a quarter of the tile's 128 tokens
+    float lm, ls;
+    {
+      float z[32];
+      tmem_ld16(ta + 128 + part * 32, z);
+      tmem_ld16(ta + 128 + part * 32 + 16, z + 16);
+      tmem_ld_wait();
+      float m = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (part * 32 + j >= nv) z[j] = -INFINITY;
+        m = fmaxf(m, z[j]);
+      }
+      m = row_max4(m, red, part, row);
+      float s = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        z[j] = part * 32 + j < nv ? __expf(z[j] - m) : 0.f;
         s += z[j];
       }
       lm = m;
-      ls = s;
-      tile_row_st(sK, i, z);
+      ls = row_sum4(s, red, part, row);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sw_st16(sK, kBlk, row, part * 32 + q * 8, pack8(z + q * 8));
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -635,28 +722,37 @@ __global__ void __launch_bounds__(128, 1)
     if (!LAST) {
       // A_E enters the Wo GEMM as hi + lo bf16 halves (sQ, sK), so the
       // attention delta keeps close to fp32 accuracy.
-      float a[kD];
-      tmem_row128(ta + 256, a);
-      split_row_st(sQ, sK, kBlk, i, a, kD);
-    }
-    if (i < HL) {  // warp-uniform: HL is a multiple of 32
-      // A warp's lanes may span two heads (L = 16), and tcgen05.ld takes one
-      // address per warp: load the whole row, then keep this lane's head.
-      const int h = i / L;
-      float row[kD], acc[kDH];
-      tmem_row128(ta + 384, row);
+      float a[32];
+      tmem_ld16(ta + 256 + part * 32, a);
+      tmem_ld16(ta + 256 + part * 32 + 16, a + 16);
+      tmem_ld_wait();
 #pragma unroll
-      for (int hh = 0; hh < kH; ++hh)
-        if (hh == h) {
+      for (int q = 0; q < 4; ++q) {
+        float h8[8], l8[8];
 #pragma unroll
-          for (int cc = 0; cc < kDH; ++cc) acc[cc] = row[hh * kDH + cc];
+        for (int k = 0; k < 8; ++k) {
+          h8[k] = __bfloat162float(__float2bfloat16_rn(a[q * 8 + k]));
+          l8[k] = a[q * 8 + k] - h8[k];
         }
-      float4* rec = reinterpret_cast<float4*>(part + ((size_t)t * HL + i) * kRec);
-      rec[0] = make_float4(lm, ls, acc[0], acc[1]);
+        sw_st16(sQ, kBlk, row, part * 32 + q * 8, pack8(h8));
+        sw_st16(sK, kBlk, row, part * 32 + q * 8, pack8(l8));
+      }
+    }
+    {
+      // link record of row p = (h, k): part h reads head h's 32 columns
+      // (warp-uniform TMEM address); rows of other heads skip the store
+      float acc[kDH];
+      tmem_ld16(ta + 384 + part * kDH, acc);
+      tmem_ld16(ta + 384 + part * kDH + 16, acc + 16);
+      tmem_ld_wait();
+      if (row < HL && row / L == part) {
+        float4* rec = reinterpret_cast<float4*>(part_rec + ((size_t)t * HL + row) * kRec);
+        rec[0] = make_float4(lm, ls, acc[0], acc[1]);
 #pragma unroll
-      for (int q = 1; q < 8; ++q)
-        rec[q] = make_float4(acc[4 * q - 2], acc[4 * q - 1], acc[4 * q], acc[4 * q + 1]);
-      rec[8] = make_float4(acc[30], acc[31], 0.f, 0.f);
+        for (int q = 1; q < 8; ++q)
+          rec[q] = make_float4(acc[4 * q - 2], acc[4 * q - 1], acc[4 * q], acc[4 * q + 1]);
+        rec[8] = make_float4(acc[30], acc[31], 0.f, 0.f);
+      }
     }
     if (!LAST) {
       fence_proxy_async_smem();
@@ -670,18 +766,20 @@ __global__ void __launch_bounds__(128, 1)
       }
       cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
       {
-        // fp32 delta rows -> staging in sQ+sK (64 KB, free after the Wo MMA) ->
+        // fp32 delta -> staging in sQ+sK (64 KB, free after the Wo MMA) ->
         // coalesced stores of the valid rows
-        float y[kD];
-        tmem_row128(ta, y);
+        float y[32];
+        tmem_ld16(ta + part * 32, y);
+        tmem_ld16(ta + part * 32 + 16, y + 16);
+        tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < kD / 4; ++q)
-          *f32_chunk(sQ, i, q) = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+        for (int q = 0; q < 8; ++q)
+          *f32_chunk(sQ, row, part * 8 + q) = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
       }
       __syncthreads();
 #pragma unroll 4
-      for (int q = 0; q < 32; ++q) {
-        const int idx = q * 128 + i, r = idx >> 5, cc = idx & 31;
+      for (int q = 0; q < 8; ++q) {
+        const int idx = q * 512 + (int)threadIdx.x, r = idx >> 5, cc = idx & 31;
         if (r < nv) reinterpret_cast<float4*>(yd + (int64_t)(r0 + r) * kD)[cc] = *f32_chunk(sQ, r, cc);
       }
     }
@@ -723,117 +821,252 @@ __global__ void k_link_merge(const uint8_t* __restrict__ ws, LayerWs Lw, int64_t
 }
 
 // ------------------------------------------------------- history GatedMLP
-// Per tile: Y = E + Yd (Yd fp32 from the attention kernel), h2 = LN2(Y) in
-// bf16, then for each 64-wide chunk of the hidden layer: G1 = h2 W1c, G3 =
-// h2 W3c (TMEM [0,128)), hid = SiLU(G1) * G3 in bf16, OUT += hid W2c (TMEM
-// [128,256)); E' = Y + OUT with Y re-read from E and Yd.  256 TMEM columns
-// and ~97 KB of shared memory let two CTAs share an SM, so one CTA's waits
-// overlap the other's work.
-__global__ void __launch_bounds__(128, 2)
+// E' = Y + GatedMLP(LN2(Y)), Y = E + Yd, for one 128-row history tile at a
+// time, as a warp-specialized pipeline (persistent, one CTA per SM):
+//   warps 0-15 (epilogue): warp w serves TMEM lane quadrant w % 4 (tile rows
+//     32*(w%4) ...) and column part p = w / 4 (a quarter of every row), so each
+//     row is shared by four threads and the per-row work has four times the
+//     warps to hide latency.  They form Y = E (TMA tile) + Yd (fp32 rows) into
+//     TMEM YR, h2 = LN2(Y) (statistics reduced over the four parts through
+//     shared memory) into smem, hid = SiLU(G1) * G3 per 64-wide hidden chunk
+//     from TMEM GB[c%2] into smem HB[c%2], and finally E' = YR + OUT.
+//   warp 16 (control, one lane): TMA of the next tile's E, bulk loads of the
+//     weight chunks into two slots, and the MMAs: G(c) = h2 [W1c|W3c] into
+//     GB[c%2], OUT += hid(c) W2c.  G(c+1) is issued before hid(c) is ready, so
+//     the tensor cores work while the epilogue computes the gate.
+// TMEM: GB[0] [0,128), GB[1] [128,256), OUT [256,384), YR [384,512).
+// A barrier used twice per tile (once per chunk parity) waits for parity
+// j = c / 2; once-per-tile barriers wait for the tile index's parity.
+constexpr int kFfnEpi = 512;   // epilogue threads
+
+__global__ void __launch_bounds__(kFfnEpi + 32, 1)
     k_hist_ffn(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ E_in,
                const bf16* __restrict__ g2, const bf16* __restrict__ b2,
                const uint8_t* __restrict__ ws, LayerWs Lw, bf16* __restrict__ E_out,
                unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
-  uint8_t* sE = sm;                 // E -> h2
-  uint8_t* sH = sm + 2 * kBlk;      // hid chunk [128 x 64]
-  uint8_t* sW = sm + 3 * kBlk;      // W1c, W3c, W2c
-  Cta c;
-  cta_setup(sm + 6 * kBlk, 3, c, 256);  // bar: 0 rows, 1 mma, 2 weights
+  uint8_t* sE0 = sm;                   // 2 x [128 x 128] bf16: E tile -> h2
+  uint8_t* sH0 = sm + 4 * kBlk;        // 2 x [128 x 64]  bf16: hid chunk
+  uint8_t* sW0 = sm + 6 * kBlk;        // 2 x (W1c, W3c, W2c)
+  constexpr uint32_t kSlot = 3 * kBlk;
+  float* red = reinterpret_cast<float*>(sm + 12 * kBlk);           // [2][4][128] LN partials
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 12 * kBlk + 4096);
+  uint64_t* barE = bar;        // [2] E tile landed (TMA)
+  uint64_t* barWt = bar + 2;   // [2] weight slot landed
+  uint64_t* barG = bar + 4;    // [2] G(c) in TMEM (MMA commit)
+  uint64_t* barHid = bar + 6;  // [2] hid(c) written, GB read (epilogue arrivals)
+  uint64_t* barW2 = bar + 8;   // [2] OUT += hid(c) W2c done (MMA commit)
+  uint64_t* barH2 = bar + 10;  // h2 written (epilogue arrivals)
+  uint64_t* barOut = bar + 11; // all of the tile's MMAs done (MMA commit)
+  uint64_t* barFree = bar + 12;  // epilogue finished the tile (epilogue arrivals)
+  uint64_t* barDrain = bar + 13; // every MMA issued by the control lane is done
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 14);
+  int* abort_flag = reinterpret_cast<int*>(bar + 15);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&barE[q], 1);
+      mbar_init(&barWt[q], 1);
+      mbar_init(&barG[q], 1);
+      mbar_init(&barHid[q], kFfnEpi);
+      mbar_init(&barW2[q], 1);
+    }
+    mbar_init(barH2, kFfnEpi);
+    mbar_init(barOut, 1);
+    mbar_init(barFree, kFfnEpi);
+    mbar_init(barDrain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
   const float* yd = reinterpret_cast<const float*>(ws + Lw.yd);
-  uint32_t lph = 0, mph = 0, wph = 0;
-  const int i = threadIdx.x;
-  const uint32_t ta = lane_addr(c);
-  auto load_chunk = [&](int ch) {
-    mbar_arrive_expect_tx(&c.bar[2], 3 * kBlk);
-    bulk_load(sW, ws + Lw.img_1 + ch * kBlk, kBlk, &c.bar[2]);
-    bulk_load(sW + kBlk, ws + Lw.img_3 + ch * kBlk, kBlk, &c.bar[2]);
-    bulk_load(sW + 2 * kBlk, ws + Lw.img_2 + ch * kBlk, kBlk, &c.bar[2]);
-  };
-  auto y_row = [&](int64_t row, float* y, bool from_smem) {
-    if (from_smem) tile_row_ld(sE, i, y);
-    else gl_row_ld(E_in + row * kD, y);
-    const float4* src = reinterpret_cast<const float4*>(yd + row * kD);
-#pragma unroll
-    for (int q = 0; q < kD / 4; ++q) {
-      const float4 v = src[q];
-      y[4 * q] += v.x; y[4 * q + 1] += v.y; y[4 * q + 2] += v.z; y[4 * q + 3] += v.w;
-    }
-  };
-  for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-    const int4 tl = tiles[t];
-    const int r0 = tl.y, nv = tl.z;
-    if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
-      tma_load_2d(sE, &tmE, 0, r0, &c.bar[0]);
-      tma_load_2d(sE + kBlk, &tmE, 64, r0, &c.bar[0]);
-      load_chunk(0);
-    }
-    mbar_wait(&c.bar[0], lph, status, c.abort_flag);
-    lph ^= 1u;
-    {
-      float y[kD];
-      if (i < nv) y_row(r0 + i, y, true);
-      else {
-#pragma unroll
-        for (int k = 0; k < kD; ++k) y[k] = 0.f;
-      }
-      layer_norm_128(y, g2, b2);
-      tile_row_st(sE, i, y);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    for (int ch = 0; ch < kF / 64; ++ch) {
-      mbar_wait(&c.bar[2], wph, status, c.abort_flag);
-      wph ^= 1u;
-      if (threadIdx.x == 0) {
+  const uint32_t T_OUT = 256, T_Y = 384;
+
+  if (warp == kFfnEpi / 32) {
+    if (lane == 0) {
+      auto load_chunk = [&](int ch) {
+        uint8_t* dst = sW0 + (ch & 1) * kSlot;
+        uint64_t* b = &barWt[ch & 1];
+        mbar_arrive_expect_tx(b, kSlot);
+        bulk_load(dst, ws + Lw.img_1 + ch * kBlk, kBlk, b);
+        bulk_load(dst + kBlk, ws + Lw.img_3 + ch * kBlk, kBlk, b);
+        bulk_load(dst + 2 * kBlk, ws + Lw.img_2 + ch * kBlk, kBlk, b);
+      };
+      auto load_e = [&](int t, int buf) {
+        const int4 tl = tiles[t];
+        mbar_arrive_expect_tx(&barE[buf], 2 * kBlk);
+        tma_load_2d(sE0 + buf * 2 * kBlk, &tmE, 0, tl.y, &barE[buf]);
+        tma_load_2d(sE0 + buf * 2 * kBlk + kBlk, &tmE, 64, tl.y, &barE[buf]);
+      };
+      prefetch_tmap(&tmE);
+      if ((int)blockIdx.x < n_tiles) load_e(blockIdx.x, 0);
+      int it = 0;
+      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+        const int cur = it & 1;
+        if (it > 0 && !mbar_wait(barFree, (it - 1) & 1, status, abort_flag)) break;
+        const int tn = t + gridDim.x;
+        if (tn < n_tiles) load_e(tn, cur ^ 1);     // buffer of tile it-1 is free
+        load_chunk(0);
+        load_chunk(1);
+        if (!mbar_wait(barH2, it & 1, status, abort_flag)) break;
         tc_fence_after();
-        mma_tile(c.tmem, smem_u32(sE), kBlk, smem_u32(sW), 8192, 64, 128, false);
-        mma_tile(c.tmem + 64, smem_u32(sE), kBlk, smem_u32(sW + kBlk), 8192, 64, 128, false);
+        const uint32_t a_h2 = smem_u32(sE0 + cur * 2 * kBlk);
+        bool ok = true;
+        for (int c = 0; c < kF / 64 && ok; ++c) {
+          const int sb = c & 1;
+          ok = mbar_wait(&barWt[sb], (uint32_t)(c >> 1), status, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t wslot = smem_u32(sW0 + sb * kSlot);
+          mma_tile(tmem + sb * 128, a_h2, kBlk, wslot, 8192, 64, 128, false);
+          mma_tile(tmem + sb * 128 + 64, a_h2, kBlk, wslot + kBlk, 8192, 64, 128, false);
+          mma_commit(&barG[sb]);
+          if (c >= 1) {
+            const int pc = c - 1, pb = pc & 1;
+            ok = mbar_wait(&barHid[pb], (uint32_t)(pc >> 1), status, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            mma_tile(tmem + T_OUT, smem_u32(sH0 + pb * kBlk), kBlk,
+                     smem_u32(sW0 + pb * kSlot + 2 * kBlk), kBlk, 128, 64, pc > 0);
+            mma_commit(&barW2[pb]);
+            if (c + 1 < kF / 64) {       // slot pb is free once W2(pc) is done
+              ok = mbar_wait(&barW2[pb], (uint32_t)(pc >> 1), status, abort_flag);
+              if (!ok) break;
+              load_chunk(c + 1);
+            }
+          }
+        }
+        if (!ok) break;
+        {
+          const int pc = kF / 64 - 1, pb = pc & 1;
+          if (!mbar_wait(&barHid[pb], (uint32_t)(pc >> 1), status, abort_flag)) break;
+          tc_fence_after();
+          mma_tile(tmem + T_OUT, smem_u32(sH0 + pb * kBlk), kBlk,
+                   smem_u32(sW0 + pb * kSlot + 2 * kBlk), kBlk, 128, 64, true);
+          mma_commit(&barW2[pb]);
+          mma_commit(barOut);
+        }
       }
-      cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+      // drain: no MMA of ours may be in flight when TMEM is freed
+      mma_commit(barDrain);
+      mbar_wait(barDrain, 0, status, abort_flag);
+    }
+  } else {
+    const int q4 = warp & 3, part = warp >> 2;     // lane quadrant, column part
+    const int row = q4 * 32 + lane;
+    const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16);
+    const int c0 = part * 32;                      // this thread's 32 columns of a row
+    int it = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+      const int cur = it & 1;
+      const int4 tl = tiles[t];
+      const int r0 = tl.y, nv = tl.z;
+      uint8_t* sE = sE0 + cur * 2 * kBlk;
+      // Yd part first: its round trip overlaps the wait for the E tile
+      float y[32];
+      if (row < nv) {
+        const float4* src = reinterpret_cast<const float4*>(yd + (int64_t)(r0 + row) * kD + c0);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 v = src[q];
+          y[4 * q] = v.x; y[4 * q + 1] = v.y; y[4 * q + 2] = v.z; y[4 * q + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) y[k] = 0.f;
+      }
+      mbar_wait(&barE[cur], (uint32_t)((it >> 1) & 1), status, abort_flag);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float e[8];
+        unpack8(sw_ld16(sE, kBlk, row, c0 + q * 8), e);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) y[q * 8 + k] += e[k];
+      }
+      tmem_st16(ta + T_Y + c0, y);
+      tmem_st16(ta + T_Y + c0 + 16, y + 16);
+      tmem_st_wait();
+      // LN2 statistics over the row's four parts
+      float* rs = red + (it & 1) * 512;
       {
-        float g[64], gg[64];
+        float s1 = 0.f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld16(ta + q * 16, g + q * 16);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld16(ta + 64 + q * 16, gg + q * 16);
-        tmem_ld_wait();
-#pragma unroll
-        for (int k = 0; k < 64; ++k) g[k] = silu_fast(g[k]) * gg[k];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) sw_st16(sH, kBlk, i, q * 8, pack8(g + q * 8));
+        for (int k = 0; k < 32; ++k) s1 += y[k];
+        rs[part * 128 + row] = s1;
       }
+      named_bar_sync(1, kFfnEpi);
+      const float mu = (rs[row] + rs[128 + row] + rs[256 + row] + rs[384 + row]) * (1.0f / kD);
+      named_bar_sync(1, kFfnEpi);
+      {
+        float s2 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) { const float d0 = y[k] - mu; s2 += d0 * d0; }
+        rs[part * 128 + row] = s2;
+      }
+      named_bar_sync(1, kFfnEpi);
+      const float rstd =
+          rsqrtf((rs[row] + rs[128 + row] + rs[256 + row] + rs[384 + row]) * (1.0f / kD) + kLnEps);
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        y[k] = (y[k] - mu) * rstd * __bfloat162float(g2[c0 + k]) + __bfloat162float(b2[c0 + k]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sw_st16(sE, kBlk, row, c0 + q * 8, pack8(y + q * 8));
       fence_proxy_async_smem();
       tc_fence_before();
-      __syncthreads();
-      if (threadIdx.x == 0) {
+      mbar_arrive(barH2);
+      for (int c = 0; c < kF / 64; ++c) {
+        const int sb = c & 1;
+        mbar_wait(&barG[sb], (uint32_t)(c >> 1), status, abort_flag);
         tc_fence_after();
-        mma_tile(c.tmem + 128, smem_u32(sH), kBlk, smem_u32(sW + 2 * kBlk), kBlk, 128, 64, ch > 0);
-      }
-      cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-      if (threadIdx.x == 0 && ch + 1 < kF / 64) load_chunk(ch + 1);
-    }
-    {
-      float o[kD];
-      tmem_row128(ta + 128, o);   // warp-collective: every thread loads
-      if (i < nv) {
-        float y[kD];
-        y_row(r0 + i, y, false);
+        float g[16], gg[16];
+        tmem_ld16(ta + sb * 128 + part * 16, g);
+        tmem_ld16(ta + sb * 128 + 64 + part * 16, gg);
+        tmem_ld_wait();
 #pragma unroll
-        for (int k = 0; k < kD; ++k) y[k] += o[k];
-        gl_row_st(E_out + (int64_t)(r0 + i) * kD, y);
+        for (int k = 0; k < 16; ++k) g[k] = silu_fast(g[k]) * gg[k];
+        // hid(c) reuses the buffer of hid(c-2): wait until its W2 MMA is done
+        if (c >= 2) mbar_wait(&barW2[sb], 0u, status, abort_flag);
+        uint8_t* sH = sH0 + sb * kBlk;
+        sw_st16(sH, kBlk, row, part * 16, pack8(g));
+        sw_st16(sH, kBlk, row, part * 16 + 8, pack8(g + 8));
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&barHid[sb]);
       }
+      mbar_wait(barOut, (uint32_t)(it & 1), status, abort_flag);
+      tc_fence_after();
+      {
+        float o[32], yy[32];
+        tmem_ld16(ta + T_OUT + c0, o);
+        tmem_ld16(ta + T_OUT + c0 + 16, o + 16);
+        tmem_ld16(ta + T_Y + c0, yy);
+        tmem_ld16(ta + T_Y + c0 + 16, yy + 16);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] += yy[k];
+        if (row < nv) {
+          uint4* dst = reinterpret_cast<uint4*>(E_out + (int64_t)(r0 + row) * kD + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[q] = pack8(o + q * 8);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(barFree);
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
   }
-  cta_teardown(c);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
 }
 
 // ---------------------------------------------------------- link outputs
@@ -842,11 +1075,12 @@ __global__ void __launch_bounds__(128, 2)
 // b Wo and LN2 for its 128 rows, then GatedMLP chunk ch only, and writes the
 // chunk's fp32 contribution to zpart[ch] (chunk 0 also writes b Wo to
 // zpart[4]); k_link_finish sums them.  Deterministic, no atomics.
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(512, 1)
     k_link_out(const bf16* __restrict__ Z, const float* __restrict__ bm, int64_t nrows,
                const bf16* __restrict__ g2, const bf16* __restrict__ b2,
                const uint8_t* __restrict__ ws_c, LayerWs Lw, float* __restrict__ zpart,
                unsigned* status) {
+  // 512 threads: thread (row, part) owns columns part*32 .. part*32+31 of its row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
   uint8_t* sAh = sm;
@@ -855,9 +1089,10 @@ __global__ void __launch_bounds__(128, 1)
   uint8_t* sHl = sm + 5 * kBlk;
   uint8_t* sWo = sm + 6 * kBlk;
   uint8_t* sW = sm + 8 * kBlk;      // W1c, W3c, W2c of chunk ch
+  float* red = reinterpret_cast<float*>(sm + 11 * kBlk);
   const int ch = blockIdx.y;
   Cta c;
-  cta_setup(sm + 11 * kBlk, 3, c);  // bar: 0 Wo, 1 mma, 2 chunk
+  cta_setup(sm + 11 * kBlk + 2048, 3, c);  // bar: 0 Wo, 1 mma, 2 chunk
   uint32_t mph = 0;
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
@@ -867,24 +1102,39 @@ __global__ void __launch_bounds__(128, 1)
     bulk_load(sW + kBlk, ws_c + Lw.img_3 + ch * kBlk, kBlk, &c.bar[2]);
     bulk_load(sW + 2 * kBlk, ws_c + Lw.img_2 + ch * kBlk, kBlk, &c.bar[2]);
   }
-  const int r = threadIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int part = warp >> 2;
+  const int r = (warp & 3) * 32 + (threadIdx.x & 31);
+  const int c0 = part * 32;
   const int64_t R = (int64_t)blockIdx.x * kTile + r;
   const bool valid = R < nrows;
-  const uint32_t ta = lane_addr(c);
-  {
-    float x[kD];
-    if (valid) {
-      const float4* src = reinterpret_cast<const float4*>(bm + R * kD);
+  const uint32_t ta = quad_addr(c);
+  auto split_store = [&](uint8_t* hi, uint8_t* lo, int col0, const float* x, int n) {
+    for (int q = 0; q < n / 8; ++q) {
+      float h8[8], l8[8];
 #pragma unroll
-      for (int q = 0; q < kD / 4; ++q) {
+      for (int k = 0; k < 8; ++k) {
+        h8[k] = __bfloat162float(__float2bfloat16_rn(x[q * 8 + k]));
+        l8[k] = x[q * 8 + k] - h8[k];
+      }
+      sw_st16(hi, kBlk, r, col0 + q * 8, pack8(h8));
+      sw_st16(lo, kBlk, r, col0 + q * 8, pack8(l8));
+    }
+  };
+  {
+    float x[32];
+    if (valid) {
+      const float4* src = reinterpret_cast<const float4*>(bm + R * kD + c0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
         const float4 v = src[q];
         x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
       }
     } else {
 #pragma unroll
-      for (int k = 0; k < kD; ++k) x[k] = 0.f;
+      for (int k = 0; k < 32; ++k) x[k] = 0.f;
     }
-    split_row_st(sAh, sAl, kBlk, r, x, kD);
+    split_store(sAh, sAl, c0, x, 32);
   }
   fence_proxy_async_smem();
   __syncthreads();
@@ -896,22 +1146,27 @@ __global__ void __launch_bounds__(128, 1)
   }
   cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
   {
-    float y[kD], z[kD];
-    tmem_row128(ta, y);
+    float y[32];
+    tmem_ld16(ta + c0, y);
+    tmem_ld16(ta + c0 + 16, y + 16);
+    tmem_ld_wait();
     if (valid && ch == 0) {
-      float4* dst = reinterpret_cast<float4*>(zpart + ((size_t)4 * nrows + R) * kD);
+      float4* dst = reinterpret_cast<float4*>(zpart + ((size_t)4 * nrows + R) * kD + c0);
 #pragma unroll
-      for (int q = 0; q < kD / 4; ++q) dst[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+      for (int q = 0; q < 8; ++q) dst[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
     }
-    if (valid) gl_row_ld(Z + R * kD, z);
-    else {
+    if (valid) {
+      const uint4* src = reinterpret_cast<const uint4*>(Z + R * kD + c0);
 #pragma unroll
-      for (int k = 0; k < kD; ++k) z[k] = 0.f;
+      for (int q = 0; q < 4; ++q) {
+        float z8[8];
+        unpack8(src[q], z8);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) y[q * 8 + k] += z8[k];
+      }
     }
-#pragma unroll
-    for (int k = 0; k < kD; ++k) y[k] += z[k];
-    layer_norm_128(y, g2, b2);
-    split_row_st(sAh, sAl, kBlk, r, y, kD);
+    layer_norm_part(y, c0, g2, b2, red, part, r);
+    split_store(sAh, sAl, c0, y, 32);
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -926,15 +1181,13 @@ __global__ void __launch_bounds__(128, 1)
   }
   cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
   {
-    float g[64], gg[64];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) tmem_ld16(ta + 128 + q * 16, g + q * 16);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) tmem_ld16(ta + 192 + q * 16, gg + q * 16);
+    float g[16], gg[16];
+    tmem_ld16(ta + 128 + part * 16, g);
+    tmem_ld16(ta + 192 + part * 16, gg);
     tmem_ld_wait();
 #pragma unroll
-    for (int k = 0; k < 64; ++k) g[k] = silu_fast(g[k]) * gg[k];
-    split_row_st(sHh, sHl, kBlk, r, g, 64);
+    for (int k = 0; k < 16; ++k) g[k] = silu_fast(g[k]) * gg[k];
+    split_store(sHh, sHl, part * 16, g, 16);
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -946,12 +1199,14 @@ __global__ void __launch_bounds__(128, 1)
   }
   cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
   {
-    float o[kD];
-    tmem_row128(ta + 256, o);    // warp-collective: every thread loads
+    float o[32];
+    tmem_ld16(ta + 256 + c0, o);    // warp-collective: every thread loads
+    tmem_ld16(ta + 256 + c0 + 16, o + 16);
+    tmem_ld_wait();
     if (valid) {
-      float4* dst = reinterpret_cast<float4*>(zpart + ((size_t)ch * nrows + R) * kD);
+      float4* dst = reinterpret_cast<float4*>(zpart + ((size_t)ch * nrows + R) * kD + c0);
 #pragma unroll
-      for (int q = 0; q < kD / 4; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
     }
   }
   cta_teardown(c);
@@ -995,9 +1250,9 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     note_launches(1);
   }
   {
-    const int smem = 1024 + 6 * kBlk + kBarBytes;
+    const int smem = 1024 + 6 * kBlk + 2048 + kBarBytes;
     if (!set_smem(k_link_proj<L>, smem)) return LIME_ERR_CUDA;
-    k_link_proj<L><<<dim3((unsigned)((nz + kTile - 1) / kTile), 3), 128, smem, st>>>(
+    k_link_proj<L><<<dim3((unsigned)((nz + kTile - 1) / kTile), 3), 512, smem, st>>>(
         (const bf16*)Z_in, nz, (const bf16*)w.g1, (const bf16*)w.b1, ws, ws, Lw, scale, status);
     note_launches(1);
   }
@@ -1011,33 +1266,32 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     const int64_t tiles_hi = Lw.max_tiles;
     const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
     if (last) {
-      const int smem = 1024 + 8 * kBlk + kBarBytes;
+      const int smem = 1024 + 8 * kBlk + 2048 + kBarBytes;
       if (!set_smem(k_hist_proj<true>, smem)) return LIME_ERR_CUDA;
-      k_hist_proj<true><<<grid, 128, smem, st>>>(tmE, (const bf16*)w.g1, (const bf16*)w.b1, ws,
+      k_hist_proj<true><<<grid, 512, smem, st>>>(tmE, (const bf16*)w.g1, (const bf16*)w.b1, ws,
                                                   Lw, status);
     } else {
-      const int smem = 1024 + 10 * kBlk + kBarBytes;
+      const int smem = 1024 + 10 * kBlk + 2048 + kBarBytes;
       if (!set_smem(k_hist_proj<false>, smem)) return LIME_ERR_CUDA;
-      k_hist_proj<false><<<grid, 128, smem, st>>>(tmE, (const bf16*)w.g1, (const bf16*)w.b1, ws,
+      k_hist_proj<false><<<grid, 512, smem, st>>>(tmE, (const bf16*)w.g1, (const bf16*)w.b1, ws,
                                                    Lw, status);
     }
     note_launches(1);
     if (last) {
-      const int smem = 1024 + 6 * kBlk + uimg_bytes(L) + kBarBytes;
+      const int smem = 1024 + 6 * kBlk + uimg_bytes(L) + 2048 + kBarBytes;
       if (!set_smem(k_hist_attn<L, true>, smem)) return LIME_ERR_CUDA;
-      k_hist_attn<L, true><<<grid, 128, smem, st>>>(tmQ, tmK, tmV, ws, Lw, status);
+      k_hist_attn<L, true><<<grid, 512, smem, st>>>(tmQ, tmK, tmV, ws, Lw, status);
     } else {
-      const int smem = 1024 + 8 * kBlk + uimg_bytes(L) + kBarBytes;
+      const int smem = 1024 + 8 * kBlk + uimg_bytes(L) + 2048 + kBarBytes;
       if (!set_smem(k_hist_attn<L, false>, smem)) return LIME_ERR_CUDA;
-      k_hist_attn<L, false><<<grid, 128, smem, st>>>(tmQ, tmK, tmV, ws, Lw, status);
+      k_hist_attn<L, false><<<grid, 512, smem, st>>>(tmQ, tmK, tmV, ws, Lw, status);
     }
     note_launches(1);
     if (!last) {
-      const int smem = 1024 + 6 * kBlk + kBarBytes;
+      const int smem = 1024 + 12 * kBlk + 4096 + 256;
       if (!set_smem(k_hist_ffn, smem)) return LIME_ERR_CUDA;
-      const int g2 = (int)(tiles_hi < 2 * sms ? tiles_hi : 2 * sms);
-      k_hist_ffn<<<g2, 128, smem, st>>>(tmE, (const bf16*)E_in, (const bf16*)w.g2,
-                                        (const bf16*)w.b2, ws, Lw, (bf16*)E_out, status);
+      k_hist_ffn<<<grid, kFfnEpi + 32, smem, st>>>(tmE, (const bf16*)E_in, (const bf16*)w.g2,
+                                                   (const bf16*)w.b2, ws, Lw, (bf16*)E_out, status);
       note_launches(1);
     }
   }
@@ -1048,10 +1302,10 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     note_launches(1);
   }
   {
-    const int smem = 1024 + 11 * kBlk + kBarBytes;
+    const int smem = 1024 + 11 * kBlk + 2048 + kBarBytes;
     if (!set_smem(k_link_out, smem)) return LIME_ERR_CUDA;
     float* zpart = reinterpret_cast<float*>(ws + Lw.zpart);
-    k_link_out<<<dim3((unsigned)((nz + kTile - 1) / kTile), kF / 64), 128, smem, st>>>(
+    k_link_out<<<dim3((unsigned)((nz + kTile - 1) / kTile), kF / 64), 512, smem, st>>>(
         (const bf16*)Z_in, reinterpret_cast<const float*>(ws + Lw.bmerge), nz,
         (const bf16*)w.g2, (const bf16*)w.b2, ws, Lw, zpart, status);
     note_launches(1);

@@ -32,7 +32,8 @@
 //                    precision), fp32 partials; k_link_finish sums them -> Z'
 //   (k_link_proj also runs one CTA per (tile, Q|K|V))
 // The last layer (E_out = NULL) skips everything only E' needs: Q_E, the
-// history branch, Wo on history rows and k_hist_ffn.
+// history branch, Wo on history rows and k_hist_ffn; its link branch runs in
+// k_hist_link, which keeps K_E and V_E on chip.
 //
 // CTAs run their phases synchronously: thread 0 issues the MMAs of a phase,
 // all 128 threads wait on an mbarrier (bounded), then each thread works on its
@@ -790,6 +791,166 @@ __global__ void __launch_bounds__(512, 1)
   cta_teardown(c);
 }
 
+// ------------------------------------------------ last layer: link branch
+// The last layer needs only the link rows' outputs, so the history side is
+// just the link branch, fused in one kernel that keeps K_E and V_E on chip:
+// TMA E -> LN1 (hi + lo) -> K_E, V_E = X^ Wk, X^ Wv (TMEM) -> bf16 in smem ->
+// S'^T = (s Q_Z)_bd K_E^T -> softmax over the tile's valid rows (per
+// (head, link) lane, statistics reduced over four token parts) -> P2 ->
+// P2 V_E (V_E read as an MN-major operand) -> per-tile records.
+// 512 threads: thread (row, part).  TMEM: K_E [0,128), V_E [128,256),
+// S'^T [256,384), P2 V_E [384,512).
+template <int L>
+__global__ void __launch_bounds__(512, 1)
+    k_hist_link(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ g1,
+                const bf16* __restrict__ b1, uint8_t* __restrict__ ws, LayerWs Lw,
+                unsigned* status) {
+  constexpr int HL = kH * L;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1k(smem_raw);
+  uint8_t* sE = sm;                // E tile -> X^ hi -> K_E -> P2
+  uint8_t* sEl = sm + 2 * kBlk;    // X^ lo -> V_E
+  uint8_t* sWk = sm + 4 * kBlk;
+  uint8_t* sWv = sm + 6 * kBlk;
+  uint8_t* sQBD = sm + 8 * kBlk;   // block-diagonal s*Q_Z, hi then lo (4 blocks)
+  float* red = reinterpret_cast<float*>(sm + 12 * kBlk);
+  Cta c;
+  cta_setup(sm + 12 * kBlk + 2048, 3, c);
+  const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
+  const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
+  float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
+  uint32_t lph = 0, mph = 0;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&c.bar[2], 4 * kBlk);
+    bulk_load(sWk, ws + Lw.img_k, 2 * kBlk, &c.bar[2]);
+    bulk_load(sWv, ws + Lw.img_v, 2 * kBlk, &c.bar[2]);
+  }
+  mbar_wait(&c.bar[2], 0, status, c.abort_flag);
+  const int warp = threadIdx.x >> 5;
+  const int part = warp >> 2;
+  const int row = (warp & 3) * 32 + (threadIdx.x & 31);
+  const int c0 = part * 32;
+  const uint32_t ta = quad_addr(c);
+  int cur_u = -1;
+  for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const int4 tl = tiles[t];
+    const int u = tl.x, r0 = tl.y, nv = tl.z;
+    if (threadIdx.x == 0) {
+      const uint32_t qbd_bytes = 4 * kBlk;
+      mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk + (u != cur_u ? qbd_bytes : 0));
+      tma_load_2d(sE, &tmE, 0, r0, &c.bar[0]);
+      tma_load_2d(sE + kBlk, &tmE, 64, r0, &c.bar[0]);
+      if (u != cur_u)
+        bulk_load(sQBD, ws + Lw.uimg + (size_t)u * Lw.uimg_bytes + kz_bytes(L) + kBlk, qbd_bytes,
+                  &c.bar[0]);
+    }
+    cur_u = u;
+    mbar_wait(&c.bar[0], lph, status, c.abort_flag);
+    lph ^= 1u;
+    {
+      float x[32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sE, kBlk, row, c0 + q * 8), x + q * 8);
+      layer_norm_part(x, c0, g1, b1, red, part, row);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float h8[8], l8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          h8[k] = __bfloat162float(__float2bfloat16_rn(x[q * 8 + k]));
+          l8[k] = x[q * 8 + k] - h8[k];
+        }
+        sw_st16(sE, kBlk, row, c0 + q * 8, pack8(h8));
+        sw_st16(sEl, kBlk, row, c0 + q * 8, pack8(l8));
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      mma_tile(c.tmem, smem_u32(sE), kBlk, smem_u32(sWk), kBlk, 128, 128, false);
+      mma_tile(c.tmem, smem_u32(sEl), kBlk, smem_u32(sWk), kBlk, 128, 128, true);
+      mma_tile(c.tmem + 128, smem_u32(sE), kBlk, smem_u32(sWv), kBlk, 128, 128, false);
+      mma_tile(c.tmem + 128, smem_u32(sEl), kBlk, smem_u32(sWv), kBlk, 128, 128, true);
+    }
+    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+    {
+      // K_E -> sE (K-major B of the score MMA), V_E -> sEl (MN-major B)
+      float v[32];
+      tmem_ld16(ta + c0, v);
+      tmem_ld16(ta + c0 + 16, v + 16);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sw_st16(sE, kBlk, row, c0 + q * 8, pack8(v + q * 8));
+      tmem_ld16(ta + 128 + c0, v);
+      tmem_ld16(ta + 128 + c0 + 16, v + 16);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sw_st16(sEl, kBlk, row, c0 + q * 8, pack8(v + q * 8));
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      mma_tile(c.tmem + 256, smem_u32(sQBD), kBlk, smem_u32(sE), kBlk, 128, 128, false);
+      mma_tile(c.tmem + 256, smem_u32(sQBD + 2 * kBlk), kBlk, smem_u32(sE), kBlk, 128, 128, true);
+    }
+    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+    float lm, ls;
+    {
+      float z[32];
+      tmem_ld16(ta + 256 + part * 32, z);
+      tmem_ld16(ta + 256 + part * 32 + 16, z + 16);
+      tmem_ld_wait();
+      float m = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (part * 32 + j >= nv) z[j] = -INFINITY;
+        m = fmaxf(m, z[j]);
+      }
+      m = row_max4(m, red, part, row);
+      float s = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        z[j] = part * 32 + j < nv ? __expf(z[j] - m) : 0.f;
+        s += z[j];
+      }
+      lm = m;
+      ls = row_sum4(s, red, part, row);
+      // P2 goes into sE: K_E's last reader (the score MMA) has completed
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sw_st16(sE, kBlk, row, part * 32 + q * 8, pack8(z + q * 8));
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      mma_tile_bmn(c.tmem + 384, smem_u32(sE), kBlk, smem_u32(sEl), kBlk, 128, 128, false);
+    }
+    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+    {
+      float acc[kDH];
+      tmem_ld16(ta + 384 + part * kDH, acc);
+      tmem_ld16(ta + 384 + part * kDH + 16, acc + 16);
+      tmem_ld_wait();
+      if (row < HL && row / L == part) {
+        float4* rec = reinterpret_cast<float4*>(part_rec + ((size_t)t * HL + row) * kRec);
+        rec[0] = make_float4(lm, ls, acc[0], acc[1]);
+#pragma unroll
+        for (int q = 1; q < 8; ++q)
+          rec[q] = make_float4(acc[4 * q - 2], acc[4 * q - 1], acc[4 * q], acc[4 * q + 1]);
+        rec[8] = make_float4(acc[30], acc[31], 0.f, 0.f);
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+  }
+  cta_teardown(c);
+}
+
 // ------------------------------------------------------------ link merge
 // b[u, k, h*32 + c] = merge over the user's tiles of (max, sum, acc) records:
 // the link-branch softmax of link k (head h) over all of the user's history.
@@ -1266,10 +1427,10 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     const int64_t tiles_hi = Lw.max_tiles;
     const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
     if (last) {
-      const int smem = 1024 + 8 * kBlk + 2048 + kBarBytes;
-      if (!set_smem(k_hist_proj<true>, smem)) return LIME_ERR_CUDA;
-      k_hist_proj<true><<<grid, 512, smem, st>>>(tmE, (const bf16*)w.g1, (const bf16*)w.b1, ws,
-                                                  Lw, status);
+      const int smem = 1024 + 12 * kBlk + 2048 + kBarBytes;
+      if (!set_smem(k_hist_link<L>, smem)) return LIME_ERR_CUDA;
+      k_hist_link<L><<<grid, 512, smem, st>>>(tmE, (const bf16*)w.g1, (const bf16*)w.b1, ws, Lw,
+                                              status);
     } else {
       const int smem = 1024 + 10 * kBlk + 2048 + kBarBytes;
       if (!set_smem(k_hist_proj<false>, smem)) return LIME_ERR_CUDA;
@@ -1277,16 +1438,12 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
                                                    Lw, status);
     }
     note_launches(1);
-    if (last) {
-      const int smem = 1024 + 6 * kBlk + uimg_bytes(L) + 2048 + kBarBytes;
-      if (!set_smem(k_hist_attn<L, true>, smem)) return LIME_ERR_CUDA;
-      k_hist_attn<L, true><<<grid, 512, smem, st>>>(tmQ, tmK, tmV, ws, Lw, status);
-    } else {
+    if (!last) {
       const int smem = 1024 + 8 * kBlk + uimg_bytes(L) + 2048 + kBarBytes;
       if (!set_smem(k_hist_attn<L, false>, smem)) return LIME_ERR_CUDA;
       k_hist_attn<L, false><<<grid, 512, smem, st>>>(tmQ, tmK, tmV, ws, Lw, status);
+      note_launches(1);
     }
-    note_launches(1);
     if (!last) {
       const int smem = 1024 + 12 * kBlk + 4096 + 256;
       if (!set_smem(k_hist_ffn, smem)) return LIME_ERR_CUDA;

@@ -136,10 +136,13 @@ int lime_build_qk_cache_noalloc(const lime_dims* dims, const void* T, int64_t n_
 /* Context links: LC[u, k, :] = SiLU([L_k ; ctx_u] Wc1 + bc1) Wc2 + bc2.
  * LIME note 整体框架 (L^C = MLP(L ⊕ E^C)) and 一个完整示例 step 2.
  *   L   device [l, d];  ctx device [B, c];  LC_out device [B, l, d].
+ *   workspace, workspace_bytes: only its status word is used (a timed-out
+ *           device wait sets LIME_FLAG_TIMEOUT there); at least
+ *           lime_workspace_bytes(dims, 0, 0) bytes.
  * Needs dims->c >= 1.                                                    */
 int lime_context_links(const lime_dims* dims, int64_t B, const void* L,
                        const void* ctx, const lime_ctx_mlp* w, void* LC_out,
-                       cudaStream_t stream);
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* One LIME-XOR layer over a batch of jagged user histories.
  * LIME note 关键设计 2: over X = [E; Z] a query attends to a key only when

@@ -124,11 +124,13 @@ int lime_build_qk_cache(const lime_dims* dims, const void* T, int64_t n_items, c
 }
 
 int lime_context_links(const lime_dims* dims, int64_t B, const void* L, const void* ctx,
-                       const lime_ctx_mlp* w, void* LC_out, cudaStream_t stream) {
+                       const lime_ctx_mlp* w, void* LC_out, void* workspace,
+                       size_t workspace_bytes, cudaStream_t stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if (dims->c < 1) return LIME_ERR_SHAPE;
   if (B < 0 || B > INT32_MAX) return LIME_ERR_ARG;
+  if ((rc = check_ws(workspace, workspace_bytes, dims, 0, 0))) return rc;
   if (B == 0) return LIME_OK;
   if (!L || !ctx || !w || !LC_out || !w->Wc1 || !w->bc1 || !w->Wc2 || !w->bc2)
     return LIME_ERR_ARG;
@@ -138,7 +140,10 @@ int lime_context_links(const lime_dims* dims, int64_t B, const void* L, const vo
   if (overlap(LC_out, out_sz, L, (size_t)dims->l * dims->d * es) ||
       overlap(LC_out, out_sz, ctx, (size_t)B * dims->c * es))
     return LIME_ERR_ALIAS;
-  if (dims->dtype == LIME_BF16)
+  if (fast_ctx_supported(*dims) && aligned16(L) && aligned16(ctx) && aligned16(LC_out)) {
+    if ((rc = fast_context_links(*dims, B, L, ctx, *w, LC_out, status_of(workspace), stream)))
+      return rc;
+  } else if (dims->dtype == LIME_BF16)
     simt_context_links<bf16>(*dims, B, L, ctx, *w, LC_out, stream);
   else
     simt_context_links<float>(*dims, B, L, ctx, *w, LC_out, stream);

@@ -18,6 +18,10 @@ int fast_score(const lime_dims& D, int64_t B, const void* cache, int64_t n_items
                const int32_t* ids, const int64_t* off, int64_t total, const void* LP, void* O,
                float* ws, unsigned* status, cudaStream_t st);
 
+bool fast_ctx_supported(const lime_dims& D);
+int fast_context_links(const lime_dims& D, int64_t B, const void* L, const void* ctx,
+                       const lime_ctx_mlp& w, void* LC, unsigned* status, cudaStream_t st);
+
 bool fast_layer_supported(const lime_dims& D);
 int fast_xor_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh,
                    const void* E_in, const void* Z_in, const lime_layer_w& w, void* E_out,

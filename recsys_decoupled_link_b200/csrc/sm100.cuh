@@ -48,16 +48,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase of `bar` with the given parity to complete.  The wait is
-// bounded (about two seconds); on expiry it sets LIME_FLAG_TIMEOUT in the
-// status word, raises the CTA's abort flag and returns false.
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Waits for the phase of `bar` with the given parity to complete.  try_wait
+// suspends the thread in hardware until the phase completes or a short
+// system time limit passes, so the loop needs no sleep of its own (a software
+// sleep would add its wake-up delay to every producer -> consumer hand-off).
+// The wait is bounded by the global timer (two seconds); on expiry it sets
+// LIME_FLAG_TIMEOUT in the status word, raises the CTA's abort flag and
+// returns false.  A raised abort flag ends every later wait of the CTA.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* status,
                                           volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  for (uint32_t it = 0; it < (1u << 25); ++it) {
+  const uint64_t t0 = global_ns();
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (it > 64) __nanosleep(64);
+    if (global_ns() - t0 > 2000000000ull) break;
   }
   raise_flag(status, LIME_FLAG_TIMEOUT);
   *abort_flag = 1;

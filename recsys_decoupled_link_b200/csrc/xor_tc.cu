@@ -53,7 +53,7 @@ constexpr float kLnEps = 1e-5f;
 constexpr int kRec = 36;  // floats per link-branch record: max, sum, 32 weighted sums, 2 pad
 
 struct LayerWs {
-  size_t img_q, img_k, img_v, img_o, img_1, img_3, img_2;
+  size_t img_q, img_k, img_v, img_o, img_13, img_2;
   size_t sched, tiles, tile_start;
   size_t qe, ke, ve, yd, uimg, part, bmerge, zpart;
   size_t total;
@@ -76,8 +76,7 @@ LayerWs layer_ws(int l, int64_t B, int64_t nh) {
   w.img_k = take(2 * kBlk);
   w.img_v = take(2 * kBlk);
   w.img_o = take(2 * kBlk);
-  w.img_1 = take(4 * kBlk);
-  w.img_3 = take(4 * kBlk);
+  w.img_13 = take(8 * kBlk);
   w.img_2 = take(4 * kBlk);
   w.max_tiles = nh / kTile + B + 1;
   w.sched = take(16);
@@ -290,10 +289,10 @@ __global__ void __launch_bounds__(1024) k_prep_weights(
     const int64_t r0 = e - 4 * n_sq;
     const int w = (int)(r0 / n_ff), r = (int)(r0 % n_ff);
     const int k = r / kF, n = r % kF;
+    // chunk n/64 of the hidden layer: K block k/64 holds W1's 64 rows, then W3's
     const bf16* src = w == 0 ? W1 : W3;
-    const size_t base = w == 0 ? L.img_1 : L.img_3;
-    *reinterpret_cast<bf16*>(ws + base + (n >> 6) * 16384 + (k >> 6) * 8192 +
-                             sw128_offset(n & 63, k & 63)) = src[r];
+    *reinterpret_cast<bf16*>(ws + L.img_13 + (n >> 6) * (2 * kBlk) + (k >> 6) * kBlk +
+                             w * 8192 + sw128_offset(n & 63, k & 63)) = src[r];
   } else if (e < 4 * n_sq + 3 * n_ff) {
     const int r = (int)(e - 4 * n_sq - 2 * n_ff);
     const int k = r / kD, n = r % kD;   // W2 is [256, 128]
@@ -985,46 +984,56 @@ __global__ void k_link_merge(const uint8_t* __restrict__ ws, LayerWs Lw, int64_t
 // E' = Y + GatedMLP(LN2(Y)), Y = E + Yd, for one 128-row history tile at a
 // time, as a warp-specialized pipeline (persistent, one CTA per SM):
 //   warps 0-15 (epilogue): warp w serves TMEM lane quadrant w % 4 (tile rows
-//     32*(w%4) ...) and column part p = w / 4 (a quarter of every row), so each
-//     row is shared by four threads and the per-row work has four times the
-//     warps to hide latency.  They form Y = E (TMA tile) + Yd (fp32 rows) into
-//     TMEM YR, h2 = LN2(Y) (statistics reduced over the four parts through
-//     shared memory) into smem, hid = SiLU(G1) * G3 per 64-wide hidden chunk
-//     from TMEM GB[c%2] into smem HB[c%2], and finally E' = YR + OUT.
-//   warp 16 (control, one lane): TMA of the next tile's E, bulk loads of the
-//     weight chunks into two slots, and the MMAs: G(c) = h2 [W1c|W3c] into
-//     GB[c%2], OUT += hid(c) W2c.  G(c+1) is issued before hid(c) is ready, so
-//     the tensor cores work while the epilogue computes the gate.
-// TMEM: GB[0] [0,128), GB[1] [128,256), OUT [256,384), YR [384,512).
-// A barrier used twice per tile (once per chunk parity) waits for parity
-// j = c / 2; once-per-tile barriers wait for the tile index's parity.
+//     32*(w%4) ...) and column part p = w / 4 (a quarter of every row).  Per
+//     tile they form Y = E (TMA tile) + Yd (fp32 rows, loaded a tile ahead
+//     into registers) and store it into the tile's output accumulator OUT,
+//     so that the W2 products add the GatedMLP onto the residual in place;
+//     write h2 = LN2(Y) (statistics reduced over the four parts through
+//     shared memory) over the E tile; compute hid = SiLU(G1) * G3 per 64-wide
+//     hidden chunk from TMEM GB[g%2] into smem HB[g%2]; and store E' = OUT.
+//     The next tile's Y and LN2 run before this tile's E' is read out, so the
+//     tensor cores start the next tile while the epilogue finishes this one.
+//   warp 16 (control, one lane): TMA of the E tiles (one tile ahead), the
+//     [W1c | W3c] chunk images through a two-slot ring (chunk g+1 is fetched
+//     as soon as G(g-1) has consumed its slot), and the MMAs: G(g) =
+//     h2 [W1c | W3c] (one N = 128 product) into GB[g%2] and OUT += hid(g) W2c
+//     with W2 resident in shared memory.
+// Chunks are counted over the CTA's whole tile sequence (g = 4*k + c for its
+// k-th tile), so every ring barrier's parity is (g / 2) % 2.
+// TMEM: GB[0] [0,128), GB[1] [128,256), OUT[k%2] [256 + 128*(k%2), +128).
 constexpr int kFfnEpi = 512;   // epilogue threads
+constexpr int kFfnTiles = 32;  // tile descriptors of a CTA kept in shared memory
+constexpr int kFfnSmem = 1024 + 14 * kBlk + 1024 + kFfnTiles * 16 + 256;
 
 __global__ void __launch_bounds__(kFfnEpi + 32, 1)
-    k_hist_ffn(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ E_in,
-               const bf16* __restrict__ g2, const bf16* __restrict__ b2,
-               const uint8_t* __restrict__ ws, LayerWs Lw, bf16* __restrict__ E_out,
-               unsigned* status) {
+    k_hist_ffn(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ g2,
+               const bf16* __restrict__ b2, const uint8_t* __restrict__ ws, LayerWs Lw,
+               bf16* __restrict__ E_out, unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
-  uint8_t* sE0 = sm;                   // 2 x [128 x 128] bf16: E tile -> h2
+  uint8_t* sE0 = sm;                   // 2 x [128 x 128] bf16: E tile -> h2 (-> LN2 scratch)
   uint8_t* sH0 = sm + 4 * kBlk;        // 2 x [128 x 64]  bf16: hid chunk
-  uint8_t* sW0 = sm + 6 * kBlk;        // 2 x (W1c, W3c, W2c)
-  constexpr uint32_t kSlot = 3 * kBlk;
-  float* red = reinterpret_cast<float*>(sm + 12 * kBlk);           // [2][4][128] LN partials
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 12 * kBlk + 4096);
+  uint8_t* sW13 = sm + 6 * kBlk;       // 2 x [W1c | W3c] ring
+  uint8_t* sW2 = sm + 10 * kBlk;       // W2 image, 4 chunks
+  float* sg = reinterpret_cast<float*>(sm + 14 * kBlk);   // g2, b2 as fp32 [2][128]
+  int4* s_tiles = reinterpret_cast<int4*>(sm + 14 * kBlk + 1024);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 14 * kBlk + 1024 + kFfnTiles * 16);
   uint64_t* barE = bar;        // [2] E tile landed (TMA)
-  uint64_t* barWt = bar + 2;   // [2] weight slot landed
-  uint64_t* barG = bar + 4;    // [2] G(c) in TMEM (MMA commit)
-  uint64_t* barHid = bar + 6;  // [2] hid(c) written, GB read (epilogue arrivals)
-  uint64_t* barW2 = bar + 8;   // [2] OUT += hid(c) W2c done (MMA commit)
-  uint64_t* barH2 = bar + 10;  // h2 written (epilogue arrivals)
+  uint64_t* barWt = bar + 2;   // [2] [W1c | W3c] ring slot landed
+  uint64_t* barG = bar + 4;    // [2] G(g) in TMEM (MMA commit)
+  uint64_t* barHid = bar + 6;  // [2] hid(g) written, GB read (epilogue arrivals)
+  uint64_t* barW2 = bar + 8;   // [2] OUT += hid(g) W2c done (MMA commit)
+  uint64_t* barH2 = bar + 10;  // Y in OUT and h2 written (epilogue arrivals)
   uint64_t* barOut = bar + 11; // all of the tile's MMAs done (MMA commit)
-  uint64_t* barFree = bar + 12;  // epilogue finished the tile (epilogue arrivals)
+  uint64_t* barW2in = bar + 12;  // W2 image landed
   uint64_t* barDrain = bar + 13; // every MMA issued by the control lane is done
   uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 14);
   int* abort_flag = reinterpret_cast<int*>(bar + 15);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
+  const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
+  const int my_tiles =
+      (int)blockIdx.x < n_tiles ? (n_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
   if (threadIdx.x == 0) {
     for (int q = 0; q < 2; ++q) {
       mbar_init(&barE[q], 1);
@@ -1035,85 +1044,85 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
     }
     mbar_init(barH2, kFfnEpi);
     mbar_init(barOut, 1);
-    mbar_init(barFree, kFfnEpi);
+    mbar_init(barW2in, 1);
     mbar_init(barDrain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (threadIdx.x < kD) {
+    sg[threadIdx.x] = __bfloat162float(g2[threadIdx.x]);
+    sg[kD + threadIdx.x] = __bfloat162float(b2[threadIdx.x]);
+  }
+  if ((int)threadIdx.x < my_tiles && threadIdx.x < kFfnTiles)
+    s_tiles[threadIdx.x] = tiles[blockIdx.x + threadIdx.x * gridDim.x];
   if (warp == 0) tmem_alloc(slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
-  const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
-  const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
-  const float* yd = reinterpret_cast<const float*>(ws + Lw.yd);
-  const uint32_t T_OUT = 256, T_Y = 384;
+  constexpr uint32_t T_OUT = 256;
+  auto tile_of = [&](int k) -> int4 {
+    return k < kFfnTiles ? s_tiles[k] : tiles[blockIdx.x + k * gridDim.x];
+  };
+  const int n_chunks = my_tiles * (kF / 64);
 
   if (warp == kFfnEpi / 32) {
-    if (lane == 0) {
-      auto load_chunk = [&](int ch) {
-        uint8_t* dst = sW0 + (ch & 1) * kSlot;
-        uint64_t* b = &barWt[ch & 1];
-        mbar_arrive_expect_tx(b, kSlot);
-        bulk_load(dst, ws + Lw.img_1 + ch * kBlk, kBlk, b);
-        bulk_load(dst + kBlk, ws + Lw.img_3 + ch * kBlk, kBlk, b);
-        bulk_load(dst + 2 * kBlk, ws + Lw.img_2 + ch * kBlk, kBlk, b);
+    if (lane == 0 && my_tiles > 0) {
+      auto load_w13 = [&](int g) {
+        const int s = g & 1, ch = g & 3;
+        mbar_arrive_expect_tx(&barWt[s], 2 * kBlk);
+        bulk_load(sW13 + s * 2 * kBlk, ws + Lw.img_13 + ch * 2 * kBlk, 2 * kBlk, &barWt[s]);
       };
-      auto load_e = [&](int t, int buf) {
-        const int4 tl = tiles[t];
-        mbar_arrive_expect_tx(&barE[buf], 2 * kBlk);
-        tma_load_2d(sE0 + buf * 2 * kBlk, &tmE, 0, tl.y, &barE[buf]);
-        tma_load_2d(sE0 + buf * 2 * kBlk + kBlk, &tmE, 64, tl.y, &barE[buf]);
+      auto load_e = [&](int k) {
+        const int4 tl = tile_of(k);
+        uint8_t* dst = sE0 + (k & 1) * 2 * kBlk;
+        mbar_arrive_expect_tx(&barE[k & 1], 2 * kBlk);
+        tma_load_2d(dst, &tmE, 0, tl.y, &barE[k & 1]);
+        tma_load_2d(dst + kBlk, &tmE, 64, tl.y, &barE[k & 1]);
       };
       prefetch_tmap(&tmE);
-      if ((int)blockIdx.x < n_tiles) load_e(blockIdx.x, 0);
-      int it = 0;
-      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
-        const int cur = it & 1;
-        if (it > 0 && !mbar_wait(barFree, (it - 1) & 1, status, abort_flag)) break;
-        const int tn = t + gridDim.x;
-        if (tn < n_tiles) load_e(tn, cur ^ 1);     // buffer of tile it-1 is free
-        load_chunk(0);
-        load_chunk(1);
-        if (!mbar_wait(barH2, it & 1, status, abort_flag)) break;
+      load_e(0);
+      load_w13(0);
+      if (n_chunks > 1) load_w13(1);
+      mbar_arrive_expect_tx(barW2in, 4 * kBlk);
+      bulk_load(sW2, ws + Lw.img_2, 4 * kBlk, barW2in);
+      bool ok = mbar_wait(barW2in, 0, status, abort_flag);
+      for (int k = 0; k < my_tiles && ok; ++k) {
+        if (!(ok = mbar_wait(barH2, k & 1, status, abort_flag))) break;
         tc_fence_after();
-        const uint32_t a_h2 = smem_u32(sE0 + cur * 2 * kBlk);
-        bool ok = true;
-        for (int c = 0; c < kF / 64 && ok; ++c) {
-          const int sb = c & 1;
-          ok = mbar_wait(&barWt[sb], (uint32_t)(c >> 1), status, abort_flag);
-          if (!ok) break;
+        const uint32_t a_h2 = smem_u32(sE0 + (k & 1) * 2 * kBlk);
+        const uint32_t t_out = tmem + T_OUT + (k & 1) * 128;
+        for (int c = 0; c < kF / 64; ++c) {
+          const int g = k * (kF / 64) + c, s = g & 1;
+          if (!(ok = mbar_wait(&barWt[s], (uint32_t)((g >> 1) & 1), status, abort_flag))) break;
           tc_fence_after();
-          const uint32_t wslot = smem_u32(sW0 + sb * kSlot);
-          mma_tile(tmem + sb * 128, a_h2, kBlk, wslot, 8192, 64, 128, false);
-          mma_tile(tmem + sb * 128 + 64, a_h2, kBlk, wslot + kBlk, 8192, 64, 128, false);
-          mma_commit(&barG[sb]);
+          mma_tile(tmem + s * 128, a_h2, kBlk, smem_u32(sW13 + s * 2 * kBlk), kBlk, 128, 128, false);
+          mma_commit(&barG[s]);
+          if (g >= 1) {
+            // G(g-1) done: its ring slot takes chunk g+1; at a tile's first
+            // chunk it also means the previous tile's h2 buffer is free
+            if (!(ok = mbar_wait(&barG[s ^ 1], (uint32_t)(((g - 1) >> 1) & 1), status, abort_flag)))
+              break;
+            if (g + 1 < n_chunks) load_w13(g + 1);
+          }
+          if (c == 0 && k + 1 < my_tiles) load_e(k + 1);
           if (c >= 1) {
-            const int pc = c - 1, pb = pc & 1;
-            ok = mbar_wait(&barHid[pb], (uint32_t)(pc >> 1), status, abort_flag);
-            if (!ok) break;
+            const int pg = g - 1, pb = pg & 1;
+            if (!(ok = mbar_wait(&barHid[pb], (uint32_t)((pg >> 1) & 1), status, abort_flag))) break;
             tc_fence_after();
-            mma_tile(tmem + T_OUT, smem_u32(sH0 + pb * kBlk), kBlk,
-                     smem_u32(sW0 + pb * kSlot + 2 * kBlk), kBlk, 128, 64, pc > 0);
+            mma_tile(t_out, smem_u32(sH0 + pb * kBlk), kBlk, smem_u32(sW2 + (c - 1) * kBlk), kBlk,
+                     128, 64, true);
             mma_commit(&barW2[pb]);
-            if (c + 1 < kF / 64) {       // slot pb is free once W2(pc) is done
-              ok = mbar_wait(&barW2[pb], (uint32_t)(pc >> 1), status, abort_flag);
-              if (!ok) break;
-              load_chunk(c + 1);
-            }
           }
         }
         if (!ok) break;
-        {
-          const int pc = kF / 64 - 1, pb = pc & 1;
-          if (!mbar_wait(&barHid[pb], (uint32_t)(pc >> 1), status, abort_flag)) break;
-          tc_fence_after();
-          mma_tile(tmem + T_OUT, smem_u32(sH0 + pb * kBlk), kBlk,
-                   smem_u32(sW0 + pb * kSlot + 2 * kBlk), kBlk, 128, 64, true);
-          mma_commit(&barW2[pb]);
-          mma_commit(barOut);
-        }
+        const int lg = k * (kF / 64) + kF / 64 - 1, lb = lg & 1;
+        if (!(ok = mbar_wait(&barHid[lb], (uint32_t)((lg >> 1) & 1), status, abort_flag))) break;
+        tc_fence_after();
+        mma_tile(t_out, smem_u32(sH0 + lb * kBlk), kBlk, smem_u32(sW2 + (kF / 64 - 1) * kBlk), kBlk,
+                 128, 64, true);
+        mma_commit(&barW2[lb]);
+        mma_commit(barOut);
       }
       // drain: no MMA of ours may be in flight when TMEM is freed
       mma_commit(barDrain);
@@ -1124,102 +1133,120 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
     const int row = q4 * 32 + lane;
     const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16);
     const int c0 = part * 32;                      // this thread's 32 columns of a row
-    int it = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
-      const int cur = it & 1;
-      const int4 tl = tiles[t];
-      const int r0 = tl.y, nv = tl.z;
-      uint8_t* sE = sE0 + cur * 2 * kBlk;
-      // Yd part first: its round trip overlaps the wait for the E tile
-      float y[32];
-      if (row < nv) {
-        const float4* src = reinterpret_cast<const float4*>(yd + (int64_t)(r0 + row) * kD + c0);
+    const float* yd = reinterpret_cast<const float*>(ws + Lw.yd);
+    float yn[32];                                  // Yd of the next tile
+    auto load_yd = [&](int k) {
+      const int4 tl = tile_of(k);
+      if (row < tl.z) {
+        const float4* src = reinterpret_cast<const float4*>(yd + (int64_t)(tl.y + row) * kD + c0);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float4 v = src[q];
-          y[4 * q] = v.x; y[4 * q + 1] = v.y; y[4 * q + 2] = v.z; y[4 * q + 3] = v.w;
+          yn[4 * q] = v.x; yn[4 * q + 1] = v.y; yn[4 * q + 2] = v.z; yn[4 * q + 3] = v.w;
         }
       } else {
 #pragma unroll
-        for (int k = 0; k < 32; ++k) y[k] = 0.f;
+        for (int j = 0; j < 32; ++j) yn[j] = 0.f;
       }
-      mbar_wait(&barE[cur], (uint32_t)((it >> 1) & 1), status, abort_flag);
+    };
+    // Y(j) = E + Yd into OUT[j%2], h2(j) = LN2(Y(j)) over E tile j%2.  The
+    // reduction scratch is the other E buffer: it holds h2(j-1), whose last
+    // reader G(j-1, 3) has completed by the time the epilogue gets here, and
+    // E(j+1) is loaded into it only after this tile's barH2 completes.
+    auto y_ln2 = [&](int j) {
+      uint8_t* sE = sE0 + (j & 1) * 2 * kBlk;
+      float* red1 = reinterpret_cast<float*>(sE0 + ((j & 1) ^ 1) * 2 * kBlk);
+      float* red2 = red1 + 4 * 128;
+      float y[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) y[i] = yn[i];
+      mbar_wait(&barE[j & 1], (uint32_t)((j >> 1) & 1), status, abort_flag);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float e[8];
         unpack8(sw_ld16(sE, kBlk, row, c0 + q * 8), e);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) y[q * 8 + k] += e[k];
+        for (int i = 0; i < 8; ++i) y[q * 8 + i] += e[i];
       }
-      tmem_st16(ta + T_Y + c0, y);
-      tmem_st16(ta + T_Y + c0 + 16, y + 16);
-      tmem_st_wait();
-      // LN2 statistics over the row's four parts
-      float* rs = red + (it & 1) * 512;
+      const uint32_t t_out = ta + T_OUT + (j & 1) * 128 + c0;
+      tmem_st16(t_out, y);
+      tmem_st16(t_out + 16, y + 16);
       {
         float s1 = 0.f;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) s1 += y[k];
-        rs[part * 128 + row] = s1;
+        for (int i = 0; i < 32; ++i) s1 += y[i];
+        red1[part * 128 + row] = s1;
       }
       named_bar_sync(1, kFfnEpi);
-      const float mu = (rs[row] + rs[128 + row] + rs[256 + row] + rs[384 + row]) * (1.0f / kD);
-      named_bar_sync(1, kFfnEpi);
+      const float mu =
+          (red1[row] + red1[128 + row] + red1[256 + row] + red1[384 + row]) * (1.0f / kD);
       {
         float s2 = 0.f;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) { const float d0 = y[k] - mu; s2 += d0 * d0; }
-        rs[part * 128 + row] = s2;
+        for (int i = 0; i < 32; ++i) { const float d0 = y[i] - mu; s2 += d0 * d0; }
+        red2[part * 128 + row] = s2;
       }
       named_bar_sync(1, kFfnEpi);
       const float rstd =
-          rsqrtf((rs[row] + rs[128 + row] + rs[256 + row] + rs[384 + row]) * (1.0f / kD) + kLnEps);
+          rsqrtf((red2[row] + red2[128 + row] + red2[256 + row] + red2[384 + row]) * (1.0f / kD) +
+                 kLnEps);
 #pragma unroll
-      for (int k = 0; k < 32; ++k)
-        y[k] = (y[k] - mu) * rstd * __bfloat162float(g2[c0 + k]) + __bfloat162float(b2[c0 + k]);
+      for (int q = 0; q < 8; ++q) {
+        const float4 gv = reinterpret_cast<const float4*>(sg + c0)[q];
+        const float4 bv = reinterpret_cast<const float4*>(sg + kD + c0)[q];
+        y[4 * q] = (y[4 * q] - mu) * rstd * gv.x + bv.x;
+        y[4 * q + 1] = (y[4 * q + 1] - mu) * rstd * gv.y + bv.y;
+        y[4 * q + 2] = (y[4 * q + 2] - mu) * rstd * gv.z + bv.z;
+        y[4 * q + 3] = (y[4 * q + 3] - mu) * rstd * gv.w + bv.w;
+      }
 #pragma unroll
       for (int q = 0; q < 4; ++q) sw_st16(sE, kBlk, row, c0 + q * 8, pack8(y + q * 8));
+      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(barH2);
+      if (j + 1 < my_tiles) load_yd(j + 1);   // in flight during the next chunk loop
+    };
+    if (my_tiles > 0) {
+      load_yd(0);
+      y_ln2(0);
+    }
+    for (int k = 0; k < my_tiles; ++k) {
       for (int c = 0; c < kF / 64; ++c) {
-        const int sb = c & 1;
-        mbar_wait(&barG[sb], (uint32_t)(c >> 1), status, abort_flag);
+        const int g = k * (kF / 64) + c, sb = g & 1;
+        mbar_wait(&barG[sb], (uint32_t)((g >> 1) & 1), status, abort_flag);
         tc_fence_after();
-        float g[16], gg[16];
-        tmem_ld16(ta + sb * 128 + part * 16, g);
-        tmem_ld16(ta + sb * 128 + 64 + part * 16, gg);
+        float gt[16], gu[16];
+        tmem_ld16(ta + sb * 128 + part * 16, gt);
+        tmem_ld16(ta + sb * 128 + 64 + part * 16, gu);
         tmem_ld_wait();
 #pragma unroll
-        for (int k = 0; k < 16; ++k) g[k] = silu_fast(g[k]) * gg[k];
-        // hid(c) reuses the buffer of hid(c-2): wait until its W2 MMA is done
-        if (c >= 2) mbar_wait(&barW2[sb], 0u, status, abort_flag);
+        for (int i = 0; i < 16; ++i) gt[i] = silu_fast(gt[i]) * gu[i];
+        // hid(g) reuses the buffer of hid(g-2): wait until its W2 MMA is done
+        if (g >= 2) mbar_wait(&barW2[sb], (uint32_t)(((g - 2) >> 1) & 1), status, abort_flag);
         uint8_t* sH = sH0 + sb * kBlk;
-        sw_st16(sH, kBlk, row, part * 16, pack8(g));
-        sw_st16(sH, kBlk, row, part * 16 + 8, pack8(g + 8));
+        sw_st16(sH, kBlk, row, part * 16, pack8(gt));
+        sw_st16(sH, kBlk, row, part * 16 + 8, pack8(gt + 8));
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&barHid[sb]);
       }
-      mbar_wait(barOut, (uint32_t)(it & 1), status, abort_flag);
+      if (k + 1 < my_tiles) y_ln2(k + 1);
+      mbar_wait(barOut, (uint32_t)(k & 1), status, abort_flag);
       tc_fence_after();
-      {
-        float o[32], yy[32];
-        tmem_ld16(ta + T_OUT + c0, o);
-        tmem_ld16(ta + T_OUT + c0 + 16, o + 16);
-        tmem_ld16(ta + T_Y + c0, yy);
-        tmem_ld16(ta + T_Y + c0 + 16, yy + 16);
+      const int4 tl = tile_of(k);
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        float o[16];
+        tmem_ld16(ta + T_OUT + (k & 1) * 128 + c0 + hf * 16, o);
         tmem_ld_wait();
-#pragma unroll
-        for (int k = 0; k < 32; ++k) o[k] += yy[k];
-        if (row < nv) {
-          uint4* dst = reinterpret_cast<uint4*>(E_out + (int64_t)(r0 + row) * kD + c0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = pack8(o + q * 8);
+        if (row < tl.z) {
+          uint4* dst = reinterpret_cast<uint4*>(E_out + (int64_t)(tl.y + row) * kD + c0 + hf * 16);
+          dst[0] = pack8(o);
+          dst[1] = pack8(o + 8);
         }
       }
       tc_fence_before();
-      mbar_arrive(barFree);
     }
   }
   tc_fence_before();
@@ -1249,7 +1276,7 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sHh = sm + 4 * kBlk;
   uint8_t* sHl = sm + 5 * kBlk;
   uint8_t* sWo = sm + 6 * kBlk;
-  uint8_t* sW = sm + 8 * kBlk;      // W1c, W3c, W2c of chunk ch
+  uint8_t* sW = sm + 8 * kBlk;      // [W1c | W3c] image, W2c of chunk ch
   float* red = reinterpret_cast<float*>(sm + 11 * kBlk);
   const int ch = blockIdx.y;
   Cta c;
@@ -1259,8 +1286,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
     bulk_load(sWo, ws_c + Lw.img_o, 2 * kBlk, &c.bar[0]);
     mbar_arrive_expect_tx(&c.bar[2], 3 * kBlk);
-    bulk_load(sW, ws_c + Lw.img_1 + ch * kBlk, kBlk, &c.bar[2]);
-    bulk_load(sW + kBlk, ws_c + Lw.img_3 + ch * kBlk, kBlk, &c.bar[2]);
+    bulk_load(sW, ws_c + Lw.img_13 + ch * 2 * kBlk, 2 * kBlk, &c.bar[2]);
     bulk_load(sW + 2 * kBlk, ws_c + Lw.img_2 + ch * kBlk, kBlk, &c.bar[2]);
   }
   const int warp = threadIdx.x >> 5;
@@ -1335,10 +1361,9 @@ __global__ void __launch_bounds__(512, 1)
   mbar_wait(&c.bar[2], 0, status, c.abort_flag);
   if (threadIdx.x == 0) {
     tc_fence_after();
-    mma_tile(c.tmem + 128, smem_u32(sAh), kBlk, smem_u32(sW), 8192, 64, 128, false);
-    mma_tile(c.tmem + 128, smem_u32(sAl), kBlk, smem_u32(sW), 8192, 64, 128, true);
-    mma_tile(c.tmem + 192, smem_u32(sAh), kBlk, smem_u32(sW + kBlk), 8192, 64, 128, false);
-    mma_tile(c.tmem + 192, smem_u32(sAl), kBlk, smem_u32(sW + kBlk), 8192, 64, 128, true);
+    // [G1 | G3] of the chunk in one N = 128 product
+    mma_tile(c.tmem + 128, smem_u32(sAh), kBlk, smem_u32(sW), kBlk, 128, 128, false);
+    mma_tile(c.tmem + 128, smem_u32(sAl), kBlk, smem_u32(sW), kBlk, 128, 128, true);
   }
   cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
   {
@@ -1445,10 +1470,9 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
       note_launches(1);
     }
     if (!last) {
-      const int smem = 1024 + 12 * kBlk + 4096 + 256;
-      if (!set_smem(k_hist_ffn, smem)) return LIME_ERR_CUDA;
-      k_hist_ffn<<<grid, kFfnEpi + 32, smem, st>>>(tmE, (const bf16*)E_in, (const bf16*)w.g2,
-                                                   (const bf16*)w.b2, ws, Lw, (bf16*)E_out, status);
+      if (!set_smem(k_hist_ffn, kFfnSmem)) return LIME_ERR_CUDA;
+      k_hist_ffn<<<grid, kFfnEpi + 32, kFfnSmem, st>>>(tmE, (const bf16*)w.g2, (const bf16*)w.b2,
+                                                       ws, Lw, (bf16*)E_out, status);
       note_launches(1);
     }
   }

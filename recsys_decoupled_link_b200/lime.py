@@ -58,7 +58,7 @@ def _load() -> ctypes.CDLL:
         "lime_workspace_bytes": (SZ, [D, I64, I64]),
         "lime_workspace_init": (I32, [P, SZ, P]),
         "lime_build_qk_cache": (I32, [D, P, I64, P, P, P, P, P, SZ, P]),
-        "lime_context_links": (I32, [D, I64, P, P, ctypes.POINTER(lime_ctx_mlp), P, P]),
+        "lime_context_links": (I32, [D, I64, P, P, ctypes.POINTER(lime_ctx_mlp), P, P, SZ, P]),
         "lime_xor_layer": (I32, [D, I64, P, I64, P, P, ctypes.POINTER(lime_layer_w), P, P, P,
                                  SZ, P]),
         "lime_score_candidates": (I32, [D, I64, P, I64, P, P, I64, P, P, P, SZ, P]),
@@ -146,13 +146,13 @@ def lime_build_qk_cache_noalloc(dims, T, L, Wq_c, Wk_c, cache_out, stream=None):
         _ptr(cache_out), _stream(stream)))
 
 
-def lime_context_links(dims, L, ctx, Wc1, bc1, Wc2, bc2, LC_out, stream=None):
+def lime_context_links(dims, L, ctx, Wc1, bc1, Wc2, bc2, LC_out, ws: Workspace, stream=None):
     w = lime_ctx_mlp(Wc1.data_ptr(), bc1.data_ptr(), Wc2.data_ptr(), bc2.data_ptr())
     for t in (Wc1, bc1, Wc2, bc2):
         _ptr(t)
     _check("lime_context_links", _lib.lime_context_links(
         ctypes.byref(dims), ctx.shape[0], _ptr(L), _ptr(ctx), ctypes.byref(w),
-        _ptr(LC_out), _stream(stream)))
+        _ptr(LC_out), ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def layer_struct(weights: Sequence[torch.Tensor]) -> lime_layer_w:

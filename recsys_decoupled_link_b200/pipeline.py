@@ -83,7 +83,7 @@ def alloc(x: DeviceInputs, n_items: Optional[int] = None, device="cuda") -> Buff
 def user_encode(x: DeviceInputs, buf: Buffers, stream=None) -> torch.Tensor:
     """Context links then the layer stack; returns L^P [B, l, d]."""
     if x.ctx_w is not None:
-        lime.lime_context_links(x.dims, x.L, x.ctx, *x.ctx_w, buf.LC, stream=stream)
+        lime.lime_context_links(x.dims, x.L, x.ctx, *x.ctx_w, buf.LC, buf.ws, stream=stream)
         Z = buf.LC
     else:
         Z = x.Z0

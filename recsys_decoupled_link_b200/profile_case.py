@@ -36,7 +36,7 @@ def main():
     buf = pipeline.alloc(x)
     Z = buf.LC
     if x.ctx_w is not None:
-        lime.lime_context_links(x.dims, x.L, x.ctx, *x.ctx_w, buf.LC)
+        lime.lime_context_links(x.dims, x.L, x.ctx, *x.ctx_w, buf.LC, buf.ws)
     else:
         Z = x.Z0
     if a.phase == "score":

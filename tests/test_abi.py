@@ -103,4 +103,4 @@ def test_host_validation_of_scoring_and_cache(lime):
     nodims = lime.make_dims(128, 4, 32, 256, 0, "bf16")
     mlp = lime.lime_ctx_mlp(0x10000, 0x20000, 0x30000, 0x40000)
     assert c(ctypes.byref(nodims), 2, 0x50000, 0x60000, ctypes.byref(mlp), 0x70000,
-             None) == lime.LIME_ERR_SHAPE
+             0x1000000, nws, None) == lime.LIME_ERR_SHAPE

@@ -23,7 +23,7 @@ pytestmark = pytest.mark.gpu
 def run_user_side(x, buf):
     """Context links + layers through the C ABI; returns Z0 and per-layer (E', Z')."""
     if x.ctx_w is not None:
-        lime.lime_context_links(x.dims, x.L, x.ctx, *x.ctx_w, buf.LC)
+        lime.lime_context_links(x.dims, x.L, x.ctx, *x.ctx_w, buf.LC, buf.ws)
         Z = buf.LC.clone()
     else:
         Z = x.Z0
@@ -118,6 +118,24 @@ def test_scoring_many_tiles_per_user(l):
     # few users with many candidates: each scoring CTA walks several tiles
     w = synth.workload("standard", B=2, l=l, n_items=20_000, layers=1, cand=("uniform",))
     check_workload(w, n_hist=[130, 40], n_cand=[5000, 3333])
+
+
+@pytest.mark.parametrize("c,l,B,dtype", [(64, 32, 5, "bf16"), (128, 16, 37, "bf16"),
+                                         (64, 64, 3, "bf16"), (64, 32, 1000, "bf16"),
+                                         (64, 32, 5, "f32")])
+def test_context_links(c, l, B, dtype):
+    # ragged last tile of B*l rows (B=37, l=16: 592 rows), more 128-row tiles
+    # than SMs (B=1000: 250 tiles), d + c = 192 and 256, and the fp32 path
+    w = synth.workload("standard", B=B, l=l, c=c, n_items=1000, layers=1, dtype=dtype)
+    us = synth.user_side(w, [1] * B)
+    cs = synth.candidate_side(w, [1] * B)
+    x = pipeline.to_device(w, us, cs, synth.item_table(w))
+    buf = pipeline.alloc(x)
+    buf.LC.fill_(float("nan"))
+    lime.lime_context_links(x.dims, x.L, x.ctx, *x.ctx_w, buf.LC, buf.ws)
+    torch.cuda.synchronize()
+    assert lime.lime_get_status(buf.ws) == 0
+    assert_close(buf.LC, oracle_Z0(w, us), dtype, "context links")
 
 
 def test_single_user_single_token():

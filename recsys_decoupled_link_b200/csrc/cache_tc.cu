@@ -55,6 +55,8 @@ __global__ void __launch_bounds__(128) k_fold_g_img(const T* __restrict__ L, con
   // link's key, split over blockDim/d_h partial sums), then G^T row j.
   __shared__ float part[8][64];
   __shared__ float kc[64];
+  pdl_launch();
+  pdl_wait();
   const int j = blockIdx.x, h = j / l, k = j % l, dh = d / H, HL = H * l;
   const int c = threadIdx.x % dh, q = threadIdx.x / dh, nq = blockDim.x / dh;
   {
@@ -120,6 +122,8 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_launch();
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -257,9 +261,8 @@ int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, unsigne
     return LIME_ERR_CUDA;
   const int n_tiles = (int)((n + kBM - 1) / kBM);
   const int grid = n_tiles < num_sms() ? n_tiles : num_sms();
-  k_cache_tc<HL, L><<<grid, 320, C::SMEM, st>>>(tmT, tmC, img, n_tiles, status);
-  note_launches(1);
-  return LIME_OK;
+  return launch_pdl(k_cache_tc<HL, L>, dim3(grid), dim3(320), C::SMEM, st, 1, tmT, tmC, img,
+                    n_tiles, status);
 }
 
 }  // namespace
@@ -280,9 +283,9 @@ int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void
   const int HL = D.H * D.l;
   bf16* img = reinterpret_cast<bf16*>(ws);
   const float scale = 1.0f / sqrtf((float)(D.d / D.H));
-  k_fold_g_img<bf16><<<HL, 128, 0, st>>>((const bf16*)L, (const bf16*)Wq, (const bf16*)Wk, D.d,
-                                         D.H, D.l, scale, img);
-  note_launches(1);
+  int rc = launch_pdl(k_fold_g_img<bf16>, dim3(HL), dim3(128), 0, st, 1, (const bf16*)L,
+                      (const bf16*)Wq, (const bf16*)Wk, D.d, D.H, D.l, scale, img);
+  if (rc) return rc;
   if (n == 0) return LIME_OK;
   switch (HL * 1000 + D.l) {
     case 64016: return launch_cache<64, 16>(T, n, img, cache, status, st);

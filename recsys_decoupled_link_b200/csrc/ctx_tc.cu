@@ -51,6 +51,10 @@ __global__ void __launch_bounds__(512, 1)
     fence_mbar_init();
   }
   if (tid < 32) tmem_alloc(slot, 256);
+  tc_fence_before();
+  __syncthreads();
+  pdl_launch();
+  pdl_wait();
   // weights: 16-byte chunk (k, n8) of a row-major [K x 128] matrix goes to
   // row k, columns n8*8.. of the MN-major image
   {
@@ -165,11 +169,9 @@ int fast_context_links(const lime_dims& D, int64_t B, const void* L, const void*
     return LIME_ERR_CUDA;
   int64_t grid = (rows + 127) / 128;
   if (grid > num_sms()) grid = num_sms();
-  k_context_tc<<<(unsigned)grid, 512, smem, st>>>(
-      D.c, D.l, rows, (const bf16*)L, (const bf16*)ctx, (const bf16*)w.Wc1, (const bf16*)w.bc1,
-      (const bf16*)w.Wc2, (const bf16*)w.bc2, (bf16*)LC, status);
-  note_launches(1);
-  return LIME_OK;
+  return launch_pdl(k_context_tc, dim3((unsigned)grid), dim3(512), smem, st, 1, D.c, D.l, rows,
+                    (const bf16*)L, (const bf16*)ctx, (const bf16*)w.Wc1, (const bf16*)w.bc1,
+                    (const bf16*)w.Wc2, (const bf16*)w.bc2, (bf16*)LC, status);
 }
 
 }  // namespace lime

@@ -4,6 +4,36 @@
 
 namespace lime {
 
+// Launches a kernel that follows the pdl_launch / pdl_wait protocol with
+// programmatic stream serialization (its launch and prologue overlap the
+// previous kernel's tail), optionally as clusters of cluster_y CTAs along y.
+template <typename... KArgs, typename... Args>
+inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, unsigned cluster_y, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_y > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 1;
+    attr[n].val.clusterDim.y = cluster_y;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) return LIME_ERR_CUDA;
+  note_launches(1);
+  return LIME_OK;
+}
+
 size_t fast_ws_bytes(const lime_dims& D, int64_t B, int64_t total_hist);
 size_t fast_cache_ws_bytes(const lime_dims& D);
 size_t fast_layer_ws_bytes(const lime_dims& D, int64_t B, int64_t total_hist);

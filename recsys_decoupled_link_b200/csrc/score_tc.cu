@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(128)
   int* abort_flag = reinterpret_cast<int*>(bar + 2);
   int64_t* s_ids = reinterpret_cast<int64_t*>(bar + 4);   // [128] candidate IDs of the tile
 
+  pdl_wait();
   const int64_t u = blockIdx.x;
   int64_t a, b;
   user_range(off, u, B, total, &a, &b, status);
@@ -61,6 +62,8 @@ __global__ void __launch_bounds__(128)
     fence_mbar_init();
   }
   if (i < 32) tmem_alloc(slot, 128);
+  __syncthreads();
+  pdl_launch();   // after the TMEM allocation (the next kernel may allocate before it waits)
   // The first tile's candidate ID is loaded together with L^P_u (one memory
   // round trip for both).
   int32_t first_id = -1;
@@ -185,10 +188,8 @@ int launch_score(int64_t B, const void* cache, int64_t n_items, const int32_t* i
   if (G < 1) G = 1;
   if (G > 65535) G = 65535;
   dim3 grid((unsigned)B, (unsigned)G);
-  k_score_tc<L><<<grid, 128, smem, st>>>((const bf16*)cache, n_items, ids, off, B, total,
-                                          (const bf16*)LP, (bf16*)O, status);
-  note_launches(1);
-  return LIME_OK;
+  return launch_pdl(k_score_tc<L>, grid, dim3(128), smem, st, 1, (const bf16*)cache, n_items,
+                    ids, off, B, total, (const bf16*)LP, (bf16*)O, status);
 }
 
 }  // namespace

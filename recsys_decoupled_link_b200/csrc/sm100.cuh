@@ -75,6 +75,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   return false;
 }
 
+// Programmatic dependent launch.  Kernels launched with launch_pdl call
+// pdl_launch once their TMEM is allocated (so that the next kernel's CTAs,
+// which may allocate TMEM before they wait, cannot take it first) and
+// pdl_wait before their first global-memory access: the previous kernel in
+// the stream has then completed and its writes are visible.
+__device__ __forceinline__ void pdl_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -331,6 +341,43 @@ __device__ __forceinline__ void mma_tile_bmn(uint32_t d_tmem, uint32_t a_base, u
     mma_bf16(d_tmem, sdesc_sw128(a_base + (k >> 2) * a_blk + off),
              sdesc_sw128_mn(b_base + (uint32_t)k * 2048, b_lbo), idesc, accumulate || k > 0);
   }
+}
+
+// ------------------------------------------------------------- clusters
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+// Bulk copy from this CTA's shared memory to another CTA's (dst and mbar are
+// cluster addresses from cluster_map); completes `bytes` on that CTA's
+// mbarrier.  Both addresses 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_push_cluster(uint32_t dst, const void* src, uint32_t bytes,
+                                                  uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "r"(smem_u32(src)), "r"(bytes), "r"(mbar)
+      : "memory");
+}
+// Every thread of every CTA of the cluster: release this CTA's shared-memory
+// writes and acquire the others'.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
 }
 
 // Cooperative, coalesced store of the first `nv` rows of a [128 x 128] bf16

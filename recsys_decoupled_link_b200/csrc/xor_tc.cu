@@ -55,7 +55,7 @@ constexpr int kRec = 36;  // floats per link-branch record: max, sum, 32 weighte
 struct LayerWs {
   size_t img_q, img_k, img_v, img_o, img_13, img_2;
   size_t sched, tiles, tile_start;
-  size_t qe, ke, ve, yd, uimg, part, bmerge, zpart;
+  size_t qe, ke, ve, yd, uimg, part;
   size_t total;
   int64_t max_tiles;
   uint32_t uimg_bytes;
@@ -89,8 +89,6 @@ LayerWs layer_ws(int l, int64_t B, int64_t nh) {
   w.uimg_bytes = uimg_bytes(l);
   w.uimg = take((size_t)B * w.uimg_bytes);
   w.part = take((size_t)w.max_tiles * kH * l * kRec * 4);
-  w.bmerge = take((size_t)B * l * kD * 4);
-  w.zpart = take((size_t)5 * B * l * kD * 4);
   w.total = o;
   return w;
 }
@@ -188,6 +186,23 @@ __device__ __forceinline__ void split_row_st(uint8_t* hi, uint8_t* lo, uint32_t 
   }
 }
 
+// Writes 32 values (columns c0 .. c0+31 of row `row`) as hi = bf16(x) and
+// lo = bf16(x - hi) into two [128 x 128] swizzled operands.
+__device__ __forceinline__ void split_part_st(uint8_t* hi, uint8_t* lo, int row, int c0,
+                                              const float* x) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float h8[8], l8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      h8[k] = __bfloat162float(__float2bfloat16_rn(x[q * 8 + k]));
+      l8[k] = x[q * 8 + k] - h8[k];
+    }
+    sw_st16(hi, kBlk, row, c0 + q * 8, pack8(h8));
+    sw_st16(lo, kBlk, row, c0 + q * 8, pack8(l8));
+  }
+}
+
 __device__ __forceinline__ float silu_fast(float x) { return x / (1.0f + __expf(-x)); }
 
 // fp32 [rows x 128] staging: row r is 512 bytes, its 16-byte chunk c sits at
@@ -233,6 +248,8 @@ __device__ __forceinline__ void cta_setup(uint8_t* bar_area, int nbar, Cta& c,
   __syncthreads();
   tc_fence_after();
   c.tmem = *c.slot;
+  pdl_launch();
+  pdl_wait();
 }
 
 __device__ __forceinline__ void cta_teardown(Cta& c) {
@@ -271,6 +288,8 @@ __global__ void __launch_bounds__(1024) k_prep_weights(
     const bf16* __restrict__ Wo, const bf16* __restrict__ W1, const bf16* __restrict__ W3,
     const bf16* __restrict__ W2, uint8_t* __restrict__ ws, LayerWs L,
     const int64_t* __restrict__ off, int64_t B, int64_t nh, unsigned* status) {
+  pdl_launch();
+  pdl_wait();
   if (blockIdx.x == 0) {
     schedule_tiles(off, B, nh, (int)L.max_tiles, reinterpret_cast<int*>(ws + L.sched),
                    reinterpret_cast<int4*>(ws + L.tiles), reinterpret_cast<int*>(ws + L.tile_start),
@@ -431,49 +450,72 @@ __global__ void __launch_bounds__(512)
   tmem_ld16(quad_addr(c) + c0, v);          // warp-collective: every thread loads
   tmem_ld16(quad_addr(c) + c0 + 16, v + 16);
   tmem_ld_wait();
-  if (valid) {
-    const int64_t u = R / L;
-    const int k = (int)(R % L);
-    uint8_t* img = ws + Lw.uimg + u * Lw.uimg_bytes;
-    if (which == 1) {           // s·K_Z row k
+  if (which != 2) {
 #pragma unroll
-      for (int i2 = 0; i2 < 32; ++i2) v[i2] *= scale;
+    for (int i2 = 0; i2 < 32; ++i2) v[i2] *= scale;
+  }
+  float lo[32];
+  if (which == 0) {         // the link query is kept as hi + lo bf16 halves
 #pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(img, (uint32_t)L * 128, k, c0 + q * 8, pack8(v + q * 8));
-    } else if (which == 2) {    // V_Z^T column k, zero padding columns k + L, ... < 64
-      uint8_t* vzt = img + kz_bytes(L);
-      for (int cc = 0; cc < 32; ++cc) {
-        *reinterpret_cast<bf16*>(vzt + sw128_offset(c0 + cc, k)) = __float2bfloat16_rn(v[cc]);
-        for (int kp = k + L; kp < 64; kp += L)
-          *reinterpret_cast<bf16*>(vzt + sw128_offset(c0 + cc, kp)) = __float2bfloat16_rn(0.f);
-      }
-    } else {                    // block-diagonal s·Q_Z rows h*L + k (hi, lo); rows >= 4L zero
-      uint8_t* qbd = img + kz_bytes(L) + kBlk;
-      uint8_t* qbl = qbd + 2 * kBlk;
-      float lo[32];
+    for (int i2 = 0; i2 < 32; ++i2) {
+      const float x = v[i2];
+      v[i2] = __bfloat162float(__float2bfloat16_rn(x));
+      lo[i2] = x - v[i2];
+    }
+  }
+  // The images are built per user in shared memory (the operands of the MMA
+  // are dead) and copied out with coalesced 16-byte stores.  Piece per user:
+  // s·K_Z (L*256 bytes), V_Z^T (one 16 KB block) or the block-diagonal s·Q_Z
+  // hi + lo (four 16 KB blocks).
+  constexpr int UP = kTile / L;                               // users per tile
+  const uint32_t piece = which == 0 ? 4 * kBlk : which == 1 ? kz_bytes(L) : kBlk;
+  const uint32_t img_off = which == 0 ? kz_bytes(L) + kBlk : which == 1 ? 0 : kz_bytes(L);
+  const int upp = which == 0 ? 1 : which == 1 ? UP : (UP < 4 ? UP : 4);   // users per pass
+  uint8_t* stage = sm;                                        // 96 KB: sAh, sAl, sW
+  const int ju = r / L, k = r % L;
+  const int64_t u0 = (int64_t)blockIdx.x * UP;
+  const int n_users = (int)((nrows - (int64_t)blockIdx.x * kTile) / L) < UP
+                          ? (int)((nrows - (int64_t)blockIdx.x * kTile) / L) : UP;
+  for (int j0 = 0; j0 < n_users; j0 += upp) {
+    __syncthreads();   // the staging area is free (MMA operands, previous pass)
+    if (ju >= j0 && ju < j0 + upp && valid) {
+      uint8_t* img = stage + (uint32_t)(ju - j0) * piece;
+      if (which == 1) {           // s·K_Z row k
 #pragma unroll
-      for (int i2 = 0; i2 < 32; ++i2) {
-        const float x = v[i2] * scale;
-        v[i2] = __bfloat162float(__float2bfloat16_rn(x));
-        lo[i2] = x - v[i2];
-      }
-      const uint4 z4 = make_uint4(0, 0, 0, 0);
-      // this thread's 32 columns belong to head `part`
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 hv = pack8(v + q * 8), lv = pack8(lo + q * 8);
-#pragma unroll
-        for (int h = 0; h < kH; ++h) {
-          sw_st16(qbd, kBlk, h * L + k, c0 + q * 8, h == part ? hv : z4);
-          sw_st16(qbl, kBlk, h * L + k, c0 + q * 8, h == part ? lv : z4);
+        for (int q = 0; q < 4; ++q) sw_st16(img, (uint32_t)L * 128, k, c0 + q * 8, pack8(v + q * 8));
+      } else if (which == 2) {    // V_Z^T column k; columns k + L, k + 2L, ... < 64 are zero
+        for (int cc = 0; cc < 32; ++cc) {
+          *reinterpret_cast<bf16*>(img + sw128_offset(c0 + cc, k)) = __float2bfloat16_rn(v[cc]);
+          for (int kp = k + L; kp < 64; kp += L)
+            *reinterpret_cast<bf16*>(img + sw128_offset(c0 + cc, kp)) = __float2bfloat16_rn(0.f);
         }
-      }
-      for (int p = kH * L + k; p < kTile; p += L)
+      } else {                    // rows h*L + k: head `part` holds s·Q_Z, the rest zero
+        uint8_t* qbl = img + 2 * kBlk;
+        const uint4 z4 = make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          sw_st16(qbd, kBlk, p, c0 + q * 8, z4);
-          sw_st16(qbl, kBlk, p, c0 + q * 8, z4);
+          const uint4 hv = pack8(v + q * 8), lv = pack8(lo + q * 8);
+#pragma unroll
+          for (int h = 0; h < kH; ++h) {
+            sw_st16(img, kBlk, h * L + k, c0 + q * 8, h == part ? hv : z4);
+            sw_st16(qbl, kBlk, h * L + k, c0 + q * 8, h == part ? lv : z4);
+          }
         }
+        for (int p2 = kH * L + k; p2 < kTile; p2 += L)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            sw_st16(img, kBlk, p2, c0 + q * 8, z4);
+            sw_st16(qbl, kBlk, p2, c0 + q * 8, z4);
+          }
+      }
+    }
+    __syncthreads();
+    const int nu = n_users - j0 < upp ? n_users - j0 : upp;
+    const uint32_t chunks = piece / 16;
+    for (uint32_t e = threadIdx.x; e < (uint32_t)nu * chunks; e += blockDim.x) {
+      const uint32_t j = e / chunks, q = e - j * chunks;
+      uint8_t* dst = ws + Lw.uimg + (size_t)(u0 + j0 + j) * Lw.uimg_bytes + img_off;
+      reinterpret_cast<uint4*>(dst)[q] = reinterpret_cast<const uint4*>(stage + j * piece)[q];
     }
   }
   cta_teardown(c);
@@ -950,36 +992,6 @@ __global__ void __launch_bounds__(512, 1)
   cta_teardown(c);
 }
 
-// ------------------------------------------------------------ link merge
-// b[u, k, h*32 + c] = merge over the user's tiles of (max, sum, acc) records:
-// the link-branch softmax of link k (head h) over all of the user's history.
-// One warp per (user, head, link); lane c owns output column h*32 + c.
-template <int L>
-__global__ void k_link_merge(const uint8_t* __restrict__ ws, LayerWs Lw, int64_t B,
-                             float* __restrict__ bout) {
-  constexpr int HL = kH * L;
-  const int64_t task = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (task >= B * HL) return;
-  const int64_t u = task / HL;
-  const int p = (int)(task % HL), h = p / L, k = p % L;
-  const int* ts = reinterpret_cast<const int*>(ws + Lw.tile_start);
-  const float* part = reinterpret_cast<const float*>(ws + Lw.part);
-  const int t0 = ts[u], t1 = ts[u + 1];
-  float M = -INFINITY, S = 0.f, acc = 0.f;
-  for (int t = t0; t < t1; ++t) {
-    const float* rec = part + ((size_t)t * HL + p) * kRec;
-    const float m = rec[0], s = rec[1], a = rec[2 + lane];
-    const float Mn = fmaxf(M, m);
-    const float so = M == -INFINITY ? 0.f : __expf(M - Mn);
-    const float sn = __expf(m - Mn);
-    S = S * so + s * sn;
-    acc = acc * so + a * sn;
-    M = Mn;
-  }
-  bout[(u * L + k) * kD + h * kDH + lane] = S > 0.f ? acc / S : 0.f;
-}
-
 // ------------------------------------------------------- history GatedMLP
 // E' = Y + GatedMLP(LN2(Y)), Y = E + Yd, for one 128-row history tile at a
 // time, as a warp-specialized pipeline (persistent, one CTA per SM):
@@ -1030,10 +1042,6 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
   uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 14);
   int* abort_flag = reinterpret_cast<int*>(bar + 15);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
-  const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
-  const int my_tiles =
-      (int)blockIdx.x < n_tiles ? (n_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
   if (threadIdx.x == 0) {
     for (int q = 0; q < 2; ++q) {
       mbar_init(&barE[q], 1);
@@ -1049,17 +1057,24 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (warp == 0) tmem_alloc(slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  pdl_launch();
+  pdl_wait();
+  const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
+  const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
+  const int my_tiles =
+      (int)blockIdx.x < n_tiles ? (n_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
   if (threadIdx.x < kD) {
     sg[threadIdx.x] = __bfloat162float(g2[threadIdx.x]);
     sg[kD + threadIdx.x] = __bfloat162float(b2[threadIdx.x]);
   }
   if ((int)threadIdx.x < my_tiles && threadIdx.x < kFfnTiles)
     s_tiles[threadIdx.x] = tiles[blockIdx.x + threadIdx.x * gridDim.x];
-  if (warp == 0) tmem_alloc(slot, 512);
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *slot;
   constexpr uint32_t T_OUT = 256;
   auto tile_of = [&](int k) -> int4 {
     return k < kFfnTiles ? s_tiles[k] : tiles[blockIdx.x + k * gridDim.x];
@@ -1257,103 +1272,172 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
   }
 }
 
-// ---------------------------------------------------------- link outputs
-// Link rows, split precision: Y_Z = Z + b Wo, h2 = LN2(Y_Z),
-// Z' = Y_Z + (SiLU(h2 W1) * (h2 W3)) W2.  CTA (tile, ch) computes Y_Z's delta
-// b Wo and LN2 for its 128 rows, then GatedMLP chunk ch only, and writes the
-// chunk's fp32 contribution to zpart[ch] (chunk 0 also writes b Wo to
-// zpart[4]); k_link_finish sums them.  Deterministic, no atomics.
+// ------------------------------------------------------------- link tail
+// Everything the link rows need after the attention records, in one kernel:
+//   b    = merge over the user's tiles of the link-branch records (max, sum,
+//          weighted V sum) — the softmax of link k (head h) over all of the
+//          user's history, as a log-sum-exp merge;
+//   Y_Z  = Z + b Wo;  h2 = LN2(Y_Z);  Z' = Y_Z + (SiLU(h2 W1) * (h2 W3)) W2.
+// A cluster of four CTAs owns 128 link rows.  CTA r merges rows 32r..32r+31
+// straight into its A operand (bf16 hi + lo) and pushes those rows to the
+// other three CTAs with shared-to-shared bulk copies (distributed shared
+// memory, completion on the receiver's mbarrier).  Every CTA then runs b Wo
+// and LN2 (split precision, identical in all four) and GatedMLP hidden chunk r
+// only (64 of the 256 hidden units), stages its fp32 partial product, and
+// pushes rows 32q..32q+31 of it to CTA q; CTA r sums the four partials of its
+// rows, adds Y_Z and writes Z'.  No atomics; the summation order is fixed.
+// 512 threads: thread (row, part) owns columns part*32 .. part*32+31.
+constexpr int kTailSmem = 1024 + 12 * kBlk + 2048 + 64;
+
+template <int L>
 __global__ void __launch_bounds__(512, 1)
-    k_link_out(const bf16* __restrict__ Z, const float* __restrict__ bm, int64_t nrows,
-               const bf16* __restrict__ g2, const bf16* __restrict__ b2,
-               const uint8_t* __restrict__ ws_c, LayerWs Lw, float* __restrict__ zpart,
-               unsigned* status) {
-  // 512 threads: thread (row, part) owns columns part*32 .. part*32+31 of its row
+    k_link_tail(const bf16* __restrict__ Z, int64_t nrows, const bf16* __restrict__ g2,
+                const bf16* __restrict__ b2, const uint8_t* __restrict__ ws, LayerWs Lw,
+                bf16* __restrict__ Z_out, unsigned* status) {
+  constexpr int HL = kH * L;
+  constexpr uint32_t kQuarter = 32 * 128;        // 32 rows of a [128 x 64] block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
-  uint8_t* sAh = sm;
-  uint8_t* sAl = sm + 2 * kBlk;
-  uint8_t* sHh = sm + 4 * kBlk;
-  uint8_t* sHl = sm + 5 * kBlk;
-  uint8_t* sWo = sm + 6 * kBlk;
-  uint8_t* sW = sm + 8 * kBlk;      // [W1c | W3c] image, W2c of chunk ch
-  float* red = reinterpret_cast<float*>(sm + 11 * kBlk);
-  const int ch = blockIdx.y;
+  uint8_t* sAh = sm;                 // A operand hi: b, then h2; later the fp32 partial
+  uint8_t* sAl = sm + 2 * kBlk;      // A operand lo
+  uint8_t* sHh = sm + 4 * kBlk;      // hid hi [128 x 64]
+  uint8_t* sHl = sm + 5 * kBlk;      // hid lo
+  uint8_t* sWo = sm + 6 * kBlk;      // Wo image
+  uint8_t* sRecv = sm + 4 * kBlk;    // 4 x 16 KB partial rows received (over hid and Wo)
+  uint8_t* sW = sm + 8 * kBlk;       // [W1c | W3c] image, W2c (chunk = cluster rank)
+  float* sY = reinterpret_cast<float*>(sm + 11 * kBlk);   // Y_Z of this CTA's 32 rows
+  float* red = reinterpret_cast<float*>(sm + 12 * kBlk);
+  uint8_t* sP = sAh;                 // fp32 partial [128 x 128] over sAh, sAl
+  const uint32_t cr = cluster_rank();
   Cta c;
-  cta_setup(sm + 11 * kBlk + 2048, 3, c);  // bar: 0 Wo, 1 mma, 2 chunk
+  cta_setup(sm + 12 * kBlk + 2048, 5, c);  // bar: 0 Wo, 1 mma, 2 chunk, 3 b rows, 4 partials
   uint32_t mph = 0;
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
-    bulk_load(sWo, ws_c + Lw.img_o, 2 * kBlk, &c.bar[0]);
+    bulk_load(sWo, ws + Lw.img_o, 2 * kBlk, &c.bar[0]);
     mbar_arrive_expect_tx(&c.bar[2], 3 * kBlk);
-    bulk_load(sW, ws_c + Lw.img_13 + ch * 2 * kBlk, 2 * kBlk, &c.bar[2]);
-    bulk_load(sW + 2 * kBlk, ws_c + Lw.img_2 + ch * kBlk, kBlk, &c.bar[2]);
+    bulk_load(sW, ws + Lw.img_13 + cr * 2 * kBlk, 2 * kBlk, &c.bar[2]);
+    bulk_load(sW + 2 * kBlk, ws + Lw.img_2 + cr * kBlk, kBlk, &c.bar[2]);
+    mbar_arrive_expect_tx(&c.bar[3], 3 * 4 * kQuarter);   // the other CTAs' b rows
+    mbar_arrive_expect_tx(&c.bar[4], 3 * 32 * 512);       // the other CTAs' partial rows
   }
+  const int64_t t0 = (int64_t)blockIdx.x * kTile;
   const int warp = threadIdx.x >> 5;
   const int part = warp >> 2;
   const int r = (warp & 3) * 32 + (threadIdx.x & 31);
   const int c0 = part * 32;
-  const int64_t R = (int64_t)blockIdx.x * kTile + r;
+  const int64_t R = t0 + r;
   const bool valid = R < nrows;
-  const uint32_t ta = quad_addr(c);
-  auto split_store = [&](uint8_t* hi, uint8_t* lo, int col0, const float* x, int n) {
-    for (int q = 0; q < n / 8; ++q) {
-      float h8[8], l8[8];
+  uint4 zr[4];                                     // this thread's Z values, loaded early
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        h8[k] = __bfloat162float(__float2bfloat16_rn(x[q * 8 + k]));
-        l8[k] = x[q * 8 + k] - h8[k];
-      }
-      sw_st16(hi, kBlk, r, col0 + q * 8, pack8(h8));
-      sw_st16(lo, kBlk, r, col0 + q * 8, pack8(l8));
-    }
-  };
+  for (int q = 0; q < 4; ++q)
+    zr[q] = valid ? reinterpret_cast<const uint4*>(Z + R * kD + c0)[q] : make_uint4(0, 0, 0, 0);
+  // 1. merge rows 32cr..32cr+31 (16 threads per row: 4 heads x 8-column groups)
   {
-    float x[32];
-    if (valid) {
-      const float4* src = reinterpret_cast<const float4*>(bm + R * kD + c0);
+    const int lr = threadIdx.x >> 4, sub = threadIdx.x & 15, h = sub >> 2, q = sub & 3;
+    const int64_t Rm = t0 + 32 * cr + lr;
+    float acc[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 v = src[q];
-        x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    float S = 0.f;
+    if (Rm < nrows) {
+      const int64_t u = Rm / L;
+      const int k = (int)(Rm - u * L);
+      const int* ts = reinterpret_cast<const int*>(ws + Lw.tile_start);
+      const float* recs = reinterpret_cast<const float*>(ws + Lw.part);
+      float M = -INFINITY;
+      const int ta_ = ts[u], tb_ = ts[u + 1];
+      for (int t = ta_; t < tb_; t += 4) {
+        // the records of up to four tiles are loaded before any is merged
+        float2 ms[4];
+        float a[4][8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (t + i < tb_) {
+            const float* rec = recs + ((size_t)(t + i) * HL + h * L + k) * kRec;
+            ms[i] = *reinterpret_cast<const float2*>(rec);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 v = *reinterpret_cast<const float2*>(rec + 2 + q * 8 + 2 * j);
+              a[i][2 * j] = v.x;
+              a[i][2 * j + 1] = v.y;
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (t + i < tb_) {
+            const float Mn = fmaxf(M, ms[i].x);
+            const float so = M == -INFINITY ? 0.f : __expf(M - Mn);
+            const float sn = __expf(ms[i].x - Mn);
+            S = S * so + ms[i].y * sn;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = acc[j] * so + a[i][j] * sn;
+            M = Mn;
+          }
+        }
       }
-    } else {
-#pragma unroll
-      for (int k = 0; k < 32; ++k) x[k] = 0.f;
     }
-    split_store(sAh, sAl, c0, x, 32);
+    const float inv = S > 0.f ? 1.0f / S : 0.f;
+    float h8[8], l8[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float x = acc[j] * inv;
+      h8[j] = __bfloat162float(__float2bfloat16_rn(x));
+      l8[j] = x - h8[j];
+    }
+    sw_st16(sAh, kBlk, 32 * cr + lr, h * kDH + q * 8, pack8(h8));
+    sw_st16(sAl, kBlk, 32 * cr + lr, h * kDH + q * 8, pack8(l8));
   }
   fence_proxy_async_smem();
-  __syncthreads();
+  cluster_sync();      // every CTA's barriers are armed and its b rows are written
+  if (threadIdx.x == 0) {
+    // rows 32cr..32cr+31 of the four 64-column blocks (hi 0, hi 1, lo 0, lo 1)
+    // are 4 KB each and contiguous in the swizzled layout
+    for (uint32_t p = 0; p < 4; ++p) {
+      if (p == cr) continue;
+      const uint32_t mb = cluster_map(&c.bar[3], p);
+      for (int blk = 0; blk < 4; ++blk) {
+        uint8_t* src = sAh + blk * kBlk + cr * kQuarter;
+        bulk_push_cluster(cluster_map(src, p), src, kQuarter, mb);
+      }
+    }
+  }
+  mbar_wait(&c.bar[3], 0, status, c.abort_flag);
   mbar_wait(&c.bar[0], 0, status, c.abort_flag);
   if (threadIdx.x == 0) {
     tc_fence_after();
     mma_tile(c.tmem, smem_u32(sAh), kBlk, smem_u32(sWo), kBlk, 128, 128, false);
     mma_tile(c.tmem, smem_u32(sAl), kBlk, smem_u32(sWo), kBlk, 128, 128, true);
+    mma_commit(&c.bar[1]);
   }
-  cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+  // every CTA has received its rows, so no copy still reads our b rows
+  cluster_sync();
+  mbar_wait(&c.bar[1], mph, status, c.abort_flag);
+  mph ^= 1u;
+  tc_fence_after();
+  const uint32_t ta = quad_addr(c);
+  const bool mine = (uint32_t)(r >> 5) == cr;   // this CTA finishes row r
+  // 2. Y_Z = Z + b Wo; LN2 -> A operand (hi + lo)
   {
     float y[32];
     tmem_ld16(ta + c0, y);
     tmem_ld16(ta + c0 + 16, y + 16);
     tmem_ld_wait();
-    if (valid && ch == 0) {
-      float4* dst = reinterpret_cast<float4*>(zpart + ((size_t)4 * nrows + R) * kD + c0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float z8[8];
+      unpack8(zr[q], z8);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) y[q * 8 + k] += z8[k];
+    }
+    if (mine) {
+      float4* dst = reinterpret_cast<float4*>(sY + (r & 31) * kD + c0);
 #pragma unroll
       for (int q = 0; q < 8; ++q) dst[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
     }
-    if (valid) {
-      const uint4* src = reinterpret_cast<const uint4*>(Z + R * kD + c0);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float z8[8];
-        unpack8(src[q], z8);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) y[q * 8 + k] += z8[k];
-      }
-    }
     layer_norm_part(y, c0, g2, b2, red, part, r);
-    split_store(sAh, sAl, c0, y, 32);
+    split_part_st(sAh, sAl, r, c0, y);
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -1361,7 +1445,7 @@ __global__ void __launch_bounds__(512, 1)
   mbar_wait(&c.bar[2], 0, status, c.abort_flag);
   if (threadIdx.x == 0) {
     tc_fence_after();
-    // [G1 | G3] of the chunk in one N = 128 product
+    // [G1 | G3] of hidden chunk cr in one N = 128 product
     mma_tile(c.tmem + 128, smem_u32(sAh), kBlk, smem_u32(sW), kBlk, 128, 128, false);
     mma_tile(c.tmem + 128, smem_u32(sAl), kBlk, smem_u32(sW), kBlk, 128, 128, true);
   }
@@ -1373,7 +1457,17 @@ __global__ void __launch_bounds__(512, 1)
     tmem_ld_wait();
 #pragma unroll
     for (int k = 0; k < 16; ++k) g[k] = silu_fast(g[k]) * gg[k];
-    split_store(sHh, sHl, part * 16, g, 16);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      float h8[8], l8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        h8[k] = __bfloat162float(__float2bfloat16_rn(g[q * 8 + k]));
+        l8[k] = g[q * 8 + k] - h8[k];
+      }
+      sw_st16(sHh, kBlk, r, part * 16 + q * 8, pack8(h8));
+      sw_st16(sHl, kBlk, r, part * 16 + q * 8, pack8(l8));
+    }
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -1384,31 +1478,50 @@ __global__ void __launch_bounds__(512, 1)
     mma_tile(c.tmem + 256, smem_u32(sHl), kBlk, smem_u32(sW + 2 * kBlk), kBlk, 128, 64, true);
   }
   cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+  // 3. this chunk's fp32 partial -> shared memory (the A operand is dead);
+  //    rows 32q..32q+31 form one contiguous 16 KB piece
   {
     float o[32];
-    tmem_ld16(ta + 256 + c0, o);    // warp-collective: every thread loads
+    tmem_ld16(ta + 256 + c0, o);
     tmem_ld16(ta + 256 + c0 + 16, o + 16);
     tmem_ld_wait();
-    if (valid) {
-      float4* dst = reinterpret_cast<float4*>(zpart + ((size_t)ch * nrows + R) * kD + c0);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    for (int q = 0; q < 8; ++q)
+      *f32_chunk(sP, r, part * 8 + q) = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+  }
+  fence_proxy_async_smem();
+  cluster_sync();      // every CTA's hid and Wo buffers are free to receive
+  if (threadIdx.x == 0) {
+    for (uint32_t p = 0; p < 4; ++p) {
+      if (p == cr) continue;
+      uint8_t* src = sP + p * 32 * 512;
+      bulk_push_cluster(cluster_map(sRecv + cr * 32 * 512, p), src, 32 * 512,
+                        cluster_map(&c.bar[4], p));
     }
   }
-  cta_teardown(c);
-}
-
-// Z' = Z + (b Wo) + sum of the four GatedMLP chunk contributions, in bf16.
-__global__ void k_link_finish(const bf16* __restrict__ Z, const float* __restrict__ zpart,
-                              int64_t nrows, bf16* __restrict__ Z_out) {
-  const int64_t n = nrows * kD;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    float v = __bfloat162float(Z[e]) + zpart[4 * n + e];
+  mbar_wait(&c.bar[4], 0, status, c.abort_flag);
+  // 4. rows 32cr..32cr+31: Z' = Y_Z + the four partials (rank order)
+  {
+    const int lr = threadIdx.x >> 4, cc = threadIdx.x & 15;   // 8 columns each
+    const int64_t Rr = t0 + 32 * cr + lr;
+    float v[8];
+    {
+      const float4* y = reinterpret_cast<const float4*>(sY + lr * kD + cc * 8);
+      const float4 a = y[0], b = y[1];
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) v += zpart[q * n + e];
-    Z_out[e] = __float2bfloat16_rn(v);
+    for (uint32_t p = 0; p < 4; ++p) {
+      uint8_t* base = p == cr ? sP + cr * 32 * 512 : sRecv + p * 32 * 512;
+      const float4 a = *f32_chunk(base, lr, cc * 2);
+      const float4 b = *f32_chunk(base, lr, cc * 2 + 1);
+      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+      v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+    }
+    if (Rr < nrows) reinterpret_cast<uint4*>(Z_out + Rr * kD)[cc] = pack8(v);
   }
+  cluster_sync();   // every CTA has received its partials: no copy still reads ours
+  cta_teardown(c);
 }
 
 constexpr int kBarBytes = 64;
@@ -1430,17 +1543,19 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
   const int sms = num_sms();
   {
     const int64_t n = 4 * kD * kD + 3 * kD * kF;
-    k_prep_weights<<<(unsigned)(1 + (n + 1023) / 1024), 1024, 0, st>>>(
-        (const bf16*)w.Wq, (const bf16*)w.Wk, (const bf16*)w.Wv, (const bf16*)w.Wo,
-        (const bf16*)w.W1, (const bf16*)w.W3, (const bf16*)w.W2, ws, Lw, off, B, nh, status);
-    note_launches(1);
+    int rc = launch_pdl(k_prep_weights, dim3((unsigned)(1 + (n + 1023) / 1024)), dim3(1024), 0, st,
+                        1, (const bf16*)w.Wq, (const bf16*)w.Wk, (const bf16*)w.Wv,
+                        (const bf16*)w.Wo, (const bf16*)w.W1, (const bf16*)w.W3, (const bf16*)w.W2,
+                        ws, Lw, off, B, nh, status);
+    if (rc) return rc;
   }
   {
-    const int smem = 1024 + 6 * kBlk + 2048 + kBarBytes;
+    const int smem = 1024 + 6 * kBlk + 2048 + kBarBytes;   // 96 KB of it stage the images
     if (!set_smem(k_link_proj<L>, smem)) return LIME_ERR_CUDA;
-    k_link_proj<L><<<dim3((unsigned)((nz + kTile - 1) / kTile), 3), 512, smem, st>>>(
-        (const bf16*)Z_in, nz, (const bf16*)w.g1, (const bf16*)w.b1, ws, ws, Lw, scale, status);
-    note_launches(1);
+    int rc = launch_pdl(k_link_proj<L>, dim3((unsigned)((nz + kTile - 1) / kTile), 3), dim3(512),
+                        smem, st, 1, (const bf16*)Z_in, nz, (const bf16*)w.g1, (const bf16*)w.b1,
+                        (const uint8_t*)ws, ws, Lw, scale, status);
+    if (rc) return rc;
   }
   if (nh > 0) {
     CUtensorMap tmE, tmQ, tmK, tmV;
@@ -1454,46 +1569,39 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     if (last) {
       const int smem = 1024 + 12 * kBlk + 2048 + kBarBytes;
       if (!set_smem(k_hist_link<L>, smem)) return LIME_ERR_CUDA;
-      k_hist_link<L><<<grid, 512, smem, st>>>(tmE, (const bf16*)w.g1, (const bf16*)w.b1, ws, Lw,
-                                              status);
+      int rc = launch_pdl(k_hist_link<L>, dim3(grid), dim3(512), smem, st, 1, tmE,
+                          (const bf16*)w.g1, (const bf16*)w.b1, ws, Lw, status);
+      if (rc) return rc;
     } else {
       const int smem = 1024 + 10 * kBlk + 2048 + kBarBytes;
       if (!set_smem(k_hist_proj<false>, smem)) return LIME_ERR_CUDA;
-      k_hist_proj<false><<<grid, 512, smem, st>>>(tmE, (const bf16*)w.g1, (const bf16*)w.b1, ws,
-                                                   Lw, status);
+      int rc = launch_pdl(k_hist_proj<false>, dim3(grid), dim3(512), smem, st, 1, tmE,
+                          (const bf16*)w.g1, (const bf16*)w.b1, ws, Lw, status);
+      if (rc) return rc;
     }
-    note_launches(1);
     if (!last) {
       const int smem = 1024 + 8 * kBlk + uimg_bytes(L) + 2048 + kBarBytes;
       if (!set_smem(k_hist_attn<L, false>, smem)) return LIME_ERR_CUDA;
-      k_hist_attn<L, false><<<grid, 512, smem, st>>>(tmQ, tmK, tmV, ws, Lw, status);
-      note_launches(1);
+      int rc = launch_pdl(k_hist_attn<L, false>, dim3(grid), dim3(512), smem, st, 1, tmQ, tmK, tmV,
+                          ws, Lw, status);
+      if (rc) return rc;
     }
     if (!last) {
       if (!set_smem(k_hist_ffn, kFfnSmem)) return LIME_ERR_CUDA;
-      k_hist_ffn<<<grid, kFfnEpi + 32, kFfnSmem, st>>>(tmE, (const bf16*)w.g2, (const bf16*)w.b2,
-                                                       ws, Lw, (bf16*)E_out, status);
-      note_launches(1);
+      int rc = launch_pdl(k_hist_ffn, dim3(grid), dim3(kFfnEpi + 32), kFfnSmem, st, 1, tmE,
+                          (const bf16*)w.g2, (const bf16*)w.b2, (const uint8_t*)ws, Lw,
+                          (bf16*)E_out, status);
+      if (rc) return rc;
     }
   }
   {
-    const int64_t tasks = B * kH * L;
-    k_link_merge<L><<<(unsigned)((tasks * 32 + 255) / 256), 256, 0, st>>>(
-        ws, Lw, B, reinterpret_cast<float*>(ws + Lw.bmerge));
-    note_launches(1);
-  }
-  {
-    const int smem = 1024 + 11 * kBlk + 2048 + kBarBytes;
-    if (!set_smem(k_link_out, smem)) return LIME_ERR_CUDA;
-    float* zpart = reinterpret_cast<float*>(ws + Lw.zpart);
-    k_link_out<<<dim3((unsigned)((nz + kTile - 1) / kTile), kF / 64), 512, smem, st>>>(
-        (const bf16*)Z_in, reinterpret_cast<const float*>(ws + Lw.bmerge), nz,
-        (const bf16*)w.g2, (const bf16*)w.b2, ws, Lw, zpart, status);
-    note_launches(1);
-    const int64_t n = nz * kD;
-    k_link_finish<<<(unsigned)((n + 255) / 256 < 148 * 8 ? (n + 255) / 256 : 148 * 8), 256, 0, st>>>(
-        (const bf16*)Z_in, zpart, nz, (bf16*)Z_out);
-    note_launches(1);
+    // one 4-CTA cluster per 128 link rows
+    if (!set_smem(k_link_tail<L>, kTailSmem)) return LIME_ERR_CUDA;
+    int rc = launch_pdl(k_link_tail<L>, dim3((unsigned)((nz + kTile - 1) / kTile), kF / 64),
+                        dim3(512), kTailSmem, st, kF / 64, (const bf16*)Z_in, nz,
+                        (const bf16*)w.g2, (const bf16*)w.b2, (const uint8_t*)ws, Lw, (bf16*)Z_out,
+                        status);
+    if (rc) return rc;
   }
   return LIME_OK;
 }

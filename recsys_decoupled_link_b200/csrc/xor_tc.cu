@@ -203,7 +203,11 @@ __device__ __forceinline__ void split_part_st(uint8_t* hi, uint8_t* lo, int row,
   }
 }
 
-__device__ __forceinline__ float silu_fast(float x) { return x / (1.0f + __expf(-x)); }
+// SiLU with the hardware exp2 and reciprocal approximations (a few ulp in
+// fp32; the result is rounded to bf16 for the next product).  An IEEE
+// division here would cost about as much as the rest of the gate's epilogue.
+// For very negative x, 1 + exp(-x) overflows to inf and the result is -0.
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 // fp32 [rows x 128] staging: row r is 512 bytes, its 16-byte chunk c sits at
 // r*512 + ((c ^ (r & 31)) * 16), so row-per-thread and row-per-warp accesses
@@ -997,19 +1001,20 @@ __global__ void __launch_bounds__(512, 1)
 // time, as a warp-specialized pipeline (persistent, one CTA per SM):
 //   warps 0-15 (epilogue): warp w serves TMEM lane quadrant w % 4 (tile rows
 //     32*(w%4) ...) and column part p = w / 4 (a quarter of every row).  Per
-//     tile they form Y = E (TMA tile) + Yd (fp32 rows, loaded a tile ahead
-//     into registers) and store it into the tile's output accumulator OUT,
+//     tile they form Y = E (TMA tile) + Yd (fp32 rows, prefetched into L2
+//     with the E tile) and store it into the tile's output accumulator OUT,
 //     so that the W2 products add the GatedMLP onto the residual in place;
 //     write h2 = LN2(Y) (statistics reduced over the four parts through
 //     shared memory) over the E tile; compute hid = SiLU(G1) * G3 per 64-wide
 //     hidden chunk from TMEM GB[g%2] into smem HB[g%2]; and store E' = OUT.
 //     The next tile's Y and LN2 run before this tile's E' is read out, so the
 //     tensor cores start the next tile while the epilogue finishes this one.
-//   warp 16 (control, one lane): TMA of the E tiles (one tile ahead), the
-//     [W1c | W3c] chunk images through a two-slot ring (chunk g+1 is fetched
-//     as soon as G(g-1) has consumed its slot), and the MMAs: G(g) =
-//     h2 [W1c | W3c] (one N = 128 product) into GB[g%2] and OUT += hid(g) W2c
-//     with W2 resident in shared memory.
+//   warp 16 (one lane) issues the MMAs: G(g) = h2 [W1c | W3c] (one N = 128
+//     product) into GB[g%2] and OUT += hid(g) W2c with W2 resident in shared
+//     memory.
+//   warp 17 (one lane) loads: the E tiles (one tile ahead) and the [W1c | W3c]
+//     chunk images through a two-slot ring (chunk g+1 is fetched as soon as
+//     G(g-1) has consumed its slot).
 // Chunks are counted over the CTA's whole tile sequence (g = 4*k + c for its
 // k-th tile), so every ring barrier's parity is (g / 2) % 2.
 // TMEM: GB[0] [0,128), GB[1] [128,256), OUT[k%2] [256 + 128*(k%2), +128).
@@ -1017,7 +1022,7 @@ constexpr int kFfnEpi = 512;   // epilogue threads
 constexpr int kFfnTiles = 32;  // tile descriptors of a CTA kept in shared memory
 constexpr int kFfnSmem = 1024 + 14 * kBlk + 1024 + kFfnTiles * 16 + 256;
 
-__global__ void __launch_bounds__(kFfnEpi + 32, 1)
+__global__ void __launch_bounds__(kFfnEpi + 64, 1)
     k_hist_ffn(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ g2,
                const bf16* __restrict__ b2, const uint8_t* __restrict__ ws, LayerWs Lw,
                bf16* __restrict__ E_out, unsigned* status) {
@@ -1081,7 +1086,10 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
   };
   const int n_chunks = my_tiles * (kF / 64);
 
-  if (warp == kFfnEpi / 32) {
+  if (warp == kFfnEpi / 32 + 1) {
+    // loader: the W1|W3 ring, the E tiles and W2.  It runs apart from the MMA
+    // issuer because tcgen05.mma issue stalls while the tensor pipe is busy,
+    // which would hold back the next loads.
     if (lane == 0 && my_tiles > 0) {
       auto load_w13 = [&](int g) {
         const int s = g & 1, ch = g & 3;
@@ -1094,6 +1102,9 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
         mbar_arrive_expect_tx(&barE[k & 1], 2 * kBlk);
         tma_load_2d(dst, &tmE, 0, tl.y, &barE[k & 1]);
         tma_load_2d(dst + kBlk, &tmE, 64, tl.y, &barE[k & 1]);
+        // the tile's Yd rows into L2, for the epilogue's plain loads
+        bulk_prefetch_l2(reinterpret_cast<const float*>(ws + Lw.yd) + (int64_t)tl.y * kD,
+                         (uint32_t)tl.z * kD * 4);
       };
       prefetch_tmap(&tmE);
       load_e(0);
@@ -1101,6 +1112,25 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
       if (n_chunks > 1) load_w13(1);
       mbar_arrive_expect_tx(barW2in, 4 * kBlk);
       bulk_load(sW2, ws + Lw.img_2, 4 * kBlk, barW2in);
+      for (int g = 0; g < n_chunks; ++g) {
+        if (g >= 1) {
+          // G(g-1) done: its ring slot takes chunk g+1
+          if (!mbar_wait(&barG[(g - 1) & 1], (uint32_t)(((g - 1) >> 1) & 1), status, abort_flag))
+            break;
+          if (g + 1 < n_chunks) load_w13(g + 1);
+        }
+        const int k = g / (kF / 64);
+        if (g % (kF / 64) == 0 && k + 1 < my_tiles) {
+          // E(k+1) goes to buffer (k+1)%2, which held h2(k-1) (dead once
+          // G(k-1, 3) is done) and is the LN2 scratch of tile k: wait for h2(k)
+          if (!mbar_wait(barH2, k & 1, status, abort_flag)) break;
+          load_e(k + 1);
+        }
+      }
+    }
+  } else if (warp == kFfnEpi / 32) {
+    // MMA issuer
+    if (lane == 0 && my_tiles > 0) {
       bool ok = mbar_wait(barW2in, 0, status, abort_flag);
       for (int k = 0; k < my_tiles && ok; ++k) {
         if (!(ok = mbar_wait(barH2, k & 1, status, abort_flag))) break;
@@ -1113,14 +1143,6 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
           tc_fence_after();
           mma_tile(tmem + s * 128, a_h2, kBlk, smem_u32(sW13 + s * 2 * kBlk), kBlk, 128, 128, false);
           mma_commit(&barG[s]);
-          if (g >= 1) {
-            // G(g-1) done: its ring slot takes chunk g+1; at a tile's first
-            // chunk it also means the previous tile's h2 buffer is free
-            if (!(ok = mbar_wait(&barG[s ^ 1], (uint32_t)(((g - 1) >> 1) & 1), status, abort_flag)))
-              break;
-            if (g + 1 < n_chunks) load_w13(g + 1);
-          }
-          if (c == 0 && k + 1 < my_tiles) load_e(k + 1);
           if (c >= 1) {
             const int pg = g - 1, pb = pg & 1;
             if (!(ok = mbar_wait(&barHid[pb], (uint32_t)((pg >> 1) & 1), status, abort_flag))) break;
@@ -1149,21 +1171,6 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
     const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16);
     const int c0 = part * 32;                      // this thread's 32 columns of a row
     const float* yd = reinterpret_cast<const float*>(ws + Lw.yd);
-    float yn[32];                                  // Yd of the next tile
-    auto load_yd = [&](int k) {
-      const int4 tl = tile_of(k);
-      if (row < tl.z) {
-        const float4* src = reinterpret_cast<const float4*>(yd + (int64_t)(tl.y + row) * kD + c0);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 v = src[q];
-          yn[4 * q] = v.x; yn[4 * q + 1] = v.y; yn[4 * q + 2] = v.z; yn[4 * q + 3] = v.w;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) yn[j] = 0.f;
-      }
-    };
     // Y(j) = E + Yd into OUT[j%2], h2(j) = LN2(Y(j)) over E tile j%2.  The
     // reduction scratch is the other E buffer: it holds h2(j-1), whose last
     // reader G(j-1, 3) has completed by the time the epilogue gets here, and
@@ -1173,8 +1180,21 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
       float* red1 = reinterpret_cast<float*>(sE0 + ((j & 1) ^ 1) * 2 * kBlk);
       float* red2 = red1 + 4 * 128;
       float y[32];
+      {
+        // Yd rows (prefetched into L2 with the E tile)
+        const int4 tl = tile_of(j);
+        if (row < tl.z) {
+          const float4* src = reinterpret_cast<const float4*>(yd + (int64_t)(tl.y + row) * kD + c0);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) y[i] = yn[i];
+          for (int q = 0; q < 8; ++q) {
+            const float4 v = src[q];
+            y[4 * q] = v.x; y[4 * q + 1] = v.y; y[4 * q + 2] = v.z; y[4 * q + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = 0.f;
+        }
+      }
       mbar_wait(&barE[j & 1], (uint32_t)((j >> 1) & 1), status, abort_flag);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -1220,12 +1240,8 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(barH2);
-      if (j + 1 < my_tiles) load_yd(j + 1);   // in flight during the next chunk loop
     };
-    if (my_tiles > 0) {
-      load_yd(0);
-      y_ln2(0);
-    }
+    if (my_tiles > 0) y_ln2(0);
     for (int k = 0; k < my_tiles; ++k) {
       for (int c = 0; c < kF / 64; ++c) {
         const int g = k * (kF / 64) + c, sb = g & 1;
@@ -1249,19 +1265,29 @@ __global__ void __launch_bounds__(kFfnEpi + 32, 1)
       if (k + 1 < my_tiles) y_ln2(k + 1);
       mbar_wait(barOut, (uint32_t)(k & 1), status, abort_flag);
       tc_fence_after();
-      const int4 tl = tile_of(k);
+      // E' = OUT -> bf16, staged in the hid buffers (every W2 product of the
+      // tile is done, and the next hid is written by these threads after the
+      // copy) and written with coalesced 16-byte stores
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         float o[16];
         tmem_ld16(ta + T_OUT + (k & 1) * 128 + c0 + hf * 16, o);
         tmem_ld_wait();
-        if (row < tl.z) {
-          uint4* dst = reinterpret_cast<uint4*>(E_out + (int64_t)(tl.y + row) * kD + c0 + hf * 16);
-          dst[0] = pack8(o);
-          dst[1] = pack8(o + 8);
-        }
+        sw_st16(sH0, kBlk, row, c0 + hf * 16, pack8(o));
+        sw_st16(sH0, kBlk, row, c0 + hf * 16 + 8, pack8(o + 8));
       }
       tc_fence_before();
+      named_bar_sync(1, kFfnEpi);
+      {
+        const int4 tl = tile_of(k);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int idx = q * kFfnEpi + (int)threadIdx.x, r = idx >> 4, cc = idx & 15;
+          if (r < tl.z)
+            reinterpret_cast<uint4*>(E_out + (int64_t)(tl.y + r) * kD)[cc] = sw_ld16(sH0, kBlk, r, cc * 8);
+        }
+      }
+      named_bar_sync(1, kFfnEpi);
     }
   }
   tc_fence_before();
@@ -1588,7 +1614,7 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     }
     if (!last) {
       if (!set_smem(k_hist_ffn, kFfnSmem)) return LIME_ERR_CUDA;
-      int rc = launch_pdl(k_hist_ffn, dim3(grid), dim3(kFfnEpi + 32), kFfnSmem, st, 1, tmE,
+      int rc = launch_pdl(k_hist_ffn, dim3(grid), dim3(kFfnEpi + 64), kFfnSmem, st, 1, tmE,
                           (const bf16*)w.g2, (const bf16*)w.b2, (const uint8_t*)ws, Lw,
                           (bf16*)E_out, status);
       if (rc) return rc;

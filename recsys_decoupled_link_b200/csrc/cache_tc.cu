@@ -47,73 +47,65 @@ struct CacheCfg {
 
 // G^T image: block b (K columns [64b, 64b+64)) of HL rows x 128 bytes,
 // element (row j = h*l + k, K index i) at b*HL*128 + sw128_offset(j, i % 64).
-// CTA (h, quarter) stages L, Wk_c[:, h-cols] and 32 rows of Wq_c[:, h-cols]
-// in shared memory (fp32), forms kc = L Wk_c[:, h-cols] ([l x dh], every
-// quarter redundantly) and writes G^T rows h*l .. h*l+l-1 for its 32 K
-// indices i.  256 threads.
-constexpr int kFoldRows = 32;   // K indices per CTA
-
-__global__ void __launch_bounds__(256) k_fold_g_img(const bf16* __restrict__ L,
+// CTA j = h*l + k stages L_k and the head-h columns of Wk_c and Wq_c in
+// shared memory (all 16-byte loads issued before any is used), forms
+// kc = L_k Wk_c[:, h-cols] (dh values; 128 threads, each a quarter of the
+// K = 128 sum for one value when dh = 32) and writes row j of G^T.
+__global__ void __launch_bounds__(128) k_fold_g_img(const bf16* __restrict__ L,
                                                     const bf16* __restrict__ Wq,
                                                     const bf16* __restrict__ Wk, int H, int l,
                                                     float scale, bf16* __restrict__ img) {
-  extern __shared__ float fsm[];
+  __shared__ __align__(16) bf16 sWk[kD * 64];   // [kD][dh]
+  __shared__ __align__(16) bf16 sWq[kD * 64];   // [kD][dh]
+  __shared__ float sL[kD];
+  __shared__ float part[8][64];   // dh >= 16: at most 8 partial sums
+  __shared__ float kc[64];
   const int dh = kD / H, HL = H * l;
-  const int h = blockIdx.x, i0 = blockIdx.y * kFoldRows;
-  float* sL = fsm;                      // [l][kD]
-  float* sWk = sL + l * kD;             // [kD][dh]
-  float* sWq = sWk + kD * dh;           // [kFoldRows][dh]
-  float* sKc = sWq + kFoldRows * dh;    // [l][dh + 1]
+  const int j = blockIdx.x, h = j / l, k = j % l;
   pdl_launch();
   pdl_wait();
-  // 16-byte loads, all issued before any is used (the latency is paid once):
-  // L is l x 16 chunks, the head-h columns of Wk are kD x dh/8 chunks, those
-  // of the CTA's 32 Wq rows 32 x dh/8 chunks; at most 1024 + 1024 + 256.
   {
-    const int cw = dh / 8;                      // 16-byte chunks per head row
-    const int nL = l * 16, nK = kD * cw, nQ = kFoldRows * cw;
-    uint4 v[10];
+    const int cw = dh / 8;                 // 16-byte chunks per head row (2, 4 or 8)
+    const int nK = kD * cw;                // <= 1024 chunks for each of Wk, Wq
+    uint4 vk[8], vq[8], vl;
 #pragma unroll
-    for (int q = 0; q < 10; ++q) {
-      const int e = q * 256 + (int)threadIdx.x;
-      if (e < nL) {
-        v[q] = reinterpret_cast<const uint4*>(L)[e];
-      } else if (e < nL + nK) {
-        const int f = e - nL;
-        v[q] = reinterpret_cast<const uint4*>(Wk + (f / cw) * kD + h * dh)[f % cw];
-      } else if (e < nL + nK + nQ) {
-        const int f = e - nL - nK;
-        v[q] = reinterpret_cast<const uint4*>(Wq + (i0 + f / cw) * kD + h * dh)[f % cw];
+    for (int q = 0; q < 8; ++q) {
+      const int e = q * 128 + (int)threadIdx.x;
+      if (e < nK) {
+        vk[q] = reinterpret_cast<const uint4*>(Wk + (e / cw) * kD + h * dh)[e % cw];
+        vq[q] = reinterpret_cast<const uint4*>(Wq + (e / cw) * kD + h * dh)[e % cw];
       }
     }
+    if (threadIdx.x < 16) vl = reinterpret_cast<const uint4*>(L + (int64_t)k * kD)[threadIdx.x];
 #pragma unroll
-    for (int q = 0; q < 10; ++q) {
-      const int e = q * 256 + (int)threadIdx.x;
-      float f8[8];
-      unpack8(v[q], f8);
-      float* dst = nullptr;
-      if (e < nL) dst = sL + e * 8;
-      else if (e < nL + nK) dst = sWk + (e - nL) * 8;
-      else if (e < nL + nK + nQ) dst = sWq + (e - nL - nK) * 8;
-      if (dst) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) dst[j] = f8[j];
+    for (int q = 0; q < 8; ++q) {
+      const int e = q * 128 + (int)threadIdx.x;
+      if (e < nK) {
+        reinterpret_cast<uint4*>(sWk)[e] = vk[q];
+        reinterpret_cast<uint4*>(sWq)[e] = vq[q];
       }
     }
+    if (threadIdx.x < 16) unpack8(vl, sL + threadIdx.x * 8);
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < l * dh; e += blockDim.x) {
-    const int k = e / dh, c = e % dh;
+  {
+    // kc[c] = sum_t L_k[t] Wk[t, h*dh + c]: thread (c, quarter of t)
+    const int nq = 128 / dh, c = threadIdx.x % dh, q = threadIdx.x / dh;
     float acc = 0.f;
-#pragma unroll 8
-    for (int t = 0; t < kD; ++t) acc += sL[k * kD + t] * sWk[t * dh + c];
-    sKc[k * (dh + 1) + c] = acc;
+    for (int t = q; t < kD; t += nq) acc += sL[t] * __bfloat162float(sWk[t * dh + c]);
+    part[q][c] = acc;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kFoldRows * l; e += blockDim.x) {
-    const int ii = e / l, k = e % l, i = i0 + ii, j = h * l + k;
+  if (threadIdx.x < dh) {
+    float s = 0.f;
+    for (int q = 0; q < 128 / dh; ++q) s += part[q][threadIdx.x];
+    kc[threadIdx.x] = s;
+  }
+  __syncthreads();
+  {
+    const int i = threadIdx.x;   // K index of G^T row j
     float acc = 0.f;
-    for (int c = 0; c < dh; ++c) acc += sWq[ii * dh + c] * sKc[k * (dh + 1) + c];
+    for (int c = 0; c < dh; ++c) acc += __bfloat162float(sWq[i * dh + c]) * kc[c];
     uint8_t* base = reinterpret_cast<uint8_t*>(img) + (size_t)(i >> 6) * HL * 128;
     *reinterpret_cast<bf16*>(base + sw128_offset(j, i & 63)) = __float2bfloat16_rn(acc * scale);
   }
@@ -322,14 +314,8 @@ int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void
   const int HL = D.H * D.l;
   bf16* img = reinterpret_cast<bf16*>(ws);
   const float scale = 1.0f / sqrtf((float)(D.d / D.H));
-  const int dh = D.d / D.H;
-  const size_t fold_smem =
-      ((size_t)D.l * kD + (size_t)kD * dh + (size_t)kFoldRows * dh + (size_t)D.l * (dh + 1)) * 4;
-  if (cudaFuncSetAttribute(k_fold_g_img, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)fold_smem) != cudaSuccess)
-    return LIME_ERR_CUDA;
-  int rc = launch_pdl(k_fold_g_img, dim3(D.H, kD / kFoldRows), dim3(256), fold_smem, st, 1,
-                      (const bf16*)L, (const bf16*)Wq, (const bf16*)Wk, D.H, D.l, scale, img);
+  int rc = launch_pdl(k_fold_g_img, dim3(HL), dim3(128), 0, st, 1, (const bf16*)L,
+                      (const bf16*)Wq, (const bf16*)Wk, D.H, D.l, scale, img);
   if (rc) return rc;
   if (n == 0) return LIME_OK;
   switch (HL * 1000 + D.l) {

@@ -65,8 +65,9 @@ __host__ __device__ constexpr size_t up1k(size_t x) { return (x + 1023) & ~(size
 
 __host__ __device__ constexpr uint32_t kz_bytes(int l) { return (uint32_t)l * 256; }  // [l x 128] bf16
 __host__ __device__ constexpr uint32_t uimg_bytes(int l) {
-  return (uint32_t)up1k(kz_bytes(l) + kBlk + 4 * kBlk);   // KZ, VZT, QBD hi, QBD lo
+  return (uint32_t)up1k(kz_bytes(l) + kBlk + 2 * kz_bytes(l));   // KZ, VZT, QZ hi, QZ lo
 }
+__host__ __device__ constexpr uint32_t qz_off(int l) { return kz_bytes(l) + kBlk; }
 
 LayerWs layer_ws(int l, int64_t B, int64_t nh) {
   LayerWs w;
@@ -183,6 +184,31 @@ __device__ __forceinline__ void split_row_st(uint8_t* hi, uint8_t* lo, uint32_t 
     }
     sw_st16(hi, blk, row, c * 8, pack8(h));
     sw_st16(lo, blk, row, c * 8, pack8(r));
+  }
+}
+
+// Expands the compact s·Q_Z image (hi [L x 128] then lo, blocks of L*128
+// bytes, bulk-loaded to the start of `qbd`) in place into the block-diagonal
+// operands: qbd (hi) and qbd + 2*kBlk (lo), [128 rows x 128] each, row h*L + k
+// = s·Q_Z[k] in head h's 32 columns and zeros elsewhere, rows >= 4L zero.
+// All 512 threads: thread (row p, part) writes row p's columns part*32..+31;
+// the thread with part == h(p) first reads its 32 compact values.
+template <int L>
+__device__ __forceinline__ void expand_qbd(uint8_t* qbd, int p, int part) {
+  const bool mine = p < kH * L && p / L == part;
+  const int k = p % L;
+  uint4 hv[4], lv[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    hv[q] = mine ? sw_ld16(qbd, (uint32_t)L * 128, k, part * 32 + q * 8) : make_uint4(0, 0, 0, 0);
+    lv[q] = mine ? sw_ld16(qbd + kz_bytes(L), (uint32_t)L * 128, k, part * 32 + q * 8)
+                 : make_uint4(0, 0, 0, 0);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    sw_st16(qbd, kBlk, p, part * 32 + q * 8, hv[q]);
+    sw_st16(qbd + 2 * kBlk, kBlk, p, part * 32 + q * 8, lv[q]);
   }
 }
 
@@ -386,10 +412,11 @@ __device__ void schedule_tiles(const int64_t* __restrict__ off, int64_t B, int64
 // Per-user operand images (at uimg + u * uimg_bytes, ℓ = L):
 //   KZ   [L rows x 128] bf16, 2 blocks of L*128 bytes:  s·K_Z
 //   VZT  [128 rows (c) x 64 cols (k)] bf16, 1 block:     V_Z^T, k >= L zero
-//   QZBD [128 rows (h,k) x 128] bf16, 2 blocks of 16 KB: row h*L + k holds
-//        s·Q_Z[k] in head h's 32 columns and zeros elsewhere; rows >= 4L zero;
-//        stored twice, as the hi and lo bf16 halves of the fp32 value (the
-//        link query is one vector per link, so its rounding is not averaged)
+//   QZ   [L rows x 128] bf16, 2 blocks of L*128 bytes, twice: s·Q_Z as the hi
+//        and lo bf16 halves of the fp32 value (the link query is one vector
+//        per link, so its rounding is not averaged).  The attention kernels
+//        expand it in shared memory to the block-diagonal [128 x 128] operand
+//        (row h*L + k = s·Q_Z[k] in head h's columns, zeros elsewhere).
 template <int L>
 __global__ void __launch_bounds__(512)
     k_link_proj(const bf16* __restrict__ Z, int64_t nrows, const bf16* __restrict__ g1,
@@ -468,19 +495,19 @@ __global__ void __launch_bounds__(512)
     }
   }
   // The images are built per user in shared memory (the operands of the MMA
-  // are dead) and copied out with coalesced 16-byte stores.  Piece per user:
-  // s·K_Z (L*256 bytes), V_Z^T (one 16 KB block) or the block-diagonal s·Q_Z
-  // hi + lo (four 16 KB blocks).
+  // are dead) and written out with one bulk copy per user.  Piece per user:
+  // s·K_Z (L*256 bytes), V_Z^T (one 16 KB block) or s·Q_Z hi + lo (2 x L*256).
   constexpr int UP = kTile / L;                               // users per tile
-  const uint32_t piece = which == 0 ? 4 * kBlk : which == 1 ? kz_bytes(L) : kBlk;
-  const uint32_t img_off = which == 0 ? kz_bytes(L) + kBlk : which == 1 ? 0 : kz_bytes(L);
-  const int upp = which == 0 ? 1 : which == 1 ? UP : (UP < 4 ? UP : 4);   // users per pass
+  const uint32_t piece = which == 0 ? 2 * kz_bytes(L) : which == 1 ? kz_bytes(L) : kBlk;
+  const uint32_t img_off = which == 0 ? qz_off(L) : which == 1 ? 0 : kz_bytes(L);
+  const int upp = which == 2 ? (UP < 4 ? UP : 4) : UP;       // users per pass
   uint8_t* stage = sm;                                        // 96 KB: sAh, sAl, sW
   const int ju = r / L, k = r % L;
   const int64_t u0 = (int64_t)blockIdx.x * UP;
   const int n_users = (int)((nrows - (int64_t)blockIdx.x * kTile) / L) < UP
                           ? (int)((nrows - (int64_t)blockIdx.x * kTile) / L) : UP;
   for (int j0 = 0; j0 < n_users; j0 += upp) {
+    if (threadIdx.x == 0) bulk_wait_read<0>();   // the previous pass's copies have read it
     __syncthreads();   // the staging area is free (MMA operands, previous pass)
     if (ju >= j0 && ju < j0 + upp && valid) {
       uint8_t* img = stage + (uint32_t)(ju - j0) * piece;
@@ -493,72 +520,63 @@ __global__ void __launch_bounds__(512)
           for (int kp = k + L; kp < 64; kp += L)
             *reinterpret_cast<bf16*>(img + sw128_offset(c0 + cc, kp)) = __float2bfloat16_rn(0.f);
         }
-      } else {                    // rows h*L + k: head `part` holds s·Q_Z, the rest zero
-        uint8_t* qbl = img + 2 * kBlk;
-        const uint4 z4 = make_uint4(0, 0, 0, 0);
+      } else {                    // s·Q_Z row k, hi then lo
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const uint4 hv = pack8(v + q * 8), lv = pack8(lo + q * 8);
-#pragma unroll
-          for (int h = 0; h < kH; ++h) {
-            sw_st16(img, kBlk, h * L + k, c0 + q * 8, h == part ? hv : z4);
-            sw_st16(qbl, kBlk, h * L + k, c0 + q * 8, h == part ? lv : z4);
-          }
+          sw_st16(img, (uint32_t)L * 128, k, c0 + q * 8, pack8(v + q * 8));
+          sw_st16(img + kz_bytes(L), (uint32_t)L * 128, k, c0 + q * 8, pack8(lo + q * 8));
         }
-        for (int p2 = kH * L + k; p2 < kTile; p2 += L)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            sw_st16(img, kBlk, p2, c0 + q * 8, z4);
-            sw_st16(qbl, kBlk, p2, c0 + q * 8, z4);
-          }
       }
     }
+    fence_proxy_async_smem();
     __syncthreads();
-    const int nu = n_users - j0 < upp ? n_users - j0 : upp;
-    const uint32_t chunks = piece / 16;
-    for (uint32_t e = threadIdx.x; e < (uint32_t)nu * chunks; e += blockDim.x) {
-      const uint32_t j = e / chunks, q = e - j * chunks;
-      uint8_t* dst = ws + Lw.uimg + (size_t)(u0 + j0 + j) * Lw.uimg_bytes + img_off;
-      reinterpret_cast<uint4*>(dst)[q] = reinterpret_cast<const uint4*>(stage + j * piece)[q];
+    if (threadIdx.x == 0) {
+      const int nu = n_users - j0 < upp ? n_users - j0 : upp;
+      for (int j = 0; j < nu; ++j)
+        bulk_store(ws + Lw.uimg + (size_t)(u0 + j0 + j) * Lw.uimg_bytes + img_off,
+                   stage + (uint32_t)j * piece, piece);
+      bulk_commit();
     }
   }
+  if (threadIdx.x == 0) bulk_wait<0>();   // the images are complete before the CTA exits
   cta_teardown(c);
 }
 
 // ----------------------------------------------------- history projections
 // One persistent CTA per SM walks the tile list.  For each tile: TMA the 128
 // history rows, LN1, Q/K/V = X^·W on the tensor cores (X^ as hi + lo bf16);
-// writes the valid rows of Q_E, K_E and V_E (row-major bf16) through a
-// swizzled staging tile with coalesced stores.  The next tile's rows are
-// loaded while this tile's outputs are written.  512 threads: thread (row,
-// part) handles a quarter of the row's columns; LN1's statistics are reduced
-// across the four parts.
-template <bool LAST>
+// the outputs go through swizzled staging tiles: a full tile (128 valid rows)
+// leaves with TMA tensor stores that overlap the next steps, a partial tile
+// (its rows end at a user boundary) with coalesced plain stores of its valid
+// rows.  The next tile's rows are loaded while this tile's outputs are
+// written.  512 threads: thread (row, part) handles a quarter of the row's
+// columns; LN1's statistics are reduced across the four parts.
 __global__ void __launch_bounds__(512, 1)
-    k_hist_proj(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ g1,
-                const bf16* __restrict__ b1, uint8_t* __restrict__ ws, LayerWs Lw,
-                unsigned* status) {
+    k_hist_proj(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmQ,
+                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                const bf16* __restrict__ g1, const bf16* __restrict__ b1, uint8_t* __restrict__ ws,
+                LayerWs Lw, unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
-  uint8_t* sE = sm;               // E tile -> LN1 output, hi half
-  uint8_t* sEl = sm + 2 * kBlk;    // LN1 output, lo half -> output staging
-  uint8_t* sW = sm + 4 * kBlk;     // [Wq,] Wk, Wv images
-  constexpr int NW = LAST ? 2 : 3;
-  float* red = reinterpret_cast<float*>(sm + (4 + 2 * NW) * kBlk);
+  uint8_t* sE = sm;                // E tile -> LN1 output, hi half
+  uint8_t* sEl = sm + 2 * kBlk;    // LN1 output, lo half -> Q, V staging
+  uint8_t* sW = sm + 4 * kBlk;     // Wq, Wk, Wv images
+  uint8_t* sS = sm + 10 * kBlk;    // K staging
+  float* red = reinterpret_cast<float*>(sm + 12 * kBlk);
   Cta c;
-  cta_setup(sm + (4 + 2 * NW) * kBlk + 2048, 3, c);
+  cta_setup(sm + 12 * kBlk + 2048, 3, c);
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
-  bf16* qe = reinterpret_cast<bf16*>(ws + Lw.qe);
-  bf16* ke = reinterpret_cast<bf16*>(ws + Lw.ke);
-  bf16* ve = reinterpret_cast<bf16*>(ws + Lw.ve);
   uint32_t eph = 0, mph = 0;
   if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(&c.bar[2], NW * 2 * kBlk);
-    int slot = 0;
-    if (!LAST) bulk_load(sW + 2 * kBlk * slot++, ws + Lw.img_q, 2 * kBlk, &c.bar[2]);
-    bulk_load(sW + 2 * kBlk * slot++, ws + Lw.img_k, 2 * kBlk, &c.bar[2]);
-    bulk_load(sW + 2 * kBlk * slot, ws + Lw.img_v, 2 * kBlk, &c.bar[2]);
+    prefetch_tmap(&tmE);
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    mbar_arrive_expect_tx(&c.bar[2], 6 * kBlk);
+    bulk_load(sW, ws + Lw.img_q, 2 * kBlk, &c.bar[2]);
+    bulk_load(sW + 2 * kBlk, ws + Lw.img_k, 2 * kBlk, &c.bar[2]);
+    bulk_load(sW + 4 * kBlk, ws + Lw.img_v, 2 * kBlk, &c.bar[2]);
     if ((int)blockIdx.x < n_tiles) {
       const int4 tl = tiles[blockIdx.x];
       mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
@@ -575,6 +593,9 @@ __global__ void __launch_bounds__(512, 1)
   for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
     const int4 tl = tiles[t];
     const int r0 = tl.y, nv = tl.z;
+    // the previous tile's tensor stores have read the staging tiles (the LN
+    // barriers below pass this on to every thread before sEl is rewritten)
+    if (threadIdx.x == 0) bulk_wait_read<0>();
     mbar_wait(&c.bar[0], eph, status, c.abort_flag);
     eph ^= 1u;
     {
@@ -584,24 +605,14 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
       for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sE, kBlk, row, c0 + q * 8), x + q * 8);
       layer_norm_part(x, c0, g1, b1, red, part, row);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float h8[8], l8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          h8[k] = __bfloat162float(__float2bfloat16_rn(x[q * 8 + k]));
-          l8[k] = x[q * 8 + k] - h8[k];
-        }
-        sw_st16(sE, kBlk, row, c0 + q * 8, pack8(h8));
-        sw_st16(sEl, kBlk, row, c0 + q * 8, pack8(l8));
-      }
+      split_part_st(sE, sEl, row, c0, x);
     }
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {
       tc_fence_after();
-      for (int w = 0; w < NW; ++w) {
-        const uint32_t d = c.tmem + (LAST ? w + 1 : w) * 128;
+      for (int w = 0; w < 3; ++w) {
+        const uint32_t d = c.tmem + w * 128;
         mma_tile(d, smem_u32(sE), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128, 128, false);
         mma_tile(d, smem_u32(sEl), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128, 128, true);
       }
@@ -614,24 +625,38 @@ __global__ void __launch_bounds__(512, 1)
       tma_load_2d(sE, &tmE, 0, tl2.y, &c.bar[0]);
       tma_load_2d(sE + kBlk, &tmE, 64, tl2.y, &c.bar[0]);
     }
-    // Q_E, K_E, V_E rows: TMEM -> bf16 -> swizzled staging tile (the lo half
-    // of LN1's output is free now) -> coalesced stores of the valid rows
-    for (int mtx = LAST ? 1 : 0; mtx < 3; ++mtx) {
+    // Q_E -> sEl, K_E -> sS, V_E -> sEl (once Q's store has read it)
+    const bool full = nv == kTile;
+    for (int mtx = 0; mtx < 3; ++mtx) {
+      uint8_t* buf = mtx == 1 ? sS : sEl;
+      if (mtx == 2) {
+        if (full && threadIdx.x == 0) bulk_wait_read<1>();
+        __syncthreads();
+      }
       float v[32];
       tmem_ld16(ta + mtx * 128 + c0, v);
       tmem_ld16(ta + mtx * 128 + c0 + 16, v + 16);
       tmem_ld_wait();
 #pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(sEl, kBlk, row, c0 + q * 8, pack8(v + q * 8));
+      for (int q = 0; q < 4; ++q) sw_st16(buf, kBlk, row, c0 + q * 8, pack8(v + q * 8));
+      fence_proxy_async_smem();
       __syncthreads();
-      bf16* dst = (mtx == 0 ? qe : mtx == 1 ? ke : ve) + (int64_t)r0 * kD;
-      tile_store_rows(sEl, dst, nv);
-      __syncthreads();
+      if (full) {
+        if (threadIdx.x == 0) {
+          const CUtensorMap* tm = mtx == 0 ? &tmQ : mtx == 1 ? &tmK : &tmV;
+          tma_store_2d(tm, buf, 0, r0);
+          tma_store_2d(tm, buf + kBlk, 64, r0);
+          bulk_commit();
+        }
+      } else {
+        const size_t off = mtx == 0 ? Lw.qe : mtx == 1 ? Lw.ke : Lw.ve;
+        tile_store_rows(buf, reinterpret_cast<bf16*>(ws + off) + (int64_t)r0 * kD, nv);
+      }
     }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
   }
+  if (threadIdx.x == 0) bulk_wait<0>();
   cta_teardown(c);
 }
 
@@ -651,13 +676,12 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sK = sm + 2 * kBlk;      // K_E -> P2 -> A_E (lo)
   uint8_t* sV = sm + 4 * kBlk;      // V_E rows (row-major, read as an MN-major operand)
   uint8_t* sWo = sm + 6 * kBlk;     // Wo image (not in the last layer)
-  uint8_t* sU = sm + (LAST ? 6 : 8) * kBlk;  // user images
-  uint8_t* sKZ = sU;
-  uint8_t* sVZT = sU + kz_bytes(L);
-  uint8_t* sQBD = sVZT + kBlk;
-  float* red = reinterpret_cast<float*>(sU + uimg_bytes(L));   // [4][128]
+  uint8_t* sQBD = sm + (LAST ? 6 : 8) * kBlk;   // block-diagonal s·Q_Z, hi then lo
+  uint8_t* sKZ = sQBD + 4 * kBlk;                // user images: s·K_Z, V_Z^T
+  uint8_t* sVZT = sKZ + kz_bytes(L);
+  float* red = reinterpret_cast<float*>(sVZT + kBlk);   // [4][128]
   Cta c;
-  cta_setup(sU + uimg_bytes(L) + 2048, 3, c);
+  cta_setup(sVZT + kBlk + 2048, 3, c);
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
   float* yd = reinterpret_cast<float*>(ws + Lw.yd);
@@ -679,7 +703,7 @@ __global__ void __launch_bounds__(512, 1)
     const int4 tl = tiles[t];
     const int u = tl.x, r0 = tl.y, nv = tl.z;
     if (threadIdx.x == 0) {
-      uint32_t bytes = 4 * kBlk + (LAST ? 0 : 2 * kBlk) + (u != cur_u ? Lw.uimg_bytes : 0);
+      uint32_t bytes = 4 * kBlk + (LAST ? 0 : 2 * kBlk) + (u != cur_u ? 3 * kz_bytes(L) + kBlk : 0);
       mbar_arrive_expect_tx(&c.bar[0], bytes);
       if (!LAST) {
         tma_load_2d(sQ, &tmQ, 0, r0, &c.bar[0]);
@@ -689,11 +713,20 @@ __global__ void __launch_bounds__(512, 1)
       tma_load_2d(sK + kBlk, &tmK, 64, r0, &c.bar[0]);
       tma_load_2d(sV, &tmV, 0, r0, &c.bar[0]);
       tma_load_2d(sV + kBlk, &tmV, 64, r0, &c.bar[0]);
-      if (u != cur_u) bulk_load(sU, ws + Lw.uimg + (size_t)u * Lw.uimg_bytes, Lw.uimg_bytes, &c.bar[0]);
+      if (u != cur_u) {
+        const uint8_t* img = ws + Lw.uimg + (size_t)u * Lw.uimg_bytes;
+        bulk_load(sKZ, img, kz_bytes(L) + kBlk, &c.bar[0]);
+        bulk_load(sQBD, img + qz_off(L), 2 * kz_bytes(L), &c.bar[0]);
+      }
     }
-    cur_u = u;
     mbar_wait(&c.bar[0], lph, status, c.abort_flag);
     lph ^= 1u;
+    if (u != cur_u) {
+      expand_qbd<L>(sQBD, row, part);
+      fence_proxy_async_smem();
+      __syncthreads();
+    }
+    cur_u = u;
     // phase 1: history scores S_h = Q_E,h (s K_Z,h)^T -> TMEM [0, HL);
     //          link scores, transposed: S'^T = (s Q_Z)_bd K_E^T -> TMEM [128, 256)
     if (threadIdx.x == 0) {
@@ -881,17 +914,17 @@ __global__ void __launch_bounds__(512, 1)
     const int4 tl = tiles[t];
     const int u = tl.x, r0 = tl.y, nv = tl.z;
     if (threadIdx.x == 0) {
-      const uint32_t qbd_bytes = 4 * kBlk;
-      mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk + (u != cur_u ? qbd_bytes : 0));
+      const uint32_t qz_bytes = 2 * kz_bytes(L);
+      mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk + (u != cur_u ? qz_bytes : 0));
       tma_load_2d(sE, &tmE, 0, r0, &c.bar[0]);
       tma_load_2d(sE + kBlk, &tmE, 64, r0, &c.bar[0]);
       if (u != cur_u)
-        bulk_load(sQBD, ws + Lw.uimg + (size_t)u * Lw.uimg_bytes + kz_bytes(L) + kBlk, qbd_bytes,
-                  &c.bar[0]);
+        bulk_load(sQBD, ws + Lw.uimg + (size_t)u * Lw.uimg_bytes + qz_off(L), qz_bytes, &c.bar[0]);
     }
-    cur_u = u;
     mbar_wait(&c.bar[0], lph, status, c.abort_flag);
     lph ^= 1u;
+    if (u != cur_u) expand_qbd<L>(sQBD, row, part);   // ordered before the MMAs by LN1's barriers
+    cur_u = u;
     {
       float x[32];
 #pragma unroll
@@ -1599,14 +1632,14 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
                           (const bf16*)w.g1, (const bf16*)w.b1, ws, Lw, status);
       if (rc) return rc;
     } else {
-      const int smem = 1024 + 10 * kBlk + 2048 + kBarBytes;
-      if (!set_smem(k_hist_proj<false>, smem)) return LIME_ERR_CUDA;
-      int rc = launch_pdl(k_hist_proj<false>, dim3(grid), dim3(512), smem, st, 1, tmE,
+      const int smem = 1024 + 12 * kBlk + 2048 + kBarBytes;
+      if (!set_smem(k_hist_proj, smem)) return LIME_ERR_CUDA;
+      int rc = launch_pdl(k_hist_proj, dim3(grid), dim3(512), smem, st, 1, tmE, tmQ, tmK, tmV,
                           (const bf16*)w.g1, (const bf16*)w.b1, ws, Lw, status);
       if (rc) return rc;
     }
     if (!last) {
-      const int smem = 1024 + 8 * kBlk + uimg_bytes(L) + 2048 + kBarBytes;
+      const int smem = 1024 + 12 * kBlk + kz_bytes(L) + kBlk + 2048 + kBarBytes;
       if (!set_smem(k_hist_attn<L, false>, smem)) return LIME_ERR_CUDA;
       int rc = launch_pdl(k_hist_attn<L, false>, dim3(grid), dim3(512), smem, st, 1, tmQ, tmK, tmV,
                           ws, Lw, status);

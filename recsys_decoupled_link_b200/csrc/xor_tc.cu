@@ -17,27 +17,30 @@
 //                    block 0 turns hist_offsets into the tile list (user,
 //                    first row, valid rows)
 //   k_link_proj      LN1(Z) -> Q_Z, K_Z, V_Z (split precision) -> per-user
-//                    operand images: s·K_Z, V_Z^T, and s·Q_Z laid out
-//                    block-diagonally over heads so that one MMA yields the
-//                    link branch's scores transposed (links on TMEM lanes)
+//                    operand images: s·K_Z, V_Z^T and s·Q_Z (hi + lo); one
+//                    CTA per (128 link rows, Q|K|V)
 //   k_hist_proj      LN1(E) (split precision) -> Q_E, K_E, V_E (row-major)
 //   k_hist_attn      history branch: softmax over the user's l links, P·V_Z,
 //                    then (P·V_Z)·Wo -> Yd (fp32 attention delta);
-//                    link branch: per tile and (head, link) the partial
-//                    softmax statistics (max, sum) and the weighted V sum
-//                    (V_E read as an MN-major operand, no transpose)
-//   k_link_merge     log-sum-exp merge of a user's tile partials -> b (fp32)
+//                    link branch: s·Q_Z laid out block-diagonally over heads
+//                    (expanded on chip) so that one MMA yields the scores
+//                    transposed (links on TMEM lanes); per tile and (head,
+//                    link) the partial softmax statistics (max, sum) and the
+//                    weighted V sum (V_E read as an MN-major operand)
 //   k_hist_ffn       Y = E + Yd, LN2, GatedMLP in 64-wide chunks, E' = Y + ·
-//   k_link_out       Y_Z = Z + b·Wo, LN2, one GatedMLP chunk per CTA (split
-//                    precision), fp32 partials; k_link_finish sums them -> Z'
-//   (k_link_proj also runs one CTA per (tile, Q|K|V))
+//                    (warp-specialized pipeline)
+//   k_link_tail      per 128 link rows, a cluster of four CTAs: log-sum-exp
+//                    merge of the tile partials -> b, Y_Z = Z + b·Wo, LN2,
+//                    GatedMLP (one hidden chunk per CTA, split precision),
+//                    Z' = Y_Z + sum of the chunks
 // The last layer (E_out = NULL) skips everything only E' needs: Q_E, the
 // history branch, Wo on history rows and k_hist_ffn; its link branch runs in
 // k_hist_link, which keeps K_E and V_E on chip.
 //
-// CTAs run their phases synchronously: thread 0 issues the MMAs of a phase,
-// all 128 threads wait on an mbarrier (bounded), then each thread works on its
-// TMEM lane (one tile row).  Every wait is bounded and sets LIME_FLAG_TIMEOUT.
+// Kernels use 512 threads (thread (row, part): a TMEM lane and a quarter of
+// the row's columns) or warp-specialized roles; one thread issues the MMAs.
+// Every kernel is launched with programmatic dependent launch (pdl_launch /
+// pdl_wait).  Every wait is bounded and sets LIME_FLAG_TIMEOUT.
 #include "lime_fast.cuh"
 #include "sm100.cuh"
 

@@ -13,8 +13,8 @@
 //   warp 0     TMA producer: 128-row tiles of T into a STAGES-deep ring
 //   warp 1     tcgen05.mma issuer (M=128, N=H*l, K=128 as 8 K-steps) into one
 //              of two TMEM accumulators
-//   warps 2-9  epilogue, two warps per TMEM lane quadrant each taking half of
-//              the heads: tcgen05.ld of its row, softmax per head over l links
+//   warps 2-   epilogue, up to four warps per TMEM lane quadrant, each taking
+//              a share of the heads: tcgen05.ld of its row, softmax per head over l links
 //              in fp32, bf16 into a 128-byte-swizzled staging tile, TMA store
 //              of the tile (rows past n_items are clipped by TMA)
 // Every wait is bounded; a timeout sets LIME_FLAG_TIMEOUT and the CTA drains
@@ -31,7 +31,7 @@ namespace {
 constexpr int kD = 128;    // model dim handled here
 constexpr int kBM = 128;   // catalogue rows per tile
 
-template <int HL>
+template <int HL, int L>
 struct CacheCfg {
   static constexpr int STAGES = HL <= 128 ? 4 : 3;
   static constexpr int OUTB = HL <= 128 ? 2 : 1;
@@ -43,6 +43,13 @@ struct CacheCfg {
   static constexpr int OFF_O = OFF_B + B_BYTES;
   static constexpr int OFF_BAR = OFF_O + OUTB * O_BYTES;
   static constexpr int SMEM = 1024 + OFF_BAR + 256;
+  // epilogue warps per TMEM lane quadrant: one head each for up to 4 heads
+  // of l <= 32 links; two (half of the heads each) for l = 64, whose rows need
+  // more registers than 18 warps leave per thread
+  static constexpr int H_ = HL / L;
+  static constexpr int WPQ = L >= 64 ? (H_ < 2 ? H_ : 2) : (H_ < 4 ? H_ : 4);
+  static constexpr int EPI = 4 * WPQ * 32;          // epilogue threads
+  static constexpr int THREADS = 64 + EPI;
 };
 
 // G^T image: block b (K columns [64b, 64b+64)) of HL rows x 128 bytes,
@@ -112,10 +119,10 @@ __global__ void __launch_bounds__(128) k_fold_g_img(const bf16* __restrict__ L,
 }
 
 template <int HL, int L>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(CacheCfg<HL, L>::THREADS, 1)
     k_cache_tc(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmC,
                const bf16* __restrict__ gimg, int n_tiles, unsigned* status) {
-  using C = CacheCfg<HL>;
+  using C = CacheCfg<HL, L>;
   constexpr int H = HL / L;
   constexpr uint32_t IDESC = idesc_bf16(kBM, HL);
   extern __shared__ uint8_t smem_raw[];
@@ -139,8 +146,8 @@ __global__ void __launch_bounds__(320, 1)
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 256);
-      mbar_init(&ofull[a], 256);
+      mbar_init(&tempty[a], C::EPI);
+      mbar_init(&ofull[a], C::EPI);
       mbar_init(&ofree[a], 1);
     }
     mbar_init(bready, 1);
@@ -207,11 +214,12 @@ __global__ void __launch_bounds__(320, 1)
       mbar_wait(mdone, 0, status, &abort_flag);
     }
   } else {
-    // epilogue: 8 warps, two per TMEM lane quadrant; the warp's lane is tile row
-    // `row` and it handles half of the heads (half = 0 for warps 2-5, 1 for 6-9)
+    // epilogue: WPQ warps per TMEM lane quadrant; the warp's lane is tile row
+    // `row` and it handles heads grp*HPW .. (group grp = (warp - 2) / 4)
     const int et = threadIdx.x - 64;
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int grp = (warp - 2) >> 2;                // 0 .. WPQ-1
+    constexpr int HPW = H / C::WPQ < 1 ? 1 : H / C::WPQ;   // heads per epilogue warp
     const int row = quad * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     int it = 0;
@@ -225,7 +233,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       uint8_t* stage = sO + ob * C::O_BYTES;
 #pragma unroll 1
-      for (int h = half * (H / 2); h < (half + 1) * (H / 2); ++h) {
+      for (int h = grp * HPW; h < (grp + 1) * HPW && h < H; ++h) {
         float z[L];
 #pragma unroll
         for (int q = 0; q < L / 16; ++q)
@@ -283,7 +291,7 @@ __global__ void __launch_bounds__(320, 1)
 template <int HL, int L>
 int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, unsigned* status,
                  cudaStream_t st) {
-  using C = CacheCfg<HL>;
+  using C = CacheCfg<HL, L>;
   CUtensorMap tmT, tmC;
   if (!make_tmap_2d_bf16(&tmT, T, kD, (uint64_t)n, kD * 2, 64, kBM)) return LIME_ERR_CUDA;
   if (!make_tmap_2d_bf16(&tmC, cache, HL, (uint64_t)n, HL * 2, 64, kBM)) return LIME_ERR_CUDA;
@@ -292,7 +300,7 @@ int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, unsigne
     return LIME_ERR_CUDA;
   const int n_tiles = (int)((n + kBM - 1) / kBM);
   const int grid = n_tiles < num_sms() ? n_tiles : num_sms();
-  return launch_pdl(k_cache_tc<HL, L>, dim3(grid), dim3(320), C::SMEM, st, 1, tmT, tmC, img,
+  return launch_pdl(k_cache_tc<HL, L>, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, tmT, tmC, img,
                     n_tiles, status);
 }
 

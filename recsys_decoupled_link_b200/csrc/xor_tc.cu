@@ -140,21 +140,48 @@ __device__ __forceinline__ float row_max4(float v, float* red, int part, int row
   return t;
 }
 
+// LayerNorm scratch of the 512-thread kernels: two [4][128] reduction
+// buffers and the affine parameters as fp32 (g, then b).
+constexpr int kLnFloats = 2 * 512 + 2 * kD;
+constexpr int kLnBytes = kLnFloats * 4;
+
+// Stages g and b (bf16 [128]) as fp32 at gb (call before the first LN; the
+// LN's own barriers order these writes before the reads).
+__device__ __forceinline__ void ln_stage(float* gb, const bf16* g, const bf16* b) {
+  if (threadIdx.x < kD) {
+    gb[threadIdx.x] = __bfloat162float(g[threadIdx.x]);
+    gb[kD + threadIdx.x] = __bfloat162float(b[threadIdx.x]);
+  }
+}
+
 // LayerNorm of one row held as four 32-column parts (x = this thread's part,
-// columns c0..c0+31), affine with g, b.
-__device__ __forceinline__ void layer_norm_part(float* x, int c0, const bf16* g, const bf16* b,
-                                                float* red, int part, int row) {
+// columns c0..c0+31), affine with the staged g, b.  `red` is a kLnFloats
+// scratch (red[0..1023] for the two reductions, g and b after them); all 512
+// threads take part (two block-wide barriers).
+__device__ __forceinline__ void layer_norm_part(float* x, int c0, float* red, int part, int row) {
   float s1 = 0.f;
 #pragma unroll
   for (int k = 0; k < 32; ++k) s1 += x[k];
-  const float mu = row_sum4(s1, red, part, row) * (1.0f / kD);
+  red[part * 128 + row] = s1;
+  __syncthreads();
+  const float mu = (red[row] + red[128 + row] + red[256 + row] + red[384 + row]) * (1.0f / kD);
   float s2 = 0.f;
 #pragma unroll
   for (int k = 0; k < 32; ++k) { const float d0 = x[k] - mu; s2 += d0 * d0; }
-  const float rstd = rsqrtf(row_sum4(s2, red, part, row) * (1.0f / kD) + kLnEps);
+  red[512 + part * 128 + row] = s2;
+  __syncthreads();
+  const float rstd = rsqrtf((red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row]) *
+                                (1.0f / kD) + kLnEps);
+  const float4* g4 = reinterpret_cast<const float4*>(red + 1024 + c0);
+  const float4* b4 = reinterpret_cast<const float4*>(red + 1024 + kD + c0);
 #pragma unroll
-  for (int k = 0; k < 32; ++k)
-    x[k] = (x[k] - mu) * rstd * __bfloat162float(g[c0 + k]) + __bfloat162float(b[c0 + k]);
+  for (int q = 0; q < 8; ++q) {
+    const float4 gv = g4[q], bv = b4[q];
+    x[4 * q] = (x[4 * q] - mu) * rstd * gv.x + bv.x;
+    x[4 * q + 1] = (x[4 * q + 1] - mu) * rstd * gv.y + bv.y;
+    x[4 * q + 2] = (x[4 * q + 2] - mu) * rstd * gv.z + bv.z;
+    x[4 * q + 3] = (x[4 * q + 3] - mu) * rstd * gv.w + bv.w;
+  }
 }
 
 // Loads 128 consecutive fp32 TMEM columns of this thread's lane.
@@ -435,7 +462,8 @@ __global__ void __launch_bounds__(512)
   float* red = reinterpret_cast<float*>(sm + 6 * kBlk);
   const int which = blockIdx.y;
   Cta c;
-  cta_setup(sm + 6 * kBlk + 2048, 2, c, 128);
+  cta_setup(sm + 6 * kBlk + kLnBytes, 2, c, 128);
+  ln_stage(red + 1024, g1, b1);
   uint32_t mph = 0;
   if (threadIdx.x == 0) {
     const size_t img = which == 0 ? Lw.img_q : which == 1 ? Lw.img_k : Lw.img_v;
@@ -458,7 +486,7 @@ __global__ void __launch_bounds__(512)
 #pragma unroll
       for (int i2 = 0; i2 < 32; ++i2) x[i2] = 0.f;
     }
-    layer_norm_part(x, c0, g1, b1, red, part, r);
+    layer_norm_part(x, c0, red, part, r);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       float h8[8], l8[8];
@@ -567,7 +595,8 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sS = sm + 10 * kBlk;    // K staging
   float* red = reinterpret_cast<float*>(sm + 12 * kBlk);
   Cta c;
-  cta_setup(sm + 12 * kBlk + 2048, 3, c);
+  cta_setup(sm + 12 * kBlk + kLnBytes, 3, c);
+  ln_stage(red + 1024, g1, b1);
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
   uint32_t eph = 0, mph = 0;
@@ -607,7 +636,7 @@ __global__ void __launch_bounds__(512, 1)
       float x[32];
 #pragma unroll
       for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sE, kBlk, row, c0 + q * 8), x + q * 8);
-      layer_norm_part(x, c0, g1, b1, red, part, row);
+      layer_norm_part(x, c0, red, part, row);
       split_part_st(sE, sEl, row, c0, x);
     }
     fence_proxy_async_smem();
@@ -896,7 +925,8 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sQBD = sm + 8 * kBlk;   // block-diagonal s*Q_Z, hi then lo (4 blocks)
   float* red = reinterpret_cast<float*>(sm + 12 * kBlk);
   Cta c;
-  cta_setup(sm + 12 * kBlk + 2048, 3, c);
+  cta_setup(sm + 12 * kBlk + kLnBytes, 3, c);
+  ln_stage(red + 1024, g1, b1);
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
   float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
@@ -932,7 +962,7 @@ __global__ void __launch_bounds__(512, 1)
       float x[32];
 #pragma unroll
       for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sE, kBlk, row, c0 + q * 8), x + q * 8);
-      layer_norm_part(x, c0, g1, b1, red, part, row);
+      layer_norm_part(x, c0, red, part, row);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float h8[8], l8[8];
@@ -1349,7 +1379,7 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
 // pushes rows 32q..32q+31 of it to CTA q; CTA r sums the four partials of its
 // rows, adds Y_Z and writes Z'.  No atomics; the summation order is fixed.
 // 512 threads: thread (row, part) owns columns part*32 .. part*32+31.
-constexpr int kTailSmem = 1024 + 12 * kBlk + 2048 + 64;
+constexpr int kTailSmem = 1024 + 12 * kBlk + kLnBytes + 64;
 
 template <int L>
 __global__ void __launch_bounds__(512, 1)
@@ -1372,7 +1402,8 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sP = sAh;                 // fp32 partial [128 x 128] over sAh, sAl
   const uint32_t cr = cluster_rank();
   Cta c;
-  cta_setup(sm + 12 * kBlk + 2048, 5, c);  // bar: 0 Wo, 1 mma, 2 chunk, 3 b rows, 4 partials
+  cta_setup(sm + 12 * kBlk + kLnBytes, 5, c);  // bar: 0 Wo, 1 mma, 2 chunk, 3 b rows, 4 partials
+  ln_stage(red + 1024, g2, b2);
   uint32_t mph = 0;
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
@@ -1498,7 +1529,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
       for (int q = 0; q < 8; ++q) dst[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
     }
-    layer_norm_part(y, c0, g2, b2, red, part, r);
+    layer_norm_part(y, c0, red, part, r);
     split_part_st(sAh, sAl, r, c0, y);
   }
   fence_proxy_async_smem();
@@ -1612,7 +1643,7 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     if (rc) return rc;
   }
   {
-    const int smem = 1024 + 6 * kBlk + 2048 + kBarBytes;   // 96 KB of it stage the images
+    const int smem = 1024 + 6 * kBlk + kLnBytes + kBarBytes;   // 96 KB of it stage the images
     if (!set_smem(k_link_proj<L>, smem)) return LIME_ERR_CUDA;
     int rc = launch_pdl(k_link_proj<L>, dim3((unsigned)((nz + kTile - 1) / kTile), 3), dim3(512),
                         smem, st, 1, (const bf16*)Z_in, nz, (const bf16*)w.g1, (const bf16*)w.b1,
@@ -1629,13 +1660,13 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     const int64_t tiles_hi = Lw.max_tiles;
     const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
     if (last) {
-      const int smem = 1024 + 12 * kBlk + 2048 + kBarBytes;
+      const int smem = 1024 + 12 * kBlk + kLnBytes + kBarBytes;
       if (!set_smem(k_hist_link<L>, smem)) return LIME_ERR_CUDA;
       int rc = launch_pdl(k_hist_link<L>, dim3(grid), dim3(512), smem, st, 1, tmE,
                           (const bf16*)w.g1, (const bf16*)w.b1, ws, Lw, status);
       if (rc) return rc;
     } else {
-      const int smem = 1024 + 12 * kBlk + 2048 + kBarBytes;
+      const int smem = 1024 + 12 * kBlk + kLnBytes + kBarBytes;
       if (!set_smem(k_hist_proj, smem)) return LIME_ERR_CUDA;
       int rc = launch_pdl(k_hist_proj, dim3(grid), dim3(512), smem, st, 1, tmE, tmQ, tmK, tmV,
                           (const bf16*)w.g1, (const bf16*)w.b1, ws, Lw, status);

@@ -42,7 +42,7 @@ import torch  # noqa: E402
 # be of the kernel as it is now, else the entry is removed.
 NCU_TRAFFIC = {
     # profiles/k_cache_tc_standard.md: k_cache_tc<128, 32>, 1M items
-    "cache": 256.134144e6 + 201.650176e6,
+    "cache": 256.093696e6 + 200.985088e6,
 }
 
 
@@ -368,6 +368,30 @@ def main():
     torch.cuda.synchronize()
     e2e_step_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in ee)], dist,
                                  "cuda")[0] / args.steps
+
+    # Scoring at scale: 16 users x 65,536 candidates drawn uniformly from the
+    # whole catalogue (gathered rows far exceed L2; L2 flushed before each
+    # call), against the cache and L^P this step built.
+    sc_users, sc_per = 16, 65536
+    g = torch.Generator(device="cpu").manual_seed(4242)
+    sc_ids = torch.randint(0, w.n_items, (sc_users * sc_per,), generator=g,
+                           dtype=torch.int64).to(torch.int32).cuda()
+    sc_off = (torch.arange(sc_users + 1, dtype=torch.int64) * sc_per).cuda()
+    sc_LP = pipeline.user_encode(x, buf)[:sc_users].contiguous()
+    sc_O = torch.empty(sc_users * sc_per, w.d, dtype=buf.O.dtype, device="cuda")
+    sc_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for _ in range(3):
+        lime.lime_score_candidates(x.dims, buf.cache, sc_ids, sc_off, sc_users * sc_per, sc_LP,
+                                   sc_O, buf.ws)
+    for k in range(args.steps):
+        flush.zero_()
+        sc_ev[k][0].record(stream)
+        lime.lime_score_candidates(x.dims, buf.cache, sc_ids, sc_off, sc_users * sc_per, sc_LP,
+                                   sc_O, buf.ws)
+        sc_ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    sc_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in sc_ev)], dist,
+                           "cuda")[0] / args.steps
     if lime.lime_get_status(buf.ws) != 0:
         raise RuntimeError("device status flags set during the timed steps")
 
@@ -398,16 +422,29 @@ def main():
                           "the k_fold_g_img prologue)")
         roof["algorithmic_bytes_per_launch"] = work["cache"][1]
         roof["peak_source"] = pk["source"] + " (MEASURED_PEAKS.json hbm_gbs copy bandwidth)"
+        ur = phase_roof("user")
+        if ur["unit"] == "TFLOP/s":
+            ur["frac_of_sustained"] = ur["achieved"] / pk["bf16_tflops_sustained"]
+        sc_pairs = sc_users * sc_per
+        sc_bytes = sc_pairs * (w.H * w.l * (2 if w.dtype == "bf16" else 4) + 4 +
+                               w.d * (2 if w.dtype == "bf16" else 4))
+        sc_gbs = sc_bytes / (sc_ms * 1e-3) / 1e9
         phases = {
             "user_encode": {"ms": phase_ms["user"],
                             "history_tokens_per_s": total_hist / (phase_ms["user"] * 1e-3),
-                            "roofline": phase_roof("user")},
+                            "roofline": ur},
             "qk_cache": {"ms": phase_ms["cache"],
                          "items_per_s": w.n_items / (phase_ms["cache"] * 1e-3),
                          "roofline": phase_roof("cache")},
             "score": {"ms": phase_ms["score"],
                       "pairs_per_s": total_cand / (phase_ms["score"] * 1e-3),
                       "roofline": phase_roof("score")},
+            "score_at_scale": {"ms": sc_ms, "pairs": sc_pairs,
+                               "pairs_per_s": sc_pairs / (sc_ms * 1e-3),
+                               "ids": f"uniform over {w.n_items} items, L2 flushed before each call",
+                               "roofline": {"bound": "hbm", "achieved": sc_gbs,
+                                            "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                            "frac": sc_gbs / pk["hbm_gbs"]}},
         }
         line = {"metric": "user-candidate pairs scored/s (full LIME step)", "value": value,
                 "unit": "pairs/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -11,13 +11,14 @@
 // kernel stays bound by the gather.
 //
 // CTA (u, g) stages L^P_u^T once (a [128 c x 64 k] 128B-swizzled block, k >= l
-// zero) and walks tiles g, g + G, ... of user u's candidates.  Per tile each
-// thread gathers one candidate's row with 16-byte loads into the swizzled A
-// tile (an out-of-range ID gives a zero row and LIME_FLAG_BAD_ID) — the
-// threads of a warp cover whole rows, so the gather is coalesced — thread 0
-// issues one MMA group per head into TMEM, each thread stages its row of O in
-// bf16, and the tile is written back with coalesced 16-byte stores.  No
-// workspace is used.
+// zero) and walks tiles g, g + G, ... of user u's candidates.  The rows of
+// tile t+G are gathered with asynchronous 16-byte copies (cp.async) into the
+// second of two stages while tile t is multiplied and written, and the IDs of
+// tile t+2G are read meanwhile.  A warp's copies cover whole cache rows, so
+// the gather is coalesced; an out-of-range ID gives a zero row and
+// LIME_FLAG_BAD_ID.  Thread 0 issues one MMA group per head into TMEM, each
+// thread stages its row of O in bf16, and the tile is written back with
+// coalesced 16-byte stores.  No workspace is used.
 #include "lime_fast.cuh"
 #include "sm100.cuh"
 
@@ -39,14 +40,16 @@ __global__ void __launch_bounds__(128)
   // A tile blocks of 64 columns; at least 2 because the same region later
   // stages the [128 x 128] output tile
   constexpr int ABLK = HL / 64 < 2 ? 2 : HL / 64;
+  constexpr uint32_t kStage = ABLK * kBlk;
+  constexpr int CH = HL / 8;                 // 16-byte chunks per cache row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = sm;
-  uint8_t* sB = sm + ABLK * kBlk;
+  uint8_t* sA0 = sm;                         // 2 stages: gathered rows, then output staging
+  uint8_t* sB = sm + 2 * kStage;
   uint64_t* bar = reinterpret_cast<uint64_t*>(sB + kBlk);
   uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 1);
   int* abort_flag = reinterpret_cast<int*>(bar + 2);
-  int64_t* s_ids = reinterpret_cast<int64_t*>(bar + 4);   // [128] candidate IDs of the tile
+  int64_t* s_ids = reinterpret_cast<int64_t*>(bar + 4);   // [2][128] candidate IDs per stage
 
   pdl_wait();
   const int64_t u = blockIdx.x;
@@ -64,23 +67,54 @@ __global__ void __launch_bounds__(128)
   if (i < 32) tmem_alloc(slot, 128);
   __syncthreads();
   pdl_launch();   // after the TMEM allocation (the next kernel may allocate before it waits)
-  // The first tile's candidate ID is loaded together with L^P_u (one memory
-  // round trip for both).
-  int32_t first_id = -1;
-  if ((int64_t)i < b - (a + (int64_t)blockIdx.y * kTile)) first_id = ids[a + (int64_t)blockIdx.y * kTile + i];
+  const int G = (int)gridDim.y;
+  // candidate ID of row i of tile t (kNoRow past the user's rows); loaded a
+  // tile ahead.  A staged ID of -1 means "zero row".
+  constexpr int64_t kNoRow = INT64_MIN;
+  auto load_id = [&](int t) -> int64_t {
+    const int64_t m = a + (int64_t)t * kTile + i;
+    return (t < nt && m < b) ? (int64_t)ids[m] : kNoRow;
+  };
+  auto put_id = [&](int stage, int64_t id) {
+    if (id == kNoRow) {
+      id = -1;
+    } else if (id < 0 || id >= n_items) {
+      raise_flag(status, LIME_FLAG_BAD_ID);
+      id = -1;
+    }
+    s_ids[stage * kTile + i] = id;
+  };
+  // gather of one tile into a stage: chunk q*128 + i is chunk (idx % CH) of
+  // row idx / CH, so a warp reads whole cache rows; bad or missing IDs give
+  // zero rows
+  auto gather = [&](int stage) {
+    uint8_t* sA = sA0 + stage * kStage;
+#pragma unroll
+    for (int q = 0; q < CH; ++q) {
+      const int idx = q * 128 + i, r = idx / CH, cc = idx % CH;
+      const int64_t id = s_ids[stage * kTile + r];
+      const bf16* src = cache + (id < 0 ? 0 : id * HL) + cc * 8;
+      cp_async16(sA + (cc >> 3) * kBlk + sw128_offset(r, (cc & 7) * 8), src, id >= 0);
+    }
+    cp_async_commit();
+  };
+  int64_t id_cur = load_id(blockIdx.y);
+  int64_t id_nxt = load_id(blockIdx.y + G);
   // L^P_u transposed into sB: element (c, k) at sw128_offset(c, k), k >= L zero.
-  // Coalesced 16-byte copies of L^P_u into the (still unused) A tile, then each
+  // Coalesced 16-byte copies of L^P_u into stage 1 (unused yet), then each
   // thread builds its own row c of the transpose with 16-byte swizzled stores.
   {
     const uint4* lp = reinterpret_cast<const uint4*>(LP + (u * L) * kD);
-    uint4* stage = reinterpret_cast<uint4*>(sA);   // [L][128] bf16, plain row-major
+    uint4* stage = reinterpret_cast<uint4*>(sA0 + kStage);   // [L][128] bf16, plain row-major
     uint4 lv[L * kD / 8 / 128];
 #pragma unroll
     for (int q = 0; q < L * kD / 8 / 128; ++q) lv[q] = __ldg(lp + q * 128 + i);
 #pragma unroll
     for (int q = 0; q < L * kD / 8 / 128; ++q) stage[q * 128 + i] = lv[q];
+    put_id(0, id_cur);
     __syncthreads();
-    const bf16* st = reinterpret_cast<const bf16*>(sA);
+    gather(0);       // the first tile's rows stream in while L^P is transposed
+    const bf16* st = reinterpret_cast<const bf16*>(sA0 + kStage);
 #pragma unroll
     for (int k8 = 0; k8 < 8; ++k8) {
       float f[8];
@@ -92,48 +126,27 @@ __global__ void __launch_bounds__(128)
       sw_st16(sB, kBlk, i, k8 * 8, pack8(f));
     }
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+  __syncthreads();   // stage 1 is free again
   const uint32_t tmem = *slot;
   const uint32_t ta = tmem + ((uint32_t)(i & ~31) << 16);
   uint32_t ph = 0;
-  for (int t = blockIdx.y; t < nt; t += gridDim.y) {
+  int it = 0;
+  for (int t = blockIdx.y; t < nt; t += G, ++it) {
+    const int cur = it & 1, nxt = cur ^ 1;
     const int64_t m0 = a + (int64_t)t * kTile;
     const int nv = b - m0 < kTile ? (int)(b - m0) : kTile;
-    {
-      int64_t id = -1;
-      if (i < nv) {
-        id = t == (int)blockIdx.y ? first_id : ids[m0 + i];
-        if (id < 0 || id >= n_items) {
-          raise_flag(status, LIME_FLAG_BAD_ID);
-          id = -1;
-        }
-      }
-      s_ids[i] = id;
+    const bool more = t + G < nt;
+    if (more) {
+      put_id(nxt, id_nxt);
+      __syncthreads();
+      gather(nxt);                  // tile t+G streams in during tile t
+      id_nxt = load_id(t + 2 * G);  // and the IDs of tile t+2G
     }
-    __syncthreads();
-    // cooperative gather: 16-byte chunk q*128 + i is chunk (idx % CH) of row idx / CH,
-    // so a warp reads whole cache rows (coalesced) instead of one row per thread
-    {
-      constexpr int CH = HL / 8;               // 16-byte chunks per cache row
-      uint4 v[CH];
-#pragma unroll
-      for (int q = 0; q < CH; ++q) {
-        const int idx = q * 128 + i, r = idx / CH, cc = idx % CH;
-        const int64_t id = s_ids[r];
-        v[q] = id < 0 ? make_uint4(0, 0, 0, 0)
-                      : __ldg(reinterpret_cast<const uint4*>(cache + id * HL) + cc);
-      }
-#pragma unroll
-      for (int q = 0; q < CH; ++q) {
-        const int idx = q * 128 + i, r = idx / CH, cc = idx % CH;
-        sw_st16(sA, kBlk, r, cc * 8, v[q]);
-      }
-    }
+    if (more) cp_async_wait<1>(); else cp_async_wait<0>();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    uint8_t* sA = sA0 + cur * kStage;
     if (i == 0) {
       tc_fence_after();
 #pragma unroll
@@ -163,7 +176,7 @@ __global__ void __launch_bounds__(128)
       if (r < nv)
         reinterpret_cast<uint4*>(O + (m0 + r) * kD)[cc] = sw_ld16(sA, kBlk, r, cc * 8);
     }
-    __syncthreads();   // sA, s_ids and TMEM are reused by the next tile
+    __syncthreads();   // this stage and TMEM are reused two tiles on
   }
   if (i < 32) {
     tc_fence_after();
@@ -176,7 +189,7 @@ int launch_score(int64_t B, const void* cache, int64_t n_items, const int32_t* i
                  const int64_t* off, int64_t total, const void* LP, void* O, unsigned* status,
                  cudaStream_t st) {
   constexpr int HL = kH * L;
-  const int smem = 1024 + ((HL / 64 < 2 ? 2 : HL / 64) + 1) * kBlk + 64 + 128 * 8;
+  const int smem = 1024 + (2 * (HL / 64 < 2 ? 2 : HL / 64) + 1) * kBlk + 64 + 2 * 128 * 8;
   if (cudaFuncSetAttribute(k_score_tc<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return LIME_ERR_CUDA;

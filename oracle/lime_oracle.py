@@ -40,6 +40,10 @@ notes of the library):
      values L^P with no projection, no output projection.
   R8 no positional term.  N_u = 0 gives the link branch a zero output; M_u = 0
      gives no output rows.
+  R14 int8 QK cache: the pages store each cached weight in one byte ("int8
+     lookup + dequant") without stating the encoding.  Softmax weights lie in
+     [0, 1], so the reading is unsigned 8-bit with the fixed scale 1/255:
+     q = round(255 w), half to even, dequantised as q / 255.
 """
 from __future__ import annotations
 
@@ -243,6 +247,32 @@ def score_candidates(cache: np.ndarray, cand_ids: np.ndarray,
             c = slice(h * dh, (h + 1) * dh)
             O[a:b, c] = W[:, h, :] @ LP[u, :, c]         # sum_k w_k L^P_k
     return O
+
+
+def quantize_cache_u8(cache: np.ndarray) -> np.ndarray:
+    """int8 QK cache: q = round(255 w) as uint8, ties to even (reading R14).
+
+    LIME listing Tables 9, 11 and 12: the production cache holds one byte per
+    (item, head, link) weight ("int8 lookup + dequant"; 12.8 GB for 100M items,
+    four heads and 32 links).
+    """
+    return np.clip(np.rint(255.0 * cache), 0, 255).astype(np.uint8)
+
+
+def dequantize_cache_u8(q: np.ndarray) -> np.ndarray:
+    """The weights an int8 cache stands for: q / 255 (reading R14)."""
+    return q.astype(np.float64) / 255.0
+
+
+def score_candidates_u8(q: np.ndarray, cand_ids: np.ndarray,
+                        cand_offsets: Sequence[int], LP: np.ndarray,
+                        users: Optional[Sequence[int]] = None) -> np.ndarray:
+    """Cached scoring from an int8 cache: O_m = sum_k (q_k / 255) L^P_k.
+
+    LIME listing Table 9 ("Int8 lookup+dequant", "Int8 total"): the bytes are
+    dequantised on lookup and then aggregated exactly as in score_candidates.
+    """
+    return score_candidates(dequantize_cache_u8(q), cand_ids, cand_offsets, LP, users)
 
 
 def candidate_attention_uncached(T_rows: np.ndarray, L: np.ndarray,

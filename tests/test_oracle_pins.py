@@ -306,3 +306,52 @@ def test_scoring_edge_cases():
     np.testing.assert_array_equal(out[3], 0.0)
     np.testing.assert_allclose(out[4, :4], cache[9, 0] @ LP[1, :, :4], atol=1e-15)
     np.testing.assert_allclose(out[4, 4:], cache[9, 1] @ LP[1, :, 4:], atol=1e-15)
+
+
+# ------------------------------------------------------------ int8 QK cache
+
+def test_u8_quantize_rounds_half_to_even_and_saturates():
+    # hand values: 255 w = 0.5 -> 0, 1.5 -> 2, 2.5 -> 2, 254.6 -> 255, w = 1 -> 255
+    w = np.array([0.5, 1.5, 2.5, 3.49, 254.6, 255.0]) / 255.0
+    assert O.quantize_cache_u8(w).tolist() == [0, 2, 2, 3, 255, 255]
+    assert O.quantize_cache_u8(np.array([0.0, 1.0, 1.2])).tolist() == [0, 255, 255]
+
+
+def test_u8_cache_error_is_within_half_a_step():
+    g = np.random.default_rng(5)
+    T, L = g.normal(size=(300, 64)), g.normal(size=(16, 64))
+    Wq, Wk = g.normal(size=(64, 64)) / 8, g.normal(size=(64, 64)) / 8
+    w = O.qk_cache(T, L, Wq, Wk, 2)
+    q = O.quantize_cache_u8(w)
+    assert q.dtype == np.uint8 and q.shape == w.shape
+    err = np.abs(O.dequantize_cache_u8(q) - w)
+    assert err.max() <= 0.5 / 255 + 1e-15
+    # one link: every weight is exactly 1 and quantises to 255 exactly
+    w1 = O.qk_cache(T, L[:1], Wq, Wk, 2)
+    assert (O.quantize_cache_u8(w1) == 255).all()
+
+
+def test_u8_scoring_worked_example():
+    # the pages' worked example with the weights stored as bytes:
+    # 0.42 -> round(107.1) = 107, 0.35 -> round(89.25) = 89
+    l, d, H = 32, 8, 1
+    g = np.random.default_rng(9)
+    LP = g.normal(size=(1, l, d))
+    cache = np.zeros((3, H, l))
+    cache[1, 0, 29], cache[1, 0, 1] = 0.42, 0.35
+    q = O.quantize_cache_u8(cache)
+    assert q[1, 0, 29] == 107 and q[1, 0, 1] == 89
+    out = O.score_candidates_u8(q, np.array([1]), [0, 1], LP)
+    np.testing.assert_allclose(out[0], (107 * LP[0, 29] + 89 * LP[0, 1]) / 255, rtol=0, atol=1e-14)
+
+
+def test_u8_scoring_with_identity_values_returns_the_dequantised_row():
+    # d_h = l and every head slice of L^P the identity: O[m, h*l + k] = q / 255
+    l, H = 16, 2
+    LP = np.zeros((1, l, H * l))
+    for h in range(H):
+        LP[0, :, h * l:(h + 1) * l] = np.eye(l)
+    q = np.random.default_rng(2).integers(0, 256, size=(7, H, l)).astype(np.uint8)
+    ids = np.array([6, 0, 3, 3])
+    out = O.score_candidates_u8(q, ids, [0, 4], LP)
+    np.testing.assert_array_equal(out, q[ids].reshape(4, H * l) / 255.0)

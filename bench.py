@@ -392,6 +392,31 @@ def main():
     torch.cuda.synchronize()
     sc_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in sc_ev)], dist,
                            "cuda")[0] / args.steps
+
+    # The int8 cache variant (one byte per weight): its build over the whole
+    # catalogue and the same scoring at scale from it.
+    u8 = None
+    if w.dtype == "bf16" and w.H * w.l >= 128:
+        q8 = torch.empty(w.n_items, w.H, w.l, dtype=torch.uint8, device="cuda")
+        u8_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        for _ in range(3):
+            lime.lime_build_qk_cache_u8(x.dims, x.T, x.L, x.Wq_c, x.Wk_c, q8, buf.ws)
+            lime.lime_score_candidates_u8(x.dims, q8, sc_ids, sc_off, sc_users * sc_per, sc_LP,
+                                          sc_O, buf.ws)
+        for k in range(args.steps):
+            flush.zero_()
+            u8_ev[k][0].record(stream)
+            lime.lime_build_qk_cache_u8(x.dims, x.T, x.L, x.Wq_c, x.Wk_c, q8, buf.ws)
+            u8_ev[k][1].record(stream)
+            flush.zero_()
+            u8_ev[k][2].record(stream)
+            lime.lime_score_candidates_u8(x.dims, q8, sc_ids, sc_off, sc_users * sc_per, sc_LP,
+                                          sc_O, buf.ws)
+            u8_ev[k][3].record(stream)
+        torch.cuda.synchronize()
+        u8 = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in u8_ev),
+                             sum(e[2].elapsed_time(e[3]) for e in u8_ev)], dist, "cuda")
+        u8 = [v / args.steps for v in u8]
     if lime.lime_get_status(buf.ws) != 0:
         raise RuntimeError("device status flags set during the timed steps")
 
@@ -446,6 +471,21 @@ def main():
                                             "peak": pk["hbm_gbs"], "unit": "GB/s",
                                             "frac": sc_gbs / pk["hbm_gbs"]}},
         }
+        if u8 is not None:
+            c8_bytes = w.n_items * (2 * w.d + w.H * w.l)
+            s8_bytes = sc_pairs * (w.H * w.l + 4 + 2 * w.d)
+            c8_gbs = c8_bytes / (u8[0] * 1e-3) / 1e9
+            s8_gbs = s8_bytes / (u8[1] * 1e-3) / 1e9
+            phases["qk_cache_u8"] = {
+                "ms": u8[0], "items_per_s": w.n_items / (u8[0] * 1e-3),
+                "note": "int8 cache variant (one byte per weight); includes the fold prologue",
+                "roofline": {"bound": "hbm", "achieved": c8_gbs, "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "frac": c8_gbs / pk["hbm_gbs"]}}
+            phases["score_u8_at_scale"] = {
+                "ms": u8[1], "pairs": sc_pairs, "pairs_per_s": sc_pairs / (u8[1] * 1e-3),
+                "ids": f"uniform over {w.n_items} items, L2 flushed before each call",
+                "roofline": {"bound": "hbm", "achieved": s8_gbs, "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "frac": s8_gbs / pk["hbm_gbs"]}}
         line = {"metric": "user-candidate pairs scored/s (full LIME step)", "value": value,
                 "unit": "pairs/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",

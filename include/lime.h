@@ -184,6 +184,31 @@ int lime_score_candidates(const lime_dims* dims, int64_t B, const void* cache,
                           const void* LP, void* O_out, void* workspace,
                           size_t workspace_bytes, cudaStream_t stream);
 
+/* int8 QK cache (LIME listing Tables 9, 11, 12: one byte per cached weight,
+ * "int8 lookup + dequant"; the encoding is not stated by the pages).  Byte
+ * q[m, h, k] = round(255 * w[m, h, k]) with w the lime_build_qk_cache
+ * weight computed in fp32 (ties to even; w lies in [0, 1]); dequantised as
+ * q / 255.  Same arguments, checks and errors as lime_build_qk_cache, with
+ *   cache_out device uint8 [n_items, H, l] (16-byte aligned).
+ * Supported: bf16, d = 128, H*l >= 128 (else LIME_ERR_SHAPE).            */
+int lime_build_qk_cache_u8(const lime_dims* dims, const void* T, int64_t n_items,
+                           const void* L, const void* Wq_c, const void* Wk_c,
+                           uint8_t* cache_out, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
+/* Cached scoring from an int8 cache: O[m, h-cols] = sum_k (q[id_m, h, k] / 255)
+ * L^P_u[k, h-cols].  Same arguments, checks and errors as
+ * lime_score_candidates, with cache a device uint8 [n_items, H, l] array
+ * (16-byte aligned).  The product runs in fp16 (the bytes are exact; L^P is
+ * converted exactly for 6.1e-5 <= |x| <= 65504, smaller magnitudes keep an
+ * absolute error below 3e-8; larger ones overflow).  Supported: bf16,
+ * d = 128, H = 4, l in {32, 64} (else LIME_ERR_SHAPE).                     */
+int lime_score_candidates_u8(const lime_dims* dims, int64_t B, const uint8_t* cache,
+                             int64_t n_items, const int32_t* cand_ids,
+                             const int64_t* cand_offsets, int64_t total_cand,
+                             const void* LP, void* O_out, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream);
+
 /* Synchronises stream, copies the sticky LIME_FLAG_* word to *flags and
  * clears it. */
 int lime_get_status(void* workspace, cudaStream_t stream, int* flags);

@@ -31,13 +31,15 @@ namespace {
 constexpr int kD = 128;    // model dim handled here
 constexpr int kBM = 128;   // catalogue rows per tile
 
-template <int HL, int L>
+// U8: the cache is stored as bytes q = round(255 w) (an int8 cache).
+template <int HL, int L, bool U8>
 struct CacheCfg {
   static constexpr int STAGES = HL <= 128 ? 4 : 3;
-  static constexpr int OUTB = HL <= 128 ? 2 : 1;
+  static constexpr int OUTB = HL <= 128 || U8 ? 2 : 1;
   static constexpr int A_BYTES = kBM * kD * 2;      // one T tile
   static constexpr int B_BYTES = HL * kD * 2;       // the G^T image
-  static constexpr int O_BYTES = kBM * HL * 2;      // one output tile
+  static constexpr int ROW_BYTES = HL * (U8 ? 1 : 2);   // one cache row
+  static constexpr int O_BYTES = kBM * ROW_BYTES;   // one output tile
   static constexpr int TMEM_COLS = 2 * HL;
   static constexpr int OFF_B = STAGES * A_BYTES;
   static constexpr int OFF_O = OFF_B + B_BYTES;
@@ -118,11 +120,11 @@ __global__ void __launch_bounds__(128) k_fold_g_img(const bf16* __restrict__ L,
   }
 }
 
-template <int HL, int L>
-__global__ void __launch_bounds__(CacheCfg<HL, L>::THREADS, 1)
+template <int HL, int L, bool U8>
+__global__ void __launch_bounds__(CacheCfg<HL, L, U8>::THREADS, 1)
     k_cache_tc(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmC,
                const bf16* __restrict__ gimg, int n_tiles, unsigned* status) {
-  using C = CacheCfg<HL, L>;
+  using C = CacheCfg<HL, L, U8>;
   constexpr int H = HL / L;
   constexpr uint32_t IDESC = idesc_bf16(kBM, HL);
   extern __shared__ uint8_t smem_raw[];
@@ -249,15 +251,41 @@ __global__ void __launch_bounds__(CacheCfg<HL, L>::THREADS, 1)
           ssum += z[k];
         }
         const float inv = 1.0f / ssum;
+        if constexpr (U8) {
+          // bytes q = round(255 w), ties to even; 16 per 16-byte chunk of the
+          // row's 128-byte swizzled block
+          const float sc = inv * 255.0f;
 #pragma unroll
-        for (int c = 0; c < L / 8; ++c) {
-          const int col = h * L + c * 8;
-          uint4 v;
-          v.x = pack_bf16(z[c * 8 + 0] * inv, z[c * 8 + 1] * inv);
-          v.y = pack_bf16(z[c * 8 + 2] * inv, z[c * 8 + 3] * inv);
-          v.z = pack_bf16(z[c * 8 + 4] * inv, z[c * 8 + 5] * inv);
-          v.w = pack_bf16(z[c * 8 + 6] * inv, z[c * 8 + 7] * inv);
-          *reinterpret_cast<uint4*>(stage + (col >> 6) * (kBM * 128) + sw128_offset(row, col & 63)) = v;
+          for (int c = 0; c < L / 16; ++c) {
+            const int bcol = h * L + c * 16;
+            // z <= 1 and sum >= 1, so 255 z / sum rounds to at most 255.  Adding
+            // 1.5 * 2^23 in the same FMA rounds the product to an integer (ties
+            // to even) in the low mantissa bits: the low byte is q.
+            uint32_t wv[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float* zz = z + c * 16 + j * 4;
+              const uint32_t q0 = __float_as_uint(fmaf(zz[0], sc, 12582912.0f));
+              const uint32_t q1 = __float_as_uint(fmaf(zz[1], sc, 12582912.0f));
+              const uint32_t q2 = __float_as_uint(fmaf(zz[2], sc, 12582912.0f));
+              const uint32_t q3 = __float_as_uint(fmaf(zz[3], sc, 12582912.0f));
+              wv[j] = __byte_perm(__byte_perm(q0, q1, 0x0040), __byte_perm(q2, q3, 0x0040), 0x5410);
+            }
+            *reinterpret_cast<uint4*>(stage + (bcol >> 7) * (kBM * 128) + row * 128 +
+                                      ((((bcol & 127) >> 4) ^ (row & 7)) << 4)) =
+                make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < L / 8; ++c) {
+            const int col = h * L + c * 8;
+            uint4 v;
+            v.x = pack_bf16(z[c * 8 + 0] * inv, z[c * 8 + 1] * inv);
+            v.y = pack_bf16(z[c * 8 + 2] * inv, z[c * 8 + 3] * inv);
+            v.z = pack_bf16(z[c * 8 + 4] * inv, z[c * 8 + 5] * inv);
+            v.w = pack_bf16(z[c * 8 + 6] * inv, z[c * 8 + 7] * inv);
+            *reinterpret_cast<uint4*>(stage + (col >> 6) * (kBM * 128) + sw128_offset(row, col & 63)) = v;
+          }
         }
       }
       tc_fence_before();
@@ -266,8 +294,11 @@ __global__ void __launch_bounds__(CacheCfg<HL, L>::THREADS, 1)
       mbar_arrive(&ofull[ob]);
       if (et == 0) {
         if (!mbar_wait(&ofull[ob], oph, status, &abort_flag)) break;
+        // 128-byte-wide boxes: 64 bf16 or 128 bytes of the cache row
+        constexpr int per_box = U8 ? 128 : 64;
 #pragma unroll
-        for (int b = 0; b < HL / 64; ++b) tma_store_2d(&tmC, stage + b * (kBM * 128), b * 64, tile * kBM);
+        for (int b = 0; b < HL / per_box; ++b)
+          tma_store_2d(&tmC, stage + b * (kBM * 128), b * per_box, tile * kBM);
         bulk_commit();
         // the store issued OUTB-1 tiles ago has finished reading its buffer
         bulk_wait_read<C::OUTB - 1>();
@@ -288,20 +319,24 @@ __global__ void __launch_bounds__(CacheCfg<HL, L>::THREADS, 1)
   }
 }
 
-template <int HL, int L>
+template <int HL, int L, bool U8>
 int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, unsigned* status,
                  cudaStream_t st) {
-  using C = CacheCfg<HL, L>;
+  using C = CacheCfg<HL, L, U8>;
   CUtensorMap tmT, tmC;
   if (!make_tmap_2d_bf16(&tmT, T, kD, (uint64_t)n, kD * 2, 64, kBM)) return LIME_ERR_CUDA;
-  if (!make_tmap_2d_bf16(&tmC, cache, HL, (uint64_t)n, HL * 2, 64, kBM)) return LIME_ERR_CUDA;
-  if (cudaFuncSetAttribute(k_cache_tc<HL, L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (U8) {
+    if (!make_tmap_2d_u8(&tmC, cache, HL, (uint64_t)n, HL, 128, kBM)) return LIME_ERR_CUDA;
+  } else if (!make_tmap_2d_bf16(&tmC, cache, HL, (uint64_t)n, HL * 2, 64, kBM)) {
+    return LIME_ERR_CUDA;
+  }
+  if (cudaFuncSetAttribute(k_cache_tc<HL, L, U8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::SMEM) != cudaSuccess)
     return LIME_ERR_CUDA;
   const int n_tiles = (int)((n + kBM - 1) / kBM);
   const int grid = n_tiles < num_sms() ? n_tiles : num_sms();
-  return launch_pdl(k_cache_tc<HL, L>, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, tmT, tmC, img,
-                    n_tiles, status);
+  return launch_pdl(k_cache_tc<HL, L, U8>, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, tmT, tmC,
+                    img, n_tiles, status);
 }
 
 }  // namespace
@@ -316,9 +351,14 @@ bool fast_cache_supported(const lime_dims& D) {
   return HL == 64 || HL == 128 || HL == 256;
 }
 
-int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void* L,
-                        const void* Wq, const void* Wk, void* cache, float* ws, unsigned* status,
-                        cudaStream_t st) {
+bool fast_cache_u8_supported(const lime_dims& D) {
+  return fast_cache_supported(D) && D.H * D.l >= 128;
+}
+
+namespace {
+int build_cache(const lime_dims& D, const void* T, int64_t n, const void* L, const void* Wq,
+                const void* Wk, void* cache, bool u8, float* ws, unsigned* status,
+                cudaStream_t st) {
   const int HL = D.H * D.l;
   bf16* img = reinterpret_cast<bf16*>(ws);
   const float scale = 1.0f / sqrtf((float)(D.d / D.H));
@@ -326,16 +366,34 @@ int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void
                       (const bf16*)Wq, (const bf16*)Wk, D.H, D.l, scale, img);
   if (rc) return rc;
   if (n == 0) return LIME_OK;
-  switch (HL * 1000 + D.l) {
-    case 64016: return launch_cache<64, 16>(T, n, img, cache, status, st);
-    case 64032: return launch_cache<64, 32>(T, n, img, cache, status, st);
-    case 128016: return launch_cache<128, 16>(T, n, img, cache, status, st);
-    case 128032: return launch_cache<128, 32>(T, n, img, cache, status, st);
-    case 128064: return launch_cache<128, 64>(T, n, img, cache, status, st);
-    case 256032: return launch_cache<256, 32>(T, n, img, cache, status, st);
-    case 256064: return launch_cache<256, 64>(T, n, img, cache, status, st);
+  switch (HL * 1000 + D.l + (u8 ? 1000000 : 0)) {
+    case 64016: return launch_cache<64, 16, false>(T, n, img, cache, status, st);
+    case 64032: return launch_cache<64, 32, false>(T, n, img, cache, status, st);
+    case 128016: return launch_cache<128, 16, false>(T, n, img, cache, status, st);
+    case 128032: return launch_cache<128, 32, false>(T, n, img, cache, status, st);
+    case 128064: return launch_cache<128, 64, false>(T, n, img, cache, status, st);
+    case 256032: return launch_cache<256, 32, false>(T, n, img, cache, status, st);
+    case 256064: return launch_cache<256, 64, false>(T, n, img, cache, status, st);
+    case 1128016: return launch_cache<128, 16, true>(T, n, img, cache, status, st);
+    case 1128032: return launch_cache<128, 32, true>(T, n, img, cache, status, st);
+    case 1128064: return launch_cache<128, 64, true>(T, n, img, cache, status, st);
+    case 1256032: return launch_cache<256, 32, true>(T, n, img, cache, status, st);
+    case 1256064: return launch_cache<256, 64, true>(T, n, img, cache, status, st);
     default: return LIME_ERR_SHAPE;
   }
+}
+}  // namespace
+
+int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void* L,
+                        const void* Wq, const void* Wk, void* cache, float* ws,
+                        unsigned* status, cudaStream_t st) {
+  return build_cache(D, T, n, L, Wq, Wk, cache, false, ws, status, st);
+}
+
+int fast_build_qk_cache_u8(const lime_dims& D, const void* T, int64_t n, const void* L,
+                           const void* Wq, const void* Wk, void* cache, float* ws,
+                           unsigned* status, cudaStream_t st) {
+  return build_cache(D, T, n, L, Wq, Wk, cache, true, ws, status, st);
 }
 
 }  // namespace lime

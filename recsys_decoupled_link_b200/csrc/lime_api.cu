@@ -222,6 +222,60 @@ int lime_score_candidates(const lime_dims* dims, int64_t B, const void* cache, i
   return launch_status("lime_score_candidates");
 }
 
+int lime_build_qk_cache_u8(const lime_dims* dims, const void* T, int64_t n_items, const void* L,
+                           const void* Wq_c, const void* Wk_c, uint8_t* cache_out,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!fast_cache_u8_supported(*dims)) return LIME_ERR_SHAPE;
+  if (n_items < 0 || n_items > (int64_t)INT32_MAX + 1) return LIME_ERR_ARG;
+  if (!L || !Wq_c || !Wk_c || (n_items > 0 && (!T || !cache_out))) return LIME_ERR_ARG;
+  if ((n_items > 0 && (!aligned16(T) || !aligned16(cache_out))) || !aligned16(L) ||
+      !aligned16(Wq_c) || !aligned16(Wk_c))
+    return LIME_ERR_ARG;
+  if ((rc = check_ws(workspace, workspace_bytes, dims, 0, 0))) return rc;
+  const size_t es = esize(dims);
+  const size_t cache_sz = (size_t)n_items * dims->H * dims->l;
+  if (overlap(cache_out, cache_sz, T, (size_t)n_items * dims->d * es) ||
+      overlap(cache_out, cache_sz, L, (size_t)dims->l * dims->d * es) ||
+      overlap(cache_out, cache_sz, Wq_c, (size_t)dims->d * dims->d * es) ||
+      overlap(cache_out, cache_sz, Wk_c, (size_t)dims->d * dims->d * es))
+    return LIME_ERR_ALIAS;
+  if ((rc = fast_build_qk_cache_u8(*dims, T, n_items, L, Wq_c, Wk_c, cache_out,
+                                   scratch_of(workspace), status_of(workspace), stream)))
+    return rc;
+  return launch_status("lime_build_qk_cache_u8");
+}
+
+int lime_score_candidates_u8(const lime_dims* dims, int64_t B, const uint8_t* cache,
+                             int64_t n_items, const int32_t* cand_ids,
+                             const int64_t* cand_offsets, int64_t total_cand, const void* LP,
+                             void* O_out, void* workspace, size_t workspace_bytes,
+                             cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!fast_score_u8_supported(*dims)) return LIME_ERR_SHAPE;
+  if (B < 0 || B > INT32_MAX || n_items < 0 || total_cand < 0) return LIME_ERR_ARG;
+  if (B == 0) return total_cand == 0 ? LIME_OK : LIME_ERR_ARG;
+  if (!cand_offsets || !LP || ((uintptr_t)cand_offsets & 7)) return LIME_ERR_ARG;
+  if (total_cand > 0 && (!cand_ids || !O_out || !cache)) return LIME_ERR_ARG;
+  if (!aligned16(LP) || (O_out && !aligned16(O_out)) || (cache && !aligned16(cache)) ||
+      ((uintptr_t)cand_ids & 3))
+    return LIME_ERR_ARG;
+  if ((rc = check_ws(workspace, workspace_bytes, dims, 0, 0))) return rc;
+  const size_t es = esize(dims);
+  const size_t o_sz = (size_t)total_cand * dims->d * es;
+  if (overlap(O_out, o_sz, cache, (size_t)n_items * dims->H * dims->l) ||
+      overlap(O_out, o_sz, LP, (size_t)B * dims->l * dims->d * es) ||
+      overlap(O_out, o_sz, cand_ids, (size_t)total_cand * 4))
+    return LIME_ERR_ALIAS;
+  if (total_cand == 0) return LIME_OK;
+  if ((rc = fast_score_u8(*dims, B, cache, n_items, cand_ids, cand_offsets, total_cand, LP, O_out,
+                          status_of(workspace), stream)))
+    return rc;
+  return launch_status("lime_score_candidates_u8");
+}
+
 int lime_get_status(void* workspace, cudaStream_t stream, int* flags) {
   if (!workspace || !flags || ((uintptr_t)workspace & 255)) return LIME_ERR_ARG;
   unsigned v = 0;

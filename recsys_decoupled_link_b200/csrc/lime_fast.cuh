@@ -43,6 +43,12 @@ int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void
                         const void* Wq, const void* Wk, void* cache, float* ws,
                         unsigned* status, cudaStream_t st);
 
+// int8 cache (bytes q = round(255 w)); needs H*l >= 128
+bool fast_cache_u8_supported(const lime_dims& D);
+int fast_build_qk_cache_u8(const lime_dims& D, const void* T, int64_t n, const void* L,
+                           const void* Wq, const void* Wk, void* cache, float* ws,
+                           unsigned* status, cudaStream_t st);
+
 bool fast_score_supported(const lime_dims& D);
 int fast_score(const lime_dims& D, int64_t B, const void* cache, int64_t n_items,
                const int32_t* ids, const int64_t* off, int64_t total, const void* LP, void* O,
@@ -51,6 +57,11 @@ int fast_score(const lime_dims& D, int64_t B, const void* cache, int64_t n_items
 bool fast_ctx_supported(const lime_dims& D);
 int fast_context_links(const lime_dims& D, int64_t B, const void* L, const void* ctx,
                        const lime_ctx_mlp& w, void* LC, unsigned* status, cudaStream_t st);
+
+bool fast_score_u8_supported(const lime_dims& D);
+int fast_score_u8(const lime_dims& D, int64_t B, const uint8_t* cache, int64_t n_items,
+                  const int32_t* ids, const int64_t* off, int64_t total, const void* LP, void* O,
+                  unsigned* status, cudaStream_t st);
 
 bool fast_layer_supported(const lime_dims& D);
 int fast_xor_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh,

@@ -31,21 +31,39 @@ namespace {
 constexpr int kD = 128, kH = 4, kDH = 32, kTile = 128;
 constexpr uint32_t kBlk = 128 * 128;
 
-template <int L>
-__global__ void __launch_bounds__(128)
-    k_score_tc(const bf16* __restrict__ cache, int64_t n_items, const int32_t* __restrict__ ids,
-               const int64_t* __restrict__ off, int64_t B, int64_t total,
-               const bf16* __restrict__ LP, bf16* __restrict__ O, unsigned* status) {
-  constexpr int HL = kH * L;
+// Shared memory of k_score_tc<L, U8>: bf16 cache = two A stages (the gather
+// lands in the MMA operand directly); int8 cache = one A tile plus two byte
+// stages (the gather lands in a byte stage, which is widened into A).
+template <int L, bool U8>
+struct ScoreCfg {
+  static constexpr int HL = kH * L;
   // A tile blocks of 64 columns; at least 2 because the same region later
   // stages the [128 x 128] output tile
-  constexpr int ABLK = HL / 64 < 2 ? 2 : HL / 64;
-  constexpr uint32_t kStage = ABLK * kBlk;
-  constexpr int CH = HL / 8;                 // 16-byte chunks per cache row
+  static constexpr int ABLK = HL / 64 < 2 ? 2 : HL / 64;
+  static constexpr uint32_t kA = ABLK * kBlk;
+  static constexpr int RB = U8 ? HL : 2 * HL;          // bytes per cache row
+  static constexpr uint32_t kG = U8 ? 128u * RB : kA;  // one gather stage
+  static constexpr uint32_t OFF_G = U8 ? kA : 0;
+  static constexpr uint32_t OFF_B = OFF_G + 2 * kG;
+  static constexpr int SMEM = 1024 + OFF_B + kBlk + 64 + 2 * 128 * 8;
+};
+
+template <int L, bool U8>
+__global__ void __launch_bounds__(128)
+    k_score_tc(const void* __restrict__ cache_v, int64_t n_items, const int32_t* __restrict__ ids,
+               const int64_t* __restrict__ off, int64_t B, int64_t total,
+               const bf16* __restrict__ LP, bf16* __restrict__ O, unsigned* status) {
+  using C = ScoreCfg<L, U8>;
+  constexpr int HL = C::HL;
+  constexpr uint32_t kStage = C::kG;
+  constexpr int CH = C::RB / 16;             // 16-byte chunks per cache row
+  constexpr int kSw = CH >= 8 ? 7 : CH - 1;  // XOR swizzle of the byte stages
+  const uint8_t* cache = reinterpret_cast<const uint8_t*>(cache_v);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA0 = sm;                         // 2 stages: gathered rows, then output staging
-  uint8_t* sB = sm + 2 * kStage;
+  uint8_t* sA0 = sm + C::OFF_G;              // 2 gather stages
+  uint8_t* sAu = sm;                         // int8 cache: the widened A tile
+  uint8_t* sB = sm + C::OFF_B;
   uint64_t* bar = reinterpret_cast<uint64_t*>(sB + kBlk);
   uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 1);
   int* abort_flag = reinterpret_cast<int*>(bar + 2);
@@ -86,15 +104,18 @@ __global__ void __launch_bounds__(128)
   };
   // gather of one tile into a stage: chunk q*128 + i is chunk (idx % CH) of
   // row idx / CH, so a warp reads whole cache rows; bad or missing IDs give
-  // zero rows
+  // zero rows.  bf16 rows land in the swizzled MMA operand; byte rows in a
+  // [128 x RB] stage with chunk c of row r at r*RB + ((c ^ (r & kSw)) * 16).
   auto gather = [&](int stage) {
-    uint8_t* sA = sA0 + stage * kStage;
+    uint8_t* sG = sA0 + stage * kStage;
 #pragma unroll
     for (int q = 0; q < CH; ++q) {
       const int idx = q * 128 + i, r = idx / CH, cc = idx % CH;
       const int64_t id = s_ids[stage * kTile + r];
-      const bf16* src = cache + (id < 0 ? 0 : id * HL) + cc * 8;
-      cp_async16(sA + (cc >> 3) * kBlk + sw128_offset(r, (cc & 7) * 8), src, id >= 0);
+      const uint8_t* src = cache + (id < 0 ? 0 : id * C::RB) + cc * 16;
+      uint8_t* dst = U8 ? sG + r * C::RB + ((cc ^ (r & kSw)) << 4)
+                        : sG + (cc >> 3) * kBlk + sw128_offset(r, (cc & 7) * 8);
+      cp_async16(dst, src, id >= 0);
     }
     cp_async_commit();
   };
@@ -105,7 +126,7 @@ __global__ void __launch_bounds__(128)
   // thread builds its own row c of the transpose with 16-byte swizzled stores.
   {
     const uint4* lp = reinterpret_cast<const uint4*>(LP + (u * L) * kD);
-    uint4* stage = reinterpret_cast<uint4*>(sA0 + kStage);   // [L][128] bf16, plain row-major
+    uint4* stage = reinterpret_cast<uint4*>(sA0 + kStage);   // [L][128] bf16 in gather stage 1
     uint4 lv[L * kD / 8 / 128];
 #pragma unroll
     for (int q = 0; q < L * kD / 8 / 128; ++q) lv[q] = __ldg(lp + q * 128 + i);
@@ -123,7 +144,8 @@ __global__ void __launch_bounds__(128)
         const int k = k8 * 8 + z;
         f[z] = k < L ? __bfloat162float(st[k * kD + i]) : 0.f;
       }
-      sw_st16(sB, kBlk, i, k8 * 8, pack8(f));
+      // int8 cache: fp16 operands (A holds the bytes exactly, L^P converts exactly)
+      sw_st16(sB, kBlk, i, k8 * 8, U8 ? pack8_f16(f) : pack8(f));
     }
   }
   __syncthreads();   // stage 1 is free again
@@ -143,16 +165,44 @@ __global__ void __launch_bounds__(128)
       id_nxt = load_id(t + 2 * G);  // and the IDs of tile t+2G
     }
     if (more) cp_async_wait<1>(); else cp_async_wait<0>();
+    uint8_t* sA = sA0 + cur * kStage;
+    if constexpr (U8) {
+      // widen this thread's row of bytes into the fp16 operand, exactly: the
+      // half with bits 0x64 | b is 1024 + b, minus 1024 gives b
+      __syncthreads();
+      const uint8_t* sG = sA0 + cur * kStage;
+      const __half2 k1024 = __float2half2_rn(1024.0f);
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(sG + i * C::RB + ((c ^ (i & kSw)) << 4));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t lo = __byte_perm(w[j], 0x64646464u, 0x4140);
+          uint32_t hi = __byte_perm(w[j], 0x64646464u, 0x4342);
+          __half2 l2 = __hsub2(*reinterpret_cast<__half2*>(&lo), k1024);
+          __half2 h2 = __hsub2(*reinterpret_cast<__half2*>(&hi), k1024);
+          h[2 * j] = *reinterpret_cast<uint32_t*>(&l2);
+          h[2 * j + 1] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+        sw_st16(sAu, kBlk, i, c * 16, make_uint4(h[0], h[1], h[2], h[3]));
+        sw_st16(sAu, kBlk, i, c * 16 + 8, make_uint4(h[4], h[5], h[6], h[7]));
+      }
+      sA = sAu;
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    uint8_t* sA = sA0 + cur * kStage;
     if (i == 0) {
       tc_fence_after();
 #pragma unroll
-      for (int h = 0; h < kH; ++h)
-        mma_tile(tmem + h * kDH, smem_u32(sA + ((h * L) >> 6) * kBlk + ((h * L) & 63) * 2), kBlk,
-                 smem_u32(sB + h * kDH * 128), kBlk, kDH, L, false);
+      for (int h = 0; h < kH; ++h) {
+        const uint32_t a = smem_u32(sA + ((h * L) >> 6) * kBlk + ((h * L) & 63) * 2);
+        const uint32_t bb = smem_u32(sB + h * kDH * 128);
+        if constexpr (U8) mma_tile_f16(tmem + h * kDH, a, kBlk, bb, kBlk, kDH, L, false);
+        else mma_tile(tmem + h * kDH, a, kBlk, bb, kBlk, kDH, L, false);
+      }
       mma_commit(bar);
     }
     mbar_wait(bar, ph, status, abort_flag);
@@ -164,6 +214,10 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
       for (int q = 0; q < 8; ++q) tmem_ld16(ta + q * 16, row + q * 16);
       tmem_ld_wait();
+      if constexpr (U8) {
+#pragma unroll
+        for (int c = 0; c < kD; ++c) row[c] *= (1.0f / 255.0f);   // dequantise
+      }
 #pragma unroll
       for (int c = 0; c < 16; ++c) sw_st16(sA, kBlk, i, c * 8, pack8(row + c * 8));
     }
@@ -184,14 +238,13 @@ __global__ void __launch_bounds__(128)
   }
 }
 
-template <int L>
+template <int L, bool U8>
 int launch_score(int64_t B, const void* cache, int64_t n_items, const int32_t* ids,
                  const int64_t* off, int64_t total, const void* LP, void* O, unsigned* status,
                  cudaStream_t st) {
-  constexpr int HL = kH * L;
-  const int smem = 1024 + (2 * (HL / 64 < 2 ? 2 : HL / 64) + 1) * kBlk + 64 + 2 * 128 * 8;
-  if (cudaFuncSetAttribute(k_score_tc<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
+  using C = ScoreCfg<L, U8>;
+  if (cudaFuncSetAttribute(k_score_tc<L, U8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM) != cudaSuccess)
     return LIME_ERR_CUDA;
   // enough (user, slot) CTAs to fill every SM a few times over
   const int64_t target = 4LL * num_sms();
@@ -201,8 +254,8 @@ int launch_score(int64_t B, const void* cache, int64_t n_items, const int32_t* i
   if (G < 1) G = 1;
   if (G > 65535) G = 65535;
   dim3 grid((unsigned)B, (unsigned)G);
-  return launch_pdl(k_score_tc<L>, grid, dim3(128), smem, st, 1, (const bf16*)cache, n_items,
-                    ids, off, B, total, (const bf16*)LP, (bf16*)O, status);
+  return launch_pdl(k_score_tc<L, U8>, grid, dim3(128), C::SMEM, st, 1, cache, n_items, ids, off, B,
+                    total, (const bf16*)LP, (bf16*)O, status);
 }
 
 }  // namespace
@@ -211,14 +264,28 @@ bool fast_score_supported(const lime_dims& D) {
   return D.dtype == LIME_BF16 && D.d == kD && D.H == kH && (D.l == 16 || D.l == 32 || D.l == 64);
 }
 
+bool fast_score_u8_supported(const lime_dims& D) {
+  return fast_score_supported(D) && D.H * D.l >= 128;
+}
+
 int fast_score(const lime_dims& D, int64_t B, const void* cache, int64_t n_items,
                const int32_t* ids, const int64_t* off, int64_t total, const void* LP, void* O,
                float* ws, unsigned* status, cudaStream_t st) {
   (void)ws;
   switch (D.l) {
-    case 16: return launch_score<16>(B, cache, n_items, ids, off, total, LP, O, status, st);
-    case 32: return launch_score<32>(B, cache, n_items, ids, off, total, LP, O, status, st);
-    default: return launch_score<64>(B, cache, n_items, ids, off, total, LP, O, status, st);
+    case 16: return launch_score<16, false>(B, cache, n_items, ids, off, total, LP, O, status, st);
+    case 32: return launch_score<32, false>(B, cache, n_items, ids, off, total, LP, O, status, st);
+    default: return launch_score<64, false>(B, cache, n_items, ids, off, total, LP, O, status, st);
+  }
+}
+
+int fast_score_u8(const lime_dims& D, int64_t B, const uint8_t* cache, int64_t n_items,
+                  const int32_t* ids, const int64_t* off, int64_t total, const void* LP, void* O,
+                  unsigned* status, cudaStream_t st) {
+  switch (D.l) {
+    case 16: return launch_score<16, true>(B, cache, n_items, ids, off, total, LP, O, status, st);
+    case 32: return launch_score<32, true>(B, cache, n_items, ids, off, total, LP, O, status, st);
+    default: return launch_score<64, true>(B, cache, n_items, ids, off, total, LP, O, status, st);
   }
 }
 

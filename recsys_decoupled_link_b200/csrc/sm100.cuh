@@ -4,6 +4,7 @@
 // descriptors of the 128-byte-swizzled K-major layout.
 #pragma once
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -218,6 +219,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
          ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction descriptor: fp16 x fp16 -> fp32, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // Shared-memory descriptor of a K-major operand stored as 128-byte-swizzled
 // 8-row x 128-byte atoms (rows 128 bytes apart, 8-row groups 1024 bytes
 // apart).  `addr` is the byte address of the first row's current K slice; a
@@ -264,6 +270,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
 
+// Host: the same for a 2-D uint8 tensor (128-byte swizzle; box_inner <= 128).
+bool make_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                     uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
+
 // Host: number of SMs of the current device (cached per device).
 int num_sms();
 
@@ -298,6 +308,18 @@ __device__ __forceinline__ void mma_tile(uint32_t d_tmem, uint32_t a_base, uint3
                                          uint32_t b_base, uint32_t b_blk, int N, int K,
                                          bool accumulate) {
   const uint32_t idesc = idesc_bf16(128, N);
+  for (int k = 0; k < K / 16; ++k) {
+    const uint32_t off = (uint32_t)(k & 3) * 32;
+    mma_bf16(d_tmem, sdesc_sw128(a_base + (k >> 2) * a_blk + off),
+             sdesc_sw128(b_base + (k >> 2) * b_blk + off), idesc, accumulate || k > 0);
+  }
+}
+
+// mma_tile with fp16 operands (both A and B fp16).
+__device__ __forceinline__ void mma_tile_f16(uint32_t d_tmem, uint32_t a_base, uint32_t a_blk,
+                                             uint32_t b_base, uint32_t b_blk, int N, int K,
+                                             bool accumulate) {
+  const uint32_t idesc = idesc_f16(128, N);
   for (int k = 0; k < K / 16; ++k) {
     const uint32_t off = (uint32_t)(k & 3) * 32;
     mma_bf16(d_tmem, sdesc_sw128(a_base + (k >> 2) * a_blk + off),
@@ -420,6 +442,18 @@ __device__ __forceinline__ void tile_store_rows(const uint8_t* tile, bf16* dst, 
     const int r = idx >> 4, cc = idx & 15;
     if (r < nv) reinterpret_cast<uint4*>(dst + (int64_t)r * 128)[cc] = sw_ld16(tile, 128 * 128, r, cc * 8);
   }
+}
+
+// 8 floats -> 8 fp16 (round to nearest even).
+__device__ __forceinline__ uint4 pack8_f16(const float* f) {
+  uint4 v;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __half2 h = __floats2half2_rn(f[2 * j], f[2 * j + 1]);
+    w[j] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return v;
 }
 
 }  // namespace sm100

@@ -65,6 +65,8 @@ def _load() -> ctypes.CDLL:
         "lime_get_status": (I32, [P, P, ctypes.POINTER(ctypes.c_int)]),
         "lime_launch_count": (ctypes.c_uint64, []),
         "lime_build_qk_cache_noalloc": (I32, [D, P, I64, P, P, P, P, P]),
+        "lime_build_qk_cache_u8": (I32, [D, P, I64, P, P, P, P, P, SZ, P]),
+        "lime_score_candidates_u8": (I32, [D, I64, P, I64, P, P, I64, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -75,7 +77,8 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 EXPORTED = ("lime_workspace_bytes", "lime_workspace_init", "lime_build_qk_cache",
             "lime_context_links", "lime_xor_layer", "lime_score_candidates",
-            "lime_get_status", "lime_launch_count", "lime_build_qk_cache_noalloc")
+            "lime_get_status", "lime_launch_count", "lime_build_qk_cache_noalloc",
+            "lime_build_qk_cache_u8", "lime_score_candidates_u8")
 
 
 def library_path() -> str:
@@ -136,6 +139,23 @@ def lime_build_qk_cache(dims, T, L, Wq_c, Wk_c, cache_out, ws: Workspace, stream
     _check("lime_build_qk_cache", _lib.lime_build_qk_cache(
         ctypes.byref(dims), _ptr(T), n_items, _ptr(L), _ptr(Wq_c), _ptr(Wk_c),
         _ptr(cache_out), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def lime_build_qk_cache_u8(dims, T, L, Wq_c, Wk_c, cache_out, ws: Workspace, stream=None):
+    """int8 QK cache: cache_out uint8 [n_items, H, l] = round(255 w)."""
+    n_items = 0 if T is None else T.shape[0]
+    _check("lime_build_qk_cache_u8", _lib.lime_build_qk_cache_u8(
+        ctypes.byref(dims), _ptr(T), n_items, _ptr(L), _ptr(Wq_c), _ptr(Wk_c),
+        _ptr(cache_out), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def lime_score_candidates_u8(dims, cache, cand_ids, cand_offsets, total_cand, LP, O_out,
+                             ws: Workspace, stream=None):
+    """Cached scoring from an int8 cache (uint8 [n_items, H, l])."""
+    B = cand_offsets.shape[0] - 1
+    _check("lime_score_candidates_u8", _lib.lime_score_candidates_u8(
+        ctypes.byref(dims), B, _ptr(cache), cache.shape[0], _ptr(cand_ids), _ptr(cand_offsets),
+        int(total_cand), _ptr(LP), _ptr(O_out), ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def lime_build_qk_cache_noalloc(dims, T, L, Wq_c, Wk_c, cache_out, stream=None):

@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
         "lime_workspace_bytes", "lime_workspace_init", "lime_build_qk_cache",
         "lime_context_links", "lime_xor_layer", "lime_score_candidates", "lime_get_status",
-        "lime_launch_count", "lime_build_qk_cache_noalloc"])
+        "lime_launch_count", "lime_build_qk_cache_noalloc", "lime_build_qk_cache_u8",
+        "lime_score_candidates_u8"])
 
 
 def test_library_exports_every_declared_symbol(lime):

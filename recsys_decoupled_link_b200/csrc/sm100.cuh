@@ -274,6 +274,10 @@ bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint6
 bool make_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                      uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
 
+// Host: the same for a 2-D fp32 tensor (128-byte swizzle; box_inner <= 32).
+bool make_tmap_2d_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                      uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
+
 // Host: number of SMs of the current device (cached per device).
 int num_sms();
 

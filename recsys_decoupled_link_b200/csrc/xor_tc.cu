@@ -695,37 +695,62 @@ __global__ void __launch_bounds__(512, 1)
 // --------------------------------------------------------- XOR attention
 // 512 threads: thread (row, part) with row = 32*(warp%4) + lane (a TMEM lane)
 // and part = warp/4, a quarter of the row's columns (or of the tile's tokens
-// for the link branch).  Thread 0 issues the MMAs.
-template <int L, bool LAST>
+// for the link branch).  Thread 0 issues the MMAs and the loads.  Loads are
+// issued a tile ahead where the buffers allow: the next tile's V_E and user
+// images as soon as phase 2 has consumed this tile's, its Q_E and K_E once
+// this tile's delta has left the staging area.  Full tiles store the fp32
+// delta with TMA tensor stores.
+template <int L>
 __global__ void __launch_bounds__(512, 1)
     k_hist_attn(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, uint8_t* __restrict__ ws, LayerWs Lw,
-                unsigned* status) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmY,
+                uint8_t* __restrict__ ws, LayerWs Lw, unsigned* status) {
   constexpr int HL = kH * L;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
   uint8_t* sQ = sm;                 // Q_E -> P -> A_E (hi); with sK: fp32 delta staging
   uint8_t* sK = sm + 2 * kBlk;      // K_E -> P2 -> A_E (lo)
   uint8_t* sV = sm + 4 * kBlk;      // V_E rows (row-major, read as an MN-major operand)
-  uint8_t* sWo = sm + 6 * kBlk;     // Wo image (not in the last layer)
-  uint8_t* sQBD = sm + (LAST ? 6 : 8) * kBlk;   // block-diagonal s·Q_Z, hi then lo
-  uint8_t* sKZ = sQBD + 4 * kBlk;                // user images: s·K_Z, V_Z^T
+  uint8_t* sWo = sm + 6 * kBlk;     // Wo image
+  uint8_t* sQBD = sm + 8 * kBlk;    // block-diagonal s·Q_Z, hi then lo
+  uint8_t* sKZ = sQBD + 4 * kBlk;   // user images: s·K_Z, V_Z^T
   uint8_t* sVZT = sKZ + kz_bytes(L);
-  float* red = reinterpret_cast<float*>(sVZT + kBlk);   // [4][128]
+  float* red = reinterpret_cast<float*>(sVZT + kBlk);   // [2][4][128]
   Cta c;
-  cta_setup(sVZT + kBlk + 2048, 3, c);
+  cta_setup(sVZT + kBlk + 4096, 4, c);   // bar: 0 Q,K  1 mma  2 Wo  3 V + user image
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
   float* yd = reinterpret_cast<float*>(ws + Lw.yd);
   float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
-  uint32_t lph = 0, mph = 0;
-  if (!LAST) {
-    if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(&c.bar[2], 2 * kBlk);
-      bulk_load(sWo, ws + Lw.img_o, 2 * kBlk, &c.bar[2]);
+  uint32_t qph = 0, vph = 0, mph = 0;
+  auto load_qk = [&](int r0) {
+    mbar_arrive_expect_tx(&c.bar[0], 4 * kBlk);
+    tma_load_2d(sQ, &tmQ, 0, r0, &c.bar[0]);
+    tma_load_2d(sQ + kBlk, &tmQ, 64, r0, &c.bar[0]);
+    tma_load_2d(sK, &tmK, 0, r0, &c.bar[0]);
+    tma_load_2d(sK + kBlk, &tmK, 64, r0, &c.bar[0]);
+  };
+  auto load_v_img = [&](int r0, int u, bool img) {
+    mbar_arrive_expect_tx(&c.bar[3], 2 * kBlk + (img ? 3 * kz_bytes(L) + kBlk : 0));
+    tma_load_2d(sV, &tmV, 0, r0, &c.bar[3]);
+    tma_load_2d(sV + kBlk, &tmV, 64, r0, &c.bar[3]);
+    if (img) {
+      const uint8_t* im = ws + Lw.uimg + (size_t)u * Lw.uimg_bytes;
+      bulk_load(sKZ, im, kz_bytes(L) + kBlk, &c.bar[3]);
+      bulk_load(sQBD, im + qz_off(L), 2 * kz_bytes(L), &c.bar[3]);
     }
-    mbar_wait(&c.bar[2], 0, status, c.abort_flag);
+  };
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmY);
+    mbar_arrive_expect_tx(&c.bar[2], 2 * kBlk);
+    bulk_load(sWo, ws + Lw.img_o, 2 * kBlk, &c.bar[2]);
+    if ((int)blockIdx.x < n_tiles) {
+      const int4 tl = tiles[blockIdx.x];
+      load_qk(tl.y);
+      load_v_img(tl.y, tl.x, true);
+    }
   }
+  mbar_wait(&c.bar[2], 0, status, c.abort_flag);
   const int warp = threadIdx.x >> 5;
   const int part = warp >> 2;
   const int row = (warp & 3) * 32 + (threadIdx.x & 31);
@@ -734,25 +759,11 @@ __global__ void __launch_bounds__(512, 1)
   for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
     const int4 tl = tiles[t];
     const int u = tl.x, r0 = tl.y, nv = tl.z;
-    if (threadIdx.x == 0) {
-      uint32_t bytes = 4 * kBlk + (LAST ? 0 : 2 * kBlk) + (u != cur_u ? 3 * kz_bytes(L) + kBlk : 0);
-      mbar_arrive_expect_tx(&c.bar[0], bytes);
-      if (!LAST) {
-        tma_load_2d(sQ, &tmQ, 0, r0, &c.bar[0]);
-        tma_load_2d(sQ + kBlk, &tmQ, 64, r0, &c.bar[0]);
-      }
-      tma_load_2d(sK, &tmK, 0, r0, &c.bar[0]);
-      tma_load_2d(sK + kBlk, &tmK, 64, r0, &c.bar[0]);
-      tma_load_2d(sV, &tmV, 0, r0, &c.bar[0]);
-      tma_load_2d(sV + kBlk, &tmV, 64, r0, &c.bar[0]);
-      if (u != cur_u) {
-        const uint8_t* img = ws + Lw.uimg + (size_t)u * Lw.uimg_bytes;
-        bulk_load(sKZ, img, kz_bytes(L) + kBlk, &c.bar[0]);
-        bulk_load(sQBD, img + qz_off(L), 2 * kz_bytes(L), &c.bar[0]);
-      }
-    }
-    mbar_wait(&c.bar[0], lph, status, c.abort_flag);
-    lph ^= 1u;
+    const int tn = t + gridDim.x;
+    mbar_wait(&c.bar[0], qph, status, c.abort_flag);
+    qph ^= 1u;
+    mbar_wait(&c.bar[3], vph, status, c.abort_flag);
+    vph ^= 1u;
     if (u != cur_u) {
       expand_qbd<L>(sQBD, row, part);
       fence_proxy_async_smem();
@@ -763,16 +774,15 @@ __global__ void __launch_bounds__(512, 1)
     //          link scores, transposed: S'^T = (s Q_Z)_bd K_E^T -> TMEM [128, 256)
     if (threadIdx.x == 0) {
       tc_fence_after();
-      if (!LAST)
-        for (int h = 0; h < kH; ++h)
-          mma_tile(c.tmem + h * L, smem_u32(sQ + (h >> 1) * kBlk + (h & 1) * 64), kBlk,
-                   smem_u32(sKZ + (h >> 1) * (L * 128) + (h & 1) * 64), L * 128, L, kDH, false);
+      for (int h = 0; h < kH; ++h)
+        mma_tile(c.tmem + h * L, smem_u32(sQ + (h >> 1) * kBlk + (h & 1) * 64), kBlk,
+                 smem_u32(sKZ + (h >> 1) * (L * 128) + (h & 1) * 64), L * 128, L, kDH, false);
       mma_tile(c.tmem + 128, smem_u32(sQBD), kBlk, smem_u32(sK), kBlk, 128, 128, false);
       mma_tile(c.tmem + 128, smem_u32(sQBD + 2 * kBlk), kBlk, smem_u32(sK), kBlk, 128, 128, true);
     }
     cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
     // history softmax over the user's L links: part = head
-    if (!LAST) {
+    {
       const int h = part;
       float z[L];
 #pragma unroll
@@ -791,7 +801,9 @@ __global__ void __launch_bounds__(512, 1)
       for (int q = 0; q < L / 8; ++q) sw_st16(sQ, kBlk, row, h * L + q * 8, pack8(z + q * 8));
     }
     // link softmax over this tile's valid history rows; row = (head, link)
-    // lane, part = a quarter of the tile's 128 tokens
+    // lane, part = a quarter of the tile's 128 tokens.  The max and the sum
+    // are each reduced over the four parts through their own scratch (one
+    // barrier each: the next writes of either come after later barriers).
     float lm, ls;
     {
       float z[32];
@@ -804,15 +816,19 @@ __global__ void __launch_bounds__(512, 1)
         if (part * 32 + j >= nv) z[j] = -INFINITY;
         m = fmaxf(m, z[j]);
       }
-      m = row_max4(m, red, part, row);
+      red[part * 128 + row] = m;
+      __syncthreads();
+      m = fmaxf(fmaxf(red[row], red[128 + row]), fmaxf(red[256 + row], red[384 + row]));
       float s = 0.f;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         z[j] = part * 32 + j < nv ? __expf(z[j] - m) : 0.f;
         s += z[j];
       }
+      red[512 + part * 128 + row] = s;
+      __syncthreads();
       lm = m;
-      ls = row_sum4(s, red, part, row);
+      ls = red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row];
 #pragma unroll
       for (int q = 0; q < 4; ++q) sw_st16(sK, kBlk, row, part * 32 + q * 8, pack8(z + q * 8));
     }
@@ -822,32 +838,27 @@ __global__ void __launch_bounds__(512, 1)
     // phase 2: A_E,h = P_h V_Z,h -> TMEM [256, 384); link P2 V_E -> TMEM [384, 512)
     if (threadIdx.x == 0) {
       tc_fence_after();
-      if (!LAST)
-        for (int h = 0; h < kH; ++h)
-          mma_tile(c.tmem + 256 + h * kDH,
-                   smem_u32(sQ + ((h * L) >> 6) * kBlk + ((h * L) & 63) * 2), kBlk,
-                   smem_u32(sVZT + h * kDH * 128), kBlk, kDH, L, false);
+      for (int h = 0; h < kH; ++h)
+        mma_tile(c.tmem + 256 + h * kDH,
+                 smem_u32(sQ + ((h * L) >> 6) * kBlk + ((h * L) & 63) * 2), kBlk,
+                 smem_u32(sVZT + h * kDH * 128), kBlk, kDH, L, false);
       mma_tile_bmn(c.tmem + 384, smem_u32(sK), kBlk, smem_u32(sV), kBlk, 128, 128, false);
     }
     cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    if (!LAST) {
+    // V_E, s·K_Z and V_Z^T are consumed (and the expanded s·Q_Z since phase
+    // 1): the next tile's V_E and, for a new user, its images come in now
+    if (threadIdx.x == 0 && tn < n_tiles) {
+      const int4 tl2 = tiles[tn];
+      load_v_img(tl2.y, tl2.x, tl2.x != u);
+    }
+    {
       // A_E enters the Wo GEMM as hi + lo bf16 halves (sQ, sK), so the
       // attention delta keeps close to fp32 accuracy.
       float a[32];
       tmem_ld16(ta + 256 + part * 32, a);
       tmem_ld16(ta + 256 + part * 32 + 16, a + 16);
       tmem_ld_wait();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float h8[8], l8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          h8[k] = __bfloat162float(__float2bfloat16_rn(a[q * 8 + k]));
-          l8[k] = a[q * 8 + k] - h8[k];
-        }
-        sw_st16(sQ, kBlk, row, part * 32 + q * 8, pack8(h8));
-        sw_st16(sK, kBlk, row, part * 32 + q * 8, pack8(l8));
-      }
+      split_part_st(sQ, sK, row, part * 32, a);
     }
     {
       // link record of row p = (h, k): part h reads head h's 32 columns
@@ -865,29 +876,43 @@ __global__ void __launch_bounds__(512, 1)
         rec[8] = make_float4(acc[30], acc[31], 0.f, 0.f);
       }
     }
-    if (!LAST) {
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      // phase 3: Yd = A_E Wo -> TMEM [0, 128)
-      if (threadIdx.x == 0) {
-        tc_fence_after();
-        mma_tile(c.tmem, smem_u32(sQ), kBlk, smem_u32(sWo), kBlk, 128, 128, false);
-        mma_tile(c.tmem, smem_u32(sK), kBlk, smem_u32(sWo), kBlk, 128, 128, true);
-      }
-      cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-      {
-        // fp32 delta -> staging in sQ+sK (64 KB, free after the Wo MMA) ->
-        // coalesced stores of the valid rows
-        float y[32];
-        tmem_ld16(ta + part * 32, y);
-        tmem_ld16(ta + part * 32 + 16, y + 16);
-        tmem_ld_wait();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // phase 3: Yd = A_E Wo -> TMEM [0, 128)
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      mma_tile(c.tmem, smem_u32(sQ), kBlk, smem_u32(sWo), kBlk, 128, 128, false);
+      mma_tile(c.tmem, smem_u32(sK), kBlk, smem_u32(sWo), kBlk, 128, 128, true);
+    }
+    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+    {
+      float y[32];
+      tmem_ld16(ta + part * 32, y);
+      tmem_ld16(ta + part * 32 + 16, y + 16);
+      tmem_ld_wait();
+      if (nv == kTile) {
+        // full tile: four [128 x 32] fp32 boxes (128-byte swizzle), box = part
+        uint8_t* box = sQ + part * kBlk;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<float4*>(box + row * 128 + ((q ^ (row & 7)) << 4)) =
+              make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+      } else {
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           *f32_chunk(sQ, row, part * 8 + q) = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
       }
-      __syncthreads();
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (nv == kTile) {
+      if (threadIdx.x == 0) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_store_2d(&tmY, sQ + b * kBlk, b * 32, r0);
+        bulk_commit();
+      }
+    } else {
 #pragma unroll 4
       for (int q = 0; q < 8; ++q) {
         const int idx = q * 512 + (int)threadIdx.x, r = idx >> 5, cc = idx & 31;
@@ -897,7 +922,13 @@ __global__ void __launch_bounds__(512, 1)
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    // the next tile's Q_E and K_E, once the delta's staging has been read
+    if (threadIdx.x == 0 && tn < n_tiles) {
+      bulk_wait_read<0>();
+      load_qk(tiles[tn].y);
+    }
   }
+  if (threadIdx.x == 0) bulk_wait<0>();
   cta_teardown(c);
 }
 
@@ -1673,9 +1704,12 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
       if (rc) return rc;
     }
     if (!last) {
-      const int smem = 1024 + 12 * kBlk + kz_bytes(L) + kBlk + 2048 + kBarBytes;
-      if (!set_smem(k_hist_attn<L, false>, smem)) return LIME_ERR_CUDA;
-      int rc = launch_pdl(k_hist_attn<L, false>, dim3(grid), dim3(512), smem, st, 1, tmQ, tmK, tmV,
+      const int smem = 1024 + 12 * kBlk + kz_bytes(L) + kBlk + 4096 + kBarBytes;
+      CUtensorMap tmY;
+      if (!make_tmap_2d_f32(&tmY, ws + Lw.yd, kD, (uint64_t)nh, kD * 4, 32, kTile))
+        return LIME_ERR_CUDA;
+      if (!set_smem(k_hist_attn<L>, smem)) return LIME_ERR_CUDA;
+      int rc = launch_pdl(k_hist_attn<L>, dim3(grid), dim3(512), smem, st, 1, tmQ, tmK, tmV, tmY,
                           ws, Lw, status);
       if (rc) return rc;
     }

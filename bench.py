@@ -420,6 +420,31 @@ def main():
     if lime.lime_get_status(buf.ws) != 0:
         raise RuntimeError("device status flags set during the timed steps")
 
+    # Linearity in N: the user side of the long workload's shape (B = 32 users,
+    # 2 layers) at N = 1,024 / 4,096 / 16,384 history tokens per user.
+    lin = None
+    if rank == 0 and w.dtype == "bf16":
+        lin = {"B": 32, "N": [], "user_encode_ms": [], "us_per_1k_tokens": []}
+        for N in (1024, 4096, 16384):
+            wl = synth.workload("long", N=N, n_items=1024, M=1)
+            xl = pipeline.to_device(wl, synth.user_side(wl), synth.candidate_side(wl),
+                                    synth.item_table(wl))
+            bl = pipeline.alloc(xl)
+            for _ in range(3):
+                pipeline.user_encode(xl, bl)
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(5)]
+            for e in ev:
+                flush.zero_()
+                e[0].record(stream)
+                pipeline.user_encode(xl, bl)
+                e[1].record(stream)
+            torch.cuda.synchronize()
+            ms = sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+            lin["N"].append(N)
+            lin["user_encode_ms"].append(ms)
+            lin["us_per_1k_tokens"].append(ms * 1e3 / (xl.total_hist / 1e3))
+            del xl, bl
+
     if rank == 0:
         pk = peaks()
         work = work_units(w, total_hist, total_cand)
@@ -471,6 +496,8 @@ def main():
                                             "peak": pk["hbm_gbs"], "unit": "GB/s",
                                             "frac": sc_gbs / pk["hbm_gbs"]}},
         }
+        if lin is not None:
+            phases["user_encode_linearity"] = lin
         if u8 is not None:
             c8_bytes = w.n_items * (2 * w.d + w.H * w.l)
             s8_bytes = sc_pairs * (w.H * w.l + 4 + 2 * w.d)

@@ -56,15 +56,29 @@ __global__ void __launch_bounds__(512, 1)
   pdl_launch();
   pdl_wait();
   // weights: 16-byte chunk (k, n8) of a row-major [K x 128] matrix goes to
-  // row k, columns n8*8.. of the MN-major image
+  // row k, columns n8*8.. of the MN-major image.  All of a thread's loads are
+  // issued before any store, so their latencies overlap.
   {
     const uint4* g1 = reinterpret_cast<const uint4*>(Wc1);
-    for (int idx = tid; idx < din * 16; idx += 512)
-      sw_st16(sW1, w1_blk, idx >> 4, (idx & 15) * 8, __ldg(g1 + idx));
     const uint4* g2 = reinterpret_cast<const uint4*>(Wc2);
-#pragma unroll 4
-    for (int idx = tid; idx < kD * 16; idx += 512)
-      sw_st16(sW2, kBlk, idx >> 4, (idx & 15) * 8, __ldg(g2 + idx));
+    uint4 v1[8], v2[4];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int idx = q * 512 + tid;
+      if (idx < din * 16) v1[q] = __ldg(g1 + idx);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v2[q] = __ldg(g2 + q * 512 + tid);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int idx = q * 512 + tid;
+      if (idx < din * 16) sw_st16(sW1, w1_blk, idx >> 4, (idx & 15) * 8, v1[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int idx = q * 512 + tid;
+      sw_st16(sW2, kBlk, idx >> 4, (idx & 15) * 8, v2[q]);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -81,15 +95,23 @@ __global__ void __launch_bounds__(512, 1)
     const int64_t r0 = t * 128;
     const int nv = rows - r0 < 128 ? (int)(rows - r0) : 128;
     // gather the input rows [L_k ⊕ ctx_u]; rows past the end are zero
-    for (int idx = tid; idx < 128 * cpr; idx += 512) {
-      const int r = idx / cpr, cc = idx - r * cpr;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < nv) {
-        const int64_t R = r0 + r, u = R / l, k = R - u * l;
-        v = cc < 16 ? __ldg(reinterpret_cast<const uint4*>(L + k * kD) + cc)
-                    : __ldg(reinterpret_cast<const uint4*>(ctx + u * c) + (cc - 16));
+    {
+      uint4 v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int idx = q * 512 + tid, r = idx / cpr, cc = idx - r * cpr;
+        v[q] = make_uint4(0, 0, 0, 0);
+        if (idx < 128 * cpr && r < nv) {
+          const int64_t R = r0 + r, u = R / l, k = R - u * l;
+          v[q] = cc < 16 ? __ldg(reinterpret_cast<const uint4*>(L + k * kD) + cc)
+                         : __ldg(reinterpret_cast<const uint4*>(ctx + u * c) + (cc - 16));
+        }
       }
-      sw_st16(sX, kBlk, r, cc * 8, v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int idx = q * 512 + tid, r = idx / cpr, cc = idx - r * cpr;
+        if (idx < 128 * cpr) sw_st16(sX, kBlk, r, cc * 8, v[q]);
+      }
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -109,7 +131,10 @@ __global__ void __launch_bounds__(512, 1)
         float h8[8], l8[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float v = silu_f(x[q * 8 + j] + __bfloat162float(bc1[c0 + q * 8 + j]));
+          // SiLU with the hardware exp2 / reciprocal approximations (a few
+          // ulp; the hidden value is kept to about 16 bits as hi + lo)
+          const float a = x[q * 8 + j] + __bfloat162float(bc1[c0 + q * 8 + j]);
+          const float v = __fdividef(a, 1.0f + __expf(-a));
           h8[j] = __bfloat162float(__float2bfloat16_rn(v));
           l8[j] = v - h8[j];
         }

@@ -356,26 +356,35 @@ __global__ void __launch_bounds__(1024) k_prep_weights(
                    status);
     return;
   }
+  // Thread (matrix, n, k8) gathers W[k8*8 .. k8*8+7][n] (loads coalesced over
+  // n) and writes them as one 16-byte chunk of row n of the image.
   const int64_t e = (blockIdx.x - 1) * (int64_t)blockDim.x + threadIdx.x;
-  const int64_t n_sq = kD * kD, n_ff = kD * kF;
+  const int64_t n_sq = kD * kD / 8, n_ff = kD * kF / 8;   // chunks per matrix
+  float f[8];
   if (e < 4 * n_sq) {
     const int w = (int)(e / n_sq), r = (int)(e % n_sq);
-    const int k = r / kD, n = r % kD;
+    const int k8 = r / kD, n = r % kD;
     const bf16* src = w == 0 ? Wq : w == 1 ? Wk : w == 2 ? Wv : Wo;
     const size_t base = w == 0 ? L.img_q : w == 1 ? L.img_k : w == 2 ? L.img_v : L.img_o;
-    *reinterpret_cast<bf16*>(ws + base + (k >> 6) * kBlk + sw128_offset(n, k & 63)) = src[r];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = __bfloat162float(src[(k8 * 8 + j) * kD + n]);
+    sw_st16(ws + base, kBlk, n, k8 * 8, pack8(f));
   } else if (e < 4 * n_sq + 2 * n_ff) {
     const int64_t r0 = e - 4 * n_sq;
     const int w = (int)(r0 / n_ff), r = (int)(r0 % n_ff);
-    const int k = r / kF, n = r % kF;
+    const int k8 = r / kF, n = r % kF;
     // chunk n/64 of the hidden layer: K block k/64 holds W1's 64 rows, then W3's
     const bf16* src = w == 0 ? W1 : W3;
-    *reinterpret_cast<bf16*>(ws + L.img_13 + (n >> 6) * (2 * kBlk) + (k >> 6) * kBlk +
-                             w * 8192 + sw128_offset(n & 63, k & 63)) = src[r];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = __bfloat162float(src[(k8 * 8 + j) * kF + n]);
+    *reinterpret_cast<uint4*>(ws + L.img_13 + (n >> 6) * (2 * kBlk) + ((k8 * 8) >> 6) * kBlk +
+                              w * 8192 + sw128_offset(n & 63, (k8 * 8) & 63)) = pack8(f);
   } else if (e < 4 * n_sq + 3 * n_ff) {
     const int r = (int)(e - 4 * n_sq - 2 * n_ff);
-    const int k = r / kD, n = r % kD;   // W2 is [256, 128]
-    *reinterpret_cast<bf16*>(ws + L.img_2 + (k >> 6) * kBlk + sw128_offset(n, k & 63)) = W2[r];
+    const int k8 = r / kD, n = r % kD;   // W2 is [256, 128]
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = __bfloat162float(W2[(k8 * 8 + j) * kD + n]);
+    sw_st16(ws + L.img_2, kBlk, n, k8 * 8, pack8(f));
   }
 }
 
@@ -1666,7 +1675,7 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
   const int64_t nz = B * L;
   const int sms = num_sms();
   {
-    const int64_t n = 4 * kD * kD + 3 * kD * kF;
+    const int64_t n = (4 * kD * kD + 3 * kD * kF) / 8;
     int rc = launch_pdl(k_prep_weights, dim3((unsigned)(1 + (n + 1023) / 1024)), dim3(1024), 0, st,
                         1, (const bf16*)w.Wq, (const bf16*)w.Wk, (const bf16*)w.Wv,
                         (const bf16*)w.Wo, (const bf16*)w.W1, (const bf16*)w.W3, (const bf16*)w.W2,

@@ -1480,12 +1480,12 @@ __global__ void __launch_bounds__(512, 1)
       const float* recs = reinterpret_cast<const float*>(ws + Lw.part);
       float M = -INFINITY;
       const int ta_ = ts[u], tb_ = ts[u + 1];
-      for (int t = ta_; t < tb_; t += 4) {
-        // the records of up to four tiles are loaded before any is merged
-        float2 ms[4];
-        float a[4][8];
+      for (int t = ta_; t < tb_; t += 8) {
+        // the records of up to eight tiles are loaded before any is merged
+        float2 ms[8];
+        float a[8][8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 8; ++i) {
           if (t + i < tb_) {
             const float* rec = recs + ((size_t)(t + i) * HL + h * L + k) * kRec;
             ms[i] = *reinterpret_cast<const float2*>(rec);
@@ -1498,7 +1498,7 @@ __global__ void __launch_bounds__(512, 1)
           }
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 8; ++i) {
           if (t + i < tb_) {
             const float Mn = fmaxf(M, ms[i].x);
             const float so = M == -INFINITY ? 0.f : __expf(M - Mn);

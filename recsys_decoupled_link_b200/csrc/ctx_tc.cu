@@ -8,9 +8,10 @@
 // is two GEMMs with B*l rows; row r is link k = r % l of user u = r / l.
 //
 // One CTA per 128 rows (persistent over more tiles when there are more tiles
-// than SMs).  Wc1 and Wc2 are staged once per CTA as MN-major operand images
-// (row-major [K x 128] tiles in 128-byte-swizzled 64-column blocks); per tile
-// the [128 x (d + c)] input rows are gathered into a K-major operand, GEMM 1
+// than SMs).  Wc1 and Wc2 are loaded once per CTA with TMA as MN-major operand
+// images (row-major [K x 128] tiles in 128-byte-swizzled 64-column blocks);
+// per tile the [128 x (d + c)] input rows are gathered with asynchronous
+// copies into a K-major operand, GEMM 1
 // runs into TMEM, the epilogue adds bc1, applies SiLU and writes the hidden
 // rows as bf16 hi + lo halves (hi = bf16(x), lo = bf16(x - hi)), GEMM 2 takes
 // both halves (so the hidden layer keeps about 16 mantissa bits), and the
@@ -29,9 +30,9 @@ constexpr int kD = 128;
 constexpr uint32_t kBlk = 128 * 128;   // one [128 x 64] bf16 block
 
 __global__ void __launch_bounds__(512, 1)
-    k_context_tc(int c, int l, int64_t rows, const bf16* __restrict__ L,
-                 const bf16* __restrict__ ctx, const bf16* __restrict__ Wc1,
-                 const bf16* __restrict__ bc1, const bf16* __restrict__ Wc2,
+    k_context_tc(const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
+                 int c, int l, int64_t rows, const bf16* __restrict__ L,
+                 const bf16* __restrict__ ctx, const bf16* __restrict__ bc1,
                  const bf16* __restrict__ bc2, bf16* __restrict__ LC, unsigned* status) {
   const int din = kD + c;                 // 192 or 256
   const uint32_t w1_blk = (uint32_t)din * 128;
@@ -41,12 +42,13 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sHlo = sm + 4 * kBlk;          // hidden lo
   uint8_t* sW2 = sm + 6 * kBlk;           // Wc2 [128 x 128] MN-major
   uint8_t* sW1 = sm + 8 * kBlk;           // Wc1 [din x 128] MN-major (2 blocks of din rows)
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sW1 + 2 * w1_blk);
-  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 1);
-  int* abort_flag = reinterpret_cast<int*>(bar + 2);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sW1 + 2 * w1_blk);   // [0] mma, [1] weights
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 2);
+  int* abort_flag = reinterpret_cast<int*>(bar + 3);
   const int tid = threadIdx.x;
   if (tid == 0) {
-    mbar_init(bar, 1);
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -55,30 +57,14 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   pdl_launch();
   pdl_wait();
-  // weights: 16-byte chunk (k, n8) of a row-major [K x 128] matrix goes to
-  // row k, columns n8*8.. of the MN-major image.  All of a thread's loads are
-  // issued before any store, so their latencies overlap.
-  {
-    const uint4* g1 = reinterpret_cast<const uint4*>(Wc1);
-    const uint4* g2 = reinterpret_cast<const uint4*>(Wc2);
-    uint4 v1[8], v2[4];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int idx = q * 512 + tid;
-      if (idx < din * 16) v1[q] = __ldg(g1 + idx);
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) v2[q] = __ldg(g2 + q * 512 + tid);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int idx = q * 512 + tid;
-      if (idx < din * 16) sw_st16(sW1, w1_blk, idx >> 4, (idx & 15) * 8, v1[q]);
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int idx = q * 512 + tid;
-      sw_st16(sW2, kBlk, idx >> 4, (idx & 15) * 8, v2[q]);
-    }
+  // weights: TMA tiles of the row-major [K x 128] matrices in 128-byte
+  // swizzle are exactly the MN-major operand images (64 columns per block)
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bar[1], 2 * w1_blk + 2 * kBlk);
+    tma_load_2d(sW1, &tmW1, 0, 0, &bar[1]);
+    tma_load_2d(sW1 + w1_blk, &tmW1, 64, 0, &bar[1]);
+    tma_load_2d(sW2, &tmW2, 0, 0, &bar[1]);
+    tma_load_2d(sW2 + kBlk, &tmW2, 64, 0, &bar[1]);
   }
   tc_fence_before();
   __syncthreads();
@@ -94,33 +80,30 @@ __global__ void __launch_bounds__(512, 1)
   for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x) {
     const int64_t r0 = t * 128;
     const int nv = rows - r0 < 128 ? (int)(rows - r0) : 128;
-    // gather the input rows [L_k ⊕ ctx_u]; rows past the end are zero
-    {
-      uint4 v[8];
+    // gather the input rows [L_k ⊕ ctx_u] with asynchronous copies; rows past
+    // the end are zero
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int idx = q * 512 + tid, r = idx / cpr, cc = idx - r * cpr;
-        v[q] = make_uint4(0, 0, 0, 0);
-        if (idx < 128 * cpr && r < nv) {
-          const int64_t R = r0 + r, u = R / l, k = R - u * l;
-          v[q] = cc < 16 ? __ldg(reinterpret_cast<const uint4*>(L + k * kD) + cc)
-                         : __ldg(reinterpret_cast<const uint4*>(ctx + u * c) + (cc - 16));
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int idx = q * 512 + tid, r = idx / cpr, cc = idx - r * cpr;
-        if (idx < 128 * cpr) sw_st16(sX, kBlk, r, cc * 8, v[q]);
+    for (int q = 0; q < 8; ++q) {
+      const int idx = q * 512 + tid, r = idx / cpr, cc = idx - r * cpr;
+      if (idx < 128 * cpr) {
+        const bool ok = r < nv;
+        const int64_t R = ok ? r0 + r : 0, u = R / l, k = R - u * l;
+        const void* src = cc < 16 ? (const void*)(L + k * kD + cc * 8)
+                                  : (const void*)(ctx + u * c + (cc - 16) * 8);
+        cp_async16(sX + (cc >> 3) * kBlk + sw128_offset(r, (cc & 7) * 8), src, ok);
       }
     }
+    cp_async_commit();
+    cp_async_wait<0>();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
+      if (t == blockIdx.x) mbar_wait(&bar[1], 0, status, abort_flag);   // weights landed
       tc_fence_after();
       mma_tile_bmn(tmem, smem_u32(sX), kBlk, smem_u32(sW1), w1_blk, 128, din, false);
     }
-    cta_mma_wait(bar, ph, status, abort_flag);
+    cta_mma_wait(&bar[0], ph, status, abort_flag);
     {
       float x[32];
       tmem_ld16(ta + c0, x);
@@ -150,7 +133,7 @@ __global__ void __launch_bounds__(512, 1)
       mma_tile_bmn(tmem + 128, smem_u32(sX), kBlk, smem_u32(sW2), kBlk, 128, kD, false);
       mma_tile_bmn(tmem + 128, smem_u32(sHlo), kBlk, smem_u32(sW2), kBlk, 128, kD, true);
     }
-    cta_mma_wait(bar, ph, status, abort_flag);
+    cta_mma_wait(&bar[0], ph, status, abort_flag);
     {
       float x[32];
       tmem_ld16(ta + 128 + c0, x);
@@ -182,7 +165,7 @@ bool fast_ctx_supported(const lime_dims& D) {
 }
 
 size_t fast_ctx_smem(const lime_dims& D) {
-  return 1024 + 8 * (size_t)kBlk + 2 * (size_t)(kD + D.c) * 128 + 64;
+  return 1024 + 8 * (size_t)kBlk + 2 * (size_t)(kD + D.c) * 128 + 64;   // + barriers
 }
 
 int fast_context_links(const lime_dims& D, int64_t B, const void* L, const void* ctx,
@@ -194,9 +177,13 @@ int fast_context_links(const lime_dims& D, int64_t B, const void* L, const void*
     return LIME_ERR_CUDA;
   int64_t grid = (rows + 127) / 128;
   if (grid > num_sms()) grid = num_sms();
-  return launch_pdl(k_context_tc, dim3((unsigned)grid), dim3(512), smem, st, 1, D.c, D.l, rows,
-                    (const bf16*)L, (const bf16*)ctx, (const bf16*)w.Wc1, (const bf16*)w.bc1,
-                    (const bf16*)w.Wc2, (const bf16*)w.bc2, (bf16*)LC, status);
+  CUtensorMap tmW1, tmW2;
+  if (!make_tmap_2d_bf16(&tmW1, w.Wc1, kD, (uint64_t)(kD + D.c), kD * 2, 64, kD + D.c) ||
+      !make_tmap_2d_bf16(&tmW2, w.Wc2, kD, kD, kD * 2, 64, kD))
+    return LIME_ERR_CUDA;
+  return launch_pdl(k_context_tc, dim3((unsigned)grid), dim3(512), smem, st, 1, tmW1, tmW2, D.c,
+                    D.l, rows, (const bf16*)L, (const bf16*)ctx, (const bf16*)w.bc1,
+                    (const bf16*)w.bc2, (bf16*)LC, status);
 }
 
 }  // namespace lime

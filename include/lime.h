@@ -109,6 +109,27 @@ int lime_build_qk_cache(const lime_dims* dims, const void* T, int64_t n_items,
                         void* cache_out, void* workspace, size_t workspace_bytes,
                         cudaStream_t stream);
 
+/* Two-stage form of lime_build_qk_cache, for callers that run the small first
+ * stage on another stream (it depends only on the weights):
+ * lime_fold_qk writes the folded per-head matrix G_h = s Wq_c[:, h-cols]
+ * (L Wk_c[:, h-cols])^T (d x H*l, the same for every item; LIME note 关键设计
+ * 1: the weights depend only on the item and the global links) to `image`
+ * as the 128-byte-swizzled operand image the build reads;
+ * lime_build_qk_cache_folded then computes cache[m, h, :] =
+ * softmax_k((T_m G_h)_k) over the catalogue.  Together they equal
+ * lime_build_qk_cache.
+ *   image  device, lime_qk_image_bytes(dims) bytes (2*d*H*l), 16-byte
+ *          aligned; written by lime_fold_qk, read by the build.
+ * Other arguments, checks and errors as lime_build_qk_cache.  Supported:
+ * the bf16 tensor-core shapes (lime_qk_image_bytes returns 0 otherwise and
+ * both calls return LIME_ERR_SHAPE).  lime_fold_qk uses no workspace.      */
+size_t lime_qk_image_bytes(const lime_dims* dims);
+int lime_fold_qk(const lime_dims* dims, const void* L, const void* Wq_c, const void* Wk_c,
+                 void* image, cudaStream_t stream);
+int lime_build_qk_cache_folded(const lime_dims* dims, const void* T, int64_t n_items,
+                               const void* image, void* cache_out, void* workspace,
+                               size_t workspace_bytes, cudaStream_t stream);
+
 /* Allocation-free variant of lime_build_qk_cache.  The paper has no
  * counterpart: it exists for callers that cannot allocate device memory, such
  * as a plug-in whose host framework owns the whole device memory pool, or a

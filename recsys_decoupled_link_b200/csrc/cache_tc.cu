@@ -356,17 +356,17 @@ bool fast_cache_u8_supported(const lime_dims& D) {
 }
 
 namespace {
-int build_cache(const lime_dims& D, const void* T, int64_t n, const void* L, const void* Wq,
-                const void* Wk, void* cache, bool u8, float* ws, unsigned* status,
+int launch_fold(const lime_dims& D, const void* L, const void* Wq, const void* Wk, bf16* img,
                 cudaStream_t st) {
-  const int HL = D.H * D.l;
-  bf16* img = reinterpret_cast<bf16*>(ws);
   const float scale = 1.0f / sqrtf((float)(D.d / D.H));
-  int rc = launch_pdl(k_fold_g_img, dim3(HL), dim3(128), 0, st, 1, (const bf16*)L,
-                      (const bf16*)Wq, (const bf16*)Wk, D.H, D.l, scale, img);
-  if (rc) return rc;
+  return launch_pdl(k_fold_g_img, dim3(D.H * D.l), dim3(128), 0, st, 1, (const bf16*)L,
+                    (const bf16*)Wq, (const bf16*)Wk, D.H, D.l, scale, img);
+}
+
+int launch_build(const lime_dims& D, const void* T, int64_t n, const bf16* img, void* cache,
+                 bool u8, unsigned* status, cudaStream_t st) {
   if (n == 0) return LIME_OK;
-  switch (HL * 1000 + D.l + (u8 ? 1000000 : 0)) {
+  switch (D.H * D.l * 1000 + D.l + (u8 ? 1000000 : 0)) {
     case 64016: return launch_cache<64, 16, false>(T, n, img, cache, status, st);
     case 64032: return launch_cache<64, 32, false>(T, n, img, cache, status, st);
     case 128016: return launch_cache<128, 16, false>(T, n, img, cache, status, st);
@@ -387,13 +387,27 @@ int build_cache(const lime_dims& D, const void* T, int64_t n, const void* L, con
 int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void* L,
                         const void* Wq, const void* Wk, void* cache, float* ws,
                         unsigned* status, cudaStream_t st) {
-  return build_cache(D, T, n, L, Wq, Wk, cache, false, ws, status, st);
+  bf16* img = reinterpret_cast<bf16*>(ws);
+  int rc = launch_fold(D, L, Wq, Wk, img, st);
+  return rc ? rc : launch_build(D, T, n, img, cache, false, status, st);
 }
 
 int fast_build_qk_cache_u8(const lime_dims& D, const void* T, int64_t n, const void* L,
                            const void* Wq, const void* Wk, void* cache, float* ws,
                            unsigned* status, cudaStream_t st) {
-  return build_cache(D, T, n, L, Wq, Wk, cache, true, ws, status, st);
+  bf16* img = reinterpret_cast<bf16*>(ws);
+  int rc = launch_fold(D, L, Wq, Wk, img, st);
+  return rc ? rc : launch_build(D, T, n, img, cache, true, status, st);
+}
+
+int fast_fold_qk(const lime_dims& D, const void* L, const void* Wq, const void* Wk, void* image,
+                 cudaStream_t st) {
+  return launch_fold(D, L, Wq, Wk, reinterpret_cast<bf16*>(image), st);
+}
+
+int fast_build_qk_cache_folded(const lime_dims& D, const void* T, int64_t n, const void* image,
+                               void* cache, unsigned* status, cudaStream_t st) {
+  return launch_build(D, T, n, reinterpret_cast<const bf16*>(image), cache, false, status, st);
 }
 
 }  // namespace lime

@@ -222,6 +222,53 @@ int lime_score_candidates(const lime_dims* dims, int64_t B, const void* cache, i
   return launch_status("lime_score_candidates");
 }
 
+size_t lime_qk_image_bytes(const lime_dims* dims) {
+  if (!dims || check_dims(dims) || dims->dtype != LIME_BF16 || !fast_cache_supported(*dims))
+    return 0;
+  return (size_t)2 * dims->d * dims->H * dims->l;
+}
+
+int lime_fold_qk(const lime_dims* dims, const void* L, const void* Wq_c, const void* Wk_c,
+                 void* image, cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!lime_qk_image_bytes(dims)) return LIME_ERR_SHAPE;
+  if (!L || !Wq_c || !Wk_c || !image) return LIME_ERR_ARG;
+  if (!aligned16(L) || !aligned16(Wq_c) || !aligned16(Wk_c) || !aligned16(image))
+    return LIME_ERR_ARG;
+  const size_t es = esize(dims), img = lime_qk_image_bytes(dims);
+  if (overlap(image, img, L, (size_t)dims->l * dims->d * es) ||
+      overlap(image, img, Wq_c, (size_t)dims->d * dims->d * es) ||
+      overlap(image, img, Wk_c, (size_t)dims->d * dims->d * es))
+    return LIME_ERR_ALIAS;
+  if ((rc = fast_fold_qk(*dims, L, Wq_c, Wk_c, image, stream))) return rc;
+  return launch_status("lime_fold_qk");
+}
+
+int lime_build_qk_cache_folded(const lime_dims* dims, const void* T, int64_t n_items,
+                               const void* image, void* cache_out, void* workspace,
+                               size_t workspace_bytes, cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!lime_qk_image_bytes(dims)) return LIME_ERR_SHAPE;
+  if (n_items < 0 || n_items > (int64_t)INT32_MAX + 1) return LIME_ERR_ARG;
+  if (!image || (n_items > 0 && (!T || !cache_out))) return LIME_ERR_ARG;
+  if (!aligned16(image) || (n_items > 0 && (!aligned16(T) || !aligned16(cache_out))))
+    return LIME_ERR_ARG;
+  if ((rc = check_ws(workspace, workspace_bytes, dims, 0, 0))) return rc;
+  const size_t es = esize(dims);
+  const size_t cache_sz = (size_t)n_items * dims->H * dims->l * es;
+  if (overlap(cache_out, cache_sz, T, (size_t)n_items * dims->d * es) ||
+      overlap(cache_out, cache_sz, image, lime_qk_image_bytes(dims)) ||
+      overlap(workspace, workspace_bytes, image, lime_qk_image_bytes(dims)) ||
+      overlap(workspace, workspace_bytes, cache_out, cache_sz))
+    return LIME_ERR_ALIAS;
+  if ((rc = fast_build_qk_cache_folded(*dims, T, n_items, image, cache_out, status_of(workspace),
+                                       stream)))
+    return rc;
+  return launch_status("lime_build_qk_cache_folded");
+}
+
 int lime_build_qk_cache_u8(const lime_dims* dims, const void* T, int64_t n_items, const void* L,
                            const void* Wq_c, const void* Wk_c, uint8_t* cache_out,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {

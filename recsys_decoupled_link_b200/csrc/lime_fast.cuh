@@ -43,6 +43,12 @@ int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void
                         const void* Wq, const void* Wk, void* cache, float* ws,
                         unsigned* status, cudaStream_t st);
 
+// the two stages of fast_build_qk_cache (bf16 cache): G^T image, catalogue
+int fast_fold_qk(const lime_dims& D, const void* L, const void* Wq, const void* Wk, void* image,
+                 cudaStream_t st);
+int fast_build_qk_cache_folded(const lime_dims& D, const void* T, int64_t n, const void* image,
+                               void* cache, unsigned* status, cudaStream_t st);
+
 // int8 cache (bytes q = round(255 w)); needs H*l >= 128
 bool fast_cache_u8_supported(const lime_dims& D);
 int fast_build_qk_cache_u8(const lime_dims& D, const void* T, int64_t n, const void* L,

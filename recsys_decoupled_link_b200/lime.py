@@ -67,6 +67,9 @@ def _load() -> ctypes.CDLL:
         "lime_build_qk_cache_noalloc": (I32, [D, P, I64, P, P, P, P, P]),
         "lime_build_qk_cache_u8": (I32, [D, P, I64, P, P, P, P, P, SZ, P]),
         "lime_score_candidates_u8": (I32, [D, I64, P, I64, P, P, I64, P, P, P, SZ, P]),
+        "lime_qk_image_bytes": (SZ, [D]),
+        "lime_fold_qk": (I32, [D, P, P, P, P, P]),
+        "lime_build_qk_cache_folded": (I32, [D, P, I64, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -78,7 +81,8 @@ _lib = _load()
 EXPORTED = ("lime_workspace_bytes", "lime_workspace_init", "lime_build_qk_cache",
             "lime_context_links", "lime_xor_layer", "lime_score_candidates",
             "lime_get_status", "lime_launch_count", "lime_build_qk_cache_noalloc",
-            "lime_build_qk_cache_u8", "lime_score_candidates_u8")
+            "lime_build_qk_cache_u8", "lime_score_candidates_u8", "lime_qk_image_bytes",
+            "lime_fold_qk", "lime_build_qk_cache_folded")
 
 
 def library_path() -> str:
@@ -147,6 +151,24 @@ def lime_build_qk_cache_u8(dims, T, L, Wq_c, Wk_c, cache_out, ws: Workspace, str
     _check("lime_build_qk_cache_u8", _lib.lime_build_qk_cache_u8(
         ctypes.byref(dims), _ptr(T), n_items, _ptr(L), _ptr(Wq_c), _ptr(Wk_c),
         _ptr(cache_out), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def lime_qk_image_bytes(dims) -> int:
+    return int(_lib.lime_qk_image_bytes(ctypes.byref(dims)))
+
+
+def lime_fold_qk(dims, L, Wq_c, Wk_c, image, stream=None):
+    """First stage of the QK cache: the folded G^T operand image (uint8 bytes)."""
+    _check("lime_fold_qk", _lib.lime_fold_qk(
+        ctypes.byref(dims), _ptr(L), _ptr(Wq_c), _ptr(Wk_c), _ptr(image), _stream(stream)))
+
+
+def lime_build_qk_cache_folded(dims, T, image, cache_out, ws: Workspace, stream=None):
+    """Second stage of the QK cache: the catalogue pass over a folded image."""
+    n_items = 0 if T is None else T.shape[0]
+    _check("lime_build_qk_cache_folded", _lib.lime_build_qk_cache_folded(
+        ctypes.byref(dims), _ptr(T), n_items, _ptr(image), _ptr(cache_out), ws.ptr, ws.nbytes,
+        _stream(stream)))
 
 
 def lime_score_candidates_u8(dims, cache, cand_ids, cand_offsets, total_cand, LP, O_out,

@@ -5,6 +5,11 @@ the library in the order the method runs them (LIME note, 整体框架 and
 一个完整示例): context links, the LIME-XOR layer stack (the last layer marked
 by E_out = NULL), the QK-cache build over the catalogue, and cached candidate
 scoring.  All arithmetic happens inside liblime.
+
+Where the library offers the two-stage cache build, ``step`` runs its first
+stage (the folded per-head matrix, which depends only on the weights) on a
+side stream at the start of the step, so it overlaps the user side; the
+catalogue pass then waits for it on the main stream.
 """
 from __future__ import annotations
 
@@ -45,6 +50,10 @@ class Buffers:
     cache: torch.Tensor
     O: torch.Tensor
     ws: lime.Workspace
+    image: Optional[torch.Tensor] = None          # folded G^T operand image
+    side: Optional[torch.cuda.Stream] = None      # stream the fold runs on
+    fold_done: Optional[torch.cuda.Event] = None
+    fold_pending: bool = False
 
 
 def to_device(w: synth.Workload, us: synth.UserSide, cs: synth.CandidateSide,
@@ -71,13 +80,32 @@ def alloc(x: DeviceInputs, n_items: Optional[int] = None, device="cuda") -> Buff
     dt = synth.torch_dtype(w)
     n_items = w.n_items if n_items is None else n_items
     nbuf = 2 if w.layers > 1 else 1
+    img_bytes = lime.lime_qk_image_bytes(x.dims)
+    two_stage = {}
+    if img_bytes:
+        two_stage = dict(image=torch.empty(img_bytes, dtype=torch.uint8, device=device),
+                         side=torch.cuda.Stream(device=device), fold_done=torch.cuda.Event())
     return Buffers(
         LC=torch.empty(w.B, w.l, w.d, dtype=dt, device=device),
         E_bufs=[torch.empty(x.total_hist, w.d, dtype=dt, device=device) for _ in range(nbuf)],
         Z_bufs=[torch.empty(w.B, w.l, w.d, dtype=dt, device=device) for _ in range(2)],
         cache=torch.empty(n_items, w.H, w.l, dtype=dt, device=device),
         O=torch.empty(x.total_cand, w.d, dtype=dt, device=device),
-        ws=lime.Workspace(x.dims, w.B, x.total_hist, device=device))
+        ws=lime.Workspace(x.dims, w.B, x.total_hist, device=device), **two_stage)
+
+
+def fold_qk(x: DeviceInputs, buf: Buffers, stream=None):
+    """Starts the first cache stage on the side stream (no-op without one).
+
+    The side stream first waits for everything already queued on ``stream``
+    (the previous step's catalogue pass still reads the image)."""
+    if buf.image is None:
+        return
+    main = torch.cuda.current_stream() if stream is None else stream
+    buf.side.wait_stream(main)
+    lime.lime_fold_qk(x.dims, x.L, x.Wq_c, x.Wk_c, buf.image, stream=buf.side)
+    buf.fold_done.record(buf.side)
+    buf.fold_pending = True
 
 
 def user_encode(x: DeviceInputs, buf: Buffers, stream=None) -> torch.Tensor:
@@ -100,7 +128,15 @@ def user_encode(x: DeviceInputs, buf: Buffers, stream=None) -> torch.Tensor:
 
 
 def build_cache(x: DeviceInputs, buf: Buffers, stream=None):
-    lime.lime_build_qk_cache(x.dims, x.T, x.L, x.Wq_c, x.Wk_c, buf.cache, buf.ws, stream=stream)
+    """The QK cache; the catalogue pass alone when fold_qk started this step."""
+    if buf.fold_pending:
+        main = torch.cuda.current_stream() if stream is None else stream
+        main.wait_event(buf.fold_done)
+        buf.fold_pending = False
+        lime.lime_build_qk_cache_folded(x.dims, x.T, buf.image, buf.cache, buf.ws, stream=main)
+    else:
+        lime.lime_build_qk_cache(x.dims, x.T, x.L, x.Wq_c, x.Wk_c, buf.cache, buf.ws,
+                                 stream=stream)
 
 
 def score(x: DeviceInputs, buf: Buffers, LP: torch.Tensor, stream=None):
@@ -110,6 +146,7 @@ def score(x: DeviceInputs, buf: Buffers, LP: torch.Tensor, stream=None):
 
 def step(x: DeviceInputs, buf: Buffers, stream=None) -> torch.Tensor:
     """One pass of the whole hot path; returns O [sum M, d]."""
+    fold_qk(x, buf, stream)
     LP = user_encode(x, buf, stream)
     build_cache(x, buf, stream)
     score(x, buf, LP, stream)

@@ -31,7 +31,8 @@ def test_header_declares_the_boundary():
         "lime_workspace_bytes", "lime_workspace_init", "lime_build_qk_cache",
         "lime_context_links", "lime_xor_layer", "lime_score_candidates", "lime_get_status",
         "lime_launch_count", "lime_build_qk_cache_noalloc", "lime_build_qk_cache_u8",
-        "lime_score_candidates_u8"])
+        "lime_score_candidates_u8", "lime_qk_image_bytes", "lime_fold_qk",
+        "lime_build_qk_cache_folded"])
 
 
 def test_library_exports_every_declared_symbol(lime):
@@ -105,3 +106,32 @@ def test_host_validation_of_scoring_and_cache(lime):
     mlp = lime.lime_ctx_mlp(0x10000, 0x20000, 0x30000, 0x40000)
     assert c(ctypes.byref(nodims), 2, 0x50000, 0x60000, ctypes.byref(mlp), 0x70000,
              0x1000000, nws, None) == lime.LIME_ERR_SHAPE
+
+
+def test_host_validation_of_two_stage_cache(lime):
+    dims = lime.make_dims(128, 4, 32, 256, 64, "bf16")
+    img = lime.lime_qk_image_bytes(dims)
+    assert img == 2 * 128 * 4 * 32
+    assert lime.lime_qk_image_bytes(lime.make_dims(128, 4, 32, 256, 64, "f32")) == 0
+    assert lime.lime_qk_image_bytes(lime.make_dims(128, 4, 48, 256, 64, "bf16")) == 0
+    fold = lime._lib.lime_fold_qk
+    assert fold(ctypes.byref(dims), 0x100000, 0x200000, 0x300000, None, None) == lime.LIME_ERR_ARG
+    assert fold(ctypes.byref(dims), 0x100000, 0x200008, 0x300000, 0x400000,
+                None) == lime.LIME_ERR_ARG                                    # unaligned
+    assert fold(ctypes.byref(dims), 0x100000, 0x200000, 0x300000, 0x100000 + 4096,
+                None) == lime.LIME_ERR_ALIAS                                  # image inside L
+    f32 = lime.make_dims(128, 4, 32, 256, 64, "f32")
+    assert fold(ctypes.byref(f32), 0x100000, 0x200000, 0x300000, 0x400000,
+                None) == lime.LIME_ERR_SHAPE
+    nws = lime.lime_workspace_bytes(dims, 0, 0)
+    g = lime._lib.lime_build_qk_cache_folded
+    assert g(ctypes.byref(dims), 0x100000, 10, 0x200000, 0x200000 + 256, 0x1000000, nws,
+             None) == lime.LIME_ERR_ALIAS                                     # cache over image
+    assert g(ctypes.byref(dims), 0x100000, 10, 0x1000000, 0x300000, 0x1000000, nws,
+             None) == lime.LIME_ERR_ALIAS                                     # image in ws
+    assert g(ctypes.byref(dims), 0x100000, 10, None, 0x300000, 0x1000000, nws,
+             None) == lime.LIME_ERR_ARG
+    assert g(ctypes.byref(dims), 0x100000, -1, 0x200000, 0x300000, 0x1000000, nws,
+             None) == lime.LIME_ERR_ARG
+    assert g(ctypes.byref(dims), 0x100000, 10, 0x200000, 0x300000, 0x1000000, 64,
+             None) == lime.LIME_ERR_ARG                                       # ws too small

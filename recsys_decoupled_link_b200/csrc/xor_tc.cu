@@ -11,31 +11,30 @@
 // work on a few rows.  History rows (the O(N) part) use bf16 operands with
 // fp32 accumulation, statistics and residual adds.  History rows are cut into
 // per-user tiles of 128 rows (a tile never spans two users; its tail rows are
-// masked).
+// masked).  The query/key products are folded per user through the link
+// rows (Q_E K_Z^T = X^ (Wq K_Z^T), Q_Z K_E^T = (Q_Z Wk^T) X^^T, P V_Z Wo =
+// P (V_Z Wo) per head), so Q_E and K_E are never formed.
 //
 //   k_prep_weights   layer weights -> K-major 128B-swizzled images (W^T); its
 //                    block 0 turns hist_offsets into the tile list (user,
 //                    first row, valid rows)
 //   k_link_proj      LN1(Z) -> Q_Z, K_Z, V_Z (split precision) -> per-user
-//                    operand images: s·K_Z, V_Z^T and s·Q_Z (hi + lo); one
-//                    CTA per (128 link rows, Q|K|V)
-//   k_hist_proj      LN1(E) (split precision) -> Q_E, K_E, V_E (row-major)
-//   k_hist_attn      history branch: softmax over the user's l links, P·V_Z,
-//                    then (P·V_Z)·Wo -> Yd (fp32 attention delta);
-//                    link branch: s·Q_Z laid out block-diagonally over heads
-//                    (expanded on chip) so that one MMA yields the scores
-//                    transposed (links on TMEM lanes); per tile and (head,
-//                    link) the partial softmax statistics (max, sum) and the
-//                    weighted V sum (V_E read as an MN-major operand)
+//                    folded images G = s Wq K_Z^T (transposed), Q' = s Q_Z
+//                    Wk^T (hi + lo) and VO = V_Z Wo, per head; one CTA per
+//                    (128 link rows, image)
+//   k_hist_xattn     LN1(E) -> history scores X^ G, softmax over l, Yd = P VO
+//                    (fp32 attention delta); link scores Q' X^^T (transposed:
+//                    (head, link) on the TMEM lanes), V_E = X^ Wv, per tile
+//                    and (head, link) the partial softmax statistics (max,
+//                    sum) and the weighted V_E sum
 //   k_hist_ffn       Y = E + Yd, LN2, GatedMLP in 64-wide chunks, E' = Y + ·
 //                    (warp-specialized pipeline)
 //   k_link_tail      per 128 link rows, a cluster of four CTAs: log-sum-exp
 //                    merge of the tile partials -> b, Y_Z = Z + b·Wo, LN2,
 //                    GatedMLP (one hidden chunk per CTA, split precision),
 //                    Z' = Y_Z + sum of the chunks
-// The last layer (E_out = NULL) skips everything only E' needs: Q_E, the
-// history branch, Wo on history rows and k_hist_ffn; its link branch runs in
-// k_hist_link, which keeps K_E and V_E on chip.
+// The last layer (E_out = NULL) skips everything only E' needs: G, VO, the
+// history branch of k_hist_xattn and k_hist_ffn.
 //
 // Kernels use 512 threads (thread (row, part): a TMEM lane and a quarter of
 // the row's columns) or warp-specialized roles; one thread issues the MMAs.
@@ -58,7 +57,7 @@ constexpr int kRec = 36;  // floats per link-branch record: max, sum, 32 weighte
 struct LayerWs {
   size_t img_q, img_k, img_v, img_o, img_13, img_2;
   size_t sched, tiles, tile_start;
-  size_t qe, ke, ve, yd, uimg, part;
+  size_t yd, uimg, part;
   size_t total;
   int64_t max_tiles;
   uint32_t uimg_bytes;
@@ -66,11 +65,8 @@ struct LayerWs {
 
 __host__ __device__ constexpr size_t up1k(size_t x) { return (x + 1023) & ~(size_t)1023; }
 
-__host__ __device__ constexpr uint32_t kz_bytes(int l) { return (uint32_t)l * 256; }  // [l x 128] bf16
-__host__ __device__ constexpr uint32_t uimg_bytes(int l) {
-  return (uint32_t)up1k(kz_bytes(l) + kBlk + 2 * kz_bytes(l));   // KZ, VZT, QZ hi, QZ lo
-}
-__host__ __device__ constexpr uint32_t qz_off(int l) { return kz_bytes(l) + kBlk; }
+// per-user folded images: G^T, Q' hi, Q' lo, VO ([128 x 128] bf16 each)
+constexpr uint32_t kUimgBytes = 8 * kBlk;
 
 LayerWs layer_ws(int l, int64_t B, int64_t nh) {
   LayerWs w;
@@ -86,11 +82,8 @@ LayerWs layer_ws(int l, int64_t B, int64_t nh) {
   w.sched = take(16);
   w.tiles = take((size_t)w.max_tiles * 16);
   w.tile_start = take((size_t)(B + 1) * 4);
-  w.qe = take((size_t)nh * kD * 2);
-  w.ke = take((size_t)nh * kD * 2);
-  w.ve = take((size_t)nh * kD * 2);
   w.yd = take((size_t)nh * kD * 4);   // fp32 attention delta
-  w.uimg_bytes = uimg_bytes(l);
+  w.uimg_bytes = kUimgBytes;
   w.uimg = take((size_t)B * w.uimg_bytes);
   w.part = take((size_t)w.max_tiles * kH * l * kRec * 4);
   w.total = o;
@@ -214,31 +207,6 @@ __device__ __forceinline__ void split_row_st(uint8_t* hi, uint8_t* lo, uint32_t 
     }
     sw_st16(hi, blk, row, c * 8, pack8(h));
     sw_st16(lo, blk, row, c * 8, pack8(r));
-  }
-}
-
-// Expands the compact s·Q_Z image (hi [L x 128] then lo, blocks of L*128
-// bytes, bulk-loaded to the start of `qbd`) in place into the block-diagonal
-// operands: qbd (hi) and qbd + 2*kBlk (lo), [128 rows x 128] each, row h*L + k
-// = s·Q_Z[k] in head h's 32 columns and zeros elsewhere, rows >= 4L zero.
-// All 512 threads: thread (row p, part) writes row p's columns part*32..+31;
-// the thread with part == h(p) first reads its 32 compact values.
-template <int L>
-__device__ __forceinline__ void expand_qbd(uint8_t* qbd, int p, int part) {
-  const bool mine = p < kH * L && p / L == part;
-  const int k = p % L;
-  uint4 hv[4], lv[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    hv[q] = mine ? sw_ld16(qbd, (uint32_t)L * 128, k, part * 32 + q * 8) : make_uint4(0, 0, 0, 0);
-    lv[q] = mine ? sw_ld16(qbd + kz_bytes(L), (uint32_t)L * 128, k, part * 32 + q * 8)
-                 : make_uint4(0, 0, 0, 0);
-  }
-  __syncthreads();
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    sw_st16(qbd, kBlk, p, part * 32 + q * 8, hv[q]);
-    sw_st16(qbd + 2 * kBlk, kBlk, p, part * 32 + q * 8, lv[q]);
   }
 }
 
@@ -448,36 +416,47 @@ __device__ void schedule_tiles(const int64_t* __restrict__ off, int64_t B, int64
 }
 
 // ----------------------------------------------------- link projections
-// Per-user operand images (at uimg + u * uimg_bytes, ℓ = L):
-//   KZ   [L rows x 128] bf16, 2 blocks of L*128 bytes:  s·K_Z
-//   VZT  [128 rows (c) x 64 cols (k)] bf16, 1 block:     V_Z^T, k >= L zero
-//   QZ   [L rows x 128] bf16, 2 blocks of L*128 bytes, twice: s·Q_Z as the hi
-//        and lo bf16 halves of the fp32 value (the link query is one vector
-//        per link, so its rounding is not averaged).  The attention kernels
-//        expand it in shared memory to the block-diagonal [128 x 128] operand
-//        (row h*L + k = s·Q_Z[k] in head h's columns, zeros elsewhere).
+// Per-user operand images, at uimg + u * uimg_bytes: four [128 rows x 128]
+// bf16 K-major 128B-swizzled images of two kBlk blocks each.  Row p = h*L + k
+// is (head h, link k); rows p >= H*L are never written and only ever reach
+// MMA output rows that nothing reads.
+//   G      [0, 2 kBlk)     G^T[p]  = s K_Z[k, h] Wq[:, h]^T      (h: head h's 32 columns)
+//   QH, QL [2, 6 kBlk)     Q'[p]   = s Q_Z[k, h] Wk[:, h]^T as bf16 hi + lo
+//   VO     [6, 8 kBlk)     VO[p]   = V_Z[k, h] Wo[h, :]          (Wo's rows of head h)
+// By associativity the history scores are Q_E,h (s K_Z,h)^T = X^ G_h, the
+// link scores (s Q_Z,h) K_E,h^T = Q'_h X^^T and the history branch through
+// Wo is (P_h V_Z,h) Wo_h = P_h VO_h (X^ = LN1(E)), so the history kernel
+// needs neither Q_E nor K_E (and the link branch keeps V_E on chip).
+//
+// CTA (128 link rows, which): which = 0 -> Q' (hi + lo), 1 -> G, 2 -> VO.
+// LN1(Z) (split) -> projection P = X^z Wm -> s P (which < 2) split hi + lo ->
+// per head h the fold P[:, h] B_h (K = 32, four MMAs per half) with B_h =
+// Wk's, Wq's or Wo's head-h slice of its weight image -> rows h*L + k of the
+// users' images, written straight from the TMEM lanes.  512 threads: thread
+// (row, part) owns columns part*32 .. part*32+31, i.e. head `part`.
 template <int L>
 __global__ void __launch_bounds__(512)
     k_link_proj(const bf16* __restrict__ Z, int64_t nrows, const bf16* __restrict__ g1,
-                const bf16* __restrict__ b1, const uint8_t* __restrict__ ws_c,
-                uint8_t* __restrict__ ws, LayerWs Lw, float scale, unsigned* status) {
-  // CTA (tile, which): which = 0 -> Q_Z (block-diagonal image), 1 -> K_Z, 2 -> V_Z^T.
-  // 512 threads: thread (row, part) owns columns part*32 .. part*32+31.
+                const bf16* __restrict__ b1, uint8_t* __restrict__ ws, LayerWs Lw, float scale,
+                unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
   uint8_t* sAh = sm;
   uint8_t* sAl = sm + 2 * kBlk;
-  uint8_t* sW = sm + 4 * kBlk;
-  float* red = reinterpret_cast<float*>(sm + 6 * kBlk);
+  uint8_t* sW = sm + 4 * kBlk;    // projection weight image (W^T, K-major)
+  uint8_t* sF = sm + 6 * kBlk;    // fold weight image
+  float* red = reinterpret_cast<float*>(sm + 8 * kBlk);
   const int which = blockIdx.y;
   Cta c;
-  cta_setup(sm + 6 * kBlk + kLnBytes, 2, c, 128);
+  cta_setup(sm + 8 * kBlk + kLnBytes, 2, c, 512);
   ln_stage(red + 1024, g1, b1);
   uint32_t mph = 0;
   if (threadIdx.x == 0) {
     const size_t img = which == 0 ? Lw.img_q : which == 1 ? Lw.img_k : Lw.img_v;
-    mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
-    bulk_load(sW, ws_c + img, 2 * kBlk, &c.bar[0]);
+    const size_t fold = which == 0 ? Lw.img_k : which == 1 ? Lw.img_q : Lw.img_o;
+    mbar_arrive_expect_tx(&c.bar[0], 4 * kBlk);
+    bulk_load(sW, ws + img, 2 * kBlk, &c.bar[0]);
+    bulk_load(sF, ws + fold, 2 * kBlk, &c.bar[0]);
   }
   const int warp = threadIdx.x >> 5;
   const int part = warp >> 2;
@@ -496,17 +475,7 @@ __global__ void __launch_bounds__(512)
       for (int i2 = 0; i2 < 32; ++i2) x[i2] = 0.f;
     }
     layer_norm_part(x, c0, red, part, r);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float h8[8], l8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        h8[k] = __bfloat162float(__float2bfloat16_rn(x[q * 8 + k]));
-        l8[k] = x[q * 8 + k] - h8[k];
-      }
-      sw_st16(sAh, kBlk, r, c0 + q * 8, pack8(h8));
-      sw_st16(sAl, kBlk, r, c0 + q * 8, pack8(l8));
-    }
+    split_part_st(sAh, sAl, r, c0, x);
   }
   fence_proxy_async_smem();
   __syncthreads();
@@ -517,281 +486,199 @@ __global__ void __launch_bounds__(512)
     mma_tile(c.tmem, smem_u32(sAl), kBlk, smem_u32(sW), kBlk, 128, 128, true);
   }
   cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-  float v[32];
-  tmem_ld16(quad_addr(c) + c0, v);          // warp-collective: every thread loads
-  tmem_ld16(quad_addr(c) + c0 + 16, v + 16);
-  tmem_ld_wait();
-  if (which != 2) {
+  const uint32_t ta = quad_addr(c);
+  {
+    // the projection (scaled for the score operands) becomes the fold's A
+    // operand, split hi + lo over the MMA operands it came from
+    float v[32];
+    tmem_ld16(ta + c0, v);
+    tmem_ld16(ta + c0 + 16, v + 16);
+    tmem_ld_wait();
+    if (which != 2) {
 #pragma unroll
-    for (int i2 = 0; i2 < 32; ++i2) v[i2] *= scale;
-  }
-  float lo[32];
-  if (which == 0) {         // the link query is kept as hi + lo bf16 halves
-#pragma unroll
-    for (int i2 = 0; i2 < 32; ++i2) {
-      const float x = v[i2];
-      v[i2] = __bfloat162float(__float2bfloat16_rn(x));
-      lo[i2] = x - v[i2];
+      for (int i2 = 0; i2 < 32; ++i2) v[i2] *= scale;
     }
+    split_part_st(sAh, sAl, r, c0, v);
   }
-  // The images are built per user in shared memory (the operands of the MMA
-  // are dead) and written out with one bulk copy per user.  Piece per user:
-  // s·K_Z (L*256 bytes), V_Z^T (one 16 KB block) or s·Q_Z hi + lo (2 x L*256).
-  constexpr int UP = kTile / L;                               // users per tile
-  const uint32_t piece = which == 0 ? 2 * kz_bytes(L) : which == 1 ? kz_bytes(L) : kBlk;
-  const uint32_t img_off = which == 0 ? qz_off(L) : which == 1 ? 0 : kz_bytes(L);
-  const int upp = which == 2 ? (UP < 4 ? UP : 4) : UP;       // users per pass
-  uint8_t* stage = sm;                                        // 96 KB: sAh, sAl, sW
-  const int ju = r / L, k = r % L;
-  const int64_t u0 = (int64_t)blockIdx.x * UP;
-  const int n_users = (int)((nrows - (int64_t)blockIdx.x * kTile) / L) < UP
-                          ? (int)((nrows - (int64_t)blockIdx.x * kTile) / L) : UP;
-  for (int j0 = 0; j0 < n_users; j0 += upp) {
-    if (threadIdx.x == 0) bulk_wait_read<0>();   // the previous pass's copies have read it
-    __syncthreads();   // the staging area is free (MMA operands, previous pass)
-    if (ju >= j0 && ju < j0 + upp && valid) {
-      uint8_t* img = stage + (uint32_t)(ju - j0) * piece;
-      if (which == 1) {           // s·K_Z row k
-#pragma unroll
-        for (int q = 0; q < 4; ++q) sw_st16(img, (uint32_t)L * 128, k, c0 + q * 8, pack8(v + q * 8));
-      } else if (which == 2) {    // V_Z^T column k; columns k + L, k + 2L, ... < 64 are zero
-        for (int cc = 0; cc < 32; ++cc) {
-          *reinterpret_cast<bf16*>(img + sw128_offset(c0 + cc, k)) = __float2bfloat16_rn(v[cc]);
-          for (int kp = k + L; kp < 64; kp += L)
-            *reinterpret_cast<bf16*>(img + sw128_offset(c0 + cc, kp)) = __float2bfloat16_rn(0.f);
-        }
-      } else {                    // s·Q_Z row k, hi then lo
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          sw_st16(img, (uint32_t)L * 128, k, c0 + q * 8, pack8(v + q * 8));
-          sw_st16(img + kz_bytes(L), (uint32_t)L * 128, k, c0 + q * 8, pack8(lo + q * 8));
-        }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    tc_fence_after();
+    for (int h = 0; h < kH; ++h) {
+      const uint32_t d = c.tmem + h * 128;
+      const uint32_t ah = smem_u32(sAh) + (h >> 1) * kBlk + (h & 1) * 64;
+      const uint32_t al = smem_u32(sAl) + (h >> 1) * kBlk + (h & 1) * 64;
+      if (which == 2) {
+        // B[n][k'] = Wo[32h + k'][n]: Wo^T's image with a K offset of 32h
+        const uint32_t b = smem_u32(sF) + (h >> 1) * kBlk + (h & 1) * 64;
+        mma_tile(d, ah, kBlk, b, kBlk, 128, kDH, false);
+        mma_tile(d, al, kBlk, b, kBlk, 128, kDH, true);
+      } else {
+        // B[n][k'] = W[n][32h + k']: rows 32h .. of W^T's image read MN-major
+        const uint32_t b = smem_u32(sF) + h * kDH * 128;
+        mma_tile_bmn(d, ah, kBlk, b, kBlk, 128, kDH, false);
+        mma_tile_bmn(d, al, kBlk, b, kBlk, 128, kDH, true);
       }
     }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      const int nu = n_users - j0 < upp ? n_users - j0 : upp;
-      for (int j = 0; j < nu; ++j)
-        bulk_store(ws + Lw.uimg + (size_t)(u0 + j0 + j) * Lw.uimg_bytes + img_off,
-                   stage + (uint32_t)j * piece, piece);
-      bulk_commit();
+  }
+  cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+  const int64_t u = R / L;
+  const int k = (int)(R % L);
+  uint8_t* img = ws + Lw.uimg + (size_t)u * Lw.uimg_bytes + (which == 0 ? 2 * kBlk : which == 1 ? 0 : 6 * kBlk);
+  for (int h = 0; h < kH; ++h) {
+    float v[32];
+    tmem_ld16(ta + h * 128 + c0, v);        // warp-collective: every thread loads
+    tmem_ld16(ta + h * 128 + c0 + 16, v + 16);
+    tmem_ld_wait();
+    if (!valid) continue;
+    const int p = h * L + k;
+    if (which == 0) {
+      split_part_st(img, img + 2 * kBlk, p, c0, v);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sw_st16(img, kBlk, p, c0 + q * 8, pack8(v + q * 8));
     }
   }
-  if (threadIdx.x == 0) bulk_wait<0>();   // the images are complete before the CTA exits
   cta_teardown(c);
 }
 
-// ----------------------------------------------------- history projections
-// One persistent CTA per SM walks the tile list.  For each tile: TMA the 128
-// history rows, LN1, Q/K/V = X^·W on the tensor cores (X^ as hi + lo bf16);
-// the outputs go through swizzled staging tiles: a full tile (128 valid rows)
-// leaves with TMA tensor stores that overlap the next steps, a partial tile
-// (its rows end at a user boundary) with coalesced plain stores of its valid
-// rows.  The next tile's rows are loaded while this tile's outputs are
-// written.  512 threads: thread (row, part) handles a quarter of the row's
-// columns; LN1's statistics are reduced across the four parts.
+// --------------------------------------------------------- XOR attention
+// One persistent CTA per SM walks the tile list.  Per 128-row history tile
+// (a tile never spans two users; rows past `nv` are masked):
+//   LN1      X^ = LN1(E) as bf16 hi (over the E tile) + lo
+//   phase 1  S = X^hi G (history scores, TMEM [0, H*L)),
+//            S'^T = Q'hi X^hi^T + Q'lo X^hi^T (link scores with (head, link)
+//            on the TMEM lanes, [128, 256)), V_E = X^ Wv (hi + lo, [256, 384))
+//   softmax  P = softmax of each head's L scores (part = head) over sP;
+//            V_E as bf16 over the G image; P2 = exp(S'^T - max) over the
+//            tile's valid rows (part = a quarter of the tokens; the lane's
+//            max and sum reduced over the parts)
+//   phase 2  Yd = P VO ([0, 128), the history branch already through Wo) and
+//            P2 V_E ([128, 256); lane (h, k) keeps head h's 32 columns)
+//   out      Yd (fp32) by TMA tensor stores (plain stores for a partial tile);
+//            the link record (max, sum, 32 weighted V sums) of each lane.
+// HIST = false (the last layer: E' is not needed) keeps the link branch only.
+//
+// Shared memory: six 32 KB slots.  Wv (resident), G -> V_E, QH -> VO, and
+// three that rotate (A, B, C): A = E tile -> X^hi -> P -> Yd staging (boxes
+// 0-1), B = X^lo -> P2 -> Yd staging (boxes 2-3), C = Q'lo -> next E tile.
+// The next tile's roles are (C, A, B).  Loads run a phase ahead: VO and the
+// next E tile as soon as phase 1 has read their slots, the next G and Q'hi
+// after phase 2, the next Q'lo once the Yd stores have read their staging.
+// 512 threads: thread (row, part), row = 32*(warp%4) + lane (a TMEM lane),
+// part = warp/4.  Thread 0 issues the loads and the MMAs.
+template <int L, bool HIST>
 __global__ void __launch_bounds__(512, 1)
-    k_hist_proj(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmQ,
-                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                const bf16* __restrict__ g1, const bf16* __restrict__ b1, uint8_t* __restrict__ ws,
-                LayerWs Lw, unsigned* status) {
+    k_hist_xattn(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
+                 const bf16* __restrict__ g1, const bf16* __restrict__ b1,
+                 uint8_t* __restrict__ ws, LayerWs Lw, unsigned* status) {
+  constexpr int HL = kH * L;
+  constexpr uint32_t kSlot = 2 * kBlk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
-  uint8_t* sE = sm;                // E tile -> LN1 output, hi half
-  uint8_t* sEl = sm + 2 * kBlk;    // LN1 output, lo half -> Q, V staging
-  uint8_t* sW = sm + 4 * kBlk;     // Wq, Wk, Wv images
-  uint8_t* sS = sm + 10 * kBlk;    // K staging
-  float* red = reinterpret_cast<float*>(sm + 12 * kBlk);
+  uint8_t* sW = sm;                 // Wv^T image
+  uint8_t* sG = sm + kSlot;         // G^T -> V_E
+  uint8_t* sQH = sm + 2 * kSlot;    // Q'hi -> VO
+  uint8_t* rot = sm + 3 * kSlot;    // three rotating slots
+  float* red = reinterpret_cast<float*>(sm + 6 * kSlot);
   Cta c;
-  cta_setup(sm + 12 * kBlk + kLnBytes, 3, c);
+  // bar: 0 Wv, 1 mma, 2 E tile, 3 G + Q'hi, 4 Q'lo, 5 VO
+  cta_setup(sm + 6 * kSlot + kLnBytes, 6, c);
   ln_stage(red + 1024, g1, b1);
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
-  uint32_t eph = 0, mph = 0;
+  float* yd = reinterpret_cast<float*>(ws + Lw.yd);
+  float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
+  auto uimg = [&](int u) { return ws + Lw.uimg + (size_t)u * Lw.uimg_bytes; };
+  auto load_e = [&](uint8_t* dst, int r0) {
+    mbar_arrive_expect_tx(&c.bar[2], kSlot);
+    tma_load_2d(dst, &tmE, 0, r0, &c.bar[2]);
+    tma_load_2d(dst + kBlk, &tmE, 64, r0, &c.bar[2]);
+  };
+  auto load_gq = [&](int u) {
+    mbar_arrive_expect_tx(&c.bar[3], HIST ? 2 * kSlot : kSlot);
+    if (HIST) bulk_load(sG, uimg(u), kSlot, &c.bar[3]);
+    bulk_load(sQH, uimg(u) + 2 * kBlk, kSlot, &c.bar[3]);
+  };
+  auto load_ql = [&](uint8_t* dst, int u) {
+    mbar_arrive_expect_tx(&c.bar[4], kSlot);
+    bulk_load(dst, uimg(u) + 4 * kBlk, kSlot, &c.bar[4]);
+  };
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmE);
-    prefetch_tmap(&tmQ);
-    prefetch_tmap(&tmK);
-    prefetch_tmap(&tmV);
-    mbar_arrive_expect_tx(&c.bar[2], 6 * kBlk);
-    bulk_load(sW, ws + Lw.img_q, 2 * kBlk, &c.bar[2]);
-    bulk_load(sW + 2 * kBlk, ws + Lw.img_k, 2 * kBlk, &c.bar[2]);
-    bulk_load(sW + 4 * kBlk, ws + Lw.img_v, 2 * kBlk, &c.bar[2]);
+    if (HIST) prefetch_tmap(&tmY);
+    mbar_arrive_expect_tx(&c.bar[0], kSlot);
+    bulk_load(sW, ws + Lw.img_v, kSlot, &c.bar[0]);
     if ((int)blockIdx.x < n_tiles) {
       const int4 tl = tiles[blockIdx.x];
-      mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
-      tma_load_2d(sE, &tmE, 0, tl.y, &c.bar[0]);
-      tma_load_2d(sE + kBlk, &tmE, 64, tl.y, &c.bar[0]);
+      load_e(rot, tl.y);
+      load_gq(tl.x);
+      load_ql(rot + 2 * kSlot, tl.x);
     }
   }
-  mbar_wait(&c.bar[2], 0, status, c.abort_flag);
   const int warp = threadIdx.x >> 5;
   const int part = warp >> 2;
   const int row = (warp & 3) * 32 + (threadIdx.x & 31);
   const int c0 = part * 32;
   const uint32_t ta = quad_addr(c);
-  for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+  uint32_t mph = 0;
+  int ia = 0;   // slot ia = A, (ia+1)%3 = B, (ia+2)%3 = C
+  for (int t = blockIdx.x, it = 0; t < n_tiles; t += gridDim.x, ++it) {
     const int4 tl = tiles[t];
-    const int r0 = tl.y, nv = tl.z;
-    // the previous tile's tensor stores have read the staging tiles (the LN
-    // barriers below pass this on to every thread before sEl is rewritten)
-    if (threadIdx.x == 0) bulk_wait_read<0>();
-    mbar_wait(&c.bar[0], eph, status, c.abort_flag);
-    eph ^= 1u;
+    const int u = tl.x, r0 = tl.y, nv = tl.z;
+    const int tn = t + gridDim.x;
+    const uint32_t ph = (uint32_t)it & 1u;
+    uint8_t* sA = rot + ia * kSlot;
+    uint8_t* sB = rot + (ia == 2 ? 0 : ia + 1) * kSlot;
+    uint8_t* sC = rot + (ia == 0 ? 2 : ia - 1) * kSlot;
+    if (threadIdx.x == 0 && it > 0) {
+      // the previous tile's Yd stores have read A's and B's old contents (this
+      // tile's B and C); LN1's first barrier passes this on before B is written
+      bulk_wait_read<0>();
+      load_ql(sC, u);
+    }
+    mbar_wait(&c.bar[2], ph, status, c.abort_flag);
     {
-      // LN1 output as hi + lo bf16 halves: K_E and V_E feed the link branch,
-      // whose softmax over a short history does not average rounding away
       float x[32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sE, kBlk, row, c0 + q * 8), x + q * 8);
+      for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sA, kBlk, row, c0 + q * 8), x + q * 8);
       layer_norm_part(x, c0, red, part, row);
-      split_part_st(sE, sEl, row, c0, x);
+      split_part_st(sA, sB, row, c0, x);
     }
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {
+      if (it == 0) mbar_wait(&c.bar[0], 0, status, c.abort_flag);
+      mbar_wait(&c.bar[3], ph, status, c.abort_flag);
+      mbar_wait(&c.bar[4], ph, status, c.abort_flag);
       tc_fence_after();
-      for (int w = 0; w < 3; ++w) {
-        const uint32_t d = c.tmem + w * 128;
-        mma_tile(d, smem_u32(sE), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128, 128, false);
-        mma_tile(d, smem_u32(sEl), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128, 128, true);
-      }
+      if (HIST) mma_tile(c.tmem, smem_u32(sA), kBlk, smem_u32(sG), kBlk, HL, 128, false);
+      mma_tile(c.tmem + 128, smem_u32(sQH), kBlk, smem_u32(sA), kBlk, 128, 128, false);
+      mma_tile(c.tmem + 128, smem_u32(sC), kBlk, smem_u32(sA), kBlk, 128, 128, true);
+      mma_tile(c.tmem + 256, smem_u32(sA), kBlk, smem_u32(sW), kBlk, 128, 128, false);
+      mma_tile(c.tmem + 256, smem_u32(sB), kBlk, smem_u32(sW), kBlk, 128, 128, true);
     }
     cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    const int tn = t + gridDim.x;
-    if (threadIdx.x == 0 && tn < n_tiles) {
-      const int4 tl2 = tiles[tn];
-      mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk);
-      tma_load_2d(sE, &tmE, 0, tl2.y, &c.bar[0]);
-      tma_load_2d(sE + kBlk, &tmE, 64, tl2.y, &c.bar[0]);
-    }
-    // Q_E -> sEl, K_E -> sS, V_E -> sEl (once Q's store has read it)
-    const bool full = nv == kTile;
-    for (int mtx = 0; mtx < 3; ++mtx) {
-      uint8_t* buf = mtx == 1 ? sS : sEl;
-      if (mtx == 2) {
-        if (full && threadIdx.x == 0) bulk_wait_read<1>();
-        __syncthreads();
+    // phase 1 has read Q'hi and Q'lo: VO and the next E tile come in now
+    if (threadIdx.x == 0) {
+      if (HIST) {
+        mbar_arrive_expect_tx(&c.bar[5], kSlot);
+        bulk_load(sQH, uimg(u) + 6 * kBlk, kSlot, &c.bar[5]);
       }
+      if (tn < n_tiles) load_e(sC, tiles[tn].y);
+    }
+    {
+      // V_E (bf16) over the G image: the MN-major B operand of P2 V_E
       float v[32];
-      tmem_ld16(ta + mtx * 128 + c0, v);
-      tmem_ld16(ta + mtx * 128 + c0 + 16, v + 16);
+      tmem_ld16(ta + 256 + c0, v);
+      tmem_ld16(ta + 256 + c0 + 16, v + 16);
       tmem_ld_wait();
 #pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(buf, kBlk, row, c0 + q * 8, pack8(v + q * 8));
-      fence_proxy_async_smem();
-      __syncthreads();
-      if (full) {
-        if (threadIdx.x == 0) {
-          const CUtensorMap* tm = mtx == 0 ? &tmQ : mtx == 1 ? &tmK : &tmV;
-          tma_store_2d(tm, buf, 0, r0);
-          tma_store_2d(tm, buf + kBlk, 64, r0);
-          bulk_commit();
-        }
-      } else {
-        const size_t off = mtx == 0 ? Lw.qe : mtx == 1 ? Lw.ke : Lw.ve;
-        tile_store_rows(buf, reinterpret_cast<bf16*>(ws + off) + (int64_t)r0 * kD, nv);
-      }
+      for (int q = 0; q < 4; ++q) sw_st16(sG, kBlk, row, c0 + q * 8, pack8(v + q * 8));
     }
-    tc_fence_before();
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) bulk_wait<0>();
-  cta_teardown(c);
-}
-
-// --------------------------------------------------------- XOR attention
-// 512 threads: thread (row, part) with row = 32*(warp%4) + lane (a TMEM lane)
-// and part = warp/4, a quarter of the row's columns (or of the tile's tokens
-// for the link branch).  Thread 0 issues the MMAs and the loads.  Loads are
-// issued a tile ahead where the buffers allow: the next tile's V_E and user
-// images as soon as phase 2 has consumed this tile's, its Q_E and K_E once
-// this tile's delta has left the staging area.  Full tiles store the fp32
-// delta with TMA tensor stores.
-template <int L>
-__global__ void __launch_bounds__(512, 1)
-    k_hist_attn(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmY,
-                uint8_t* __restrict__ ws, LayerWs Lw, unsigned* status) {
-  constexpr int HL = kH * L;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = align1k(smem_raw);
-  uint8_t* sQ = sm;                 // Q_E -> P -> A_E (hi); with sK: fp32 delta staging
-  uint8_t* sK = sm + 2 * kBlk;      // K_E -> P2 -> A_E (lo)
-  uint8_t* sV = sm + 4 * kBlk;      // V_E rows (row-major, read as an MN-major operand)
-  uint8_t* sWo = sm + 6 * kBlk;     // Wo image
-  uint8_t* sQBD = sm + 8 * kBlk;    // block-diagonal s·Q_Z, hi then lo
-  uint8_t* sKZ = sQBD + 4 * kBlk;   // user images: s·K_Z, V_Z^T
-  uint8_t* sVZT = sKZ + kz_bytes(L);
-  float* red = reinterpret_cast<float*>(sVZT + kBlk);   // [2][4][128]
-  Cta c;
-  cta_setup(sVZT + kBlk + 4096, 4, c);   // bar: 0 Q,K  1 mma  2 Wo  3 V + user image
-  const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
-  const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
-  float* yd = reinterpret_cast<float*>(ws + Lw.yd);
-  float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
-  uint32_t qph = 0, vph = 0, mph = 0;
-  auto load_qk = [&](int r0) {
-    mbar_arrive_expect_tx(&c.bar[0], 4 * kBlk);
-    tma_load_2d(sQ, &tmQ, 0, r0, &c.bar[0]);
-    tma_load_2d(sQ + kBlk, &tmQ, 64, r0, &c.bar[0]);
-    tma_load_2d(sK, &tmK, 0, r0, &c.bar[0]);
-    tma_load_2d(sK + kBlk, &tmK, 64, r0, &c.bar[0]);
-  };
-  auto load_v_img = [&](int r0, int u, bool img) {
-    mbar_arrive_expect_tx(&c.bar[3], 2 * kBlk + (img ? 3 * kz_bytes(L) + kBlk : 0));
-    tma_load_2d(sV, &tmV, 0, r0, &c.bar[3]);
-    tma_load_2d(sV + kBlk, &tmV, 64, r0, &c.bar[3]);
-    if (img) {
-      const uint8_t* im = ws + Lw.uimg + (size_t)u * Lw.uimg_bytes;
-      bulk_load(sKZ, im, kz_bytes(L) + kBlk, &c.bar[3]);
-      bulk_load(sQBD, im + qz_off(L), 2 * kz_bytes(L), &c.bar[3]);
-    }
-  };
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&tmY);
-    mbar_arrive_expect_tx(&c.bar[2], 2 * kBlk);
-    bulk_load(sWo, ws + Lw.img_o, 2 * kBlk, &c.bar[2]);
-    if ((int)blockIdx.x < n_tiles) {
-      const int4 tl = tiles[blockIdx.x];
-      load_qk(tl.y);
-      load_v_img(tl.y, tl.x, true);
-    }
-  }
-  mbar_wait(&c.bar[2], 0, status, c.abort_flag);
-  const int warp = threadIdx.x >> 5;
-  const int part = warp >> 2;
-  const int row = (warp & 3) * 32 + (threadIdx.x & 31);
-  const uint32_t ta = quad_addr(c);
-  int cur_u = -1;
-  for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-    const int4 tl = tiles[t];
-    const int u = tl.x, r0 = tl.y, nv = tl.z;
-    const int tn = t + gridDim.x;
-    mbar_wait(&c.bar[0], qph, status, c.abort_flag);
-    qph ^= 1u;
-    mbar_wait(&c.bar[3], vph, status, c.abort_flag);
-    vph ^= 1u;
-    if (u != cur_u) {
-      expand_qbd<L>(sQBD, row, part);
-      fence_proxy_async_smem();
-      __syncthreads();
-    }
-    cur_u = u;
-    // phase 1: history scores S_h = Q_E,h (s K_Z,h)^T -> TMEM [0, HL);
-    //          link scores, transposed: S'^T = (s Q_Z)_bd K_E^T -> TMEM [128, 256)
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      for (int h = 0; h < kH; ++h)
-        mma_tile(c.tmem + h * L, smem_u32(sQ + (h >> 1) * kBlk + (h & 1) * 64), kBlk,
-                 smem_u32(sKZ + (h >> 1) * (L * 128) + (h & 1) * 64), L * 128, L, kDH, false);
-      mma_tile(c.tmem + 128, smem_u32(sQBD), kBlk, smem_u32(sK), kBlk, 128, 128, false);
-      mma_tile(c.tmem + 128, smem_u32(sQBD + 2 * kBlk), kBlk, smem_u32(sK), kBlk, 128, 128, true);
-    }
-    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    // history softmax over the user's L links: part = head
-    {
+    if (HIST) {
+      // history softmax over the user's L links: part = head, P over X^hi
       const int h = part;
       float z[L];
 #pragma unroll
@@ -807,22 +694,21 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
       for (int k = 0; k < L; ++k) z[k] *= inv;
 #pragma unroll
-      for (int q = 0; q < L / 8; ++q) sw_st16(sQ, kBlk, row, h * L + q * 8, pack8(z + q * 8));
+      for (int q = 0; q < L / 8; ++q) sw_st16(sA, kBlk, row, h * L + q * 8, pack8(z + q * 8));
     }
-    // link softmax over this tile's valid history rows; row = (head, link)
-    // lane, part = a quarter of the tile's 128 tokens.  The max and the sum
-    // are each reduced over the four parts through their own scratch (one
-    // barrier each: the next writes of either come after later barriers).
+    // link softmax over the tile's valid rows: row = (head, link) lane, part =
+    // a quarter of the tokens; P2 over X^lo.  Lanes >= H*L carry no link.
     float lm, ls;
     {
       float z[32];
-      tmem_ld16(ta + 128 + part * 32, z);
-      tmem_ld16(ta + 128 + part * 32 + 16, z + 16);
+      tmem_ld16(ta + 128 + c0, z);
+      tmem_ld16(ta + 128 + c0 + 16, z + 16);
       tmem_ld_wait();
+      const bool link = row < HL;
       float m = -INFINITY;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        if (part * 32 + j >= nv) z[j] = -INFINITY;
+        if (c0 + j >= nv || !link) z[j] = -INFINITY;
         m = fmaxf(m, z[j]);
       }
       red[part * 128 + row] = m;
@@ -831,7 +717,7 @@ __global__ void __launch_bounds__(512, 1)
       float s = 0.f;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        z[j] = part * 32 + j < nv ? __expf(z[j] - m) : 0.f;
+        z[j] = c0 + j < nv && link ? __expf(z[j] - m) : 0.f;
         s += z[j];
       }
       red[512 + part * 128 + row] = s;
@@ -839,42 +725,26 @@ __global__ void __launch_bounds__(512, 1)
       lm = m;
       ls = red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(sK, kBlk, row, part * 32 + q * 8, pack8(z + q * 8));
+      for (int q = 0; q < 4; ++q) sw_st16(sB, kBlk, row, c0 + q * 8, pack8(z + q * 8));
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    // phase 2: A_E,h = P_h V_Z,h -> TMEM [256, 384); link P2 V_E -> TMEM [384, 512)
     if (threadIdx.x == 0) {
+      if (HIST) mbar_wait(&c.bar[5], ph, status, c.abort_flag);
       tc_fence_after();
-      for (int h = 0; h < kH; ++h)
-        mma_tile(c.tmem + 256 + h * kDH,
-                 smem_u32(sQ + ((h * L) >> 6) * kBlk + ((h * L) & 63) * 2), kBlk,
-                 smem_u32(sVZT + h * kDH * 128), kBlk, kDH, L, false);
-      mma_tile_bmn(c.tmem + 384, smem_u32(sK), kBlk, smem_u32(sV), kBlk, 128, 128, false);
+      if (HIST) mma_tile_bmn(c.tmem, smem_u32(sA), kBlk, smem_u32(sQH), kBlk, 128, HL, false);
+      mma_tile_bmn(c.tmem + 128, smem_u32(sB), kBlk, smem_u32(sG), kBlk, 128, 128, false);
     }
     cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    // V_E, s·K_Z and V_Z^T are consumed (and the expanded s·Q_Z since phase
-    // 1): the next tile's V_E and, for a new user, its images come in now
-    if (threadIdx.x == 0 && tn < n_tiles) {
-      const int4 tl2 = tiles[tn];
-      load_v_img(tl2.y, tl2.x, tl2.x != u);
-    }
-    {
-      // A_E enters the Wo GEMM as hi + lo bf16 halves (sQ, sK), so the
-      // attention delta keeps close to fp32 accuracy.
-      float a[32];
-      tmem_ld16(ta + 256 + part * 32, a);
-      tmem_ld16(ta + 256 + part * 32 + 16, a + 16);
-      tmem_ld_wait();
-      split_part_st(sQ, sK, row, part * 32, a);
-    }
+    // phase 2 has read V_E and VO: the next tile's G and Q'hi come in now
+    if (threadIdx.x == 0 && tn < n_tiles) load_gq(tiles[tn].x);
     {
       // link record of row p = (h, k): part h reads head h's 32 columns
       // (warp-uniform TMEM address); rows of other heads skip the store
       float acc[kDH];
-      tmem_ld16(ta + 384 + part * kDH, acc);
-      tmem_ld16(ta + 384 + part * kDH + 16, acc + 16);
+      tmem_ld16(ta + 128 + part * kDH, acc);
+      tmem_ld16(ta + 128 + part * kDH + 16, acc + 16);
       tmem_ld_wait();
       if (row < HL && row / L == part) {
         float4* rec = reinterpret_cast<float4*>(part_rec + ((size_t)t * HL + row) * kRec);
@@ -885,219 +755,51 @@ __global__ void __launch_bounds__(512, 1)
         rec[8] = make_float4(acc[30], acc[31], 0.f, 0.f);
       }
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // phase 3: Yd = A_E Wo -> TMEM [0, 128)
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      mma_tile(c.tmem, smem_u32(sQ), kBlk, smem_u32(sWo), kBlk, 128, 128, false);
-      mma_tile(c.tmem, smem_u32(sK), kBlk, smem_u32(sWo), kBlk, 128, 128, true);
-    }
-    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    {
+    if (HIST) {
       float y[32];
-      tmem_ld16(ta + part * 32, y);
-      tmem_ld16(ta + part * 32 + 16, y + 16);
+      tmem_ld16(ta + c0, y);
+      tmem_ld16(ta + c0 + 16, y + 16);
       tmem_ld_wait();
       if (nv == kTile) {
         // full tile: four [128 x 32] fp32 boxes (128-byte swizzle), box = part
-        uint8_t* box = sQ + part * kBlk;
+        uint8_t* box = (part < 2 ? sA : sB) + (part & 1) * kBlk;
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           *reinterpret_cast<float4*>(box + row * 128 + ((q ^ (row & 7)) << 4)) =
               make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
       } else {
+        // rows 0-63 staged in A, 64-127 in B (512 bytes a row)
+        uint8_t* half = row < 64 ? sA : sB;
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          *f32_chunk(sQ, row, part * 8 + q) = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+          *f32_chunk(half, row & 63, part * 8 + q) =
+              make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
       }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (nv == kTile) {
-      if (threadIdx.x == 0) {
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (nv == kTile) {
+        if (threadIdx.x == 0) {
 #pragma unroll
-        for (int b = 0; b < 4; ++b) tma_store_2d(&tmY, sQ + b * kBlk, b * 32, r0);
-        bulk_commit();
-      }
-    } else {
-#pragma unroll 4
-      for (int q = 0; q < 8; ++q) {
-        const int idx = q * 512 + (int)threadIdx.x, r = idx >> 5, cc = idx & 31;
-        if (r < nv) reinterpret_cast<float4*>(yd + (int64_t)(r0 + r) * kD)[cc] = *f32_chunk(sQ, r, cc);
-      }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // the next tile's Q_E and K_E, once the delta's staging has been read
-    if (threadIdx.x == 0 && tn < n_tiles) {
-      bulk_wait_read<0>();
-      load_qk(tiles[tn].y);
-    }
-  }
-  if (threadIdx.x == 0) bulk_wait<0>();
-  cta_teardown(c);
-}
-
-// ------------------------------------------------ last layer: link branch
-// The last layer needs only the link rows' outputs, so the history side is
-// just the link branch, fused in one kernel that keeps K_E and V_E on chip:
-// TMA E -> LN1 (hi + lo) -> K_E, V_E = X^ Wk, X^ Wv (TMEM) -> bf16 in smem ->
-// S'^T = (s Q_Z)_bd K_E^T -> softmax over the tile's valid rows (per
-// (head, link) lane, statistics reduced over four token parts) -> P2 ->
-// P2 V_E (V_E read as an MN-major operand) -> per-tile records.
-// 512 threads: thread (row, part).  TMEM: K_E [0,128), V_E [128,256),
-// S'^T [256,384), P2 V_E [384,512).
-template <int L>
-__global__ void __launch_bounds__(512, 1)
-    k_hist_link(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ g1,
-                const bf16* __restrict__ b1, uint8_t* __restrict__ ws, LayerWs Lw,
-                unsigned* status) {
-  constexpr int HL = kH * L;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = align1k(smem_raw);
-  uint8_t* sE = sm;                // E tile -> X^ hi -> K_E -> P2
-  uint8_t* sEl = sm + 2 * kBlk;    // X^ lo -> V_E
-  uint8_t* sWk = sm + 4 * kBlk;
-  uint8_t* sWv = sm + 6 * kBlk;
-  uint8_t* sQBD = sm + 8 * kBlk;   // block-diagonal s*Q_Z, hi then lo (4 blocks)
-  float* red = reinterpret_cast<float*>(sm + 12 * kBlk);
-  Cta c;
-  cta_setup(sm + 12 * kBlk + kLnBytes, 3, c);
-  ln_stage(red + 1024, g1, b1);
-  const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
-  const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
-  float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
-  uint32_t lph = 0, mph = 0;
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(&c.bar[2], 4 * kBlk);
-    bulk_load(sWk, ws + Lw.img_k, 2 * kBlk, &c.bar[2]);
-    bulk_load(sWv, ws + Lw.img_v, 2 * kBlk, &c.bar[2]);
-  }
-  mbar_wait(&c.bar[2], 0, status, c.abort_flag);
-  const int warp = threadIdx.x >> 5;
-  const int part = warp >> 2;
-  const int row = (warp & 3) * 32 + (threadIdx.x & 31);
-  const int c0 = part * 32;
-  const uint32_t ta = quad_addr(c);
-  int cur_u = -1;
-  for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-    const int4 tl = tiles[t];
-    const int u = tl.x, r0 = tl.y, nv = tl.z;
-    if (threadIdx.x == 0) {
-      const uint32_t qz_bytes = 2 * kz_bytes(L);
-      mbar_arrive_expect_tx(&c.bar[0], 2 * kBlk + (u != cur_u ? qz_bytes : 0));
-      tma_load_2d(sE, &tmE, 0, r0, &c.bar[0]);
-      tma_load_2d(sE + kBlk, &tmE, 64, r0, &c.bar[0]);
-      if (u != cur_u)
-        bulk_load(sQBD, ws + Lw.uimg + (size_t)u * Lw.uimg_bytes + qz_off(L), qz_bytes, &c.bar[0]);
-    }
-    mbar_wait(&c.bar[0], lph, status, c.abort_flag);
-    lph ^= 1u;
-    if (u != cur_u) expand_qbd<L>(sQBD, row, part);   // ordered before the MMAs by LN1's barriers
-    cur_u = u;
-    {
-      float x[32];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sE, kBlk, row, c0 + q * 8), x + q * 8);
-      layer_norm_part(x, c0, red, part, row);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float h8[8], l8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          h8[k] = __bfloat162float(__float2bfloat16_rn(x[q * 8 + k]));
-          l8[k] = x[q * 8 + k] - h8[k];
+          for (int b = 0; b < 4; ++b) tma_store_2d(&tmY, (b < 2 ? sA : sB) + (b & 1) * kBlk, b * 32, r0);
+          bulk_commit();
         }
-        sw_st16(sE, kBlk, row, c0 + q * 8, pack8(h8));
-        sw_st16(sEl, kBlk, row, c0 + q * 8, pack8(l8));
+      } else {
+#pragma unroll 4
+        for (int q = 0; q < 8; ++q) {
+          const int idx = q * 512 + (int)threadIdx.x, r = idx >> 5, cc = idx & 31;
+          if (r < nv)
+            reinterpret_cast<float4*>(yd + (int64_t)(r0 + r) * kD)[cc] = *f32_chunk(r < 64 ? sA : sB, r & 63, cc);
+        }
       }
     }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      mma_tile(c.tmem, smem_u32(sE), kBlk, smem_u32(sWk), kBlk, 128, 128, false);
-      mma_tile(c.tmem, smem_u32(sEl), kBlk, smem_u32(sWk), kBlk, 128, 128, true);
-      mma_tile(c.tmem + 128, smem_u32(sE), kBlk, smem_u32(sWv), kBlk, 128, 128, false);
-      mma_tile(c.tmem + 128, smem_u32(sEl), kBlk, smem_u32(sWv), kBlk, 128, 128, true);
-    }
-    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    {
-      // K_E -> sE (K-major B of the score MMA), V_E -> sEl (MN-major B)
-      float v[32];
-      tmem_ld16(ta + c0, v);
-      tmem_ld16(ta + c0 + 16, v + 16);
-      tmem_ld_wait();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(sE, kBlk, row, c0 + q * 8, pack8(v + q * 8));
-      tmem_ld16(ta + 128 + c0, v);
-      tmem_ld16(ta + 128 + c0 + 16, v + 16);
-      tmem_ld_wait();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(sEl, kBlk, row, c0 + q * 8, pack8(v + q * 8));
-    }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      mma_tile(c.tmem + 256, smem_u32(sQBD), kBlk, smem_u32(sE), kBlk, 128, 128, false);
-      mma_tile(c.tmem + 256, smem_u32(sQBD + 2 * kBlk), kBlk, smem_u32(sE), kBlk, 128, 128, true);
-    }
-    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    float lm, ls;
-    {
-      float z[32];
-      tmem_ld16(ta + 256 + part * 32, z);
-      tmem_ld16(ta + 256 + part * 32 + 16, z + 16);
-      tmem_ld_wait();
-      float m = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (part * 32 + j >= nv) z[j] = -INFINITY;
-        m = fmaxf(m, z[j]);
-      }
-      m = row_max4(m, red, part, row);
-      float s = 0.f;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        z[j] = part * 32 + j < nv ? __expf(z[j] - m) : 0.f;
-        s += z[j];
-      }
-      lm = m;
-      ls = row_sum4(s, red, part, row);
-      // P2 goes into sE: K_E's last reader (the score MMA) has completed
-#pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(sE, kBlk, row, part * 32 + q * 8, pack8(z + q * 8));
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      mma_tile_bmn(c.tmem + 384, smem_u32(sE), kBlk, smem_u32(sEl), kBlk, 128, 128, false);
-    }
-    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    {
-      float acc[kDH];
-      tmem_ld16(ta + 384 + part * kDH, acc);
-      tmem_ld16(ta + 384 + part * kDH + 16, acc + 16);
-      tmem_ld_wait();
-      if (row < HL && row / L == part) {
-        float4* rec = reinterpret_cast<float4*>(part_rec + ((size_t)t * HL + row) * kRec);
-        rec[0] = make_float4(lm, ls, acc[0], acc[1]);
-#pragma unroll
-        for (int q = 1; q < 8; ++q)
-          rec[q] = make_float4(acc[4 * q - 2], acc[4 * q - 1], acc[4 * q], acc[4 * q + 1]);
-        rec[8] = make_float4(acc[30], acc[31], 0.f, 0.f);
-      }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
+    ia = ia == 0 ? 2 : ia - 1;   // next (A, B, C) = (C, A, B)
+  }
+  if (threadIdx.x == 0) {
+    // a CTA without tiles still lets its Wv load land before it exits
+    if ((int)blockIdx.x >= n_tiles) mbar_wait(&c.bar[0], 0, status, c.abort_flag);
+    bulk_wait<0>();
   }
   cta_teardown(c);
 }
@@ -1683,43 +1385,27 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     if (rc) return rc;
   }
   {
-    const int smem = 1024 + 6 * kBlk + kLnBytes + kBarBytes;   // 96 KB of it stage the images
+    // the last layer needs only Q' (its history branch is skipped)
+    const int smem = 1024 + 8 * kBlk + kLnBytes + kBarBytes;
     if (!set_smem(k_link_proj<L>, smem)) return LIME_ERR_CUDA;
-    int rc = launch_pdl(k_link_proj<L>, dim3((unsigned)((nz + kTile - 1) / kTile), 3), dim3(512),
-                        smem, st, 1, (const bf16*)Z_in, nz, (const bf16*)w.g1, (const bf16*)w.b1,
-                        (const uint8_t*)ws, ws, Lw, scale, status);
+    int rc = launch_pdl(k_link_proj<L>, dim3((unsigned)((nz + kTile - 1) / kTile), last ? 1 : 3),
+                        dim3(512), smem, st, 1, (const bf16*)Z_in, nz, (const bf16*)w.g1,
+                        (const bf16*)w.b1, ws, Lw, scale, status);
     if (rc) return rc;
   }
   if (nh > 0) {
-    CUtensorMap tmE, tmQ, tmK, tmV;
+    CUtensorMap tmE, tmY;
     if (!make_tmap_2d_bf16(&tmE, E_in, kD, (uint64_t)nh, kD * 2, 64, kTile) ||
-        !make_tmap_2d_bf16(&tmQ, ws + Lw.qe, kD, (uint64_t)nh, kD * 2, 64, kTile) ||
-        !make_tmap_2d_bf16(&tmK, ws + Lw.ke, kD, (uint64_t)nh, kD * 2, 64, kTile) ||
-        !make_tmap_2d_bf16(&tmV, ws + Lw.ve, kD, (uint64_t)nh, kD * 2, 64, kTile))
+        !make_tmap_2d_f32(&tmY, ws + Lw.yd, kD, (uint64_t)nh, kD * 4, 32, kTile))
       return LIME_ERR_CUDA;
     const int64_t tiles_hi = Lw.max_tiles;
     const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
-    if (last) {
+    {
       const int smem = 1024 + 12 * kBlk + kLnBytes + kBarBytes;
-      if (!set_smem(k_hist_link<L>, smem)) return LIME_ERR_CUDA;
-      int rc = launch_pdl(k_hist_link<L>, dim3(grid), dim3(512), smem, st, 1, tmE,
-                          (const bf16*)w.g1, (const bf16*)w.b1, ws, Lw, status);
-      if (rc) return rc;
-    } else {
-      const int smem = 1024 + 12 * kBlk + kLnBytes + kBarBytes;
-      if (!set_smem(k_hist_proj, smem)) return LIME_ERR_CUDA;
-      int rc = launch_pdl(k_hist_proj, dim3(grid), dim3(512), smem, st, 1, tmE, tmQ, tmK, tmV,
-                          (const bf16*)w.g1, (const bf16*)w.b1, ws, Lw, status);
-      if (rc) return rc;
-    }
-    if (!last) {
-      const int smem = 1024 + 12 * kBlk + kz_bytes(L) + kBlk + 4096 + kBarBytes;
-      CUtensorMap tmY;
-      if (!make_tmap_2d_f32(&tmY, ws + Lw.yd, kD, (uint64_t)nh, kD * 4, 32, kTile))
-        return LIME_ERR_CUDA;
-      if (!set_smem(k_hist_attn<L>, smem)) return LIME_ERR_CUDA;
-      int rc = launch_pdl(k_hist_attn<L>, dim3(grid), dim3(512), smem, st, 1, tmQ, tmK, tmV, tmY,
-                          ws, Lw, status);
+      auto kern = last ? k_hist_xattn<L, false> : k_hist_xattn<L, true>;
+      if (!set_smem(kern, smem)) return LIME_ERR_CUDA;
+      int rc = launch_pdl(kern, dim3(grid), dim3(512), smem, st, 1, tmE, tmY, (const bf16*)w.g1,
+                          (const bf16*)w.b1, ws, Lw, status);
       if (rc) return rc;
     }
     if (!last) {

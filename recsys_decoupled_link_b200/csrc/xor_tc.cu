@@ -148,23 +148,22 @@ __device__ __forceinline__ void ln_stage(float* gb, const bf16* g, const bf16* b
 }
 
 // LayerNorm of one row held as four 32-column parts (x = this thread's part,
-// columns c0..c0+31), affine with the staged g, b.  `red` is a kLnFloats
-// scratch (red[0..1023] for the two reductions, g and b after them); all 512
-// threads take part (two block-wide barriers).
+// columns c0..c0+31), affine with the staged g, b.  The sum and the sum of
+// squares are reduced in one pass (var = E[x^2] - mu^2 in fp32; LN inputs
+// here are O(1) with |mu| of the order of the spread, so the cancellation
+// costs a few ulp).  `red` is a kLnFloats scratch (red[0..1023] for the
+// reductions, g and b after them); all 512 threads take part (one block-wide
+// barrier; the caller's next barrier must come before red is written again).
 __device__ __forceinline__ void layer_norm_part(float* x, int c0, float* red, int part, int row) {
-  float s1 = 0.f;
+  float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-  for (int k = 0; k < 32; ++k) s1 += x[k];
+  for (int k = 0; k < 32; ++k) { s1 += x[k]; s2 = fmaf(x[k], x[k], s2); }
   red[part * 128 + row] = s1;
-  __syncthreads();
-  const float mu = (red[row] + red[128 + row] + red[256 + row] + red[384 + row]) * (1.0f / kD);
-  float s2 = 0.f;
-#pragma unroll
-  for (int k = 0; k < 32; ++k) { const float d0 = x[k] - mu; s2 += d0 * d0; }
   red[512 + part * 128 + row] = s2;
   __syncthreads();
-  const float rstd = rsqrtf((red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row]) *
-                                (1.0f / kD) + kLnEps);
+  const float mu = (red[row] + red[128 + row] + red[256 + row] + red[384 + row]) * (1.0f / kD);
+  const float ex2 = (red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row]) * (1.0f / kD);
+  const float rstd = rsqrtf(fmaxf(ex2 - mu * mu, 0.f) + kLnEps);
   const float4* g4 = reinterpret_cast<const float4*>(red + 1024 + c0);
   const float4* b4 = reinterpret_cast<const float4*>(red + 1024 + kD + c0);
 #pragma unroll
@@ -632,32 +631,39 @@ __global__ void __launch_bounds__(512, 1)
     uint8_t* sA = rot + ia * kSlot;
     uint8_t* sB = rot + (ia == 2 ? 0 : ia + 1) * kSlot;
     uint8_t* sC = rot + (ia == 0 ? 2 : ia - 1) * kSlot;
-    if (threadIdx.x == 0 && it > 0) {
-      // the previous tile's Yd stores have read A's and B's old contents (this
-      // tile's B and C); LN1's first barrier passes this on before B is written
-      bulk_wait_read<0>();
-      load_ql(sC, u);
-    }
+    // (last layer) B's old contents, P2, were read by the previous phase 2
+    if (!HIST && threadIdx.x == 0 && it > 0) load_ql(sC, u);
     mbar_wait(&c.bar[2], ph, status, c.abort_flag);
     {
       float x[32];
 #pragma unroll
       for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sA, kBlk, row, c0 + q * 8), x + q * 8);
       layer_norm_part(x, c0, red, part, row);
+      if (HIST && it > 0) {
+        // the previous tile's Yd stores have read A's and B's old contents
+        // (this tile's B and C) before B is written and Q'lo loads into C
+        if (threadIdx.x == 0) {
+          bulk_wait_read<0>();
+          load_ql(sC, u);
+        }
+        __syncthreads();
+      }
       split_part_st(sA, sB, row, c0, x);
     }
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {
+      // Q'lo (the latest load) is waited for only before its own MMA
       if (it == 0) mbar_wait(&c.bar[0], 0, status, c.abort_flag);
       mbar_wait(&c.bar[3], ph, status, c.abort_flag);
-      mbar_wait(&c.bar[4], ph, status, c.abort_flag);
       tc_fence_after();
       if (HIST) mma_tile(c.tmem, smem_u32(sA), kBlk, smem_u32(sG), kBlk, HL, 128, false);
-      mma_tile(c.tmem + 128, smem_u32(sQH), kBlk, smem_u32(sA), kBlk, 128, 128, false);
-      mma_tile(c.tmem + 128, smem_u32(sC), kBlk, smem_u32(sA), kBlk, 128, 128, true);
       mma_tile(c.tmem + 256, smem_u32(sA), kBlk, smem_u32(sW), kBlk, 128, 128, false);
       mma_tile(c.tmem + 256, smem_u32(sB), kBlk, smem_u32(sW), kBlk, 128, 128, true);
+      mma_tile(c.tmem + 128, smem_u32(sQH), kBlk, smem_u32(sA), kBlk, 128, 128, false);
+      mbar_wait(&c.bar[4], ph, status, c.abort_flag);
+      tc_fence_after();
+      mma_tile(c.tmem + 128, smem_u32(sC), kBlk, smem_u32(sA), kBlk, 128, 128, true);
     }
     cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
     // phase 1 has read Q'hi and Q'lo: VO and the next E tile come in now
@@ -739,6 +745,11 @@ __global__ void __launch_bounds__(512, 1)
     cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
     // phase 2 has read V_E and VO: the next tile's G and Q'hi come in now
     if (threadIdx.x == 0 && tn < n_tiles) load_gq(tiles[tn].x);
+    float y[32];
+    if (HIST) {
+      tmem_ld16(ta + c0, y);
+      tmem_ld16(ta + c0 + 16, y + 16);
+    }
     {
       // link record of row p = (h, k): part h reads head h's 32 columns
       // (warp-uniform TMEM address); rows of other heads skip the store
@@ -756,10 +767,6 @@ __global__ void __launch_bounds__(512, 1)
       }
     }
     if (HIST) {
-      float y[32];
-      tmem_ld16(ta + c0, y);
-      tmem_ld16(ta + c0 + 16, y + 16);
-      tmem_ld_wait();
       if (nv == kTile) {
         // full tile: four [128 x 32] fp32 boxes (128-byte swizzle), box = part
         uint8_t* box = (part < 2 ? sA : sB) + (part & 1) * kBlk;
@@ -1015,24 +1022,19 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
       tmem_st16(t_out, y);
       tmem_st16(t_out + 16, y + 16);
       {
-        float s1 = 0.f;
+        // one-pass statistics (see layer_norm_part)
+        float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s1 += y[i];
+        for (int i = 0; i < 32; ++i) { s1 += y[i]; s2 = fmaf(y[i], y[i], s2); }
         red1[part * 128 + row] = s1;
+        red2[part * 128 + row] = s2;
       }
       named_bar_sync(1, kFfnEpi);
       const float mu =
           (red1[row] + red1[128 + row] + red1[256 + row] + red1[384 + row]) * (1.0f / kD);
-      {
-        float s2 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) { const float d0 = y[i] - mu; s2 += d0 * d0; }
-        red2[part * 128 + row] = s2;
-      }
-      named_bar_sync(1, kFfnEpi);
-      const float rstd =
-          rsqrtf((red2[row] + red2[128 + row] + red2[256 + row] + red2[384 + row]) * (1.0f / kD) +
-                 kLnEps);
+      const float ex2 =
+          (red2[row] + red2[128 + row] + red2[256 + row] + red2[384 + row]) * (1.0f / kD);
+      const float rstd = rsqrtf(fmaxf(ex2 - mu * mu, 0.f) + kLnEps);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const float4 gv = reinterpret_cast<const float4*>(sg + c0)[q];

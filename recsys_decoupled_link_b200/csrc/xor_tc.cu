@@ -427,14 +427,16 @@ __device__ void schedule_tiles(const int64_t* __restrict__ off, int64_t B, int64
 // Wo is (P_h V_Z,h) Wo_h = P_h VO_h (X^ = LN1(E)), so the history kernel
 // needs neither Q_E nor K_E (and the link branch keeps V_E on chip).
 //
-// CTA (128 link rows, which): which = 0 -> Q' (hi + lo), 1 -> G, 2 -> VO.
+// CTA (128 link rows, which, z): which = 0 -> Q' (hi + lo), 1 -> G, 2 -> VO,
+// for heads z*hpc .. z*hpc + hpc - 1 (hpc = H / gridDim.z; more CTAs spread
+// the image writes, which dominate, over more SMs).
 // LN1(Z) (split) -> projection P = X^z Wm -> s P (which < 2) split hi + lo ->
-// per head h the fold P[:, h] B_h (K = 32, four MMAs per half) with B_h =
+// per head h of the CTA the fold P[:, h] B_h (K = 32, two MMAs per half), B_h =
 // Wk's, Wq's or Wo's head-h slice of its weight image -> rows h*L + k of the
-// users' images, written straight from the TMEM lanes.  512 threads: thread
+// users' images, staged and written with bulk copies.  512 threads: thread
 // (row, part) owns columns part*32 .. part*32+31, i.e. head `part`.
 template <int L>
-__global__ void __launch_bounds__(512)
+__global__ void __launch_bounds__(512, 1)
     k_link_proj(const bf16* __restrict__ Z, int64_t nrows, const bf16* __restrict__ g1,
                 const bf16* __restrict__ b1, uint8_t* __restrict__ ws, LayerWs Lw, float scale,
                 unsigned* status) {
@@ -446,6 +448,7 @@ __global__ void __launch_bounds__(512)
   uint8_t* sF = sm + 6 * kBlk;    // fold weight image
   float* red = reinterpret_cast<float*>(sm + 8 * kBlk);
   const int which = blockIdx.y;
+  const int hpc = kH / (int)gridDim.z, h0 = (int)blockIdx.z * hpc;   // this CTA's heads
   Cta c;
   cta_setup(sm + 8 * kBlk + kLnBytes, 2, c, 512);
   ln_stage(red + 1024, g1, b1);
@@ -504,8 +507,8 @@ __global__ void __launch_bounds__(512)
   __syncthreads();
   if (threadIdx.x == 0) {
     tc_fence_after();
-    for (int h = 0; h < kH; ++h) {
-      const uint32_t d = c.tmem + h * 128;
+    for (int h = h0; h < h0 + hpc; ++h) {
+      const uint32_t d = c.tmem + (h - h0) * 128;
       const uint32_t ah = smem_u32(sAh) + (h >> 1) * kBlk + (h & 1) * 64;
       const uint32_t al = smem_u32(sAl) + (h >> 1) * kBlk + (h & 1) * 64;
       if (which == 2) {
@@ -522,23 +525,54 @@ __global__ void __launch_bounds__(512)
     }
   }
   cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-  const int64_t u = R / L;
-  const int k = (int)(R % L);
-  uint8_t* img = ws + Lw.uimg + (size_t)u * Lw.uimg_bytes + (which == 0 ? 2 * kBlk : which == 1 ? 0 : 6 * kBlk);
-  for (int h = 0; h < kH; ++h) {
-    float v[32];
-    tmem_ld16(ta + h * 128 + c0, v);        // warp-collective: every thread loads
-    tmem_ld16(ta + h * 128 + c0 + 16, v + 16);
-    tmem_ld_wait();
-    if (!valid) continue;
-    const int p = h * L + k;
-    if (which == 0) {
-      split_part_st(img, img + 2 * kBlk, p, c0, v);
-    } else {
+  // The fold outputs are staged (the MMA operands are dead) in the images'
+  // own swizzled layout: lane r = j*L + k of user j lands at row r, which has
+  // the swizzle phase of its image row h*L + k, so user j's L rows of a head
+  // leave as one L*128-byte bulk copy per 64-column block.  Items are (head,
+  // half): Q' has a hi and a lo half per head; four 32 KB buffers per pass.
+  constexpr int UP = kTile / L;   // users per tile
+  const int64_t u0 = (int64_t)blockIdx.x * UP;
+  const int64_t left = nrows / L - u0;
+  const int n_users = left < UP ? (int)left : UP;
+  const int halves = which == 0 ? 2 : 1;
+  const int n_items = hpc * halves;
+  for (int i0 = 0; i0 < n_items; i0 += 4) {
+    if (i0 > 0) {
+      if (threadIdx.x == 0) bulk_wait_read<0>();
+      __syncthreads();
+    }
+    const int ni = n_items - i0 < 4 ? n_items - i0 : 4;
+    for (int i = 0; i < ni; i += halves) {
+      const int h = h0 + (i0 + i) / halves;
+      float v[32];
+      tmem_ld16(ta + (h - h0) * 128 + c0, v);
+      tmem_ld16(ta + (h - h0) * 128 + c0 + 16, v + 16);
+      tmem_ld_wait();
+      uint8_t* buf = sm + i * 2 * kBlk;
+      if (which == 0)
+        split_part_st(buf, buf + 2 * kBlk, r, c0, v);
+      else {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(img, kBlk, p, c0 + q * 8, pack8(v + q * 8));
+        for (int q = 0; q < 4; ++q) sw_st16(buf, kBlk, r, c0 + q * 8, pack8(v + q * 8));
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int i = 0; i < ni; ++i) {
+        const int h = h0 + (i0 + i) / halves;
+        const uint32_t img_off = which == 0 ? (2 + 2 * ((i0 + i) & 1)) * kBlk : which == 1 ? 0 : 6 * kBlk;
+        for (int j = 0; j < n_users; ++j) {
+          uint8_t* dst = ws + Lw.uimg + (size_t)(u0 + j) * Lw.uimg_bytes + img_off + h * L * 128;
+          const uint8_t* src = sm + i * 2 * kBlk + j * L * 128;
+          bulk_store(dst, src, L * 128);
+          bulk_store(dst + kBlk, src + kBlk, L * 128);
+        }
+      }
+      bulk_commit();
     }
   }
+  if (threadIdx.x == 0) bulk_wait<0>();   // the images are complete before the CTA exits
   cta_teardown(c);
 }
 
@@ -1390,7 +1424,8 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     // the last layer needs only Q' (its history branch is skipped)
     const int smem = 1024 + 8 * kBlk + kLnBytes + kBarBytes;
     if (!set_smem(k_link_proj<L>, smem)) return LIME_ERR_CUDA;
-    int rc = launch_pdl(k_link_proj<L>, dim3((unsigned)((nz + kTile - 1) / kTile), last ? 1 : 3),
+    int rc = launch_pdl(k_link_proj<L>, dim3((unsigned)((nz + kTile - 1) / kTile), last ? 1 : 3,
+                                             last ? 4 : 2),
                         dim3(512), smem, st, 1, (const bf16*)Z_in, nz, (const bf16*)w.g1,
                         (const bf16*)w.b1, ws, Lw, scale, status);
     if (rc) return rc;

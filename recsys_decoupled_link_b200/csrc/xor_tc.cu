@@ -52,7 +52,7 @@ namespace {
 constexpr int kD = 128, kH = 4, kDH = 32, kF = 256, kTile = 128;
 constexpr uint32_t kBlk = 128 * 128;  // bytes of one [128 rows x 64 cols] bf16 block
 constexpr float kLnEps = 1e-5f;
-constexpr int kRec = 36;  // floats per link-branch record: max, sum, 32 weighted sums, 2 pad
+constexpr int kRec = 36;  // floats per link-branch record: max, sum, 2 pad, 32 weighted sums
 
 struct LayerWs {
   size_t img_q, img_k, img_v, img_o, img_13, img_2;
@@ -793,11 +793,10 @@ __global__ void __launch_bounds__(512, 1)
       tmem_ld_wait();
       if (row < HL && row / L == part) {
         float4* rec = reinterpret_cast<float4*>(part_rec + ((size_t)t * HL + row) * kRec);
-        rec[0] = make_float4(lm, ls, acc[0], acc[1]);
+        rec[0] = make_float4(lm, ls, 0.f, 0.f);
 #pragma unroll
-        for (int q = 1; q < 8; ++q)
-          rec[q] = make_float4(acc[4 * q - 2], acc[4 * q - 1], acc[4 * q], acc[4 * q + 1]);
-        rec[8] = make_float4(acc[30], acc[31], 0.f, 0.f);
+        for (int q = 0; q < 8; ++q)
+          rec[1 + q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
       }
     }
     if (HIST) {
@@ -1203,9 +1202,12 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
   for (int q = 0; q < 4; ++q)
     zr[q] = valid ? reinterpret_cast<const uint4*>(Z + R * kD + c0)[q] : make_uint4(0, 0, 0, 0);
-  // 1. merge rows 32cr..32cr+31 (16 threads per row: 4 heads x 8-column groups)
+  // 1. merge rows 32cr..32cr+31: four threads per (row, head) pair, 8
+  //    columns each; pair p = 32h + row, so a warp reads the records of eight
+  //    consecutive links of one head (contiguous, float4-aligned)
   {
-    const int lr = threadIdx.x >> 4, sub = threadIdx.x & 15, h = sub >> 2, q = sub & 3;
+    const int pr = threadIdx.x >> 2, q = threadIdx.x & 3;
+    const int h = pr >> 5, lr = pr & 31;
     const int64_t Rm = t0 + 32 * cr + lr;
     float acc[8];
 #pragma unroll
@@ -1221,18 +1223,15 @@ __global__ void __launch_bounds__(512, 1)
       for (int t = ta_; t < tb_; t += 8) {
         // the records of up to eight tiles are loaded before any is merged
         float2 ms[8];
-        float a[8][8];
+        float4 a[8][2];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           if (t + i < tb_) {
-            const float* rec = recs + ((size_t)(t + i) * HL + h * L + k) * kRec;
+            const float4* rec =
+                reinterpret_cast<const float4*>(recs + ((size_t)(t + i) * HL + h * L + k) * kRec);
             ms[i] = *reinterpret_cast<const float2*>(rec);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float2 v = *reinterpret_cast<const float2*>(rec + 2 + q * 8 + 2 * j);
-              a[i][2 * j] = v.x;
-              a[i][2 * j + 1] = v.y;
-            }
+            a[i][0] = rec[1 + 2 * q];
+            a[i][1] = rec[2 + 2 * q];
           }
         }
 #pragma unroll
@@ -1242,8 +1241,14 @@ __global__ void __launch_bounds__(512, 1)
             const float so = M == -INFINITY ? 0.f : __expf(M - Mn);
             const float sn = __expf(ms[i].x - Mn);
             S = S * so + ms[i].y * sn;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = acc[j] * so + a[i][j] * sn;
+            acc[0] = acc[0] * so + a[i][0].x * sn;
+            acc[1] = acc[1] * so + a[i][0].y * sn;
+            acc[2] = acc[2] * so + a[i][0].z * sn;
+            acc[3] = acc[3] * so + a[i][0].w * sn;
+            acc[4] = acc[4] * so + a[i][1].x * sn;
+            acc[5] = acc[5] * so + a[i][1].y * sn;
+            acc[6] = acc[6] * so + a[i][1].z * sn;
+            acc[7] = acc[7] * so + a[i][1].w * sn;
             M = Mn;
           }
         }

@@ -270,6 +270,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
 
+// Host: the same for a 2-D fp16 tensor (128-byte swizzle; box_inner <= 64).
+bool make_tmap_2d_f16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                      uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
+
 // Host: the same for a 2-D uint8 tensor (128-byte swizzle; box_inner <= 128).
 bool make_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                      uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
@@ -445,6 +449,17 @@ __device__ __forceinline__ void tile_store_rows(const uint8_t* tile, bf16* dst, 
   for (int idx = (int)threadIdx.x; idx < 2048; idx += (int)blockDim.x) {
     const int r = idx >> 4, cc = idx & 15;
     if (r < nv) reinterpret_cast<uint4*>(dst + (int64_t)r * 128)[cc] = sw_ld16(tile, 128 * 128, r, cc * 8);
+  }
+}
+
+// 8 fp16 -> 8 floats (exact).
+__device__ __forceinline__ void unpack8_f16(uint4 v, float* f) {
+  const __half2* p = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(p[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
   }
 }
 

@@ -23,7 +23,7 @@
 //                    Wk^T (hi + lo) and VO = V_Z Wo, per head; one CTA per
 //                    (128 link rows, image)
 //   k_hist_xattn     LN1(E) -> history scores X^ G, softmax over l, Yd = P VO
-//                    (fp32 attention delta); link scores Q' X^^T (transposed:
+//                    (fp16 attention delta); link scores Q' X^^T (transposed:
 //                    (head, link) on the TMEM lanes), V_E = X^ Wv, per tile
 //                    and (head, link) the partial softmax statistics (max,
 //                    sum) and the weighted V_E sum
@@ -82,7 +82,7 @@ LayerWs layer_ws(int l, int64_t B, int64_t nh) {
   w.sched = take(16);
   w.tiles = take((size_t)w.max_tiles * 16);
   w.tile_start = take((size_t)(B + 1) * 4);
-  w.yd = take((size_t)nh * kD * 4);   // fp32 attention delta
+  w.yd = take((size_t)nh * kD * 2);   // attention delta (fp16)
   w.uimg_bytes = kUimgBytes;
   w.uimg = take((size_t)B * w.uimg_bytes);
   w.part = take((size_t)w.max_tiles * kH * l * kRec * 4);
@@ -580,27 +580,31 @@ __global__ void __launch_bounds__(512, 1)
 // One persistent CTA per SM walks the tile list.  Per 128-row history tile
 // (a tile never spans two users; rows past `nv` are masked):
 //   LN1      X^ = LN1(E) as bf16 hi (over the E tile) + lo
-//   phase 1  S = X^hi G (history scores, TMEM [0, H*L)),
-//            S'^T = Q'hi X^hi^T + Q'lo X^hi^T (link scores with (head, link)
-//            on the TMEM lanes, [128, 256)), V_E = X^ Wv (hi + lo, [256, 384))
-//   softmax  P = softmax of each head's L scores (part = head) over sP;
-//            V_E as bf16 over the G image; P2 = exp(S'^T - max) over the
-//            tile's valid rows (part = a quarter of the tokens; the lane's
-//            max and sum reduced over the parts)
-//   phase 2  Yd = P VO ([0, 128), the history branch already through Wo) and
-//            P2 V_E ([128, 256); lane (h, k) keeps head h's 32 columns)
-//   out      Yd (fp32) by TMA tensor stores (plain stores for a partial tile);
-//            the link record (max, sum, 32 weighted V sums) of each lane.
+//   MMAs     S'^T = Q'hi X^hi^T + Q'lo X^hi^T (link scores, (head, link) on
+//            the TMEM lanes, [128, 256)), V_E = X^ Wv (hi + lo, [256, 384)),
+//            S = X^hi G (history scores, [0, H*L)); each group is committed
+//            to its own barrier, so the epilogue starts on the link scores
+//            while the tensor cores finish V_E and S
+//   softmax  P2 = exp(S'^T - max) over the tile's valid rows (part = a
+//            quarter of the tokens; the lane's max and sum reduced over the
+//            parts) over X^lo; V_E as bf16 over the G image; P = softmax of
+//            each head's L scores (part = head) over X^hi
+//   MMAs     P2 V_E ([128, 256); lane (h, k) keeps head h's 32 columns) and
+//            Yd = P VO ([0, 128), the history branch already through Wo)
+//   out      the link record (max, sum, 32 weighted V sums) of each lane;
+//            Yd as fp16 by TMA tensor stores (plain stores for a partial
+//            tile); fp16 keeps 11 bits of the delta, which the residual adds
+//            to E (bf16 would cost E' up to 2^-9 |Yd|)
 // HIST = false (the last layer: E' is not needed) keeps the link branch only.
 //
 // Shared memory: six 32 KB slots.  Wv (resident), G -> V_E, QH -> VO, and
-// three that rotate (A, B, C): A = E tile -> X^hi -> P -> Yd staging (boxes
-// 0-1), B = X^lo -> P2 -> Yd staging (boxes 2-3), C = Q'lo -> next E tile.
-// The next tile's roles are (C, A, B).  Loads run a phase ahead: VO and the
-// next E tile as soon as phase 1 has read their slots, the next G and Q'hi
-// after phase 2, the next Q'lo once the Yd stores have read their staging.
-// 512 threads: thread (row, part), row = 32*(warp%4) + lane (a TMEM lane),
-// part = warp/4.  Thread 0 issues the loads and the MMAs.
+// three that rotate (A, B, C): A = E tile -> X^hi -> P -> Yd staging, B = X^lo
+// -> P2, C = Q'lo -> the next E tile; the next tile's roles are (C, A, B).
+// Every load is issued as soon as its slot's last reader has completed: the
+// next E tile and VO once the link scores are done, the next G and Q'lo once
+// P2 V_E is done, the next Q'hi once Yd is done.  512 threads: thread (row,
+// part), row = 32*(warp%4) + lane (a TMEM lane), part = warp/4.  Thread 0
+// issues the loads and the MMAs.
 template <int L, bool HIST>
 __global__ void __launch_bounds__(512, 1)
     k_hist_xattn(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
@@ -616,38 +620,35 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* rot = sm + 3 * kSlot;    // three rotating slots
   float* red = reinterpret_cast<float*>(sm + 6 * kSlot);
   Cta c;
-  // bar: 0 Wv, 1 mma, 2 E tile, 3 G + Q'hi, 4 Q'lo, 5 VO
-  cta_setup(sm + 6 * kSlot + kLnBytes, 6, c);
+  // bar: 0 Wv, 1 S' done, 2 E tile, 3 G, 4 Q'hi, 5 Q'lo, 6 VO, 7 V_E done,
+  //      8 S done, 9 P2 V_E done, 10 Yd done
+  cta_setup(sm + 6 * kSlot + kLnBytes, 11, c);
+  uint64_t* bar = c.bar;
   ln_stage(red + 1024, g1, b1);
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
-  float* yd = reinterpret_cast<float*>(ws + Lw.yd);
+  bf16* yd = reinterpret_cast<bf16*>(ws + Lw.yd);   // fp16 bits; rows copied as bytes
   float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
   auto uimg = [&](int u) { return ws + Lw.uimg + (size_t)u * Lw.uimg_bytes; };
+  auto load = [&](uint64_t* b, uint8_t* dst, const uint8_t* src) {
+    mbar_arrive_expect_tx(b, kSlot);
+    bulk_load(dst, src, kSlot, b);
+  };
   auto load_e = [&](uint8_t* dst, int r0) {
-    mbar_arrive_expect_tx(&c.bar[2], kSlot);
-    tma_load_2d(dst, &tmE, 0, r0, &c.bar[2]);
-    tma_load_2d(dst + kBlk, &tmE, 64, r0, &c.bar[2]);
-  };
-  auto load_gq = [&](int u) {
-    mbar_arrive_expect_tx(&c.bar[3], HIST ? 2 * kSlot : kSlot);
-    if (HIST) bulk_load(sG, uimg(u), kSlot, &c.bar[3]);
-    bulk_load(sQH, uimg(u) + 2 * kBlk, kSlot, &c.bar[3]);
-  };
-  auto load_ql = [&](uint8_t* dst, int u) {
-    mbar_arrive_expect_tx(&c.bar[4], kSlot);
-    bulk_load(dst, uimg(u) + 4 * kBlk, kSlot, &c.bar[4]);
+    mbar_arrive_expect_tx(&bar[2], kSlot);
+    tma_load_2d(dst, &tmE, 0, r0, &bar[2]);
+    tma_load_2d(dst + kBlk, &tmE, 64, r0, &bar[2]);
   };
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmE);
     if (HIST) prefetch_tmap(&tmY);
-    mbar_arrive_expect_tx(&c.bar[0], kSlot);
-    bulk_load(sW, ws + Lw.img_v, kSlot, &c.bar[0]);
+    load(&bar[0], sW, ws + Lw.img_v);
     if ((int)blockIdx.x < n_tiles) {
       const int4 tl = tiles[blockIdx.x];
       load_e(rot, tl.y);
-      load_gq(tl.x);
-      load_ql(rot + 2 * kSlot, tl.x);
+      if (HIST) load(&bar[3], sG, uimg(tl.x));
+      load(&bar[4], sQH, uimg(tl.x) + 2 * kBlk);
+      load(&bar[5], rot + 2 * kSlot, uimg(tl.x) + 4 * kBlk);
     }
   }
   const int warp = threadIdx.x >> 5;
@@ -655,31 +656,25 @@ __global__ void __launch_bounds__(512, 1)
   const int row = (warp & 3) * 32 + (threadIdx.x & 31);
   const int c0 = part * 32;
   const uint32_t ta = quad_addr(c);
-  uint32_t mph = 0;
   int ia = 0;   // slot ia = A, (ia+1)%3 = B, (ia+2)%3 = C
   for (int t = blockIdx.x, it = 0; t < n_tiles; t += gridDim.x, ++it) {
     const int4 tl = tiles[t];
     const int u = tl.x, r0 = tl.y, nv = tl.z;
     const int tn = t + gridDim.x;
+    const int un = tn < n_tiles ? tiles[tn].x : 0;
     const uint32_t ph = (uint32_t)it & 1u;
     uint8_t* sA = rot + ia * kSlot;
     uint8_t* sB = rot + (ia == 2 ? 0 : ia + 1) * kSlot;
     uint8_t* sC = rot + (ia == 0 ? 2 : ia - 1) * kSlot;
-    // (last layer) B's old contents, P2, were read by the previous phase 2
-    if (!HIST && threadIdx.x == 0 && it > 0) load_ql(sC, u);
-    mbar_wait(&c.bar[2], ph, status, c.abort_flag);
+    mbar_wait(&bar[2], ph, status, c.abort_flag);
     {
       float x[32];
 #pragma unroll
       for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sA, kBlk, row, c0 + q * 8), x + q * 8);
       layer_norm_part(x, c0, red, part, row);
       if (HIST && it > 0) {
-        // the previous tile's Yd stores have read A's and B's old contents
-        // (this tile's B and C) before B is written and Q'lo loads into C
-        if (threadIdx.x == 0) {
-          bulk_wait_read<0>();
-          load_ql(sC, u);
-        }
+        // the previous tile's Yd store has read its staging (this tile's B)
+        if (threadIdx.x == 0) bulk_wait_read<0>();
         __syncthreads();
       }
       split_part_st(sA, sB, row, c0, x);
@@ -687,57 +682,33 @@ __global__ void __launch_bounds__(512, 1)
     fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0) {
-      // Q'lo (the latest load) is waited for only before its own MMA
-      if (it == 0) mbar_wait(&c.bar[0], 0, status, c.abort_flag);
-      mbar_wait(&c.bar[3], ph, status, c.abort_flag);
+      if (it == 0) mbar_wait(&bar[0], 0, status, c.abort_flag);
+      mbar_wait(&bar[4], ph, status, c.abort_flag);
+      mbar_wait(&bar[5], ph, status, c.abort_flag);
       tc_fence_after();
-      if (HIST) mma_tile(c.tmem, smem_u32(sA), kBlk, smem_u32(sG), kBlk, HL, 128, false);
+      mma_tile(c.tmem + 128, smem_u32(sQH), kBlk, smem_u32(sA), kBlk, 128, 128, false);
+      mma_tile(c.tmem + 128, smem_u32(sC), kBlk, smem_u32(sA), kBlk, 128, 128, true);
+      mma_commit(&bar[1]);
       mma_tile(c.tmem + 256, smem_u32(sA), kBlk, smem_u32(sW), kBlk, 128, 128, false);
       mma_tile(c.tmem + 256, smem_u32(sB), kBlk, smem_u32(sW), kBlk, 128, 128, true);
-      mma_tile(c.tmem + 128, smem_u32(sQH), kBlk, smem_u32(sA), kBlk, 128, 128, false);
-      mbar_wait(&c.bar[4], ph, status, c.abort_flag);
-      tc_fence_after();
-      mma_tile(c.tmem + 128, smem_u32(sC), kBlk, smem_u32(sA), kBlk, 128, 128, true);
-    }
-    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    // phase 1 has read Q'hi and Q'lo: VO and the next E tile come in now
-    if (threadIdx.x == 0) {
+      mma_commit(&bar[7]);
       if (HIST) {
-        mbar_arrive_expect_tx(&c.bar[5], kSlot);
-        bulk_load(sQH, uimg(u) + 6 * kBlk, kSlot, &c.bar[5]);
+        mbar_wait(&bar[3], ph, status, c.abort_flag);
+        tc_fence_after();
+        mma_tile(c.tmem, smem_u32(sA), kBlk, smem_u32(sG), kBlk, HL, 128, false);
+        mma_commit(&bar[8]);
       }
+    }
+    mbar_wait(&bar[1], ph, status, c.abort_flag);
+    tc_fence_after();
+    // the link scores have read Q'hi and Q'lo
+    if (threadIdx.x == 0) {
+      if (HIST) load(&bar[6], sQH, uimg(u) + 6 * kBlk);
+      else if (tn < n_tiles) load(&bar[4], sQH, uimg(un) + 2 * kBlk);
       if (tn < n_tiles) load_e(sC, tiles[tn].y);
     }
-    {
-      // V_E (bf16) over the G image: the MN-major B operand of P2 V_E
-      float v[32];
-      tmem_ld16(ta + 256 + c0, v);
-      tmem_ld16(ta + 256 + c0 + 16, v + 16);
-      tmem_ld_wait();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(sG, kBlk, row, c0 + q * 8, pack8(v + q * 8));
-    }
-    if (HIST) {
-      // history softmax over the user's L links: part = head, P over X^hi
-      const int h = part;
-      float z[L];
-#pragma unroll
-      for (int q = 0; q < L / 16; ++q) tmem_ld16(ta + h * L + q * 16, z + q * 16);
-      tmem_ld_wait();
-      float m = z[0];
-#pragma unroll
-      for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
-      float s = 0.f;
-#pragma unroll
-      for (int k = 0; k < L; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
-      const float inv = 1.0f / s;
-#pragma unroll
-      for (int k = 0; k < L; ++k) z[k] *= inv;
-#pragma unroll
-      for (int q = 0; q < L / 8; ++q) sw_st16(sA, kBlk, row, h * L + q * 8, pack8(z + q * 8));
-    }
     // link softmax over the tile's valid rows: row = (head, link) lane, part =
-    // a quarter of the tokens; P2 over X^lo.  Lanes >= H*L carry no link.
+    // a quarter of the tokens.  Lanes >= H*L carry no link.
     float lm, ls;
     {
       float z[32];
@@ -764,25 +735,61 @@ __global__ void __launch_bounds__(512, 1)
       __syncthreads();
       lm = m;
       ls = red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row];
+      // P2 over X^lo, whose last reader is the V_E product
+      mbar_wait(&bar[7], ph, status, c.abort_flag);
 #pragma unroll
       for (int q = 0; q < 4; ++q) sw_st16(sB, kBlk, row, c0 + q * 8, pack8(z + q * 8));
+    }
+    {
+      // V_E (bf16) over the G image (read by S): the MN-major B of P2 V_E
+      if (HIST) mbar_wait(&bar[8], ph, status, c.abort_flag);
+      tc_fence_after();
+      float v[32];
+      tmem_ld16(ta + 256 + c0, v);
+      tmem_ld16(ta + 256 + c0 + 16, v + 16);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sw_st16(sG, kBlk, row, c0 + q * 8, pack8(v + q * 8));
+    }
+    if (HIST) {
+      // history softmax over the user's L links: part = head, P over X^hi
+      const int h = part;
+      float z[L];
+#pragma unroll
+      for (int q = 0; q < L / 16; ++q) tmem_ld16(ta + h * L + q * 16, z + q * 16);
+      tmem_ld_wait();
+      float m = z[0];
+#pragma unroll
+      for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
+      float s = 0.f;
+#pragma unroll
+      for (int k = 0; k < L; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
+      const float inv = 1.0f / s;
+#pragma unroll
+      for (int k = 0; k < L; ++k) z[k] *= inv;
+#pragma unroll
+      for (int q = 0; q < L / 8; ++q) sw_st16(sA, kBlk, row, h * L + q * 8, pack8(z + q * 8));
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x == 0) {
-      if (HIST) mbar_wait(&c.bar[5], ph, status, c.abort_flag);
       tc_fence_after();
-      if (HIST) mma_tile_bmn(c.tmem, smem_u32(sA), kBlk, smem_u32(sQH), kBlk, 128, HL, false);
       mma_tile_bmn(c.tmem + 128, smem_u32(sB), kBlk, smem_u32(sG), kBlk, 128, 128, false);
+      mma_commit(&bar[9]);
+      if (HIST) {
+        mbar_wait(&bar[6], ph, status, c.abort_flag);
+        tc_fence_after();
+        mma_tile_bmn(c.tmem, smem_u32(sA), kBlk, smem_u32(sQH), kBlk, 128, HL, false);
+        mma_commit(&bar[10]);
+      }
     }
-    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-    // phase 2 has read V_E and VO: the next tile's G and Q'hi come in now
-    if (threadIdx.x == 0 && tn < n_tiles) load_gq(tiles[tn].x);
-    float y[32];
-    if (HIST) {
-      tmem_ld16(ta + c0, y);
-      tmem_ld16(ta + c0 + 16, y + 16);
+    mbar_wait(&bar[9], ph, status, c.abort_flag);
+    tc_fence_after();
+    // P2 V_E has read V_E and P2: the next G, and the next Q'lo (the next C)
+    if (threadIdx.x == 0 && tn < n_tiles) {
+      if (HIST) load(&bar[3], sG, uimg(un));
+      load(&bar[5], sB, uimg(un) + 4 * kBlk);
     }
     {
       // link record of row p = (h, k): part h reads head h's 32 columns
@@ -800,36 +807,26 @@ __global__ void __launch_bounds__(512, 1)
       }
     }
     if (HIST) {
-      if (nv == kTile) {
-        // full tile: four [128 x 32] fp32 boxes (128-byte swizzle), box = part
-        uint8_t* box = (part < 2 ? sA : sB) + (part & 1) * kBlk;
+      mbar_wait(&bar[10], ph, status, c.abort_flag);
+      tc_fence_after();
+      // Yd has read P and VO: the next Q'hi
+      if (threadIdx.x == 0 && tn < n_tiles) load(&bar[4], sQH, uimg(un) + 2 * kBlk);
+      float y[32];
+      tmem_ld16(ta + c0, y);
+      tmem_ld16(ta + c0 + 16, y + 16);
+      tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          *reinterpret_cast<float4*>(box + row * 128 + ((q ^ (row & 7)) << 4)) =
-              make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
-      } else {
-        // rows 0-63 staged in A, 64-127 in B (512 bytes a row)
-        uint8_t* half = row < 64 ? sA : sB;
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          *f32_chunk(half, row & 63, part * 8 + q) =
-              make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
-      }
+      for (int q = 0; q < 4; ++q) sw_st16(sA, kBlk, row, c0 + q * 8, pack8_f16(y + q * 8));
       fence_proxy_async_smem();
       __syncthreads();
       if (nv == kTile) {
         if (threadIdx.x == 0) {
-#pragma unroll
-          for (int b = 0; b < 4; ++b) tma_store_2d(&tmY, (b < 2 ? sA : sB) + (b & 1) * kBlk, b * 32, r0);
+          tma_store_2d(&tmY, sA, 0, r0);
+          tma_store_2d(&tmY, sA + kBlk, 64, r0);
           bulk_commit();
         }
       } else {
-#pragma unroll 4
-        for (int q = 0; q < 8; ++q) {
-          const int idx = q * 512 + (int)threadIdx.x, r = idx >> 5, cc = idx & 31;
-          if (r < nv)
-            reinterpret_cast<float4*>(yd + (int64_t)(r0 + r) * kD)[cc] = *f32_chunk(r < 64 ? sA : sB, r & 63, cc);
-        }
+        tile_store_rows(sA, yd + (int64_t)r0 * kD, nv);
       }
     }
     tc_fence_before();
@@ -838,7 +835,7 @@ __global__ void __launch_bounds__(512, 1)
   }
   if (threadIdx.x == 0) {
     // a CTA without tiles still lets its Wv load land before it exits
-    if ((int)blockIdx.x >= n_tiles) mbar_wait(&c.bar[0], 0, status, c.abort_flag);
+    if ((int)blockIdx.x >= n_tiles) mbar_wait(&bar[0], 0, status, c.abort_flag);
     bulk_wait<0>();
   }
   cta_teardown(c);
@@ -849,7 +846,7 @@ __global__ void __launch_bounds__(512, 1)
 // time, as a warp-specialized pipeline (persistent, one CTA per SM):
 //   warps 0-15 (epilogue): warp w serves TMEM lane quadrant w % 4 (tile rows
 //     32*(w%4) ...) and column part p = w / 4 (a quarter of every row).  Per
-//     tile they form Y = E (TMA tile) + Yd (fp32 rows, prefetched into L2
+//     tile they form Y = E (TMA tile) + Yd (fp16 rows, prefetched into L2
 //     with the E tile) and store it into the tile's output accumulator OUT,
 //     so that the W2 products add the GatedMLP onto the residual in place;
 //     write h2 = LN2(Y) (statistics reduced over the four parts through
@@ -951,8 +948,8 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
         tma_load_2d(dst, &tmE, 0, tl.y, &barE[k & 1]);
         tma_load_2d(dst + kBlk, &tmE, 64, tl.y, &barE[k & 1]);
         // the tile's Yd rows into L2, for the epilogue's plain loads
-        bulk_prefetch_l2(reinterpret_cast<const float*>(ws + Lw.yd) + (int64_t)tl.y * kD,
-                         (uint32_t)tl.z * kD * 4);
+        bulk_prefetch_l2(reinterpret_cast<const __half*>(ws + Lw.yd) + (int64_t)tl.y * kD,
+                         (uint32_t)tl.z * kD * 2);
       };
       prefetch_tmap(&tmE);
       load_e(0);
@@ -1018,7 +1015,7 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
     const int row = q4 * 32 + lane;
     const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16);
     const int c0 = part * 32;                      // this thread's 32 columns of a row
-    const float* yd = reinterpret_cast<const float*>(ws + Lw.yd);
+    const __half* yd = reinterpret_cast<const __half*>(ws + Lw.yd);
     // Y(j) = E + Yd into OUT[j%2], h2(j) = LN2(Y(j)) over E tile j%2.  The
     // reduction scratch is the other E buffer: it holds h2(j-1), whose last
     // reader G(j-1, 3) has completed by the time the epilogue gets here, and
@@ -1032,12 +1029,9 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
         // Yd rows (prefetched into L2 with the E tile)
         const int4 tl = tile_of(j);
         if (row < tl.z) {
-          const float4* src = reinterpret_cast<const float4*>(yd + (int64_t)(tl.y + row) * kD + c0);
+          const uint4* src = reinterpret_cast<const uint4*>(yd + (int64_t)(tl.y + row) * kD + c0);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 v = src[q];
-            y[4 * q] = v.x; y[4 * q + 1] = v.y; y[4 * q + 2] = v.z; y[4 * q + 3] = v.w;
-          }
+          for (int q = 0; q < 4; ++q) unpack8_f16(src[q], y + q * 8);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) y[i] = 0.f;
@@ -1438,12 +1432,12 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
   if (nh > 0) {
     CUtensorMap tmE, tmY;
     if (!make_tmap_2d_bf16(&tmE, E_in, kD, (uint64_t)nh, kD * 2, 64, kTile) ||
-        !make_tmap_2d_f32(&tmY, ws + Lw.yd, kD, (uint64_t)nh, kD * 4, 32, kTile))
+        !make_tmap_2d_f16(&tmY, ws + Lw.yd, kD, (uint64_t)nh, kD * 2, 64, kTile))
       return LIME_ERR_CUDA;
     const int64_t tiles_hi = Lw.max_tiles;
     const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
     {
-      const int smem = 1024 + 12 * kBlk + kLnBytes + kBarBytes;
+      const int smem = 1024 + 12 * kBlk + kLnBytes + 128;   // 11 barriers
       auto kern = last ? k_hist_xattn<L, false> : k_hist_xattn<L, true>;
       if (!set_smem(kern, smem)) return LIME_ERR_CUDA;
       int rc = launch_pdl(kern, dim3(grid), dim3(512), smem, st, 1, tmE, tmY, (const bf16*)w.g1,

@@ -152,15 +152,19 @@ __device__ __forceinline__ void ln_stage(float* gb, const bf16* g, const bf16* b
 // squares are reduced in one pass (var = E[x^2] - mu^2 in fp32; LN inputs
 // here are O(1) with |mu| of the order of the spread, so the cancellation
 // costs a few ulp).  `red` is a kLnFloats scratch (red[0..1023] for the
-// reductions, g and b after them); all 512 threads take part (one block-wide
-// barrier; the caller's next barrier must come before red is written again).
+// reductions, g and b after them); 512 threads take part (one barrier: the
+// whole block, or named barrier 1 over threads 0-511 when NB = 512 and the
+// block has more threads; the caller's next barrier must come before red is
+// written again).
+template <int NB = 0>
 __device__ __forceinline__ void layer_norm_part(float* x, int c0, float* red, int part, int row) {
   float s1 = 0.f, s2 = 0.f;
 #pragma unroll
   for (int k = 0; k < 32; ++k) { s1 += x[k]; s2 = fmaf(x[k], x[k], s2); }
   red[part * 128 + row] = s1;
   red[512 + part * 128 + row] = s2;
-  __syncthreads();
+  if (NB) named_bar_sync(1, NB);
+  else __syncthreads();
   const float mu = (red[row] + red[128 + row] + red[256 + row] + red[384 + row]) * (1.0f / kD);
   const float ex2 = (red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row]) * (1.0f / kD);
   const float rstd = rsqrtf(fmaxf(ex2 - mu * mu, 0.f) + kLnEps);
@@ -602,11 +606,18 @@ __global__ void __launch_bounds__(512, 1)
 // -> P2, C = Q'lo -> the next E tile; the next tile's roles are (C, A, B).
 // Every load is issued as soon as its slot's last reader has completed: the
 // next E tile and VO once the link scores are done, the next G and Q'lo once
-// P2 V_E is done, the next Q'hi once Yd is done.  512 threads: thread (row,
-// part), row = 32*(warp%4) + lane (a TMEM lane), part = warp/4.  Thread 0
-// issues the loads and the MMAs.
+// P2 V_E is done, the next Q'hi once Yd is done.
+// Warps 0-15 (epilogue): thread (row, part), row = 32*(warp%4) + lane (a TMEM
+// lane), part = warp/4; they synchronise among themselves with a named
+// barrier.  Warp 16 (one lane) issues the MMAs and the loads: tcgen05.mma
+// issue stalls while the tensor pipe is busy, which would otherwise hold an
+// epilogue warp, and with it every barrier of the epilogue, until the last
+// MMA group has started.
+constexpr int kXaEpi = 512;
+constexpr int kXaThreads = kXaEpi + 32;
+
 template <int L, bool HIST>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(kXaThreads, 1)
     k_hist_xattn(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
                  const bf16* __restrict__ g1, const bf16* __restrict__ b1,
                  uint8_t* __restrict__ ws, LayerWs Lw, unsigned* status) {
@@ -621,222 +632,243 @@ __global__ void __launch_bounds__(512, 1)
   float* red = reinterpret_cast<float*>(sm + 6 * kSlot);
   Cta c;
   // bar: 0 Wv, 1 S' done, 2 E tile, 3 G, 4 Q'hi, 5 Q'lo, 6 VO, 7 V_E done,
-  //      8 S done, 9 P2 V_E done, 10 Yd done
-  cta_setup(sm + 6 * kSlot + kLnBytes, 11, c);
+  //      8 S done, 9 P2 V_E done, 10 Yd done, 11 X^ written, 12 P2, V_E, P written
+  cta_setup(sm + 6 * kSlot + kLnBytes, 13, c);
   uint64_t* bar = c.bar;
   ln_stage(red + 1024, g1, b1);
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
-  bf16* yd = reinterpret_cast<bf16*>(ws + Lw.yd);   // fp16 bits; rows copied as bytes
-  float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
-  auto uimg = [&](int u) { return ws + Lw.uimg + (size_t)u * Lw.uimg_bytes; };
-  auto load = [&](uint64_t* b, uint8_t* dst, const uint8_t* src) {
-    mbar_arrive_expect_tx(b, kSlot);
-    bulk_load(dst, src, kSlot, b);
-  };
-  auto load_e = [&](uint8_t* dst, int r0) {
-    mbar_arrive_expect_tx(&bar[2], kSlot);
-    tma_load_2d(dst, &tmE, 0, r0, &bar[2]);
-    tma_load_2d(dst + kBlk, &tmE, 64, r0, &bar[2]);
-  };
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&tmE);
-    if (HIST) prefetch_tmap(&tmY);
-    load(&bar[0], sW, ws + Lw.img_v);
-    if ((int)blockIdx.x < n_tiles) {
-      const int4 tl = tiles[blockIdx.x];
-      load_e(rot, tl.y);
-      if (HIST) load(&bar[3], sG, uimg(tl.x));
-      load(&bar[4], sQH, uimg(tl.x) + 2 * kBlk);
-      load(&bar[5], rot + 2 * kSlot, uimg(tl.x) + 4 * kBlk);
-    }
-  }
   const int warp = threadIdx.x >> 5;
-  const int part = warp >> 2;
-  const int row = (warp & 3) * 32 + (threadIdx.x & 31);
-  const int c0 = part * 32;
-  const uint32_t ta = quad_addr(c);
-  int ia = 0;   // slot ia = A, (ia+1)%3 = B, (ia+2)%3 = C
-  for (int t = blockIdx.x, it = 0; t < n_tiles; t += gridDim.x, ++it) {
-    const int4 tl = tiles[t];
-    const int u = tl.x, r0 = tl.y, nv = tl.z;
-    const int tn = t + gridDim.x;
-    const int un = tn < n_tiles ? tiles[tn].x : 0;
-    const uint32_t ph = (uint32_t)it & 1u;
-    uint8_t* sA = rot + ia * kSlot;
-    uint8_t* sB = rot + (ia == 2 ? 0 : ia + 1) * kSlot;
-    uint8_t* sC = rot + (ia == 0 ? 2 : ia - 1) * kSlot;
-    mbar_wait(&bar[2], ph, status, c.abort_flag);
-    {
-      float x[32];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sA, kBlk, row, c0 + q * 8), x + q * 8);
-      layer_norm_part(x, c0, red, part, row);
-      if (HIST && it > 0) {
-        // the previous tile's Yd store has read its staging (this tile's B)
-        if (threadIdx.x == 0) bulk_wait_read<0>();
-        __syncthreads();
-      }
-      split_part_st(sA, sB, row, c0, x);
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      if (it == 0) mbar_wait(&bar[0], 0, status, c.abort_flag);
-      mbar_wait(&bar[4], ph, status, c.abort_flag);
-      mbar_wait(&bar[5], ph, status, c.abort_flag);
-      tc_fence_after();
-      mma_tile(c.tmem + 128, smem_u32(sQH), kBlk, smem_u32(sA), kBlk, 128, 128, false);
-      mma_tile(c.tmem + 128, smem_u32(sC), kBlk, smem_u32(sA), kBlk, 128, 128, true);
-      mma_commit(&bar[1]);
-      mma_tile(c.tmem + 256, smem_u32(sA), kBlk, smem_u32(sW), kBlk, 128, 128, false);
-      mma_tile(c.tmem + 256, smem_u32(sB), kBlk, smem_u32(sW), kBlk, 128, 128, true);
-      mma_commit(&bar[7]);
-      if (HIST) {
-        mbar_wait(&bar[3], ph, status, c.abort_flag);
-        tc_fence_after();
-        mma_tile(c.tmem, smem_u32(sA), kBlk, smem_u32(sG), kBlk, HL, 128, false);
-        mma_commit(&bar[8]);
-      }
-    }
-    mbar_wait(&bar[1], ph, status, c.abort_flag);
-    tc_fence_after();
-    // the link scores have read Q'hi and Q'lo
-    if (threadIdx.x == 0) {
-      if (HIST) load(&bar[6], sQH, uimg(u) + 6 * kBlk);
-      else if (tn < n_tiles) load(&bar[4], sQH, uimg(un) + 2 * kBlk);
-      if (tn < n_tiles) load_e(sC, tiles[tn].y);
-    }
-    // link softmax over the tile's valid rows: row = (head, link) lane, part =
-    // a quarter of the tokens.  Lanes >= H*L carry no link.
-    float lm, ls;
-    {
-      float z[32];
-      tmem_ld16(ta + 128 + c0, z);
-      tmem_ld16(ta + 128 + c0 + 16, z + 16);
-      tmem_ld_wait();
-      const bool link = row < HL;
-      float m = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (c0 + j >= nv || !link) z[j] = -INFINITY;
-        m = fmaxf(m, z[j]);
-      }
-      red[part * 128 + row] = m;
-      __syncthreads();
-      m = fmaxf(fmaxf(red[row], red[128 + row]), fmaxf(red[256 + row], red[384 + row]));
-      float s = 0.f;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        z[j] = c0 + j < nv && link ? __expf(z[j] - m) : 0.f;
-        s += z[j];
-      }
-      red[512 + part * 128 + row] = s;
-      __syncthreads();
-      lm = m;
-      ls = red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row];
-      // P2 over X^lo, whose last reader is the V_E product
-      mbar_wait(&bar[7], ph, status, c.abort_flag);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(sB, kBlk, row, c0 + q * 8, pack8(z + q * 8));
-    }
-    {
-      // V_E (bf16) over the G image (read by S): the MN-major B of P2 V_E
-      if (HIST) mbar_wait(&bar[8], ph, status, c.abort_flag);
-      tc_fence_after();
-      float v[32];
-      tmem_ld16(ta + 256 + c0, v);
-      tmem_ld16(ta + 256 + c0 + 16, v + 16);
-      tmem_ld_wait();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(sG, kBlk, row, c0 + q * 8, pack8(v + q * 8));
-    }
-    if (HIST) {
-      // history softmax over the user's L links: part = head, P over X^hi
-      const int h = part;
-      float z[L];
-#pragma unroll
-      for (int q = 0; q < L / 16; ++q) tmem_ld16(ta + h * L + q * 16, z + q * 16);
-      tmem_ld_wait();
-      float m = z[0];
-#pragma unroll
-      for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
-      float s = 0.f;
-#pragma unroll
-      for (int k = 0; k < L; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
-      const float inv = 1.0f / s;
-#pragma unroll
-      for (int k = 0; k < L; ++k) z[k] *= inv;
-#pragma unroll
-      for (int q = 0; q < L / 8; ++q) sw_st16(sA, kBlk, row, h * L + q * 8, pack8(z + q * 8));
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      mma_tile_bmn(c.tmem + 128, smem_u32(sB), kBlk, smem_u32(sG), kBlk, 128, 128, false);
-      mma_commit(&bar[9]);
-      if (HIST) {
-        mbar_wait(&bar[6], ph, status, c.abort_flag);
-        tc_fence_after();
-        mma_tile_bmn(c.tmem, smem_u32(sA), kBlk, smem_u32(sQH), kBlk, 128, HL, false);
-        mma_commit(&bar[10]);
-      }
-    }
-    mbar_wait(&bar[9], ph, status, c.abort_flag);
-    tc_fence_after();
-    // P2 V_E has read V_E and P2: the next G, and the next Q'lo (the next C)
-    if (threadIdx.x == 0 && tn < n_tiles) {
-      if (HIST) load(&bar[3], sG, uimg(un));
-      load(&bar[5], sB, uimg(un) + 4 * kBlk);
-    }
-    {
-      // link record of row p = (h, k): part h reads head h's 32 columns
-      // (warp-uniform TMEM address); rows of other heads skip the store
-      float acc[kDH];
-      tmem_ld16(ta + 128 + part * kDH, acc);
-      tmem_ld16(ta + 128 + part * kDH + 16, acc + 16);
-      tmem_ld_wait();
-      if (row < HL && row / L == part) {
-        float4* rec = reinterpret_cast<float4*>(part_rec + ((size_t)t * HL + row) * kRec);
-        rec[0] = make_float4(lm, ls, 0.f, 0.f);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          rec[1 + q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
-      }
-    }
-    if (HIST) {
-      mbar_wait(&bar[10], ph, status, c.abort_flag);
-      tc_fence_after();
-      // Yd has read P and VO: the next Q'hi
-      if (threadIdx.x == 0 && tn < n_tiles) load(&bar[4], sQH, uimg(un) + 2 * kBlk);
-      float y[32];
-      tmem_ld16(ta + c0, y);
-      tmem_ld16(ta + c0 + 16, y + 16);
-      tmem_ld_wait();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(sA, kBlk, row, c0 + q * 8, pack8_f16(y + q * 8));
-      fence_proxy_async_smem();
-      __syncthreads();
-      if (nv == kTile) {
-        if (threadIdx.x == 0) {
-          tma_store_2d(&tmY, sA, 0, r0);
-          tma_store_2d(&tmY, sA + kBlk, 64, r0);
-          bulk_commit();
-        }
+  auto slots = [&](int ia, uint8_t*& sA, uint8_t*& sB, uint8_t*& sC) {
+    sA = rot + ia * kSlot;
+    sB = rot + (ia == 2 ? 0 : ia + 1) * kSlot;
+    sC = rot + (ia == 0 ? 2 : ia - 1) * kSlot;
+  };
+  if (warp == kXaEpi / 32) {
+    if ((threadIdx.x & 31) == 0) {
+      // ---- the issuer: loads and MMAs
+      auto uimg = [&](int u) { return ws + Lw.uimg + (size_t)u * Lw.uimg_bytes; };
+      auto load = [&](uint64_t* b, uint8_t* dst, const uint8_t* src) {
+        mbar_arrive_expect_tx(b, kSlot);
+        bulk_load(dst, src, kSlot, b);
+      };
+      auto load_e = [&](uint8_t* dst, int r0) {
+        mbar_arrive_expect_tx(&bar[2], kSlot);
+        tma_load_2d(dst, &tmE, 0, r0, &bar[2]);
+        tma_load_2d(dst + kBlk, &tmE, 64, r0, &bar[2]);
+      };
+      prefetch_tmap(&tmE);
+      load(&bar[0], sW, ws + Lw.img_v);
+      if ((int)blockIdx.x < n_tiles) {
+        const int4 tl = tiles[blockIdx.x];
+        load_e(rot, tl.y);
+        if (HIST) load(&bar[3], sG, uimg(tl.x));
+        load(&bar[4], sQH, uimg(tl.x) + 2 * kBlk);
+        load(&bar[5], rot + 2 * kSlot, uimg(tl.x) + 4 * kBlk);
       } else {
-        tile_store_rows(sA, yd + (int64_t)r0 * kD, nv);
+        mbar_wait(&bar[0], 0, status, c.abort_flag);   // lands before the CTA exits
+      }
+      int ia = 0;
+      for (int t = blockIdx.x, it = 0; t < n_tiles; t += gridDim.x, ++it) {
+        const int u = tiles[t].x;
+        const int tn = t + gridDim.x;
+        const int un = tn < n_tiles ? tiles[tn].x : 0;
+        const uint32_t ph = (uint32_t)it & 1u;
+        uint8_t *sA, *sB, *sC;
+        slots(ia, sA, sB, sC);
+        mbar_wait(&bar[11], ph, status, c.abort_flag);
+        if (it == 0) mbar_wait(&bar[0], 0, status, c.abort_flag);
+        mbar_wait(&bar[4], ph, status, c.abort_flag);
+        mbar_wait(&bar[5], ph, status, c.abort_flag);
+        tc_fence_after();
+        mma_tile(c.tmem + 128, smem_u32(sQH), kBlk, smem_u32(sA), kBlk, 128, 128, false);
+        mma_tile(c.tmem + 128, smem_u32(sC), kBlk, smem_u32(sA), kBlk, 128, 128, true);
+        mma_commit(&bar[1]);
+        mma_tile(c.tmem + 256, smem_u32(sA), kBlk, smem_u32(sW), kBlk, 128, 128, false);
+        mma_tile(c.tmem + 256, smem_u32(sB), kBlk, smem_u32(sW), kBlk, 128, 128, true);
+        mma_commit(&bar[7]);
+        if (HIST) {
+          mbar_wait(&bar[3], ph, status, c.abort_flag);
+          tc_fence_after();
+          mma_tile(c.tmem, smem_u32(sA), kBlk, smem_u32(sG), kBlk, HL, 128, false);
+          mma_commit(&bar[8]);
+        }
+        // the link scores have read Q'hi and Q'lo
+        mbar_wait(&bar[1], ph, status, c.abort_flag);
+        if (HIST) load(&bar[6], sQH, uimg(u) + 6 * kBlk);
+        else if (tn < n_tiles) load(&bar[4], sQH, uimg(un) + 2 * kBlk);
+        if (tn < n_tiles) load_e(sC, tiles[tn].y);
+        mbar_wait(&bar[12], ph, status, c.abort_flag);
+        tc_fence_after();
+        mma_tile_bmn(c.tmem + 128, smem_u32(sB), kBlk, smem_u32(sG), kBlk, 128, 128, false);
+        mma_commit(&bar[9]);
+        if (HIST) {
+          mbar_wait(&bar[6], ph, status, c.abort_flag);
+          tc_fence_after();
+          mma_tile_bmn(c.tmem, smem_u32(sA), kBlk, smem_u32(sQH), kBlk, 128, HL, false);
+          mma_commit(&bar[10]);
+        }
+        // P2 V_E has read V_E and P2: the next G, and the next Q'lo (the next C)
+        mbar_wait(&bar[9], ph, status, c.abort_flag);
+        if (tn < n_tiles) {
+          if (HIST) load(&bar[3], sG, uimg(un));
+          load(&bar[5], sB, uimg(un) + 4 * kBlk);
+        }
+        if (HIST) {
+          // Yd has read P and VO: the next Q'hi
+          mbar_wait(&bar[10], ph, status, c.abort_flag);
+          if (tn < n_tiles) load(&bar[4], sQH, uimg(un) + 2 * kBlk);
+        }
+        ia = ia == 0 ? 2 : ia - 1;
       }
     }
-    tc_fence_before();
-    __syncthreads();
-    ia = ia == 0 ? 2 : ia - 1;   // next (A, B, C) = (C, A, B)
-  }
-  if (threadIdx.x == 0) {
-    // a CTA without tiles still lets its Wv load land before it exits
-    if ((int)blockIdx.x >= n_tiles) mbar_wait(&bar[0], 0, status, c.abort_flag);
-    bulk_wait<0>();
+  } else {
+    // ---- the epilogue (512 threads)
+    const int part = warp >> 2;
+    const int row = (warp & 3) * 32 + (threadIdx.x & 31);
+    const int c0 = part * 32;
+    const uint32_t ta = quad_addr(c);
+    bf16* yd = reinterpret_cast<bf16*>(ws + Lw.yd);   // fp16 bits; rows copied as bytes
+    float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
+    if (HIST && threadIdx.x == 0) prefetch_tmap(&tmY);
+    int ia = 0;
+    for (int t = blockIdx.x, it = 0; t < n_tiles; t += gridDim.x, ++it) {
+      const int4 tl = tiles[t];
+      const int r0 = tl.y, nv = tl.z;
+      const uint32_t ph = (uint32_t)it & 1u;
+      uint8_t *sA, *sB, *sC;
+      slots(ia, sA, sB, sC);
+      mbar_wait(&bar[2], ph, status, c.abort_flag);
+      {
+        float x[32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sA, kBlk, row, c0 + q * 8), x + q * 8);
+        layer_norm_part<kXaEpi>(x, c0, red, part, row);
+        if (HIST && it > 0) {
+          // the previous tile's Yd store has read its staging (this tile's B)
+          if (threadIdx.x == 0) bulk_wait_read<0>();
+          named_bar_sync(1, kXaEpi);
+        }
+        split_part_st(sA, sB, row, c0, x);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(1, kXaEpi);
+      if (threadIdx.x == 0) mbar_arrive(&bar[11]);
+      mbar_wait(&bar[1], ph, status, c.abort_flag);
+      tc_fence_after();
+      // link softmax over the tile's valid rows: row = (head, link) lane,
+      // part = a quarter of the tokens.  Lanes >= H*L carry no link.
+      float lm, ls;
+      {
+        float z[32];
+        tmem_ld16(ta + 128 + c0, z);
+        tmem_ld16(ta + 128 + c0 + 16, z + 16);
+        tmem_ld_wait();
+        const bool link = row < HL;
+        float m = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (c0 + j >= nv || !link) z[j] = -INFINITY;
+          m = fmaxf(m, z[j]);
+        }
+        red[part * 128 + row] = m;
+        named_bar_sync(1, kXaEpi);
+        m = fmaxf(fmaxf(red[row], red[128 + row]), fmaxf(red[256 + row], red[384 + row]));
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          z[j] = c0 + j < nv && link ? __expf(z[j] - m) : 0.f;
+          s += z[j];
+        }
+        red[512 + part * 128 + row] = s;
+        named_bar_sync(1, kXaEpi);
+        lm = m;
+        ls = red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row];
+        // P2 over X^lo, whose last reader is the V_E product
+        mbar_wait(&bar[7], ph, status, c.abort_flag);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sw_st16(sB, kBlk, row, c0 + q * 8, pack8(z + q * 8));
+      }
+      {
+        // V_E (bf16) over the G image (read by S): the MN-major B of P2 V_E
+        if (HIST) mbar_wait(&bar[8], ph, status, c.abort_flag);
+        tc_fence_after();
+        float v[32];
+        tmem_ld16(ta + 256 + c0, v);
+        tmem_ld16(ta + 256 + c0 + 16, v + 16);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sw_st16(sG, kBlk, row, c0 + q * 8, pack8(v + q * 8));
+      }
+      if (HIST) {
+        // history softmax over the user's L links: part = head, P over X^hi
+        const int h = part;
+        float z[L];
+#pragma unroll
+        for (int q = 0; q < L / 16; ++q) tmem_ld16(ta + h * L + q * 16, z + q * 16);
+        tmem_ld_wait();
+        float m = z[0];
+#pragma unroll
+        for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < L; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
+        const float inv = 1.0f / s;
+#pragma unroll
+        for (int k = 0; k < L; ++k) z[k] *= inv;
+#pragma unroll
+        for (int q = 0; q < L / 8; ++q) sw_st16(sA, kBlk, row, h * L + q * 8, pack8(z + q * 8));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(1, kXaEpi);
+      if (threadIdx.x == 0) mbar_arrive(&bar[12]);
+      mbar_wait(&bar[9], ph, status, c.abort_flag);
+      tc_fence_after();
+      {
+        // link record of row p = (h, k): part h reads head h's 32 columns
+        // (warp-uniform TMEM address); rows of other heads skip the store
+        float acc[kDH];
+        tmem_ld16(ta + 128 + part * kDH, acc);
+        tmem_ld16(ta + 128 + part * kDH + 16, acc + 16);
+        tmem_ld_wait();
+        if (row < HL && row / L == part) {
+          float4* rec = reinterpret_cast<float4*>(part_rec + ((size_t)t * HL + row) * kRec);
+          rec[0] = make_float4(lm, ls, 0.f, 0.f);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            rec[1 + q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+        }
+      }
+      if (HIST) {
+        mbar_wait(&bar[10], ph, status, c.abort_flag);
+        tc_fence_after();
+        float y[32];
+        tmem_ld16(ta + c0, y);
+        tmem_ld16(ta + c0 + 16, y + 16);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sw_st16(sA, kBlk, row, c0 + q * 8, pack8_f16(y + q * 8));
+        fence_proxy_async_smem();
+        named_bar_sync(1, kXaEpi);
+        if (nv == kTile) {
+          if (threadIdx.x == 0) {
+            tma_store_2d(&tmY, sA, 0, r0);
+            tma_store_2d(&tmY, sA + kBlk, 64, r0);
+            bulk_commit();
+          }
+        } else {
+          for (int idx = (int)threadIdx.x; idx < 2048; idx += kXaEpi) {
+            const int r = idx >> 4, cc = idx & 15;
+            if (r < nv) reinterpret_cast<uint4*>(yd + (int64_t)(r0 + r) * kD)[cc] = sw_ld16(sA, kBlk, r, cc * 8);
+          }
+        }
+      }
+      tc_fence_before();
+      ia = ia == 0 ? 2 : ia - 1;   // next (A, B, C) = (C, A, B)
+    }
+    if (threadIdx.x == 0) bulk_wait<0>();
   }
   cta_teardown(c);
 }
@@ -1437,10 +1469,10 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     const int64_t tiles_hi = Lw.max_tiles;
     const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
     {
-      const int smem = 1024 + 12 * kBlk + kLnBytes + 128;   // 11 barriers
+      const int smem = 1024 + 12 * kBlk + kLnBytes + 128;   // 13 barriers
       auto kern = last ? k_hist_xattn<L, false> : k_hist_xattn<L, true>;
       if (!set_smem(kern, smem)) return LIME_ERR_CUDA;
-      int rc = launch_pdl(kern, dim3(grid), dim3(512), smem, st, 1, tmE, tmY, (const bf16*)w.g1,
+      int rc = launch_pdl(kern, dim3(grid), dim3(kXaThreads), smem, st, 1, tmE, tmY, (const bf16*)w.g1,
                           (const bf16*)w.b1, ws, Lw, status);
       if (rc) return rc;
     }

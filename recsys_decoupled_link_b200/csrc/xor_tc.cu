@@ -56,6 +56,7 @@ constexpr int kRec = 36;  // floats per link-branch record: max, sum, 2 pad, 32 
 
 struct LayerWs {
   size_t img_q, img_k, img_v, img_o, img_13, img_2;
+  size_t img_vg;   // (g1 Wv)^T as hi, lo images, then cv = colsum(g1 Wv), dv = b1 Wv (fp32)
   size_t sched, tiles, tile_start;
   size_t yd, uimg, part;
   size_t total;
@@ -65,8 +66,10 @@ struct LayerWs {
 
 __host__ __device__ constexpr size_t up1k(size_t x) { return (x + 1023) & ~(size_t)1023; }
 
-// per-user folded images: G^T, Q' hi, Q' lo, VO ([128 x 128] bf16 each)
-constexpr uint32_t kUimgBytes = 8 * kBlk;
+// per-user folded images: G'^T, Q'g, VO ([128 x 128] bf16 each), then the
+// fp32 vectors cQ, dQ, cG, dG ([128] each)
+constexpr uint32_t kUimgVec = 6 * kBlk;
+constexpr uint32_t kUimgBytes = 6 * kBlk + 4 * 128 * 4;
 
 LayerWs layer_ws(int l, int64_t B, int64_t nh) {
   LayerWs w;
@@ -78,6 +81,7 @@ LayerWs layer_ws(int l, int64_t B, int64_t nh) {
   w.img_o = take(2 * kBlk);
   w.img_13 = take(8 * kBlk);
   w.img_2 = take(4 * kBlk);
+  w.img_vg = take(4 * kBlk + 2 * kD * 4);
   w.max_tiles = nh / kTile + B + 1;
   w.sched = take(16);
   w.tiles = take((size_t)w.max_tiles * 16);
@@ -88,49 +92,6 @@ LayerWs layer_ws(int l, int64_t B, int64_t nh) {
   w.part = take((size_t)w.max_tiles * kH * l * kRec * 4);
   w.total = o;
   return w;
-}
-
-// Reads row `row` (128 bf16) of a [128 x 128] swizzled tile into fp32.
-__device__ __forceinline__ void tile_row_ld(const uint8_t* t, int row, float* x) {
-#pragma unroll
-  for (int c = 0; c < 16; ++c) unpack8(sw_ld16(t, kBlk, row, c * 8), x + c * 8);
-}
-__device__ __forceinline__ void tile_row_st(uint8_t* t, int row, const float* x) {
-#pragma unroll
-  for (int c = 0; c < 16; ++c) sw_st16(t, kBlk, row, c * 8, pack8(x + c * 8));
-}
-
-// x <- LayerNorm(x) * g + b over 128 values (biased variance).
-__device__ __forceinline__ void layer_norm_128(float* x, const bf16* g, const bf16* b) {
-  float mu = 0.f;
-#pragma unroll
-  for (int i = 0; i < kD; ++i) mu += x[i];
-  mu *= (1.0f / kD);
-  float var = 0.f;
-#pragma unroll
-  for (int i = 0; i < kD; ++i) { const float t = x[i] - mu; var += t * t; }
-  const float rstd = rsqrtf(var * (1.0f / kD) + kLnEps);
-#pragma unroll
-  for (int i = 0; i < kD; ++i)
-    x[i] = (x[i] - mu) * rstd * __bfloat162float(g[i]) + __bfloat162float(b[i]);
-}
-
-// Row reductions over the four column parts of a row (thread = (row, part),
-// 512 threads): every thread gets the total.  `red` holds 512 floats; all
-// threads of the block take part (two block-wide barriers).
-__device__ __forceinline__ float row_sum4(float v, float* red, int part, int row) {
-  red[part * 128 + row] = v;
-  __syncthreads();
-  const float t = red[row] + red[128 + row] + red[256 + row] + red[384 + row];
-  __syncthreads();
-  return t;
-}
-__device__ __forceinline__ float row_max4(float v, float* red, int part, int row) {
-  red[part * 128 + row] = v;
-  __syncthreads();
-  const float t = fmaxf(fmaxf(red[row], red[128 + row]), fmaxf(red[256 + row], red[384 + row]));
-  __syncthreads();
-  return t;
 }
 
 // LayerNorm scratch of the 512-thread kernels: two [4][128] reduction
@@ -152,19 +113,15 @@ __device__ __forceinline__ void ln_stage(float* gb, const bf16* g, const bf16* b
 // squares are reduced in one pass (var = E[x^2] - mu^2 in fp32; LN inputs
 // here are O(1) with |mu| of the order of the spread, so the cancellation
 // costs a few ulp).  `red` is a kLnFloats scratch (red[0..1023] for the
-// reductions, g and b after them); 512 threads take part (one barrier: the
-// whole block, or named barrier 1 over threads 0-511 when NB = 512 and the
-// block has more threads; the caller's next barrier must come before red is
-// written again).
-template <int NB = 0>
+// reductions, g and b after them); all 512 threads take part (one block-wide
+// barrier; the caller's next barrier must come before red is written again).
 __device__ __forceinline__ void layer_norm_part(float* x, int c0, float* red, int part, int row) {
   float s1 = 0.f, s2 = 0.f;
 #pragma unroll
   for (int k = 0; k < 32; ++k) { s1 += x[k]; s2 = fmaf(x[k], x[k], s2); }
   red[part * 128 + row] = s1;
   red[512 + part * 128 + row] = s2;
-  if (NB) named_bar_sync(1, NB);
-  else __syncthreads();
+  __syncthreads();
   const float mu = (red[row] + red[128 + row] + red[256 + row] + red[384 + row]) * (1.0f / kD);
   const float ex2 = (red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row]) * (1.0f / kD);
   const float rstd = rsqrtf(fmaxf(ex2 - mu * mu, 0.f) + kLnEps);
@@ -177,39 +134,6 @@ __device__ __forceinline__ void layer_norm_part(float* x, int c0, float* red, in
     x[4 * q + 1] = (x[4 * q + 1] - mu) * rstd * gv.y + bv.y;
     x[4 * q + 2] = (x[4 * q + 2] - mu) * rstd * gv.z + bv.z;
     x[4 * q + 3] = (x[4 * q + 3] - mu) * rstd * gv.w + bv.w;
-  }
-}
-
-// Loads 128 consecutive fp32 TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_row128(uint32_t taddr, float* x) {
-#pragma unroll
-  for (int q = 0; q < 8; ++q) tmem_ld16(taddr + q * 16, x + q * 16);
-  tmem_ld_wait();
-}
-
-__device__ __forceinline__ void gl_row_st(bf16* dst, const float* x) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int c = 0; c < 16; ++c) d[c] = pack8(x + c * 8);
-}
-__device__ __forceinline__ void gl_row_ld(const bf16* src, float* x) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int c = 0; c < 16; ++c) unpack8(s[c], x + c * 8);
-}
-
-// Writes x (fp32) as hi = bf16(x) and lo = bf16(x - hi) rows of two operands.
-__device__ __forceinline__ void split_row_st(uint8_t* hi, uint8_t* lo, uint32_t blk, int row,
-                                             const float* x, int n) {
-  for (int c = 0; c < n / 8; ++c) {
-    float h[8], r[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      h[i] = __bfloat162float(__float2bfloat16_rn(x[c * 8 + i]));
-      r[i] = x[c * 8 + i] - h[i];
-    }
-    sw_st16(hi, blk, row, c * 8, pack8(h));
-    sw_st16(lo, blk, row, c * 8, pack8(r));
   }
 }
 
@@ -241,17 +165,6 @@ __device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f 
 // are both free of bank conflicts.
 __device__ __forceinline__ float4* f32_chunk(uint8_t* base, int r, int c) {
   return reinterpret_cast<float4*>(base + r * 512 + ((c ^ (r & 31)) << 4));
-}
-
-// Cooperatively loads fp32 rows p*32 .. p*32+31 of `src` (128 columns, row 0 =
-// the tile's first row) into staging rows 0..31; rows at or past `nv` are not read.
-__device__ __forceinline__ void f32_stage32(uint8_t* stage, const float* src, int p, int nv) {
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const int idx = q * 128 + (int)threadIdx.x, r = idx >> 5, c = idx & 31;
-    if (p * 32 + r < nv)
-      *f32_chunk(stage, r, c) = reinterpret_cast<const float4*>(src + (int64_t)(p * 32 + r) * kD)[c];
-  }
 }
 
 // Common CTA prologue: barriers, abort flag, TMEM allocation (`ncols` columns).
@@ -292,9 +205,6 @@ __device__ __forceinline__ void cta_teardown(Cta& c) {
   }
 }
 
-__device__ __forceinline__ uint32_t lane_addr(const Cta& c) {
-  return c.tmem + ((uint32_t)(threadIdx.x & ~31) << 16);
-}
 // 512-thread kernels: warp w serves TMEM lane quadrant w % 4.
 __device__ __forceinline__ uint32_t quad_addr(const Cta& c) {
   return c.tmem + ((uint32_t)(((threadIdx.x >> 5) & 3) * 32) << 16);
@@ -313,12 +223,14 @@ __device__ void schedule_tiles(const int64_t* __restrict__ off, int64_t B, int64
                                int max_tiles, int* __restrict__ sched, int4* __restrict__ tiles,
                                int* __restrict__ tile_start, unsigned* status);
 
-// Block 0 builds the tile schedule; the other blocks write the weight images.
+// Block 0 builds the tile schedule, block 1 the V_E vectors (cv, dv); the
+// other blocks write the weight images.
 __global__ void __launch_bounds__(1024) k_prep_weights(
     const bf16* __restrict__ Wq, const bf16* __restrict__ Wk, const bf16* __restrict__ Wv,
     const bf16* __restrict__ Wo, const bf16* __restrict__ W1, const bf16* __restrict__ W3,
-    const bf16* __restrict__ W2, uint8_t* __restrict__ ws, LayerWs L,
-    const int64_t* __restrict__ off, int64_t B, int64_t nh, unsigned* status) {
+    const bf16* __restrict__ W2, const bf16* __restrict__ g1, const bf16* __restrict__ b1,
+    uint8_t* __restrict__ ws, LayerWs L, const int64_t* __restrict__ off, int64_t B, int64_t nh,
+    unsigned* status) {
   pdl_launch();
   pdl_wait();
   if (blockIdx.x == 0) {
@@ -327,9 +239,35 @@ __global__ void __launch_bounds__(1024) k_prep_weights(
                    status);
     return;
   }
+  if (blockIdx.x == 1) {
+    // cv[n] = sum_i g1[i] Wv[i][n] (each product is exact in fp32, and equal to
+    // the hi + lo image pair), dv[n] = sum_i b1[i] Wv[i][n]: thread (n, g)
+    // sums rows 16g .. 16g+15, then thread n adds the eight partials
+    __shared__ float part_cd[2][8][kD];
+    const int n = threadIdx.x & (kD - 1), g = threadIdx.x >> 7;
+    float cv = 0.f, dv = 0.f;
+#pragma unroll
+    for (int i = g * 16; i < g * 16 + 16; ++i) {
+      const float w = __bfloat162float(Wv[i * kD + n]);
+      cv = fmaf(__bfloat162float(g1[i]), w, cv);
+      dv = fmaf(__bfloat162float(b1[i]), w, dv);
+    }
+    part_cd[0][g][n] = cv;
+    part_cd[1][g][n] = dv;
+    __syncthreads();
+    if (threadIdx.x < kD) {
+      float* vec = reinterpret_cast<float*>(ws + L.img_vg + 4 * kBlk);
+      float a = 0.f, b = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { a += part_cd[0][j][n]; b += part_cd[1][j][n]; }
+      vec[n] = a;
+      vec[kD + n] = b;
+    }
+    return;
+  }
   // Thread (matrix, n, k8) gathers W[k8*8 .. k8*8+7][n] (loads coalesced over
   // n) and writes them as one 16-byte chunk of row n of the image.
-  const int64_t e = (blockIdx.x - 1) * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t e = (blockIdx.x - 2) * (int64_t)blockDim.x + threadIdx.x;
   const int64_t n_sq = kD * kD / 8, n_ff = kD * kF / 8;   // chunks per matrix
   float f[8];
   if (e < 4 * n_sq) {
@@ -356,6 +294,19 @@ __global__ void __launch_bounds__(1024) k_prep_weights(
 #pragma unroll
     for (int j = 0; j < 8; ++j) f[j] = __bfloat162float(W2[(k8 * 8 + j) * kD + n]);
     sw_st16(ws + L.img_2, kBlk, n, k8 * 8, pack8(f));
+  } else if (e < 5 * n_sq + 3 * n_ff) {
+    // (g1 Wv)^T split hi + lo: LN1's scale folded into the V_E weights
+    const int r = (int)(e - 4 * n_sq - 3 * n_ff);
+    const int k8 = r / kD, n = r % kD;
+    float lo[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float x = __bfloat162float(g1[k8 * 8 + j]) * __bfloat162float(Wv[(k8 * 8 + j) * kD + n]);
+      f[j] = __bfloat162float(__float2bfloat16_rn(x));
+      lo[j] = x - f[j];
+    }
+    sw_st16(ws + L.img_vg, kBlk, n, k8 * 8, pack8(f));
+    sw_st16(ws + L.img_vg + 2 * kBlk, kBlk, n, k8 * 8, pack8(lo));
   }
 }
 
@@ -419,26 +370,30 @@ __device__ void schedule_tiles(const int64_t* __restrict__ off, int64_t B, int64
 }
 
 // ----------------------------------------------------- link projections
-// Per-user operand images, at uimg + u * uimg_bytes: four [128 rows x 128]
-// bf16 K-major 128B-swizzled images of two kBlk blocks each.  Row p = h*L + k
-// is (head h, link k); rows p >= H*L are never written and only ever reach
-// MMA output rows that nothing reads.
-//   G      [0, 2 kBlk)     G^T[p]  = s K_Z[k, h] Wq[:, h]^T      (h: head h's 32 columns)
-//   QH, QL [2, 6 kBlk)     Q'[p]   = s Q_Z[k, h] Wk[:, h]^T as bf16 hi + lo
-//   VO     [6, 8 kBlk)     VO[p]   = V_Z[k, h] Wo[h, :]          (Wo's rows of head h)
+// Per-user operand images, at uimg + u * uimg_bytes: three [128 rows x 128]
+// bf16 K-major 128B-swizzled images of two kBlk blocks each, then fp32
+// vectors.  Row p = h*L + k is (head h, link k); rows p >= H*L are never
+// written and only ever reach MMA output rows that nothing reads.
+//   G'   [0, 2 kBlk)   G'[p, i] = g1[i] (s K_Z[k, h] Wq[:, h]^T)[i]   (h: head h's 32 columns)
+//   Q'g  [2, 4 kBlk)   Q'g[p, i] = g1[i] (s Q_Z[k, h] Wk[:, h]^T)[i]
+//   VO   [4, 6 kBlk)   VO[p] = V_Z[k, h] Wo[h, :]                     (Wo's rows of head h)
+//   vec  cQ, dQ, cG, dG [128] each: c[p] = sum_i of the stored row p of Q'g
+//        (G'), d[p] = sum_i b1[i] of the unscaled row
 // By associativity the history scores are Q_E,h (s K_Z,h)^T = X^ G_h, the
 // link scores (s Q_Z,h) K_E,h^T = Q'_h X^^T and the history branch through
-// Wo is (P_h V_Z,h) Wo_h = P_h VO_h (X^ = LN1(E)), so the history kernel
-// needs neither Q_E nor K_E (and the link branch keeps V_E on chip).
+// Wo is (P_h V_Z,h) Wo_h = P_h VO_h.  With X^ = LN1(E) = rstd (E - mu) g1 + b1
+// per history row, Q' X^^T = rstd (Q'g E^T - mu cQ) + dQ (and likewise X^ G),
+// so the history kernel multiplies the raw rows E and needs only each row's
+// mean and rstd; it never forms Q_E, K_E or X^.
 //
-// CTA (128 link rows, which, z): which = 0 -> Q' (hi + lo), 1 -> G, 2 -> VO,
-// for heads z*hpc .. z*hpc + hpc - 1 (hpc = H / gridDim.z; more CTAs spread
-// the image writes, which dominate, over more SMs).
-// LN1(Z) (split) -> projection P = X^z Wm -> s P (which < 2) split hi + lo ->
-// per head h of the CTA the fold P[:, h] B_h (K = 32, two MMAs per half), B_h =
-// Wk's, Wq's or Wo's head-h slice of its weight image -> rows h*L + k of the
-// users' images, staged and written with bulk copies.  512 threads: thread
-// (row, part) owns columns part*32 .. part*32+31, i.e. head `part`.
+// CTA (128 link rows, which, z): which = 0 -> Q'g, 1 -> G', 2 -> VO, for heads
+// z*hpc .. z*hpc + hpc - 1 (hpc = H / gridDim.z; more CTAs spread the image
+// writes, which dominate, over more SMs).  LN1(Z) (split) -> projection P =
+// X^z Wm -> s P (which < 2) split hi + lo -> per head h of the CTA the fold
+// P[:, h] B_h (K = 32, two MMAs), B_h = Wk's, Wq's or Wo's head-h slice of its
+// weight image -> rows h*L + k of the users' images, staged and written with
+// bulk copies.  512 threads: thread (row, part) owns columns part*32 ..
+// part*32+31.
 template <int L>
 __global__ void __launch_bounds__(512, 1)
     k_link_proj(const bf16* __restrict__ Z, int64_t nrows, const bf16* __restrict__ g1,
@@ -532,49 +487,64 @@ __global__ void __launch_bounds__(512, 1)
   // The fold outputs are staged (the MMA operands are dead) in the images'
   // own swizzled layout: lane r = j*L + k of user j lands at row r, which has
   // the swizzle phase of its image row h*L + k, so user j's L rows of a head
-  // leave as one L*128-byte bulk copy per 64-column block.  Items are (head,
-  // half): Q' has a hi and a lo half per head; four 32 KB buffers per pass.
+  // leave as one L*128-byte bulk copy per 64-column block (up to four heads
+  // per CTA, one 32 KB buffer each).  Q' and G carry LN1's affine map of the
+  // history rows: they are stored scaled by g1 along d (Q'g, G'), with
+  // c[p] = sum_i Q'g[p, i] (of the stored bf16 values) and d[p] = sum_i
+  // Q'[p, i] b1[i] (likewise for G) in the user's vector area, so that
+  // Q' X^^T = rstd (Q'g E^T - mu c) + d for the raw history rows E.
   constexpr int UP = kTile / L;   // users per tile
   const int64_t u0 = (int64_t)blockIdx.x * UP;
   const int64_t left = nrows / L - u0;
   const int n_users = left < UP ? (int)left : UP;
-  const int halves = which == 0 ? 2 : 1;
-  const int n_items = hpc * halves;
-  for (int i0 = 0; i0 < n_items; i0 += 4) {
-    if (i0 > 0) {
-      if (threadIdx.x == 0) bulk_wait_read<0>();
+  const float* gb = red + 1024;   // g1, b1 as fp32
+  for (int i = 0; i < hpc; ++i) {
+    const int h = h0 + i;
+    float v[32];
+    tmem_ld16(ta + i * 128 + c0, v);
+    tmem_ld16(ta + i * 128 + c0 + 16, v + 16);
+    tmem_ld_wait();
+    uint8_t* buf = sm + i * 2 * kBlk;
+    if (which == 2) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sw_st16(buf, kBlk, r, c0 + q * 8, pack8(v + q * 8));
+    } else {
+      float cs = 0.f, ds = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        ds = fmaf(v[j], gb[kD + c0 + j], ds);
+        v[j] = __bfloat162float(__float2bfloat16_rn(v[j] * gb[c0 + j]));
+        cs += v[j];
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sw_st16(buf, kBlk, r, c0 + q * 8, pack8(v + q * 8));
+      red[part * 128 + r] = cs;
+      red[512 + part * 128 + r] = ds;
+      __syncthreads();
+      if (part == 0 && valid) {
+        float* vec = reinterpret_cast<float*>(ws + Lw.uimg + (size_t)(R / L) * Lw.uimg_bytes + kUimgVec) +
+                     (which == 0 ? 0 : 2 * 128);
+        const int p = h * L + (int)(R % L);
+        vec[p] = red[r] + red[128 + r] + red[256 + r] + red[384 + r];
+        vec[128 + p] = red[512 + r] + red[640 + r] + red[768 + r] + red[896 + r];
+      }
       __syncthreads();
     }
-    const int ni = n_items - i0 < 4 ? n_items - i0 : 4;
-    for (int i = 0; i < ni; i += halves) {
-      const int h = h0 + (i0 + i) / halves;
-      float v[32];
-      tmem_ld16(ta + (h - h0) * 128 + c0, v);
-      tmem_ld16(ta + (h - h0) * 128 + c0 + 16, v + 16);
-      tmem_ld_wait();
-      uint8_t* buf = sm + i * 2 * kBlk;
-      if (which == 0)
-        split_part_st(buf, buf + 2 * kBlk, r, c0, v);
-      else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) sw_st16(buf, kBlk, r, c0 + q * 8, pack8(v + q * 8));
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t img_off = which == 0 ? 2 * kBlk : which == 1 ? 0 : 4 * kBlk;
+    for (int i = 0; i < hpc; ++i) {
+      const int h = h0 + i;
+      for (int j = 0; j < n_users; ++j) {
+        uint8_t* dst = ws + Lw.uimg + (size_t)(u0 + j) * Lw.uimg_bytes + img_off + h * L * 128;
+        const uint8_t* src = sm + i * 2 * kBlk + j * L * 128;
+        bulk_store(dst, src, L * 128);
+        bulk_store(dst + kBlk, src + kBlk, L * 128);
       }
     }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      for (int i = 0; i < ni; ++i) {
-        const int h = h0 + (i0 + i) / halves;
-        const uint32_t img_off = which == 0 ? (2 + 2 * ((i0 + i) & 1)) * kBlk : which == 1 ? 0 : 6 * kBlk;
-        for (int j = 0; j < n_users; ++j) {
-          uint8_t* dst = ws + Lw.uimg + (size_t)(u0 + j) * Lw.uimg_bytes + img_off + h * L * 128;
-          const uint8_t* src = sm + i * 2 * kBlk + j * L * 128;
-          bulk_store(dst, src, L * 128);
-          bulk_store(dst + kBlk, src + kBlk, L * 128);
-        }
-      }
-      bulk_commit();
-    }
+    bulk_commit();
   }
   if (threadIdx.x == 0) bulk_wait<0>();   // the images are complete before the CTA exits
   cta_teardown(c);
@@ -582,31 +552,35 @@ __global__ void __launch_bounds__(512, 1)
 
 // --------------------------------------------------------- XOR attention
 // One persistent CTA per SM walks the tile list.  Per 128-row history tile
-// (a tile never spans two users; rows past `nv` are masked):
-//   LN1      X^ = LN1(E) as bf16 hi (over the E tile) + lo
-//   MMAs     S'^T = Q'hi X^hi^T + Q'lo X^hi^T (link scores, (head, link) on
-//            the TMEM lanes, [128, 256)), V_E = X^ Wv (hi + lo, [256, 384)),
-//            S = X^hi G (history scores, [0, H*L)); each group is committed
-//            to its own barrier, so the epilogue starts on the link scores
-//            while the tensor cores finish V_E and S
-//   softmax  P2 = exp(S'^T - max) over the tile's valid rows (part = a
-//            quarter of the tokens; the lane's max and sum reduced over the
-//            parts) over X^lo; V_E as bf16 over the G image; P = softmax of
-//            each head's L scores (part = head) over X^hi
-//   MMAs     P2 V_E ([128, 256); lane (h, k) keeps head h's 32 columns) and
-//            Yd = P VO ([0, 128), the history branch already through Wo)
+// (a tile never spans two users; rows past `nv` are masked), with mu, rstd the
+// LN1 statistics of each raw history row E (the affine part of LN1 is folded
+// into the images: see the link projections):
+//   MMAs     S'^T = Q'g E^T (link scores, (head, link) on the TMEM lanes;
+//            [128, 256) or [384, 512) by tile parity), V_E = E (g1 Wv) (hi +
+//            lo, [256, 384)), S = E G' (history scores, [0, H*L)), each group
+//            committed to its own barrier.  They need only the raw E tile, so
+//            they start as soon as it lands, while the epilogue finishes the
+//            previous tile.
+//   stats    mu, rstd per row (reduced over the four column parts)
+//   softmax  P2 = exp(z - max), z = rstd (S'^T - mu cQ) + dQ per token column,
+//            over the tile's valid rows (part = a quarter of the tokens; the
+//            lane's max and sum reduced over the parts); V_E = rstd (. - mu
+//            cv) + dv as bf16 over the G' image; P = softmax of each head's L
+//            scores rstd (S - mu cG) + dG (part = head) over the E tile
+//   MMAs     P2 V_E (into the link-score columns; lane (h, k) keeps head h's
+//            32 columns) and Yd = P VO ([0, 128), already through Wo)
 //   out      the link record (max, sum, 32 weighted V sums) of each lane;
 //            Yd as fp16 by TMA tensor stores (plain stores for a partial
 //            tile); fp16 keeps 11 bits of the delta, which the residual adds
 //            to E (bf16 would cost E' up to 2^-9 |Yd|)
 // HIST = false (the last layer: E' is not needed) keeps the link branch only.
 //
-// Shared memory: six 32 KB slots.  Wv (resident), G -> V_E, QH -> VO, and
-// three that rotate (A, B, C): A = E tile -> X^hi -> P -> Yd staging, B = X^lo
-// -> P2, C = Q'lo -> the next E tile; the next tile's roles are (C, A, B).
-// Every load is issued as soon as its slot's last reader has completed: the
-// next E tile and VO once the link scores are done, the next G and Q'lo once
-// P2 V_E is done, the next Q'hi once Yd is done.
+// Shared memory: six 32 KB slots.  (g1 Wv)^T hi and lo (resident), G' -> V_E,
+// Q'g -> VO, and two that alternate (A, B): A = E tile -> P -> Yd staging,
+// B = P2 -> the next E tile.  Every load is issued as soon as its slot's last
+// reader has completed: VO (and, in the last layer, the next Q'g) once the
+// link scores are done, the next E tile and G' once P2 V_E is done, the next
+// Q'g once Yd is done.
 // Warps 0-15 (epilogue): thread (row, part), row = 32*(warp%4) + lane (a TMEM
 // lane), part = warp/4; they synchronise among themselves with a named
 // barrier.  Warp 16 (one lane) issues the MMAs and the loads: tcgen05.mma
@@ -615,35 +589,35 @@ __global__ void __launch_bounds__(512, 1)
 // MMA group has started.
 constexpr int kXaEpi = 512;
 constexpr int kXaThreads = kXaEpi + 32;
+constexpr uint32_t kXaSmem = 1024 + 12 * kBlk + 1024 /* mu, rstd */ + 4096 /* red */ +
+                             1024 /* cv, dv */ + 2 * 2048 /* vec x2 */ + 128 /* 14 barriers */;
 
 template <int L, bool HIST>
 __global__ void __launch_bounds__(kXaThreads, 1)
     k_hist_xattn(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
-                 const bf16* __restrict__ g1, const bf16* __restrict__ b1,
                  uint8_t* __restrict__ ws, LayerWs Lw, unsigned* status) {
   constexpr int HL = kH * L;
   constexpr uint32_t kSlot = 2 * kBlk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
-  uint8_t* sW = sm;                 // Wv^T image
-  uint8_t* sG = sm + kSlot;         // G^T -> V_E
-  uint8_t* sQH = sm + 2 * kSlot;    // Q'hi -> VO
-  uint8_t* rot = sm + 3 * kSlot;    // three rotating slots
-  float* red = reinterpret_cast<float*>(sm + 6 * kSlot);
+  uint8_t* sWh = sm;                // (g1 Wv)^T hi
+  uint8_t* sWl = sm + kSlot;        // (g1 Wv)^T lo
+  uint8_t* sG = sm + 2 * kSlot;     // G' -> V_E
+  uint8_t* sQ = sm + 3 * kSlot;     // Q'g -> VO
+  uint8_t* rot = sm + 4 * kSlot;    // two alternating slots
+  float* smu = reinterpret_cast<float*>(sm + 6 * kSlot);   // [128] mu, then [128] rstd
+  float* red = smu + 256;                                   // [1024]
+  float* cvd = red + 1024;                                  // cv [128], dv [128]
+  float* vecs = cvd + 256;                                  // 2 x (cQ, dQ, cG, dG)
   Cta c;
-  // bar: 0 Wv, 1 S' done, 2 E tile, 3 G, 4 Q'hi, 5 Q'lo, 6 VO, 7 V_E done,
-  //      8 S done, 9 P2 V_E done, 10 Yd done, 11 X^ written, 12 P2, V_E, P written
-  cta_setup(sm + 6 * kSlot + kLnBytes, 13, c);
+  // bar: 0 weights, 1 S' done, 2 E tile, 3 G', 4 Q'g + vec, 6 VO, 7 V_E done,
+  //      8 S done, 9 P2 V_E done, 10 Yd done, 11 TMEM read out, 12 P2 and V_E
+  //      written, 13 P written
+  cta_setup(reinterpret_cast<uint8_t*>(vecs + 1024), 14, c);
   uint64_t* bar = c.bar;
-  ln_stage(red + 1024, g1, b1);
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
   const int warp = threadIdx.x >> 5;
-  auto slots = [&](int ia, uint8_t*& sA, uint8_t*& sB, uint8_t*& sC) {
-    sA = rot + ia * kSlot;
-    sB = rot + (ia == 2 ? 0 : ia + 1) * kSlot;
-    sC = rot + (ia == 0 ? 2 : ia - 1) * kSlot;
-  };
   if (warp == kXaEpi / 32) {
     if ((threadIdx.x & 31) == 0) {
       // ---- the issuer: loads and MMAs
@@ -652,74 +626,79 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         mbar_arrive_expect_tx(b, kSlot);
         bulk_load(dst, src, kSlot, b);
       };
+      auto load_q = [&](int u, int it) {   // Q'g and the user's vectors
+        mbar_arrive_expect_tx(&bar[4], kSlot + 2048);
+        bulk_load(sQ, uimg(u) + 2 * kBlk, kSlot, &bar[4]);
+        bulk_load(vecs + (it & 1) * 512, uimg(u) + kUimgVec, 2048, &bar[4]);
+      };
       auto load_e = [&](uint8_t* dst, int r0) {
         mbar_arrive_expect_tx(&bar[2], kSlot);
         tma_load_2d(dst, &tmE, 0, r0, &bar[2]);
         tma_load_2d(dst + kBlk, &tmE, 64, r0, &bar[2]);
       };
       prefetch_tmap(&tmE);
-      load(&bar[0], sW, ws + Lw.img_v);
+      mbar_arrive_expect_tx(&bar[0], 2 * kSlot + 1024);
+      bulk_load(sWh, ws + Lw.img_vg, 2 * kSlot, &bar[0]);
+      bulk_load(cvd, ws + Lw.img_vg + 4 * kBlk, 1024, &bar[0]);
       if ((int)blockIdx.x < n_tiles) {
         const int4 tl = tiles[blockIdx.x];
         load_e(rot, tl.y);
         if (HIST) load(&bar[3], sG, uimg(tl.x));
-        load(&bar[4], sQH, uimg(tl.x) + 2 * kBlk);
-        load(&bar[5], rot + 2 * kSlot, uimg(tl.x) + 4 * kBlk);
+        load_q(tl.x, 0);
       } else {
         mbar_wait(&bar[0], 0, status, c.abort_flag);   // lands before the CTA exits
       }
-      int ia = 0;
+      int ab = 0;
       for (int t = blockIdx.x, it = 0; t < n_tiles; t += gridDim.x, ++it) {
         const int u = tiles[t].x;
         const int tn = t + gridDim.x;
         const int un = tn < n_tiles ? tiles[tn].x : 0;
         const uint32_t ph = (uint32_t)it & 1u;
-        uint8_t *sA, *sB, *sC;
-        slots(ia, sA, sB, sC);
-        mbar_wait(&bar[11], ph, status, c.abort_flag);
+        uint8_t* sA = rot + ab * kSlot;
+        uint8_t* sB = rot + (ab ^ 1) * kSlot;
+        const uint32_t tS2 = c.tmem + 128 + (uint32_t)(it & 1) * 256;
+        mbar_wait(&bar[2], ph, status, c.abort_flag);
         if (it == 0) mbar_wait(&bar[0], 0, status, c.abort_flag);
         mbar_wait(&bar[4], ph, status, c.abort_flag);
-        mbar_wait(&bar[5], ph, status, c.abort_flag);
         tc_fence_after();
-        mma_tile(c.tmem + 128, smem_u32(sQH), kBlk, smem_u32(sA), kBlk, 128, 128, false);
-        mma_tile(c.tmem + 128, smem_u32(sC), kBlk, smem_u32(sA), kBlk, 128, 128, true);
+        mma_tile(tS2, smem_u32(sQ), kBlk, smem_u32(sA), kBlk, 128, 128, false);
         mma_commit(&bar[1]);
-        mma_tile(c.tmem + 256, smem_u32(sA), kBlk, smem_u32(sW), kBlk, 128, 128, false);
-        mma_tile(c.tmem + 256, smem_u32(sB), kBlk, smem_u32(sW), kBlk, 128, 128, true);
+        mma_tile(c.tmem + 256, smem_u32(sA), kBlk, smem_u32(sWh), kBlk, 128, 128, false);
+        mma_tile(c.tmem + 256, smem_u32(sA), kBlk, smem_u32(sWl), kBlk, 128, 128, true);
         mma_commit(&bar[7]);
         if (HIST) {
+          // S overwrites the previous tile's Yd columns: wait for their readout
+          if (it > 0) mbar_wait(&bar[11], ph ^ 1u, status, c.abort_flag);
           mbar_wait(&bar[3], ph, status, c.abort_flag);
           tc_fence_after();
           mma_tile(c.tmem, smem_u32(sA), kBlk, smem_u32(sG), kBlk, HL, 128, false);
           mma_commit(&bar[8]);
         }
-        // the link scores have read Q'hi and Q'lo
+        // the link scores have read Q'g
         mbar_wait(&bar[1], ph, status, c.abort_flag);
-        if (HIST) load(&bar[6], sQH, uimg(u) + 6 * kBlk);
-        else if (tn < n_tiles) load(&bar[4], sQH, uimg(un) + 2 * kBlk);
-        if (tn < n_tiles) load_e(sC, tiles[tn].y);
+        if (HIST) load(&bar[6], sQ, uimg(u) + 4 * kBlk);
+        else if (tn < n_tiles) load_q(un, it + 1);
         mbar_wait(&bar[12], ph, status, c.abort_flag);
         tc_fence_after();
-        mma_tile_bmn(c.tmem + 128, smem_u32(sB), kBlk, smem_u32(sG), kBlk, 128, 128, false);
+        mma_tile_bmn(tS2, smem_u32(sB), kBlk, smem_u32(sG), kBlk, 128, 128, false);
         mma_commit(&bar[9]);
-        if (HIST) {
-          mbar_wait(&bar[6], ph, status, c.abort_flag);
-          tc_fence_after();
-          mma_tile_bmn(c.tmem, smem_u32(sA), kBlk, smem_u32(sQH), kBlk, 128, HL, false);
-          mma_commit(&bar[10]);
-        }
-        // P2 V_E has read V_E and P2: the next G, and the next Q'lo (the next C)
+        // P2 V_E has read P2 and V_E: the next E tile, and the next G'
         mbar_wait(&bar[9], ph, status, c.abort_flag);
         if (tn < n_tiles) {
+          load_e(sB, tiles[tn].y);
           if (HIST) load(&bar[3], sG, uimg(un));
-          load(&bar[5], sB, uimg(un) + 4 * kBlk);
         }
         if (HIST) {
-          // Yd has read P and VO: the next Q'hi
+          mbar_wait(&bar[13], ph, status, c.abort_flag);
+          mbar_wait(&bar[6], ph, status, c.abort_flag);
+          tc_fence_after();
+          mma_tile_bmn(c.tmem, smem_u32(sA), kBlk, smem_u32(sQ), kBlk, 128, HL, false);
+          mma_commit(&bar[10]);
+          // Yd has read P and VO: the next Q'g
           mbar_wait(&bar[10], ph, status, c.abort_flag);
-          if (tn < n_tiles) load(&bar[4], sQH, uimg(un) + 2 * kBlk);
+          if (tn < n_tiles) load_q(un, it + 1);
         }
-        ia = ia == 0 ? 2 : ia - 1;
+        ab ^= 1;
       }
     }
   } else {
@@ -731,30 +710,42 @@ __global__ void __launch_bounds__(kXaThreads, 1)
     bf16* yd = reinterpret_cast<bf16*>(ws + Lw.yd);   // fp16 bits; rows copied as bytes
     float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
     if (HIST && threadIdx.x == 0) prefetch_tmap(&tmY);
-    int ia = 0;
+    int ab = 0;
     for (int t = blockIdx.x, it = 0; t < n_tiles; t += gridDim.x, ++it) {
       const int4 tl = tiles[t];
       const int r0 = tl.y, nv = tl.z;
       const uint32_t ph = (uint32_t)it & 1u;
-      uint8_t *sA, *sB, *sC;
-      slots(ia, sA, sB, sC);
+      uint8_t* sA = rot + ab * kSlot;
+      uint8_t* sB = rot + (ab ^ 1) * kSlot;
+      const uint32_t tS2 = ta + 128 + (uint32_t)(it & 1) * 256;
+      const float* vec = vecs + (it & 1) * 512;   // cQ, dQ, cG, dG
       mbar_wait(&bar[2], ph, status, c.abort_flag);
+      if (it == 0) mbar_wait(&bar[0], 0, status, c.abort_flag);
+      mbar_wait(&bar[4], ph, status, c.abort_flag);
+      // LN1 statistics of this thread's row (biased variance; see layer_norm_part)
+      float mu_r, rs_r;
       {
-        float x[32];
+        float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sA, kBlk, row, c0 + q * 8), x + q * 8);
-        layer_norm_part<kXaEpi>(x, c0, red, part, row);
-        if (HIST && it > 0) {
-          // the previous tile's Yd store has read its staging (this tile's B)
-          if (threadIdx.x == 0) bulk_wait_read<0>();
-          named_bar_sync(1, kXaEpi);
+        for (int q = 0; q < 4; ++q) {
+          float x[8];
+          unpack8(sw_ld16(sA, kBlk, row, c0 + q * 8), x);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) { s1 += x[k]; s2 = fmaf(x[k], x[k], s2); }
         }
-        split_part_st(sA, sB, row, c0, x);
+        red[part * 128 + row] = s1;
+        red[512 + part * 128 + row] = s2;
+        named_bar_sync(1, kXaEpi);
+        mu_r = (red[row] + red[128 + row] + red[256 + row] + red[384 + row]) * (1.0f / kD);
+        const float ex2 =
+            (red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row]) * (1.0f / kD);
+        rs_r = rsqrtf(fmaxf(ex2 - mu_r * mu_r, 0.f) + kLnEps);
+        if (part == 0) {
+          smu[row] = mu_r;
+          smu[128 + row] = rs_r;
+        }
+        named_bar_sync(1, kXaEpi);
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      named_bar_sync(1, kXaEpi);
-      if (threadIdx.x == 0) mbar_arrive(&bar[11]);
       mbar_wait(&bar[1], ph, status, c.abort_flag);
       tc_fence_after();
       // link softmax over the tile's valid rows: row = (head, link) lane,
@@ -762,17 +753,29 @@ __global__ void __launch_bounds__(kXaThreads, 1)
       float lm, ls;
       {
         float z[32];
-        tmem_ld16(ta + 128 + c0, z);
-        tmem_ld16(ta + 128 + c0 + 16, z + 16);
+        tmem_ld16(tS2 + c0, z);
+        tmem_ld16(tS2 + c0 + 16, z + 16);
         tmem_ld_wait();
         const bool link = row < HL;
+        const float cq = link ? vec[row] : 0.f, dq = link ? vec[128 + row] : 0.f;
+        const float4* mu4 = reinterpret_cast<const float4*>(smu + c0);
+        const float4* rs4 = reinterpret_cast<const float4*>(smu + 128 + c0);
         float m = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (c0 + j >= nv || !link) z[j] = -INFINITY;
-          m = fmaxf(m, z[j]);
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 mv = mu4[j4], rv = rs4[j4];
+          const float mj[4] = {mv.x, mv.y, mv.z, mv.w}, rj[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = j4 * 4 + e;
+            z[j] = fmaf(rj[e], fmaf(-mj[e], cq, z[j]), dq);
+            if (c0 + j >= nv || !link) z[j] = -INFINITY;
+            m = fmaxf(m, z[j]);
+          }
         }
         red[part * 128 + row] = m;
+        // B held the previous tile's Yd staging: its store must have read it
+        if (HIST && it > 0 && threadIdx.x == 0) bulk_wait_read<0>();
         named_bar_sync(1, kXaEpi);
         m = fmaxf(fmaxf(red[row], red[128 + row]), fmaxf(red[256 + row], red[384 + row]));
         float s = 0.f;
@@ -785,13 +788,12 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         named_bar_sync(1, kXaEpi);
         lm = m;
         ls = red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row];
-        // P2 over X^lo, whose last reader is the V_E product
-        mbar_wait(&bar[7], ph, status, c.abort_flag);
 #pragma unroll
         for (int q = 0; q < 4; ++q) sw_st16(sB, kBlk, row, c0 + q * 8, pack8(z + q * 8));
       }
       {
-        // V_E (bf16) over the G image (read by S): the MN-major B of P2 V_E
+        // V_E (bf16) over the G' image (read by S): the MN-major B of P2 V_E
+        mbar_wait(&bar[7], ph, status, c.abort_flag);
         if (HIST) mbar_wait(&bar[8], ph, status, c.abort_flag);
         tc_fence_after();
         float v[32];
@@ -799,15 +801,24 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         tmem_ld16(ta + 256 + c0 + 16, v + 16);
         tmem_ld_wait();
 #pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = fmaf(rs_r, fmaf(-mu_r, cvd[c0 + j], v[j]), cvd[kD + c0 + j]);
+#pragma unroll
         for (int q = 0; q < 4; ++q) sw_st16(sG, kBlk, row, c0 + q * 8, pack8(v + q * 8));
       }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(1, kXaEpi);
+      if (threadIdx.x == 0) mbar_arrive(&bar[12]);   // P2 V_E can start
       if (HIST) {
-        // history softmax over the user's L links: part = head, P over X^hi
+        // history softmax over the user's L links: part = head, P over the E tile
         const int h = part;
         float z[L];
 #pragma unroll
         for (int q = 0; q < L / 16; ++q) tmem_ld16(ta + h * L + q * 16, z + q * 16);
         tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < L; ++k)
+          z[k] = fmaf(rs_r, fmaf(-mu_r, vec[256 + h * L + k], z[k]), vec[384 + h * L + k]);
         float m = z[0];
 #pragma unroll
         for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
@@ -819,19 +830,19 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         for (int k = 0; k < L; ++k) z[k] *= inv;
 #pragma unroll
         for (int q = 0; q < L / 8; ++q) sw_st16(sA, kBlk, row, h * L + q * 8, pack8(z + q * 8));
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar_sync(1, kXaEpi);
+        if (threadIdx.x == 0) mbar_arrive(&bar[13]);   // Yd = P VO can start
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      named_bar_sync(1, kXaEpi);
-      if (threadIdx.x == 0) mbar_arrive(&bar[12]);
       mbar_wait(&bar[9], ph, status, c.abort_flag);
       tc_fence_after();
       {
         // link record of row p = (h, k): part h reads head h's 32 columns
         // (warp-uniform TMEM address); rows of other heads skip the store
         float acc[kDH];
-        tmem_ld16(ta + 128 + part * kDH, acc);
-        tmem_ld16(ta + 128 + part * kDH + 16, acc + 16);
+        tmem_ld16(tS2 + part * kDH, acc);
+        tmem_ld16(tS2 + part * kDH + 16, acc + 16);
         tmem_ld_wait();
         if (row < HL && row / L == part) {
           float4* rec = reinterpret_cast<float4*>(part_rec + ((size_t)t * HL + row) * kRec);
@@ -848,6 +859,9 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         tmem_ld16(ta + c0, y);
         tmem_ld16(ta + c0 + 16, y + 16);
         tmem_ld_wait();
+        tc_fence_before();
+        named_bar_sync(1, kXaEpi);   // every thread has read P (the MMA is done) and Yd
+        if (threadIdx.x == 0) mbar_arrive(&bar[11]);
 #pragma unroll
         for (int q = 0; q < 4; ++q) sw_st16(sA, kBlk, row, c0 + q * 8, pack8_f16(y + q * 8));
         fence_proxy_async_smem();
@@ -865,8 +879,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
           }
         }
       }
-      tc_fence_before();
-      ia = ia == 0 ? 2 : ia - 1;   // next (A, B, C) = (C, A, B)
+      ab ^= 1;
     }
     if (threadIdx.x == 0) bulk_wait<0>();
   }
@@ -1444,11 +1457,11 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
   const int64_t nz = B * L;
   const int sms = num_sms();
   {
-    const int64_t n = (4 * kD * kD + 3 * kD * kF) / 8;
-    int rc = launch_pdl(k_prep_weights, dim3((unsigned)(1 + (n + 1023) / 1024)), dim3(1024), 0, st,
+    const int64_t n = (5 * kD * kD + 3 * kD * kF) / 8;
+    int rc = launch_pdl(k_prep_weights, dim3((unsigned)(2 + (n + 1023) / 1024)), dim3(1024), 0, st,
                         1, (const bf16*)w.Wq, (const bf16*)w.Wk, (const bf16*)w.Wv,
                         (const bf16*)w.Wo, (const bf16*)w.W1, (const bf16*)w.W3, (const bf16*)w.W2,
-                        ws, Lw, off, B, nh, status);
+                        (const bf16*)w.g1, (const bf16*)w.b1, ws, Lw, off, B, nh, status);
     if (rc) return rc;
   }
   {
@@ -1469,11 +1482,10 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     const int64_t tiles_hi = Lw.max_tiles;
     const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
     {
-      const int smem = 1024 + 12 * kBlk + kLnBytes + 128;   // 13 barriers
       auto kern = last ? k_hist_xattn<L, false> : k_hist_xattn<L, true>;
-      if (!set_smem(kern, smem)) return LIME_ERR_CUDA;
-      int rc = launch_pdl(kern, dim3(grid), dim3(kXaThreads), smem, st, 1, tmE, tmY, (const bf16*)w.g1,
-                          (const bf16*)w.b1, ws, Lw, status);
+      if (!set_smem(kern, kXaSmem)) return LIME_ERR_CUDA;
+      int rc = launch_pdl(kern, dim3(grid), dim3(kXaThreads), kXaSmem, st, 1, tmE, tmY, ws, Lw,
+                          status);
       if (rc) return rc;
     }
     if (!last) {

@@ -268,6 +268,8 @@ def main():
     ap.add_argument("--impl", default="lime", choices=["lime", "reference"])
     ap.add_argument("--workload", default="standard")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="time the step as eager library calls instead of CUDA graph replays")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -294,17 +296,27 @@ def main():
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def step_events():
-        return [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-
     for _ in range(args.warmup):
         flush.zero_()
         pipeline.step(x, buf)
     torch.cuda.synchronize()
     if lime.lime_get_status(buf.ws) != 0:
         raise RuntimeError("device status flags set during warm-up")
+    l0 = lime.lime_launch_count()
+    pipeline.step(x, buf)
+    launches_per_step = lime.lime_launch_count() - l0
 
-    evs = [step_events() for _ in range(args.steps)]
+    # The step's launches are captured once in CUDA graphs (the whole step, and
+    # its three phases for the per-phase times) and replayed; --eager times
+    # the same library calls issued one by one from Python instead.
+    graphs = None if args.eager else pipeline.step_graphs(x, buf)
+    if graphs:
+        for _ in range(args.warmup):
+            flush.zero_()
+            graphs[0].replay()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     sampler = ClockSampler(local)
     if dist:
         dist.barrier()
@@ -314,30 +326,50 @@ def main():
     with sampler:
         for k in range(args.steps):
             flush.zero_()
-            e = evs[k]
-            e[0].record(stream)
+            evs[k][0].record(stream)
+            if graphs:
+                graphs[0].replay()
+            else:
+                pipeline.step(x, buf)
+            evs[k][1].record(stream)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+    t_wall = time.perf_counter() - t_wall
+    launches = (launches_per_step * args.steps if graphs
+                else lime.lime_launch_count() - launches0)
+    total_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    total_ms = max_over_ranks([total_ms], dist, "cuda")[0]
+    ms_step = total_ms / args.steps
+    value = job_throughput(world, total_cand, ms_step)
+
+    # per-phase times: the same step as three consecutive phases
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush.zero_()
+        e = pev[k]
+        e[0].record(stream)
+        if graphs:
+            graphs[1].replay()
+            e[1].record(stream)
+            graphs[2].replay()
+            e[2].record(stream)
+            graphs[3].replay()
+        else:
             pipeline.fold_qk(x, buf)
             LP = pipeline.user_encode(x, buf)
             e[1].record(stream)
             pipeline.build_cache(x, buf)
             e[2].record(stream)
             pipeline.score(x, buf, LP)
-            e[3].record(stream)
-        torch.cuda.synchronize()
-        if dist:
-            dist.barrier()
-    t_wall = time.perf_counter() - t_wall
-    launches = lime.lime_launch_count() - launches0
+        e[3].record(stream)
+    torch.cuda.synchronize()
     ph = {"user": 0.0, "cache": 0.0, "score": 0.0}
-    total_ms = 0.0
-    for e in evs:
+    for e in pev:
         ph["user"] += e[0].elapsed_time(e[1])
         ph["cache"] += e[1].elapsed_time(e[2])
         ph["score"] += e[2].elapsed_time(e[3])
-        total_ms += e[0].elapsed_time(e[3])
-    total_ms = max_over_ranks([total_ms], dist, "cuda")[0]
-    ms_step = total_ms / args.steps
-    value = job_throughput(world, total_cand, ms_step)
+    ph = dict(zip(ph, max_over_ranks(list(ph.values()), dist, "cuda")))
 
     # end to end through the public API: pinned host inputs in, scores out
     host = {"E": x.E.cpu().pin_memory(), "ctx": x.ctx.cpu().pin_memory() if x.ctx is not None else None,
@@ -522,7 +554,9 @@ def main():
                 "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
                 "data": "synthetic (seeded; shapes of the pages' workloads)",
-                "config": config_of(w, total_cand, total_hist),
+                "config": dict(config_of(w, total_cand, total_hist),
+                               launch="eager library calls" if args.eager else
+                               "CUDA graph replay of the step's captured library launches"),
                 "phases": phases, "roofline": roof,
                 "clocks": sampler.summary(),
                 "e2e": {"value": job_throughput(world, total_cand, e2e_step_ms), "unit": "pairs/s",

@@ -53,7 +53,7 @@ class Buffers:
     image: Optional[torch.Tensor] = None          # folded G^T operand image
     side: Optional[torch.cuda.Stream] = None      # stream the fold runs on
     fold_done: Optional[torch.cuda.Event] = None
-    fold_pending: bool = False
+    fold_state: Optional[str] = None              # None, "pending" (forked) or "joined"
 
 
 def to_device(w: synth.Workload, us: synth.UserSide, cs: synth.CandidateSide,
@@ -105,7 +105,15 @@ def fold_qk(x: DeviceInputs, buf: Buffers, stream=None):
     buf.side.wait_stream(main)
     lime.lime_fold_qk(x.dims, x.L, x.Wq_c, x.Wk_c, buf.image, stream=buf.side)
     buf.fold_done.record(buf.side)
-    buf.fold_pending = True
+    buf.fold_state = "pending"
+
+
+def join_fold(buf: Buffers, stream=None):
+    """Makes ``stream`` wait for a forked fold (no-op if none is pending)."""
+    if buf.fold_state == "pending":
+        main = torch.cuda.current_stream() if stream is None else stream
+        main.wait_event(buf.fold_done)
+        buf.fold_state = "joined"
 
 
 def user_encode(x: DeviceInputs, buf: Buffers, stream=None) -> torch.Tensor:
@@ -129,10 +137,10 @@ def user_encode(x: DeviceInputs, buf: Buffers, stream=None) -> torch.Tensor:
 
 def build_cache(x: DeviceInputs, buf: Buffers, stream=None):
     """The QK cache; the catalogue pass alone when fold_qk started this step."""
-    if buf.fold_pending:
+    if buf.fold_state is not None:
         main = torch.cuda.current_stream() if stream is None else stream
-        main.wait_event(buf.fold_done)
-        buf.fold_pending = False
+        join_fold(buf, main)
+        buf.fold_state = None
         lime.lime_build_qk_cache_folded(x.dims, x.T, buf.image, buf.cache, buf.ws, stream=main)
     else:
         lime.lime_build_qk_cache(x.dims, x.T, x.L, x.Wq_c, x.Wk_c, buf.cache, buf.ws,
@@ -151,3 +159,29 @@ def step(x: DeviceInputs, buf: Buffers, stream=None) -> torch.Tensor:
     build_cache(x, buf, stream)
     score(x, buf, LP, stream)
     return buf.O
+
+
+def capture(fn) -> torch.cuda.CUDAGraph:
+    """Captures ``fn`` (library calls on the current stream, and the fold's side
+    stream forked and joined inside it) into a CUDA graph."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def step_graphs(x: DeviceInputs, buf: Buffers):
+    """CUDA graphs of one step: (whole step, user side, cache, scoring).
+
+    The user-side graph forks the fold stage and joins it at its end; the
+    cache graph then runs the catalogue pass alone."""
+    def user():
+        fold_qk(x, buf)
+        user_encode(x, buf)
+        join_fold(buf)
+    LP = buf.Z_bufs[(len(x.layers) - 1) % 2]
+    g_step = capture(lambda: step(x, buf))
+    g_user = capture(user)
+    g_cache = capture(lambda: build_cache(x, buf))
+    g_score = capture(lambda: score(x, buf, LP))
+    return g_step, g_user, g_cache, g_score

@@ -59,3 +59,21 @@ def test_forked_step_matches_single_stream_step():
     torch.cuda.synchronize()
     assert lime.lime_get_status(buf.ws) == 0
     assert torch.equal(O_fork.view(torch.int16), buf.O.view(torch.int16))
+
+
+def test_graph_replay_matches_eager():
+    # the step captured in CUDA graphs (whole step; and user side, cache,
+    # scoring as three graphs) replays to the eager step's scores bit for bit
+    w = synth.workload("standard", B=8, n_items=5000)
+    x = pipeline.to_device(w, synth.user_side(w), synth.candidate_side(w), synth.item_table(w))
+    buf = pipeline.alloc(x)
+    O_eager = pipeline.step(x, buf).clone()
+    graphs = pipeline.step_graphs(x, buf)
+    for replay in ([graphs[0]], graphs[1:]):
+        buf.O.zero_()
+        buf.cache.zero_()
+        for g in replay:
+            g.replay()
+        torch.cuda.synchronize()
+        assert lime.lime_get_status(buf.ws) == 0
+        assert torch.equal(O_eager.view(torch.int16), buf.O.view(torch.int16))

@@ -426,6 +426,24 @@ def main():
     sc_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in sc_ev)], dist,
                            "cuda")[0] / args.steps
 
+    # Uncached (online) scoring at scale: the same IDs, with the weights computed
+    # per candidate from the item table and the folded G image.
+    on_ms = None
+    if buf.image is not None and w.l in (16, 32):
+        on_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        for _ in range(3):
+            lime.lime_score_candidates_uncached(x.dims, x.T, buf.image, sc_ids, sc_off,
+                                                sc_users * sc_per, sc_LP, sc_O, buf.ws)
+        for k in range(args.steps):
+            flush.zero_()
+            on_ev[k][0].record(stream)
+            lime.lime_score_candidates_uncached(x.dims, x.T, buf.image, sc_ids, sc_off,
+                                                sc_users * sc_per, sc_LP, sc_O, buf.ws)
+            on_ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        on_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in on_ev)], dist,
+                               "cuda")[0] / args.steps
+
     # The int8 cache variant (one byte per weight): its build over the whole
     # catalogue and the same scoring at scale from it.
     u8 = None
@@ -534,6 +552,15 @@ def main():
         }
         if lin is not None:
             phases["user_encode_linearity"] = lin
+        if on_ms is not None:
+            on_bytes = sc_pairs * (4 * w.d + 4)   # item row in, score row out, ID
+            on_gbs = on_bytes / (on_ms * 1e-3) / 1e9
+            phases["score_uncached_at_scale"] = {
+                "ms": on_ms, "pairs": sc_pairs, "pairs_per_s": sc_pairs / (on_ms * 1e-3),
+                "note": "weights computed per candidate from the item table (no cache)",
+                "ids": f"uniform over {w.n_items} items, L2 flushed before each call",
+                "roofline": {"bound": "hbm", "achieved": on_gbs, "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "frac": on_gbs / pk["hbm_gbs"]}}
         if u8 is not None:
             c8_bytes = w.n_items * (2 * w.d + w.H * w.l)
             s8_bytes = sc_pairs * (w.H * w.l + 4 + 2 * w.d)

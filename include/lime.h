@@ -130,6 +130,24 @@ int lime_build_qk_cache_folded(const lime_dims* dims, const void* T, int64_t n_i
                                const void* image, void* cache_out, void* workspace,
                                size_t workspace_bytes, cudaStream_t stream);
 
+/* Uncached (online) candidate scoring: the same O_m as
+ * lime_score_candidates, with the weights computed per candidate from the item
+ * table instead of read from a QK cache,
+ *   O[m, h-cols] = sum_k softmax_k(s (T[id_m] Wq_c)_h . (L Wk_c)_{k,h}) LP_u[k, h-cols]
+ * (LIME note 关键设计 1, O = MHA(T, L, L^P); LIME listing Table 10
+ * "uncached global"; the cold-start path for items not in the cache).
+ *   T        device [n_items, d] item table, 16-byte aligned.
+ *   image    device, the folded G image written by lime_fold_qk for the same
+ *            dims, L, Wq_c, Wk_c (lime_qk_image_bytes(dims) bytes).
+ * Other arguments, checks, flags and errors as lime_score_candidates (an
+ * out-of-range ID sets LIME_FLAG_BAD_ID and its row of O is zero).
+ * Supported: bf16, d = 128, H = 4, l in {16, 32} (else LIME_ERR_SHAPE).    */
+int lime_score_candidates_uncached(const lime_dims* dims, int64_t B, const void* T,
+                                   int64_t n_items, const void* image, const int32_t* cand_ids,
+                                   const int64_t* cand_offsets, int64_t total_cand, const void* LP,
+                                   void* O_out, void* workspace, size_t workspace_bytes,
+                                   cudaStream_t stream);
+
 /* Allocation-free variant of lime_build_qk_cache.  The paper has no
  * counterpart: it exists for callers that cannot allocate device memory, such
  * as a plug-in whose host framework owns the whole device memory pool, or a

@@ -222,6 +222,37 @@ int lime_score_candidates(const lime_dims* dims, int64_t B, const void* cache, i
   return launch_status("lime_score_candidates");
 }
 
+int lime_score_candidates_uncached(const lime_dims* dims, int64_t B, const void* T,
+                                   int64_t n_items, const void* image, const int32_t* cand_ids,
+                                   const int64_t* cand_offsets, int64_t total_cand, const void* LP,
+                                   void* O_out, void* workspace, size_t workspace_bytes,
+                                   cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->dtype != LIME_BF16 || !fast_online_supported(*dims) || !lime_qk_image_bytes(dims))
+    return LIME_ERR_SHAPE;
+  if (B < 0 || B > INT32_MAX || n_items < 0 || total_cand < 0) return LIME_ERR_ARG;
+  if (B == 0) return total_cand == 0 ? LIME_OK : LIME_ERR_ARG;
+  if (!cand_offsets || !LP || !image || ((uintptr_t)cand_offsets & 7)) return LIME_ERR_ARG;
+  if (total_cand > 0 && (!cand_ids || !O_out || !T)) return LIME_ERR_ARG;
+  if (!aligned16(LP) || !aligned16(image) || (O_out && !aligned16(O_out)) ||
+      (T && !aligned16(T)) || ((uintptr_t)cand_ids & 3))
+    return LIME_ERR_ARG;
+  if ((rc = check_ws(workspace, workspace_bytes, dims, 0, 0))) return rc;
+  const size_t es = esize(dims);
+  const size_t o_sz = (size_t)total_cand * dims->d * es;
+  if (overlap(O_out, o_sz, T, (size_t)n_items * dims->d * es) ||
+      overlap(O_out, o_sz, image, lime_qk_image_bytes(dims)) ||
+      overlap(O_out, o_sz, LP, (size_t)B * dims->l * dims->d * es) ||
+      overlap(O_out, o_sz, cand_ids, (size_t)total_cand * 4))
+    return LIME_ERR_ALIAS;
+  if (total_cand == 0) return LIME_OK;
+  if ((rc = fast_score_online(*dims, B, T, n_items, image, cand_ids, cand_offsets, total_cand, LP,
+                              O_out, status_of(workspace), stream)))
+    return rc;
+  return launch_status("lime_score_candidates_uncached");
+}
+
 size_t lime_qk_image_bytes(const lime_dims* dims) {
   if (!dims || check_dims(dims) || dims->dtype != LIME_BF16 || !fast_cache_supported(*dims))
     return 0;

@@ -49,6 +49,12 @@ int fast_fold_qk(const lime_dims& D, const void* L, const void* Wq, const void* 
 int fast_build_qk_cache_folded(const lime_dims& D, const void* T, int64_t n, const void* image,
                                void* cache, unsigned* status, cudaStream_t st);
 
+// uncached (online) scoring from the item table and the folded G image
+bool fast_online_supported(const lime_dims& D);
+int fast_score_online(const lime_dims& D, int64_t B, const void* T, int64_t n_items,
+                      const void* image, const int32_t* ids, const int64_t* off, int64_t total,
+                      const void* LP, void* O, unsigned* status, cudaStream_t st);
+
 // int8 cache (bytes q = round(255 w)); needs H*l >= 128
 bool fast_cache_u8_supported(const lime_dims& D);
 int fast_build_qk_cache_u8(const lime_dims& D, const void* T, int64_t n, const void* L,

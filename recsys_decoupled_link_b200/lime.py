@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "lime_qk_image_bytes": (SZ, [D]),
         "lime_fold_qk": (I32, [D, P, P, P, P, P]),
         "lime_build_qk_cache_folded": (I32, [D, P, I64, P, P, P, SZ, P]),
+        "lime_score_candidates_uncached": (I32, [D, I64, P, I64, P, P, P, I64, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -82,7 +83,7 @@ EXPORTED = ("lime_workspace_bytes", "lime_workspace_init", "lime_build_qk_cache"
             "lime_context_links", "lime_xor_layer", "lime_score_candidates",
             "lime_get_status", "lime_launch_count", "lime_build_qk_cache_noalloc",
             "lime_build_qk_cache_u8", "lime_score_candidates_u8", "lime_qk_image_bytes",
-            "lime_fold_qk", "lime_build_qk_cache_folded")
+            "lime_fold_qk", "lime_build_qk_cache_folded", "lime_score_candidates_uncached")
 
 
 def library_path() -> str:
@@ -168,6 +169,16 @@ def lime_build_qk_cache_folded(dims, T, image, cache_out, ws: Workspace, stream=
     n_items = 0 if T is None else T.shape[0]
     _check("lime_build_qk_cache_folded", _lib.lime_build_qk_cache_folded(
         ctypes.byref(dims), _ptr(T), n_items, _ptr(image), _ptr(cache_out), ws.ptr, ws.nbytes,
+        _stream(stream)))
+
+
+def lime_score_candidates_uncached(dims, T, image, cand_ids, cand_offsets, total_cand, LP, O_out,
+                                   ws: Workspace, stream=None):
+    """Uncached scoring: weights computed per candidate from T and the G image."""
+    B = cand_offsets.shape[0] - 1
+    _check("lime_score_candidates_uncached", _lib.lime_score_candidates_uncached(
+        ctypes.byref(dims), B, _ptr(T), T.shape[0], _ptr(image), _ptr(cand_ids),
+        _ptr(cand_offsets), int(total_cand), _ptr(LP), _ptr(O_out), ws.ptr, ws.nbytes,
         _stream(stream)))
 
 

@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
         "lime_context_links", "lime_xor_layer", "lime_score_candidates", "lime_get_status",
         "lime_launch_count", "lime_build_qk_cache_noalloc", "lime_build_qk_cache_u8",
         "lime_score_candidates_u8", "lime_qk_image_bytes", "lime_fold_qk",
-        "lime_build_qk_cache_folded"])
+        "lime_build_qk_cache_folded", "lime_score_candidates_uncached"])
 
 
 def test_library_exports_every_declared_symbol(lime):
@@ -135,3 +135,18 @@ def test_host_validation_of_two_stage_cache(lime):
              None) == lime.LIME_ERR_ARG
     assert g(ctypes.byref(dims), 0x100000, 10, 0x200000, 0x300000, 0x1000000, 64,
              None) == lime.LIME_ERR_ARG                                       # ws too small
+
+
+def test_host_validation_of_uncached_scoring(lime):
+    dims = lime.make_dims(128, 4, 32, 256, 64, "bf16")
+    nws = lime.lime_workspace_bytes(dims, 0, 0)
+    f = lime._lib.lime_score_candidates_uncached
+    args = lambda **k: [ctypes.byref(k.get("dims", dims)), 1, k.get("T", 0x100000), 100,
+                        k.get("image", 0x200000), 0x300000, 0x400000, 5, 0x500000,
+                        k.get("O", 0x600000), 0x1000000, nws, None]
+    assert f(*args(image=None)) == lime.LIME_ERR_ARG
+    assert f(*args(image=0x200008)) == lime.LIME_ERR_ARG                    # unaligned
+    assert f(*args(O=0x100000 + 512)) == lime.LIME_ERR_ALIAS               # O inside T
+    assert f(*args(O=0x200000)) == lime.LIME_ERR_ALIAS                     # O over the image
+    assert f(*args(dims=lime.make_dims(128, 4, 64, 256, 64, "bf16"))) == lime.LIME_ERR_SHAPE
+    assert f(*args(dims=lime.make_dims(128, 4, 32, 256, 64, "f32"))) == lime.LIME_ERR_SHAPE

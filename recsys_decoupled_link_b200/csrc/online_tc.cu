@@ -15,7 +15,11 @@
 //   MMA 2    per head [128 x l] x [l x 32] against L^P_u^T, as in cached
 //            scoring (TMEM [128, 256))
 //   out      O rows in bf16 through the same stage, coalesced 16-byte stores.
-// CTA (u, g) walks tiles g, g + G, ... of user u's candidates; 128 threads.
+// CTA (u, g) walks tiles g, g + G, ... of user u's candidates with four
+// warpgroups that take turns (tile j of the CTA goes to group j % 4): each has
+// its own gather stage, 128 TMEM columns (S, then O over it) and MMA barrier,
+// so the groups' gathers, MMAs and softmaxes overlap one another.  Thread =
+// candidate row (a TMEM lane) within its group.
 // An out-of-range ID gives a zero row of T (so uniform weights) and
 // LIME_FLAG_BAD_ID; its O row is written as zero.  No workspace is used.
 #include "lime_fast.cuh"
@@ -34,14 +38,17 @@ template <int L>
 struct OnlineCfg {
   static constexpr int HL = kH * L;
   static constexpr uint32_t kStage = 2 * kBlk;         // [128 x 128] bf16 gather stage
-  static constexpr uint32_t OFF_B = 2 * kStage;        // L^P_u^T
+  static constexpr uint32_t OFF_B = 4 * kStage;        // L^P_u^T (after 4 groups' stages)
   static constexpr uint32_t OFF_G = OFF_B + kBlk;      // G image: 2 blocks of HL x 128 bytes
   static constexpr uint32_t OFF_BAR = OFF_G + 2 * HL * 128;
-  static constexpr int SMEM = 1024 + OFF_BAR + 64 + 2 * 128 * 8;
+  static constexpr int SMEM = 1024 + OFF_BAR + 64 + 4 * 128 * 4;
 };
 
+constexpr int kGroups = 4;
+constexpr int kOnThreads = 128 * kGroups;
+
 template <int L>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kOnThreads, 1)
     k_score_online(const bf16* __restrict__ T, int64_t n_items, const uint8_t* __restrict__ gimg,
                    const int32_t* __restrict__ ids, const int64_t* __restrict__ off, int64_t B,
                    int64_t total, const bf16* __restrict__ LP, bf16* __restrict__ O,
@@ -51,13 +58,12 @@ __global__ void __launch_bounds__(128)
   constexpr int CH = 2 * kD / 16;            // 16-byte chunks per item row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA0 = sm;                         // 2 gather stages
   uint8_t* sB = sm + C::OFF_B;
   uint8_t* sG = sm + C::OFF_G;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);   // [0] mma, [1] G image
-  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 2);
-  int* abort_flag = reinterpret_cast<int*>(bar + 3);
-  int64_t* s_ids = reinterpret_cast<int64_t*>(bar + 4);   // [2][128] IDs per stage (-1: zero row)
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);   // [0..3] mma per group, [4] G
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 5);
+  int* abort_flag = reinterpret_cast<int*>(bar + 6);
+  int32_t* s_ids_all = reinterpret_cast<int32_t*>(bar + 8);   // [group][128]
 
   pdl_wait();
   const int64_t u = blockIdx.x;
@@ -66,65 +72,31 @@ __global__ void __launch_bounds__(128)
   const int nt = (int)((b - a + kTile - 1) / kTile);
   if ((int)blockIdx.y >= nt) return;   // uniform over the CTA: nothing allocated yet
 
-  const int i = threadIdx.x;
-  if (i == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+  const int tid = threadIdx.x;
+  const int i = tid & 127;                   // row (and TMEM lane) within the group
+  const int grp = tid >> 7;                  // warpgroup 0 .. kGroups-1
+  if (tid == 0) {
+    for (int q = 0; q <= kGroups; ++q) mbar_init(&bar[q], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (i < 32) tmem_alloc(slot, 256);
+  if (tid < 32) tmem_alloc(slot, 512);
   __syncthreads();
   pdl_launch();   // after the TMEM allocation (the next kernel may allocate before it waits)
-  if (i == 0) {
-    mbar_arrive_expect_tx(&bar[1], 2 * HL * 128);
-    bulk_load(sG, gimg, 2 * HL * 128, &bar[1]);
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bar[kGroups], 2 * HL * 128);
+    bulk_load(sG, gimg, 2 * HL * 128, &bar[kGroups]);
   }
-  const int G = (int)gridDim.y;
-  constexpr int64_t kNoRow = INT64_MIN;
-  auto load_id = [&](int t) -> int64_t {
-    const int64_t m = a + (int64_t)t * kTile + i;
-    return (t < nt && m < b) ? (int64_t)ids[m] : kNoRow;
-  };
-  auto put_id = [&](int stage, int64_t id) {
-    if (id == kNoRow) {
-      id = -1;
-    } else if (id < 0 || id >= n_items) {
-      raise_flag(status, LIME_FLAG_BAD_ID);
-      id = -2;   // a zero row whose output is written as zero
-    }
-    s_ids[stage * kTile + i] = id;
-  };
-  // gather of one tile's item rows: chunk q*128 + i is chunk (idx % CH) of
-  // row idx / CH, so a warp reads whole rows; rows without an item are zero
-  auto gather = [&](int stage) {
-    uint8_t* dstA = sA0 + stage * C::kStage;
-#pragma unroll
-    for (int q = 0; q < CH; ++q) {
-      const int idx = q * 128 + i, r = idx / CH, cc = idx % CH;
-      const int64_t id = s_ids[stage * kTile + r];
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(T) + (id < 0 ? 0 : id * 2 * kD) + cc * 16;
-      cp_async16(dstA + (cc >> 3) * kBlk + sw128_offset(r, (cc & 7) * 8), src, id >= 0);
-    }
-    cp_async_commit();
-  };
-  int64_t id_cur = load_id(blockIdx.y);
-  int64_t id_nxt = load_id(blockIdx.y + G);
-  // L^P_u transposed into sB: element (c, k) at sw128_offset(c, k), k >= L zero
+  // L^P_u transposed into sB: element (c, k) at sw128_offset(c, k), k >= L zero;
+  // staged through the first gather stage (unused yet)
   {
     const uint4* lp = reinterpret_cast<const uint4*>(LP + (u * L) * kD);
-    uint4* stage = reinterpret_cast<uint4*>(sA0 + C::kStage);   // [L][128] bf16 in stage 1
-    uint4 lv[L * kD / 8 / 128];
-#pragma unroll
-    for (int q = 0; q < L * kD / 8 / 128; ++q) lv[q] = __ldg(lp + q * 128 + i);
-#pragma unroll
-    for (int q = 0; q < L * kD / 8 / 128; ++q) stage[q * 128 + i] = lv[q];
-    put_id(0, id_cur);
+    uint4* stage = reinterpret_cast<uint4*>(sm);
+    for (int idx = tid; idx < L * kD / 8; idx += kOnThreads) stage[idx] = __ldg(lp + idx);
     __syncthreads();
-    gather(0);
-    const bf16* st = reinterpret_cast<const bf16*>(sA0 + C::kStage);
+    const bf16* st = reinterpret_cast<const bf16*>(sm);
 #pragma unroll
-    for (int k8 = 0; k8 < 8; ++k8) {
+    for (int k8 = grp * (8 / kGroups); k8 < (grp + 1) * (8 / kGroups); ++k8) {
       float f[8];
 #pragma unroll
       for (int z = 0; z < 8; ++z) {
@@ -134,35 +106,67 @@ __global__ void __launch_bounds__(128)
       sw_st16(sB, kBlk, i, k8 * 8, pack8(f));
     }
   }
-  __syncthreads();   // stage 1 is free again
-  mbar_wait(&bar[1], 0, status, abort_flag);   // the G image
-  const uint32_t tmem = *slot;
+  fence_proxy_async_smem();
+  __syncthreads();   // sB is complete and the staging stage is free again
+  mbar_wait(&bar[kGroups], 0, status, abort_flag);   // the G image
+  const uint32_t tmem = *slot + (uint32_t)grp * 128;   // this group's S, then O
   const uint32_t ta = tmem + ((uint32_t)(i & ~31) << 16);
+  const int G = (int)gridDim.y;
+  const int step = kGroups * G;              // a group's stride over the user's tiles
+  const int t0 = blockIdx.y + grp * G;
+  uint8_t* sA = sm + grp * C::kStage;        // this group's stage
+  int32_t* s_ids = s_ids_all + grp * 128;
+  uint64_t* mbar = &bar[grp];
+  auto gsync = [&]() { named_bar_sync(1 + grp, 128); };
+  constexpr int64_t kNoRow = INT64_MIN;
+  auto load_id = [&](int t) -> int64_t {
+    const int64_t m = a + (int64_t)t * kTile + i;
+    return (t < nt && m < b) ? (int64_t)ids[m] : kNoRow;
+  };
+  auto put_id = [&](int64_t id) {
+    int32_t v;
+    if (id == kNoRow) {
+      v = -1;
+    } else if (id < 0 || id >= n_items) {
+      raise_flag(status, LIME_FLAG_BAD_ID);
+      v = -2;   // a zero row whose output is written as zero
+    } else {
+      v = (int32_t)id;
+    }
+    s_ids[i] = v;
+  };
+  // gather of one tile's item rows: chunk q*128 + i is chunk (idx % CH) of row
+  // idx / CH, so a warp reads whole rows; rows without an item are zero
+  auto gather = [&]() {
+#pragma unroll
+    for (int q = 0; q < CH; ++q) {
+      const int idx = q * 128 + i, r = idx / CH, cc = idx % CH;
+      const int64_t id = s_ids[r];
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(T) + (id < 0 ? 0 : id * 2 * kD) + cc * 16;
+      cp_async16(sA + (cc >> 3) * kBlk + sw128_offset(r, (cc & 7) * 8), src, id >= 0);
+    }
+    cp_async_commit();
+  };
+  int64_t id_cur = load_id(t0);
   uint32_t ph = 0;
-  int it = 0;
-  for (int t = blockIdx.y; t < nt; t += G, ++it) {
-    const int cur = it & 1, nxt = cur ^ 1;
+  for (int t = t0; t < nt; t += step) {
     const int64_t m0 = a + (int64_t)t * kTile;
     const int nv = b - m0 < kTile ? (int)(b - m0) : kTile;
-    const bool more = t + G < nt;
-    if (more) {
-      put_id(nxt, id_nxt);
-      __syncthreads();
-      gather(nxt);                  // tile t+G streams in during tile t
-      id_nxt = load_id(t + 2 * G);
-    }
-    if (more) cp_async_wait<1>(); else cp_async_wait<0>();
-    uint8_t* sA = sA0 + cur * C::kStage;
-    const bool bad = s_ids[cur * kTile + i] == -2;
+    put_id(id_cur);
+    gsync();
+    gather();
+    id_cur = load_id(t + step);     // the group's next IDs while the rows stream in
+    cp_async_wait<0>();
+    const bool bad = s_ids[i] == -2;
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    gsync();
     if (i == 0) {
       tc_fence_after();
       mma_tile(tmem, smem_u32(sA), kBlk, smem_u32(sG), HL * 128, HL, kD, false);
-      mma_commit(&bar[0]);
+      mma_commit(mbar);
     }
-    mbar_wait(&bar[0], ph, status, abort_flag);
+    mbar_wait(mbar, ph, status, abort_flag);
     ph ^= 1u;
     tc_fence_after();
     {
@@ -189,46 +193,49 @@ __global__ void __launch_bounds__(128)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    gsync();
     if (i == 0) {
       tc_fence_after();
+      // O over the score columns (every thread has read its scores)
 #pragma unroll
       for (int h = 0; h < kH; ++h) {
         const uint32_t aa = smem_u32(sA + ((h * L) >> 6) * kBlk + ((h * L) & 63) * 2);
         const uint32_t bb = smem_u32(sB + h * kDH * 128);
-        mma_tile(tmem + 128 + h * kDH, aa, kBlk, bb, kBlk, kDH, L, false);
+        mma_tile(tmem + h * kDH, aa, kBlk, bb, kBlk, kDH, L, false);
       }
-      mma_commit(&bar[0]);
+      mma_commit(mbar);
     }
-    mbar_wait(&bar[0], ph, status, abort_flag);
+    mbar_wait(mbar, ph, status, abort_flag);
     ph ^= 1u;
     tc_fence_after();
-    {
-      // thread = row: TMEM -> bf16 -> swizzled staging in sA (MMA 2 is done with it)
-      float row[kD];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) tmem_ld16(ta + 128 + q * 16, row + q * 16);
+    for (int hf = 0; hf < 2; ++hf) {
+      // thread = row, half hf of its columns: TMEM -> bf16 -> swizzled staging
+      // in sA (MMA 2 is done with it)
+      float row[64];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld16(ta + hf * 64 + q * 16, row + q * 16);
       tmem_ld_wait();
       if (bad) {
 #pragma unroll
-        for (int c = 0; c < kD; ++c) row[c] = 0.f;
+        for (int c = 0; c < 64; ++c) row[c] = 0.f;
       }
 #pragma unroll
-      for (int c = 0; c < 16; ++c) sw_st16(sA, kBlk, i, c * 8, pack8(row + c * 8));
+      for (int c = 0; c < 8; ++c) sw_st16(sA, kBlk, i, hf * 64 + c * 8, pack8(row + c * 8));
     }
     tc_fence_before();
-    __syncthreads();
+    gsync();
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
       const int idx = q * 128 + i, r = idx / 16, cc = idx % 16;
       if (r < nv)
         reinterpret_cast<uint4*>(O + (m0 + r) * kD)[cc] = sw_ld16(sA, kBlk, r, cc * 8);
     }
-    __syncthreads();   // this stage and TMEM are reused two tiles on
   }
-  if (i < 32) {
+  __syncthreads();
+  if (tid < 32) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(*slot, 512);
   }
 }
 
@@ -240,13 +247,14 @@ int launch_online(int64_t B, const void* T, int64_t n_items, const void* image, 
   if (cudaFuncSetAttribute(k_score_online<L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::SMEM) != cudaSuccess)
     return LIME_ERR_CUDA;
-  const int64_t target = 2LL * num_sms();
-  int64_t G = (target + B - 1) / B;
+  // one CTA per SM (its TMEM allocation is all 512 columns): (user, slot) CTAs
+  // in a single wave, as many slots per user as fit
+  int64_t G = num_sms() / B;
   const int64_t tiles_hi = (total + kTile - 1) / kTile;
   if (G > tiles_hi) G = tiles_hi;
   if (G < 1) G = 1;
   if (G > 65535) G = 65535;
-  return launch_pdl(k_score_online<L>, dim3((unsigned)B, (unsigned)G), dim3(128), C::SMEM, st, 1,
+  return launch_pdl(k_score_online<L>, dim3((unsigned)B, (unsigned)G), dim3(kOnThreads), C::SMEM, st, 1,
                     (const bf16*)T, n_items, (const uint8_t*)image, ids, off, B, total,
                     (const bf16*)LP, (bf16*)O, status);
 }

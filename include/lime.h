@@ -120,6 +120,11 @@ int lime_build_qk_cache(const lime_dims* dims, const void* T, int64_t n_items,
  * lime_build_qk_cache.
  *   image  device, lime_qk_image_bytes(dims) bytes (2*d*H*l), 16-byte
  *          aligned; written by lime_fold_qk, read by the build.
+ *   tiles_per_cta  0: one persistent CTA per SM (fastest alone); k > 0:
+ *          CTAs of about k 128-item tiles each, so that a build issued on a
+ *          low-priority stream yields SMs to higher-priority work (every
+ *          kernel is launched with its stream's priority).  Negative:
+ *          LIME_ERR_ARG.
  * Other arguments, checks and errors as lime_build_qk_cache.  Supported:
  * the bf16 tensor-core shapes (lime_qk_image_bytes returns 0 otherwise and
  * both calls return LIME_ERR_SHAPE).  lime_fold_qk uses no workspace.      */
@@ -127,8 +132,8 @@ size_t lime_qk_image_bytes(const lime_dims* dims);
 int lime_fold_qk(const lime_dims* dims, const void* L, const void* Wq_c, const void* Wk_c,
                  void* image, cudaStream_t stream);
 int lime_build_qk_cache_folded(const lime_dims* dims, const void* T, int64_t n_items,
-                               const void* image, void* cache_out, void* workspace,
-                               size_t workspace_bytes, cudaStream_t stream);
+                               const void* image, void* cache_out, int32_t tiles_per_cta,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Uncached (online) candidate scoring: the same O_m as
  * lime_score_candidates, with the weights computed per candidate from the item

@@ -320,8 +320,8 @@ __global__ void __launch_bounds__(CacheCfg<HL, L, U8>::THREADS, 1)
 }
 
 template <int HL, int L, bool U8>
-int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, unsigned* status,
-                 cudaStream_t st) {
+int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, int tiles_per_cta,
+                 unsigned* status, cudaStream_t st) {
   using C = CacheCfg<HL, L, U8>;
   CUtensorMap tmT, tmC;
   if (!make_tmap_2d_bf16(&tmT, T, kD, (uint64_t)n, kD * 2, 64, kBM)) return LIME_ERR_CUDA;
@@ -334,7 +334,10 @@ int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, unsigne
                            C::SMEM) != cudaSuccess)
     return LIME_ERR_CUDA;
   const int n_tiles = (int)((n + kBM - 1) / kBM);
-  const int grid = n_tiles < num_sms() ? n_tiles : num_sms();
+  // persistent (one CTA per SM), or CTAs of about tiles_per_cta tiles each, so
+  // that the build can share the GPU with higher-priority work
+  int grid = n_tiles < num_sms() ? n_tiles : num_sms();
+  if (tiles_per_cta > 0) grid = (n_tiles + tiles_per_cta - 1) / tiles_per_cta;
   return launch_pdl(k_cache_tc<HL, L, U8>, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, tmT, tmC,
                     img, n_tiles, status);
 }
@@ -364,21 +367,21 @@ int launch_fold(const lime_dims& D, const void* L, const void* Wq, const void* W
 }
 
 int launch_build(const lime_dims& D, const void* T, int64_t n, const bf16* img, void* cache,
-                 bool u8, unsigned* status, cudaStream_t st) {
+                 bool u8, int tpc, unsigned* status, cudaStream_t st) {
   if (n == 0) return LIME_OK;
   switch (D.H * D.l * 1000 + D.l + (u8 ? 1000000 : 0)) {
-    case 64016: return launch_cache<64, 16, false>(T, n, img, cache, status, st);
-    case 64032: return launch_cache<64, 32, false>(T, n, img, cache, status, st);
-    case 128016: return launch_cache<128, 16, false>(T, n, img, cache, status, st);
-    case 128032: return launch_cache<128, 32, false>(T, n, img, cache, status, st);
-    case 128064: return launch_cache<128, 64, false>(T, n, img, cache, status, st);
-    case 256032: return launch_cache<256, 32, false>(T, n, img, cache, status, st);
-    case 256064: return launch_cache<256, 64, false>(T, n, img, cache, status, st);
-    case 1128016: return launch_cache<128, 16, true>(T, n, img, cache, status, st);
-    case 1128032: return launch_cache<128, 32, true>(T, n, img, cache, status, st);
-    case 1128064: return launch_cache<128, 64, true>(T, n, img, cache, status, st);
-    case 1256032: return launch_cache<256, 32, true>(T, n, img, cache, status, st);
-    case 1256064: return launch_cache<256, 64, true>(T, n, img, cache, status, st);
+    case 64016: return launch_cache<64, 16, false>(T, n, img, cache, tpc, status, st);
+    case 64032: return launch_cache<64, 32, false>(T, n, img, cache, tpc, status, st);
+    case 128016: return launch_cache<128, 16, false>(T, n, img, cache, tpc, status, st);
+    case 128032: return launch_cache<128, 32, false>(T, n, img, cache, tpc, status, st);
+    case 128064: return launch_cache<128, 64, false>(T, n, img, cache, tpc, status, st);
+    case 256032: return launch_cache<256, 32, false>(T, n, img, cache, tpc, status, st);
+    case 256064: return launch_cache<256, 64, false>(T, n, img, cache, tpc, status, st);
+    case 1128016: return launch_cache<128, 16, true>(T, n, img, cache, tpc, status, st);
+    case 1128032: return launch_cache<128, 32, true>(T, n, img, cache, tpc, status, st);
+    case 1128064: return launch_cache<128, 64, true>(T, n, img, cache, tpc, status, st);
+    case 1256032: return launch_cache<256, 32, true>(T, n, img, cache, tpc, status, st);
+    case 1256064: return launch_cache<256, 64, true>(T, n, img, cache, tpc, status, st);
     default: return LIME_ERR_SHAPE;
   }
 }
@@ -389,7 +392,7 @@ int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void
                         unsigned* status, cudaStream_t st) {
   bf16* img = reinterpret_cast<bf16*>(ws);
   int rc = launch_fold(D, L, Wq, Wk, img, st);
-  return rc ? rc : launch_build(D, T, n, img, cache, false, status, st);
+  return rc ? rc : launch_build(D, T, n, img, cache, false, 0, status, st);
 }
 
 int fast_build_qk_cache_u8(const lime_dims& D, const void* T, int64_t n, const void* L,
@@ -397,7 +400,7 @@ int fast_build_qk_cache_u8(const lime_dims& D, const void* T, int64_t n, const v
                            unsigned* status, cudaStream_t st) {
   bf16* img = reinterpret_cast<bf16*>(ws);
   int rc = launch_fold(D, L, Wq, Wk, img, st);
-  return rc ? rc : launch_build(D, T, n, img, cache, true, status, st);
+  return rc ? rc : launch_build(D, T, n, img, cache, true, 0, status, st);
 }
 
 int fast_fold_qk(const lime_dims& D, const void* L, const void* Wq, const void* Wk, void* image,
@@ -406,8 +409,9 @@ int fast_fold_qk(const lime_dims& D, const void* L, const void* Wq, const void* 
 }
 
 int fast_build_qk_cache_folded(const lime_dims& D, const void* T, int64_t n, const void* image,
-                               void* cache, unsigned* status, cudaStream_t st) {
-  return launch_build(D, T, n, reinterpret_cast<const bf16*>(image), cache, false, status, st);
+                               void* cache, int tiles_per_cta, unsigned* status, cudaStream_t st) {
+  return launch_build(D, T, n, reinterpret_cast<const bf16*>(image), cache, false, tiles_per_cta,
+                      status, st);
 }
 
 }  // namespace lime

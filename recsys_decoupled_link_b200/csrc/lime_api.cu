@@ -277,12 +277,12 @@ int lime_fold_qk(const lime_dims* dims, const void* L, const void* Wq_c, const v
 }
 
 int lime_build_qk_cache_folded(const lime_dims* dims, const void* T, int64_t n_items,
-                               const void* image, void* cache_out, void* workspace,
-                               size_t workspace_bytes, cudaStream_t stream) {
+                               const void* image, void* cache_out, int32_t tiles_per_cta,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if (!lime_qk_image_bytes(dims)) return LIME_ERR_SHAPE;
-  if (n_items < 0 || n_items > (int64_t)INT32_MAX + 1) return LIME_ERR_ARG;
+  if (n_items < 0 || n_items > (int64_t)INT32_MAX + 1 || tiles_per_cta < 0) return LIME_ERR_ARG;
   if (!image || (n_items > 0 && (!T || !cache_out))) return LIME_ERR_ARG;
   if (!aligned16(image) || (n_items > 0 && (!aligned16(T) || !aligned16(cache_out))))
     return LIME_ERR_ARG;
@@ -294,8 +294,8 @@ int lime_build_qk_cache_folded(const lime_dims* dims, const void* T, int64_t n_i
       overlap(workspace, workspace_bytes, image, lime_qk_image_bytes(dims)) ||
       overlap(workspace, workspace_bytes, cache_out, cache_sz))
     return LIME_ERR_ALIAS;
-  if ((rc = fast_build_qk_cache_folded(*dims, T, n_items, image, cache_out, status_of(workspace),
-                                       stream)))
+  if ((rc = fast_build_qk_cache_folded(*dims, T, n_items, image, cache_out, tiles_per_cta,
+                                       status_of(workspace), stream)))
     return rc;
   return launch_status("lime_build_qk_cache_folded");
 }

@@ -15,11 +15,19 @@ inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   unsigned n = 0;
   attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[n].val.programmaticStreamSerializationAllowed = 1;
   ++n;
+  // the stream's priority travels with the launch (and into a captured graph's
+  // kernel node), so a low-priority stream's CTAs yield SMs to a high one's
+  int prio = 0;
+  if (cudaStreamGetPriority(st, &prio) == cudaSuccess && prio != 0) {
+    attr[n].id = cudaLaunchAttributePriority;
+    attr[n].val.priority = prio;
+    ++n;
+  }
   if (cluster_y > 1) {
     attr[n].id = cudaLaunchAttributeClusterDimension;
     attr[n].val.clusterDim.x = 1;
@@ -47,7 +55,7 @@ int fast_build_qk_cache(const lime_dims& D, const void* T, int64_t n, const void
 int fast_fold_qk(const lime_dims& D, const void* L, const void* Wq, const void* Wk, void* image,
                  cudaStream_t st);
 int fast_build_qk_cache_folded(const lime_dims& D, const void* T, int64_t n, const void* image,
-                               void* cache, unsigned* status, cudaStream_t st);
+                               void* cache, int tiles_per_cta, unsigned* status, cudaStream_t st);
 
 // uncached (online) scoring from the item table and the folded G image
 bool fast_online_supported(const lime_dims& D);

@@ -69,7 +69,7 @@ def _load() -> ctypes.CDLL:
         "lime_score_candidates_u8": (I32, [D, I64, P, I64, P, P, I64, P, P, P, SZ, P]),
         "lime_qk_image_bytes": (SZ, [D]),
         "lime_fold_qk": (I32, [D, P, P, P, P, P]),
-        "lime_build_qk_cache_folded": (I32, [D, P, I64, P, P, P, SZ, P]),
+        "lime_build_qk_cache_folded": (I32, [D, P, I64, P, P, I32, P, SZ, P]),
         "lime_score_candidates_uncached": (I32, [D, I64, P, I64, P, P, P, I64, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
@@ -164,12 +164,14 @@ def lime_fold_qk(dims, L, Wq_c, Wk_c, image, stream=None):
         ctypes.byref(dims), _ptr(L), _ptr(Wq_c), _ptr(Wk_c), _ptr(image), _stream(stream)))
 
 
-def lime_build_qk_cache_folded(dims, T, image, cache_out, ws: Workspace, stream=None):
-    """Second stage of the QK cache: the catalogue pass over a folded image."""
+def lime_build_qk_cache_folded(dims, T, image, cache_out, ws: Workspace, stream=None,
+                               tiles_per_cta: int = 0):
+    """Second stage of the QK cache: the catalogue pass over a folded image
+    (tiles_per_cta > 0: short CTAs that yield SMs to higher-priority streams)."""
     n_items = 0 if T is None else T.shape[0]
     _check("lime_build_qk_cache_folded", _lib.lime_build_qk_cache_folded(
-        ctypes.byref(dims), _ptr(T), n_items, _ptr(image), _ptr(cache_out), ws.ptr, ws.nbytes,
-        _stream(stream)))
+        ctypes.byref(dims), _ptr(T), n_items, _ptr(image), _ptr(cache_out), int(tiles_per_cta),
+        ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def lime_score_candidates_uncached(dims, T, image, cand_ids, cand_offsets, total_cand, LP, O_out,

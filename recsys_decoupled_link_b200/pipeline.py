@@ -9,7 +9,10 @@ scoring.  All arithmetic happens inside liblime.
 Where the library offers the two-stage cache build, ``step`` runs its first
 stage (the folded per-head matrix, which depends only on the weights) on a
 side stream at the start of the step, so it overlaps the user side; the
-catalogue pass then waits for it on the main stream.
+catalogue pass then waits for it on the main stream.  (Running the whole
+catalogue pass beside the user side, in short CTAs on a low-priority stream,
+measured no faster: its CTAs need most of an SM's shared memory, so they
+cannot share SMs with the user-side kernels and only delay their launches.)
 """
 from __future__ import annotations
 

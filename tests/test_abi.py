@@ -125,15 +125,17 @@ def test_host_validation_of_two_stage_cache(lime):
                 None) == lime.LIME_ERR_SHAPE
     nws = lime.lime_workspace_bytes(dims, 0, 0)
     g = lime._lib.lime_build_qk_cache_folded
-    assert g(ctypes.byref(dims), 0x100000, 10, 0x200000, 0x200000 + 256, 0x1000000, nws,
+    assert g(ctypes.byref(dims), 0x100000, 10, 0x200000, 0x200000 + 256, 0, 0x1000000, nws,
              None) == lime.LIME_ERR_ALIAS                                     # cache over image
-    assert g(ctypes.byref(dims), 0x100000, 10, 0x1000000, 0x300000, 0x1000000, nws,
+    assert g(ctypes.byref(dims), 0x100000, 10, 0x1000000, 0x300000, 0, 0x1000000, nws,
              None) == lime.LIME_ERR_ALIAS                                     # image in ws
-    assert g(ctypes.byref(dims), 0x100000, 10, None, 0x300000, 0x1000000, nws,
+    assert g(ctypes.byref(dims), 0x100000, 10, None, 0x300000, 0, 0x1000000, nws,
              None) == lime.LIME_ERR_ARG
-    assert g(ctypes.byref(dims), 0x100000, -1, 0x200000, 0x300000, 0x1000000, nws,
+    assert g(ctypes.byref(dims), 0x100000, -1, 0x200000, 0x300000, 0, 0x1000000, nws,
              None) == lime.LIME_ERR_ARG
-    assert g(ctypes.byref(dims), 0x100000, 10, 0x200000, 0x300000, 0x1000000, 64,
+    assert g(ctypes.byref(dims), 0x100000, 10, 0x200000, 0x300000, -1, 0x1000000, nws,
+             None) == lime.LIME_ERR_ARG                                       # tiles_per_cta < 0
+    assert g(ctypes.byref(dims), 0x100000, 10, 0x200000, 0x300000, 0, 0x1000000, 64,
              None) == lime.LIME_ERR_ARG                                       # ws too small
 
 

@@ -426,6 +426,32 @@ def main():
     sc_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in sc_ev)], dist,
                            "cuda")[0] / args.steps
 
+    # phi = SiLU (pointwise attention weights): the same step, inputs and
+    # timing, with the SiLU variant of every attention
+    silu_ms = None
+    if w.dtype == "bf16" and not args.eager:
+        import dataclasses
+        ws_ = dataclasses.replace(w, phi="silu")
+        xs = dataclasses.replace(x, w=ws_, dims=lime.make_dims(w.d, w.H, w.l, w.f, w.c, w.dtype,
+                                                                "silu"))
+        bs = pipeline.alloc(xs)
+        gs = pipeline.step_graphs(xs, bs)[0]
+        for _ in range(3):
+            flush.zero_()
+            gs.replay()
+        sev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        for k in range(args.steps):
+            flush.zero_()
+            sev[k][0].record(stream)
+            gs.replay()
+            sev[k][1].record(stream)
+        torch.cuda.synchronize()
+        if lime.lime_get_status(bs.ws) != 0:
+            raise RuntimeError("device status flags set during the SiLU steps")
+        silu_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in sev)], dist,
+                                 "cuda")[0] / args.steps
+        del gs, bs, xs
+
     # Uncached (online) scoring at scale: the same IDs, with the weights computed
     # per candidate from the item table and the folded G image.
     on_ms = None
@@ -552,6 +578,11 @@ def main():
         }
         if lin is not None:
             phases["user_encode_linearity"] = lin
+        if silu_ms is not None:
+            phases["step_silu"] = {
+                "ms": silu_ms, "pairs_per_s": total_cand / (silu_ms * 1e-3),
+                "note": "the whole step with phi = SiLU (pointwise attention weights) in both "
+                        "XOR branches and the cache"}
         if on_ms is not None:
             on_bytes = sc_pairs * (4 * w.d + 4)   # item row in, score row out, ID
             on_gbs = on_bytes / (on_ms * 1e-3) / 1e9

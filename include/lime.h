@@ -46,6 +46,15 @@ extern "C" {
 
 typedef enum { LIME_F32 = 0, LIME_BF16 = 1 } lime_dtype;
 
+/* The attention weight function phi of both XOR branches and the candidate
+ * side (LIME note, 关键设计 1: "scaled Softmax or SiLU"; 损失函数 / 训练策略:
+ * softmax for single-layer models, SiLU in deep stacks).  LIME_PHI_SILU uses
+ * SiLU of each scaled score divided by the number of keys the query may attend
+ * to: l for a history query and for a candidate, N_u for a link query (the
+ * pages state no normaliser; this keeps an average's scale).  The int8 cache
+ * supports softmax only (SiLU weights can be negative).                     */
+typedef enum { LIME_PHI_SOFTMAX = 0, LIME_PHI_SILU = 1 } lime_phi;
+
 enum {
   LIME_OK = 0,
   LIME_ERR_ARG = -1,    /* null pointer, negative size, workspace too small  */
@@ -69,6 +78,7 @@ typedef struct {
   int32_t f;      /* GatedMLP hidden width                                   */
   int32_t c;      /* user context feature dim (0: no context MLP)            */
   int32_t dtype;  /* lime_dtype                                              */
+  int32_t phi;    /* lime_phi: the attention weight function (0 = softmax)   */
 } lime_dims;
 
 /* One LIME-XOR layer's parameters (device pointers, dims->dtype):

@@ -44,6 +44,13 @@ notes of the library):
      lookup + dequant") without stating the encoding.  Softmax weights lie in
      [0, 1], so the reading is unsigned 8-bit with the fixed scale 1/255:
      q = round(255 w), half to even, dequantised as q / 255.
+  R15 phi = SiLU (the variant the LIME note, 关键设计 1 and 损失函数 /
+     训练策略, names for deep stacks, with no normaliser stated): each weight
+     is SiLU of the same scaled score, divided by the number of keys the query
+     may attend to: ell for a history query and for a candidate, N_u for a link
+     query (a user with N_u = 0 gives the link branch a zero output, as in R8).
+     Division by the key count keeps the weights' scale that of an average, as
+     the softmax's are; the pages give no other normaliser.
 """
 from __future__ import annotations
 
@@ -72,6 +79,19 @@ def layer_norm(x: np.ndarray, gamma: np.ndarray, beta: np.ndarray,
 def silu(x: np.ndarray) -> np.ndarray:
     """SiLU(x) = x * sigmoid(x)."""
     return x / (1.0 + np.exp(-x))
+
+
+PHIS = ("softmax", "silu")
+
+
+def attention_weights(scores: np.ndarray, axis: int, phi: str) -> np.ndarray:
+    """phi over the keys of `axis` (readings R2, R15): the scaled softmax, or
+    SiLU of each score divided by the number of keys."""
+    if phi == "softmax":
+        return softmax(scores, axis=axis)
+    if phi == "silu":
+        return silu(scores) / scores.shape[axis]
+    raise ValueError(phi)
 
 
 def softmax(x: np.ndarray, axis: int = -1) -> np.ndarray:
@@ -105,7 +125,7 @@ def context_links_batch(L, ctx, Wc1, bc1, Wc2, bc2) -> np.ndarray:
 # ------------------------------------------------------ user side: XOR layer
 
 def xor_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, N: int,
-                  H: int) -> np.ndarray:
+                  H: int, phi: str = "softmax") -> np.ndarray:
     """Two-branch XOR attention over X = [E; L^C] for one user.
 
     LIME note, 关键设计 2 (XORA decomposition):
@@ -115,6 +135,7 @@ def xor_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, N: int,
     rows [0, N) are history, rows [N, N + l) are links.  Returns the per-row
     attention output [N + l, d] before the output projection.  With N = 0 the
     link rows have no key to attend to and get a zero output (reading R8).
+    phi: "softmax" (R2) or "silu" (R15).
     """
     n_rows, d = Q.shape
     dh = d // H
@@ -125,10 +146,10 @@ def xor_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, N: int,
     for h in range(H):
         c = slice(h * dh, (h + 1) * dh)
         # history -> link branch: MHA(E, L^C, L^C)
-        P_hist = softmax(s * (Q[:N, c] @ K[N:, c].T), axis=1)      # [N, l]
+        P_hist = attention_weights(s * (Q[:N, c] @ K[N:, c].T), 1, phi)   # [N, l]
         A[:N, c] = P_hist @ V[N:, c]
         # link -> history branch: MHA(L^C, E, E)
-        P_link = softmax(s * (Q[N:, c] @ K[:N, c].T), axis=1)      # [l, N]
+        P_link = attention_weights(s * (Q[N:, c] @ K[:N, c].T), 1, phi)   # [l, N]
         A[N:, c] = P_link @ V[:N, c]
     return A
 
@@ -144,7 +165,7 @@ def gated_mlp(x: np.ndarray, W1: np.ndarray, W3: np.ndarray,
 
 
 def xor_layer_user(E: np.ndarray, Z: np.ndarray, w: Dict[str, np.ndarray],
-                   H: int):
+                   H: int, phi: str = "softmax"):
     """One LIME-XOR layer for one user: (E [N, d], Z [l, d]) -> (E', Z').
 
     LIME note, 关键设计 2 (XOR mask, XORA decomposition, residual + GatedMLP)
@@ -160,13 +181,14 @@ def xor_layer_user(E: np.ndarray, Z: np.ndarray, w: Dict[str, np.ndarray],
     X = np.concatenate([E, Z], axis=0)
     Xh = layer_norm(X, w["g1"], w["b1"])
     Q, K, V = Xh @ w["Wq"], Xh @ w["Wk"], Xh @ w["Wv"]
-    Y = X + xor_attention(Q, K, V, N, H) @ w["Wo"]
+    Y = X + xor_attention(Q, K, V, N, H, phi) @ w["Wo"]
     Xp = Y + gated_mlp(layer_norm(Y, w["g2"], w["b2"]), w["W1"], w["W3"], w["W2"])
     return Xp[:N], Xp[N:]
 
 
 def xor_layer(E: np.ndarray, hist_offsets: Sequence[int], Z: np.ndarray,
-              w: Dict[str, np.ndarray], H: int, users: Optional[Sequence[int]] = None):
+              w: Dict[str, np.ndarray], H: int, users: Optional[Sequence[int]] = None,
+              phi: str = "softmax"):
     """xor_layer_user over a packed batch.
 
     E [sum N, d] packed by hist_offsets [B + 1]; Z [B, l, d].
@@ -179,12 +201,12 @@ def xor_layer(E: np.ndarray, hist_offsets: Sequence[int], Z: np.ndarray,
     Zp = np.full_like(Z, np.nan)
     for u in users:
         a, b = int(hist_offsets[u]), int(hist_offsets[u + 1])
-        Ep[a:b], Zp[u] = xor_layer_user(E[a:b], Z[u], w, H)
+        Ep[a:b], Zp[u] = xor_layer_user(E[a:b], Z[u], w, H, phi)
     return Ep, Zp
 
 
 def user_encode(E, hist_offsets, Z0, layers: List[Dict[str, np.ndarray]], H,
-                users=None):
+                users=None, phi: str = "softmax"):
     """Stack of LIME-XOR layers; returns (E after the last layer, L^P).
 
     LIME note, 整体框架 / 一个完整示例 step 2: the context links pass through
@@ -193,15 +215,15 @@ def user_encode(E, hist_offsets, Z0, layers: List[Dict[str, np.ndarray]], H,
     """
     Ecur, Zcur = E, Z0
     for w in layers:
-        Ecur, Zcur = xor_layer(Ecur, hist_offsets, Zcur, w, H, users)
+        Ecur, Zcur = xor_layer(Ecur, hist_offsets, Zcur, w, H, users, phi)
     return Ecur, Zcur
 
 
 # ------------------------------------------------------------ candidate side
 
 def qk_cache(T: np.ndarray, L: np.ndarray, Wq_c: np.ndarray, Wk_c: np.ndarray,
-             H: int) -> np.ndarray:
-    """QK cache phi(T L^T): [n_items, H, l] (readings R2, R3, R7).
+             H: int, phi: str = "softmax") -> np.ndarray:
+    """QK cache phi(T L^T): [n_items, H, l] (readings R2, R3, R7, R15).
 
     LIME note, 关键设计 1: the candidate-side attention weights depend only on
     the item embedding and the global links, so they are computed offline for
@@ -216,7 +238,7 @@ def qk_cache(T: np.ndarray, L: np.ndarray, Wq_c: np.ndarray, Wk_c: np.ndarray,
     out = np.empty((n, H, L.shape[0]))
     for h in range(H):
         c = slice(h * dh, (h + 1) * dh)
-        out[:, h, :] = softmax(s * (Qc[:, c] @ Kc[:, c].T), axis=1)
+        out[:, h, :] = attention_weights(s * (Qc[:, c] @ Kc[:, c].T), 1, phi)
     return out
 
 
@@ -277,7 +299,7 @@ def score_candidates_u8(q: np.ndarray, cand_ids: np.ndarray,
 
 def candidate_attention_uncached(T_rows: np.ndarray, L: np.ndarray,
                                  Wq_c: np.ndarray, Wk_c: np.ndarray,
-                                 LP_u: np.ndarray, H: int) -> np.ndarray:
+                                 LP_u: np.ndarray, H: int, phi: str = "softmax") -> np.ndarray:
     """MHA(T, L, L^P) computed directly, without a cache.
 
     LIME note, 关键设计 1: O = MHA(T, L, L^P; J) with an all-ones mask J, query
@@ -292,5 +314,5 @@ def candidate_attention_uncached(T_rows: np.ndarray, L: np.ndarray,
     O = np.empty((T_rows.shape[0], d))
     for h in range(H):
         c = slice(h * dh, (h + 1) * dh)
-        O[:, c] = softmax(s * (Q[:, c] @ K[:, c].T), axis=1) @ LP_u[:, c]
+        O[:, c] = attention_weights(s * (Q[:, c] @ K[:, c].T), 1, phi) @ LP_u[:, c]
     return O

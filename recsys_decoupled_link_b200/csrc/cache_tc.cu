@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(128) k_fold_g_img(const bf16* __restrict__ L,
 template <int HL, int L, bool U8>
 __global__ void __launch_bounds__(CacheCfg<HL, L, U8>::THREADS, 1)
     k_cache_tc(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmC,
-               const bf16* __restrict__ gimg, int n_tiles, unsigned* status) {
+               const bf16* __restrict__ gimg, int n_tiles, int phi, unsigned* status) {
   using C = CacheCfg<HL, L, U8>;
   constexpr int H = HL / L;
   constexpr uint32_t IDESC = idesc_bf16(kBM, HL);
@@ -241,16 +241,24 @@ __global__ void __launch_bounds__(CacheCfg<HL, L, U8>::THREADS, 1)
         for (int q = 0; q < L / 16; ++q)
           tmem_ld16(tmem + lane_base + acc * HL + h * L + q * 16, z + q * 16);
         tmem_ld_wait();
-        float m = z[0];
+        float inv;
+        if (!U8 && phi == LIME_PHI_SILU) {
+          // SiLU of each score over the l links (the int8 cache is softmax only)
 #pragma unroll
-        for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
-        float ssum = 0.f;
+          for (int k = 0; k < L; ++k) z[k] = __fdividef(z[k], 1.0f + __expf(-z[k]));
+          inv = 1.0f / L;
+        } else {
+          float m = z[0];
 #pragma unroll
-        for (int k = 0; k < L; ++k) {
-          z[k] = __expf(z[k] - m);
-          ssum += z[k];
+          for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
+          float ssum = 0.f;
+#pragma unroll
+          for (int k = 0; k < L; ++k) {
+            z[k] = __expf(z[k] - m);
+            ssum += z[k];
+          }
+          inv = 1.0f / ssum;
         }
-        const float inv = 1.0f / ssum;
         if constexpr (U8) {
           // bytes q = round(255 w), ties to even; 16 per 16-byte chunk of the
           // row's 128-byte swizzled block
@@ -321,7 +329,7 @@ __global__ void __launch_bounds__(CacheCfg<HL, L, U8>::THREADS, 1)
 
 template <int HL, int L, bool U8>
 int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, int tiles_per_cta,
-                 unsigned* status, cudaStream_t st) {
+                 int phi, unsigned* status, cudaStream_t st) {
   using C = CacheCfg<HL, L, U8>;
   CUtensorMap tmT, tmC;
   if (!make_tmap_2d_bf16(&tmT, T, kD, (uint64_t)n, kD * 2, 64, kBM)) return LIME_ERR_CUDA;
@@ -339,7 +347,7 @@ int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, int til
   int grid = n_tiles < num_sms() ? n_tiles : num_sms();
   if (tiles_per_cta > 0) grid = (n_tiles + tiles_per_cta - 1) / tiles_per_cta;
   return launch_pdl(k_cache_tc<HL, L, U8>, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, tmT, tmC,
-                    img, n_tiles, status);
+                    img, n_tiles, phi, status);
 }
 
 }  // namespace
@@ -370,18 +378,18 @@ int launch_build(const lime_dims& D, const void* T, int64_t n, const bf16* img, 
                  bool u8, int tpc, unsigned* status, cudaStream_t st) {
   if (n == 0) return LIME_OK;
   switch (D.H * D.l * 1000 + D.l + (u8 ? 1000000 : 0)) {
-    case 64016: return launch_cache<64, 16, false>(T, n, img, cache, tpc, status, st);
-    case 64032: return launch_cache<64, 32, false>(T, n, img, cache, tpc, status, st);
-    case 128016: return launch_cache<128, 16, false>(T, n, img, cache, tpc, status, st);
-    case 128032: return launch_cache<128, 32, false>(T, n, img, cache, tpc, status, st);
-    case 128064: return launch_cache<128, 64, false>(T, n, img, cache, tpc, status, st);
-    case 256032: return launch_cache<256, 32, false>(T, n, img, cache, tpc, status, st);
-    case 256064: return launch_cache<256, 64, false>(T, n, img, cache, tpc, status, st);
-    case 1128016: return launch_cache<128, 16, true>(T, n, img, cache, tpc, status, st);
-    case 1128032: return launch_cache<128, 32, true>(T, n, img, cache, tpc, status, st);
-    case 1128064: return launch_cache<128, 64, true>(T, n, img, cache, tpc, status, st);
-    case 1256032: return launch_cache<256, 32, true>(T, n, img, cache, tpc, status, st);
-    case 1256064: return launch_cache<256, 64, true>(T, n, img, cache, tpc, status, st);
+    case 64016: return launch_cache<64, 16, false>(T, n, img, cache, tpc, D.phi, status, st);
+    case 64032: return launch_cache<64, 32, false>(T, n, img, cache, tpc, D.phi, status, st);
+    case 128016: return launch_cache<128, 16, false>(T, n, img, cache, tpc, D.phi, status, st);
+    case 128032: return launch_cache<128, 32, false>(T, n, img, cache, tpc, D.phi, status, st);
+    case 128064: return launch_cache<128, 64, false>(T, n, img, cache, tpc, D.phi, status, st);
+    case 256032: return launch_cache<256, 32, false>(T, n, img, cache, tpc, D.phi, status, st);
+    case 256064: return launch_cache<256, 64, false>(T, n, img, cache, tpc, D.phi, status, st);
+    case 1128016: return launch_cache<128, 16, true>(T, n, img, cache, tpc, D.phi, status, st);
+    case 1128032: return launch_cache<128, 32, true>(T, n, img, cache, tpc, D.phi, status, st);
+    case 1128064: return launch_cache<128, 64, true>(T, n, img, cache, tpc, D.phi, status, st);
+    case 1256032: return launch_cache<256, 32, true>(T, n, img, cache, tpc, D.phi, status, st);
+    case 1256064: return launch_cache<256, 64, true>(T, n, img, cache, tpc, D.phi, status, st);
     default: return LIME_ERR_SHAPE;
   }
 }

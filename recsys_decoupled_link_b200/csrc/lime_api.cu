@@ -22,6 +22,7 @@ constexpr size_t kStatusBytes = 256;  // status word + padding at the workspace 
 bool dims_ok(const lime_dims* D) {
   if (!D) return false;
   if (D->dtype != LIME_F32 && D->dtype != LIME_BF16) return false;
+  if (D->phi != LIME_PHI_SOFTMAX && D->phi != LIME_PHI_SILU) return false;
   return true;
 }
 
@@ -305,7 +306,7 @@ int lime_build_qk_cache_u8(const lime_dims* dims, const void* T, int64_t n_items
                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
-  if (!fast_cache_u8_supported(*dims)) return LIME_ERR_SHAPE;
+  if (!fast_cache_u8_supported(*dims) || dims->phi != LIME_PHI_SOFTMAX) return LIME_ERR_SHAPE;
   if (n_items < 0 || n_items > (int64_t)INT32_MAX + 1) return LIME_ERR_ARG;
   if (!L || !Wq_c || !Wk_c || (n_items > 0 && (!T || !cache_out))) return LIME_ERR_ARG;
   if ((n_items > 0 && (!aligned16(T) || !aligned16(cache_out))) || !aligned16(L) ||

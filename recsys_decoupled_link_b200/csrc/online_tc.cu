@@ -51,7 +51,7 @@ template <int L>
 __global__ void __launch_bounds__(kOnThreads, 1)
     k_score_online(const bf16* __restrict__ T, int64_t n_items, const uint8_t* __restrict__ gimg,
                    const int32_t* __restrict__ ids, const int64_t* __restrict__ off, int64_t B,
-                   int64_t total, const bf16* __restrict__ LP, bf16* __restrict__ O,
+                   int64_t total, const bf16* __restrict__ LP, bf16* __restrict__ O, int phi,
                    unsigned* status) {
   using C = OnlineCfg<L>;
   constexpr int HL = C::HL;
@@ -178,15 +178,20 @@ __global__ void __launch_bounds__(kOnThreads, 1)
 #pragma unroll
         for (int q = 0; q < L / 16; ++q) tmem_ld16(ta + h * L + q * 16, z + q * 16);
         tmem_ld_wait();
-        float m = z[0];
+        if (phi == LIME_PHI_SILU) {
 #pragma unroll
-        for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
-        float s = 0.f;
+          for (int k = 0; k < L; ++k) z[k] = __fdividef(z[k], 1.0f + __expf(-z[k])) * (1.0f / L);
+        } else {
+          float m = z[0];
 #pragma unroll
-        for (int k = 0; k < L; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
-        const float inv = 1.0f / s;
+          for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
+          float s = 0.f;
 #pragma unroll
-        for (int k = 0; k < L; ++k) z[k] *= inv;
+          for (int k = 0; k < L; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
+          const float inv = 1.0f / s;
+#pragma unroll
+          for (int k = 0; k < L; ++k) z[k] *= inv;
+        }
 #pragma unroll
         for (int q = 0; q < L / 8; ++q) sw_st16(sA, kBlk, i, h * L + q * 8, pack8(z + q * 8));
       }
@@ -241,8 +246,8 @@ __global__ void __launch_bounds__(kOnThreads, 1)
 
 template <int L>
 int launch_online(int64_t B, const void* T, int64_t n_items, const void* image, const int32_t* ids,
-                  const int64_t* off, int64_t total, const void* LP, void* O, unsigned* status,
-                  cudaStream_t st) {
+                  const int64_t* off, int64_t total, const void* LP, void* O, int phi,
+                  unsigned* status, cudaStream_t st) {
   using C = OnlineCfg<L>;
   if (cudaFuncSetAttribute(k_score_online<L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::SMEM) != cudaSuccess)
@@ -256,7 +261,7 @@ int launch_online(int64_t B, const void* T, int64_t n_items, const void* image, 
   if (G > 65535) G = 65535;
   return launch_pdl(k_score_online<L>, dim3((unsigned)B, (unsigned)G), dim3(kOnThreads), C::SMEM, st, 1,
                     (const bf16*)T, n_items, (const uint8_t*)image, ids, off, B, total,
-                    (const bf16*)LP, (bf16*)O, status);
+                    (const bf16*)LP, (bf16*)O, phi, status);
 }
 
 }  // namespace
@@ -269,8 +274,8 @@ int fast_score_online(const lime_dims& D, int64_t B, const void* T, int64_t n_it
                       const void* image, const int32_t* ids, const int64_t* off, int64_t total,
                       const void* LP, void* O, unsigned* status, cudaStream_t st) {
   if (D.l == 16)
-    return launch_online<16>(B, T, n_items, image, ids, off, total, LP, O, status, st);
-  return launch_online<32>(B, T, n_items, image, ids, off, total, LP, O, status, st);
+    return launch_online<16>(B, T, n_items, image, ids, off, total, LP, O, D.phi, status, st);
+  return launch_online<32>(B, T, n_items, image, ids, off, total, LP, O, D.phi, status, st);
 }
 
 }  // namespace lime

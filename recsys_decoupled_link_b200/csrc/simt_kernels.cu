@@ -208,7 +208,7 @@ __global__ void k_unpack_rows(const float* __restrict__ X, int64_t nh, int64_t n
 __global__ void k_attn_hist(const float* __restrict__ Q, const float* __restrict__ K,
                             const float* __restrict__ V, const int64_t* __restrict__ off,
                             int64_t B, int64_t nh, int d, int H, int l, float scale,
-                            float* __restrict__ A) {
+                            int phi, float* __restrict__ A) {
   extern __shared__ float sp[];  // [warps][l]
   int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int64_t task = blockIdx.x * (int64_t)(blockDim.x >> 5) + warp;
@@ -230,8 +230,14 @@ __global__ void k_attn_hist(const float* __restrict__ Q, const float* __restrict
   }
   mx = warp_max(mx);
   float sum = 0.f;
-  for (int k = lane; k < l; k += 32) { float e = expf(p[k] - mx); p[k] = e; sum += e; }
-  sum = warp_sum(sum);
+  if (phi == LIME_PHI_SILU) {
+    // SiLU of each score over the l keys
+    for (int k = lane; k < l; k += 32) p[k] = p[k] / (1.0f + expf(-p[k]));
+    sum = (float)l;
+  } else {
+    for (int k = lane; k < l; k += 32) { float e = expf(p[k] - mx); p[k] = e; sum += e; }
+    sum = warp_sum(sum);
+  }
   __syncwarp();
   for (int c = lane; c < dh; c += 32) {
     float acc = 0.f;
@@ -243,12 +249,14 @@ __global__ void k_attn_hist(const float* __restrict__ Q, const float* __restrict
 // Link branch, MHA(L^C, E, E): link k of user u attends to the user's history
 // rows, per head.  One warp per (user, head, link); each lane keeps an online
 // softmax over a strided subset of the history, merged through shared memory.
-// A user with no history gets a zero output.
+// A user with no history gets a zero output.  With phi = SiLU a lane keeps the
+// SiLU-weighted sum and its key count (max 0), and the same merge divides the
+// total by N_u.
 template <int DH>
 __global__ void k_attn_link(const float* __restrict__ Q, const float* __restrict__ K,
                             const float* __restrict__ V, const int64_t* __restrict__ off,
                             int64_t B, int64_t nh, int d, int H, int l, float scale,
-                            float* __restrict__ A, unsigned* status) {
+                            int phi, float* __restrict__ A, unsigned* status) {
   __shared__ float sm_m[4][32], sm_s[4][32];
   __shared__ float sm_acc[4][32][DH + 1];
   int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -262,7 +270,8 @@ __global__ void k_attn_link(const float* __restrict__ Q, const float* __restrict
     k = task % l;
   }
   float q[DH], acc[DH];
-  float m = -INFINITY, s = 0.f;
+  const bool silu = phi == LIME_PHI_SILU;
+  float m = silu ? 0.f : -INFINITY, s = 0.f;
 #pragma unroll
   for (int c = 0; c < DH; ++c) acc[c] = 0.f;
   int64_t a = 0, b = 0;
@@ -277,9 +286,16 @@ __global__ void k_attn_link(const float* __restrict__ Q, const float* __restrict
 #pragma unroll
       for (int c = 0; c < DH; ++c) sc += q[c] * kp[c];
       sc *= scale;
+      const float* vp = V + j * d + h * DH;
+      if (silu) {
+        const float e = sc / (1.0f + expf(-sc));
+        s += 1.0f;
+#pragma unroll
+        for (int c = 0; c < DH; ++c) acc[c] += e * vp[c];
+        continue;
+      }
       float mn = fmaxf(m, sc);
       float corr = expf(m - mn), e = expf(sc - mn);
-      const float* vp = V + j * d + h * DH;
       s = s * corr + e;
 #pragma unroll
       for (int c = 0; c < DH; ++c) acc[c] = acc[c] * corr + e * vp[c];
@@ -333,11 +349,11 @@ __global__ void k_fold_g(const T* __restrict__ Wq, const float* __restrict__ Kc,
   }
 }
 
-// cache[m, h, :] = softmax_k(T_m · Gfold[:, h*l + k]).  One block of H*l
-// threads (rounded up to a warp multiple) per group of 8 items.
+// cache[m, h, :] = phi_k(T_m · Gfold[:, h*l + k]) (softmax, or SiLU / l).
+// One block of H*l threads (rounded up to a warp multiple) per group of 8 items.
 template <class T>
 __global__ void k_cache_simt(const T* __restrict__ Tm, int64_t n_items, int d, int H, int l,
-                             const float* __restrict__ G, T* __restrict__ cache) {
+                             const float* __restrict__ G, int phi, T* __restrict__ cache) {
   extern __shared__ float sm[];
   float* trow = sm;             // [8][d]
   float* logit = sm + 8 * d;    // [8][H*l]
@@ -367,6 +383,11 @@ __global__ void k_cache_simt(const T* __restrict__ Tm, int64_t n_items, int d, i
     int64_t m = m0 + t;
     if (m >= n_items) continue;
     float* z = logit + t * HL + h * l;
+    if (phi == LIME_PHI_SILU) {
+      for (int k = 0; k < l; ++k)
+        cache[(m * H + h) * l + k] = from_f<T>(z[k] / (1.0f + expf(-z[k])) / (float)l);
+      continue;
+    }
     float mx = -INFINITY;
     for (int k = 0; k < l; ++k) mx = fmaxf(mx, z[k]);
     float s = 0.f;
@@ -477,18 +498,18 @@ void simt_xor_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t n
   if (nh > 0) {
     int64_t tasks = nh * H;
     k_attn_hist<<<(unsigned)((tasks + 7) / 8), 256, 8 * l * sizeof(float), st>>>(
-        Q, K, V, off, B, nh, d, H, l, scale, A);
+        Q, K, V, off, B, nh, d, H, l, scale, D.phi, A);
     note_launches(1);
   }
   {
     int64_t tasks = B * H * l;
     unsigned grid = (unsigned)((tasks + 3) / 4);
     if (dh == 16)
-      k_attn_link<16><<<grid, 128, 0, st>>>(Q, K, V, off, B, nh, d, H, l, scale, A, status);
+      k_attn_link<16><<<grid, 128, 0, st>>>(Q, K, V, off, B, nh, d, H, l, scale, D.phi, A, status);
     else if (dh == 32)
-      k_attn_link<32><<<grid, 128, 0, st>>>(Q, K, V, off, B, nh, d, H, l, scale, A, status);
+      k_attn_link<32><<<grid, 128, 0, st>>>(Q, K, V, off, B, nh, d, H, l, scale, D.phi, A, status);
     else
-      k_attn_link<64><<<grid, 128, 0, st>>>(Q, K, V, off, B, nh, d, H, l, scale, A, status);
+      k_attn_link<64><<<grid, 128, 0, st>>>(Q, K, V, off, B, nh, d, H, l, scale, D.phi, A, status);
     note_launches(1);
   }
   gemm(A, d, w.Wo, bf, d, d, R, X, Y, st);          // Y = X + A Wo
@@ -525,7 +546,7 @@ void simt_build_qk_cache(const lime_dims& D, const void* Tm, int64_t n, const vo
   if (threads > 1024) threads = 1024;
   size_t smem = (size_t)8 * (d + HL) * sizeof(float);
   k_cache_simt<T><<<(unsigned)((n + 7) / 8), threads, smem, st>>>((const T*)Tm, n, d, H, l, G,
-                                                                 (T*)cache);
+                                                                 D.phi, (T*)cache);
   note_launches(1);
 }
 

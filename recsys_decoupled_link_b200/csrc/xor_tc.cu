@@ -67,11 +67,13 @@ struct LayerWs {
 __host__ __device__ constexpr size_t up1k(size_t x) { return (x + 1023) & ~(size_t)1023; }
 
 // per-user folded images: G'^T, Q'g, VO ([128 x 128] bf16 each), then the
-// fp32 vectors cQ, dQ, cG, dG ([128] each)
+// fp32 vectors cQ, dQ, cG, dG ([128] each); with phi = SiLU also the low half
+// of G' (G' = hi + lo)
 constexpr uint32_t kUimgVec = 6 * kBlk;
 constexpr uint32_t kUimgBytes = 6 * kBlk + 4 * 128 * 4;
+constexpr uint32_t kUimgGlo = kUimgBytes;
 
-LayerWs layer_ws(int l, int64_t B, int64_t nh) {
+LayerWs layer_ws(int l, int64_t B, int64_t nh, bool silu) {
   LayerWs w;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t r = o; o = up1k(o + bytes); return r; };
@@ -87,7 +89,7 @@ LayerWs layer_ws(int l, int64_t B, int64_t nh) {
   w.tiles = take((size_t)w.max_tiles * 16);
   w.tile_start = take((size_t)(B + 1) * 4);
   w.yd = take((size_t)nh * kD * 2);   // attention delta (fp16)
-  w.uimg_bytes = kUimgBytes;
+  w.uimg_bytes = kUimgBytes + (silu ? 2 * kBlk : 0);
   w.uimg = take((size_t)B * w.uimg_bytes);
   w.part = take((size_t)w.max_tiles * kH * l * kRec * 4);
   w.total = o;
@@ -412,7 +414,7 @@ template <int L>
 __global__ void __launch_bounds__(512, 1)
     k_link_proj(const bf16* __restrict__ Z, int64_t nrows, const bf16* __restrict__ g1,
                 const bf16* __restrict__ b1, uint8_t* __restrict__ ws, LayerWs Lw, float scale,
-                unsigned* status) {
+                bool silu, unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
   uint8_t* sAh = sm;
@@ -512,13 +514,16 @@ __global__ void __launch_bounds__(512, 1)
   const int64_t left = nrows / L - u0;
   const int n_users = left < UP ? (int)left : UP;
   const float* gb = red + 1024;   // g1, b1 as fp32
+  // phi = SiLU: G' is stored as hi + lo (two buffers per head): SiLU weights are
+  // signed, so the history scores' operand rounding is not averaged away
+  const bool split = which == 1 && silu;
   for (int i = 0; i < hpc; ++i) {
     const int h = h0 + i;
     float v[32];
     tmem_ld16(ta + i * 128 + c0, v);
     tmem_ld16(ta + i * 128 + c0 + 16, v + 16);
     tmem_ld_wait();
-    uint8_t* buf = sm + i * 2 * kBlk;
+    uint8_t* buf = sm + (split ? 2 * i : i) * 2 * kBlk;
     if (which == 2) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) sw_st16(buf, kBlk, r, c0 + q * 8, pack8(v + q * 8));
@@ -527,11 +532,16 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         ds = fmaf(v[j], gb[kD + c0 + j], ds);
-        v[j] = __bfloat162float(__float2bfloat16_rn(v[j] * gb[c0 + j]));
+        v[j] *= gb[c0 + j];
+        if (!split) v[j] = __bfloat162float(__float2bfloat16_rn(v[j]));
         cs += v[j];
       }
+      if (split)
+        split_part_st(buf, buf + 2 * kBlk, r, c0, v);
+      else {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(buf, kBlk, r, c0 + q * 8, pack8(v + q * 8));
+        for (int q = 0; q < 4; ++q) sw_st16(buf, kBlk, r, c0 + q * 8, pack8(v + q * 8));
+      }
       red[part * 128 + r] = cs;
       red[512 + part * 128 + r] = ds;
       __syncthreads();
@@ -549,10 +559,11 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   if (threadIdx.x == 0) {
     const uint32_t img_off = which == 0 ? 2 * kBlk : which == 1 ? 0 : 4 * kBlk;
-    for (int i = 0; i < hpc; ++i) {
-      const int h = h0 + i;
+    for (int i = 0; i < hpc * (split ? 2 : 1); ++i) {
+      const int h = h0 + (split ? i >> 1 : i);
+      const uint32_t off = split && (i & 1) ? kUimgGlo : img_off;
       for (int j = 0; j < n_users; ++j) {
-        uint8_t* dst = ws + Lw.uimg + (size_t)(u0 + j) * Lw.uimg_bytes + img_off + h * L * 128;
+        uint8_t* dst = ws + Lw.uimg + (size_t)(u0 + j) * Lw.uimg_bytes + off + h * L * 128;
         const uint8_t* src = sm + i * 2 * kBlk + j * L * 128;
         bulk_store(dst, src, L * 128);
         bulk_store(dst + kBlk, src + kBlk, L * 128);
@@ -576,7 +587,8 @@ __global__ void __launch_bounds__(512, 1)
 //            they start as soon as it lands, while the epilogue finishes the
 //            previous tile.
 //   stats    mu, rstd per row (reduced over the four column parts)
-//   softmax  P2 = exp(z - max), z = rstd (S'^T - mu cQ) + dQ per token column,
+//   softmax  (phi = SiLU: pointwise SiLU weights, see the lime_phi notes)
+//            P2 = exp(z - max), z = rstd (S'^T - mu cQ) + dQ per token column,
 //            over the tile's valid rows (part = a quarter of the tokens; the
 //            lane's max and sum reduced over the parts); V_E = rstd (. - mu
 //            cv) + dv as bf16 over the G' image; P = softmax of each head's L
@@ -604,12 +616,13 @@ __global__ void __launch_bounds__(512, 1)
 constexpr int kXaEpi = 512;
 constexpr int kXaThreads = kXaEpi + 32;
 constexpr uint32_t kXaSmem = 1024 + 12 * kBlk + 1024 /* mu, rstd */ + 4096 /* red */ +
-                             1024 /* cv, dv */ + 2 * 2048 /* vec x2 */ + 128 /* 14 barriers */;
+                             1024 /* cv, dv */ + 2 * 2048 /* vec x2 */ +
+                             kBlk /* one block of G'lo (phi = SiLU) */ + 256 /* barriers */;
 
 template <int L, bool HIST>
 __global__ void __launch_bounds__(kXaThreads, 1)
     k_hist_xattn(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
-                 uint8_t* __restrict__ ws, LayerWs Lw, unsigned* status) {
+                 uint8_t* __restrict__ ws, LayerWs Lw, int phi, unsigned* status) {
   constexpr int HL = kH * L;
   constexpr uint32_t kSlot = 2 * kBlk;
   extern __shared__ uint8_t smem_raw[];
@@ -623,11 +636,12 @@ __global__ void __launch_bounds__(kXaThreads, 1)
   float* red = smu + 256;                                   // [1024]
   float* cvd = red + 1024;                                  // cv [128], dv [128]
   float* vecs = cvd + 256;                                  // 2 x (cQ, dQ, cG, dG)
+  uint8_t* sGl = reinterpret_cast<uint8_t*>(vecs + 1024);   // a 64-column block of G'lo
   Cta c;
   // bar: 0 weights, 1 S' done, 2 E tile, 3 G', 4 Q'g + vec, 6 VO, 7 V_E done,
   //      8 S done, 9 P2 V_E done, 10 Yd done, 11 TMEM read out, 12 P2 and V_E
-  //      written, 13 P written
-  cta_setup(reinterpret_cast<uint8_t*>(vecs + 1024), 14, c);
+  //      written, 13 P written, 14 G'lo block landed, 15 its product done
+  cta_setup(sGl + kBlk, 16, c);
   uint64_t* bar = c.bar;
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
@@ -686,6 +700,20 @@ __global__ void __launch_bounds__(kXaThreads, 1)
           mbar_wait(&bar[3], ph, status, c.abort_flag);
           tc_fence_after();
           mma_tile(c.tmem, smem_u32(sA), kBlk, smem_u32(sG), kBlk, HL, 128, false);
+          if (phi == LIME_PHI_SILU) {
+            // + E G'lo, one 64-column block at a time through sGl
+            for (int j = 0; j < 2; ++j) {
+              const uint32_t pj = (uint32_t)(2 * it + j) & 1u;
+              if (j > 0) mbar_wait(&bar[15], pj ^ 1u, status, c.abort_flag);
+              mbar_arrive_expect_tx(&bar[14], kBlk);
+              bulk_load(sGl, uimg(u) + kUimgGlo + j * kBlk, kBlk, &bar[14]);
+              mbar_wait(&bar[14], pj, status, c.abort_flag);
+              tc_fence_after();
+              mma_tile(c.tmem, smem_u32(sA + j * kBlk), kBlk, smem_u32(sGl), kBlk, HL, 64, true);
+              mma_commit(&bar[15]);
+            }
+            mbar_wait(&bar[15], 1u, status, c.abort_flag);   // the block's buffer is free
+          }
           mma_commit(&bar[8]);
         }
         // the link scores have read Q'g
@@ -787,21 +815,32 @@ __global__ void __launch_bounds__(kXaThreads, 1)
             m = fmaxf(m, z[j]);
           }
         }
-        red[part * 128 + row] = m;
-        // B held the previous tile's Yd staging: its store must have read it
-        if (HIST && it > 0 && threadIdx.x == 0) bulk_wait_read<0>();
-        named_bar_sync(1, kXaEpi);
-        m = fmaxf(fmaxf(red[row], red[128 + row]), fmaxf(red[256 + row], red[384 + row]));
-        float s = 0.f;
+        if (phi == LIME_PHI_SILU) {
+          // pointwise weights: SiLU of each valid score; the record's (max,
+          // sum) = (0, valid tokens) makes the merge's total divide by N_u
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          z[j] = c0 + j < nv && link ? __expf(z[j] - m) : 0.f;
-          s += z[j];
+          for (int j = 0; j < 32; ++j) z[j] = c0 + j < nv && link ? silu_fast(z[j]) : 0.f;
+          if (HIST && it > 0 && threadIdx.x == 0) bulk_wait_read<0>();
+          named_bar_sync(1, kXaEpi);
+          lm = 0.f;
+          ls = (float)nv;
+        } else {
+          red[part * 128 + row] = m;
+          // B held the previous tile's Yd staging: its store must have read it
+          if (HIST && it > 0 && threadIdx.x == 0) bulk_wait_read<0>();
+          named_bar_sync(1, kXaEpi);
+          m = fmaxf(fmaxf(red[row], red[128 + row]), fmaxf(red[256 + row], red[384 + row]));
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            z[j] = c0 + j < nv && link ? __expf(z[j] - m) : 0.f;
+            s += z[j];
+          }
+          red[512 + part * 128 + row] = s;
+          named_bar_sync(1, kXaEpi);
+          lm = m;
+          ls = red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row];
         }
-        red[512 + part * 128 + row] = s;
-        named_bar_sync(1, kXaEpi);
-        lm = m;
-        ls = red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row];
 #pragma unroll
         for (int q = 0; q < 4; ++q) sw_st16(sB, kBlk, row, c0 + q * 8, pack8(z + q * 8));
       }
@@ -833,15 +872,20 @@ __global__ void __launch_bounds__(kXaThreads, 1)
 #pragma unroll
         for (int k = 0; k < L; ++k)
           z[k] = fmaf(rs_r, fmaf(-mu_r, vec[256 + h * L + k], z[k]), vec[384 + h * L + k]);
-        float m = z[0];
+        if (phi == LIME_PHI_SILU) {
 #pragma unroll
-        for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
-        float s = 0.f;
+          for (int k = 0; k < L; ++k) z[k] = silu_fast(z[k]) * (1.0f / L);
+        } else {
+          float m = z[0];
 #pragma unroll
-        for (int k = 0; k < L; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
-        const float inv = 1.0f / s;
+          for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
+          float s = 0.f;
 #pragma unroll
-        for (int k = 0; k < L; ++k) z[k] *= inv;
+          for (int k = 0; k < L; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
+          const float inv = 1.0f / s;
+#pragma unroll
+          for (int k = 0; k < L; ++k) z[k] *= inv;
+        }
 #pragma unroll
         for (int q = 0; q < L / 8; ++q) sw_st16(sA, kBlk, row, h * L + q * 8, pack8(z + q * 8));
         fence_proxy_async_smem();
@@ -1465,7 +1509,7 @@ template <int L>
 int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, const void* E_in,
               const void* Z_in, const lime_layer_w& w, void* E_out, void* Z_out, uint8_t* ws,
               unsigned* status, cudaStream_t st) {
-  const LayerWs Lw = layer_ws(L, B, nh);
+  const LayerWs Lw = layer_ws(L, B, nh, D.phi == LIME_PHI_SILU);
   const bool last = E_out == nullptr;
   const float scale = 1.0f / sqrtf((float)kDH);
   const int64_t nz = B * L;
@@ -1485,7 +1529,7 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     int rc = launch_pdl(k_link_proj<L>, dim3((unsigned)((nz + kTile - 1) / kTile), last ? 1 : 3,
                                              last ? 4 : 2),
                         dim3(512), smem, st, 1, (const bf16*)Z_in, nz, (const bf16*)w.g1,
-                        (const bf16*)w.b1, ws, Lw, scale, status);
+                        (const bf16*)w.b1, ws, Lw, scale, D.phi == LIME_PHI_SILU, status);
     if (rc) return rc;
   }
   if (nh > 0) {
@@ -1499,7 +1543,7 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
       auto kern = last ? k_hist_xattn<L, false> : k_hist_xattn<L, true>;
       if (!set_smem(kern, kXaSmem)) return LIME_ERR_CUDA;
       int rc = launch_pdl(kern, dim3(grid), dim3(kXaThreads), kXaSmem, st, 1, tmE, tmY, ws, Lw,
-                          status);
+                          D.phi, status);
       if (rc) return rc;
     }
     if (!last) {
@@ -1530,7 +1574,7 @@ bool fast_layer_supported(const lime_dims& D) {
 
 size_t fast_layer_ws_bytes(const lime_dims& D, int64_t B, int64_t total_hist) {
   if (!fast_layer_supported(D)) return 0;
-  return layer_ws(D.l, B, total_hist).total;
+  return layer_ws(D.l, B, total_hist, D.phi == LIME_PHI_SILU).total;
 }
 
 int fast_xor_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh,

@@ -17,6 +17,7 @@ import torch
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblime.so")
 
 LIME_F32, LIME_BF16 = 0, 1
+LIME_PHI_SOFTMAX, LIME_PHI_SILU = 0, 1
 LIME_OK, LIME_ERR_ARG, LIME_ERR_SHAPE, LIME_ERR_ALIAS, LIME_ERR_CUDA = 0, -1, -2, -3, -4
 LIME_ERR_SCRATCH = -5
 LIME_NOALLOC_SCRATCH_BYTES = 1 << 20
@@ -35,7 +36,8 @@ class LimeError(RuntimeError):
 
 class lime_dims(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("H", ctypes.c_int32), ("l", ctypes.c_int32),
-                ("f", ctypes.c_int32), ("c", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+                ("f", ctypes.c_int32), ("c", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("phi", ctypes.c_int32)]
 
 
 class lime_layer_w(ctypes.Structure):
@@ -110,9 +112,10 @@ def _check(fn: str, rc: int):
         raise LimeError(fn, rc)
 
 
-def make_dims(d: int, H: int, l: int, f: int, c: int, dtype) -> lime_dims:
+def make_dims(d: int, H: int, l: int, f: int, c: int, dtype, phi="softmax") -> lime_dims:
     dt = LIME_BF16 if dtype in (torch.bfloat16, "bf16", LIME_BF16) else LIME_F32
-    return lime_dims(d, H, l, f, c, dt)
+    ph = LIME_PHI_SILU if phi in ("silu", LIME_PHI_SILU) else LIME_PHI_SOFTMAX
+    return lime_dims(d, H, l, f, c, dt, ph)
 
 
 def lime_workspace_bytes(dims: lime_dims, B: int, total_hist: int) -> int:

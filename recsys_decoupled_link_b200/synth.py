@@ -47,6 +47,7 @@ class Workload:
     cand: tuple            # ("uniform_noreplace",) | ("uniform",) | ("zipf", s)
     dtype: str             # "bf16" | "f32"
     seed: int
+    phi: str = "softmax"   # attention weight function: "softmax" | "silu"
 
     @property
     def f(self) -> int:

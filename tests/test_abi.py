@@ -152,3 +152,16 @@ def test_host_validation_of_uncached_scoring(lime):
     assert f(*args(O=0x200000)) == lime.LIME_ERR_ALIAS                     # O over the image
     assert f(*args(dims=lime.make_dims(128, 4, 64, 256, 64, "bf16"))) == lime.LIME_ERR_SHAPE
     assert f(*args(dims=lime.make_dims(128, 4, 32, 256, 64, "f32"))) == lime.LIME_ERR_SHAPE
+
+
+def test_phi_validation(lime):
+    d = lime.make_dims(128, 4, 32, 256, 64, "bf16", phi="silu")
+    assert d.phi == lime.LIME_PHI_SILU
+    assert lime.lime_workspace_bytes(d, 1, 10) > 0
+    bad = lime.lime_dims(128, 4, 32, 256, 64, lime.LIME_BF16, 7)
+    assert lime.lime_workspace_bytes(bad, 1, 10) == 0
+    # the int8 cache holds softmax weights only
+    nws = lime.lime_workspace_bytes(d, 0, 0)
+    g = lime._lib.lime_build_qk_cache_u8
+    assert g(ctypes.byref(d), 0x100000, 10, 0x200000, 0x300000, 0x400000, 0x500000,
+             0x1000000, nws, None) == lime.LIME_ERR_SHAPE

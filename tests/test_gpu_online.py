@@ -19,9 +19,9 @@ from parity_util import assert_close, f64
 pytestmark = pytest.mark.gpu
 
 
-def _run(l, n_cand, n_items=20_000, bad=()):
+def _run(l, n_cand, n_items=20_000, bad=(), phi="softmax"):
     w = synth.workload("standard", l=l, n_items=n_items, B=len(n_cand), layers=1,
-                       cand=("uniform",))
+                       cand=("uniform",), phi=phi)
     us = synth.user_side(w, [1] * w.B)
     cs = synth.candidate_side(w, n_cand)
     T = synth.item_table(w)
@@ -30,7 +30,7 @@ def _run(l, n_cand, n_items=20_000, bad=()):
     ids = cs.cand_ids.clone()
     for pos in bad:
         ids[pos] = n_items + 5 if pos % 2 else -3
-    dims = lime.make_dims(w.d, w.H, l, w.f, w.c, "bf16")
+    dims = lime.make_dims(w.d, w.H, l, w.f, w.c, "bf16", phi)
     Td, Ld, Wq, Wk, LPd = (t.cuda() for t in (T, us.L, cs.Wq_c, cs.Wk_c, LP))
     idd, offd = ids.cuda(), cs.cand_offsets.cuda()
     ws = lime.Workspace(dims, 0, 0)
@@ -44,9 +44,10 @@ def _run(l, n_cand, n_items=20_000, bad=()):
     return w, us, cs, T, LP, ids, Od, flags
 
 
+@pytest.mark.parametrize("phi", ["softmax", "silu"])
 @pytest.mark.parametrize("l,n_cand", [(32, [5, 0, 300, 128]), (16, [257, 1, 0, 3])])
-def test_uncached_scoring_matches_direct_attention(l, n_cand):
-    w, us, cs, T, LP, ids, Od, flags = _run(l, n_cand)
+def test_uncached_scoring_matches_direct_attention(l, n_cand, phi):
+    w, us, cs, T, LP, ids, Od, flags = _run(l, n_cand, phi=phi)
     assert flags == 0
     offs = cs.cand_offsets.numpy()
     ref = np.zeros((int(offs[-1]), w.d))
@@ -54,7 +55,8 @@ def test_uncached_scoring_matches_direct_attention(l, n_cand):
         a, b = offs[u], offs[u + 1]
         if a < b:
             ref[a:b] = O.candidate_attention_uncached(f64(T)[ids[a:b].numpy()], f64(us.L),
-                                                      f64(cs.Wq_c), f64(cs.Wk_c), f64(LP[u]), w.H)
+                                                      f64(cs.Wq_c), f64(cs.Wk_c), f64(LP[u]), w.H,
+                                                      phi=phi)
     assert_close(Od, ref, "bf16", "uncached scoring")
 
 

@@ -62,7 +62,7 @@ def check_workload(w, n_hist=None, n_cand=None, check_e2e=True):
     # each layer in isolation
     E_prev, Z_prev = f64(us.E), f64(Z0_gpu)
     for i, (E_out, Z_out) in enumerate(outs):
-        E_ref, Z_ref = O.xor_layer(E_prev, offs, Z_prev, layers[i], w.H)
+        E_ref, Z_ref = O.xor_layer(E_prev, offs, Z_prev, layers[i], w.H, phi=w.phi)
         assert_close(Z_out, Z_ref, dt, f"layer {i} links")
         if E_out is not None:
             assert_close(E_out, E_ref, dt, f"layer {i} history")
@@ -70,11 +70,12 @@ def check_workload(w, n_hist=None, n_cand=None, check_e2e=True):
         Z_prev = f64(Z_out)
     # end to end user side: a chain of the context-link and layer stores
     chain = w.layers + (1 if w.c > 0 else 0)
-    _, LP_ref = O.user_encode(f64(us.E), offs, Z0_ref, layers, w.H)
+    _, LP_ref = O.user_encode(f64(us.E), offs, Z0_ref, layers, w.H, phi=w.phi)
     if check_e2e:
-        assert_close(LP_gpu, LP_ref, dt, "L^P end to end", stages=chain)
+        assert_close(LP_gpu, LP_ref, dt, "L^P end to end", stages=chain,
+                     chain_rel=w.phi == "silu")
     # cache
-    cache_ref = O.qk_cache(f64(T), f64(us.L), f64(cs.Wq_c), f64(cs.Wk_c), w.H)
+    cache_ref = O.qk_cache(f64(T), f64(us.L), f64(cs.Wq_c), f64(cs.Wk_c), w.H, phi=w.phi)
     assert_close(buf.cache, cache_ref, dt, "QK cache")
     # scoring, isolated and end to end
     O_iso = O.score_candidates(f64(buf.cache), cs.cand_ids.numpy(), cs.cand_offsets.numpy(),
@@ -82,7 +83,8 @@ def check_workload(w, n_hist=None, n_cand=None, check_e2e=True):
     assert_close(buf.O, O_iso, dt, "scoring (GPU cache and L^P)")
     if check_e2e:
         O_e2e = O.score_candidates(cache_ref, cs.cand_ids.numpy(), cs.cand_offsets.numpy(), LP_ref)
-        assert_close(buf.O, O_e2e, dt, "scoring end to end", stages=chain + 2)
+        assert_close(buf.O, O_e2e, dt, "scoring end to end", stages=chain + 2,
+                     chain_rel=w.phi == "silu")
 
 
 SMALL = {
@@ -291,3 +293,28 @@ def test_full_size_sampled(case):
         rows_u = buf.cache[ids.long().cuda()].cpu()
         ref = O.score_candidates(f64(rows_u), np.arange(b - a), [0, b - a], f64(LP_cpu[u:u + 1]))
         assert_close(buf.O[a:b], ref, w.dtype, f"scores user {u}")
+
+
+# phi = SiLU (reading R15): the same checks, oracle and library both in SiLU
+# mode, on the tensor-core path (bf16; l = 16 and 32), the CUDA-core path
+# (fp32 tiny; bf16 l = 64) and the edge users (empty and one-row histories)
+SILU = {
+    "tiny": dict(),
+    "standard": dict(B=3, n_items=200_000),
+    "ragged16": dict(B=5, l=16, n_items=100_000),
+    "ragged64": dict(B=3, l=64, n_items=50_000),
+}
+
+
+@pytest.mark.parametrize("case", list(SILU))
+def test_silu_workload_parity(case):
+    base = "ragged" if case.startswith("ragged") else case
+    check_workload(synth.workload(base, phi="silu", **SILU[case]))
+
+
+def test_silu_edge_cases():
+    n_hist = [0, 1, 127, 128, 129, 300, 0]
+    n_cand = [5, 0, 1, 130, 7, 0, 3]
+    w = synth.workload("standard", B=len(n_hist), n_items=5000, cand=("uniform",), layers=2,
+                       phi="silu")
+    check_workload(w, n_hist=n_hist, n_cand=n_cand)

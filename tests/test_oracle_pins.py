@@ -355,3 +355,80 @@ def test_u8_scoring_with_identity_values_returns_the_dequantised_row():
     ids = np.array([6, 0, 3, 3])
     out = O.score_candidates_u8(q, ids, [0, 4], LP)
     np.testing.assert_array_equal(out, q[ids].reshape(4, H * l) / 255.0)
+
+
+# ------------------------------------------------------- phi = SiLU (R15)
+
+def brute_force_xor_silu(Q, K, V, N, H):
+    """One masked attention over all N + l rows with an explicit (N + l)^2 XOR
+    mask and pointwise weights: weight(i, j) = SiLU(score) / (visible keys of
+    row i), written with torch's SiLU; fully masked rows give 0."""
+    n, d = Q.shape
+    dh = d // H
+    mask = np.array([[(i < N) != (j < N) for j in range(n)] for i in range(n)])
+    out = np.zeros((n, d))
+    for h in range(H):
+        c = slice(h * dh, (h + 1) * dh)
+        S = t64(Q[:, c] @ K[:, c].T) / math.sqrt(dh)
+        W = F.silu(S).numpy() * mask
+        cnt = mask.sum(1, keepdims=True)
+        W = np.divide(W, cnt, out=np.zeros_like(W), where=cnt > 0)
+        out[:, c] = W @ V[:, c]
+    return out
+
+
+@pytest.mark.parametrize("N", [1, 2, 7, 33])
+@pytest.mark.parametrize("l", [1, 4])
+@pytest.mark.parametrize("H", [1, 2])
+def test_silu_xor_attention_equals_full_mask_attention(N, l, H):
+    d = 8 * H
+    Q, K, V = rand(N + l, d), rand(N + l, d), rand(N + l, d)
+    ref = brute_force_xor_silu(Q, K, V, N, H)
+    got = O.xor_attention(Q, K, V, N, H, phi="silu")
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    # and it differs from the softmax form (the switch takes effect)
+    assert np.abs(got - O.xor_attention(Q, K, V, N, H)).max() > 1e-3
+
+
+def test_silu_empty_history_gives_zero_link_output():
+    l, d = 4, 16
+    Q, K, V = rand(l, d), rand(l, d), rand(l, d)
+    assert np.all(O.xor_attention(Q, K, V, 0, 2, phi="silu") == 0.0)
+
+
+def test_silu_weights_hand_computed():
+    # d = 2, one head: T = (1, 0), L = I, Wq = Wk = I -> scores (1/sqrt 2, 0);
+    # SiLU(1/sqrt 2) = 0.70710678 / (1 + 0.49306869) = 0.47359293...,
+    # SiLU(0) = 0, each divided by l = 2
+    T = np.array([[1.0, 0.0]])
+    c = O.qk_cache(T, np.eye(2), np.eye(2), np.eye(2), 1, phi="silu")
+    np.testing.assert_allclose(c[0, 0], [0.4735929333 / 2, 0.0], rtol=0, atol=1e-10)
+
+
+@pytest.mark.parametrize("H", [1, 4])
+def test_silu_cached_scoring_equals_uncached_attention(H):
+    n, l, d, B = 40, 8, 16, 3
+    T, L = rand(n, d), rand(l, d)
+    Wq, Wk = rand(d, d, scale=0.5), rand(d, d, scale=0.5)
+    LP = rand(B, l, d)
+    counts = [5, 0, 9]
+    offs = np.concatenate([[0], np.cumsum(counts)])
+    ids = rng.integers(0, n, sum(counts))
+    cache = O.qk_cache(T, L, Wq, Wk, H, phi="silu")
+    got = O.score_candidates(cache, ids, offs, LP)
+    for u in range(B):
+        a, b = offs[u], offs[u + 1]
+        if a < b:
+            direct = O.candidate_attention_uncached(T[ids[a:b]], L, Wq, Wk, LP[u], H, phi="silu")
+            np.testing.assert_allclose(got[a:b], direct, rtol=0, atol=1e-12)
+
+
+def test_silu_layer_is_permutation_invariant_for_links():
+    N, l, d, H = 9, 4, 16, 2
+    E, Z = rand(N, d), rand(l, d)
+    w = rand_layer(d, 2 * d)
+    perm = rng.permutation(N)
+    E1, Z1 = O.xor_layer_user(E, Z, w, H, phi="silu")
+    E2, Z2 = O.xor_layer_user(E[perm], Z, w, H, phi="silu")
+    np.testing.assert_allclose(Z2, Z1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(E2, E1[perm], rtol=0, atol=1e-12)

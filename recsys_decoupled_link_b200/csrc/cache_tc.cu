@@ -120,10 +120,10 @@ __global__ void __launch_bounds__(128) k_fold_g_img(const bf16* __restrict__ L,
   }
 }
 
-template <int HL, int L, bool U8>
+template <int HL, int L, bool U8, bool SILU>
 __global__ void __launch_bounds__(CacheCfg<HL, L, U8>::THREADS, 1)
     k_cache_tc(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmC,
-               const bf16* __restrict__ gimg, int n_tiles, int phi, unsigned* status) {
+               const bf16* __restrict__ gimg, int n_tiles, unsigned* status) {
   using C = CacheCfg<HL, L, U8>;
   constexpr int H = HL / L;
   constexpr uint32_t IDESC = idesc_bf16(kBM, HL);
@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(CacheCfg<HL, L, U8>::THREADS, 1)
           tmem_ld16(tmem + lane_base + acc * HL + h * L + q * 16, z + q * 16);
         tmem_ld_wait();
         float inv;
-        if (!U8 && phi == LIME_PHI_SILU) {
+        if constexpr (SILU) {
           // SiLU of each score over the l links (the int8 cache is softmax only)
 #pragma unroll
           for (int k = 0; k < L; ++k) z[k] = __fdividef(z[k], 1.0f + __expf(-z[k]));
@@ -327,9 +327,9 @@ __global__ void __launch_bounds__(CacheCfg<HL, L, U8>::THREADS, 1)
   }
 }
 
-template <int HL, int L, bool U8>
+template <int HL, int L, bool U8, bool SILU>
 int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, int tiles_per_cta,
-                 int phi, unsigned* status, cudaStream_t st) {
+                 unsigned* status, cudaStream_t st) {
   using C = CacheCfg<HL, L, U8>;
   CUtensorMap tmT, tmC;
   if (!make_tmap_2d_bf16(&tmT, T, kD, (uint64_t)n, kD * 2, 64, kBM)) return LIME_ERR_CUDA;
@@ -338,7 +338,7 @@ int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, int til
   } else if (!make_tmap_2d_bf16(&tmC, cache, HL, (uint64_t)n, HL * 2, 64, kBM)) {
     return LIME_ERR_CUDA;
   }
-  if (cudaFuncSetAttribute(k_cache_tc<HL, L, U8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(k_cache_tc<HL, L, U8, SILU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::SMEM) != cudaSuccess)
     return LIME_ERR_CUDA;
   const int n_tiles = (int)((n + kBM - 1) / kBM);
@@ -346,8 +346,8 @@ int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, int til
   // that the build can share the GPU with higher-priority work
   int grid = n_tiles < num_sms() ? n_tiles : num_sms();
   if (tiles_per_cta > 0) grid = (n_tiles + tiles_per_cta - 1) / tiles_per_cta;
-  return launch_pdl(k_cache_tc<HL, L, U8>, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, tmT, tmC,
-                    img, n_tiles, phi, status);
+  return launch_pdl(k_cache_tc<HL, L, U8, SILU>, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, tmT, tmC,
+                    img, n_tiles, status);
 }
 
 }  // namespace
@@ -378,18 +378,25 @@ int launch_build(const lime_dims& D, const void* T, int64_t n, const bf16* img, 
                  bool u8, int tpc, unsigned* status, cudaStream_t st) {
   if (n == 0) return LIME_OK;
   switch (D.H * D.l * 1000 + D.l + (u8 ? 1000000 : 0)) {
-    case 64016: return launch_cache<64, 16, false>(T, n, img, cache, tpc, D.phi, status, st);
-    case 64032: return launch_cache<64, 32, false>(T, n, img, cache, tpc, D.phi, status, st);
-    case 128016: return launch_cache<128, 16, false>(T, n, img, cache, tpc, D.phi, status, st);
-    case 128032: return launch_cache<128, 32, false>(T, n, img, cache, tpc, D.phi, status, st);
-    case 128064: return launch_cache<128, 64, false>(T, n, img, cache, tpc, D.phi, status, st);
-    case 256032: return launch_cache<256, 32, false>(T, n, img, cache, tpc, D.phi, status, st);
-    case 256064: return launch_cache<256, 64, false>(T, n, img, cache, tpc, D.phi, status, st);
-    case 1128016: return launch_cache<128, 16, true>(T, n, img, cache, tpc, D.phi, status, st);
-    case 1128032: return launch_cache<128, 32, true>(T, n, img, cache, tpc, D.phi, status, st);
-    case 1128064: return launch_cache<128, 64, true>(T, n, img, cache, tpc, D.phi, status, st);
-    case 1256032: return launch_cache<256, 32, true>(T, n, img, cache, tpc, D.phi, status, st);
-    case 1256064: return launch_cache<256, 64, true>(T, n, img, cache, tpc, D.phi, status, st);
+    case 64016: return (D.phi == LIME_PHI_SILU ? launch_cache<64, 16, false, true>(T, n, img, cache, tpc, status, st)
+                                          : launch_cache<64, 16, false, false>(T, n, img, cache, tpc, status, st));
+    case 64032: return (D.phi == LIME_PHI_SILU ? launch_cache<64, 32, false, true>(T, n, img, cache, tpc, status, st)
+                                          : launch_cache<64, 32, false, false>(T, n, img, cache, tpc, status, st));
+    case 128016: return (D.phi == LIME_PHI_SILU ? launch_cache<128, 16, false, true>(T, n, img, cache, tpc, status, st)
+                                          : launch_cache<128, 16, false, false>(T, n, img, cache, tpc, status, st));
+    case 128032: return (D.phi == LIME_PHI_SILU ? launch_cache<128, 32, false, true>(T, n, img, cache, tpc, status, st)
+                                          : launch_cache<128, 32, false, false>(T, n, img, cache, tpc, status, st));
+    case 128064: return (D.phi == LIME_PHI_SILU ? launch_cache<128, 64, false, true>(T, n, img, cache, tpc, status, st)
+                                          : launch_cache<128, 64, false, false>(T, n, img, cache, tpc, status, st));
+    case 256032: return (D.phi == LIME_PHI_SILU ? launch_cache<256, 32, false, true>(T, n, img, cache, tpc, status, st)
+                                          : launch_cache<256, 32, false, false>(T, n, img, cache, tpc, status, st));
+    case 256064: return (D.phi == LIME_PHI_SILU ? launch_cache<256, 64, false, true>(T, n, img, cache, tpc, status, st)
+                                          : launch_cache<256, 64, false, false>(T, n, img, cache, tpc, status, st));
+    case 1128016: return launch_cache<128, 16, true, false>(T, n, img, cache, tpc, status, st);
+    case 1128032: return launch_cache<128, 32, true, false>(T, n, img, cache, tpc, status, st);
+    case 1128064: return launch_cache<128, 64, true, false>(T, n, img, cache, tpc, status, st);
+    case 1256032: return launch_cache<256, 32, true, false>(T, n, img, cache, tpc, status, st);
+    case 1256064: return launch_cache<256, 64, true, false>(T, n, img, cache, tpc, status, st);
     default: return LIME_ERR_SHAPE;
   }
 }

@@ -619,10 +619,10 @@ constexpr uint32_t kXaSmem = 1024 + 12 * kBlk + 1024 /* mu, rstd */ + 4096 /* re
                              1024 /* cv, dv */ + 2 * 2048 /* vec x2 */ +
                              kBlk /* one block of G'lo (phi = SiLU) */ + 256 /* barriers */;
 
-template <int L, bool HIST>
+template <int L, bool HIST, bool SILU>
 __global__ void __launch_bounds__(kXaThreads, 1)
     k_hist_xattn(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
-                 uint8_t* __restrict__ ws, LayerWs Lw, int phi, unsigned* status) {
+                 uint8_t* __restrict__ ws, LayerWs Lw, unsigned* status) {
   constexpr int HL = kH * L;
   constexpr uint32_t kSlot = 2 * kBlk;
   extern __shared__ uint8_t smem_raw[];
@@ -700,7 +700,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
           mbar_wait(&bar[3], ph, status, c.abort_flag);
           tc_fence_after();
           mma_tile(c.tmem, smem_u32(sA), kBlk, smem_u32(sG), kBlk, HL, 128, false);
-          if (phi == LIME_PHI_SILU) {
+          if constexpr (SILU) {
             // + E G'lo, one 64-column block at a time through sGl
             for (int j = 0; j < 2; ++j) {
               const uint32_t pj = (uint32_t)(2 * it + j) & 1u;
@@ -815,7 +815,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
             m = fmaxf(m, z[j]);
           }
         }
-        if (phi == LIME_PHI_SILU) {
+        if constexpr (SILU) {
           // pointwise weights: SiLU of each valid score; the record's (max,
           // sum) = (0, valid tokens) makes the merge's total divide by N_u
 #pragma unroll
@@ -872,7 +872,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
 #pragma unroll
         for (int k = 0; k < L; ++k)
           z[k] = fmaf(rs_r, fmaf(-mu_r, vec[256 + h * L + k], z[k]), vec[384 + h * L + k]);
-        if (phi == LIME_PHI_SILU) {
+        if constexpr (SILU) {
 #pragma unroll
           for (int k = 0; k < L; ++k) z[k] = silu_fast(z[k]) * (1.0f / L);
         } else {
@@ -1540,10 +1540,12 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     const int64_t tiles_hi = Lw.max_tiles;
     const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
     {
-      auto kern = last ? k_hist_xattn<L, false> : k_hist_xattn<L, true>;
+      const bool silu = D.phi == LIME_PHI_SILU;
+      auto kern = last ? (silu ? k_hist_xattn<L, false, true> : k_hist_xattn<L, false, false>)
+                       : (silu ? k_hist_xattn<L, true, true> : k_hist_xattn<L, true, false>);
       if (!set_smem(kern, kXaSmem)) return LIME_ERR_CUDA;
       int rc = launch_pdl(kern, dim3(grid), dim3(kXaThreads), kXaSmem, st, 1, tmE, tmY, ws, Lw,
-                          D.phi, status);
+                          status);
       if (rc) return rc;
     }
     if (!last) {

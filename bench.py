@@ -428,29 +428,34 @@ def main():
 
     # phi = SiLU (pointwise attention weights): the same step, inputs and
     # timing, with the SiLU variant of every attention
-    silu_ms = None
-    if w.dtype == "bf16" and not args.eager:
+    # and LIME-XOR+Window (history queries also see l/2 neighbours on each side;
+    # the CUDA-core layer kernels)
+    def variant_ms(phi="softmax", window=0, steps=args.steps):
         import dataclasses
-        ws_ = dataclasses.replace(w, phi="silu")
-        xs = dataclasses.replace(x, w=ws_, dims=lime.make_dims(w.d, w.H, w.l, w.f, w.c, w.dtype,
-                                                                "silu"))
-        bs = pipeline.alloc(xs)
-        gs = pipeline.step_graphs(xs, bs)[0]
+        wv = dataclasses.replace(w, phi=phi, window=window)
+        xv = dataclasses.replace(x, w=wv, dims=lime.make_dims(w.d, w.H, w.l, w.f, w.c, w.dtype,
+                                                               phi, window))
+        bv = pipeline.alloc(xv)
+        gv = pipeline.step_graphs(xv, bv)[0]
         for _ in range(3):
             flush.zero_()
-            gs.replay()
-        sev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-        for k in range(args.steps):
+            gv.replay()
+        vev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for k in range(steps):
             flush.zero_()
-            sev[k][0].record(stream)
-            gs.replay()
-            sev[k][1].record(stream)
+            vev[k][0].record(stream)
+            gv.replay()
+            vev[k][1].record(stream)
         torch.cuda.synchronize()
-        if lime.lime_get_status(bs.ws) != 0:
-            raise RuntimeError("device status flags set during the SiLU steps")
-        silu_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in sev)], dist,
-                                 "cuda")[0] / args.steps
-        del gs, bs, xs
+        if lime.lime_get_status(bv.ws) != 0:
+            raise RuntimeError(f"device status flags set during the {phi}/{window} steps")
+        return max_over_ranks([sum(a.elapsed_time(b) for a, b in vev)], dist,
+                              "cuda")[0] / steps
+
+    silu_ms = win_ms = None
+    if w.dtype == "bf16" and not args.eager:
+        silu_ms = variant_ms(phi="silu")
+        win_ms = variant_ms(window=w.l // 2, steps=min(args.steps, 5))
 
     # Uncached (online) scoring at scale: the same IDs, with the weights computed
     # per candidate from the item table and the folded G image.
@@ -583,6 +588,12 @@ def main():
                 "ms": silu_ms, "pairs_per_s": total_cand / (silu_ms * 1e-3),
                 "note": "the whole step with phi = SiLU (pointwise attention weights) in both "
                         "XOR branches and the cache"}
+        if win_ms is not None:
+            phases["step_xor_window"] = {
+                "ms": win_ms, "pairs_per_s": total_cand / (win_ms * 1e-3),
+                "history_tokens_per_s": total_hist / (win_ms * 1e-3),
+                "note": f"the whole step with LIME-XOR+Window (window {w.l // 2} on each side); "
+                        "its layers run on the CUDA-core kernels"}
         if on_ms is not None:
             on_bytes = sc_pairs * (4 * w.d + 4)   # item row in, score row out, ID
             on_gbs = on_bytes / (on_ms * 1e-3) / 1e9

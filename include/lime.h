@@ -55,6 +55,13 @@ typedef enum { LIME_F32 = 0, LIME_BF16 = 1 } lime_dtype;
  * supports softmax only (SiLU weights can be negative).                     */
 typedef enum { LIME_PHI_SOFTMAX = 0, LIME_PHI_SILU = 1 } lime_phi;
 
+/* LIME-XOR+Window (LIME note, 关键设计 3): besides the l links, each history
+ * token attends to the neighbouring history tokens of its own user, window
+ * rows on each side (itself excluded, fewer at the ends of the history), all
+ * in one phi over the union of keys; link queries are unchanged.  The pages'
+ * variant has l neighbours in all: window = l / 2.  0 <= window <= 64; a
+ * nonzero window runs the CUDA-core layer kernels.                          */
+
 enum {
   LIME_OK = 0,
   LIME_ERR_ARG = -1,    /* null pointer, negative size, workspace too small  */
@@ -79,6 +86,8 @@ typedef struct {
   int32_t c;      /* user context feature dim (0: no context MLP)            */
   int32_t dtype;  /* lime_dtype                                              */
   int32_t phi;    /* lime_phi: the attention weight function (0 = softmax)   */
+  int32_t window; /* LIME-XOR+Window: a history query also attends to the    */
+                  /* user's history rows within this distance (0: XOR only) */
 } lime_dims;
 
 /* One LIME-XOR layer's parameters (device pointers, dims->dtype):

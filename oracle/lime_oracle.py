@@ -51,6 +51,12 @@ notes of the library):
      query (a user with N_u = 0 gives the link branch a zero output, as in R8).
      Division by the key count keeps the weights' scale that of an average, as
      the softmax's are; the pages give no other normaliser.
+  R17 LIME-XOR+Window (LIME note, 关键设计 3): each history token also attends
+     to the neighbouring history tokens of its own user, "the l tokens before
+     and after it", for 2l key dependencies in all (l links + l neighbours):
+     the history rows j with 0 < |i - j| <= w, w = l / 2 (fewer at the ends of
+     the history; no self-attention, as in the XOR mask), in one phi over the
+     union of the link and window keys.  Link queries are unchanged.
 """
 from __future__ import annotations
 
@@ -125,7 +131,7 @@ def context_links_batch(L, ctx, Wc1, bc1, Wc2, bc2) -> np.ndarray:
 # ------------------------------------------------------ user side: XOR layer
 
 def xor_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, N: int,
-                  H: int, phi: str = "softmax") -> np.ndarray:
+                  H: int, phi: str = "softmax", window: int = 0) -> np.ndarray:
     """Two-branch XOR attention over X = [E; L^C] for one user.
 
     LIME note, 关键设计 2 (XORA decomposition):
@@ -135,7 +141,8 @@ def xor_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, N: int,
     rows [0, N) are history, rows [N, N + l) are links.  Returns the per-row
     attention output [N + l, d] before the output projection.  With N = 0 the
     link rows have no key to attend to and get a zero output (reading R8).
-    phi: "softmax" (R2) or "silu" (R15).
+    phi: "softmax" (R2) or "silu" (R15).  window > 0 (R17): a history query
+    also attends to the history rows within `window` positions of it.
     """
     n_rows, d = Q.shape
     dh = d // H
@@ -146,8 +153,18 @@ def xor_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, N: int,
     for h in range(H):
         c = slice(h * dh, (h + 1) * dh)
         # history -> link branch: MHA(E, L^C, L^C)
-        P_hist = attention_weights(s * (Q[:N, c] @ K[N:, c].T), 1, phi)   # [N, l]
-        A[:N, c] = P_hist @ V[N:, c]
+        if window == 0:
+            P_hist = attention_weights(s * (Q[:N, c] @ K[N:, c].T), 1, phi)   # [N, l]
+            A[:N, c] = P_hist @ V[N:, c]
+        else:
+            # + the window of neighbouring history rows, one phi per row over
+            # the union of its keys
+            for i in range(N):
+                nb = [j for j in range(max(0, i - window), min(N, i + window + 1)) if j != i]
+                keys = np.concatenate([K[N:, c], K[nb, c]])
+                vals = np.concatenate([V[N:, c], V[nb, c]])
+                p = attention_weights(s * (keys @ Q[i, c]), 0, phi)
+                A[i, c] = p @ vals
         # link -> history branch: MHA(L^C, E, E)
         P_link = attention_weights(s * (Q[N:, c] @ K[:N, c].T), 1, phi)   # [l, N]
         A[N:, c] = P_link @ V[:N, c]
@@ -165,7 +182,7 @@ def gated_mlp(x: np.ndarray, W1: np.ndarray, W3: np.ndarray,
 
 
 def xor_layer_user(E: np.ndarray, Z: np.ndarray, w: Dict[str, np.ndarray],
-                   H: int, phi: str = "softmax"):
+                   H: int, phi: str = "softmax", window: int = 0):
     """One LIME-XOR layer for one user: (E [N, d], Z [l, d]) -> (E', Z').
 
     LIME note, 关键设计 2 (XOR mask, XORA decomposition, residual + GatedMLP)
@@ -181,14 +198,14 @@ def xor_layer_user(E: np.ndarray, Z: np.ndarray, w: Dict[str, np.ndarray],
     X = np.concatenate([E, Z], axis=0)
     Xh = layer_norm(X, w["g1"], w["b1"])
     Q, K, V = Xh @ w["Wq"], Xh @ w["Wk"], Xh @ w["Wv"]
-    Y = X + xor_attention(Q, K, V, N, H, phi) @ w["Wo"]
+    Y = X + xor_attention(Q, K, V, N, H, phi, window) @ w["Wo"]
     Xp = Y + gated_mlp(layer_norm(Y, w["g2"], w["b2"]), w["W1"], w["W3"], w["W2"])
     return Xp[:N], Xp[N:]
 
 
 def xor_layer(E: np.ndarray, hist_offsets: Sequence[int], Z: np.ndarray,
               w: Dict[str, np.ndarray], H: int, users: Optional[Sequence[int]] = None,
-              phi: str = "softmax"):
+              phi: str = "softmax", window: int = 0):
     """xor_layer_user over a packed batch.
 
     E [sum N, d] packed by hist_offsets [B + 1]; Z [B, l, d].
@@ -201,12 +218,12 @@ def xor_layer(E: np.ndarray, hist_offsets: Sequence[int], Z: np.ndarray,
     Zp = np.full_like(Z, np.nan)
     for u in users:
         a, b = int(hist_offsets[u]), int(hist_offsets[u + 1])
-        Ep[a:b], Zp[u] = xor_layer_user(E[a:b], Z[u], w, H, phi)
+        Ep[a:b], Zp[u] = xor_layer_user(E[a:b], Z[u], w, H, phi, window)
     return Ep, Zp
 
 
 def user_encode(E, hist_offsets, Z0, layers: List[Dict[str, np.ndarray]], H,
-                users=None, phi: str = "softmax"):
+                users=None, phi: str = "softmax", window: int = 0):
     """Stack of LIME-XOR layers; returns (E after the last layer, L^P).
 
     LIME note, 整体框架 / 一个完整示例 step 2: the context links pass through
@@ -215,7 +232,7 @@ def user_encode(E, hist_offsets, Z0, layers: List[Dict[str, np.ndarray]], H,
     """
     Ecur, Zcur = E, Z0
     for w in layers:
-        Ecur, Zcur = xor_layer(Ecur, hist_offsets, Zcur, w, H, users, phi)
+        Ecur, Zcur = xor_layer(Ecur, hist_offsets, Zcur, w, H, users, phi, window)
     return Ecur, Zcur
 
 

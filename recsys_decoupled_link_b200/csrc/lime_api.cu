@@ -23,6 +23,7 @@ bool dims_ok(const lime_dims* D) {
   if (!D) return false;
   if (D->dtype != LIME_F32 && D->dtype != LIME_BF16) return false;
   if (D->phi != LIME_PHI_SOFTMAX && D->phi != LIME_PHI_SILU) return false;
+  if (D->window < 0 || D->window > 64) return false;
   return true;
 }
 

@@ -203,13 +203,15 @@ __global__ void k_unpack_rows(const float* __restrict__ X, int64_t nh, int64_t n
 
 // ---------------------------------------------------------- XOR attention
 // History branch, MHA(E, L^C, L^C): history row i of user u attends to the l
-// link rows of u, per head (LIME note, 关键设计 2).  One warp per (row, head).
-// Q, K, V are fp32 [nh + B*l, d]; link row k of user u is row nh + u*l + k.
+// link rows of u, per head (LIME note, 关键设计 2), and with LIME-XOR+Window
+// (关键设计 3) also to the user's history rows j with 0 < |i - j| <= window,
+// in one phi over the union of keys.  One warp per (row, head).  Q, K, V are
+// fp32 [nh + B*l, d]; link row k of user u is row nh + u*l + k.
 __global__ void k_attn_hist(const float* __restrict__ Q, const float* __restrict__ K,
                             const float* __restrict__ V, const int64_t* __restrict__ off,
                             int64_t B, int64_t nh, int d, int H, int l, float scale,
-                            int phi, float* __restrict__ A) {
-  extern __shared__ float sp[];  // [warps][l]
+                            int phi, int window, float* __restrict__ A, unsigned* status) {
+  extern __shared__ float sp[];  // [warps][l + 2 window]
   int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int64_t task = blockIdx.x * (int64_t)(blockDim.x >> 5) + warp;
   if (task >= nh * H) return;
@@ -217,31 +219,44 @@ __global__ void k_attn_hist(const float* __restrict__ Q, const float* __restrict
   int h = task % H;
   int dh = d / H;
   int64_t u = owner_of(off, B, i);
+  // the window: history rows [wa, wb) of the same user, row i itself skipped
+  int64_t ua = 0, ub = 0;
+  if (window > 0) user_range(off, u, B, nh, &ua, &ub, status);
+  const int64_t wa = i - window > ua ? i - window : ua;
+  const int64_t wb = i + window + 1 < ub ? i + window + 1 : ub;
+  const int nw = window > 0 ? (int)(wb - wa) : 0;   // window keys including i
+  const int nk = l + nw;                             // key slots; slot l + (i - wa) is i
   const float* q = Q + i * d + h * dh;
-  float* p = sp + warp * l;
+  float* p = sp + warp * (l + 2 * window + 1);
+  auto key_row = [&](int k) -> int64_t { return k < l ? nh + u * l + k : wa + (k - l); };
   float mx = -INFINITY;
-  for (int k = lane; k < l; k += 32) {
-    const float* kk = K + (nh + u * l + k) * d + h * dh;
-    float s = 0.f;
-    for (int c = 0; c < dh; ++c) s += q[c] * kk[c];
-    s *= scale;
+  for (int k = lane; k < nk; k += 32) {
+    const int64_t r = key_row(k);
+    float s = -INFINITY;
+    if (r != i || k < l) {
+      const float* kk = K + r * d + h * dh;
+      s = 0.f;
+      for (int c = 0; c < dh; ++c) s += q[c] * kk[c];
+      s *= scale;
+    }
     p[k] = s;
     mx = fmaxf(mx, s);
   }
   mx = warp_max(mx);
+  const int n_keys = l + (nw > 0 ? nw - 1 : 0);
   float sum = 0.f;
   if (phi == LIME_PHI_SILU) {
-    // SiLU of each score over the l keys
-    for (int k = lane; k < l; k += 32) p[k] = p[k] / (1.0f + expf(-p[k]));
-    sum = (float)l;
+    // SiLU of each score over the visible keys
+    for (int k = lane; k < nk; k += 32) p[k] = p[k] == -INFINITY ? 0.f : p[k] / (1.0f + expf(-p[k]));
+    sum = (float)n_keys;
   } else {
-    for (int k = lane; k < l; k += 32) { float e = expf(p[k] - mx); p[k] = e; sum += e; }
+    for (int k = lane; k < nk; k += 32) { float e = expf(p[k] - mx); p[k] = e; sum += e; }
     sum = warp_sum(sum);
   }
   __syncwarp();
   for (int c = lane; c < dh; c += 32) {
     float acc = 0.f;
-    for (int k = 0; k < l; ++k) acc += p[k] * V[(nh + u * l + k) * d + h * dh + c];
+    for (int k = 0; k < nk; ++k) acc += p[k] * V[key_row(k) * d + h * dh + c];
     A[i * d + h * dh + c] = acc / sum;
   }
 }
@@ -497,8 +512,8 @@ void simt_xor_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t n
   gemm(Xh, d, w.Wv, bf, d, d, R, nullptr, V, st);
   if (nh > 0) {
     int64_t tasks = nh * H;
-    k_attn_hist<<<(unsigned)((tasks + 7) / 8), 256, 8 * l * sizeof(float), st>>>(
-        Q, K, V, off, B, nh, d, H, l, scale, D.phi, A);
+    k_attn_hist<<<(unsigned)((tasks + 7) / 8), 256, 8 * (l + 2 * D.window + 1) * sizeof(float),
+                  st>>>(Q, K, V, off, B, nh, d, H, l, scale, D.phi, D.window, A, status);
     note_launches(1);
   }
   {

@@ -1571,7 +1571,8 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
 }  // namespace
 
 bool fast_layer_supported(const lime_dims& D) {
-  return D.dtype == LIME_BF16 && D.d == kD && D.H == kH && D.f == kF && (D.l == 16 || D.l == 32);
+  return D.dtype == LIME_BF16 && D.d == kD && D.H == kH && D.f == kF && (D.l == 16 || D.l == 32) &&
+         D.window == 0;
 }
 
 size_t fast_layer_ws_bytes(const lime_dims& D, int64_t B, int64_t total_hist) {

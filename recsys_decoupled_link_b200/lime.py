@@ -37,7 +37,7 @@ class LimeError(RuntimeError):
 class lime_dims(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("H", ctypes.c_int32), ("l", ctypes.c_int32),
                 ("f", ctypes.c_int32), ("c", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("phi", ctypes.c_int32)]
+                ("phi", ctypes.c_int32), ("window", ctypes.c_int32)]
 
 
 class lime_layer_w(ctypes.Structure):
@@ -112,10 +112,11 @@ def _check(fn: str, rc: int):
         raise LimeError(fn, rc)
 
 
-def make_dims(d: int, H: int, l: int, f: int, c: int, dtype, phi="softmax") -> lime_dims:
+def make_dims(d: int, H: int, l: int, f: int, c: int, dtype, phi="softmax",
+              window: int = 0) -> lime_dims:
     dt = LIME_BF16 if dtype in (torch.bfloat16, "bf16", LIME_BF16) else LIME_F32
     ph = LIME_PHI_SILU if phi in ("silu", LIME_PHI_SILU) else LIME_PHI_SOFTMAX
-    return lime_dims(d, H, l, f, c, dt, ph)
+    return lime_dims(d, H, l, f, c, dt, ph, int(window))
 
 
 def lime_workspace_bytes(dims: lime_dims, B: int, total_hist: int) -> int:

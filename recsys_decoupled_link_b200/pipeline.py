@@ -62,7 +62,7 @@ class Buffers:
 def to_device(w: synth.Workload, us: synth.UserSide, cs: synth.CandidateSide,
               T: Optional[torch.Tensor], device="cuda") -> DeviceInputs:
     dev = lambda t: None if t is None else t.to(device).contiguous()
-    dims = lime.make_dims(w.d, w.H, w.l, w.f, w.c, w.dtype, w.phi)
+    dims = lime.make_dims(w.d, w.H, w.l, w.f, w.c, w.dtype, w.phi, w.window)
     layer_tensors = [[dev(t) for t in lw.as_dict().values()] for lw in us.layers]
     if w.c > 0:
         ctx_w = [dev(us.ctx_w.Wc1), dev(us.ctx_w.bc1), dev(us.ctx_w.Wc2), dev(us.ctx_w.bc2)]

@@ -48,6 +48,7 @@ class Workload:
     dtype: str             # "bf16" | "f32"
     seed: int
     phi: str = "softmax"   # attention weight function: "softmax" | "silu"
+    window: int = 0        # LIME-XOR+Window half-width (0: XOR only; the pages' variant l/2)
 
     @property
     def f(self) -> int:

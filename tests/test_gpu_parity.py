@@ -62,7 +62,8 @@ def check_workload(w, n_hist=None, n_cand=None, check_e2e=True):
     # each layer in isolation
     E_prev, Z_prev = f64(us.E), f64(Z0_gpu)
     for i, (E_out, Z_out) in enumerate(outs):
-        E_ref, Z_ref = O.xor_layer(E_prev, offs, Z_prev, layers[i], w.H, phi=w.phi)
+        E_ref, Z_ref = O.xor_layer(E_prev, offs, Z_prev, layers[i], w.H, phi=w.phi,
+                                   window=w.window)
         assert_close(Z_out, Z_ref, dt, f"layer {i} links")
         if E_out is not None:
             assert_close(E_out, E_ref, dt, f"layer {i} history")
@@ -70,7 +71,7 @@ def check_workload(w, n_hist=None, n_cand=None, check_e2e=True):
         Z_prev = f64(Z_out)
     # end to end user side: a chain of the context-link and layer stores
     chain = w.layers + (1 if w.c > 0 else 0)
-    _, LP_ref = O.user_encode(f64(us.E), offs, Z0_ref, layers, w.H, phi=w.phi)
+    _, LP_ref = O.user_encode(f64(us.E), offs, Z0_ref, layers, w.H, phi=w.phi, window=w.window)
     if check_e2e:
         assert_close(LP_gpu, LP_ref, dt, "L^P end to end", stages=chain,
                      chain_rel=w.phi == "silu")
@@ -317,4 +318,28 @@ def test_silu_edge_cases():
     n_cand = [5, 0, 1, 130, 7, 0, 3]
     w = synth.workload("standard", B=len(n_hist), n_items=5000, cand=("uniform",), layers=2,
                        phi="silu")
+    check_workload(w, n_hist=n_hist, n_cand=n_cand)
+
+
+# LIME-XOR+Window (reading R17): history queries also attend to the l/2
+# neighbouring history rows on each side (the CUDA-core layer kernels)
+WINDOW = {
+    "tiny": dict(window=16),
+    "standard": dict(B=3, n_items=50_000, window=16),
+    "standard_silu": dict(B=3, n_items=50_000, window=16, phi="silu"),
+    "ragged16": dict(B=4, l=16, n_items=50_000, window=8),
+}
+
+
+@pytest.mark.parametrize("case", list(WINDOW))
+def test_window_workload_parity(case):
+    base = "ragged" if case.startswith("ragged") else case.split("_")[0]
+    check_workload(synth.workload(base, **WINDOW[case]))
+
+
+def test_window_edge_cases():
+    n_hist = [0, 1, 2, 17, 300, 0]
+    n_cand = [5, 0, 1, 130, 7, 3]
+    w = synth.workload("standard", B=len(n_hist), n_items=5000, cand=("uniform",), layers=2,
+                       window=16)
     check_workload(w, n_hist=n_hist, n_cand=n_cand)

@@ -432,3 +432,53 @@ def test_silu_layer_is_permutation_invariant_for_links():
     E2, Z2 = O.xor_layer_user(E[perm], Z, w, H, phi="silu")
     np.testing.assert_allclose(Z2, Z1, rtol=0, atol=1e-12)
     np.testing.assert_allclose(E2, E1[perm], rtol=0, atol=1e-12)
+
+
+# ------------------------------------------ LIME-XOR+Window (R17)
+
+def window_mask(N, l, w):
+    n = N + l
+    return np.array([[((i < N) != (j < N)) or (i < N and j < N and 0 < abs(i - j) <= w)
+                      for j in range(n)] for i in range(n)])
+
+
+@pytest.mark.parametrize("N,l,w", [(1, 2, 1), (7, 4, 2), (33, 4, 2), (20, 8, 4), (5, 2, 9)])
+@pytest.mark.parametrize("H", [1, 2])
+def test_window_attention_equals_library_masked_attention(N, l, w, H):
+    # the XOR + window mask written out in full, through torch's masked SDPA
+    d = 8 * H
+    Q, K, V = rand(N + l, d), rand(N + l, d), rand(N + l, d)
+    got = O.xor_attention(Q, K, V, N, H, window=w)
+    dh = d // H
+    q = t64(Q).view(N + l, H, dh).transpose(0, 1)
+    k = t64(K).view(N + l, H, dh).transpose(0, 1)
+    v = t64(V).view(N + l, H, dh).transpose(0, 1)
+    sd = F.scaled_dot_product_attention(q, k, v, attn_mask=t64(window_mask(N, l, w)))
+    np.testing.assert_allclose(got, sd.transpose(0, 1).reshape(N + l, d).numpy(),
+                               rtol=0, atol=1e-12)
+    # link rows do not see the window: they equal the plain XOR attention
+    np.testing.assert_allclose(got[N:], O.xor_attention(Q, K, V, N, H)[N:], rtol=0, atol=1e-12)
+
+
+def test_window_silu_equals_masked_pointwise_attention():
+    N, l, w, H, d = 12, 4, 2, 2, 16
+    Q, K, V = rand(N + l, d), rand(N + l, d), rand(N + l, d)
+    M = window_mask(N, l, w)
+    dh = d // H
+    ref = np.zeros((N + l, d))
+    for h in range(H):
+        c = slice(h * dh, (h + 1) * dh)
+        W = F.silu(t64(Q[:, c] @ K[:, c].T) / math.sqrt(dh)).numpy() * M
+        ref[:, c] = (W / M.sum(1, keepdims=True)) @ V[:, c]
+    got = O.xor_attention(Q, K, V, N, H, phi="silu", window=w)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_window_zero_is_plain_xor_and_one_token_history_has_no_neighbours():
+    N, l, d = 6, 4, 16
+    Q, K, V = rand(N + l, d), rand(N + l, d), rand(N + l, d)
+    np.testing.assert_array_equal(O.xor_attention(Q, K, V, N, 2, window=0),
+                                  O.xor_attention(Q, K, V, N, 2))
+    Q1, K1, V1 = Q[N - 1:], K[N - 1:], V[N - 1:]
+    np.testing.assert_allclose(O.xor_attention(Q1, K1, V1, 1, 2, window=3),
+                               O.xor_attention(Q1, K1, V1, 1, 2), rtol=0, atol=1e-15)

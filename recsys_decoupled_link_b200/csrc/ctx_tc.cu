@@ -42,7 +42,8 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sHlo = sm + 4 * kBlk;          // hidden lo
   uint8_t* sW2 = sm + 6 * kBlk;           // Wc2 [128 x 128] MN-major
   uint8_t* sW1 = sm + 8 * kBlk;           // Wc1 [din x 128] MN-major (2 blocks of din rows)
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sW1 + 2 * w1_blk);   // [0] mma, [1] weights
+  float* sbias = reinterpret_cast<float*>(sW1 + 2 * w1_blk);        // bc1 [128], bc2 [128]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sbias + 2 * kD);      // [0] mma, [1] weights
   uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 2);
   int* abort_flag = reinterpret_cast<int*>(bar + 3);
   const int tid = threadIdx.x;
@@ -57,6 +58,9 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   pdl_launch();
   pdl_wait();
+  // the biases as fp32 in shared memory (the epilogues read them per column;
+  // the gather's barrier below orders these writes before those reads)
+  if (tid < 2 * kD) sbias[tid] = __bfloat162float(tid < kD ? bc1[tid] : bc2[tid - kD]);
   // weights: TMA tiles of the row-major [K x 128] matrices in 128-byte
   // swizzle are exactly the MN-major operand images (64 columns per block)
   if (tid == 0) {
@@ -116,7 +120,7 @@ __global__ void __launch_bounds__(512, 1)
         for (int j = 0; j < 8; ++j) {
           // SiLU with the hardware exp2 / reciprocal approximations (a few
           // ulp; the hidden value is kept to about 16 bits as hi + lo)
-          const float a = x[q * 8 + j] + __bfloat162float(bc1[c0 + q * 8 + j]);
+          const float a = x[q * 8 + j] + sbias[c0 + q * 8 + j];
           const float v = __fdividef(a, 1.0f + __expf(-a));
           h8[j] = __bfloat162float(__float2bfloat16_rn(v));
           l8[j] = v - h8[j];
@@ -140,7 +144,7 @@ __global__ void __launch_bounds__(512, 1)
       tmem_ld16(ta + 128 + c0 + 16, x + 16);
       tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) x[j] += __bfloat162float(bc2[c0 + j]);
+      for (int j = 0; j < 32; ++j) x[j] += sbias[kD + c0 + j];
       // the hidden-hi operand (GEMM 2 is done with it) becomes the output staging
 #pragma unroll
       for (int q = 0; q < 4; ++q) sw_st16(sX, kBlk, row, c0 + q * 8, pack8(x + q * 8));
@@ -165,7 +169,7 @@ bool fast_ctx_supported(const lime_dims& D) {
 }
 
 size_t fast_ctx_smem(const lime_dims& D) {
-  return 1024 + 8 * (size_t)kBlk + 2 * (size_t)(kD + D.c) * 128 + 64;   // + barriers
+  return 1024 + 8 * (size_t)kBlk + 2 * (size_t)(kD + D.c) * 128 + 2 * kD * 4 + 64;   // + biases, barriers
 }
 
 int fast_context_links(const lime_dims& D, int64_t B, const void* L, const void* ctx,

@@ -19,6 +19,13 @@ times come from CUDA events on the launching stream; the job time is the max
 over ranks.  With N > 1 each rank runs an independent replica of the step
 (users and catalogue rows are independent; no collective on the data path),
 so scaling is weak.
+
+At 1 GPU the other workloads (tiny fp32; long history; large candidate set
+over a 10M-item catalogue; ragged histories and candidate counts at l = 16,
+32 and 64) are then timed at full size under "configs": the whole step and
+each phase replayed as CUDA graphs, L2 flushed before every replay, the
+median of up to 20 replays (ragged: warm-L2 step times too).  --configs none
+skips them.
 """
 from __future__ import annotations
 
@@ -240,6 +247,116 @@ def config_of(w, total_cand, total_hist=None):
     return c
 
 
+# ----------------------------------------------------- the other workloads
+
+CONFIG_CASES = {
+    # name: (workload, overrides)
+    "tiny": ("tiny", {}),
+    "long": ("long", {}),
+    "large_cand": ("large_cand", {}),
+    "ragged_l16": ("ragged", {"l": 16}),
+    "ragged_l32": ("ragged", {"l": 32}),
+    "ragged_l64": ("ragged", {"l": 64}),
+}
+
+
+def roofline_of(kind, flops, nbytes, sec, pk, dtype):
+    """Achieved rate against the measured peak: the tensor peak for the user
+    side in bf16, the copy bandwidth for everything else."""
+    if kind == "user" and dtype == "bf16":
+        r = {"bound": "tensor", "achieved": flops / sec / 1e12, "peak": pk["bf16_tflops"],
+             "unit": "TFLOP/s"}
+        r["frac"] = r["achieved"] / r["peak"]
+        r["frac_of_sustained"] = r["achieved"] / pk["bf16_tflops_sustained"]
+        return r
+    r = {"bound": "hbm", "achieved": nbytes / sec / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s"}
+    r["frac"] = r["achieved"] / r["peak"]
+    return r
+
+
+def distinct_row_bytes(w, cand_ids, total_cand):
+    """Scoring bytes when every distinct cache row is read once (Zipf reuse)."""
+    es = 2 if w.dtype == "bf16" else 4
+    n_uniq = int(torch.unique(cand_ids).numel())
+    return n_uniq * w.H * w.l * es + total_cand * (4 + w.d * es)
+
+
+def time_graph(g, flush, stream, runs):
+    """Per-replay times (ms) of a CUDA graph, L2 flushed before each replay when
+    `flush` is given."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(runs)]
+    for e in ev:
+        if flush is not None:
+            flush.zero_()
+        e[0].record(stream)
+        g.replay()
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def time_config(name, flush, stream, pk, T_cache):
+    """One of the other workloads at full size: the whole step and its three
+    phases, each replayed as a CUDA graph with L2 flushed before every replay
+    (plus warm-L2 step times for the ragged workload); median and mean of up to
+    20 replays.  T_cache keeps one device item table per catalogue seed (the
+    table does not depend on the number of links)."""
+    from recsys_decoupled_link_b200 import lime, pipeline, synth
+    base, over = CONFIG_CASES[name]
+    w = synth.workload(base, **over)
+    us, cs = synth.user_side(w), synth.candidate_side(w)
+    x = pipeline.to_device(w, us, cs, None)
+    key = (w.seed, w.n_items, w.d, w.dtype)
+    if key not in T_cache:
+        T_cache.clear()
+        torch.cuda.empty_cache()
+        T_cache[key] = pipeline.item_table_device(w)
+    x.T = T_cache[key]
+    buf = pipeline.alloc(x)
+    graphs = pipeline.step_graphs(x, buf)
+    for _ in range(3):
+        flush.zero_()
+        graphs[0].replay()
+    one = time_graph(graphs[0], flush, stream, 1)[0]
+    runs = max(3, min(20, int(3000.0 / max(one, 1e-3))))
+    step = time_graph(graphs[0], flush, stream, runs)
+    user = time_graph(graphs[1], flush, stream, runs)
+    cache = time_graph(graphs[2], flush, stream, runs)
+    score = time_graph(graphs[3], flush, stream, runs)
+    warm = time_graph(graphs[0], None, stream, runs) if base == "ragged" else None
+    if lime.lime_get_status(buf.ws) != 0:
+        raise RuntimeError(f"device status flags set during the {name} steps")
+    work = work_units(w, x.total_hist, x.total_cand)
+    med = statistics.median
+    fast_layers = w.dtype == "bf16" and w.d == 128 and w.H == 4 and w.l in (16, 32)
+    out = {
+        "workload": config_of(w, x.total_cand, x.total_hist)["workload"],
+        "history_tokens": x.total_hist, "pairs": x.total_cand, "runs": runs,
+        "layer_kernels": "tensor-core" if fast_layers else "CUDA-core",
+        "step_ms": med(step), "step_ms_mean": statistics.mean(step),
+        "pairs_per_s": x.total_cand / (med(step) * 1e-3),
+        "user_encode": {"ms": med(user),
+                        "history_tokens_per_s": x.total_hist / (med(user) * 1e-3),
+                        "roofline": roofline_of("user", *work["user"], med(user) * 1e-3, pk,
+                                                w.dtype)},
+        "qk_cache": {"ms": med(cache), "items_per_s": w.n_items / (med(cache) * 1e-3),
+                     "roofline": roofline_of("cache", *work["cache"], med(cache) * 1e-3, pk,
+                                             w.dtype)},
+        "score": {"ms": med(score), "pairs_per_s": x.total_cand / (med(score) * 1e-3),
+                  "roofline": roofline_of("score", *work["score"], med(score) * 1e-3, pk,
+                                          w.dtype),
+                  "distinct_row_gbs": distinct_row_bytes(w, x.cand_ids, x.total_cand) /
+                  (med(score) * 1e-3) / 1e9},
+    }
+    if warm is not None:
+        out["warm_l2_step_ms"] = med(warm)
+        out["warm_l2_pairs_per_s"] = x.total_cand / (med(warm) * 1e-3)
+    del graphs, buf, x
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------- multi-rank
 
 def max_over_ranks(values, dist=None, device="cpu"):
@@ -268,6 +385,9 @@ def main():
     ap.add_argument("--impl", default="lime", choices=["lime", "reference"])
     ap.add_argument("--workload", default="standard")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", default=",".join(CONFIG_CASES),
+                    help="comma-separated other workloads timed after the main step at 1 GPU "
+                         f"({', '.join(CONFIG_CASES)}), or 'none'")
     ap.add_argument("--eager", action="store_true",
                     help="time the step as eager library calls instead of CUDA graph replays")
     args = ap.parse_args()
@@ -531,22 +651,22 @@ def main():
             lin["us_per_1k_tokens"].append(ms * 1e3 / (xl.total_hist / 1e3))
             del xl, bl
 
+    # The other workloads at full size (1 GPU only: per-GPU measurements, and
+    # the ranks of a replica run would wait on rank 0 meanwhile)
+    cfg = None
+    if world == 1 and args.configs != "none":
+        T_cache, cfg = {}, {}
+        for name in args.configs.split(","):
+            cfg[name] = time_config(name, flush, stream, peaks(), T_cache)
+        T_cache.clear()
+
     if rank == 0:
         pk = peaks()
         work = work_units(w, total_hist, total_cand)
         phase_ms = {k: v / args.steps for k, v in ph.items()}
 
         def phase_roof(name):
-            fl, by = work[name]
-            sec = phase_ms[name] * 1e-3
-            if name == "user" and w.dtype == "bf16":
-                r = {"bound": "tensor", "achieved": fl / sec / 1e12, "peak": pk["bf16_tflops"],
-                     "unit": "TFLOP/s"}
-            else:
-                r = {"bound": "hbm", "achieved": by / sec / 1e9, "peak": pk["hbm_gbs"],
-                     "unit": "GB/s"}
-            r["frac"] = r["achieved"] / r["peak"]
-            return r
+            return roofline_of(name, *work[name], phase_ms[name] * 1e-3, pk, w.dtype)
 
         # The dominant kernel of the step is k_cache_tc (largest single-kernel share
         # in profiles/launches_standard_step.md).  Its duration is taken from the
@@ -562,8 +682,6 @@ def main():
         roof["algorithmic_bytes_per_launch"] = work["cache"][1]
         roof["peak_source"] = pk["source"] + " (MEASURED_PEAKS.json hbm_gbs copy bandwidth)"
         ur = phase_roof("user")
-        if ur["unit"] == "TFLOP/s":
-            ur["frac_of_sustained"] = ur["achieved"] / pk["bf16_tflops_sustained"]
         sc_pairs = sc_users * sc_per
         sc_bytes = sc_pairs * (w.H * w.l * (2 if w.dtype == "bf16" else 4) + 4 +
                                w.d * (2 if w.dtype == "bf16" else 4))
@@ -577,7 +695,9 @@ def main():
                          "roofline": phase_roof("cache")},
             "score": {"ms": phase_ms["score"],
                       "pairs_per_s": total_cand / (phase_ms["score"] * 1e-3),
-                      "roofline": phase_roof("score")},
+                      "roofline": phase_roof("score"),
+                      "distinct_row_gbs": distinct_row_bytes(w, x.cand_ids, total_cand) /
+                      (phase_ms["score"] * 1e-3) / 1e9},
             "score_at_scale": {"ms": sc_ms, "pairs": sc_pairs,
                                "pairs_per_s": sc_pairs / (sc_ms * 1e-3),
                                "ids": f"uniform over {w.n_items} items, L2 flushed before each call",
@@ -630,7 +750,7 @@ def main():
                 "config": dict(config_of(w, total_cand, total_hist),
                                launch="eager library calls" if args.eager else
                                "CUDA graph replay of the step's captured library launches"),
-                "phases": phases, "roofline": roof,
+                "phases": phases, "configs": cfg, "roofline": roof,
                 "clocks": sampler.summary(),
                 "e2e": {"value": job_throughput(world, total_cand, e2e_step_ms), "unit": "pairs/s",
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

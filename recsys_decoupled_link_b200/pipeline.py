@@ -78,6 +78,18 @@ def to_device(w: synth.Workload, us: synth.UserSide, cs: synth.CandidateSide,
         cand_offsets=dev(cs.cand_offsets), total_cand=int(cs.cand_offsets[-1]))
 
 
+def item_table_device(w: synth.Workload, device="cuda") -> torch.Tensor:
+    """The item table T [n_items, d] on the device, copied block by block from
+    the seeded host blocks (host memory stays at one block)."""
+    T = torch.empty(w.n_items, w.d, dtype=synth.torch_dtype(w), device=device)
+    nb = (w.n_items + synth.BLOCK_ROWS - 1) // synth.BLOCK_ROWS
+    for b in range(nb):
+        r0 = b * synth.BLOCK_ROWS
+        blk = synth.item_block(w, b)
+        T[r0:r0 + blk.shape[0]].copy_(blk)
+    return T
+
+
 def alloc(x: DeviceInputs, n_items: Optional[int] = None, device="cuda") -> Buffers:
     w = x.w
     dt = synth.torch_dtype(w)

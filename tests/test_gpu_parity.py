@@ -259,13 +259,7 @@ def test_full_size_sampled(case):
     cs = synth.candidate_side(w)
     x = pipeline.to_device(w, us, cs, None)
     # item table straight to the device block by block (keeps host memory low)
-    dt = synth.torch_dtype(w)
-    x.T = torch.empty(w.n_items, w.d, dtype=dt, device="cuda")
-    nb = (w.n_items + synth.BLOCK_ROWS - 1) // synth.BLOCK_ROWS
-    for b in range(nb):
-        r0 = b * synth.BLOCK_ROWS
-        blk = synth.item_block(w, b)
-        x.T[r0:r0 + blk.shape[0]].copy_(blk)
+    x.T = pipeline.item_table_device(w)
     buf = pipeline.alloc(x)
     LP = pipeline.user_encode(x, buf)
     pipeline.build_cache(x, buf)

@@ -328,7 +328,7 @@ def time_config(name, flush, stream, pk, T_cache):
         raise RuntimeError(f"device status flags set during the {name} steps")
     work = work_units(w, x.total_hist, x.total_cand)
     med = statistics.median
-    fast_layers = w.dtype == "bf16" and w.d == 128 and w.H == 4 and w.l in (16, 32)
+    fast_layers = w.dtype == "bf16" and w.d == 128 and w.H == 4 and w.l in (16, 32, 64)
     out = {
         "workload": config_of(w, x.total_cand, x.total_hist)["workload"],
         "history_tokens": x.total_hist, "pairs": x.total_cand, "runs": runs,

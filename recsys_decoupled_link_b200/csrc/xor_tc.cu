@@ -1,5 +1,5 @@
 // One LIME-XOR layer on the 5th-generation tensor cores (bf16 storage,
-// d = 128, 4 heads of 32, l in {16, 32}, GatedMLP width 256).
+// d = 128, 4 heads of 32, l in {16, 32, 64}, GatedMLP width 256).
 //
 // LIME note, 关键设计 2: over X = [E; Z] the XOR mask keeps only history<->link
 // attention, XORA(X,X,X) = MHA(E, Z, Z) ⊕ MHA(Z, E, E), at O(l·N) cost; the
@@ -61,14 +61,16 @@ struct LayerWs {
   size_t yd, uimg, part;
   size_t total;
   int64_t max_tiles;
-  uint32_t uimg_bytes;
+  uint32_t uimg_bytes;   // per user: nhalf half images
+  uint32_t half_bytes;   // one half image (128 (head, link) rows)
 };
 
 __host__ __device__ constexpr size_t up1k(size_t x) { return (x + 1023) & ~(size_t)1023; }
 
-// per-user folded images: G'^T, Q'g, VO ([128 x 128] bf16 each), then the
-// fp32 vectors cQ, dQ, cG, dG ([128] each); with phi = SiLU also the low half
-// of G' (G' = hi + lo)
+// per-user folded images, in halves of 128 (head, link) rows (one half for
+// l <= 32, two for l = 64: half i holds heads 2i and 2i+1): G'^T, Q'g, VO
+// ([128 x 128] bf16 each), then the fp32 vectors cQ, dQ, cG, dG ([128] each);
+// with phi = SiLU also the low half of G' (G' = hi + lo)
 constexpr uint32_t kUimgVec = 6 * kBlk;
 constexpr uint32_t kUimgBytes = 6 * kBlk + 4 * 128 * 4;
 constexpr uint32_t kUimgGlo = kUimgBytes;
@@ -89,7 +91,8 @@ LayerWs layer_ws(int l, int64_t B, int64_t nh, bool silu) {
   w.tiles = take((size_t)w.max_tiles * 16);
   w.tile_start = take((size_t)(B + 1) * 4);
   w.yd = take((size_t)nh * kD * 2);   // attention delta (fp16)
-  w.uimg_bytes = kUimgBytes + (silu ? 2 * kBlk : 0);
+  w.half_bytes = kUimgBytes + (silu ? 2 * kBlk : 0);
+  w.uimg_bytes = (uint32_t)((kH * l + 127) / 128) * w.half_bytes;
   w.uimg = take((size_t)B * w.uimg_bytes);
   w.part = take((size_t)w.max_tiles * kH * l * kRec * 4);
   w.total = o;
@@ -546,11 +549,12 @@ __global__ void __launch_bounds__(512, 1)
       red[512 + part * 128 + r] = ds;
       __syncthreads();
       if (part == 0 && valid) {
-        float* vec = reinterpret_cast<float*>(ws + Lw.uimg + (size_t)(R / L) * Lw.uimg_bytes + kUimgVec) +
+        const int p = h * L + (int)(R % L);   // row p & 127 of half p >> 7
+        float* vec = reinterpret_cast<float*>(ws + Lw.uimg + (size_t)(R / L) * Lw.uimg_bytes +
+                                              (size_t)(p >> 7) * Lw.half_bytes + kUimgVec) +
                      (which == 0 ? 0 : 2 * 128);
-        const int p = h * L + (int)(R % L);
-        vec[p] = red[r] + red[128 + r] + red[256 + r] + red[384 + r];
-        vec[128 + p] = red[512 + r] + red[640 + r] + red[768 + r] + red[896 + r];
+        vec[p & 127] = red[r] + red[128 + r] + red[256 + r] + red[384 + r];
+        vec[128 + (p & 127)] = red[512 + r] + red[640 + r] + red[768 + r] + red[896 + r];
       }
       __syncthreads();
     }
@@ -562,8 +566,10 @@ __global__ void __launch_bounds__(512, 1)
     for (int i = 0; i < hpc * (split ? 2 : 1); ++i) {
       const int h = h0 + (split ? i >> 1 : i);
       const uint32_t off = split && (i & 1) ? kUimgGlo : img_off;
+      const int p0 = h * L;   // the head's first image row: row p0 & 127 of half p0 >> 7
       for (int j = 0; j < n_users; ++j) {
-        uint8_t* dst = ws + Lw.uimg + (size_t)(u0 + j) * Lw.uimg_bytes + off + h * L * 128;
+        uint8_t* dst = ws + Lw.uimg + (size_t)(u0 + j) * Lw.uimg_bytes +
+                       (size_t)(p0 >> 7) * Lw.half_bytes + off + (p0 & 127) * 128;
         const uint8_t* src = sm + i * 2 * kBlk + j * L * 128;
         bulk_store(dst, src, L * 128);
         bulk_store(dst + kBlk, src + kBlk, L * 128);
@@ -624,6 +630,13 @@ __global__ void __launch_bounds__(kXaThreads, 1)
     k_hist_xattn(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
                  uint8_t* __restrict__ ws, LayerWs Lw, unsigned* status) {
   constexpr int HL = kH * L;
+  constexpr int NH = (HL + 127) / 128;        // halves of the (head, link) pairs
+  constexpr int HLH = HL < 128 ? HL : 128;    // pairs per half
+  constexpr bool SPLIT = NH > 1;
+  // TMEM columns: one half -> [0,128) S, then Yd; S' at [128,256) / [384,512)
+  // by tile parity; V_E [256,384).  Two halves -> [0,128) S, [128,256) S',
+  // [256,384) V_E, [384,512) Yd, accumulated over the tile's two halves.
+  constexpr uint32_t kYd = SPLIT ? 384 : 0;
   constexpr uint32_t kSlot = 2 * kBlk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
@@ -638,9 +651,10 @@ __global__ void __launch_bounds__(kXaThreads, 1)
   float* vecs = cvd + 256;                                  // 2 x (cQ, dQ, cG, dG)
   uint8_t* sGl = reinterpret_cast<uint8_t*>(vecs + 1024);   // a 64-column block of G'lo
   Cta c;
-  // bar: 0 weights, 1 S' done, 2 E tile, 3 G', 4 Q'g + vec, 6 VO, 7 V_E done,
-  //      8 S done, 9 P2 V_E done, 10 Yd done, 11 TMEM read out, 12 P2 and V_E
-  //      written, 13 P written, 14 G'lo block landed, 15 its product done
+  // bar: 0 weights, 1 S' done, 2 E tile, 3 G', 4 Q'g + vec, 5 records read
+  //      out (two halves), 6 VO, 7 V_E done, 8 S done, 9 P2 V_E done, 10 Yd
+  //      done, 11 Yd read out, 12 P2 and V_E written, 13 P written, 14 G'lo
+  //      block landed, 15 its product done
   cta_setup(sGl + kBlk, 16, c);
   uint64_t* bar = c.bar;
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
@@ -649,15 +663,17 @@ __global__ void __launch_bounds__(kXaThreads, 1)
   if (warp == kXaEpi / 32) {
     if ((threadIdx.x & 31) == 0) {
       // ---- the issuer: loads and MMAs
-      auto uimg = [&](int u) { return ws + Lw.uimg + (size_t)u * Lw.uimg_bytes; };
+      auto uimg = [&](int u, int hf) {   // half hf of user u's images
+        return ws + Lw.uimg + (size_t)u * Lw.uimg_bytes + (size_t)hf * Lw.half_bytes;
+      };
       auto load = [&](uint64_t* b, uint8_t* dst, const uint8_t* src) {
         mbar_arrive_expect_tx(b, kSlot);
         bulk_load(dst, src, kSlot, b);
       };
-      auto load_q = [&](int u, int it) {   // Q'g and the user's vectors
+      auto load_q = [&](int u, int hf, int it) {   // Q'g and the half's vectors
         mbar_arrive_expect_tx(&bar[4], kSlot + 2048);
-        bulk_load(sQ, uimg(u) + 2 * kBlk, kSlot, &bar[4]);
-        bulk_load(vecs + (it & 1) * 512, uimg(u) + kUimgVec, 2048, &bar[4]);
+        bulk_load(sQ, uimg(u, hf) + 2 * kBlk, kSlot, &bar[4]);
+        bulk_load(vecs + (it & 1) * 512, uimg(u, hf) + kUimgVec, 2048, &bar[4]);
       };
       auto load_e = [&](uint8_t* dst, int r0) {
         mbar_arrive_expect_tx(&bar[2], kSlot);
@@ -671,23 +687,28 @@ __global__ void __launch_bounds__(kXaThreads, 1)
       if ((int)blockIdx.x < n_tiles) {
         const int4 tl = tiles[blockIdx.x];
         load_e(rot, tl.y);
-        if (HIST) load(&bar[3], sG, uimg(tl.x));
-        load_q(tl.x, 0);
+        if (HIST) load(&bar[3], sG, uimg(tl.x, 0));
+        load_q(tl.x, 0, 0);
       } else {
         mbar_wait(&bar[0], 0, status, c.abort_flag);   // lands before the CTA exits
       }
-      int ab = 0;
-      for (int t = blockIdx.x, it = 0; t < n_tiles; t += gridDim.x, ++it) {
+      // virtual tiles (tile t, half hf), the halves of a tile back to back;
+      // kt counts this CTA's tiles
+      int ab = 0, t = blockIdx.x, hf = 0, kt = 0;
+      for (int it = 0; t < n_tiles; ++it) {
         const int u = tiles[t].x;
-        const int tn = t + gridDim.x;
+        const int tn = hf + 1 < NH ? t : t + (int)gridDim.x;   // the next virtual tile
+        const int hn = hf + 1 < NH ? hf + 1 : 0;
         const int un = tn < n_tiles ? tiles[tn].x : 0;
         const uint32_t ph = (uint32_t)it & 1u;
         uint8_t* sA = rot + ab * kSlot;
         uint8_t* sB = rot + (ab ^ 1) * kSlot;
-        const uint32_t tS2 = c.tmem + 128 + (uint32_t)(it & 1) * 256;
+        const uint32_t tS2 = c.tmem + 128 + (SPLIT ? 0u : (uint32_t)(it & 1) * 256);
         mbar_wait(&bar[2], ph, status, c.abort_flag);
         if (it == 0) mbar_wait(&bar[0], 0, status, c.abort_flag);
         mbar_wait(&bar[4], ph, status, c.abort_flag);
+        // one S' buffer: the previous records must have been read out
+        if (SPLIT && it > 0) mbar_wait(&bar[5], ph ^ 1u, status, c.abort_flag);
         tc_fence_after();
         mma_tile(tS2, smem_u32(sQ), kBlk, smem_u32(sA), kBlk, 128, 128, false);
         mma_commit(&bar[1]);
@@ -696,20 +717,20 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         mma_commit(&bar[7]);
         if (HIST) {
           // S overwrites the previous tile's Yd columns: wait for their readout
-          if (it > 0) mbar_wait(&bar[11], ph ^ 1u, status, c.abort_flag);
+          if (!SPLIT && it > 0) mbar_wait(&bar[11], ph ^ 1u, status, c.abort_flag);
           mbar_wait(&bar[3], ph, status, c.abort_flag);
           tc_fence_after();
-          mma_tile(c.tmem, smem_u32(sA), kBlk, smem_u32(sG), kBlk, HL, 128, false);
+          mma_tile(c.tmem, smem_u32(sA), kBlk, smem_u32(sG), kBlk, HLH, 128, false);
           if constexpr (SILU) {
             // + E G'lo, one 64-column block at a time through sGl
             for (int j = 0; j < 2; ++j) {
               const uint32_t pj = (uint32_t)(2 * it + j) & 1u;
               if (j > 0) mbar_wait(&bar[15], pj ^ 1u, status, c.abort_flag);
               mbar_arrive_expect_tx(&bar[14], kBlk);
-              bulk_load(sGl, uimg(u) + kUimgGlo + j * kBlk, kBlk, &bar[14]);
+              bulk_load(sGl, uimg(u, hf) + kUimgGlo + j * kBlk, kBlk, &bar[14]);
               mbar_wait(&bar[14], pj, status, c.abort_flag);
               tc_fence_after();
-              mma_tile(c.tmem, smem_u32(sA + j * kBlk), kBlk, smem_u32(sGl), kBlk, HL, 64, true);
+              mma_tile(c.tmem, smem_u32(sA + j * kBlk), kBlk, smem_u32(sGl), kBlk, HLH, 64, true);
               mma_commit(&bar[15]);
             }
             mbar_wait(&bar[15], 1u, status, c.abort_flag);   // the block's buffer is free
@@ -718,8 +739,8 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         }
         // the link scores have read Q'g
         mbar_wait(&bar[1], ph, status, c.abort_flag);
-        if (HIST) load(&bar[6], sQ, uimg(u) + 4 * kBlk);
-        else if (tn < n_tiles) load_q(un, it + 1);
+        if (HIST) load(&bar[6], sQ, uimg(u, hf) + 4 * kBlk);
+        else if (tn < n_tiles) load_q(un, hn, it + 1);
         mbar_wait(&bar[12], ph, status, c.abort_flag);
         tc_fence_after();
         mma_tile_bmn(tS2, smem_u32(sB), kBlk, smem_u32(sG), kBlk, 128, 128, false);
@@ -728,19 +749,28 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         mbar_wait(&bar[9], ph, status, c.abort_flag);
         if (tn < n_tiles) {
           load_e(sB, tiles[tn].y);
-          if (HIST) load(&bar[3], sG, uimg(un));
+          if (HIST) load(&bar[3], sG, uimg(un, hn));
         }
         if (HIST) {
           mbar_wait(&bar[13], ph, status, c.abort_flag);
           mbar_wait(&bar[6], ph, status, c.abort_flag);
+          // two halves: the first half's product starts the tile's Yd, so the
+          // previous tile's Yd must have been read out
+          if (SPLIT && hf == 0 && kt > 0)
+            mbar_wait(&bar[11], (uint32_t)(kt - 1) & 1u, status, c.abort_flag);
           tc_fence_after();
-          mma_tile_bmn(c.tmem, smem_u32(sA), kBlk, smem_u32(sQ), kBlk, 128, HL, false);
+          mma_tile_bmn(c.tmem + kYd, smem_u32(sA), kBlk, smem_u32(sQ), kBlk, 128, HLH, hf > 0);
           mma_commit(&bar[10]);
           // Yd has read P and VO: the next Q'g
           mbar_wait(&bar[10], ph, status, c.abort_flag);
-          if (tn < n_tiles) load_q(un, it + 1);
+          if (tn < n_tiles) load_q(un, hn, it + 1);
         }
         ab ^= 1;
+        if (++hf == NH) {
+          hf = 0;
+          t += gridDim.x;
+          ++kt;
+        }
       }
     }
   } else {
@@ -752,14 +782,15 @@ __global__ void __launch_bounds__(kXaThreads, 1)
     bf16* yd = reinterpret_cast<bf16*>(ws + Lw.yd);   // fp16 bits; rows copied as bytes
     float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
     if (HIST && threadIdx.x == 0) prefetch_tmap(&tmY);
-    int ab = 0;
-    for (int t = blockIdx.x, it = 0; t < n_tiles; t += gridDim.x, ++it) {
+    int ab = 0, t = blockIdx.x, hf = 0;
+    for (int it = 0; t < n_tiles; ++it) {
       const int4 tl = tiles[t];
       const int r0 = tl.y, nv = tl.z;
       const uint32_t ph = (uint32_t)it & 1u;
       uint8_t* sA = rot + ab * kSlot;
       uint8_t* sB = rot + (ab ^ 1) * kSlot;
-      const uint32_t tS2 = ta + 128 + (uint32_t)(it & 1) * 256;
+      const uint32_t tS2 = ta + 128 + (SPLIT ? 0u : (uint32_t)(it & 1) * 256);
+      const int pr = hf * 128 + row;   // this lane's (head, link) pair in the link branch
       const float* vec = vecs + (it & 1) * 512;   // cQ, dQ, cG, dG
       mbar_wait(&bar[2], ph, status, c.abort_flag);
       if (it == 0) mbar_wait(&bar[0], 0, status, c.abort_flag);
@@ -790,15 +821,15 @@ __global__ void __launch_bounds__(kXaThreads, 1)
       }
       mbar_wait(&bar[1], ph, status, c.abort_flag);
       tc_fence_after();
-      // link softmax over the tile's valid rows: row = (head, link) lane,
-      // part = a quarter of the tokens.  Lanes >= H*L carry no link.
+      // link softmax over the tile's valid rows: row = (head, link) lane of
+      // the half, part = a quarter of the tokens.  Pairs >= H*L carry no link.
       float lm, ls;
       {
         float z[32];
         tmem_ld16(tS2 + c0, z);
         tmem_ld16(tS2 + c0 + 16, z + 16);
         tmem_ld_wait();
-        const bool link = row < HL;
+        const bool link = pr < HL;
         const float cq = link ? vec[row] : 0.f, dq = link ? vec[128 + row] : 0.f;
         const float4* mu4 = reinterpret_cast<const float4*>(smu + c0);
         const float4* rs4 = reinterpret_cast<const float4*>(smu + 128 + c0);
@@ -862,7 +893,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
       tc_fence_before();
       named_bar_sync(1, kXaEpi);
       if (threadIdx.x == 0) mbar_arrive(&bar[12]);   // P2 V_E can start
-      if (HIST) {
+      if constexpr (HIST && !SPLIT) {
         // history softmax over the user's L links: part = head, P over the E tile
         const int h = part;
         float z[L];
@@ -888,6 +919,41 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         }
 #pragma unroll
         for (int q = 0; q < L / 8; ++q) sw_st16(sA, kBlk, row, h * L + q * 8, pack8(z + q * 8));
+      }
+      if constexpr (HIST && SPLIT) {
+        // two halves: the half's 128 score columns are heads 2hf and 2hf+1
+        // with L = 64 links each; part p holds 32 links of head 2hf + p/2, and
+        // the parts p, p^1 of a head combine their max and sum
+        float z[32];
+        tmem_ld16(ta + c0, z);
+        tmem_ld16(ta + c0 + 16, z + 16);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          z[k] = fmaf(rs_r, fmaf(-mu_r, vec[256 + c0 + k], z[k]), vec[384 + c0 + k]);
+        if constexpr (SILU) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) z[k] = silu_fast(z[k]) * (1.0f / L);
+        } else {
+          float m = z[0];
+#pragma unroll
+          for (int k = 1; k < 32; ++k) m = fmaxf(m, z[k]);
+          red[part * 128 + row] = m;
+          named_bar_sync(1, kXaEpi);
+          m = fmaxf(m, red[(part ^ 1) * 128 + row]);
+          float s = 0.f;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
+          red[512 + part * 128 + row] = s;
+          named_bar_sync(1, kXaEpi);
+          const float inv = 1.0f / (s + red[512 + (part ^ 1) * 128 + row]);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) z[k] *= inv;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sw_st16(sA, kBlk, row, c0 + q * 8, pack8(z + q * 8));
+      }
+      if (HIST) {
         fence_proxy_async_smem();
         tc_fence_before();
         named_bar_sync(1, kXaEpi);
@@ -902,20 +968,27 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         tmem_ld16(tS2 + part * kDH, acc);
         tmem_ld16(tS2 + part * kDH + 16, acc + 16);
         tmem_ld_wait();
-        if (row < HL && row / L == part) {
-          float4* rec = reinterpret_cast<float4*>(part_rec + ((size_t)t * HL + row) * kRec);
+        if (pr < HL && pr / L == part) {
+          float4* rec = reinterpret_cast<float4*>(part_rec + ((size_t)t * HL + pr) * kRec);
           rec[0] = make_float4(lm, ls, 0.f, 0.f);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             rec[1 + q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
         }
+        if constexpr (SPLIT) {
+          // the next half's link scores reuse these columns
+          tc_fence_before();
+          named_bar_sync(1, kXaEpi);
+          if (threadIdx.x == 0) mbar_arrive(&bar[5]);
+        }
       }
-      if (HIST) {
-        mbar_wait(&bar[10], ph, status, c.abort_flag);
+      if (HIST) mbar_wait(&bar[10], ph, status, c.abort_flag);   // P has been read
+      if (HIST && hf == NH - 1) {
+        // the tile's Yd (two halves: accumulated over both)
         tc_fence_after();
         float y[32];
-        tmem_ld16(ta + c0, y);
-        tmem_ld16(ta + c0 + 16, y + 16);
+        tmem_ld16(ta + kYd + c0, y);
+        tmem_ld16(ta + kYd + c0 + 16, y + 16);
         tmem_ld_wait();
         tc_fence_before();
         named_bar_sync(1, kXaEpi);   // every thread has read P (the MMA is done) and Yd
@@ -938,6 +1011,10 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         }
       }
       ab ^= 1;
+      if (++hf == NH) {
+        hf = 0;
+        t += gridDim.x;
+      }
     }
     if (threadIdx.x == 0) bulk_wait<0>();
   }
@@ -1571,8 +1648,8 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
 }  // namespace
 
 bool fast_layer_supported(const lime_dims& D) {
-  return D.dtype == LIME_BF16 && D.d == kD && D.H == kH && D.f == kF && (D.l == 16 || D.l == 32) &&
-         D.window == 0;
+  return D.dtype == LIME_BF16 && D.d == kD && D.H == kH && D.f == kF &&
+         (D.l == 16 || D.l == 32 || D.l == 64) && D.window == 0;
 }
 
 size_t fast_layer_ws_bytes(const lime_dims& D, int64_t B, int64_t total_hist) {
@@ -1585,6 +1662,7 @@ int fast_xor_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh
                    void* Z_out, float* ws, unsigned* status, cudaStream_t st) {
   uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
   if (D.l == 16) return run_layer<16>(D, B, off, nh, E_in, Z_in, w, E_out, Z_out, wsb, status, st);
+  if (D.l == 64) return run_layer<64>(D, B, off, nh, E_in, Z_in, w, E_out, Z_out, wsb, status, st);
   return run_layer<32>(D, B, off, nh, E_in, Z_in, w, E_out, Z_out, wsb, status, st);
 }
 

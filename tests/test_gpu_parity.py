@@ -105,14 +105,15 @@ def test_workload_parity(case):
     check_workload(synth.workload(base, **SMALL[case]))
 
 
-@pytest.mark.parametrize("base", ["tiny", "standard"])
-def test_edge_cases(base):
+@pytest.mark.parametrize("base,l", [("tiny", 32), ("standard", 32), ("standard", 64)])
+def test_edge_cases(base, l):
     # empty histories, one-row history, exact tiles and ragged tails; users with
-    # no candidates; the batch starts and ends with edge users
+    # no candidates; the batch starts and ends with edge users (l = 64: the
+    # layer's two halves of (head, link) pairs per history tile)
     n_hist = [0, 1, 127, 128, 129, 300, 0]
     n_cand = [5, 0, 1, 130, 7, 0, 3]
     w = synth.workload(base, B=len(n_hist), n_items=5000,
-                       cand=("uniform",), layers=2)
+                       cand=("uniform",), layers=2, l=l)
     check_workload(w, n_hist=n_hist, n_cand=n_cand)
 
 

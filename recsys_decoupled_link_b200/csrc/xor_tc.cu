@@ -40,6 +40,8 @@
 // the row's columns) or warp-specialized roles; one thread issues the MMAs.
 // Every kernel is launched with programmatic dependent launch (pdl_launch /
 // pdl_wait).  Every wait is bounded and sets LIME_FLAG_TIMEOUT.
+#include <type_traits>
+
 #include "lime_fast.cuh"
 #include "sm100.cuh"
 
@@ -177,6 +179,17 @@ __device__ __forceinline__ float tanh_approx(float x) {
 __device__ __forceinline__ float silu_tanh(float x) {
   const float h = 0.5f * x;
   return fmaf(h, tanh_approx(h), h);
+}
+
+// 2^x with the hardware approximation (ex2.approx: relative error about
+// 2^-22; -inf -> +0).  The softmax kernels keep their scores in log2 units
+// (scaled by log2 e in the folded constants), so e^(z - m) is one ex2.
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // fp32 [rows x 128] staging: row r is 512 bytes, its 16-byte chunk c sits at
@@ -397,7 +410,8 @@ __device__ void schedule_tiles(const int64_t* __restrict__ off, int64_t B, int64
 //   Q'g  [2, 4 kBlk)   Q'g[p, i] = g1[i] (s Q_Z[k, h] Wk[:, h]^T)[i]
 //   VO   [4, 6 kBlk)   VO[p] = V_Z[k, h] Wo[h, :]                     (Wo's rows of head h)
 //   vec  cQ, dQ, cG, dG [128] each: c[p] = sum_i of the stored row p of Q'g
-//        (G'), d[p] = sum_i b1[i] of the unscaled row
+//        (G'), d[p] = sum_i b1[i] of the unscaled row (times log2 e for phi =
+//        softmax: the history kernel's scores are in log2 units)
 // By associativity the history scores are Q_E,h (s K_Z,h)^T = X^ G_h, the
 // link scores (s Q_Z,h) K_E,h^T = Q'_h X^^T and the history branch through
 // Wo is (P_h V_Z,h) Wo_h = P_h VO_h.  With X^ = LN1(E) = rstd (E - mu) g1 + b1
@@ -553,8 +567,10 @@ __global__ void __launch_bounds__(512, 1)
         float* vec = reinterpret_cast<float*>(ws + Lw.uimg + (size_t)(R / L) * Lw.uimg_bytes +
                                               (size_t)(p >> 7) * Lw.half_bytes + kUimgVec) +
                      (which == 0 ? 0 : 2 * 128);
+        // softmax: d in log2 units (the history kernel scales rstd alike)
         vec[p & 127] = red[r] + red[128 + r] + red[256 + r] + red[384 + r];
-        vec[128 + (p & 127)] = red[512 + r] + red[640 + r] + red[768 + r] + red[896 + r];
+        vec[128 + (p & 127)] = (red[512 + r] + red[640 + r] + red[768 + r] + red[896 + r]) *
+                               (silu ? 1.0f : kLog2e);
       }
       __syncthreads();
     }
@@ -815,7 +831,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         rs_r = rsqrtf(fmaxf(ex2 - mu_r * mu_r, 0.f) + kLnEps);
         if (part == 0) {
           smu[row] = mu_r;
-          smu[128 + row] = rs_r;
+          smu[128 + row] = SILU ? rs_r : rs_r * kLog2e;   // softmax: log2 units
         }
         named_bar_sync(1, kXaEpi);
       }
@@ -829,23 +845,35 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         tmem_ld16(tS2 + c0, z);
         tmem_ld16(tS2 + c0 + 16, z + 16);
         tmem_ld_wait();
-        const bool link = pr < HL;
+        // all pairs of a half are links once H*L fills it; masking is only
+        // needed for a tile's invalid rows (a partial tile) or missing links
+        constexpr bool kAllLinks = HL % 128 == 0;
+        const bool link = kAllLinks || pr < HL;
+        const bool full = nv == kTile && kAllLinks;
         const float cq = link ? vec[row] : 0.f, dq = link ? vec[128 + row] : 0.f;
         const float4* mu4 = reinterpret_cast<const float4*>(smu + c0);
         const float4* rs4 = reinterpret_cast<const float4*>(smu + 128 + c0);
         float m = -INFINITY;
+        auto scores = [&](auto masked) {
 #pragma unroll
-        for (int j4 = 0; j4 < 8; ++j4) {
-          const float4 mv = mu4[j4], rv = rs4[j4];
-          const float mj[4] = {mv.x, mv.y, mv.z, mv.w}, rj[4] = {rv.x, rv.y, rv.z, rv.w};
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 mv = mu4[j4], rv = rs4[j4];
+            const float mj[4] = {mv.x, mv.y, mv.z, mv.w}, rj[4] = {rv.x, rv.y, rv.z, rv.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = j4 * 4 + e;
-            z[j] = fmaf(rj[e], fmaf(-mj[e], cq, z[j]), dq);
-            if (c0 + j >= nv || !link) z[j] = -INFINITY;
-            m = fmaxf(m, z[j]);
+            for (int e = 0; e < 4; ++e) {
+              const int j = j4 * 4 + e;
+              z[j] = fmaf(rj[e], fmaf(-mj[e], cq, z[j]), dq);
+              if constexpr (decltype(masked)::value) {
+                if (c0 + j >= nv || !link) z[j] = -INFINITY;
+              }
+              m = fmaxf(m, z[j]);
+            }
           }
-        }
+        };
+        if (full)
+          scores(std::false_type{});
+        else
+          scores(std::true_type{});
         if constexpr (SILU) {
           // pointwise weights: SiLU of each valid score; the record's (max,
           // sum) = (0, valid tokens) makes the merge's total divide by N_u
@@ -861,15 +889,18 @@ __global__ void __launch_bounds__(kXaThreads, 1)
           if (HIST && it > 0 && threadIdx.x == 0) bulk_wait_read<0>();
           named_bar_sync(1, kXaEpi);
           m = fmaxf(fmaxf(red[row], red[128 + row]), fmaxf(red[256 + row], red[384 + row]));
+          // masked scores are -inf and give 0; a lane with no link at all
+          // has m = -inf and takes m = 0 instead
+          if (m == -INFINITY) m = 0.f;
           float s = 0.f;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            z[j] = c0 + j < nv && link ? __expf(z[j] - m) : 0.f;
+            z[j] = ex2_approx(z[j] - m);
             s += z[j];
           }
           red[512 + part * 128 + row] = s;
           named_bar_sync(1, kXaEpi);
-          lm = m;
+          lm = m * kLn2;   // the record's max in natural-log units
           ls = red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row];
         }
 #pragma unroll
@@ -900,9 +931,10 @@ __global__ void __launch_bounds__(kXaThreads, 1)
 #pragma unroll
         for (int q = 0; q < L / 16; ++q) tmem_ld16(ta + h * L + q * 16, z + q * 16);
         tmem_ld_wait();
+        const float rsl = SILU ? rs_r : rs_r * kLog2e;   // softmax: log2 units
 #pragma unroll
         for (int k = 0; k < L; ++k)
-          z[k] = fmaf(rs_r, fmaf(-mu_r, vec[256 + h * L + k], z[k]), vec[384 + h * L + k]);
+          z[k] = fmaf(rsl, fmaf(-mu_r, vec[256 + h * L + k], z[k]), vec[384 + h * L + k]);
         if constexpr (SILU) {
 #pragma unroll
           for (int k = 0; k < L; ++k) z[k] = silu_fast(z[k]) * (1.0f / L);
@@ -912,7 +944,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
           for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
           float s = 0.f;
 #pragma unroll
-          for (int k = 0; k < L; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
+          for (int k = 0; k < L; ++k) { z[k] = ex2_approx(z[k] - m); s += z[k]; }
           const float inv = 1.0f / s;
 #pragma unroll
           for (int k = 0; k < L; ++k) z[k] *= inv;
@@ -928,9 +960,10 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         tmem_ld16(ta + c0, z);
         tmem_ld16(ta + c0 + 16, z + 16);
         tmem_ld_wait();
+        const float rsl = SILU ? rs_r : rs_r * kLog2e;   // softmax: log2 units
 #pragma unroll
         for (int k = 0; k < 32; ++k)
-          z[k] = fmaf(rs_r, fmaf(-mu_r, vec[256 + c0 + k], z[k]), vec[384 + c0 + k]);
+          z[k] = fmaf(rsl, fmaf(-mu_r, vec[256 + c0 + k], z[k]), vec[384 + c0 + k]);
         if constexpr (SILU) {
 #pragma unroll
           for (int k = 0; k < 32; ++k) z[k] = silu_fast(z[k]) * (1.0f / L);
@@ -943,7 +976,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
           m = fmaxf(m, red[(part ^ 1) * 128 + row]);
           float s = 0.f;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) { z[k] = __expf(z[k] - m); s += z[k]; }
+          for (int k = 0; k < 32; ++k) { z[k] = ex2_approx(z[k] - m); s += z[k]; }
           red[512 + part * 128 + row] = s;
           named_bar_sync(1, kXaEpi);
           const float inv = 1.0f / (s + red[512 + (part ^ 1) * 128 + row]);
@@ -1285,13 +1318,13 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
       // E' = OUT -> bf16, staged in the hid buffers (every W2 product of the
       // tile is done, and the next hid is written by these threads after the
       // copy) and written with coalesced 16-byte stores
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float o[16];
-        tmem_ld16(ta + T_OUT + (k & 1) * 128 + c0 + hf * 16, o);
+      {
+        float o[32];
+        tmem_ld16(ta + T_OUT + (k & 1) * 128 + c0, o);
+        tmem_ld16(ta + T_OUT + (k & 1) * 128 + c0 + 16, o + 16);
         tmem_ld_wait();
-        sw_st16(sH0, kBlk, row, c0 + hf * 16, pack8(o));
-        sw_st16(sH0, kBlk, row, c0 + hf * 16 + 8, pack8(o + 8));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sw_st16(sH0, kBlk, row, c0 + q * 8, pack8(o + q * 8));
       }
       tc_fence_before();
       named_bar_sync(1, kFfnEpi);

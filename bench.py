@@ -491,40 +491,39 @@ def main():
         ph["score"] += e[2].elapsed_time(e[3])
     ph = dict(zip(ph, max_over_ranks(list(ph.values()), dist, "cuda")))
 
-    # end to end through the public API: the step's per-request inputs (the users'
-    # histories, context features and candidate IDs with their offsets) copied
-    # in from pinned host memory and the scores copied back; the model state
-    # (weights, global links and the item table the cache is built from) stays
-    # resident, as it would in a serving process
-    host = {"E": x.E.cpu().pin_memory(), "ctx": x.ctx.cpu().pin_memory() if x.ctx is not None else None,
-            "hist_offsets": x.hist_offsets.cpu().pin_memory(),
-            "cand_ids": x.cand_ids.cpu().pin_memory(),
-            "cand_offsets": x.cand_offsets.cpu().pin_memory()}
+    # end to end through the public API: every step's per-request inputs (the
+    # users' histories, context features and candidate IDs with their offsets)
+    # copied in from pinned host memory and its scores copied back, with the
+    # model state (weights, global links and the item table the cache is built
+    # from) resident, as in a serving process.  pipeline.HostPipeline runs the
+    # steps over two request slots, so step k's copies overlap the compute of
+    # its neighbours; the timed region spans the first step's input copy to
+    # the last step's score copy.  No L2 flush between steps: every step
+    # streams the 256 MB item table and writes the 256 MB cache, which turns
+    # the 126 MB L2 over by itself.
+    host = {k: (None if getattr(x, k) is None else getattr(x, k).cpu().pin_memory())
+            for k in pipeline.REQUEST_FIELDS}
     h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
-    O_host = torch.empty(buf.O.shape, dtype=buf.O.dtype).pin_memory()
-    d2h = O_host.numel() * O_host.element_size()
-    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-
-    def e2e_step():
-        for k, t in host.items():
-            if t is not None:
-                getattr(x, k).copy_(t, non_blocking=True)
-        out = pipeline.step(x, buf)
-        O_host.copy_(out, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
+    O_hosts = [torch.empty(buf.O.shape, dtype=buf.O.dtype).pin_memory() for _ in range(2)]
+    d2h = O_hosts[0].numel() * O_hosts[0].element_size()
+    hp = pipeline.HostPipeline(x, buf)
+    for k in range(4):
+        hp.submit(host, O_hosts[k % 2])
+    hp.drain()
     torch.cuda.synchronize()
+    e2e_match = all(torch.equal(o, buf.O.cpu()) for o in O_hosts)
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     if dist:
         dist.barrier()
-    for k in range(args.steps):
-        flush.zero_()
-        ee[k][0].record(stream)
-        e2e_step()
-        ee[k][1].record(stream)
     torch.cuda.synchronize()
-    e2e_step_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in ee)], dist,
-                                 "cuda")[0] / args.steps
+    ee[0].record(stream)
+    hp.start()
+    for k in range(args.steps):
+        hp.submit(host, O_hosts[k % 2])
+    hp.drain()
+    ee[1].record(stream)
+    torch.cuda.synchronize()
+    e2e_step_ms = max_over_ranks([ee[0].elapsed_time(ee[1])], dist, "cuda")[0] / args.steps
 
     # Scoring at scale: 16 users x 65,536 candidates drawn uniformly from the
     # whole catalogue (gathered rows far exceed L2; L2 flushed before each
@@ -754,10 +753,14 @@ def main():
                 "clocks": sampler.summary(),
                 "e2e": {"value": job_throughput(world, total_cand, e2e_step_ms), "unit": "pairs/s",
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                        "note": "per-request inputs (history, context, offsets, candidate IDs) "
-                                "copied from pinned host memory and scores copied back inside "
-                                "each timed step; weights, links and the item table stay "
-                                "resident (the cache is still rebuilt from it every step)"},
+                        "ms_per_step": e2e_step_ms, "scores_match_device_step": e2e_match,
+                        "note": "every step's per-request inputs (history, context, offsets, "
+                                "candidate IDs) copied from pinned host memory and its scores "
+                                "copied back, inside the timed region; steps pipelined over two "
+                                "request slots (copies on two copy streams overlap the "
+                                "neighbouring steps' compute); weights, links and the item table "
+                                "stay resident (the cache is still rebuilt from it every step); "
+                                "no L2 flush: each step streams 512 MB through the 126 MB L2"},
                 "gpu_launches": launches, "wall_s_timed": t_wall}
         if world == 1 and not args.no_cpu_baseline:
             # whole steps (every user, as many catalogue rows as the catalogue

@@ -200,3 +200,81 @@ def step_graphs(x: DeviceInputs, buf: Buffers):
     g_cache = capture(lambda: build_cache(x, buf))
     g_score = capture(lambda: score(x, buf, LP))
     return g_step, g_user, g_cache, g_score
+
+
+# Per-request inputs of a step: what changes from one batch of users to the
+# next (the weights, the global links and the item table stay resident).
+REQUEST_FIELDS = ("E", "ctx", "hist_offsets", "cand_ids", "cand_offsets")
+
+
+class HostPipeline:
+    """Steps fed from pinned host memory, overlapped over two request slots.
+
+    ``submit(host, O_host)`` copies one batch's per-request inputs (a dict of
+    pinned CPU tensors keyed by ``REQUEST_FIELDS``, shaped as the device
+    inputs) to the device on a copy stream, runs ``step`` on the caller's
+    current stream and copies the scores back into the pinned ``O_host`` on a
+    second copy stream.  Consecutive submissions alternate between two slots
+    (inputs and output buffer), so while step k computes, the inputs of step
+    k+1 are on their way in and the scores of step k-1 on their way out.  A
+    slot is reused only after its previous step has finished reading its
+    inputs and its scores have left the device; the workspace and the
+    layers' intermediates are shared, since the steps themselves run in order
+    on one stream.  All calls are asynchronous; ``drain(stream)`` makes
+    ``stream`` wait for every copy issued so far.
+    """
+
+    def __init__(self, x: DeviceInputs, buf: Buffers):
+        self.slots = []
+        for s in range(2):
+            if s == 0:
+                xs, bs = x, buf
+            else:
+                fresh = {k: None if getattr(x, k) is None else torch.empty_like(getattr(x, k))
+                         for k in REQUEST_FIELDS}
+                xs = dataclasses.replace(x, **fresh)
+                bs = dataclasses.replace(buf, O=torch.empty_like(buf.O))
+            self.slots.append((xs, bs))
+        dev = buf.O.device
+        self.h2d = torch.cuda.Stream(device=dev)
+        self.d2h = torch.cuda.Stream(device=dev)
+        self.inputs_free = [torch.cuda.Event() for _ in range(2)]
+        self.inputs_ready = [torch.cuda.Event() for _ in range(2)]
+        self.output_free = [torch.cuda.Event() for _ in range(2)]
+        self.n = 0
+
+    def submit(self, host: dict, O_host: torch.Tensor, stream=None):
+        s = self.n % 2
+        self.n += 1
+        xs, bs = self.slots[s]
+        main = torch.cuda.current_stream() if stream is None else stream
+        # inputs in: after the step that last used this slot has read them
+        # (an event never recorded is complete, so the first two pass at once)
+        self.h2d.wait_event(self.inputs_free[s])
+        with torch.cuda.stream(self.h2d):
+            for k in REQUEST_FIELDS:
+                if host.get(k) is not None:
+                    getattr(xs, k).copy_(host[k], non_blocking=True)
+        self.inputs_ready[s].record(self.h2d)
+        # the step: after its inputs arrived and this slot's last scores left
+        main.wait_event(self.inputs_ready[s])
+        main.wait_event(self.output_free[s])
+        with torch.cuda.stream(main):
+            out = step(xs, bs)
+        self.inputs_free[s].record(main)
+        # scores out
+        self.d2h.wait_event(self.inputs_free[s])
+        with torch.cuda.stream(self.d2h):
+            O_host.copy_(out, non_blocking=True)
+        self.output_free[s].record(self.d2h)
+
+    def drain(self, stream=None):
+        main = torch.cuda.current_stream() if stream is None else stream
+        main.wait_stream(self.h2d)
+        main.wait_stream(self.d2h)
+
+    def start(self, stream=None):
+        """Orders both copy streams after the work queued on ``stream``."""
+        main = torch.cuda.current_stream() if stream is None else stream
+        self.h2d.wait_stream(main)
+        self.d2h.wait_stream(main)

@@ -77,3 +77,34 @@ def test_graph_replay_matches_eager():
         torch.cuda.synchronize()
         assert lime.lime_get_status(buf.ws) == 0
         assert torch.equal(O_eager.view(torch.int16), buf.O.view(torch.int16))
+
+
+def test_host_pipeline_alternating_batches_match_single_steps():
+    # two request batches of the same shapes (different histories, contexts
+    # and candidate IDs; shared weights and catalogue) submitted as A, B, A, B
+    # through the two-slot host pipeline give each batch's single-step scores
+    # bit for bit: neither slot's inputs nor scores leak into the other's
+    import dataclasses
+    w = synth.workload("standard", B=4, n_items=5000)
+    n_hist, n_cand = [300, 0, 129, 1024], [64, 3, 100, 200]
+    xa = pipeline.to_device(w, synth.user_side(w, n_hist), synth.candidate_side(w, n_cand),
+                            synth.item_table(w))
+    w2 = dataclasses.replace(w, seed=w.seed + 77)
+    src = pipeline.to_device(w2, synth.user_side(w2, n_hist), synth.candidate_side(w2, n_cand),
+                             None)
+    xb = dataclasses.replace(xa, **{k: getattr(src, k) for k in pipeline.REQUEST_FIELDS})
+    buf = pipeline.alloc(xa)
+    ref = [pipeline.step(xa, buf).clone(), pipeline.step(xb, buf).clone()]
+    assert not torch.equal(ref[0], ref[1])
+    host = [{k: getattr(xs, k).cpu().pin_memory() for k in pipeline.REQUEST_FIELDS}
+            for xs in (xa, xb)]
+    outs = [torch.empty(buf.O.shape, dtype=buf.O.dtype).pin_memory() for _ in range(4)]
+    hp = pipeline.HostPipeline(xa, buf)
+    hp.start()
+    for k in range(4):
+        hp.submit(host[k % 2], outs[k])
+    hp.drain()
+    torch.cuda.synchronize()
+    assert lime.lime_get_status(buf.ws) == 0
+    for k in range(4):
+        assert torch.equal(outs[k].view(torch.int16), ref[k % 2].cpu().view(torch.int16)), k

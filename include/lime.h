@@ -223,7 +223,14 @@ int lime_context_links(const lime_dims* dims, int64_t B, const void* L,
  *   workspace, workspace_bytes: at least lime_workspace_bytes(dims, B,
  *          total_hist) bytes (ERR_ARG when smaller).
  * No output may overlap an input or the other output (ERR_ALIAS).
- * A user with no history gets a zero link-branch attention output.        */
+ * A user with no history gets a zero link-branch attention output.
+ * Streams: on the bf16 tensor-core path a non-final layer runs its link-row
+ * tail on a library-owned side stream (the device's highest priority),
+ * forked from `stream` with an event and joined back before the call
+ * returns, so all of the layer's work stays ordered on `stream` (and inside a
+ * graph captured from it).  The side stream is created by the first call on
+ * the device that is not being captured; until then the layer runs in order
+ * on `stream` alone.                                                      */
 int lime_xor_layer(const lime_dims* dims, int64_t B,
                    const int64_t* hist_offsets, int64_t total_hist,
                    const void* E_in, const void* Z_in, const lime_layer_w* w,

@@ -246,10 +246,15 @@ int launch_score(int64_t B, const void* cache, int64_t n_items, const int32_t* i
   if (cudaFuncSetAttribute(k_score_tc<L, U8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::SMEM) != cudaSuccess)
     return LIME_ERR_CUDA;
-  // enough (user, slot) CTAs to fill every SM a few times over
+  // enough (user, slot) CTAs to fill every SM a few times over, but at least
+  // two tiles per CTA on average: a CTA overlaps its next tile's gather with
+  // the current tile's MMA and epilogue, which one-tile CTAs in two waves of
+  // residency cannot do
   const int64_t target = 4LL * num_sms();
   int64_t G = (target + B - 1) / B;
   const int64_t tiles_hi = (total + kTile - 1) / kTile;
+  const int64_t two_per_cta = (tiles_hi / (B > 0 ? B : 1) + 1) / 2;
+  if (G > two_per_cta) G = two_per_cta;
   if (G > tiles_hi) G = tiles_hi;
   if (G < 1) G = 1;
   if (G > 65535) G = 65535;

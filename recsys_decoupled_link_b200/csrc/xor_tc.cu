@@ -40,6 +40,7 @@
 // the row's columns) or warp-specialized roles; one thread issues the MMAs.
 // Every kernel is launched with programmatic dependent launch (pdl_launch /
 // pdl_wait).  Every wait is bounded and sets LIME_FLAG_TIMEOUT.
+#include <mutex>
 #include <type_traits>
 
 #include "lime_fast.cuh"
@@ -1615,6 +1616,48 @@ bool set_smem(K kernel, int bytes) {
          cudaSuccess;
 }
 
+// A library-owned side stream (the device's highest priority) and two events
+// per device, for running the link tail beside the history GatedMLP: both
+// depend only on the attention kernel.  Created on the first call on the
+// device that is not being captured into a graph (creating them during a
+// capture could invalidate it); until then, and if creation fails, the layer
+// runs its kernels in order on the caller's stream.  The mutex makes each
+// fork (record, wait, launch, record, wait) atomic across host threads that
+// share a device.
+struct SideStream {
+  bool tried = false;
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxDevices = 64;
+SideStream g_side[kMaxDevices];
+std::mutex g_side_mu;
+
+SideStream* side_stream(cudaStream_t st) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  SideStream& r = g_side[dev];
+  if (!r.tried) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+      return nullptr;
+    r.tried = true;
+    int least = 0, greatest = 0;
+    bool ok = cudaDeviceGetStreamPriorityRange(&least, &greatest) == cudaSuccess &&
+              cudaStreamCreateWithPriority(&r.s, cudaStreamNonBlocking, greatest) == cudaSuccess;
+    ok = ok && cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming) == cudaSuccess;
+    ok = ok && cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      if (r.fork) cudaEventDestroy(r.fork);
+      if (r.s) cudaStreamDestroy(r.s);
+      r.s = nullptr;
+      r.fork = r.join = nullptr;
+      cudaGetLastError();
+    }
+  }
+  return r.s ? &r : nullptr;
+}
+
 template <int L>
 int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, const void* E_in,
               const void* Z_in, const lime_layer_w& w, void* E_out, void* Z_out, uint8_t* ws,
@@ -1642,11 +1685,13 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
                         (const bf16*)w.b1, ws, Lw, scale, D.phi == LIME_PHI_SILU, status);
     if (rc) return rc;
   }
+  CUtensorMap tmE_ffn{};
   if (nh > 0) {
     CUtensorMap tmE, tmY;
     if (!make_tmap_2d_bf16(&tmE, E_in, kD, (uint64_t)nh, kD * 2, 64, kTile) ||
         !make_tmap_2d_f16(&tmY, ws + Lw.yd, kD, (uint64_t)nh, kD * 2, 64, kTile))
       return LIME_ERR_CUDA;
+    tmE_ffn = tmE;
     const int64_t tiles_hi = Lw.max_tiles;
     const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
     {
@@ -1658,23 +1703,44 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
                           status);
       if (rc) return rc;
     }
-    if (!last) {
-      if (!set_smem(k_hist_ffn, kFfnSmem)) return LIME_ERR_CUDA;
-      int rc = launch_pdl(k_hist_ffn, dim3(grid), dim3(kFfnEpi + 64), kFfnSmem, st, 1, tmE,
-                          (const bf16*)w.g2, (const bf16*)w.b2, (const uint8_t*)ws, Lw,
-                          (bf16*)E_out, status);
-      if (rc) return rc;
-    }
   }
-  {
-    // one 4-CTA cluster per 128 link rows
-    if (!set_smem(k_link_tail<L>, kTailSmem)) return LIME_ERR_CUDA;
-    int rc = launch_pdl(k_link_tail<L>, dim3((unsigned)((nz + kTile - 1) / kTile), kF / 64),
-                        dim3(512), kTailSmem, st, kF / 64, (const bf16*)Z_in, nz,
-                        (const bf16*)w.g2, (const bf16*)w.b2, (const uint8_t*)ws, Lw, (bf16*)Z_out,
-                        status);
-    if (rc) return rc;
+  // one 4-CTA cluster per 128 link rows
+  if (!set_smem(k_link_tail<L>, kTailSmem)) return LIME_ERR_CUDA;
+  auto tail = [&](cudaStream_t s) {
+    return launch_pdl(k_link_tail<L>, dim3((unsigned)((nz + kTile - 1) / kTile), kF / 64),
+                      dim3(512), kTailSmem, s, kF / 64, (const bf16*)Z_in, nz,
+                      (const bf16*)w.g2, (const bf16*)w.b2, (const uint8_t*)ws, Lw, (bf16*)Z_out,
+                      status);
+  };
+  if (last || nh == 0) return tail(st);
+  // the history GatedMLP and the link tail both read only what the attention
+  // kernel left: the tail runs on the high-priority side stream, so its 4-CTA
+  // clusters take SMs as the attention kernel's CTAs retire and the GatedMLP's
+  // persistent CTAs fill the rest
+  if (!set_smem(k_hist_ffn, kFfnSmem)) return LIME_ERR_CUDA;
+  const int64_t tiles_hi = Lw.max_tiles;
+  const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
+  auto ffn = [&]() {
+    return launch_pdl(k_hist_ffn, dim3(grid), dim3(kFfnEpi + 64), kFfnSmem, st, 1, tmE_ffn,
+                      (const bf16*)w.g2, (const bf16*)w.b2, (const uint8_t*)ws, Lw,
+                      (bf16*)E_out, status);
+  };
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* side = side_stream(st);
+  if (!side) {
+    int rc = ffn();
+    return rc ? rc : tail(st);
   }
+  if (cudaEventRecord(side->fork, st) != cudaSuccess ||
+      cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
+    return LIME_ERR_CUDA;
+  int rc = tail(side->s);
+  if (rc) return rc;
+  rc = ffn();
+  if (rc) return rc;
+  if (cudaEventRecord(side->join, side->s) != cudaSuccess ||
+      cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess)
+    return LIME_ERR_CUDA;
   return LIME_OK;
 }
 

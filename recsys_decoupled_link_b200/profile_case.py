@@ -3,7 +3,9 @@
     python -m recsys_decoupled_link_b200.profile_case --phase cache --workload standard --reps 3
 
 Phases: ``cache`` (QK-cache build over the catalogue), ``score`` (cached
-scoring; the cache is built once first), ``layer`` (one LIME-XOR layer, the
+scoring; the cache is built once first), ``score_scale`` (cached scoring of
+16 users x 65,536 candidate IDs drawn uniformly from the whole catalogue, so
+the gathered rows far exceed L2), ``layer`` (one LIME-XOR layer, the
 first of the stack, with history outputs), ``last`` (the last-layer variant
 without history outputs), ``step`` (the whole pass).  Inputs are the seeded
 synthetic workloads of ``synth``; ``--items`` and ``--users`` shrink them.
@@ -19,7 +21,7 @@ from . import lime, pipeline, synth
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--phase", default="cache", choices=["cache", "score", "layer", "last", "step"])
+    ap.add_argument("--phase", default="cache", choices=["cache", "score", "score_scale", "layer", "last", "step"])
     ap.add_argument("--workload", default="standard")
     ap.add_argument("--items", type=int, default=None)
     ap.add_argument("--users", type=int, default=None)
@@ -39,13 +41,23 @@ def main():
         lime.lime_context_links(x.dims, x.L, x.ctx, *x.ctx_w, buf.LC, buf.ws)
     else:
         Z = x.Z0
-    if a.phase == "score":
+    if a.phase in ("score", "score_scale"):
         pipeline.build_cache(x, buf)
+    if a.phase == "score_scale":
+        users, per = 16, 65536
+        g = torch.Generator().manual_seed(4242)
+        sc_ids = torch.randint(0, w.n_items, (users * per,), generator=g).to(torch.int32).cuda()
+        sc_off = (torch.arange(users + 1, dtype=torch.int64) * per).cuda()
+        sc_LP = Z[:users].contiguous()
+        sc_O = torch.empty(users * per, w.d, dtype=buf.O.dtype, device="cuda")
     for _ in range(a.reps):
         if a.phase == "cache":
             pipeline.build_cache(x, buf)
         elif a.phase == "score":
             pipeline.score(x, buf, Z)
+        elif a.phase == "score_scale":
+            lime.lime_score_candidates(x.dims, buf.cache, sc_ids, sc_off, users * per, sc_LP,
+                                       sc_O, buf.ws)
         elif a.phase == "layer":
             lime.lime_xor_layer(x.dims, x.hist_offsets, x.total_hist, x.E, Z, x.layers[0],
                                 buf.E_bufs[0], buf.Z_bufs[0], buf.ws)

@@ -439,6 +439,15 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
 }
+// The two halves of cluster_sync, for overlapping the barrier with work that
+// neither needs the other CTAs nor is needed by them.  Every thread calls
+// them alternately (arrive, wait, arrive, wait, ...), converged per warp.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 // Cooperative, coalesced store of the first `nv` rows of a [128 x 128] bf16
 // tile held in the swizzled layout (2 blocks of [128 x 64]) to row-major

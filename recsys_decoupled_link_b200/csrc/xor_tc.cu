@@ -1399,6 +1399,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_arrive_expect_tx(&c.bar[3], 3 * 4 * kQuarter);   // the other CTAs' b rows
     mbar_arrive_expect_tx(&c.bar[4], 3 * 32 * 512);       // the other CTAs' partial rows
   }
+  cluster_arrive();    // (1) this CTA's barriers are initialised and armed
   const int64_t t0 = (int64_t)blockIdx.x * kTile;
   const int warp = threadIdx.x >> 5;
   const int part = warp >> 2;
@@ -1474,7 +1475,8 @@ __global__ void __launch_bounds__(512, 1)
     sw_st16(sAl, kBlk, 32 * cr + lr, h * kDH + q * 8, pack8(l8));
   }
   fence_proxy_async_smem();
-  cluster_sync();      // every CTA's barriers are armed and its b rows are written
+  __syncthreads();     // this CTA's b rows are written
+  cluster_wait();      // (1) every CTA's barriers are armed
   if (threadIdx.x == 0) {
     // rows 32cr..32cr+31 of the four 64-column blocks (hi 0, hi 1, lo 0, lo 1)
     // are 4 KB each and contiguous in the swizzled layout
@@ -1488,6 +1490,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   }
   mbar_wait(&c.bar[3], 0, status, c.abort_flag);
+  cluster_arrive();    // (2) this CTA has received every row it was sent
   mbar_wait(&c.bar[0], 0, status, c.abort_flag);
   if (threadIdx.x == 0) {
     tc_fence_after();
@@ -1495,8 +1498,6 @@ __global__ void __launch_bounds__(512, 1)
     mma_tile(c.tmem, smem_u32(sAl), kBlk, smem_u32(sWo), kBlk, 128, 128, true);
     mma_commit(&c.bar[1]);
   }
-  // every CTA has received its rows, so no copy still reads our b rows
-  cluster_sync();
   mbar_wait(&c.bar[1], mph, status, c.abort_flag);
   mph ^= 1u;
   tc_fence_after();
@@ -1521,6 +1522,8 @@ __global__ void __launch_bounds__(512, 1)
       for (int q = 0; q < 8; ++q) dst[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
     }
     layer_norm_part(y, c0, red, part, r);
+    // (2) every CTA has received its rows, so no copy still reads our b rows
+    cluster_wait();
     split_part_st(sAh, sAl, r, c0, y);
   }
   fence_proxy_async_smem();
@@ -1562,6 +1565,7 @@ __global__ void __launch_bounds__(512, 1)
     mma_tile(c.tmem + 256, smem_u32(sHl), kBlk, smem_u32(sW + 2 * kBlk), kBlk, 128, 64, true);
   }
   cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+  cluster_arrive();    // (3) this CTA's hid and Wo buffers are free to receive
   // 3. this chunk's fp32 partial -> shared memory (the A operand is dead);
   //    rows 32q..32q+31 form one contiguous 16 KB piece
   {
@@ -1574,7 +1578,8 @@ __global__ void __launch_bounds__(512, 1)
       *f32_chunk(sP, r, part * 8 + q) = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
   }
   fence_proxy_async_smem();
-  cluster_sync();      // every CTA's hid and Wo buffers are free to receive
+  __syncthreads();     // this CTA's partial rows are written
+  cluster_wait();      // (3) every CTA's hid and Wo buffers are free to receive
   if (threadIdx.x == 0) {
     for (uint32_t p = 0; p < 4; ++p) {
       if (p == cr) continue;
@@ -1584,6 +1589,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   }
   mbar_wait(&c.bar[4], 0, status, c.abort_flag);
+  cluster_arrive();    // (4) this CTA has received every partial it was sent
   // 4. rows 32cr..32cr+31: Z' = Y_Z + the four partials (rank order)
   {
     const int lr = threadIdx.x >> 4, cc = threadIdx.x & 15;   // 8 columns each
@@ -1604,7 +1610,7 @@ __global__ void __launch_bounds__(512, 1)
     }
     if (Rr < nrows) reinterpret_cast<uint4*>(Z_out + Rr * kD)[cc] = pack8(v);
   }
-  cluster_sync();   // every CTA has received its partials: no copy still reads ours
+  cluster_wait();   // (4) every CTA has received its partials: no copy still reads ours
   cta_teardown(c);
 }
 

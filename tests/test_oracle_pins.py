@@ -482,3 +482,22 @@ def test_window_zero_is_plain_xor_and_one_token_history_has_no_neighbours():
     Q1, K1, V1 = Q[N - 1:], K[N - 1:], V[N - 1:]
     np.testing.assert_allclose(O.xor_attention(Q1, K1, V1, 1, 2, window=3),
                                O.xor_attention(Q1, K1, V1, 1, 2), rtol=0, atol=1e-15)
+
+
+def test_int8_cache_layout_matches_printed_cache_sizes():
+    # LIME listing, Table 12: the int8 cache of 100M items x 4 heads takes
+    # 3.2 / 6.4 / 12.8 / 25.6 / 51.2 GB at l = 8 / 16 / 32 / 64 / 128, i.e. one
+    # byte per (item, head, link).  The oracle's int8 cache is [items, H, l]
+    # bytes; its per-item size, scaled to the table's catalogue, gives the
+    # printed sizes.
+    g = json.load(open(os.path.join(HERE, "golden", "int8_cache_sizes.json")))
+    H = g["heads"]
+    rng = np.random.default_rng(7)
+    for l_str, gb in g["gb_by_links"].items():
+        l = int(l_str)
+        w = rng.random((3, H, l))
+        cache = w / w.sum(axis=-1, keepdims=True)
+        q = O.quantize_cache_u8(cache)
+        assert q.dtype == np.uint8 and q.shape == (3, H, l)
+        per_item = q.nbytes // q.shape[0]
+        assert per_item * g["items"] == pytest.approx(gb * 1e9, rel=1e-12)

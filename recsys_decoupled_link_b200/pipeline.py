@@ -221,7 +221,8 @@ class HostPipeline:
     inputs and its scores have left the device; the workspace and the
     layers' intermediates are shared, since the steps themselves run in order
     on one stream.  All calls are asynchronous; ``drain(stream)`` makes
-    ``stream`` wait for every copy issued so far.
+    ``stream`` wait for every copy issued so far, so an ``O_host`` may be read
+    on the host once ``drain`` has been called and ``stream`` synchronised.
     """
 
     def __init__(self, x: DeviceInputs, buf: Buffers):

@@ -183,6 +183,47 @@ def test_layer_matches_library_composition(N, l, H):
     np.testing.assert_allclose(Zp, rZ, rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("n_layers", [2, 3])
+def test_user_encode_chains_layers_like_the_library_composition(n_layers):
+    # the stack (LIME note, 整体框架: history and context links pass through
+    # the layers together): layer i + 1 takes layer i's history AND link rows.
+    # Reference: torch's layer composition applied layer after layer per user,
+    # with distinct weights per layer, so that feeding the original E (or Z)
+    # to every layer, reusing one layer's weights, or returning an earlier
+    # layer's link rows all fail.
+    d, H, l = 16, 2, 4
+    layers = [rand_layer(d, 2 * d) for _ in range(n_layers)]
+    ns = [5, 1, 9]
+    offs = np.concatenate([[0], np.cumsum(ns)])
+    E, Z0 = rand(sum(ns), d, scale=0.5), rand(3, l, d, scale=0.5)
+    E_out, LP = O.user_encode(E, offs, Z0, layers, H)
+    for u in range(3):
+        a, b = offs[u], offs[u + 1]
+        e, z = E[a:b], Z0[u]
+        for w in layers:
+            e, z = library_layer(e, z, w, H)
+        np.testing.assert_allclose(LP[u], z, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(E_out[a:b], e, rtol=0, atol=1e-12)
+        # the same chain through explicit single-layer oracle calls
+        e2, z2 = E[a:b], Z0[u]
+        for w in layers:
+            e2, z2 = O.xor_layer_user(e2, z2, w, H)
+        np.testing.assert_allclose(LP[u], z2, rtol=0, atol=1e-12)
+        # the pin is sensitive to the chaining: the last layer fed the
+        # original history lands far from the chained result
+        _, z_wrong = library_layer(E[a:b], _chain_z(E[a:b], Z0[u], layers[:-1], H),
+                                   layers[-1], H)
+        assert np.abs(z_wrong - z).max() > 1e-3
+
+
+def _chain_z(E, Z, layers, H):
+    """Link rows after `layers`, each layer fed the ORIGINAL history E (the
+    slip the chaining pin has to catch)."""
+    for w in layers:
+        _, Z = library_layer(E, Z, w, H)
+    return Z
+
+
 def test_history_permutation_invariance():
     N, l, d, H = 23, 4, 16, 2
     layers = [rand_layer(d, 2 * d) for _ in range(2)]

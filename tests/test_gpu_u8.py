@@ -6,8 +6,10 @@ encoding): q = round(255 w), ties to even, dequantised as q / 255.
 The byte is an integer decided by floating point, so the cache is checked in
 two ways: against the GPU's own bf16 cache (the same weight the kernel
 rounds, to a few bf16 ulps), where the byte must be the correct rounding
-except where 255 w lies within 0.05 of a tie; and against the oracle's
-weights, within half a step plus the weight tolerance of the bf16 cache.
+except where 255 w lies within 0.05 of a tie; and against the oracle's byte
+quantize_cache_u8(w_ref), which it must equal exactly wherever 255 w_ref lies
+more than 0.02 from a tie (the kernel's weight error, from its bf16 operands,
+is at most 0.001 on that scale), and within one step near a tie.
 Scoring is checked against the oracle fed the GPU's bytes (isolated), and
 bit-exactly with identity values.
 """
@@ -50,11 +52,22 @@ def test_u8_cache_rounds_the_kernel_weight_and_tracks_the_oracle(l):
     exact = np.rint(x).astype(np.int64)
     assert (qg[~near_tie] == exact[~near_tie]).all()
     assert (np.abs(qg[near_tie] - exact[near_tie]) <= 1).all()
-    # 2. against the oracle's weights: half a step plus the weight error
+    # 2. against the oracle's byte: the kernel's fp32 weight differs from the
+    #    oracle's by the rounding of its bf16 operands; emulating those
+    #    roundings on the CPU (T exact in bf16, the folded G rounded to bf16)
+    #    puts 255 |w_kernel - w_ref| at or below 0.001 on these inputs.  So
+    #    wherever 255 w_ref lies more than 0.02 from a tie the byte must equal
+    #    quantize_cache_u8(ref) exactly, and within 0.02 of a tie it may be
+    #    either neighbour.
     ref = O.qk_cache(f64(T), f64(us.L), f64(cs.Wq_c), f64(cs.Wk_c), w.H)
+    xr = 255.0 * ref
+    tie = np.abs(xr - np.floor(xr) - 0.5) < 0.02
+    qr = O.quantize_cache_u8(ref).astype(np.int64)
+    away = qg[~tie] == qr[~tie]
+    assert away.all(), f"{(~away).sum()} of {away.size} bytes away from ties differ"
+    assert (np.abs(qg[tie] - qr[tie]) <= 1).all()
     err = np.abs(qg / 255.0 - ref)
-    assert err.max() <= 0.5 / 255 + 2e-3, err.max()
-    assert (qg == O.quantize_cache_u8(ref)).mean() > 0.7
+    assert err.max() <= 0.5 / 255 + 2e-3 / 255, err.max()
 
 
 @pytest.mark.parametrize("l", [32, 64])

@@ -116,23 +116,50 @@ __device__ __forceinline__ void ln_stage(float* gb, const bf16* g, const bf16* b
   }
 }
 
+// Statistics of one 32-value part of a row: its mean and the sum of squared
+// deviations from that mean (two passes over the registers, so no
+// cancellation between E[x^2] and mu^2 however large the row's mean is).
+__device__ __forceinline__ void part_stats(const float* x, float& mean, float& m2) {
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) s += x[k];
+  mean = s * (1.0f / 32);
+  float q = 0.f;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const float dlt = x[k] - mean;
+    q = fmaf(dlt, dlt, q);
+  }
+  m2 = q;
+}
+
+// Row mean and rstd from the four parts' (mean, m2): the parallel-variance
+// merge for equal counts, M2 = sum m2_p + 32 sum (mean_p - mu)^2 (biased
+// variance M2 / 128, eps as in LayerNorm).
+__device__ __forceinline__ void merge4_stats(float m0, float m1, float m2_, float m3, float q0,
+                                             float q1, float q2, float q3, float& mu,
+                                             float& rstd) {
+  mu = (m0 + m1 + m2_ + m3) * 0.25f;
+  const float d0 = m0 - mu, d1 = m1 - mu, d2 = m2_ - mu, d3 = m3 - mu;
+  const float M2 = (q0 + q1) + (q2 + q3) + 32.0f * (d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3);
+  rstd = rsqrtf(M2 * (1.0f / kD) + kLnEps);
+}
+
 // LayerNorm of one row held as four 32-column parts (x = this thread's part,
-// columns c0..c0+31), affine with the staged g, b.  The sum and the sum of
-// squares are reduced in one pass (var = E[x^2] - mu^2 in fp32; LN inputs
-// here are O(1) with |mu| of the order of the spread, so the cancellation
-// costs a few ulp).  `red` is a kLnFloats scratch (red[0..1023] for the
+// columns c0..c0+31), affine with the staged g, b.  Each part's mean and
+// centred sum of squares are exchanged through `red` and merged (see
+// merge4_stats).  `red` is a kLnFloats scratch (red[0..1023] for the
 // reductions, g and b after them); all 512 threads take part (one block-wide
 // barrier; the caller's next barrier must come before red is written again).
 __device__ __forceinline__ void layer_norm_part(float* x, int c0, float* red, int part, int row) {
-  float s1 = 0.f, s2 = 0.f;
-#pragma unroll
-  for (int k = 0; k < 32; ++k) { s1 += x[k]; s2 = fmaf(x[k], x[k], s2); }
-  red[part * 128 + row] = s1;
-  red[512 + part * 128 + row] = s2;
+  float pm, pq;
+  part_stats(x, pm, pq);
+  red[part * 128 + row] = pm;
+  red[512 + part * 128 + row] = pq;
   __syncthreads();
-  const float mu = (red[row] + red[128 + row] + red[256 + row] + red[384 + row]) * (1.0f / kD);
-  const float ex2 = (red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row]) * (1.0f / kD);
-  const float rstd = rsqrtf(fmaxf(ex2 - mu * mu, 0.f) + kLnEps);
+  float mu, rstd;
+  merge4_stats(red[row], red[128 + row], red[256 + row], red[384 + row], red[512 + row],
+               red[640 + row], red[768 + row], red[896 + row], mu, rstd);
   const float4* g4 = reinterpret_cast<const float4*>(red + 1024 + c0);
   const float4* b4 = reinterpret_cast<const float4*>(red + 1024 + kD + c0);
 #pragma unroll
@@ -815,21 +842,32 @@ __global__ void __launch_bounds__(kXaThreads, 1)
       // LN1 statistics of this thread's row (biased variance; see layer_norm_part)
       float mu_r, rs_r;
       {
-        float s1 = 0.f, s2 = 0.f;
+        // the part's mean, then its centred sum of squares (a second read of
+        // the tile's 32 values; see part_stats)
+        float pm = 0.f, pq = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float x[8];
           unpack8(sw_ld16(sA, kBlk, row, c0 + q * 8), x);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) { s1 += x[k]; s2 = fmaf(x[k], x[k], s2); }
+          for (int k = 0; k < 8; ++k) pm += x[k];
         }
-        red[part * 128 + row] = s1;
-        red[512 + part * 128 + row] = s2;
+        pm *= 1.0f / 32;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float x[8];
+          unpack8(sw_ld16(sA, kBlk, row, c0 + q * 8), x);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float dlt = x[k] - pm;
+            pq = fmaf(dlt, dlt, pq);
+          }
+        }
+        red[part * 128 + row] = pm;
+        red[512 + part * 128 + row] = pq;
         named_bar_sync(1, kXaEpi);
-        mu_r = (red[row] + red[128 + row] + red[256 + row] + red[384 + row]) * (1.0f / kD);
-        const float ex2 =
-            (red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row]) * (1.0f / kD);
-        rs_r = rsqrtf(fmaxf(ex2 - mu_r * mu_r, 0.f) + kLnEps);
+        merge4_stats(red[row], red[128 + row], red[256 + row], red[384 + row], red[512 + row],
+                     red[640 + row], red[768 + row], red[896 + row], mu_r, rs_r);
         if (part == 0) {
           smu[row] = mu_r;
           smu[128 + row] = SILU ? rs_r : rs_r * kLog2e;   // softmax: log2 units
@@ -1242,7 +1280,11 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
       const int4 tl = tile_of(g + 2 * j);
       // Y = E + Yd into OUT (own 64 columns); LN2 statistics over all 128
       mbar_wait(&b[kE], (uint32_t)j & 1u, status, abort_flag);
-      float s1 = 0.f, s2 = 0.f;
+      // the row's sums of (y - K) and (y - K)^2 with the shift K = the row's
+      // first value: the shifted one-pass variance loses nothing to
+      // cancellation however large the row's mean is, since |mu - K| is of
+      // the order of the row's spread
+      float K = 0.f, s1 = 0.f, s2 = 0.f;
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         float y[32];
@@ -1261,15 +1303,21 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
 #pragma unroll
           for (int i = 0; i < 8; ++i) y[q * 8 + i] += e[i];
         }
+        if (p == 0) K = y[0];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) { s1 += y[i]; s2 = fmaf(y[i], y[i], s2); }
+        for (int i = 0; i < 32; ++i) {
+          const float t = y[i] - K;
+          s1 += t;
+          s2 = fmaf(t, t, s2);
+        }
         if ((p >> 1) == half) {
           tmem_st16(tOUT + p * 32, y);
           tmem_st16(tOUT + p * 32 + 16, y + 16);
         }
       }
-      const float mu = s1 * (1.0f / kD);
-      const float rstd = rsqrtf(fmaxf(s2 * (1.0f / kD) - mu * mu, 0.f) + kLnEps);
+      const float ms = s1 * (1.0f / kD);
+      const float mu = K + ms;
+      const float rstd = rsqrtf(fmaxf(s2 * (1.0f / kD) - ms * ms, 0.f) + kLnEps);
       tmem_st_wait();
       group_sync();   // every thread of the group has read the E tile
 #pragma unroll

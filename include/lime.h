@@ -180,14 +180,18 @@ int lime_score_candidates_uncached(const lime_dims* dims, int64_t B, const void*
  * cache_out (same meaning, layout and checks as lime_build_qk_cache); the
  * scratch lives in a static device array of LIME_NOALLOC_SCRATCH_BYTES bytes
  * that every GPU loading the library holds until the process exits.
- *   - The first call on a device (with that device current) looks up the
- *     array's device address; make that first call before any stream capture.
+ *   - Each call made outside a stream capture (with the device current) looks
+ *     up the array's device address; a call made during a capture reuses the
+ *     address found by the last such call on that device, so make the first
+ *     call on a device before any stream capture.
+ *   - Arguments are checked exactly as lime_build_qk_cache checks them, with
+ *     the same return codes, before the array is touched.
  *   - All calls share the array and it keeps the last call's contents; each
  *     call clears the status word it uses.  Calls that overlap on the GPU (on
  *     different streams, say) race on the array.
- *   - Sizes whose scratch exceeds the maximum (2*d*H*l bytes on the bf16
- *     tensor-core path, 4*(l*d + d*H*l) bytes otherwise, plus 256) return
- *     LIME_ERR_SCRATCH; use lime_build_qk_cache with a workspace instead.
+ *   - The scratch a call needs is lime_workspace_bytes(dims, 0, 0); when that
+ *     exceeds LIME_NOALLOC_SCRATCH_BYTES the call returns LIME_ERR_SCRATCH
+ *     (use lime_build_qk_cache with a workspace instead).
  *   - Device-side status flags of these calls are not reported.
  * Calls no cudaMalloc, cudaFree or allocating library routine.            */
 #define LIME_NOALLOC_SCRATCH_BYTES (1u << 20)

@@ -12,6 +12,8 @@ using namespace lime;
 
 namespace lime {
 static std::atomic<uint64_t> g_launches{0};
+int check_cache_args(const lime_dims* dims, const void* T, int64_t n_items, const void* L,
+                     const void* Wq_c, const void* Wk_c, const void* cache_out);
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 }  // namespace lime
 
@@ -80,6 +82,29 @@ float* scratch_of(void* ws) { return (float*)((char*)ws + kStatusBytes); }
 
 }  // namespace
 
+namespace lime {
+// Argument checks of the QK-cache build, apart from the workspace: dims,
+// sizes, null pointers, 16-byte alignment and output/input aliasing.
+int check_cache_args(const lime_dims* dims, const void* T, int64_t n_items, const void* L,
+                     const void* Wq_c, const void* Wk_c, const void* cache_out) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (n_items < 0 || n_items > (int64_t)INT32_MAX + 1) return LIME_ERR_ARG;
+  if (!L || !Wq_c || !Wk_c || (n_items > 0 && (!T || !cache_out))) return LIME_ERR_ARG;
+  if ((n_items > 0 && (!aligned16(T) || !aligned16(cache_out))) || !aligned16(L) ||
+      !aligned16(Wq_c) || !aligned16(Wk_c))
+    return LIME_ERR_ARG;
+  const size_t es = esize(dims);
+  const size_t cache_sz = (size_t)n_items * dims->H * dims->l * es;
+  if (overlap(cache_out, cache_sz, T, (size_t)n_items * dims->d * es) ||
+      overlap(cache_out, cache_sz, L, (size_t)dims->l * dims->d * es) ||
+      overlap(cache_out, cache_sz, Wq_c, (size_t)dims->d * dims->d * es) ||
+      overlap(cache_out, cache_sz, Wk_c, (size_t)dims->d * dims->d * es))
+    return LIME_ERR_ALIAS;
+  return LIME_OK;
+}
+}  // namespace lime
+
 extern "C" {
 
 size_t lime_workspace_bytes(const lime_dims* dims, int64_t B, int64_t total_hist) {
@@ -96,21 +121,9 @@ int lime_workspace_init(void* workspace, size_t bytes, cudaStream_t stream) {
 int lime_build_qk_cache(const lime_dims* dims, const void* T, int64_t n_items, const void* L,
                         const void* Wq_c, const void* Wk_c, void* cache_out, void* workspace,
                         size_t workspace_bytes, cudaStream_t stream) {
-  int rc = check_dims(dims);
+  int rc = lime::check_cache_args(dims, T, n_items, L, Wq_c, Wk_c, cache_out);
   if (rc) return rc;
-  if (n_items < 0 || n_items > (int64_t)INT32_MAX + 1) return LIME_ERR_ARG;
-  if (!L || !Wq_c || !Wk_c || (n_items > 0 && (!T || !cache_out))) return LIME_ERR_ARG;
-  if ((n_items > 0 && (!aligned16(T) || !aligned16(cache_out))) || !aligned16(L) ||
-      !aligned16(Wq_c) || !aligned16(Wk_c))
-    return LIME_ERR_ARG;
   if ((rc = check_ws(workspace, workspace_bytes, dims, 0, 0))) return rc;
-  const size_t es = esize(dims);
-  const size_t cache_sz = (size_t)n_items * dims->H * dims->l * es;
-  if (overlap(cache_out, cache_sz, T, (size_t)n_items * dims->d * es) ||
-      overlap(cache_out, cache_sz, L, (size_t)dims->l * dims->d * es) ||
-      overlap(cache_out, cache_sz, Wq_c, (size_t)dims->d * dims->d * es) ||
-      overlap(cache_out, cache_sz, Wk_c, (size_t)dims->d * dims->d * es))
-    return LIME_ERR_ALIAS;
   if (dims->dtype == LIME_BF16 && fast_cache_supported(*dims)) {
     rc = fast_build_qk_cache(*dims, T, n_items, L, Wq_c, Wk_c, cache_out,
                              scratch_of(workspace), status_of(workspace), stream);

@@ -12,9 +12,10 @@
 // The array is part of the library's device image: every GPU that loads the
 // library holds it until the process exits.  Host code cannot use the array's
 // name as a device address (on the host it names a stand-in object), so the
-// first call on each device, with that device current, looks its device
-// address up with cudaGetSymbolAddress and keeps it; that first call should
-// therefore come before any stream capture.  All calls share the one array and
+// entry point, with the device current, looks its device address up with
+// cudaGetSymbolAddress on every call outside a stream capture and keeps it for
+// calls made during one; the first call on each device should therefore come
+// before any stream capture.  All calls share the one array and
 // it keeps the last call's contents: each call clears the status word at its
 // head before use, and calls that overlap on the GPU (e.g. on two streams) race
 // on it.  Nothing here calls cudaMalloc, cudaFree or an allocating library
@@ -33,13 +34,19 @@ constexpr int kMaxDevices = 64;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
 std::mutex g_scratch_mu;
 
-// Device address of g_noalloc_scratch on the current device, looked up once per
-// device; nullptr if the runtime refuses.
-void* scratch_address() {
+// Device address of g_noalloc_scratch on the current device, nullptr if the
+// runtime refuses.  Looked up again on every call made outside a stream
+// capture (the address can change if the device's context is reset and the
+// module reloaded); a call made while `stream` is capturing uses the address
+// the last uncaptured call on this device found, so the first call on a device
+// has to come before any capture.
+void* scratch_address(cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return nullptr;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (cs == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) {
@@ -54,12 +61,20 @@ void* scratch_address() {
 
 }  // namespace
 
+namespace lime {
+int check_cache_args(const lime_dims* dims, const void* T, int64_t n_items, const void* L,
+                     const void* Wq_c, const void* Wk_c, const void* cache_out);
+}
+
 extern "C" int lime_build_qk_cache_noalloc(const lime_dims* dims, const void* T,
                                            int64_t n_items, const void* L, const void* Wq_c,
                                            const void* Wk_c, void* cache_out,
                                            cudaStream_t stream) {
+  // the same argument checks as lime_build_qk_cache, with the same codes,
+  // before the shared array is touched
+  int rc = lime::check_cache_args(dims, T, n_items, L, Wq_c, Wk_c, cache_out);
+  if (rc != LIME_OK) return rc;
   const size_t need = lime_workspace_bytes(dims, 0, 0);
-  if (need == 0) return dims == nullptr ? LIME_ERR_ARG : LIME_ERR_SHAPE;
   if (need > (size_t)LIME_NOALLOC_SCRATCH_BYTES) {
     fprintf(stderr,
             "liblime: lime_build_qk_cache_noalloc needs %zu bytes of scratch, more than its "
@@ -67,9 +82,9 @@ extern "C" int lime_build_qk_cache_noalloc(const lime_dims* dims, const void* T,
             need, (unsigned)LIME_NOALLOC_SCRATCH_BYTES);
     return LIME_ERR_SCRATCH;
   }
-  void* scratch = scratch_address();
+  void* scratch = scratch_address(stream);
   if (!scratch) return LIME_ERR_CUDA;
-  int rc = lime_workspace_init(scratch, LIME_NOALLOC_SCRATCH_BYTES, stream);
+  rc = lime_workspace_init(scratch, LIME_NOALLOC_SCRATCH_BYTES, stream);
   if (rc != LIME_OK) return rc;
   return lime_build_qk_cache(dims, T, n_items, L, Wq_c, Wk_c, cache_out, scratch,
                              LIME_NOALLOC_SCRATCH_BYTES, stream);

@@ -165,3 +165,27 @@ def test_phi_validation(lime):
     g = lime._lib.lime_build_qk_cache_u8
     assert g(ctypes.byref(d), 0x100000, 10, 0x200000, 0x300000, 0x400000, 0x500000,
              0x1000000, nws, None) == lime.LIME_ERR_SHAPE
+
+
+def test_noalloc_checks_arguments_like_the_workspace_call(lime):
+    # the allocation-free cache build rejects bad calls with the codes of
+    # lime_build_qk_cache, before it touches its static scratch array (so
+    # these calls return before any CUDA API call)
+    g = lime._lib.lime_build_qk_cache
+    na = lime._lib.lime_build_qk_cache_noalloc
+    dims = lime.make_dims(128, 4, 32, 256, 64, "bf16")
+    nws = lime.lime_workspace_bytes(dims, 0, 0)
+    cases = [
+        (dims, 0x100000, 10, 0x200000, 0x300000, 0x400000, 0x100000),   # cache over T
+        (dims, 0x100000, 10, None, 0x300000, 0x400000, 0x500000),       # no L
+        (dims, 0x100008, 10, 0x200000, 0x300000, 0x400000, 0x500000),   # T unaligned
+        (dims, 0x100000, -1, 0x200000, 0x300000, 0x400000, 0x500000),   # negative size
+        (lime.make_dims(128, 3, 32, 256, 64, "bf16"), 0x100000, 10, 0x200000, 0x300000,
+         0x400000, 0x500000),                                           # d % H != 0
+        (lime.lime_dims(128, 4, 32, 256, 64, 7), 0x100000, 10, 0x200000, 0x300000,
+         0x400000, 0x500000),                                           # bad dtype
+    ]
+    for d, T, n, L, Wq, Wk, out in cases:
+        want = g(ctypes.byref(d), T, n, L, Wq, Wk, out, 0x1000000, nws, None)
+        assert want != lime.LIME_OK
+        assert na(ctypes.byref(d), T, n, L, Wq, Wk, out, None) == want

@@ -6,8 +6,8 @@ that cannot accept cudaMalloc's implicit synchronisation); it keeps its scratch
 in a static device array instead of a caller workspace.  These tests call it
 through the C ABI twice in a row with different inputs — the second call runs
 on scratch the first one left behind — and compare each result with
-lime_build_qk_cache on a workspace, within the parity tolerance the other
-tests use.  The file is named to be collected last; it also passes alone in a
+lime_build_qk_cache on a workspace.  Both run the same kernels on the same
+inputs, so the results must be identical bit for bit.  The file is named to be collected last; it also passes alone in a
 fresh process, where its first call performs the per-device set-up.
 """
 import ctypes
@@ -16,7 +16,6 @@ import pytest
 import torch
 
 from recsys_decoupled_link_b200 import lime, synth
-from parity_util import assert_close, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -51,7 +50,7 @@ def test_noalloc_cache_matches_workspace_entry_point(case):
         assert rc == lime.LIME_OK
         torch.cuda.synchronize()
         assert lime.lime_get_status(ws) == 0
-        assert_close(got, f64(ref.cpu()), w.dtype, f"no-alloc cache, call {call + 1}")
+        assert torch.equal(got, ref), f"no-alloc cache, call {call + 1}"
 
 
 def test_noalloc_rejects_sizes_beyond_its_maximum():

@@ -1094,32 +1094,28 @@ __global__ void __launch_bounds__(kXaThreads, 1)
 }
 
 // ------------------------------------------------------- history GatedMLP
-// E' = Y + GatedMLP(LN2(Y)), Y = E + Yd, per 128-row history tile, with two
-// tiles in flight per SM (persistent, one CTA per SM).  The CTA's tiles
-// alternate between two groups; group g owns TMEM columns [256g, 256g + 256)
-// (the gate accumulator GB and the output accumulator OUT), one E/h2 tile
-// buffer, one hidden-chunk buffer and one [W1c | W3c] chunk slot, so while one
-// group's warps run a CUDA-core phase (LN2, SiLU, the E' readout) the tensor
-// cores run the other group's products.
-//   warps 8g .. 8g+7 (group g's epilogue): warp w serves TMEM lane quadrant
-//     w % 4 and half (w % 8) / 4 of every row (64 columns, handled as two
-//     32-column passes).  Per tile: Y = E (TMA tile) + Yd (fp16 rows,
-//     prefetched into L2 with the E tile) into OUT, so the W2 products add
-//     the GatedMLP onto the residual in place; each thread sums all 128
-//     columns of its row for the LN2 statistics (the two halves of a row
-//     compute them alike, so no reduction is exchanged); h2 = LN2(Y) over the
-//     E tile; per 64-wide hidden chunk hid = SiLU(G1) * G3 from GB into the
-//     chunk buffer; at the end E' = OUT staged over the E tile and written
-//     with coalesced 16-byte stores.
-//   warp 16 + g (lane 0): group g's loads and MMAs: G = h2 [W1c | W3c] (one
-//     N = 128 product) into GB, OUT += hid W2c with W2 resident in shared
-//     memory, the next chunk image once G has read the slot, the group's next
-//     E tile once its E' staging has been read out.
-// Group-local chunk counter gc = 4 j + c for the group's j-th tile: every
-// per-chunk barrier completes once per chunk (parity gc & 1), every per-tile
-// barrier once per tile (parity j & 1).
-constexpr int kFfnEpi = 512;   // epilogue threads (two groups of 256)
-constexpr int kFfnGrp = 256;
+// E' = Y + GatedMLP(LN2(Y)), Y = E + Yd, for one 128-row history tile at a
+// time, as a warp-specialized pipeline (persistent, one CTA per SM):
+//   warps 0-15 (epilogue): warp w serves TMEM lane quadrant w % 4 (tile rows
+//     32*(w%4) ...) and column part p = w / 4 (a quarter of every row).  Per
+//     tile they form Y = E (TMA tile) + Yd (fp16 rows, prefetched into L2
+//     with the E tile) and store it into the tile's output accumulator OUT,
+//     so that the W2 products add the GatedMLP onto the residual in place;
+//     write h2 = LN2(Y) (statistics reduced over the four parts through
+//     shared memory) over the E tile; compute hid = SiLU(G1) * G3 per 64-wide
+//     hidden chunk from TMEM GB[g%2] into smem HB[g%2]; and store E' = OUT.
+//     The next tile's Y and LN2 run before this tile's E' is read out, so the
+//     tensor cores start the next tile while the epilogue finishes this one.
+//   warp 16 (one lane) issues the MMAs: G(g) = h2 [W1c | W3c] (one N = 128
+//     product) into GB[g%2] and OUT += hid(g) W2c with W2 resident in shared
+//     memory.
+//   warp 17 (one lane) loads: the E tiles (one tile ahead) and the [W1c | W3c]
+//     chunk images through a two-slot ring (chunk g+1 is fetched as soon as
+//     G(g-1) has consumed its slot).
+// Chunks are counted over the CTA's whole tile sequence (g = 4*k + c for its
+// k-th tile), so every ring barrier's parity is (g / 2) % 2.
+// TMEM: GB[0] [0,128), GB[1] [128,256), OUT[k%2] [256 + 128*(k%2), +128).
+constexpr int kFfnEpi = 512;   // epilogue threads
 constexpr int kFfnTiles = 32;  // tile descriptors of a CTA kept in shared memory
 constexpr int kFfnSmem = 1024 + 14 * kBlk + 1024 + kFfnTiles * 16 + 256;
 
@@ -1129,35 +1125,37 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
                bf16* __restrict__ E_out, unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
-  uint8_t* sE0 = sm;                   // [2 groups] x [128 x 128] bf16: E tile -> h2 -> E' staging
-  uint8_t* sH0 = sm + 4 * kBlk;        // [2 groups] x [128 x 64] bf16: hidden chunk
-  uint8_t* sW0 = sm + 6 * kBlk;        // [2 groups] x [W1c | W3c] chunk slot
+  uint8_t* sE0 = sm;                   // 2 x [128 x 128] bf16: E tile -> h2 (-> LN2 scratch)
+  uint8_t* sH0 = sm + 4 * kBlk;        // 2 x [128 x 64]  bf16: hid chunk
+  uint8_t* sW13 = sm + 6 * kBlk;       // 2 x [W1c | W3c] ring
   uint8_t* sW2 = sm + 10 * kBlk;       // W2 image, 4 chunks
   float* sg = reinterpret_cast<float*>(sm + 14 * kBlk);   // g2, b2 as fp32 [2][128]
   int4* s_tiles = reinterpret_cast<int4*>(sm + 14 * kBlk + 1024);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 14 * kBlk + 1024 + kFfnTiles * 16);
-  // per group g: bar[g * 10 + i]
-  constexpr int kE = 0, kWt = 1, kG = 2, kGBf = 3, kHid = 4, kW2 = 5, kH2 = 6, kOut = 7,
-                kSE = 8, kDrain = 9;
-  uint64_t* barW2in = bar + 20;        // W2 image landed
-  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 21);
-  int* abort_flag = reinterpret_cast<int*>(bar + 22);
+  uint64_t* barE = bar;        // [2] E tile landed (TMA)
+  uint64_t* barWt = bar + 2;   // [2] [W1c | W3c] ring slot landed
+  uint64_t* barG = bar + 4;    // [2] G(g) in TMEM (MMA commit)
+  uint64_t* barHid = bar + 6;  // [2] hid(g) written, GB read (epilogue arrivals)
+  uint64_t* barW2 = bar + 8;   // [2] OUT += hid(g) W2c done (MMA commit)
+  uint64_t* barH2 = bar + 10;  // Y in OUT and h2 written (epilogue arrivals)
+  uint64_t* barOut = bar + 11; // all of the tile's MMAs done (MMA commit)
+  uint64_t* barW2in = bar + 12;  // W2 image landed
+  uint64_t* barDrain = bar + 13; // every MMA issued by the control lane is done
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 14);
+  int* abort_flag = reinterpret_cast<int*>(bar + 15);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int g = 0; g < 2; ++g) {
-      uint64_t* b = bar + g * 10;
-      mbar_init(&b[kE], 1);
-      mbar_init(&b[kWt], 1);
-      mbar_init(&b[kG], 1);
-      mbar_init(&b[kGBf], kFfnGrp);
-      mbar_init(&b[kHid], kFfnGrp);
-      mbar_init(&b[kW2], 1);
-      mbar_init(&b[kH2], kFfnGrp);
-      mbar_init(&b[kOut], 1);
-      mbar_init(&b[kSE], kFfnGrp);
-      mbar_init(&b[kDrain], 1);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&barE[q], 1);
+      mbar_init(&barWt[q], 1);
+      mbar_init(&barG[q], 1);
+      mbar_init(&barHid[q], kFfnEpi);
+      mbar_init(&barW2[q], 1);
     }
+    mbar_init(barH2, kFfnEpi);
+    mbar_init(barOut, 1);
     mbar_init(barW2in, 1);
+    mbar_init(barDrain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -1179,30 +1177,28 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
   if ((int)threadIdx.x < my_tiles && threadIdx.x < kFfnTiles)
     s_tiles[threadIdx.x] = tiles[blockIdx.x + threadIdx.x * gridDim.x];
   __syncthreads();
+  constexpr uint32_t T_OUT = 256;
   auto tile_of = [&](int k) -> int4 {
     return k < kFfnTiles ? s_tiles[k] : tiles[blockIdx.x + k * gridDim.x];
   };
-  constexpr int NC = kF / 64;          // hidden chunks per tile
+  const int n_chunks = my_tiles * (kF / 64);
 
-  if (warp >= kFfnEpi / 32) {
-    // ---- control: group g's loads and MMAs (one lane)
-    const int g = warp - kFfnEpi / 32;
-    const int n_g = my_tiles > g ? (my_tiles - g + 1) / 2 : 0;
-    uint64_t* b = bar + g * 10;
-    uint8_t* sE = sE0 + g * 2 * kBlk;
-    uint8_t* sH = sH0 + g * kBlk;
-    uint8_t* sW = sW0 + g * 2 * kBlk;
-    const uint32_t tGB = tmem + 256 * g, tOUT = tGB + 128;
-    if (lane == 0 && n_g > 0) {
-      auto load_w13 = [&](int gc) {
-        mbar_arrive_expect_tx(&b[kWt], 2 * kBlk);
-        bulk_load(sW, ws + Lw.img_13 + (gc % NC) * 2 * kBlk, 2 * kBlk, &b[kWt]);
+  if (warp == kFfnEpi / 32 + 1) {
+    // loader: the W1|W3 ring, the E tiles and W2.  It runs apart from the MMA
+    // issuer because tcgen05.mma issue stalls while the tensor pipe is busy,
+    // which would hold back the next loads.
+    if (lane == 0 && my_tiles > 0) {
+      auto load_w13 = [&](int g) {
+        const int s = g & 1, ch = g & 3;
+        mbar_arrive_expect_tx(&barWt[s], 2 * kBlk);
+        bulk_load(sW13 + s * 2 * kBlk, ws + Lw.img_13 + ch * 2 * kBlk, 2 * kBlk, &barWt[s]);
       };
-      auto load_e = [&](int j) {
-        const int4 tl = tile_of(g + 2 * j);
-        mbar_arrive_expect_tx(&b[kE], 2 * kBlk);
-        tma_load_2d(sE, &tmE, 0, tl.y, &b[kE]);
-        tma_load_2d(sE + kBlk, &tmE, 64, tl.y, &b[kE]);
+      auto load_e = [&](int k) {
+        const int4 tl = tile_of(k);
+        uint8_t* dst = sE0 + (k & 1) * 2 * kBlk;
+        mbar_arrive_expect_tx(&barE[k & 1], 2 * kBlk);
+        tma_load_2d(dst, &tmE, 0, tl.y, &barE[k & 1]);
+        tma_load_2d(dst + kBlk, &tmE, 64, tl.y, &barE[k & 1]);
         // the tile's Yd rows into L2, for the epilogue's plain loads
         bulk_prefetch_l2(reinterpret_cast<const __half*>(ws + Lw.yd) + (int64_t)tl.y * kD,
                          (uint32_t)tl.z * kD * 2);
@@ -1210,188 +1206,173 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
       prefetch_tmap(&tmE);
       load_e(0);
       load_w13(0);
-      if (g == 0) {
-        mbar_arrive_expect_tx(barW2in, 4 * kBlk);
-        bulk_load(sW2, ws + Lw.img_2, 4 * kBlk, barW2in);
-      }
-      bool ok = mbar_wait(barW2in, 0, status, abort_flag);
-      const int n_chunks = n_g * NC;
-      for (int j = 0; j < n_g && ok; ++j) {
-        if (!(ok = mbar_wait(&b[kH2], (uint32_t)j & 1u, status, abort_flag))) break;
-        for (int c = 0; c < NC; ++c) {
-          const int gc = j * NC + c;
-          if (!(ok = mbar_wait(&b[kWt], (uint32_t)gc & 1u, status, abort_flag))) break;
-          // GB is single: the epilogue must have read the previous chunk's gates
-          if (gc > 0 && !(ok = mbar_wait(&b[kGBf], (uint32_t)(gc - 1) & 1u, status, abort_flag)))
+      if (n_chunks > 1) load_w13(1);
+      mbar_arrive_expect_tx(barW2in, 4 * kBlk);
+      bulk_load(sW2, ws + Lw.img_2, 4 * kBlk, barW2in);
+      for (int g = 0; g < n_chunks; ++g) {
+        if (g >= 1) {
+          // G(g-1) done: its ring slot takes chunk g+1
+          if (!mbar_wait(&barG[(g - 1) & 1], (uint32_t)(((g - 1) >> 1) & 1), status, abort_flag))
             break;
+          if (g + 1 < n_chunks) load_w13(g + 1);
+        }
+        const int k = g / (kF / 64);
+        if (g % (kF / 64) == 0 && k + 1 < my_tiles) {
+          // E(k+1) goes to buffer (k+1)%2, which held h2(k-1) (dead once
+          // G(k-1, 3) is done) and is the LN2 scratch of tile k: wait for h2(k)
+          if (!mbar_wait(barH2, k & 1, status, abort_flag)) break;
+          load_e(k + 1);
+        }
+      }
+    }
+  } else if (warp == kFfnEpi / 32) {
+    // MMA issuer
+    if (lane == 0 && my_tiles > 0) {
+      bool ok = mbar_wait(barW2in, 0, status, abort_flag);
+      for (int k = 0; k < my_tiles && ok; ++k) {
+        if (!(ok = mbar_wait(barH2, k & 1, status, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t a_h2 = smem_u32(sE0 + (k & 1) * 2 * kBlk);
+        const uint32_t t_out = tmem + T_OUT + (k & 1) * 128;
+        for (int c = 0; c < kF / 64; ++c) {
+          const int g = k * (kF / 64) + c, s = g & 1;
+          if (!(ok = mbar_wait(&barWt[s], (uint32_t)((g >> 1) & 1), status, abort_flag))) break;
           tc_fence_after();
-          mma_tile(tGB, smem_u32(sE), kBlk, smem_u32(sW), kBlk, 128, 128, false);
-          mma_commit(&b[kG]);
+          mma_tile(tmem + s * 128, a_h2, kBlk, smem_u32(sW13 + s * 2 * kBlk), kBlk, 128, 128, false);
+          mma_commit(&barG[s]);
           if (c >= 1) {
-            if (!(ok = mbar_wait(&b[kHid], (uint32_t)(gc - 1) & 1u, status, abort_flag))) break;
+            const int pg = g - 1, pb = pg & 1;
+            if (!(ok = mbar_wait(&barHid[pb], (uint32_t)((pg >> 1) & 1), status, abort_flag))) break;
             tc_fence_after();
-            mma_tile(tOUT, smem_u32(sH), kBlk, smem_u32(sW2 + (c - 1) * kBlk), kBlk, 128, 64, true);
-            mma_commit(&b[kW2]);
+            mma_tile(t_out, smem_u32(sH0 + pb * kBlk), kBlk, smem_u32(sW2 + (c - 1) * kBlk), kBlk,
+                     128, 64, true);
+            mma_commit(&barW2[pb]);
           }
-          // G has read the slot: the next chunk image
-          if (!(ok = mbar_wait(&b[kG], (uint32_t)gc & 1u, status, abort_flag))) break;
-          if (gc + 1 < n_chunks) load_w13(gc + 1);
         }
         if (!ok) break;
-        const int lg = j * NC + NC - 1;
-        if (!(ok = mbar_wait(&b[kHid], (uint32_t)lg & 1u, status, abort_flag))) break;
+        const int lg = k * (kF / 64) + kF / 64 - 1, lb = lg & 1;
+        if (!(ok = mbar_wait(&barHid[lb], (uint32_t)((lg >> 1) & 1), status, abort_flag))) break;
         tc_fence_after();
-        mma_tile(tOUT, smem_u32(sH), kBlk, smem_u32(sW2 + (NC - 1) * kBlk), kBlk, 128, 64, true);
-        mma_commit(&b[kW2]);
-        mma_commit(&b[kOut]);
-        // the group's next E tile, once this tile's E' staging has been read out
-        if (j + 1 < n_g) {
-          if (!(ok = mbar_wait(&b[kSE], (uint32_t)j & 1u, status, abort_flag))) break;
-          load_e(j + 1);
-        }
+        mma_tile(t_out, smem_u32(sH0 + lb * kBlk), kBlk, smem_u32(sW2 + (kF / 64 - 1) * kBlk), kBlk,
+                 128, 64, true);
+        mma_commit(&barW2[lb]);
+        mma_commit(barOut);
       }
       // drain: no MMA of ours may be in flight when TMEM is freed
-      mma_commit(&b[kDrain]);
-      mbar_wait(&b[kDrain], 0, status, abort_flag);
+      mma_commit(barDrain);
+      mbar_wait(barDrain, 0, status, abort_flag);
     }
   } else {
-    // ---- group g's epilogue (256 threads)
-    const int g = warp >> 3, wl = warp & 7;
-    const int q4 = wl & 3, half = wl >> 2;
+    const int q4 = warp & 3, part = warp >> 2;     // lane quadrant, column part
     const int row = q4 * 32 + lane;
-    const int tid = (int)threadIdx.x - g * kFfnGrp;
-    const int n_g = my_tiles > g ? (my_tiles - g + 1) / 2 : 0;
-    uint64_t* b = bar + g * 10;
-    uint8_t* sE = sE0 + g * 2 * kBlk;
-    uint8_t* sH = sH0 + g * kBlk;
     const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16);
-    const uint32_t tGB = ta + 256 * g, tOUT = tGB + 128;
-    const int c0 = half * 64;          // this thread's 64 columns of a row
+    const int c0 = part * 32;                      // this thread's 32 columns of a row
     const __half* yd = reinterpret_cast<const __half*>(ws + Lw.yd);
-    // the group's named barrier (a constant id per branch, so that only
-    // barriers 0-2 are reserved)
-    auto group_sync = [&]() {
-      if (g == 0)
-        named_bar_sync(1, kFfnGrp);
-      else
-        named_bar_sync(2, kFfnGrp);
-    };
-    for (int j = 0; j < n_g; ++j) {
-      const int4 tl = tile_of(g + 2 * j);
-      // Y = E + Yd into OUT (own 64 columns); LN2 statistics over all 128
-      mbar_wait(&b[kE], (uint32_t)j & 1u, status, abort_flag);
-      // the row's sums of (y - K) and (y - K)^2 with the shift K = the row's
-      // first value: the shifted one-pass variance loses nothing to
-      // cancellation however large the row's mean is, since |mu - K| is of
-      // the order of the row's spread
-      float K = 0.f, s1 = 0.f, s2 = 0.f;
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        float y[32];
+    // Y(j) = E + Yd into OUT[j%2], h2(j) = LN2(Y(j)) over E tile j%2.  The
+    // reduction scratch is the other E buffer: it holds h2(j-1), whose last
+    // reader G(j-1, 3) has completed by the time the epilogue gets here, and
+    // E(j+1) is loaded into it only after this tile's barH2 completes.
+    auto y_ln2 = [&](int j) {
+      uint8_t* sE = sE0 + (j & 1) * 2 * kBlk;
+      float* red1 = reinterpret_cast<float*>(sE0 + ((j & 1) ^ 1) * 2 * kBlk);
+      float* red2 = red1 + 4 * 128;
+      float y[32];
+      {
+        // Yd rows (prefetched into L2 with the E tile)
+        const int4 tl = tile_of(j);
         if (row < tl.z) {
-          const uint4* src = reinterpret_cast<const uint4*>(yd + (int64_t)(tl.y + row) * kD + p * 32);
+          const uint4* src = reinterpret_cast<const uint4*>(yd + (int64_t)(tl.y + row) * kD + c0);
 #pragma unroll
           for (int q = 0; q < 4; ++q) unpack8_f16(src[q], y + q * 8);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) y[i] = 0.f;
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float e[8];
-          unpack8(sw_ld16(sE, kBlk, row, p * 32 + q * 8), e);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) y[q * 8 + i] += e[i];
-        }
-        if (p == 0) K = y[0];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float t = y[i] - K;
-          s1 += t;
-          s2 = fmaf(t, t, s2);
-        }
-        if ((p >> 1) == half) {
-          tmem_st16(tOUT + p * 32, y);
-          tmem_st16(tOUT + p * 32 + 16, y + 16);
-        }
       }
-      const float ms = s1 * (1.0f / kD);
-      const float mu = K + ms;
-      const float rstd = rsqrtf(fmaxf(s2 * (1.0f / kD) - ms * ms, 0.f) + kLnEps);
-      tmem_st_wait();
-      group_sync();   // every thread of the group has read the E tile
+      mbar_wait(&barE[j & 1], (uint32_t)((j >> 1) & 1), status, abort_flag);
 #pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        const int cc = c0 + p * 32;
-        float y[32];
-        tmem_ld16(tOUT + cc, y);
-        tmem_ld16(tOUT + cc + 16, y + 16);
-        tmem_ld_wait();
+      for (int q = 0; q < 4; ++q) {
+        float e[8];
+        unpack8(sw_ld16(sE, kBlk, row, c0 + q * 8), e);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 gv = reinterpret_cast<const float4*>(sg + cc)[q];
-          const float4 bv = reinterpret_cast<const float4*>(sg + kD + cc)[q];
-          y[4 * q] = (y[4 * q] - mu) * rstd * gv.x + bv.x;
-          y[4 * q + 1] = (y[4 * q + 1] - mu) * rstd * gv.y + bv.y;
-          y[4 * q + 2] = (y[4 * q + 2] - mu) * rstd * gv.z + bv.z;
-          y[4 * q + 3] = (y[4 * q + 3] - mu) * rstd * gv.w + bv.w;
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) sw_st16(sE, kBlk, row, cc + q * 8, pack8(y + q * 8));
+        for (int i = 0; i < 8; ++i) y[q * 8 + i] += e[i];
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&b[kH2]);
-      // hidden chunks: this thread's 32 of the chunk's 64 hidden units
-      for (int c = 0; c < NC; ++c) {
-        const int gc = j * NC + c;
-        mbar_wait(&b[kG], (uint32_t)gc & 1u, status, abort_flag);
-        tc_fence_after();
-        float h[32];
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          float gt[16], gu[16];
-          tmem_ld16(tGB + half * 32 + p * 16, gt);
-          tmem_ld16(tGB + 64 + half * 32 + p * 16, gu);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) h[p * 16 + i] = silu_tanh(gt[i]) * gu[i];
-        }
-        tc_fence_before();
-        mbar_arrive(&b[kGBf]);           // GB may take the next chunk's gates
-        // the chunk buffer held the previous chunk: its W2 product must be done
-        if (gc >= 1) mbar_wait(&b[kW2], (uint32_t)(gc - 1) & 1u, status, abort_flag);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) sw_st16(sH, kBlk, row, half * 32 + q * 8, pack8(h + q * 8));
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&b[kHid]);
+      const uint32_t t_out = ta + T_OUT + (j & 1) * 128 + c0;
+      tmem_st16(t_out, y);
+      tmem_st16(t_out + 16, y + 16);
+      {
+        float pm, pq;
+        part_stats(y, pm, pq);
+        red1[part * 128 + row] = pm;
+        red2[part * 128 + row] = pq;
       }
-      // E' = OUT -> bf16, staged over the E tile (every product of the tile,
-      // the gate products reading h2 included, is done), then coalesced stores
-      mbar_wait(&b[kOut], (uint32_t)j & 1u, status, abort_flag);
-      tc_fence_after();
-#pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        const int cc = c0 + p * 32;
-        float o[32];
-        tmem_ld16(tOUT + cc, o);
-        tmem_ld16(tOUT + cc + 16, o + 16);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < 4; ++q) sw_st16(sE, kBlk, row, cc + q * 8, pack8(o + q * 8));
-      }
-      tc_fence_before();
-      group_sync();
+      named_bar_sync(1, kFfnEpi);
+      float mu, rstd;
+      merge4_stats(red1[row], red1[128 + row], red1[256 + row], red1[384 + row], red2[row],
+                   red2[128 + row], red2[256 + row], red2[384 + row], mu, rstd);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        const int idx = q * kFfnGrp + tid, r = idx >> 4, cc = idx & 15;
-        if (r < tl.z)
-          reinterpret_cast<uint4*>(E_out + (int64_t)(tl.y + r) * kD)[cc] = sw_ld16(sE, kBlk, r, cc * 8);
+        const float4 gv = reinterpret_cast<const float4*>(sg + c0)[q];
+        const float4 bv = reinterpret_cast<const float4*>(sg + kD + c0)[q];
+        y[4 * q] = (y[4 * q] - mu) * rstd * gv.x + bv.x;
+        y[4 * q + 1] = (y[4 * q + 1] - mu) * rstd * gv.y + bv.y;
+        y[4 * q + 2] = (y[4 * q + 2] - mu) * rstd * gv.z + bv.z;
+        y[4 * q + 3] = (y[4 * q + 3] - mu) * rstd * gv.w + bv.w;
       }
-      // the staging has been read: the E buffer may take the group's next tile
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sw_st16(sE, kBlk, row, c0 + q * 8, pack8(y + q * 8));
+      tmem_st_wait();
       fence_proxy_async_smem();
-      mbar_arrive(&b[kSE]);
+      tc_fence_before();
+      mbar_arrive(barH2);
+    };
+    if (my_tiles > 0) y_ln2(0);
+    for (int k = 0; k < my_tiles; ++k) {
+      for (int c = 0; c < kF / 64; ++c) {
+        const int g = k * (kF / 64) + c, sb = g & 1;
+        mbar_wait(&barG[sb], (uint32_t)((g >> 1) & 1), status, abort_flag);
+        tc_fence_after();
+        float gt[16], gu[16];
+        tmem_ld16(ta + sb * 128 + part * 16, gt);
+        tmem_ld16(ta + sb * 128 + 64 + part * 16, gu);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) gt[i] = silu_tanh(gt[i]) * gu[i];
+        // hid(g) reuses the buffer of hid(g-2): wait until its W2 MMA is done
+        if (g >= 2) mbar_wait(&barW2[sb], (uint32_t)(((g - 2) >> 1) & 1), status, abort_flag);
+        uint8_t* sH = sH0 + sb * kBlk;
+        sw_st16(sH, kBlk, row, part * 16, pack8(gt));
+        sw_st16(sH, kBlk, row, part * 16 + 8, pack8(gt + 8));
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&barHid[sb]);
+      }
+      if (k + 1 < my_tiles) y_ln2(k + 1);
+      mbar_wait(barOut, (uint32_t)(k & 1), status, abort_flag);
+      tc_fence_after();
+      // E' = OUT -> bf16, staged in the hid buffers (every W2 product of the
+      // tile is done, and the next hid is written by these threads after the
+      // copy) and written with coalesced 16-byte stores
+      {
+        float o[32];
+        tmem_ld16(ta + T_OUT + (k & 1) * 128 + c0, o);
+        tmem_ld16(ta + T_OUT + (k & 1) * 128 + c0 + 16, o + 16);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sw_st16(sH0, kBlk, row, c0 + q * 8, pack8(o + q * 8));
+      }
+      tc_fence_before();
+      named_bar_sync(1, kFfnEpi);
+      {
+        const int4 tl = tile_of(k);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int idx = q * kFfnEpi + (int)threadIdx.x, r = idx >> 4, cc = idx & 15;
+          if (r < tl.z)
+            reinterpret_cast<uint4*>(E_out + (int64_t)(tl.y + r) * kD)[cc] = sw_ld16(sH0, kBlk, r, cc * 8);
+        }
+      }
+      named_bar_sync(1, kFfnEpi);
     }
   }
   tc_fence_before();

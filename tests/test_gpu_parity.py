@@ -64,12 +64,18 @@ def check_workload(w, n_hist=None, n_cand=None, check_e2e=True, hist_shift=0.0):
     assert_close(Z0_gpu, Z0_ref, dt, "context links")
     # each layer in isolation
     E_prev, Z_prev = f64(us.E), f64(Z0_gpu)
+    # phi = SiLU: signed pointwise weights turn the bf16 roundings of the
+    # attention operands into a second rounding stage of a layer's outputs
+    # (measured: E' up to 2.02e-2 over the per-element storage slack, link rows
+    # up to 2.31e-2 max-abs on one-row histories, rel-L2 at most 3.3e-3)
+    silu = w.phi == "silu"
     for i, (E_out, Z_out) in enumerate(outs):
         E_ref, Z_ref = O.xor_layer(E_prev, offs, Z_prev, layers[i], w.H, phi=w.phi,
                                    window=w.window)
-        assert_close(Z_out, Z_ref, dt, f"layer {i} links")
+        assert_close(Z_out, Z_ref, dt, f"layer {i} links", storage=silu, stages=2 if silu else 1)
         if E_out is not None:
-            assert_close(E_out, E_ref, dt, f"layer {i} history", storage=True)
+            assert_close(E_out, E_ref, dt, f"layer {i} history", storage=True,
+                         stages=2 if silu else 1)
             E_prev = f64(E_out)
         Z_prev = f64(Z_out)
     # end to end user side: a chain of the context-link and layer stores

@@ -168,10 +168,19 @@ def score(x: DeviceInputs, buf: Buffers, LP: torch.Tensor, stream=None):
 
 
 def step(x: DeviceInputs, buf: Buffers, stream=None) -> torch.Tensor:
-    """One pass of the whole hot path; returns O [sum M, d]."""
+    """One pass of the whole hot path, cache build included; returns O [sum M, d]."""
     fold_qk(x, buf, stream)
     LP = user_encode(x, buf, stream)
     build_cache(x, buf, stream)
+    score(x, buf, LP, stream)
+    return buf.O
+
+
+def online_step(x: DeviceInputs, buf: Buffers, stream=None) -> torch.Tensor:
+    """The per-request part of the path: context links, the layer stack and
+    cached scoring against the QK cache already in ``buf.cache`` (built offline
+    over the catalogue: LIME note, 整体框架); returns O [sum M, d]."""
+    LP = user_encode(x, buf, stream)
     score(x, buf, LP, stream)
     return buf.O
 
@@ -202,6 +211,19 @@ def step_graphs(x: DeviceInputs, buf: Buffers):
     return g_step, g_user, g_cache, g_score
 
 
+def online_graphs(x: DeviceInputs, buf: Buffers):
+    """CUDA graphs of the online step and its parts: (online step, user side,
+    scoring, cache build).  The cache graph is the whole offline build (fold
+    and catalogue pass); the others read the cache it left."""
+    LP = buf.Z_bufs[(len(x.layers) - 1) % 2]
+    g_online = capture(lambda: online_step(x, buf))
+    g_user = capture(lambda: user_encode(x, buf))
+    g_score = capture(lambda: score(x, buf, LP))
+    g_cache = capture(lambda: lime.lime_build_qk_cache(x.dims, x.T, x.L, x.Wq_c, x.Wk_c,
+                                                       buf.cache, buf.ws))
+    return g_online, g_user, g_score, g_cache
+
+
 # Per-request inputs of a step: what changes from one batch of users to the
 # next (the weights, the global links and the item table stay resident).
 REQUEST_FIELDS = ("E", "ctx", "hist_offsets", "cand_ids", "cand_offsets")
@@ -212,7 +234,8 @@ class HostPipeline:
 
     ``submit(host, O_host)`` copies one batch's per-request inputs (a dict of
     pinned CPU tensors keyed by ``REQUEST_FIELDS``, shaped as the device
-    inputs) to the device on a copy stream, runs ``step`` on the caller's
+    inputs) to the device on a copy stream, runs ``step`` (or ``online_step``
+    when built with ``online=True``) on the caller's
     current stream and copies the scores back into the pinned ``O_host`` on a
     second copy stream.  Consecutive submissions alternate between two slots
     (inputs and output buffer), so while step k computes, the inputs of step
@@ -225,7 +248,9 @@ class HostPipeline:
     on the host once ``drain`` has been called and ``stream`` synchronised.
     """
 
-    def __init__(self, x: DeviceInputs, buf: Buffers):
+    def __init__(self, x: DeviceInputs, buf: Buffers, online: bool = False):
+        # online=True runs online_step (the cache in buf.cache stays as built)
+        self.run = online_step if online else step
         self.slots = []
         for s in range(2):
             if s == 0:
@@ -261,7 +286,7 @@ class HostPipeline:
         main.wait_event(self.inputs_ready[s])
         main.wait_event(self.output_free[s])
         with torch.cuda.stream(main):
-            out = step(xs, bs)
+            out = self.run(xs, bs)
         self.inputs_free[s].record(main)
         # scores out
         self.d2h.wait_event(self.inputs_free[s])

@@ -20,11 +20,16 @@ def test_reference_arm_prints_one_contract_line():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference"
-    assert d["metric"] == "user-candidate pairs scored/s (full LIME step)"
+    import bench
+    assert d["metric"] == bench.METRIC
     assert d["unit"] == "pairs/s" and d["higher_is_better"] is True
     assert d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 3
     assert d["value"] > 0 and d["ms_per_step"] > 0
     assert d["config"]["workload"].startswith("tiny:")
+    # the same config dict as the library arm of the same workload
+    assert d["config"] == bench.config_of(bench.case_workload("tiny"))
+    # steps really timed: the sampled seconds cover steps x ms_per_step
+    assert d["sampled_seconds"] >= 0.99 * d["steps"] * d["ms_per_step"] / 1e3
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"]
     assert cb["value"] == d["value"]

@@ -224,10 +224,117 @@ __global__ void __launch_bounds__(CacheCfg<HL, L, U8>::THREADS, 1)
     constexpr int HPW = H / C::WPQ < 1 ? 1 : H / C::WPQ;   // heads per epilogue warp
     const int row = quad * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    // softmax (or SiLU) of head h of this thread's row, into the staging tile
+    auto emit_head = [&](int h, uint32_t acc, uint8_t* stage) {
+      float z[L];
+#pragma unroll
+      for (int q = 0; q < L / 16; ++q)
+        tmem_ld16(tmem + lane_base + acc * HL + h * L + q * 16, z + q * 16);
+      tmem_ld_wait();
+      float inv;
+      if constexpr (SILU) {
+        // SiLU of each score over the l links (the int8 cache is softmax only)
+#pragma unroll
+        for (int k = 0; k < L; ++k) z[k] = __fdividef(z[k], 1.0f + __expf(-z[k]));
+        inv = 1.0f / L;
+      } else {
+        float m = z[0];
+#pragma unroll
+        for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
+        float ssum = 0.f;
+#pragma unroll
+        for (int k = 0; k < L; ++k) {
+          z[k] = __expf(z[k] - m);
+          ssum += z[k];
+        }
+        inv = 1.0f / ssum;
+      }
+      if constexpr (U8) {
+        // bytes q = round(255 w), ties to even; 16 per 16-byte chunk of the
+        // row's 128-byte swizzled block
+        const float sc = inv * 255.0f;
+#pragma unroll
+        for (int c = 0; c < L / 16; ++c) {
+          const int bcol = h * L + c * 16;
+          // z <= 1 and sum >= 1, so 255 z / sum rounds to at most 255.  Adding
+          // 1.5 * 2^23 in the same FMA rounds the product to an integer (ties
+          // to even) in the low mantissa bits: the low byte is q.
+          uint32_t wv[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float* zz = z + c * 16 + j * 4;
+            const uint32_t q0 = __float_as_uint(fmaf(zz[0], sc, 12582912.0f));
+            const uint32_t q1 = __float_as_uint(fmaf(zz[1], sc, 12582912.0f));
+            const uint32_t q2 = __float_as_uint(fmaf(zz[2], sc, 12582912.0f));
+            const uint32_t q3 = __float_as_uint(fmaf(zz[3], sc, 12582912.0f));
+            wv[j] = __byte_perm(__byte_perm(q0, q1, 0x0040), __byte_perm(q2, q3, 0x0040), 0x5410);
+          }
+          *reinterpret_cast<uint4*>(stage + (bcol >> 7) * (kBM * 128) + row * 128 +
+                                    ((((bcol & 127) >> 4) ^ (row & 7)) << 4)) =
+              make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < L / 8; ++c) {
+          const int col = h * L + c * 8;
+          uint4 v;
+          v.x = pack_bf16(z[c * 8 + 0] * inv, z[c * 8 + 1] * inv);
+          v.y = pack_bf16(z[c * 8 + 2] * inv, z[c * 8 + 3] * inv);
+          v.z = pack_bf16(z[c * 8 + 4] * inv, z[c * 8 + 5] * inv);
+          v.w = pack_bf16(z[c * 8 + 6] * inv, z[c * 8 + 7] * inv);
+          *reinterpret_cast<uint4*>(stage + (col >> 6) * (kBM * 128) + sw128_offset(row, col & 63)) = v;
+        }
+      }
+    };
+    // HL = 256 with bf16 weights leaves room for one 64 KB staging tile only;
+    // it is written and stored in two halves (the first half of the heads,
+    // then the second), so that one half's TMA store overlaps the other
+    // half's softmax instead of draining before the next tile may start.
+    constexpr bool SPLIT = C::OUTB == 1;
+    static_assert(!SPLIT || (HPW == 2 && C::WPQ * L == HL / 2), "two passes of one head each");
+    constexpr int per_box = U8 ? 128 : 64;   // 128-byte-wide boxes: 64 bf16 or 128 bytes
     int it = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
+      if constexpr (SPLIT) {
+        // ofull[p] / ofree[p]: half p of the staging tile written / its store
+        // has read it (each completes once per tile)
+        const uint32_t prev = (uint32_t)(it - 1) & 1u;
+        if (it > 0 && !mbar_wait(&ofree[0], prev, status, &abort_flag)) break;
+        if (!mbar_wait(&tfull[acc], aph, status, &abort_flag)) break;
+        tc_fence_after();
+        emit_head(grp, acc, sO);
+        fence_proxy_async_smem();
+        mbar_arrive(&ofull[0]);
+        if (et == 0) {
+          if (!mbar_wait(&ofull[0], (uint32_t)it & 1u, status, &abort_flag)) break;
+#pragma unroll
+          for (int b = 0; b < HL / per_box / 2; ++b)
+            tma_store_2d(&tmC, sO + b * (kBM * 128), b * per_box, tile * kBM);
+          bulk_commit();
+          if (it > 0) {
+            bulk_wait_read<1>();   // the previous tile's second half has been read
+            mbar_arrive(&ofree[1]);
+          }
+        }
+        if (it > 0 && !mbar_wait(&ofree[1], prev, status, &abort_flag)) break;
+        emit_head(grp + C::WPQ, acc, sO);
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+        fence_proxy_async_smem();
+        mbar_arrive(&ofull[1]);
+        if (et == 0) {
+          if (!mbar_wait(&ofull[1], (uint32_t)it & 1u, status, &abort_flag)) break;
+#pragma unroll
+          for (int b = HL / per_box / 2; b < HL / per_box; ++b)
+            tma_store_2d(&tmC, sO + b * (kBM * 128), b * per_box, tile * kBM);
+          bulk_commit();
+          bulk_wait_read<1>();     // this tile's first half has been read
+          mbar_arrive(&ofree[0]);
+        }
+        continue;
+      }
       const int ob = C::OUTB == 2 ? (it & 1) : 0;
       const uint32_t oph = (it / C::OUTB) & 1;
       if (!mbar_wait(&ofree[ob], oph ^ 1, status, &abort_flag)) break;
@@ -235,75 +342,13 @@ __global__ void __launch_bounds__(CacheCfg<HL, L, U8>::THREADS, 1)
       tc_fence_after();
       uint8_t* stage = sO + ob * C::O_BYTES;
 #pragma unroll 1
-      for (int h = grp * HPW; h < (grp + 1) * HPW && h < H; ++h) {
-        float z[L];
-#pragma unroll
-        for (int q = 0; q < L / 16; ++q)
-          tmem_ld16(tmem + lane_base + acc * HL + h * L + q * 16, z + q * 16);
-        tmem_ld_wait();
-        float inv;
-        if constexpr (SILU) {
-          // SiLU of each score over the l links (the int8 cache is softmax only)
-#pragma unroll
-          for (int k = 0; k < L; ++k) z[k] = __fdividef(z[k], 1.0f + __expf(-z[k]));
-          inv = 1.0f / L;
-        } else {
-          float m = z[0];
-#pragma unroll
-          for (int k = 1; k < L; ++k) m = fmaxf(m, z[k]);
-          float ssum = 0.f;
-#pragma unroll
-          for (int k = 0; k < L; ++k) {
-            z[k] = __expf(z[k] - m);
-            ssum += z[k];
-          }
-          inv = 1.0f / ssum;
-        }
-        if constexpr (U8) {
-          // bytes q = round(255 w), ties to even; 16 per 16-byte chunk of the
-          // row's 128-byte swizzled block
-          const float sc = inv * 255.0f;
-#pragma unroll
-          for (int c = 0; c < L / 16; ++c) {
-            const int bcol = h * L + c * 16;
-            // z <= 1 and sum >= 1, so 255 z / sum rounds to at most 255.  Adding
-            // 1.5 * 2^23 in the same FMA rounds the product to an integer (ties
-            // to even) in the low mantissa bits: the low byte is q.
-            uint32_t wv[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float* zz = z + c * 16 + j * 4;
-              const uint32_t q0 = __float_as_uint(fmaf(zz[0], sc, 12582912.0f));
-              const uint32_t q1 = __float_as_uint(fmaf(zz[1], sc, 12582912.0f));
-              const uint32_t q2 = __float_as_uint(fmaf(zz[2], sc, 12582912.0f));
-              const uint32_t q3 = __float_as_uint(fmaf(zz[3], sc, 12582912.0f));
-              wv[j] = __byte_perm(__byte_perm(q0, q1, 0x0040), __byte_perm(q2, q3, 0x0040), 0x5410);
-            }
-            *reinterpret_cast<uint4*>(stage + (bcol >> 7) * (kBM * 128) + row * 128 +
-                                      ((((bcol & 127) >> 4) ^ (row & 7)) << 4)) =
-                make_uint4(wv[0], wv[1], wv[2], wv[3]);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < L / 8; ++c) {
-            const int col = h * L + c * 8;
-            uint4 v;
-            v.x = pack_bf16(z[c * 8 + 0] * inv, z[c * 8 + 1] * inv);
-            v.y = pack_bf16(z[c * 8 + 2] * inv, z[c * 8 + 3] * inv);
-            v.z = pack_bf16(z[c * 8 + 4] * inv, z[c * 8 + 5] * inv);
-            v.w = pack_bf16(z[c * 8 + 6] * inv, z[c * 8 + 7] * inv);
-            *reinterpret_cast<uint4*>(stage + (col >> 6) * (kBM * 128) + sw128_offset(row, col & 63)) = v;
-          }
-        }
-      }
+      for (int h = grp * HPW; h < (grp + 1) * HPW && h < H; ++h) emit_head(h, acc, stage);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       fence_proxy_async_smem();
       mbar_arrive(&ofull[ob]);
       if (et == 0) {
         if (!mbar_wait(&ofull[ob], oph, status, &abort_flag)) break;
-        // 128-byte-wide boxes: 64 bf16 or 128 bytes of the cache row
-        constexpr int per_box = U8 ? 128 : 64;
 #pragma unroll
         for (int b = 0; b < HL / per_box; ++b)
           tma_store_2d(&tmC, stage + b * (kBM * 128), b * per_box, tile * kBM);

@@ -7,7 +7,9 @@ scoring; the cache is built once first), ``score_scale`` (cached scoring of
 16 users x 65,536 candidate IDs drawn uniformly from the whole catalogue, so
 the gathered rows far exceed L2), ``layer`` (one LIME-XOR layer, the
 first of the stack, with history outputs), ``last`` (the last-layer variant
-without history outputs), ``step`` (the whole pass).  Inputs are the seeded
+without history outputs), ``step`` (the whole pass), ``online`` (the online
+step: context links, the layer stack and cached scoring against a cache built
+once beforehand).  Inputs are the seeded
 synthetic workloads of ``synth``; ``--items`` and ``--users`` shrink them.
 """
 from __future__ import annotations
@@ -21,10 +23,11 @@ from . import lime, pipeline, synth
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--phase", default="cache", choices=["cache", "score", "score_scale", "layer", "last", "step"])
+    ap.add_argument("--phase", default="cache", choices=["cache", "score", "score_scale", "layer", "last", "step", "online"])
     ap.add_argument("--workload", default="standard")
     ap.add_argument("--items", type=int, default=None)
     ap.add_argument("--users", type=int, default=None)
+    ap.add_argument("--links", type=int, default=None)
     ap.add_argument("--reps", type=int, default=3)
     a = ap.parse_args()
     over = {}
@@ -32,6 +35,8 @@ def main():
         over["n_items"] = a.items
     if a.users:
         over["B"] = a.users
+    if a.links:
+        over["l"] = a.links
     w = synth.workload(a.workload, **over)
     us, cs = synth.user_side(w), synth.candidate_side(w)
     x = pipeline.to_device(w, us, cs, synth.item_table(w))
@@ -41,7 +46,7 @@ def main():
         lime.lime_context_links(x.dims, x.L, x.ctx, *x.ctx_w, buf.LC, buf.ws)
     else:
         Z = x.Z0
-    if a.phase in ("score", "score_scale"):
+    if a.phase in ("score", "score_scale", "online"):
         pipeline.build_cache(x, buf)
     if a.phase == "score_scale":
         users, per = 16, 65536
@@ -64,6 +69,8 @@ def main():
         elif a.phase == "last":
             lime.lime_xor_layer(x.dims, x.hist_offsets, x.total_hist, x.E, Z, x.layers[-1],
                                 None, buf.Z_bufs[0], buf.ws)
+        elif a.phase == "online":
+            pipeline.online_step(x, buf)
         else:
             pipeline.step(x, buf)
     torch.cuda.synchronize()

@@ -1,5 +1,5 @@
 // Uncached (online) candidate scoring on the 5th-generation tensor cores
-// (bf16, d = 128, 4 heads of 32, l in {16, 32}).
+// (bf16, d = 128, 4 heads of 32, l in {16, 32, 64}).
 //
 // LIME note, 关键设计 1: O_m = MHA(T_m, L, L^P), whose weights phi(T_m L^T)
 // depend only on the item and the global links.  Cached scoring reads them
@@ -16,10 +16,12 @@
 //            scoring (TMEM [128, 256))
 //   out      O rows in bf16 through the same stage, coalesced 16-byte stores.
 // CTA (u, g) walks tiles g, g + G, ... of user u's candidates with four
-// warpgroups that take turns (tile j of the CTA goes to group j % 4): each has
-// its own gather stage, 128 TMEM columns (S, then O over it) and MMA barrier,
-// so the groups' gathers, MMAs and softmaxes overlap one another.  Thread =
-// candidate row (a TMEM lane) within its group.
+// warpgroups (two for l = 64) that take turns (tile j of the CTA goes to
+// group j % groups): each has its own gather stage, H*l TMEM columns (S, then
+// O over it) and MMA barrier, so the groups' gathers, MMAs and softmaxes
+// overlap one another.  With l = 64 a stage is 64 KB, since the [128 x 256]
+// bf16 weights overwrite the gathered rows.  Thread = candidate row (a TMEM
+// lane) within its group.
 // An out-of-range ID gives a zero row of T (so uniform weights) and
 // LIME_FLAG_BAD_ID; its O row is written as zero.  No workspace is used.
 #include "lime_fast.cuh"
@@ -37,24 +39,26 @@ constexpr uint32_t kBlk = 128 * 128;
 template <int L>
 struct OnlineCfg {
   static constexpr int HL = kH * L;
-  static constexpr uint32_t kStage = 2 * kBlk;         // [128 x 128] bf16 gather stage
-  static constexpr uint32_t OFF_B = 4 * kStage;        // L^P_u^T (after 4 groups' stages)
+  static constexpr int GROUPS = HL > 128 ? 2 : 4;      // warpgroups (HL TMEM columns each)
+  static constexpr int THREADS = 128 * GROUPS;
+  static constexpr uint32_t TCOLS = HL > 128 ? 256 : 128;   // TMEM columns per group
+  // a gather stage: the [128 x 128] bf16 item rows, later the [128 x HL] weights
+  static constexpr uint32_t kStage = (HL > 128 ? HL / 64 : 2) * kBlk;
+  static constexpr uint32_t OFF_B = GROUPS * kStage;   // L^P_u^T (after the groups' stages)
   static constexpr uint32_t OFF_G = OFF_B + kBlk;      // G image: 2 blocks of HL x 128 bytes
   static constexpr uint32_t OFF_BAR = OFF_G + 2 * HL * 128;
   static constexpr int SMEM = 1024 + OFF_BAR + 64 + 4 * 128 * 4;
 };
 
-constexpr int kGroups = 4;
-constexpr int kOnThreads = 128 * kGroups;
-
 template <int L>
-__global__ void __launch_bounds__(kOnThreads, 1)
+__global__ void __launch_bounds__(OnlineCfg<L>::THREADS, 1)
     k_score_online(const bf16* __restrict__ T, int64_t n_items, const uint8_t* __restrict__ gimg,
                    const int32_t* __restrict__ ids, const int64_t* __restrict__ off, int64_t B,
                    int64_t total, const bf16* __restrict__ LP, bf16* __restrict__ O, int phi,
                    unsigned* status) {
   using C = OnlineCfg<L>;
   constexpr int HL = C::HL;
+  constexpr int kGroups = C::GROUPS, kOnThreads = C::THREADS;
   constexpr int CH = 2 * kD / 16;            // 16-byte chunks per item row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -109,7 +113,7 @@ __global__ void __launch_bounds__(kOnThreads, 1)
   fence_proxy_async_smem();
   __syncthreads();   // sB is complete and the staging stage is free again
   mbar_wait(&bar[kGroups], 0, status, abort_flag);   // the G image
-  const uint32_t tmem = *slot + (uint32_t)grp * 128;   // this group's S, then O
+  const uint32_t tmem = *slot + (uint32_t)grp * C::TCOLS;   // this group's S, then O
   const uint32_t ta = tmem + ((uint32_t)(i & ~31) << 16);
   const int G = (int)gridDim.y;
   const int step = kGroups * G;              // a group's stride over the user's tiles
@@ -248,6 +252,7 @@ template <int L>
 int launch_online(int64_t B, const void* T, int64_t n_items, const void* image, const int32_t* ids,
                   const int64_t* off, int64_t total, const void* LP, void* O, int phi,
                   unsigned* status, cudaStream_t st) {
+  constexpr int kOnThreads = OnlineCfg<L>::THREADS;
   using C = OnlineCfg<L>;
   if (cudaFuncSetAttribute(k_score_online<L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::SMEM) != cudaSuccess)
@@ -267,7 +272,7 @@ int launch_online(int64_t B, const void* T, int64_t n_items, const void* image, 
 }  // namespace
 
 bool fast_online_supported(const lime_dims& D) {
-  return D.dtype == LIME_BF16 && D.d == kD && D.H == kH && (D.l == 16 || D.l == 32);
+  return D.dtype == LIME_BF16 && D.d == kD && D.H == kH && (D.l == 16 || D.l == 32 || D.l == 64);
 }
 
 int fast_score_online(const lime_dims& D, int64_t B, const void* T, int64_t n_items,
@@ -275,6 +280,8 @@ int fast_score_online(const lime_dims& D, int64_t B, const void* T, int64_t n_it
                       const void* LP, void* O, unsigned* status, cudaStream_t st) {
   if (D.l == 16)
     return launch_online<16>(B, T, n_items, image, ids, off, total, LP, O, D.phi, status, st);
+  if (D.l == 64)
+    return launch_online<64>(B, T, n_items, image, ids, off, total, LP, O, D.phi, status, st);
   return launch_online<32>(B, T, n_items, image, ids, off, total, LP, O, D.phi, status, st);
 }
 

@@ -150,7 +150,7 @@ def test_host_validation_of_uncached_scoring(lime):
     assert f(*args(image=0x200008)) == lime.LIME_ERR_ARG                    # unaligned
     assert f(*args(O=0x100000 + 512)) == lime.LIME_ERR_ALIAS               # O inside T
     assert f(*args(O=0x200000)) == lime.LIME_ERR_ALIAS                     # O over the image
-    assert f(*args(dims=lime.make_dims(128, 4, 64, 256, 64, "bf16"))) == lime.LIME_ERR_SHAPE
+    assert f(*args(dims=lime.make_dims(128, 4, 8, 256, 64, "bf16"))) == lime.LIME_ERR_SHAPE
     assert f(*args(dims=lime.make_dims(128, 4, 32, 256, 64, "f32"))) == lime.LIME_ERR_SHAPE
 
 

@@ -45,7 +45,8 @@ def _run(l, n_cand, n_items=20_000, bad=(), phi="softmax"):
 
 
 @pytest.mark.parametrize("phi", ["softmax", "silu"])
-@pytest.mark.parametrize("l,n_cand", [(32, [5, 0, 300, 128]), (16, [257, 1, 0, 3])])
+@pytest.mark.parametrize("l,n_cand", [(32, [5, 0, 300, 128]), (16, [257, 1, 0, 3]),
+                                      (64, [130, 0, 1, 513])])
 def test_uncached_scoring_matches_direct_attention(l, n_cand, phi):
     w, us, cs, T, LP, ids, Od, flags = _run(l, n_cand, phi=phi)
     assert flags == 0
@@ -60,11 +61,12 @@ def test_uncached_scoring_matches_direct_attention(l, n_cand, phi):
     assert_close(Od, ref, "bf16", "uncached scoring")
 
 
-def test_uncached_scoring_many_tiles_and_bad_ids():
+@pytest.mark.parametrize("l", [32, 64])
+def test_uncached_scoring_many_tiles_and_bad_ids(l):
     # one user with many tiles (each CTA walks several), bad IDs -> zero rows + flag
     n_cand = [3000, 200]
     bad = (7, 130, 3100)
-    w, us, cs, T, LP, ids, Od, flags = _run(32, n_cand, bad=bad)
+    w, us, cs, T, LP, ids, Od, flags = _run(l, n_cand, bad=bad)
     assert flags & lime.LIME_FLAG_BAD_ID
     offs = cs.cand_offsets.numpy()
     got = Od.cpu()

@@ -165,7 +165,7 @@ int lime_build_qk_cache_folded(const lime_dims* dims, const void* T, int64_t n_i
  *            dims, L, Wq_c, Wk_c (lime_qk_image_bytes(dims) bytes).
  * Other arguments, checks, flags and errors as lime_score_candidates (an
  * out-of-range ID sets LIME_FLAG_BAD_ID and its row of O is zero).
- * Supported: bf16, d = 128, H = 4, l in {16, 32} (else LIME_ERR_SHAPE).    */
+ * Supported: bf16, d = 128, H = 4, l in {16, 32, 64} (else LIME_ERR_SHAPE). */
 int lime_score_candidates_uncached(const lime_dims* dims, int64_t B, const void* T,
                                    int64_t n_items, const void* image, const int32_t* cand_ids,
                                    const int64_t* cand_offsets, int64_t total_cand, const void* LP,
@@ -264,7 +264,8 @@ int lime_score_candidates(const lime_dims* dims, int64_t B, const void* cache,
  * weight computed in fp32 (ties to even; w lies in [0, 1]); dequantised as
  * q / 255.  Same arguments, checks and errors as lime_build_qk_cache, with
  *   cache_out device uint8 [n_items, H, l] (16-byte aligned).
- * Supported: bf16, d = 128, H*l >= 128 (else LIME_ERR_SHAPE).            */
+ * Supported: bf16, d = 128, H = 4 with l in {16, 32, 64}, or H*l = 256     *
+ * (else LIME_ERR_SHAPE).                                                  */
 int lime_build_qk_cache_u8(const lime_dims* dims, const void* T, int64_t n_items,
                            const void* L, const void* Wq_c, const void* Wk_c,
                            uint8_t* cache_out, void* workspace, size_t workspace_bytes,

@@ -269,9 +269,12 @@ __global__ void __launch_bounds__(CacheCfg<HL, L, U8>::THREADS, 1)
             const uint32_t q3 = __float_as_uint(fmaf(zz[3], sc, 12582912.0f));
             wv[j] = __byte_perm(__byte_perm(q0, q1, 0x0040), __byte_perm(q2, q3, 0x0040), 0x5410);
           }
-          *reinterpret_cast<uint4*>(stage + (bcol >> 7) * (kBM * 128) + row * 128 +
-                                    ((((bcol & 127) >> 4) ^ (row & 7)) << 4)) =
-              make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          // 64-byte rows (H*l = 64) are staged row-major without swizzle;
+          // 128-byte boxes of wider rows in the 128-byte swizzle
+          uint8_t* dst = HL == 64 ? stage + row * 64 + (bcol >> 4) * 16
+                                  : stage + (bcol >> 7) * (kBM * 128) + row * 128 +
+                                        ((((bcol & 127) >> 4) ^ (row & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
       } else {
 #pragma unroll
@@ -292,7 +295,8 @@ __global__ void __launch_bounds__(CacheCfg<HL, L, U8>::THREADS, 1)
     // half's softmax instead of draining before the next tile may start.
     constexpr bool SPLIT = C::OUTB == 1;
     static_assert(!SPLIT || (HPW == 2 && C::WPQ * L == HL / 2), "two passes of one head each");
-    constexpr int per_box = U8 ? 128 : 64;   // 128-byte-wide boxes: 64 bf16 or 128 bytes
+    // 128-byte-wide boxes: 64 bf16 or 128 bytes (one 64-byte box for H*l = 64 bytes)
+    constexpr int per_box = U8 ? (HL == 64 ? 64 : 128) : 64;
     int it = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
@@ -378,7 +382,9 @@ int launch_cache(const void* T, int64_t n, const bf16* img, void* cache, int til
   using C = CacheCfg<HL, L, U8>;
   CUtensorMap tmT, tmC;
   if (!make_tmap_2d_bf16(&tmT, T, kD, (uint64_t)n, kD * 2, 64, kBM)) return LIME_ERR_CUDA;
-  if (U8) {
+  if (U8 && HL == 64) {
+    if (!make_tmap_2d_u8_plain(&tmC, cache, HL, (uint64_t)n, HL, 64, kBM)) return LIME_ERR_CUDA;
+  } else if (U8) {
     if (!make_tmap_2d_u8(&tmC, cache, HL, (uint64_t)n, HL, 128, kBM)) return LIME_ERR_CUDA;
   } else if (!make_tmap_2d_bf16(&tmC, cache, HL, (uint64_t)n, HL * 2, 64, kBM)) {
     return LIME_ERR_CUDA;
@@ -408,7 +414,8 @@ bool fast_cache_supported(const lime_dims& D) {
 }
 
 bool fast_cache_u8_supported(const lime_dims& D) {
-  return fast_cache_supported(D) && D.H * D.l >= 128;
+  // 64-byte rows only with 16 links (the byte epilogue's 16-weight chunks)
+  return fast_cache_supported(D) && (D.H * D.l >= 128 || D.l == 16);
 }
 
 namespace {
@@ -437,6 +444,7 @@ int launch_build(const lime_dims& D, const void* T, int64_t n, const bf16* img, 
                                           : launch_cache<256, 32, false, false>(T, n, img, cache, tpc, status, st));
     case 256064: return (D.phi == LIME_PHI_SILU ? launch_cache<256, 64, false, true>(T, n, img, cache, tpc, status, st)
                                           : launch_cache<256, 64, false, false>(T, n, img, cache, tpc, status, st));
+    case 1064016: return launch_cache<64, 16, true, false>(T, n, img, cache, tpc, status, st);
     case 1128016: return launch_cache<128, 16, true, false>(T, n, img, cache, tpc, status, st);
     case 1128032: return launch_cache<128, 32, true, false>(T, n, img, cache, tpc, status, st);
     case 1128064: return launch_cache<128, 64, true, false>(T, n, img, cache, tpc, status, st);

@@ -263,6 +263,304 @@ int launch_score(int64_t B, const void* cache, int64_t n_items, const int32_t* i
                     total, (const bf16*)LP, (bf16*)O, status);
 }
 
+struct ScoreTile {
+  int64_t p;   // first packed position
+  int n;       // candidates (1 .. 128)
+  int64_t u;   // user, or -1 when no valid user range holds position p
+};
+
+// The tile starting at packed position p of a range ending at r1: the user
+// holding p (the last u with off[u] <= p, by binary search) and its rows up to
+// 128, the user's end or the range's end.  Offsets that do not give p a valid
+// owner yield u = -1 (zero rows) for up to 128 positions.
+__device__ __forceinline__ ScoreTile score_tile_at(int64_t p, int64_t r1, const int64_t* off,
+                                                   int64_t B, int64_t total) {
+  ScoreTile t;
+  t.p = p;
+  const int64_t u = owner_of(off, B, p);
+  int64_t a = off[u], b = off[u + 1];
+  a = a < 0 ? 0 : a;
+  b = b > total ? total : b;
+  int64_t e = p + kTile < r1 ? p + kTile : r1;
+  if (a <= p && p < b) {
+    t.u = u;
+    e = e < b ? e : b;
+  } else {
+    t.u = -1;
+  }
+  t.n = (int)(e - p);
+  return t;
+}
+
+// ------------------------------------------------ cached scoring, bf16 cache
+// k_score_ws<L>: one persistent CTA per SM with warp-specialised roles and a
+// flat, balanced schedule.  The packed candidate positions [0, total) are cut
+// into one contiguous range per CTA (a multiple of 128 positions); inside its
+// range a CTA walks tiles of at most 128 candidates that never cross a user
+// boundary (a user's last tile in the range may be partial).  Every role
+// derives the same tile sequence from the offsets on its own, so nothing but
+// the barriers passes between them.
+//   warps 0-3  producers: a tile's candidate IDs (validated: a bad ID gives a
+//              zero row and LIME_FLAG_BAD_ID) and its row gather with 16-byte
+//              asynchronous copies (a warp's copies cover whole rows) into a
+//              ring of NS stages, in the swizzled K-major operand layout; the
+//              hardware arrives on the stage's barrier for each producer once
+//              that thread's copies have landed, so up to NS tiles are in
+//              flight and no stage waits for later progress.  On every change of user
+//              they stage L^P_u transposed ([128 c x 64 k] bf16, k >= l zero)
+//              into one of two B slots.
+//   warp 4     one lane issues, per tile and head, the [128 x l] x [l x 32]
+//              product into one of two TMEM accumulators.
+//   warps 5-8  epilogue: TMEM -> bf16 -> a swizzled staging tile -> coalesced
+//              16-byte stores of the tile's rows.
+// The gather ring holds about 128 KB (NS = 8, 4, 2 tiles for l = 16, 32, 64),
+// which keeps an SM's share of the HBM bandwidth in flight at every l.
+template <int L>
+struct WsCfg {
+  static constexpr int HL = kH * L;
+  static constexpr int ABLK = HL / 64 < 1 ? 1 : HL / 64;   // 64-column blocks of a gathered tile
+  static constexpr uint32_t kStage = ABLK * kBlk;           // = 128 rows x 2*HL bytes
+  static constexpr int NS = L == 16 ? 8 : (L == 32 ? 4 : 2);
+  static constexpr int RB = 2 * HL;                         // bytes per cache row
+  static constexpr int CH = RB / 16;                        // 16-byte chunks per row
+  static constexpr uint32_t OFF_OUT = NS * kStage;          // [128 x 128] bf16 output staging
+  static constexpr uint32_t OFF_B = OFF_OUT + 2 * kBlk;     // two B slots, one block each
+  static constexpr uint32_t OFF_T = OFF_B + 2 * kBlk;       // L^P_u row-major [L x 128] bf16
+  static constexpr uint32_t OFF_IDS = OFF_T + L * kD * 2;   // [NS][128] int64 candidate IDs
+  static constexpr uint32_t OFF_BAR = OFF_IDS + NS * 128 * 8;
+  static constexpr int SMEM = 1024 + OFF_BAR + 256;
+  static constexpr int THREADS = 288;
+};
+
+template <int L>
+__global__ void __launch_bounds__(WsCfg<L>::THREADS, 1)
+    k_score_ws(const bf16* __restrict__ cache, int64_t n_items, const int32_t* __restrict__ ids,
+               const int64_t* __restrict__ off, int64_t B, int64_t total, int64_t span,
+               const bf16* __restrict__ LP, bf16* __restrict__ O, unsigned* status) {
+  using C = WsCfg<L>;
+  constexpr int NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sOut = sm + C::OFF_OUT;
+  uint8_t* sBs = sm + C::OFF_B;
+  bf16* sT = reinterpret_cast<bf16*>(sm + C::OFF_T);
+  int64_t* s_ids = reinterpret_cast<int64_t*>(sm + C::OFF_IDS);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
+  uint64_t* empty = full + NS;
+  uint64_t* bready = empty + NS;    // [2] B slot staged (128 producer arrivals)
+  uint64_t* bfree = bready + 2;     // [2] B slot's last MMA done (commit)
+  uint64_t* tfull = bfree + 2;      // [2] accumulator ready (commit)
+  uint64_t* tempty = tfull + 2;     // [2] accumulator read (128 epilogue arrivals)
+  uint64_t* mdone = tempty + 2;
+  uint32_t* slot = reinterpret_cast<uint32_t*>(mdone + 1);
+  int* abort_flag = reinterpret_cast<int*>(mdone + 2);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int q = 0; q < NS; ++q) {
+      mbar_init(&full[q], 128);
+      mbar_init(&empty[q], 1);
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&bready[q], 128);
+      mbar_init(&bfree[q], 1);
+      mbar_init(&tfull[q], 1);
+      mbar_init(&tempty[q], 128);
+    }
+    mbar_init(mdone, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) tmem_alloc(slot, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  pdl_launch();
+  pdl_wait();
+  const int64_t r0 = (int64_t)blockIdx.x * span;
+  const int64_t r1 = r0 + span < total ? r0 + span : total;
+
+  if (warp < 4) {
+    // ---- producers (128 threads, i = tid)
+    const int i = tid;
+    if (blockIdx.x == 0) {
+      // the offsets as a whole: monotone, from 0 to total
+      for (int64_t u = i; u < B; u += 128) {
+        const int64_t x = off[u], y = off[u + 1];
+        if (x > y || x < 0 || y > total || (u == 0 && x != 0) || (u == B - 1 && y != total))
+          raise_flag(status, LIME_FLAG_BAD_OFFSETS);
+      }
+    }
+    int64_t p = r0, cur_u = -1;
+    int k = 0, nsw = 0;
+    while (p < r1) {
+      const ScoreTile t = score_tile_at(p, r1, off, B, total);
+      const int s = k % NS;
+      if (k >= NS && !mbar_wait(&empty[s], (uint32_t)((k / NS) - 1) & 1u, status, abort_flag)) break;
+      if (t.u >= 0 && t.u != cur_u) {
+        // L^P_u transposed into B slot nsw % 2, once the MMAs of the user
+        // that held it before (user nsw - 2) are done
+        if (nsw >= 2 && !mbar_wait(&bfree[nsw & 1], (uint32_t)((nsw - 2) >> 1) & 1u, status,
+                                   abort_flag))
+          break;
+        const uint4* src = reinterpret_cast<const uint4*>(LP + t.u * L * kD);
+#pragma unroll
+        for (int q = 0; q < L * kD / 8 / 128; ++q)
+          reinterpret_cast<uint4*>(sT)[q * 128 + i] = __ldg(src + q * 128 + i);
+        named_bar_sync(1, 128);
+        uint8_t* sB = sBs + (nsw & 1) * kBlk;
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {
+          float f[8];
+#pragma unroll
+          for (int z = 0; z < 8; ++z) {
+            const int kk = k8 * 8 + z;
+            f[z] = kk < L ? __bfloat162float(sT[kk * kD + i]) : 0.f;
+          }
+          sw_st16(sB, kBlk, i, k8 * 8, pack8(f));
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bready[nsw & 1]);
+        cur_u = t.u;
+        ++nsw;
+      }
+      int64_t id = -1;
+      if (t.u >= 0 && i < t.n) {
+        id = (int64_t)ids[t.p + i];
+        if (id < 0 || id >= n_items) {
+          raise_flag(status, LIME_FLAG_BAD_ID);
+          id = -1;
+        }
+      }
+      if (t.u < 0 && i == 0) raise_flag(status, LIME_FLAG_BAD_OFFSETS);
+      s_ids[s * kTile + i] = id;
+      named_bar_sync(1, 128);
+      // chunk q*128 + i is chunk (idx % CH) of row idx / CH: a warp reads whole rows
+      uint8_t* sA = sm + s * C::kStage;
+#pragma unroll
+      for (int q = 0; q < C::CH; ++q) {
+        const int idx = q * 128 + i, r = idx / C::CH, cc = idx % C::CH;
+        const int64_t rid = s_ids[s * kTile + r];
+        const bf16* srow = cache + (rid < 0 ? 0 : rid * C::HL) + cc * 8;
+        cp_async16(sA + (cc >> 3) * kBlk + sw128_offset(r, (cc & 7) * 8), srow, rid >= 0);
+      }
+      // the stage is full once every producer's copies have landed (the
+      // hardware arrives for this thread; no later progress is needed)
+      cp_async_arrive_noinc(&full[s]);
+      p += t.n;
+      ++k;
+    }
+    cp_async_wait_all();   // nothing of ours is in flight when the CTA exits
+  } else if (warp == 4) {
+    // ---- MMA issuer (one lane)
+    if (lane == 0) {
+      int64_t p = r0, cur_u = -1;
+      int k = 0, nsw = 0, bs = 0;
+      bool ok = true;
+      while (p < r1 && ok) {
+        const ScoreTile t = score_tile_at(p, r1, off, B, total);
+        const int s = k % NS, acc = k & 1;
+        if (!(ok = mbar_wait(&full[s], (uint32_t)(k / NS) & 1u, status, abort_flag))) break;
+        if (t.u >= 0 && t.u != cur_u) {
+          if (nsw >= 1) mma_commit(&bfree[(nsw - 1) & 1]);   // the previous user's slot
+          if (!(ok = mbar_wait(&bready[nsw & 1], (uint32_t)(nsw >> 1) & 1u, status, abort_flag)))
+            break;
+          bs = nsw & 1;
+          cur_u = t.u;
+          ++nsw;
+        }
+        if (k >= 2 && !(ok = mbar_wait(&tempty[acc], (uint32_t)((k >> 1) - 1) & 1u, status,
+                                       abort_flag)))
+          break;
+        fence_proxy_async_smem();   // the gathered rows (generic-proxy copies) -> the MMA
+        tc_fence_after();
+        if (t.u >= 0) {
+          const uint8_t* sA = sm + s * C::kStage;
+#pragma unroll
+          for (int h = 0; h < kH; ++h)
+            mma_tile(tmem + acc * 128 + h * kDH,
+                     smem_u32(sA + ((h * L) >> 6) * kBlk + ((h * L) & 63) * 2), kBlk,
+                     smem_u32(sBs + bs * kBlk + h * kDH * 128), kBlk, kDH, L, false);
+        }
+        mma_commit(&empty[s]);
+        mma_commit(&tfull[acc]);
+        p += t.n;
+        ++k;
+      }
+      // drain: no MMA of ours may be in flight when TMEM is freed
+      mma_commit(mdone);
+      mbar_wait(mdone, 0, status, abort_flag);
+    }
+  } else {
+    // ---- epilogue (128 threads): row = TMEM lane of this warp's quadrant
+    const int e = tid - 160;
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    int64_t p = r0;
+    int k = 0;
+    while (p < r1) {
+      const ScoreTile t = score_tile_at(p, r1, off, B, total);
+      const int acc = k & 1;
+      if (!mbar_wait(&tfull[acc], (uint32_t)(k >> 1) & 1u, status, abort_flag)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float v[64];
+        if (t.u >= 0) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmem_ld16(ta + acc * 128 + hh * 64 + q * 16, v + q * 16);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) v[c] = 0.f;
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) sw_st16(sOut, kBlk, row, hh * 64 + c * 8, pack8(v + c * 8));
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      named_bar_sync(2, 128);   // the staging tile is complete
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const int idx = q * 128 + e, r = idx >> 4, cc = idx & 15;
+        if (r < t.n)
+          reinterpret_cast<uint4*>(O + (t.p + r) * kD)[cc] = sw_ld16(sOut, kBlk, r, cc * 8);
+      }
+      named_bar_sync(2, 128);   // every thread has read the staging tile
+      p += t.n;
+      ++k;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+template <int L>
+int launch_score_ws(int64_t B, const void* cache, int64_t n_items, const int32_t* ids,
+                    const int64_t* off, int64_t total, const void* LP, void* O, unsigned* status,
+                    cudaStream_t st) {
+  using C = WsCfg<L>;
+  if (cudaFuncSetAttribute(k_score_ws<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+      cudaSuccess)
+    return LIME_ERR_CUDA;
+  // one CTA per SM, each a contiguous range of a whole number of 128-position
+  // tiles (users split across ranges freely)
+  const int64_t tiles = (total + kTile - 1) / kTile;
+  int64_t G = num_sms();
+  if (G > tiles) G = tiles;
+  if (G < 1) G = 1;
+  const int64_t span = ((tiles + G - 1) / G) * kTile;
+  G = (total + span - 1) / span;
+  return launch_pdl(k_score_ws<L>, dim3((unsigned)G), dim3(C::THREADS), C::SMEM, st, 1,
+                    (const bf16*)cache, n_items, ids, off, B, total, span, (const bf16*)LP,
+                    (bf16*)O, status);
+}
+
 }  // namespace
 
 bool fast_score_supported(const lime_dims& D) {
@@ -270,7 +568,7 @@ bool fast_score_supported(const lime_dims& D) {
 }
 
 bool fast_score_u8_supported(const lime_dims& D) {
-  return fast_score_supported(D) && D.H * D.l >= 128;
+  return fast_score_supported(D) && D.H * D.l >= 64;
 }
 
 int fast_score(const lime_dims& D, int64_t B, const void* cache, int64_t n_items,
@@ -278,9 +576,11 @@ int fast_score(const lime_dims& D, int64_t B, const void* cache, int64_t n_items
                float* ws, unsigned* status, cudaStream_t st) {
   (void)ws;
   switch (D.l) {
+    // l <= 32: (user, slot) CTAs of 128 threads that gather, multiply and store
+    // in turn; l = 64 (one CTA per SM either way): the warp-specialised kernel
     case 16: return launch_score<16, false>(B, cache, n_items, ids, off, total, LP, O, status, st);
     case 32: return launch_score<32, false>(B, cache, n_items, ids, off, total, LP, O, status, st);
-    default: return launch_score<64, false>(B, cache, n_items, ids, off, total, LP, O, status, st);
+    default: return launch_score_ws<64>(B, cache, n_items, ids, off, total, LP, O, status, st);
   }
 }
 

@@ -142,6 +142,18 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Arrive-on `bar` (without incrementing its pending count) once every
+// cp.async this thread has issued so far has landed: the barrier's expected
+// count must include one such arrival per producing thread and phase.  The
+// copies are generic-proxy writes: a consumer that reads them through the
+// async proxy fences (fence_proxy_async_smem) after its wait.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Bulk prefetch of global memory into L2 (16-byte aligned, bytes % 16 == 0).
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
@@ -278,6 +290,10 @@ bool make_tmap_2d_f16(CUtensorMap* map, const void* base, uint64_t inner, uint64
 bool make_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                      uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
 
+// Host: a 2-D uint8 tensor without swizzle (row-major staging; box_inner a
+// multiple of 16).
+bool make_tmap_2d_u8_plain(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                           uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
 // Host: the same for a 2-D fp32 tensor (128-byte swizzle; box_inner <= 32).
 bool make_tmap_2d_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                       uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);

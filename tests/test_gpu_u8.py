@@ -5,8 +5,8 @@ encoding): q = round(255 w), ties to even, dequantised as q / 255.
 
 The byte is an integer decided by floating point, so the cache is checked in
 two ways: against the GPU's own bf16 cache (the same weight the kernel
-rounds, to a few bf16 ulps), where the byte must be the correct rounding
-except where 255 w lies within 0.05 of a tie; and against the oracle's byte
+rounds, to half a bf16 ulp), where the byte must be the correct rounding
+except where 255 w lies within that rounding of a tie; and against the oracle's byte
 quantize_cache_u8(w_ref), which it must equal exactly wherever 255 w_ref lies
 more than 0.02 from a tie (the kernel's weight error, from its bf16 operands,
 is at most 0.001 on that scale), and within one step near a tie.
@@ -35,7 +35,7 @@ def _cache_inputs(l, n_items, seed=11):
     return w, dims, T, us, cs, dev
 
 
-@pytest.mark.parametrize("l", [32, 64])
+@pytest.mark.parametrize("l", [16, 32, 64])
 def test_u8_cache_rounds_the_kernel_weight_and_tracks_the_oracle(l):
     w, dims, T, us, cs, (Td, Ld, Wq, Wk) = _cache_inputs(l, 40_000)
     ws = lime.Workspace(dims, 0, 0)
@@ -48,7 +48,9 @@ def test_u8_cache_rounds_the_kernel_weight_and_tracks_the_oracle(l):
     qg = q.cpu().numpy().astype(np.int64)
     # 1. the byte is the rounding of the kernel's weight, away from ties
     x = 255.0 * c16.float().cpu().numpy().astype(np.float64)
-    near_tie = np.abs(x - np.floor(x) - 0.5) < 0.05
+    # the bf16 weight is within half a bf16 ulp (2^-8 relative) of the fp32
+    # weight the kernel rounds: 255 w moves by up to 2^-8 * 255 w
+    near_tie = np.abs(x - np.floor(x) - 0.5) < 0.02 + x * 2.0 ** -8
     exact = np.rint(x).astype(np.int64)
     assert (qg[~near_tie] == exact[~near_tie]).all()
     assert (np.abs(qg[near_tie] - exact[near_tie]) <= 1).all()
@@ -70,7 +72,7 @@ def test_u8_cache_rounds_the_kernel_weight_and_tracks_the_oracle(l):
     assert err.max() <= 0.5 / 255 + 2e-3 / 255, err.max()
 
 
-@pytest.mark.parametrize("l", [32, 64])
+@pytest.mark.parametrize("l", [16, 32, 64])
 def test_u8_scoring_matches_the_oracle_on_the_gpu_bytes(l):
     d, H, n_items = 128, 4, 30_000
     dims = lime.make_dims(d, H, l, 2 * d, 64, "bf16")
@@ -130,11 +132,11 @@ def test_u8_bad_ids_give_zero_rows_and_flag():
 
 
 def test_u8_unsupported_shapes_are_rejected():
-    dims = lime.make_dims(128, 4, 16, 256, 64, "bf16")    # H*l = 64
+    dims = lime.make_dims(128, 2, 32, 256, 64, "bf16")    # 2 heads of 64: no int8 path
     ws = lime.Workspace(dims, 1, 0)
-    q = torch.zeros(10, 4, 16, dtype=torch.uint8, device="cuda")
+    q = torch.zeros(10, 2, 32, dtype=torch.uint8, device="cuda")
     with pytest.raises(lime.LimeError):
         lime.lime_build_qk_cache_u8(dims, torch.zeros(10, 128, dtype=torch.bfloat16, device="cuda"),
-                                    torch.zeros(16, 128, dtype=torch.bfloat16, device="cuda"),
+                                    torch.zeros(32, 128, dtype=torch.bfloat16, device="cuda"),
                                     torch.zeros(128, 128, dtype=torch.bfloat16, device="cuda"),
                                     torch.zeros(128, 128, dtype=torch.bfloat16, device="cuda"), q, ws)

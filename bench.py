@@ -393,6 +393,23 @@ def time_case(name, flush, stream, pk, T_cache):
            "cache_frac": roofline_of("cache", *work["cache"], cache * 1e-3, pk, w.dtype)["frac"]}
     if w.dtype != "bf16":
         out["user_frac"] = None   # fp32 CUDA-core path: absolute numbers only
+    else:
+        # scoring at scale: 16 users x 65,536 IDs uniform over the catalogue
+        # (cold L2), apart from the workload's own (Zipf) candidates
+        n_sc = 16 * 65536
+        gsc = torch.Generator().manual_seed(4243)
+        ids_sc = torch.randint(0, w.n_items, (n_sc,), generator=gsc).to(torch.int32).cuda()
+        off_sc = (torch.arange(17, dtype=torch.int64) * 65536).cuda()
+        LP_sc = buf.Z_bufs[(len(x.layers) - 1) % 2][:16].contiguous()
+        O_sc = torch.empty(n_sc, w.d, dtype=buf.O.dtype, device="cuda")
+        call = lambda: lime.lime_score_candidates(x.dims, buf.cache, ids_sc, off_sc, n_sc, LP_sc,
+                                                  O_sc, buf.ws)
+        call()
+        ms_sc = timed(call, flush, stream, 10)
+        es = 2
+        out["score_uniform_frac"] = r4(n_sc * (w.H * w.l * es + 4 + w.d * es) / (ms_sc * 1e-3) /
+                                       1e9 / pk["hbm_gbs"])
+        del O_sc, ids_sc
     del g_on, g_user, g_score, g_cache, buf, x
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
@@ -713,7 +730,8 @@ def main():
         if lin is not None:
             line["user_encode_us_per_1k_tokens"] = lin
         line["configs"] = {c["name"]: {k: c.get(k) for k in ("pairs_per_s", "user_frac",
-                                                             "score_frac", "cache_frac")
+                                                             "score_frac", "score_uniform_frac",
+                                                             "cache_frac")
                                        if k in c} for c in cfg}
         line["clocks"] = sampler.summary()
         line["e2e"] = {"value": r4(job_throughput(world, total_cand, e2e_step_ms)),

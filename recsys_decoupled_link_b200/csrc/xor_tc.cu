@@ -62,6 +62,7 @@ struct LayerWs {
   size_t img_vg;   // (g1 Wv)^T as hi, lo images, then cv = colsum(g1 Wv), dv = b1 Wv (fp32)
   size_t sched, tiles, tile_start;
   size_t yd, uimg, part;
+  size_t qe, ke, ve, att, kz, vz;   // window layers: history Q, K, V and A; link K, V (fp32)
   size_t total;
   int64_t max_tiles;
   uint32_t uimg_bytes;   // per user: nhalf half images
@@ -78,7 +79,7 @@ constexpr uint32_t kUimgVec = 6 * kBlk;
 constexpr uint32_t kUimgBytes = 6 * kBlk + 4 * 128 * 4;
 constexpr uint32_t kUimgGlo = kUimgBytes;
 
-LayerWs layer_ws(int l, int64_t B, int64_t nh, bool silu) {
+LayerWs layer_ws(int l, int64_t B, int64_t nh, bool silu, int window) {
   LayerWs w;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t r = o; o = up1k(o + bytes); return r; };
@@ -98,6 +99,15 @@ LayerWs layer_ws(int l, int64_t B, int64_t nh, bool silu) {
   w.uimg_bytes = (uint32_t)((kH * l + 127) / 128) * w.half_bytes;
   w.uimg = take((size_t)B * w.uimg_bytes);
   w.part = take((size_t)w.max_tiles * kH * l * kRec * 4);
+  w.qe = w.ke = w.ve = w.att = w.kz = w.vz = 0;
+  if (window > 0) {
+    w.qe = take((size_t)nh * kD * 4);
+    w.ke = take((size_t)nh * kD * 4);
+    w.ve = take((size_t)nh * kD * 4);
+    w.att = take((size_t)nh * kD * 4);
+    w.kz = take((size_t)B * l * kD * 4);
+    w.vz = take((size_t)B * l * kD * 4);
+  }
   w.total = o;
   return w;
 }
@@ -826,6 +836,48 @@ __global__ void __launch_bounds__(kXaThreads, 1)
     bf16* yd = reinterpret_cast<bf16*>(ws + Lw.yd);   // fp16 bits; rows copied as bytes
     float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
     if (HIST && threadIdx.x == 0) prefetch_tmap(&tmY);
+    // LN1 statistics of this thread's row of an E tile (biased variance; see
+    // layer_norm_part): mean and rstd into mu, rs, and every row's pair into
+    // smu (rstd in log2 units for phi = softmax).  Two epilogue barriers.
+    auto ln1_stats = [&](const uint8_t* tileE, float& mu, float& rs) {
+      // the part's mean, then its centred sum of squares (a second read of
+      // the tile's 32 values; see part_stats)
+      float pm = 0.f, pq = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float x[8];
+        unpack8(sw_ld16(tileE, kBlk, row, c0 + q * 8), x);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) pm += x[k];
+      }
+      pm *= 1.0f / 32;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float x[8];
+        unpack8(sw_ld16(tileE, kBlk, row, c0 + q * 8), x);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float dlt = x[k] - pm;
+          pq = fmaf(dlt, dlt, pq);
+        }
+      }
+      red[part * 128 + row] = pm;
+      red[512 + part * 128 + row] = pq;
+      named_bar_sync(1, kXaEpi);
+      merge4_stats(red[row], red[128 + row], red[256 + row], red[384 + row], red[512 + row],
+                   red[640 + row], red[768 + row], red[896 + row], mu, rs);
+      if (part == 0) {
+        smu[row] = mu;
+        smu[128 + row] = SILU ? rs : rs * kLog2e;   // softmax: log2 units
+      }
+      named_bar_sync(1, kXaEpi);
+    };
+    // History layers with l <= 32 compute the next tile's statistics while
+    // this tile's Yd product runs (after its link records), instead of at
+    // the head of the next tile's chain.
+    constexpr bool kPre = HIST && !SPLIT;
+    float mu_n = 0.f, rs_n = 0.f;
+    bool pre = false;
     int ab = 0, t = blockIdx.x, hf = 0;
     for (int it = 0; t < n_tiles; ++it) {
       const int4 tl = tiles[t];
@@ -839,40 +891,13 @@ __global__ void __launch_bounds__(kXaThreads, 1)
       mbar_wait(&bar[2], ph, status, c.abort_flag);
       if (it == 0) mbar_wait(&bar[0], 0, status, c.abort_flag);
       mbar_wait(&bar[4], ph, status, c.abort_flag);
-      // LN1 statistics of this thread's row (biased variance; see layer_norm_part)
+      // LN1 statistics of this thread's row (computed ahead, or now)
       float mu_r, rs_r;
-      {
-        // the part's mean, then its centred sum of squares (a second read of
-        // the tile's 32 values; see part_stats)
-        float pm = 0.f, pq = 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float x[8];
-          unpack8(sw_ld16(sA, kBlk, row, c0 + q * 8), x);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) pm += x[k];
-        }
-        pm *= 1.0f / 32;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float x[8];
-          unpack8(sw_ld16(sA, kBlk, row, c0 + q * 8), x);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float dlt = x[k] - pm;
-            pq = fmaf(dlt, dlt, pq);
-          }
-        }
-        red[part * 128 + row] = pm;
-        red[512 + part * 128 + row] = pq;
-        named_bar_sync(1, kXaEpi);
-        merge4_stats(red[row], red[128 + row], red[256 + row], red[384 + row], red[512 + row],
-                     red[640 + row], red[768 + row], red[896 + row], mu_r, rs_r);
-        if (part == 0) {
-          smu[row] = mu_r;
-          smu[128 + row] = SILU ? rs_r : rs_r * kLog2e;   // softmax: log2 units
-        }
-        named_bar_sync(1, kXaEpi);
+      if (pre) {
+        mu_r = mu_n;
+        rs_r = rs_n;
+      } else {
+        ln1_stats(sA, mu_r, rs_r);
       }
       mbar_wait(&bar[1], ph, status, c.abort_flag);
       tc_fence_after();
@@ -955,7 +980,17 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         tmem_ld16(ta + 256 + c0 + 16, v + 16);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = fmaf(rs_r, fmaf(-mu_r, cvd[c0 + j], v[j]), cvd[kD + c0 + j]);
+        for (int j4 = 0; j4 < 8; ++j4) {
+          // cv, dv of this part's columns as float4 (shared by the warp: broadcast)
+          const float4 cv4 = reinterpret_cast<const float4*>(cvd + c0)[j4];
+          const float4 dv4 = reinterpret_cast<const float4*>(cvd + kD + c0)[j4];
+          const float cvj[4] = {cv4.x, cv4.y, cv4.z, cv4.w}, dvj[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * j4 + e;
+            v[j] = fmaf(rs_r, fmaf(-mu_r, cvj[e], v[j]), dvj[e]);
+          }
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) sw_st16(sG, kBlk, row, c0 + q * 8, pack8(v + q * 8));
       }
@@ -971,9 +1006,19 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         for (int q = 0; q < L / 16; ++q) tmem_ld16(ta + h * L + q * 16, z + q * 16);
         tmem_ld_wait();
         const float rsl = SILU ? rs_r : rs_r * kLog2e;   // softmax: log2 units
+        {
+          // cG, dG of head h's links as float4 (shared by the warp: broadcast)
+          const float4* cg4 = reinterpret_cast<const float4*>(vec + 256 + h * L);
+          const float4* dg4 = reinterpret_cast<const float4*>(vec + 384 + h * L);
 #pragma unroll
-        for (int k = 0; k < L; ++k)
-          z[k] = fmaf(rsl, fmaf(-mu_r, vec[256 + h * L + k], z[k]), vec[384 + h * L + k]);
+          for (int q = 0; q < L / 4; ++q) {
+            const float4 a = cg4[q], b = dg4[q];
+            z[4 * q] = fmaf(rsl, fmaf(-mu_r, a.x, z[4 * q]), b.x);
+            z[4 * q + 1] = fmaf(rsl, fmaf(-mu_r, a.y, z[4 * q + 1]), b.y);
+            z[4 * q + 2] = fmaf(rsl, fmaf(-mu_r, a.z, z[4 * q + 2]), b.z);
+            z[4 * q + 3] = fmaf(rsl, fmaf(-mu_r, a.w, z[4 * q + 3]), b.w);
+          }
+        }
         if constexpr (SILU) {
 #pragma unroll
           for (int k = 0; k < L; ++k) z[k] = silu_fast(z[k]) * (1.0f / L);
@@ -1000,9 +1045,18 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         tmem_ld16(ta + c0 + 16, z + 16);
         tmem_ld_wait();
         const float rsl = SILU ? rs_r : rs_r * kLog2e;   // softmax: log2 units
+        {
+          const float4* cg4 = reinterpret_cast<const float4*>(vec + 256 + c0);
+          const float4* dg4 = reinterpret_cast<const float4*>(vec + 384 + c0);
 #pragma unroll
-        for (int k = 0; k < 32; ++k)
-          z[k] = fmaf(rsl, fmaf(-mu_r, vec[256 + c0 + k], z[k]), vec[384 + c0 + k]);
+          for (int q = 0; q < 8; ++q) {
+            const float4 a = cg4[q], b = dg4[q];
+            z[4 * q] = fmaf(rsl, fmaf(-mu_r, a.x, z[4 * q]), b.x);
+            z[4 * q + 1] = fmaf(rsl, fmaf(-mu_r, a.y, z[4 * q + 1]), b.y);
+            z[4 * q + 2] = fmaf(rsl, fmaf(-mu_r, a.z, z[4 * q + 2]), b.z);
+            z[4 * q + 3] = fmaf(rsl, fmaf(-mu_r, a.w, z[4 * q + 3]), b.w);
+          }
+        }
         if constexpr (SILU) {
 #pragma unroll
           for (int k = 0; k < 32; ++k) z[k] = silu_fast(z[k]) * (1.0f / L);
@@ -1052,6 +1106,15 @@ __global__ void __launch_bounds__(kXaThreads, 1)
           tc_fence_before();
           named_bar_sync(1, kXaEpi);
           if (threadIdx.x == 0) mbar_arrive(&bar[5]);
+        }
+      }
+      if constexpr (kPre) {
+        // the next tile's E rows land in B once P2 V_E is done (above):
+        // their statistics now, while this tile's Yd product runs
+        pre = t + (int)gridDim.x < n_tiles;
+        if (pre) {
+          mbar_wait(&bar[2], ph ^ 1u, status, c.abort_flag);
+          ln1_stats(sB, mu_n, rs_n);
         }
       }
       if (HIST) mbar_wait(&bar[10], ph, status, c.abort_flag);   // P has been read
@@ -1272,23 +1335,25 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
     // reduction scratch is the other E buffer: it holds h2(j-1), whose last
     // reader G(j-1, 3) has completed by the time the epilogue gets here, and
     // E(j+1) is loaded into it only after this tile's barH2 completes.
-    auto y_ln2 = [&](int j) {
+    // this thread's 32 fp16 Yd values of tile j (zeros past the tile's rows)
+    auto load_yd = [&](int j, uint4* v) {
+      const int4 tl = tile_of(j);
+      if (row < tl.z) {
+        const uint4* src = reinterpret_cast<const uint4*>(yd + (int64_t)(tl.y + row) * kD + c0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[q] = src[q];
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[q] = make_uint4(0, 0, 0, 0);
+      }
+    };
+    auto y_ln2 = [&](int j, const uint4* ydv) {
       uint8_t* sE = sE0 + (j & 1) * 2 * kBlk;
       float* red1 = reinterpret_cast<float*>(sE0 + ((j & 1) ^ 1) * 2 * kBlk);
       float* red2 = red1 + 4 * 128;
       float y[32];
-      {
-        // Yd rows (prefetched into L2 with the E tile)
-        const int4 tl = tile_of(j);
-        if (row < tl.z) {
-          const uint4* src = reinterpret_cast<const uint4*>(yd + (int64_t)(tl.y + row) * kD + c0);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) unpack8_f16(src[q], y + q * 8);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] = 0.f;
-        }
-      }
+      for (int q = 0; q < 4; ++q) unpack8_f16(ydv[q], y + q * 8);
       mbar_wait(&barE[j & 1], (uint32_t)((j >> 1) & 1), status, abort_flag);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -1326,10 +1391,18 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
       tc_fence_before();
       mbar_arrive(barH2);
     };
-    if (my_tiles > 0) y_ln2(0);
+    if (my_tiles > 0) {
+      uint4 v[4];
+      load_yd(0, v);
+      y_ln2(0, v);
+    }
     for (int k = 0; k < my_tiles; ++k) {
+      // the next tile's Yd rows, loaded during this tile's last hidden chunk
+      // so that their latency hides behind it
+      uint4 ydn[4];
       for (int c = 0; c < kF / 64; ++c) {
         const int g = k * (kF / 64) + c, sb = g & 1;
+        if (c == kF / 64 - 1 && k + 1 < my_tiles) load_yd(k + 1, ydn);
         mbar_wait(&barG[sb], (uint32_t)((g >> 1) & 1), status, abort_flag);
         tc_fence_after();
         float gt[16], gu[16];
@@ -1347,12 +1420,14 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
         tc_fence_before();
         mbar_arrive(&barHid[sb]);
       }
-      if (k + 1 < my_tiles) y_ln2(k + 1);
+      if (k + 1 < my_tiles) y_ln2(k + 1, ydn);
       mbar_wait(barOut, (uint32_t)(k & 1), status, abort_flag);
       tc_fence_after();
       // E' = OUT -> bf16, staged in the hid buffers (every W2 product of the
       // tile is done, and the next hid is written by these threads after the
-      // copy) and written with coalesced 16-byte stores
+      // copy) and written with coalesced 16-byte stores (a TMA store measured
+      // slower here: its issuing thread holds the tile's barrier until the
+      // copy has read the staging)
       {
         float o[32];
         tmem_ld16(ta + T_OUT + (k & 1) * 128 + c0, o);
@@ -1380,6 +1455,277 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------ LIME-XOR+Window history
+// With a window (LIME note, 关键设计 3: a history token also attends to its
+// neighbouring history tokens), a history query's keys are the user's l links
+// and the history rows j with 0 < |i - j| <= window, under one phi.  The link
+// branch is unchanged (k_hist_xattn without its history branch); the history
+// branch runs as
+//   k_rows_proj  LN1 and the Q, K, V projections of the history rows, and K, V
+//                of the link rows (tensor cores; bf16 outputs)
+//   k_win_attn   per (history row, head): phi over the l link keys and the
+//                window keys (CUDA cores: 2 * window + l keys of 32 dims each,
+//                far too little work per query for a tensor-core tile)
+//   k_rows_proj  Yd = A Wo (fp16), which the GatedMLP kernel reads as usual.
+
+// out_w[r, :] = x_r W_w for w < NW, x_r = LN1(X[r, :]) (LN) or X[r, :] (X bf16,
+// or fp32 for IN_F32), with W_w^T's K-major image at ws + img[w].  x_r enters
+// the products split into bf16 hi + lo (two MMAs each), so the fp32 outputs
+// carry no bf16 rounding of the operand.  One CTA per 128 rows, 512 threads:
+// thread (row, part) loads, normalises and splits its 32 columns, one thread
+// issues the products, and each thread writes its row's 32 columns of every
+// output (fp32, or fp16 for F16).
+struct RowsProjArgs {
+  uint32_t img[3];
+  void* out[3];
+};
+
+template <int NW, bool LN, bool IN_F32, bool F16>
+__global__ void __launch_bounds__(512, 1)
+    k_rows_proj(const void* __restrict__ Xv, int64_t n, const bf16* __restrict__ g,
+                const bf16* __restrict__ b, const uint8_t* __restrict__ ws, RowsProjArgs args,
+                unsigned* status) {
+  constexpr uint32_t kCols = NW == 1 ? 128 : (NW == 2 ? 256 : 512);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1k(smem_raw);
+  uint8_t* sAh = sm;
+  uint8_t* sAl = sm + 2 * kBlk;
+  uint8_t* sW = sm + 4 * kBlk;
+  float* red = reinterpret_cast<float*>(sm + (4 + 2 * NW) * kBlk);
+  Cta c;
+  cta_setup(sm + (4 + 2 * NW) * kBlk + kLnBytes, 2, c, kCols);
+  if (LN) ln_stage(red + 1024, g, b);
+  uint32_t mph = 0;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&c.bar[0], NW * 2 * kBlk);
+#pragma unroll
+    for (int w = 0; w < NW; ++w) bulk_load(sW + w * 2 * kBlk, ws + args.img[w], 2 * kBlk, &c.bar[0]);
+  }
+  const int warp = threadIdx.x >> 5;
+  const int part = warp >> 2;
+  const int r = (warp & 3) * 32 + (threadIdx.x & 31);
+  const int c0 = part * 32;
+  const int64_t R = (int64_t)blockIdx.x * kTile + r;
+  const bool valid = R < n;
+  {
+    float x[32];
+    if (valid) {
+      if constexpr (IN_F32) {
+        const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(Xv) + R * kD + c0);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 v = src[q];
+          x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+        }
+      } else {
+        const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(Xv) + R * kD + c0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) unpack8(src[q], x + q * 8);
+      }
+    } else {
+#pragma unroll
+      for (int i2 = 0; i2 < 32; ++i2) x[i2] = 0.f;
+    }
+    if (LN) layer_norm_part(x, c0, red, part, r);
+    split_part_st(sAh, sAl, r, c0, x);
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  mbar_wait(&c.bar[0], 0, status, c.abort_flag);
+  if (threadIdx.x == 0) {
+    tc_fence_after();
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      mma_tile(c.tmem + w * 128, smem_u32(sAh), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128, 128,
+               false);
+      mma_tile(c.tmem + w * 128, smem_u32(sAl), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128, 128,
+               true);
+    }
+  }
+  cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+  const uint32_t ta = quad_addr(c);
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    float v[32];
+    tmem_ld16(ta + w * 128 + c0, v);
+    tmem_ld16(ta + w * 128 + c0 + 16, v + 16);
+    tmem_ld_wait();
+    if (valid) {
+      if constexpr (F16) {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(args.out[w]) + R * kD + c0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = pack8_f16(v + q * 8);
+      } else {
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(args.out[w]) + R * kD + c0);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      }
+    }
+  }
+  cta_teardown(c);
+}
+
+// A[i, head h] = sum over keys phi(s q_i . k) v for history row i of user u
+// (fp32 throughout): the keys are u's l link rows (Kz, Vz) and its history
+// rows j with 0 < |i - j| <= win (Ke, Ve); phi = softmax (online: running max
+// and sum) or SiLU / (number of keys).  Thread = (row, head): four consecutive
+// threads share a row, so their 128-byte slices of a key row are one
+// coalesced 512 bytes.
+__global__ void __launch_bounds__(128)
+    k_win_attn(const float* __restrict__ Qe, const float* __restrict__ Ke, const float* __restrict__ Ve,
+               const float* __restrict__ Kz, const float* __restrict__ Vz,
+               const int64_t* __restrict__ off, int64_t B, int64_t nh, int L, int win, float scale,
+               int silu, float* __restrict__ att) {
+  pdl_launch();
+  pdl_wait();
+  const int64_t i = (int64_t)blockIdx.x * 32 + (threadIdx.x >> 2);
+  const int h = threadIdx.x & 3;
+  if (i >= nh) return;
+  const int64_t u = owner_of(off, B, i);
+  int64_t a = off[u], b = off[u + 1];
+  a = a < 0 ? 0 : a;
+  b = b > nh ? nh : b;
+  if (!(a <= i && i < b)) {
+    a = i;   // offsets that give no owner (flagged by the layer's schedule)
+    b = i + 1;
+  }
+  float q[32];
+  {
+    const float4* src = reinterpret_cast<const float4*>(Qe + i * kD + h * kDH);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 v = src[k];
+      q[4 * k] = v.x; q[4 * k + 1] = v.y; q[4 * k + 2] = v.z; q[4 * k + 3] = v.w;
+    }
+  }
+  const int64_t j0 = i - win > a ? i - win : a;
+  const int64_t j1 = i + win < b - 1 ? i + win : b - 1;
+  const float nkeys = (float)(L + (j1 - j0));   // the window excludes row i itself
+  float m = -INFINITY, ssum = 0.f, acc[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+  auto visit = [&](const float* krow, const float* vrow) {
+    const float4* ks = reinterpret_cast<const float4*>(krow);
+    float sdot = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 kv = __ldg(ks + k);
+      sdot = fmaf(q[4 * k], kv.x, sdot);
+      sdot = fmaf(q[4 * k + 1], kv.y, sdot);
+      sdot = fmaf(q[4 * k + 2], kv.z, sdot);
+      sdot = fmaf(q[4 * k + 3], kv.w, sdot);
+    }
+    sdot *= scale;
+    float p, corr;
+    if (silu) {
+      p = sdot / (1.0f + __expf(-sdot)) / nkeys;
+      corr = 1.f;
+    } else {
+      const float mn = fmaxf(m, sdot);
+      corr = m == -INFINITY ? 0.f : __expf(m - mn);
+      p = __expf(sdot - mn);
+      ssum = fmaf(ssum, corr, p);
+      m = mn;
+    }
+    const float4* vs = reinterpret_cast<const float4*>(vrow);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 vv = __ldg(vs + k);
+      acc[4 * k] = fmaf(acc[4 * k], corr, p * vv.x);
+      acc[4 * k + 1] = fmaf(acc[4 * k + 1], corr, p * vv.y);
+      acc[4 * k + 2] = fmaf(acc[4 * k + 2], corr, p * vv.z);
+      acc[4 * k + 3] = fmaf(acc[4 * k + 3], corr, p * vv.w);
+    }
+  };
+  for (int k = 0; k < L; ++k) {
+    const int64_t zr = u * L + k;
+    visit(Kz + zr * kD + h * kDH, Vz + zr * kD + h * kDH);
+  }
+  for (int64_t j = j0; j <= j1; ++j)
+    if (j != i) visit(Ke + j * kD + h * kDH, Ve + j * kD + h * kDH);
+  const float inv = silu ? 1.0f : 1.0f / ssum;
+  float4* dst = reinterpret_cast<float4*>(att + i * kD + h * kDH);
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    dst[k] = make_float4(acc[4 * k] * inv, acc[4 * k + 1] * inv, acc[4 * k + 2] * inv, acc[4 * k + 3] * inv);
+}
+
+// ------------------------------------------------------- record pre-merge
+// The link-branch records of a user's tiles (max, sum, 32 weighted sums per
+// (tile, head, link)) are merged in runs of consecutive tiles: block b takes
+// tiles [kRun b, kRun b + kRun) of the tile list, splits them at user
+// boundaries and merges each run into the record slot of its first tile (in
+// place, log-sum-exp, the tail's formula).  Runs therefore start at every
+// user's first tile and at every multiple of kRun inside a user's tiles, and
+// the link tail merges only those slots: a user with n tiles leaves it about
+// n / kRun records, which keeps the tail's merge short for long histories.
+// Thread (pair, q): the pair's max and sum and its weighted sums 8q .. 8q+7.
+constexpr int kRun = 8;
+
+template <int L>
+__global__ void __launch_bounds__(kH * L * 4 < 512 ? kH * L * 4 : 512)
+    k_rec_merge(uint8_t* __restrict__ ws, LayerWs Lw) {
+  constexpr int HL = kH * L;
+  pdl_launch();
+  pdl_wait();
+  const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
+  const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
+  const int t0 = (int)blockIdx.x * kRun;
+  if (t0 >= n_tiles) return;
+  const int t1 = t0 + kRun < n_tiles ? t0 + kRun : n_tiles;
+  const int q = threadIdx.x & 3;
+  float* recs = reinterpret_cast<float*>(ws + Lw.part);
+  // pairs in groups of blockDim / 4 (two groups for l = 64)
+  for (int pr = threadIdx.x >> 2; pr < HL; pr += (int)blockDim.x >> 2) {
+    int s0 = t0;
+    while (s0 < t1) {
+      const int u = tiles[s0].x;
+      int e = s0 + 1;
+      while (e < t1 && tiles[e].x == u) ++e;
+      if (e - s0 > 1) {
+        float2 ms[kRun];
+        float4 a[kRun][2];
+#pragma unroll
+        for (int i = 0; i < kRun; ++i) {
+          if (s0 + i < e) {
+            const float4* rec = reinterpret_cast<const float4*>(recs + ((size_t)(s0 + i) * HL + pr) * kRec);
+            ms[i] = *reinterpret_cast<const float2*>(rec);
+            a[i][0] = rec[1 + 2 * q];
+            a[i][1] = rec[2 + 2 * q];
+          }
+        }
+        float M = -INFINITY, S = 0.f, acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+#pragma unroll
+        for (int i = 0; i < kRun; ++i) {
+          if (s0 + i < e) {
+            const float Mn = fmaxf(M, ms[i].x);
+            const float so = M == -INFINITY ? 0.f : __expf(M - Mn);
+            const float sn = __expf(ms[i].x - Mn);
+            S = S * so + ms[i].y * sn;
+            acc[0] = acc[0] * so + a[i][0].x * sn;
+            acc[1] = acc[1] * so + a[i][0].y * sn;
+            acc[2] = acc[2] * so + a[i][0].z * sn;
+            acc[3] = acc[3] * so + a[i][0].w * sn;
+            acc[4] = acc[4] * so + a[i][1].x * sn;
+            acc[5] = acc[5] * so + a[i][1].y * sn;
+            acc[6] = acc[6] * so + a[i][1].z * sn;
+            acc[7] = acc[7] * so + a[i][1].w * sn;
+            M = Mn;
+          }
+        }
+        __syncwarp();   // the pair's four threads have read the run's first record
+        float4* dst = reinterpret_cast<float4*>(recs + ((size_t)s0 * HL + pr) * kRec);
+        if (q == 0) *reinterpret_cast<float2*>(dst) = make_float2(M, S);
+        dst[1 + 2 * q] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        dst[2 + 2 * q] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
+      s0 = e;
+    }
   }
 }
 
@@ -1463,15 +1809,23 @@ __global__ void __launch_bounds__(512, 1)
       const float* recs = reinterpret_cast<const float*>(ws + Lw.part);
       float M = -INFINITY;
       const int ta_ = ts[u], tb_ = ts[u + 1];
-      for (int t = ta_; t < tb_; t += 8) {
-        // the records of up to eight tiles are loaded before any is merged
+      // the user's run records (k_rec_merge): at its first tile and at every
+      // multiple of kRun after it
+      for (int t = ta_; t < tb_;) {
+        // the records of up to eight runs are loaded before any is merged
+        int slot[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          slot[i] = t;
+          if (t < tb_) t = (t / kRun + 1) * kRun;
+        }
         float2 ms[8];
         float4 a[8][2];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          if (t + i < tb_) {
+          if (slot[i] < tb_) {
             const float4* rec =
-                reinterpret_cast<const float4*>(recs + ((size_t)(t + i) * HL + h * L + k) * kRec);
+                reinterpret_cast<const float4*>(recs + ((size_t)slot[i] * HL + h * L + k) * kRec);
             ms[i] = *reinterpret_cast<const float2*>(rec);
             a[i][0] = rec[1 + 2 * q];
             a[i][1] = rec[2 + 2 * q];
@@ -1479,7 +1833,7 @@ __global__ void __launch_bounds__(512, 1)
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          if (t + i < tb_) {
+          if (slot[i] < tb_) {
             const float Mn = fmaxf(M, ms[i].x);
             const float so = M == -INFINITY ? 0.f : __expf(M - Mn);
             const float sn = __expf(ms[i].x - Mn);
@@ -1702,8 +2056,12 @@ template <int L>
 int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, const void* E_in,
               const void* Z_in, const lime_layer_w& w, void* E_out, void* Z_out, uint8_t* ws,
               unsigned* status, cudaStream_t st) {
-  const LayerWs Lw = layer_ws(L, B, nh, D.phi == LIME_PHI_SILU);
+  const LayerWs Lw = layer_ws(L, B, nh, D.phi == LIME_PHI_SILU, D.window);
   const bool last = E_out == nullptr;
+  // a window layer's history branch runs on its own kernels (after the link
+  // branch); its link projections are those of a last layer (Q'g only)
+  const bool window = D.window > 0 && !last;
+  const bool link_only = last || window;
   const float scale = 1.0f / sqrtf((float)kDH);
   const int64_t nz = B * L;
   const int sms = num_sms();
@@ -1719,8 +2077,8 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     // the last layer needs only Q' (its history branch is skipped)
     const int smem = 1024 + 8 * kBlk + kLnBytes + kBarBytes;
     if (!set_smem(k_link_proj<L>, smem)) return LIME_ERR_CUDA;
-    int rc = launch_pdl(k_link_proj<L>, dim3((unsigned)((nz + kTile - 1) / kTile), last ? 1 : 3,
-                                             last ? 4 : 2),
+    int rc = launch_pdl(k_link_proj<L>, dim3((unsigned)((nz + kTile - 1) / kTile), link_only ? 1 : 3,
+                                             link_only ? 4 : 2),
                         dim3(512), smem, st, 1, (const bf16*)Z_in, nz, (const bf16*)w.g1,
                         (const bf16*)w.b1, ws, Lw, scale, D.phi == LIME_PHI_SILU, status);
     if (rc) return rc;
@@ -1736,17 +2094,57 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
     const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
     {
       const bool silu = D.phi == LIME_PHI_SILU;
-      auto kern = last ? (silu ? k_hist_xattn<L, false, true> : k_hist_xattn<L, false, false>)
-                       : (silu ? k_hist_xattn<L, true, true> : k_hist_xattn<L, true, false>);
+      auto kern = link_only ? (silu ? k_hist_xattn<L, false, true> : k_hist_xattn<L, false, false>)
+                            : (silu ? k_hist_xattn<L, true, true> : k_hist_xattn<L, true, false>);
       if (!set_smem(kern, kXaSmem)) return LIME_ERR_CUDA;
       int rc = launch_pdl(kern, dim3(grid), dim3(kXaThreads), kXaSmem, st, 1, tmE, tmY, ws, Lw,
                           status);
+      if (rc) return rc;
+    }
+    if (window) {
+      const bool silu = D.phi == LIME_PHI_SILU;
+      const bf16* g1 = (const bf16*)w.g1;
+      const bf16* b1 = (const bf16*)w.b1;
+      // LN1 and Q, K, V of the history rows; K, V of the link rows (fp32)
+      constexpr int smem3 = 1024 + 10 * kBlk + kLnBytes + kBarBytes;
+      constexpr int smem2 = 1024 + 8 * kBlk + kLnBytes + kBarBytes;
+      constexpr int smem1 = 1024 + 6 * kBlk + kLnBytes + kBarBytes;
+      auto kq = k_rows_proj<3, true, false, false>;
+      auto kz = k_rows_proj<2, true, false, false>;
+      auto ko = k_rows_proj<1, false, true, true>;
+      if (!set_smem(kq, smem3) || !set_smem(kz, smem2) || !set_smem(ko, smem1))
+        return LIME_ERR_CUDA;
+      RowsProjArgs a3{{(uint32_t)Lw.img_q, (uint32_t)Lw.img_k, (uint32_t)Lw.img_v},
+                      {ws + Lw.qe, ws + Lw.ke, ws + Lw.ve}};
+      int rc = launch_pdl(kq, dim3((unsigned)((nh + kTile - 1) / kTile)), dim3(512), smem3, st, 1,
+                          (const void*)E_in, nh, g1, b1, (const uint8_t*)ws, a3, status);
+      if (rc) return rc;
+      RowsProjArgs a2{{(uint32_t)Lw.img_k, (uint32_t)Lw.img_v, 0u},
+                      {ws + Lw.kz, ws + Lw.vz, nullptr}};
+      rc = launch_pdl(kz, dim3((unsigned)((nz + kTile - 1) / kTile)), dim3(512), smem2, st, 1,
+                      (const void*)Z_in, nz, g1, b1, (const uint8_t*)ws, a2, status);
+      if (rc) return rc;
+      rc = launch_pdl(k_win_attn, dim3((unsigned)((nh + 31) / 32)), dim3(128), 0, st, 1,
+                      (const float*)(ws + Lw.qe), (const float*)(ws + Lw.ke),
+                      (const float*)(ws + Lw.ve), (const float*)(ws + Lw.kz),
+                      (const float*)(ws + Lw.vz), off, B, nh, L, D.window, scale, silu ? 1 : 0,
+                      (float*)(ws + Lw.att));
+      if (rc) return rc;
+      // Yd = A Wo (fp16), the attention delta the GatedMLP kernel adds to E
+      RowsProjArgs a1{{(uint32_t)Lw.img_o, 0u, 0u}, {ws + Lw.yd, nullptr, nullptr}};
+      rc = launch_pdl(ko, dim3((unsigned)((nh + kTile - 1) / kTile)), dim3(512), smem1, st, 1,
+                      (const void*)(ws + Lw.att), nh, g1, b1, (const uint8_t*)ws, a1, status);
       if (rc) return rc;
     }
   }
   // one 4-CTA cluster per 128 link rows
   if (!set_smem(k_link_tail<L>, kTailSmem)) return LIME_ERR_CUDA;
   auto tail = [&](cudaStream_t s) {
+    if (nh > 0) {
+      int rc = launch_pdl(k_rec_merge<L>, dim3((unsigned)((Lw.max_tiles + kRun - 1) / kRun)),
+                          dim3(kH * L * 4 < 512 ? kH * L * 4 : 512), 0, s, 1, ws, Lw);
+      if (rc) return rc;
+    }
     return launch_pdl(k_link_tail<L>, dim3((unsigned)((nz + kTile - 1) / kTile), kF / 64),
                       dim3(512), kTailSmem, s, kF / 64, (const bf16*)Z_in, nz,
                       (const bf16*)w.g2, (const bf16*)w.b2, (const uint8_t*)ws, Lw, (bf16*)Z_out,
@@ -1788,12 +2186,12 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
 
 bool fast_layer_supported(const lime_dims& D) {
   return D.dtype == LIME_BF16 && D.d == kD && D.H == kH && D.f == kF &&
-         (D.l == 16 || D.l == 32 || D.l == 64) && D.window == 0;
+         (D.l == 16 || D.l == 32 || D.l == 64);
 }
 
 size_t fast_layer_ws_bytes(const lime_dims& D, int64_t B, int64_t total_hist) {
   if (!fast_layer_supported(D)) return 0;
-  return layer_ws(D.l, B, total_hist, D.phi == LIME_PHI_SILU).total;
+  return layer_ws(D.l, B, total_hist, D.phi == LIME_PHI_SILU, D.window).total;
 }
 
 int fast_xor_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh,

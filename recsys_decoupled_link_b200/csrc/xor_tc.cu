@@ -1178,7 +1178,8 @@ __global__ void __launch_bounds__(kXaThreads, 1)
 // Chunks are counted over the CTA's whole tile sequence (g = 4*k + c for its
 // k-th tile), so every ring barrier's parity is (g / 2) % 2.
 // TMEM: GB[0] [0,128), GB[1] [128,256), OUT[k%2] [256 + 128*(k%2), +128).
-constexpr int kFfnEpi = 512;   // epilogue threads
+constexpr int kFfnEpi = 512;   // epilogue threads (two groups of 256)
+constexpr int kFfnGrp = 256;
 constexpr int kFfnTiles = 32;  // tile descriptors of a CTA kept in shared memory
 constexpr int kFfnSmem = 1024 + 14 * kBlk + 1024 + kFfnTiles * 16 + 256;
 
@@ -1204,18 +1205,20 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
   uint64_t* barOut = bar + 11; // all of the tile's MMAs done (MMA commit)
   uint64_t* barW2in = bar + 12;  // W2 image landed
   uint64_t* barDrain = bar + 13; // every MMA issued by the control lane is done
-  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 14);
-  int* abort_flag = reinterpret_cast<int*>(bar + 15);
+  uint64_t* barSE = bar + 14;    // E'(j) staging read out of E buffer j%2 (row-group arrivals)
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 15);
+  int* abort_flag = reinterpret_cast<int*>(bar + 16);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int q = 0; q < 2; ++q) {
       mbar_init(&barE[q], 1);
       mbar_init(&barWt[q], 1);
       mbar_init(&barG[q], 1);
-      mbar_init(&barHid[q], kFfnEpi);
+      mbar_init(&barHid[q], kFfnGrp);
       mbar_init(&barW2[q], 1);
     }
-    mbar_init(barH2, kFfnEpi);
+    mbar_init(barH2, kFfnGrp);
+    mbar_init(barSE, kFfnGrp);
     mbar_init(barOut, 1);
     mbar_init(barW2in, 1);
     mbar_init(barDrain, 1);
@@ -1268,6 +1271,7 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
       };
       prefetch_tmap(&tmE);
       load_e(0);
+      if (my_tiles > 1) load_e(1);
       load_w13(0);
       if (n_chunks > 1) load_w13(1);
       mbar_arrive_expect_tx(barW2in, 4 * kBlk);
@@ -1280,11 +1284,11 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
           if (g + 1 < n_chunks) load_w13(g + 1);
         }
         const int k = g / (kF / 64);
-        if (g % (kF / 64) == 0 && k + 1 < my_tiles) {
-          // E(k+1) goes to buffer (k+1)%2, which held h2(k-1) (dead once
-          // G(k-1, 3) is done) and is the LN2 scratch of tile k: wait for h2(k)
-          if (!mbar_wait(barH2, k & 1, status, abort_flag)) break;
-          load_e(k + 1);
+        if (g % (kF / 64) == kF / 64 - 1 && k + 2 < my_tiles) {
+          // E(k+2) goes to buffer k%2, which held h2(k) and then tile k's E'
+          // staging: wait until the row group has read the staging out
+          if (!mbar_wait(barSE, k & 1, status, abort_flag)) break;
+          load_e(k + 2);
         }
       }
     }
@@ -1325,129 +1329,160 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
       mma_commit(barDrain);
       mbar_wait(barDrain, 0, status, abort_flag);
     }
-  } else {
-    const int q4 = warp & 3, part = warp >> 2;     // lane quadrant, column part
+  } else if (warp < kFfnGrp / 32) {
+    // ---- row group (warps 0-7): thread (row, half), 64 columns of the row
+    const int q4 = warp & 3, half = warp >> 2;
     const int row = q4 * 32 + lane;
+    const int tid = (int)threadIdx.x;
     const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16);
-    const int c0 = part * 32;                      // this thread's 32 columns of a row
+    const int c0 = half * 64;
     const __half* yd = reinterpret_cast<const __half*>(ws + Lw.yd);
-    // Y(j) = E + Yd into OUT[j%2], h2(j) = LN2(Y(j)) over E tile j%2.  The
-    // reduction scratch is the other E buffer: it holds h2(j-1), whose last
-    // reader G(j-1, 3) has completed by the time the epilogue gets here, and
-    // E(j+1) is loaded into it only after this tile's barH2 completes.
-    // this thread's 32 fp16 Yd values of tile j (zeros past the tile's rows)
+    // this thread's 64 fp16 Yd values of tile j (zeros past the tile's rows)
     auto load_yd = [&](int j, uint4* v) {
       const int4 tl = tile_of(j);
       if (row < tl.z) {
         const uint4* src = reinterpret_cast<const uint4*>(yd + (int64_t)(tl.y + row) * kD + c0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) v[q] = src[q];
+        for (int q = 0; q < 8; ++q) v[q] = src[q];
       } else {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) v[q] = make_uint4(0, 0, 0, 0);
+        for (int q = 0; q < 8; ++q) v[q] = make_uint4(0, 0, 0, 0);
       }
     };
+    // Y(j) = E + Yd into OUT[j%2]; h2(j) = LN2(Y(j)) over E buffer j%2.  Once
+    // both halves have stored their Y, each thread reads the whole row back
+    // from TMEM in column order for the statistics (so both halves normalise
+    // with identical mu and rstd; shifted one-pass sums, shift = the row's
+    // first value), then its own 64 columns again for h2.
     auto y_ln2 = [&](int j, const uint4* ydv) {
       uint8_t* sE = sE0 + (j & 1) * 2 * kBlk;
-      float* red1 = reinterpret_cast<float*>(sE0 + ((j & 1) ^ 1) * 2 * kBlk);
-      float* red2 = red1 + 4 * 128;
-      float y[32];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) unpack8_f16(ydv[q], y + q * 8);
+      const uint32_t t_out = ta + T_OUT + (j & 1) * 128;
       mbar_wait(&barE[j & 1], (uint32_t)((j >> 1) & 1), status, abort_flag);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float e[8];
-        unpack8(sw_ld16(sE, kBlk, row, c0 + q * 8), e);
+      for (int p2 = 0; p2 < 2; ++p2) {
+        float y[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) y[q * 8 + i] += e[i];
-      }
-      const uint32_t t_out = ta + T_OUT + (j & 1) * 128 + c0;
-      tmem_st16(t_out, y);
-      tmem_st16(t_out + 16, y + 16);
-      {
-        float pm, pq;
-        part_stats(y, pm, pq);
-        red1[part * 128 + row] = pm;
-        red2[part * 128 + row] = pq;
-      }
-      named_bar_sync(1, kFfnEpi);
-      float mu, rstd;
-      merge4_stats(red1[row], red1[128 + row], red1[256 + row], red1[384 + row], red2[row],
-                   red2[128 + row], red2[256 + row], red2[384 + row], mu, rstd);
+        for (int q = 0; q < 4; ++q) {
+          float e[8];
+          unpack8_f16(ydv[p2 * 4 + q], y + q * 8);
+          unpack8(sw_ld16(sE, kBlk, row, c0 + p2 * 32 + q * 8), e);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 gv = reinterpret_cast<const float4*>(sg + c0)[q];
-        const float4 bv = reinterpret_cast<const float4*>(sg + kD + c0)[q];
-        y[4 * q] = (y[4 * q] - mu) * rstd * gv.x + bv.x;
-        y[4 * q + 1] = (y[4 * q + 1] - mu) * rstd * gv.y + bv.y;
-        y[4 * q + 2] = (y[4 * q + 2] - mu) * rstd * gv.z + bv.z;
-        y[4 * q + 3] = (y[4 * q + 3] - mu) * rstd * gv.w + bv.w;
+          for (int i = 0; i < 8; ++i) y[q * 8 + i] += e[i];
+        }
+        tmem_st16(t_out + c0 + p2 * 32, y);
+        tmem_st16(t_out + c0 + p2 * 32 + 16, y + 16);
       }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) sw_st16(sE, kBlk, row, c0 + q * 8, pack8(y + q * 8));
       tmem_st_wait();
+      tc_fence_before();
+      named_bar_sync(1, kFfnGrp);   // both halves of every row are in OUT (and E is read)
+      tc_fence_after();
+      // statistics over all 128 columns, read back from TMEM in column order
+      float K = 0.f, s1 = 0.f, s2 = 0.f;
+#pragma unroll 1
+      for (int q = 0; q < 8; ++q) {
+        float o[16];
+        tmem_ld16(t_out + q * 16, o);
+        tmem_ld_wait();
+        if (q == 0) K = o[0];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float t = o[i] - K;
+          s1 += t;
+          s2 = fmaf(t, t, s2);
+        }
+      }
+      const float ms = s1 * (1.0f / kD);
+      const float mu = K + ms;
+      const float rstd = rsqrtf(fmaxf(s2 * (1.0f / kD) - ms * ms, 0.f) + kLnEps);
+      // h2 of this thread's 64 columns, 16 at a time from TMEM
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        float o[16];
+        tmem_ld16(t_out + c0 + q * 16, o);
+        tmem_ld_wait();
+        const int cc = c0 + q * 16;
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+          const float4 gv = reinterpret_cast<const float4*>(sg + cc)[i4];
+          const float4 bv = reinterpret_cast<const float4*>(sg + kD + cc)[i4];
+          o[4 * i4] = (o[4 * i4] - mu) * rstd * gv.x + bv.x;
+          o[4 * i4 + 1] = (o[4 * i4 + 1] - mu) * rstd * gv.y + bv.y;
+          o[4 * i4 + 2] = (o[4 * i4 + 2] - mu) * rstd * gv.z + bv.z;
+          o[4 * i4 + 3] = (o[4 * i4 + 3] - mu) * rstd * gv.w + bv.w;
+        }
+        sw_st16(sE, kBlk, row, cc, pack8(o));
+        sw_st16(sE, kBlk, row, cc + 8, pack8(o + 8));
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(barH2);
     };
-    if (my_tiles > 0) {
-      uint4 v[4];
-      load_yd(0, v);
-      y_ln2(0, v);
-    }
-    for (int k = 0; k < my_tiles; ++k) {
-      // the next tile's Yd rows, loaded during this tile's last hidden chunk
-      // so that their latency hides behind it
-      uint4 ydn[4];
-      for (int c = 0; c < kF / 64; ++c) {
-        const int g = k * (kF / 64) + c, sb = g & 1;
-        if (c == kF / 64 - 1 && k + 1 < my_tiles) load_yd(k + 1, ydn);
-        mbar_wait(&barG[sb], (uint32_t)((g >> 1) & 1), status, abort_flag);
-        tc_fence_after();
-        float gt[16], gu[16];
-        tmem_ld16(ta + sb * 128 + part * 16, gt);
-        tmem_ld16(ta + sb * 128 + 64 + part * 16, gu);
+    // E'(j) = OUT[j%2] -> bf16, staged over E buffer j%2 (h2(j) is dead once
+    // every product of the tile is done) and written with coalesced stores
+    auto out = [&](int j) {
+      mbar_wait(barOut, (uint32_t)(j & 1), status, abort_flag);
+      tc_fence_after();
+      uint8_t* sE = sE0 + (j & 1) * 2 * kBlk;
+#pragma unroll
+      for (int p2 = 0; p2 < 2; ++p2) {
+        float o[32];
+        tmem_ld16(ta + T_OUT + (j & 1) * 128 + c0 + p2 * 32, o);
+        tmem_ld16(ta + T_OUT + (j & 1) * 128 + c0 + p2 * 32 + 16, o + 16);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) gt[i] = silu_tanh(gt[i]) * gu[i];
+        for (int q = 0; q < 4; ++q) sw_st16(sE, kBlk, row, c0 + p2 * 32 + q * 8, pack8(o + q * 8));
+      }
+      tc_fence_before();
+      named_bar_sync(1, kFfnGrp);   // the staging tile is complete
+      const int4 tl = tile_of(j);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int idx = q * kFfnGrp + tid, r = idx >> 4, cc = idx & 15;
+        if (r < tl.z)
+          reinterpret_cast<uint4*>(E_out + (int64_t)(tl.y + r) * kD)[cc] = sw_ld16(sE, kBlk, r, cc * 8);
+      }
+      mbar_arrive(barSE);   // this thread has read its part of the staging
+    };
+    uint4 ydv[8];
+    if (my_tiles > 0) load_yd(0, ydv);
+    for (int j = 0; j <= my_tiles; ++j) {
+      if (j < my_tiles) {
+        y_ln2(j, ydv);
+        // the next tile's Yd rows, in flight while this group reads out E'(j-1)
+        if (j + 1 < my_tiles) load_yd(j + 1, ydv);
+      }
+      if (j >= 1) out(j - 1);
+    }
+  } else {
+    // ---- chunk group (warps 8-15): thread (row, half): hidden units
+    //      32 half .. 32 half + 31 of every 64-wide chunk
+    const int q4 = warp & 3, half = (warp >> 2) & 1;
+    const int row = q4 * 32 + lane;
+    const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16);
+    for (int k = 0; k < my_tiles; ++k) {
+      for (int c = 0; c < kF / 64; ++c) {
+        const int g = k * (kF / 64) + c, sb = g & 1;
+        mbar_wait(&barG[sb], (uint32_t)((g >> 1) & 1), status, abort_flag);
+        tc_fence_after();
+        float h[32];
+#pragma unroll
+        for (int p2 = 0; p2 < 2; ++p2) {
+          float gt[16], gu[16];
+          tmem_ld16(ta + sb * 128 + half * 32 + p2 * 16, gt);
+          tmem_ld16(ta + sb * 128 + 64 + half * 32 + p2 * 16, gu);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) h[p2 * 16 + i] = silu_tanh(gt[i]) * gu[i];
+        }
         // hid(g) reuses the buffer of hid(g-2): wait until its W2 MMA is done
         if (g >= 2) mbar_wait(&barW2[sb], (uint32_t)(((g - 2) >> 1) & 1), status, abort_flag);
         uint8_t* sH = sH0 + sb * kBlk;
-        sw_st16(sH, kBlk, row, part * 16, pack8(gt));
-        sw_st16(sH, kBlk, row, part * 16 + 8, pack8(gt + 8));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sw_st16(sH, kBlk, row, half * 32 + q * 8, pack8(h + q * 8));
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&barHid[sb]);
       }
-      if (k + 1 < my_tiles) y_ln2(k + 1, ydn);
-      mbar_wait(barOut, (uint32_t)(k & 1), status, abort_flag);
-      tc_fence_after();
-      // E' = OUT -> bf16, staged in the hid buffers (every W2 product of the
-      // tile is done, and the next hid is written by these threads after the
-      // copy) and written with coalesced 16-byte stores (a TMA store measured
-      // slower here: its issuing thread holds the tile's barrier until the
-      // copy has read the staging)
-      {
-        float o[32];
-        tmem_ld16(ta + T_OUT + (k & 1) * 128 + c0, o);
-        tmem_ld16(ta + T_OUT + (k & 1) * 128 + c0 + 16, o + 16);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < 4; ++q) sw_st16(sH0, kBlk, row, c0 + q * 8, pack8(o + q * 8));
-      }
-      tc_fence_before();
-      named_bar_sync(1, kFfnEpi);
-      {
-        const int4 tl = tile_of(k);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int idx = q * kFfnEpi + (int)threadIdx.x, r = idx >> 4, cc = idx & 15;
-          if (r < tl.z)
-            reinterpret_cast<uint4*>(E_out + (int64_t)(tl.y + r) * kD)[cc] = sw_ld16(sH0, kBlk, r, cc * 8);
-        }
-      }
-      named_bar_sync(1, kFfnEpi);
     }
   }
   tc_fence_before();

@@ -28,6 +28,7 @@ def main():
     ap.add_argument("--items", type=int, default=None)
     ap.add_argument("--users", type=int, default=None)
     ap.add_argument("--links", type=int, default=None)
+    ap.add_argument("--window", type=int, default=None)
     ap.add_argument("--reps", type=int, default=3)
     a = ap.parse_args()
     over = {}
@@ -37,6 +38,8 @@ def main():
         over["B"] = a.users
     if a.links:
         over["l"] = a.links
+    if a.window:
+        over["window"] = a.window
     w = synth.workload(a.workload, **over)
     us, cs = synth.user_side(w), synth.candidate_side(w)
     x = pipeline.to_device(w, us, cs, synth.item_table(w))

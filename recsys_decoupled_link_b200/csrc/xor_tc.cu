@@ -1379,13 +1379,14 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
       // statistics over all 128 columns, read back from TMEM in column order
       float K = 0.f, s1 = 0.f, s2 = 0.f;
 #pragma unroll 1
-      for (int q = 0; q < 8; ++q) {
-        float o[16];
-        tmem_ld16(t_out + q * 16, o);
+      for (int q = 0; q < 4; ++q) {
+        float o[32];
+        tmem_ld16(t_out + q * 32, o);
+        tmem_ld16(t_out + q * 32 + 16, o + 16);
         tmem_ld_wait();
         if (q == 0) K = o[0];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 32; ++i) {
           const float t = o[i] - K;
           s1 += t;
           s2 = fmaf(t, t, s2);
@@ -1509,10 +1510,12 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
 // out_w[r, :] = x_r W_w for w < NW, x_r = LN1(X[r, :]) (LN) or X[r, :] (X bf16,
 // or fp32 for IN_F32), with W_w^T's K-major image at ws + img[w].  x_r enters
 // the products split into bf16 hi + lo (two MMAs each), so the fp32 outputs
-// carry no bf16 rounding of the operand.  One CTA per 128 rows, 512 threads:
-// thread (row, part) loads, normalises and splits its 32 columns, one thread
-// issues the products, and each thread writes its row's 32 columns of every
-// output (fp32, or fp16 for F16).
+// carry no bf16 rounding of the operand.  Persistent CTAs of 512 threads take
+// tiles of 128 rows (the weight images are loaded once per CTA): thread
+// (row, part) loads, normalises and splits its 32 columns, one thread issues
+// the products, and each output leaves through a [128 x 128] fp32 staging
+// buffer over the dead operands, a warp writing whole 512-byte rows (fp32, or
+// 256-byte fp16 rows for F16).
 struct RowsProjArgs {
   uint32_t img[3];
   void* out[3];
@@ -1528,6 +1531,7 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sm = align1k(smem_raw);
   uint8_t* sAh = sm;
   uint8_t* sAl = sm + 2 * kBlk;
+  uint8_t* stage = sm;   // 64 KB over sAh and sAl once a tile's products are done
   uint8_t* sW = sm + 4 * kBlk;
   float* red = reinterpret_cast<float*>(sm + (4 + 2 * NW) * kBlk);
   Cta c;
@@ -1543,61 +1547,82 @@ __global__ void __launch_bounds__(512, 1)
   const int part = warp >> 2;
   const int r = (warp & 3) * 32 + (threadIdx.x & 31);
   const int c0 = part * 32;
-  const int64_t R = (int64_t)blockIdx.x * kTile + r;
-  const bool valid = R < n;
-  {
-    float x[32];
-    if (valid) {
-      if constexpr (IN_F32) {
-        const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(Xv) + R * kD + c0);
+  const uint32_t ta = quad_addr(c);
+  const int64_t ntiles = (n + kTile - 1) / kTile;
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int64_t R = tile * kTile + r;
+    const bool valid = R < n;
+    {
+      float x[32];
+      if (valid) {
+        if constexpr (IN_F32) {
+          const float4* src =
+              reinterpret_cast<const float4*>(reinterpret_cast<const float*>(Xv) + R * kD + c0);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 v = src[q];
-          x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+          for (int q = 0; q < 8; ++q) {
+            const float4 v = src[q];
+            x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+          }
+        } else {
+          const uint4* src =
+              reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(Xv) + R * kD + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) unpack8(src[q], x + q * 8);
         }
       } else {
-        const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(Xv) + R * kD + c0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) unpack8(src[q], x + q * 8);
+        for (int i2 = 0; i2 < 32; ++i2) x[i2] = 0.f;
       }
-    } else {
-#pragma unroll
-      for (int i2 = 0; i2 < 32; ++i2) x[i2] = 0.f;
+      if (LN) layer_norm_part(x, c0, red, part, r);
+      split_part_st(sAh, sAl, r, c0, x);
     }
-    if (LN) layer_norm_part(x, c0, red, part, r);
-    split_part_st(sAh, sAl, r, c0, x);
-  }
-  fence_proxy_async_smem();
-  __syncthreads();
-  mbar_wait(&c.bar[0], 0, status, c.abort_flag);
-  if (threadIdx.x == 0) {
-    tc_fence_after();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tile == blockIdx.x) mbar_wait(&c.bar[0], 0, status, c.abort_flag);
+    if (threadIdx.x == 0) {
+      tc_fence_after();
 #pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        mma_tile(c.tmem + w * 128, smem_u32(sAh), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128,
+                 128, false);
+        mma_tile(c.tmem + w * 128, smem_u32(sAl), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128,
+                 128, true);
+      }
+    }
+    cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
+#pragma unroll 1
     for (int w = 0; w < NW; ++w) {
-      mma_tile(c.tmem + w * 128, smem_u32(sAh), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128, 128,
-               false);
-      mma_tile(c.tmem + w * 128, smem_u32(sAl), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128, 128,
-               true);
-    }
-  }
-  cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
-  const uint32_t ta = quad_addr(c);
+      float v[32];
+      tmem_ld16(ta + w * 128 + c0, v);
+      tmem_ld16(ta + w * 128 + c0 + 16, v + 16);
+      tmem_ld_wait();
 #pragma unroll
-  for (int w = 0; w < NW; ++w) {
-    float v[32];
-    tmem_ld16(ta + w * 128 + c0, v);
-    tmem_ld16(ta + w * 128 + c0 + 16, v + 16);
-    tmem_ld_wait();
-    if (valid) {
+      for (int q = 0; q < 8; ++q)
+        *f32_chunk(stage, r, c0 / 4 + q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      tc_fence_before();
+      __syncthreads();
+      const int64_t row0 = tile * kTile;
       if constexpr (F16) {
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(args.out[w]) + R * kD + c0);
+        __half* out = reinterpret_cast<__half*>(args.out[w]);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) dst[q] = pack8_f16(v + q * 8);
+        for (int t = threadIdx.x; t < kTile * 16; t += 512) {
+          const int rr = t >> 4, cp = t & 15;
+          if (row0 + rr < n) {
+            const float4 x0 = *f32_chunk(stage, rr, 2 * cp), x1 = *f32_chunk(stage, rr, 2 * cp + 1);
+            const float f8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            reinterpret_cast<uint4*>(out + (row0 + rr) * kD)[cp] = pack8_f16(f8);
+          }
+        }
       } else {
-        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(args.out[w]) + R * kD + c0);
+        float* out = reinterpret_cast<float*>(args.out[w]);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        for (int t = threadIdx.x; t < kTile * 32; t += 512) {
+          const int rr = t >> 5, cc = t & 31;
+          if (row0 + rr < n) reinterpret_cast<float4*>(out + (row0 + rr) * kD)[cc] = *f32_chunk(stage, rr, cc);
+        }
       }
+      __syncthreads();
     }
   }
   cta_teardown(c);
@@ -1605,87 +1630,215 @@ __global__ void __launch_bounds__(512, 1)
 
 // A[i, head h] = sum over keys phi(s q_i . k) v for history row i of user u
 // (fp32 throughout): the keys are u's l link rows (Kz, Vz) and its history
-// rows j with 0 < |i - j| <= win (Ke, Ve); phi = softmax (online: running max
-// and sum) or SiLU / (number of keys).  Thread = (row, head): four consecutive
-// threads share a row, so their 128-byte slices of a key row are one
-// coalesced 512 bytes.
-__global__ void __launch_bounds__(128)
+// rows j with 0 < |i - j| <= win (Ke, Ve); phi = softmax or SiLU / (number of
+// keys).  A block takes kWinRows consecutive history rows, warp w the eight
+// rows r0 + 8 w .. r0 + 8 w + 7.  Lane = (row group g, head h, quarter c):
+// it holds dims 8c .. 8c + 7 of head h of the four rows 4g .. 4g + 3 of the
+// warp, so every key value it loads feeds four rows.  Key rows are staged in
+// shared memory, kWinBuf at a time (first each user's link rows, then the
+// block's window range), and a warp walks its keys in lockstep: at a step the
+// lanes read one key row (the heads padded to 36 floats so that the eight
+// 16-byte slices of a load sit in distinct banks).  The four quarter sums of
+// a row are combined by a reduce-scatter over the lane's quad, after which
+// lane c owns row 4g + c: it applies the row's mask, keeps the row's softmax
+// state and hands its weight to the quad (four shuffles).  The softmax keeps
+// a reference value m per row and rescales only when a score passes
+// m + 8 (in log2 units; weights stay below 2^8), the warp then broadcasting
+// each row's factor; the result acc / sum is the same quotient as with the
+// running maximum.
+constexpr int kWinRows = 64;
+constexpr int kWinBuf = 96;
+constexpr int kWinPitch = 4 * (kDH + 4);
+constexpr int kWinSmem = 2 * kWinBuf * kWinPitch * 4;
+static_assert(kWinRows == 8 * 8, "eight warps of eight rows");
+
+__device__ __forceinline__ void win_stage(float* sK, float* sV, const float* __restrict__ K,
+                                          const float* __restrict__ V, int64_t row0, int nrows) {
+  for (int t = threadIdx.x; t < nrows * 32; t += blockDim.x) {
+    const int r = t >> 5, c4 = t & 31;
+    const int dst = r * kWinPitch + (c4 >> 3) * (kDH + 4) + (c4 & 7) * 4;
+    const int64_t src = (row0 + r) * kD + c4 * 4;
+    cp_async16(sK + dst, K + src, true);
+    cp_async16(sV + dst, V + src, true);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(256, 2)
     k_win_attn(const float* __restrict__ Qe, const float* __restrict__ Ke, const float* __restrict__ Ve,
                const float* __restrict__ Kz, const float* __restrict__ Vz,
                const int64_t* __restrict__ off, int64_t B, int64_t nh, int L, int win, float scale,
                int silu, float* __restrict__ att) {
+  constexpr unsigned kAll = 0xffffffffu;
+  extern __shared__ float4 win_smem[];
+  float* sK = reinterpret_cast<float*>(win_smem);
+  float* sV = sK + kWinBuf * kWinPitch;
   pdl_launch();
   pdl_wait();
-  const int64_t i = (int64_t)blockIdx.x * 32 + (threadIdx.x >> 2);
-  const int h = threadIdx.x & 3;
-  if (i >= nh) return;
-  const int64_t u = owner_of(off, B, i);
-  int64_t a = off[u], b = off[u + 1];
-  a = a < 0 ? 0 : a;
-  b = b > nh ? nh : b;
-  if (!(a <= i && i < b)) {
-    a = i;   // offsets that give no owner (flagged by the layer's schedule)
-    b = i + 1;
-  }
-  float q[32];
-  {
-    const float4* src = reinterpret_cast<const float4*>(Qe + i * kD + h * kDH);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c = lane & 3, h = (lane >> 2) & 3, g = lane >> 4;
+  const bool b0 = c & 1, b1 = c & 2;
+  const int quad = lane & ~3;
+  const int64_t r0 = (int64_t)blockIdx.x * kWinRows;
+  const int64_t w0 = r0 + warp * 8;      // the warp's first row
+  const int64_t rg = w0 + 4 * g;         // the lane's first row
+  const int64_t i = rg + c;              // the row this lane keeps the state of
+  const int64_t rlast = (r0 + kWinRows < nh ? r0 + kWinRows : nh) - 1;
+  // softmax scores in log2 units (exp(x) = 2^(x log2 e))
+  const float qs = silu ? scale : scale * kLog2e;
+  float q[4][8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float4 v = src[k];
-      q[4 * k] = v.x; q[4 * k + 1] = v.y; q[4 * k + 2] = v.z; q[4 * k + 3] = v.w;
-    }
-  }
-  const int64_t j0 = i - win > a ? i - win : a;
-  const int64_t j1 = i + win < b - 1 ? i + win : b - 1;
-  const float nkeys = (float)(L + (j1 - j0));   // the window excludes row i itself
-  float m = -INFINITY, ssum = 0.f, acc[32];
-#pragma unroll
-  for (int k = 0; k < 32; ++k) acc[k] = 0.f;
-  auto visit = [&](const float* krow, const float* vrow) {
-    const float4* ks = reinterpret_cast<const float4*>(krow);
-    float sdot = 0.f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float4 kv = __ldg(ks + k);
-      sdot = fmaf(q[4 * k], kv.x, sdot);
-      sdot = fmaf(q[4 * k + 1], kv.y, sdot);
-      sdot = fmaf(q[4 * k + 2], kv.z, sdot);
-      sdot = fmaf(q[4 * k + 3], kv.w, sdot);
-    }
-    sdot *= scale;
-    float p, corr;
-    if (silu) {
-      p = sdot / (1.0f + __expf(-sdot)) / nkeys;
-      corr = 1.f;
+  for (int r = 0; r < 4; ++r) {
+    const int64_t ir = rg + r;
+    if (ir < nh) {
+      const float4* src = reinterpret_cast<const float4*>(Qe + ir * kD + h * kDH + 8 * c);
+      const float4 v0 = src[0], v1 = src[1];
+      q[r][0] = v0.x * qs; q[r][1] = v0.y * qs; q[r][2] = v0.z * qs; q[r][3] = v0.w * qs;
+      q[r][4] = v1.x * qs; q[r][5] = v1.y * qs; q[r][6] = v1.z * qs; q[r][7] = v1.w * qs;
     } else {
-      const float mn = fmaxf(m, sdot);
-      corr = m == -INFINITY ? 0.f : __expf(m - mn);
-      p = __expf(sdot - mn);
-      ssum = fmaf(ssum, corr, p);
-      m = mn;
-    }
-    const float4* vs = reinterpret_cast<const float4*>(vrow);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float4 vv = __ldg(vs + k);
-      acc[4 * k] = fmaf(acc[4 * k], corr, p * vv.x);
-      acc[4 * k + 1] = fmaf(acc[4 * k + 1], corr, p * vv.y);
-      acc[4 * k + 2] = fmaf(acc[4 * k + 2], corr, p * vv.z);
-      acc[4 * k + 3] = fmaf(acc[4 * k + 3], corr, p * vv.w);
+      for (int k = 0; k < 8; ++k) q[r][k] = 0.f;
+    }
+  }
+  int64_t u = -1, j0 = 0, j1 = -1;
+  if (i < nh) {
+    u = owner_of(off, B, i);
+    int64_t a = off[u], b = off[u + 1];
+    a = a < 0 ? 0 : a;
+    b = b > nh ? nh : b;
+    if (!(a <= i && i < b)) {
+      a = i;   // offsets that give no owner (flagged by the layer's schedule)
+      b = i + 1;
+    }
+    j0 = i - win > a ? i - win : a;
+    j1 = i + win < b - 1 ? i + win : b - 1;
+  }
+  const float inv_n = 1.0f / (float)(L + (j1 - j0 > 0 ? j1 - j0 : 0));   // row i itself excluded
+  const int loff = h * (kDH + 4) + 8 * c;   // the lane's floats in a staged row
+  float m = -INFINITY, mthr = -INFINITY, ssum = 0.f, acc[4][8];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[r][k] = 0.f;
+  // The lane's four quarter dots of one key, reduced over the quad: lane c
+  // ends with the whole dot of row c.
+  auto dot = [&](const float* krow) {
+    const float4 k0 = reinterpret_cast<const float4*>(krow)[0];
+    const float4 k1 = reinterpret_cast<const float4*>(krow)[1];
+    float P[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      float x = q[r][0] * k0.x;
+      float y = q[r][1] * k0.y;
+      x = fmaf(q[r][2], k0.z, x);
+      y = fmaf(q[r][3], k0.w, y);
+      x = fmaf(q[r][4], k1.x, x);
+      y = fmaf(q[r][5], k1.y, y);
+      x = fmaf(q[r][6], k1.z, x);
+      y = fmaf(q[r][7], k1.w, y);
+      P[r] = x + y;
+    }
+    float s0 = b1 ? P[2] : P[0], s1 = b1 ? P[3] : P[1];
+    const float t0 = b1 ? P[0] : P[2], t1 = b1 ? P[1] : P[3];
+    s0 += __shfl_xor_sync(kAll, t0, 2);
+    s1 += __shfl_xor_sync(kAll, t1, 2);
+    return (b0 ? s1 : s0) + __shfl_xor_sync(kAll, b0 ? s0 : s1, 1);
+  };
+  auto accumulate = [&](const float* vrow, float p) {
+    const float4 v0 = reinterpret_cast<const float4*>(vrow)[0];
+    const float4 v1 = reinterpret_cast<const float4*>(vrow)[1];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float pr = __shfl_sync(kAll, p, quad | r);
+      acc[r][0] = fmaf(pr, v0.x, acc[r][0]);
+      acc[r][1] = fmaf(pr, v0.y, acc[r][1]);
+      acc[r][2] = fmaf(pr, v0.z, acc[r][2]);
+      acc[r][3] = fmaf(pr, v0.w, acc[r][3]);
+      acc[r][4] = fmaf(pr, v1.x, acc[r][4]);
+      acc[r][5] = fmaf(pr, v1.y, acc[r][5]);
+      acc[r][6] = fmaf(pr, v1.z, acc[r][6]);
+      acc[r][7] = fmaf(pr, v1.w, acc[r][7]);
     }
   };
-  for (int k = 0; k < L; ++k) {
-    const int64_t zr = u * L + k;
-    visit(Kz + zr * kD + h * kDH, Vz + zr * kD + h * kDH);
-  }
-  for (int64_t j = j0; j <= j1; ++j)
-    if (j != i) visit(Ke + j * kD + h * kDH, Ve + j * kD + h * kDH);
-  const float inv = silu ? 1.0f : 1.0f / ssum;
-  float4* dst = reinterpret_cast<float4*>(att + i * kD + h * kDH);
+  // two keys per step (independent dots, one rescale vote): staged rows ra, rb
+  auto visit2 = [&](int ra, bool va, int rb, bool vb) {
+    const float sa = dot(sK + ra * kWinPitch + loff);
+    const float sb = dot(sK + rb * kWinPitch + loff);
+    float pa, pb;
+    if (silu) {
+      pa = va ? sa * __frcp_rn(1.0f + __expf(-sa)) * inv_n : 0.f;
+      pb = vb ? sb * __frcp_rn(1.0f + __expf(-sb)) * inv_n : 0.f;
+    } else {
+      const float smax = fmaxf(va ? sa : -INFINITY, vb ? sb : -INFINITY);
+      const bool need = smax > mthr;
+      if (__any_sync(kAll, need)) {   // a new reference value in some row
+        float corr = 1.f;
+        if (need) {
+          corr = ex2_approx(m - smax);   // 0 while m is -inf
+          ssum *= corr;
+          m = smax;
+          mthr = smax + 8.0f;
+        }
 #pragma unroll
-  for (int k = 0; k < 8; ++k)
-    dst[k] = make_float4(acc[4 * k] * inv, acc[4 * k + 1] * inv, acc[4 * k + 2] * inv, acc[4 * k + 3] * inv);
+        for (int r = 0; r < 4; ++r) {
+          const float cr = __shfl_sync(kAll, corr, quad | r);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[r][k] *= cr;
+        }
+      }
+      pa = va ? ex2_approx(sa - m) : 0.f;
+      pb = vb ? ex2_approx(sb - m) : 0.f;
+      ssum += pa + pb;
+    }
+    accumulate(sV + ra * kWinPitch + loff, pa);
+    accumulate(sV + rb * kWinPitch + loff, pb);
+  };
+  // link keys, one pass per user owning rows of the block
+  const int64_t u_lo = owner_of(off, B, r0), u_hi = owner_of(off, B, rlast);
+  for (int64_t uu = u_lo; uu <= u_hi; ++uu) {
+    if (off[uu + 1] <= off[uu]) continue;   // no history rows
+    __syncthreads();
+    win_stage(sK, sV, Kz, Vz, uu * L, L);
+    if (!__any_sync(kAll, u == uu)) continue;
+    const bool mine = u == uu;
+#pragma unroll 1
+    for (int k = 0; k < L; k += 2) {
+      const bool second = k + 1 < L;
+      visit2(k, mine, second ? k + 1 : k, mine && second);
+    }
+  }
+  // window keys: rows [r0 - win, rlast + win] clipped to the history rows
+  const int64_t lo = r0 - win > 0 ? r0 - win : 0;
+  const int64_t hi = rlast + win < nh - 1 ? rlast + win : nh - 1;
+  const int64_t wlo = w0 - win, whi = w0 + 7 + win;   // the warp's key range
+  for (int64_t c0 = lo; c0 <= hi; c0 += kWinBuf) {
+    const int n = (int)(hi - c0 + 1 < kWinBuf ? hi - c0 + 1 : kWinBuf);
+    __syncthreads();
+    win_stage(sK, sV, Ke, Ve, c0, n);
+    // the lane's row's keys and the row itself, relative to c0 (clamped)
+    auto rel = [&](int64_t x) { return (int)(x < c0 - 1 ? -1 : (x > c0 + kWinBuf ? kWinBuf : x - c0)); };
+    const int klo = rel(j0), khi = rel(j1), kme = rel(i);
+    const int a = (int)((wlo > c0 ? wlo : c0) - c0);
+    const int b = (int)((whi < c0 + n - 1 ? whi : c0 + n - 1) - c0);
+#pragma unroll 1
+    for (int k = a; k <= b; k += 2) {
+      const int k2 = k + 1 <= b ? k + 1 : k;
+      visit2(k, klo <= k && k <= khi && k != kme, k2, k2 != k && klo <= k2 && k2 <= khi && k2 != kme);
+    }
+  }
+  const float den = silu ? 1.0f : ssum;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float inv = 1.0f / __shfl_sync(kAll, den, quad | r);
+    const int64_t ir = rg + r;
+    if (ir < nh) {
+      float4* dst = reinterpret_cast<float4*>(att + ir * kD + h * kDH + 8 * c);
+      dst[0] = make_float4(acc[r][0] * inv, acc[r][1] * inv, acc[r][2] * inv, acc[r][3] * inv);
+      dst[1] = make_float4(acc[r][4] * inv, acc[r][5] * inv, acc[r][6] * inv, acc[r][7] * inv);
+    }
+  }
 }
 
 // ------------------------------------------------------- record pre-merge
@@ -2151,15 +2304,21 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
         return LIME_ERR_CUDA;
       RowsProjArgs a3{{(uint32_t)Lw.img_q, (uint32_t)Lw.img_k, (uint32_t)Lw.img_v},
                       {ws + Lw.qe, ws + Lw.ke, ws + Lw.ve}};
-      int rc = launch_pdl(kq, dim3((unsigned)((nh + kTile - 1) / kTile)), dim3(512), smem3, st, 1,
+      auto pgrid = [&](int64_t rows) {
+        const int64_t t = (rows + kTile - 1) / kTile;
+        return dim3((unsigned)(t < sms ? t : sms));
+      };
+      int rc = launch_pdl(kq, pgrid(nh), dim3(512), smem3, st, 1,
                           (const void*)E_in, nh, g1, b1, (const uint8_t*)ws, a3, status);
       if (rc) return rc;
       RowsProjArgs a2{{(uint32_t)Lw.img_k, (uint32_t)Lw.img_v, 0u},
                       {ws + Lw.kz, ws + Lw.vz, nullptr}};
-      rc = launch_pdl(kz, dim3((unsigned)((nz + kTile - 1) / kTile)), dim3(512), smem2, st, 1,
+      rc = launch_pdl(kz, pgrid(nz), dim3(512), smem2, st, 1,
                       (const void*)Z_in, nz, g1, b1, (const uint8_t*)ws, a2, status);
       if (rc) return rc;
-      rc = launch_pdl(k_win_attn, dim3((unsigned)((nh + 31) / 32)), dim3(128), 0, st, 1,
+      if (!set_smem(k_win_attn, kWinSmem)) return LIME_ERR_CUDA;
+      rc = launch_pdl(k_win_attn, dim3((unsigned)((nh + kWinRows - 1) / kWinRows)), dim3(256),
+                      kWinSmem, st, 1,
                       (const float*)(ws + Lw.qe), (const float*)(ws + Lw.ke),
                       (const float*)(ws + Lw.ve), (const float*)(ws + Lw.kz),
                       (const float*)(ws + Lw.vz), off, B, nh, L, D.window, scale, silu ? 1 : 0,
@@ -2167,7 +2326,7 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
       if (rc) return rc;
       // Yd = A Wo (fp16), the attention delta the GatedMLP kernel adds to E
       RowsProjArgs a1{{(uint32_t)Lw.img_o, 0u, 0u}, {ws + Lw.yd, nullptr, nullptr}};
-      rc = launch_pdl(ko, dim3((unsigned)((nh + kTile - 1) / kTile)), dim3(512), smem1, st, 1,
+      rc = launch_pdl(ko, pgrid(nh), dim3(512), smem1, st, 1,
                       (const void*)(ws + Lw.att), nh, g1, b1, (const uint8_t*)ws, a1, status);
       if (rc) return rc;
     }

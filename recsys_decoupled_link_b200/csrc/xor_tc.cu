@@ -675,7 +675,7 @@ __global__ void __launch_bounds__(512, 1)
 // MMA group has started.
 constexpr int kXaEpi = 512;
 constexpr int kXaThreads = kXaEpi + 32;
-constexpr uint32_t kXaSmem = 1024 + 12 * kBlk + 1024 /* mu, rstd */ + 4096 /* red */ +
+constexpr uint32_t kXaSmem = 1024 + 12 * kBlk + 2048 /* mu, rstd x2 */ + 8192 /* red x2 */ +
                              1024 /* cv, dv */ + 2 * 2048 /* vec x2 */ +
                              kBlk /* one block of G'lo (phi = SiLU) */ + 256 /* barriers */;
 
@@ -699,9 +699,11 @@ __global__ void __launch_bounds__(kXaThreads, 1)
   uint8_t* sG = sm + 2 * kSlot;     // G' -> V_E
   uint8_t* sQ = sm + 3 * kSlot;     // Q'g -> VO
   uint8_t* rot = sm + 4 * kSlot;    // two alternating slots
-  float* smu = reinterpret_cast<float*>(sm + 6 * kSlot);   // [128] mu, then [128] rstd
-  float* red = smu + 256;                                   // [1024]
-  float* cvd = red + 1024;                                  // cv [128], dv [128]
+  // [128] mu, then [128] rstd, by tile parity
+  float* smu2 = reinterpret_cast<float*>(sm + 6 * kSlot);
+  float* redS = smu2 + 512;                                 // [1024] LN1 statistics
+  float* redX = redS + 1024;                                // [1024] softmax max / sum
+  float* cvd = redX + 1024;                                 // cv [128], dv [128]
   float* vecs = cvd + 256;                                  // 2 x (cQ, dQ, cG, dG)
   uint8_t* sGl = reinterpret_cast<uint8_t*>(vecs + 1024);   // a 64-column block of G'lo
   Cta c;
@@ -711,6 +713,12 @@ __global__ void __launch_bounds__(kXaThreads, 1)
   //      block landed, 15 its product done
   cta_setup(sGl + kBlk, 16, c);
   uint64_t* bar = c.bar;
+  // the epilogue's hand-offs to the issuer: one arrival per epilogue warp
+  if (threadIdx.x == 0) {
+    for (int i : {5, 11, 12, 13}) mbar_init(&bar[i], kXaEpi / 32);
+    fence_mbar_init();
+  }
+  __syncthreads();
   const int n_tiles = *reinterpret_cast<const int*>(ws + Lw.sched);
   const int4* tiles = reinterpret_cast<const int4*>(ws + Lw.tiles);
   const int warp = threadIdx.x >> 5;
@@ -835,11 +843,23 @@ __global__ void __launch_bounds__(kXaThreads, 1)
     const uint32_t ta = quad_addr(c);
     bf16* yd = reinterpret_cast<bf16*>(ws + Lw.yd);   // fp16 bits; rows copied as bytes
     float* part_rec = reinterpret_cast<float*>(ws + Lw.part);
-    if (HIST && threadIdx.x == 0) prefetch_tmap(&tmY);
+    // The four warps of a TMEM lane quadrant hold the same 32 rows (one part
+    // each): reductions over a row's parts synchronise the quadrant only, the
+    // hand-offs to the issuer are one arrival per warp, and each quadrant
+    // stores its own rows of Yd (its leader's bulk group).
+    const int quad = warp & 3;
+    const bool qlead = part == 0 && (threadIdx.x & 31) == 0;
+    auto qbar = [&]() { named_bar_sync(2 + quad, 128); };
+    auto warp_arrive = [&](uint64_t* b) {
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(b);
+    };
+    if (HIST && qlead) prefetch_tmap(&tmY);
     // LN1 statistics of this thread's row of an E tile (biased variance; see
     // layer_norm_part): mean and rstd into mu, rs, and every row's pair into
-    // smu (rstd in log2 units for phi = softmax).  Two epilogue barriers.
-    auto ln1_stats = [&](const uint8_t* tileE, float& mu, float& rs) {
+    // smu (rstd in log2 units for phi = softmax).  A quadrant barrier, then an
+    // epilogue barrier (the link softmax reads every row's pair).
+    auto ln1_stats = [&](const uint8_t* tileE, float* smu, float& mu, float& rs) {
       // the part's mean, then its centred sum of squares (a second read of
       // the tile's 32 values; see part_stats)
       float pm = 0.f, pq = 0.f;
@@ -861,11 +881,11 @@ __global__ void __launch_bounds__(kXaThreads, 1)
           pq = fmaf(dlt, dlt, pq);
         }
       }
-      red[part * 128 + row] = pm;
-      red[512 + part * 128 + row] = pq;
-      named_bar_sync(1, kXaEpi);
-      merge4_stats(red[row], red[128 + row], red[256 + row], red[384 + row], red[512 + row],
-                   red[640 + row], red[768 + row], red[896 + row], mu, rs);
+      redS[part * 128 + row] = pm;
+      redS[512 + part * 128 + row] = pq;
+      qbar();
+      merge4_stats(redS[row], redS[128 + row], redS[256 + row], redS[384 + row], redS[512 + row],
+                   redS[640 + row], redS[768 + row], redS[896 + row], mu, rs);
       if (part == 0) {
         smu[row] = mu;
         smu[128 + row] = SILU ? rs : rs * kLog2e;   // softmax: log2 units
@@ -888,6 +908,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
       const uint32_t tS2 = ta + 128 + (SPLIT ? 0u : (uint32_t)(it & 1) * 256);
       const int pr = hf * 128 + row;   // this lane's (head, link) pair in the link branch
       const float* vec = vecs + (it & 1) * 512;   // cQ, dQ, cG, dG
+      float* smu = smu2 + (it & 1) * 256;
       mbar_wait(&bar[2], ph, status, c.abort_flag);
       if (it == 0) mbar_wait(&bar[0], 0, status, c.abort_flag);
       mbar_wait(&bar[4], ph, status, c.abort_flag);
@@ -897,7 +918,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         mu_r = mu_n;
         rs_r = rs_n;
       } else {
-        ln1_stats(sA, mu_r, rs_r);
+        ln1_stats(sA, smu, mu_r, rs_r);
       }
       mbar_wait(&bar[1], ph, status, c.abort_flag);
       tc_fence_after();
@@ -943,16 +964,17 @@ __global__ void __launch_bounds__(kXaThreads, 1)
           // sum) = (0, valid tokens) makes the merge's total divide by N_u
 #pragma unroll
           for (int j = 0; j < 32; ++j) z[j] = c0 + j < nv && link ? silu_fast(z[j]) : 0.f;
-          if (HIST && it > 0 && threadIdx.x == 0) bulk_wait_read<0>();
-          named_bar_sync(1, kXaEpi);
+          if (HIST && it > 0 && qlead) bulk_wait_read<0>();
+          qbar();
           lm = 0.f;
           ls = (float)nv;
         } else {
-          red[part * 128 + row] = m;
-          // B held the previous tile's Yd staging: its store must have read it
-          if (HIST && it > 0 && threadIdx.x == 0) bulk_wait_read<0>();
-          named_bar_sync(1, kXaEpi);
-          m = fmaxf(fmaxf(red[row], red[128 + row]), fmaxf(red[256 + row], red[384 + row]));
+          redX[part * 128 + row] = m;
+          // B held the previous tile's Yd staging: the quadrant's store must
+          // have read its rows
+          if (HIST && it > 0 && qlead) bulk_wait_read<0>();
+          qbar();
+          m = fmaxf(fmaxf(redX[row], redX[128 + row]), fmaxf(redX[256 + row], redX[384 + row]));
           // masked scores are -inf and give 0; a lane with no link at all
           // has m = -inf and takes m = 0 instead
           if (m == -INFINITY) m = 0.f;
@@ -962,10 +984,10 @@ __global__ void __launch_bounds__(kXaThreads, 1)
             z[j] = ex2_approx(z[j] - m);
             s += z[j];
           }
-          red[512 + part * 128 + row] = s;
-          named_bar_sync(1, kXaEpi);
+          redX[512 + part * 128 + row] = s;
+          qbar();
           lm = m * kLn2;   // the record's max in natural-log units
-          ls = red[512 + row] + red[640 + row] + red[768 + row] + red[896 + row];
+          ls = redX[512 + row] + redX[640 + row] + redX[768 + row] + redX[896 + row];
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) sw_st16(sB, kBlk, row, c0 + q * 8, pack8(z + q * 8));
@@ -996,8 +1018,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_bar_sync(1, kXaEpi);
-      if (threadIdx.x == 0) mbar_arrive(&bar[12]);   // P2 V_E can start
+      warp_arrive(&bar[12]);   // P2 V_E starts once every warp has arrived
       if constexpr (HIST && !SPLIT) {
         // history softmax over the user's L links: part = head, P over the E tile
         const int h = part;
@@ -1064,15 +1085,15 @@ __global__ void __launch_bounds__(kXaThreads, 1)
           float m = z[0];
 #pragma unroll
           for (int k = 1; k < 32; ++k) m = fmaxf(m, z[k]);
-          red[part * 128 + row] = m;
-          named_bar_sync(1, kXaEpi);
-          m = fmaxf(m, red[(part ^ 1) * 128 + row]);
+          redX[part * 128 + row] = m;
+          qbar();
+          m = fmaxf(m, redX[(part ^ 1) * 128 + row]);
           float s = 0.f;
 #pragma unroll
           for (int k = 0; k < 32; ++k) { z[k] = ex2_approx(z[k] - m); s += z[k]; }
-          red[512 + part * 128 + row] = s;
-          named_bar_sync(1, kXaEpi);
-          const float inv = 1.0f / (s + red[512 + (part ^ 1) * 128 + row]);
+          redX[512 + part * 128 + row] = s;
+          qbar();
+          const float inv = 1.0f / (s + redX[512 + (part ^ 1) * 128 + row]);
 #pragma unroll
           for (int k = 0; k < 32; ++k) z[k] *= inv;
         }
@@ -1082,8 +1103,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
       if (HIST) {
         fence_proxy_async_smem();
         tc_fence_before();
-        named_bar_sync(1, kXaEpi);
-        if (threadIdx.x == 0) mbar_arrive(&bar[13]);   // Yd = P VO can start
+        warp_arrive(&bar[13]);   // Yd = P VO starts once every warp has arrived
       }
       mbar_wait(&bar[9], ph, status, c.abort_flag);
       tc_fence_after();
@@ -1104,8 +1124,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         if constexpr (SPLIT) {
           // the next half's link scores reuse these columns
           tc_fence_before();
-          named_bar_sync(1, kXaEpi);
-          if (threadIdx.x == 0) mbar_arrive(&bar[5]);
+          warp_arrive(&bar[5]);
         }
       }
       if constexpr (kPre) {
@@ -1114,7 +1133,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         pre = t + (int)gridDim.x < n_tiles;
         if (pre) {
           mbar_wait(&bar[2], ph ^ 1u, status, c.abort_flag);
-          ln1_stats(sB, mu_n, rs_n);
+          ln1_stats(sB, smu2 + ((it + 1) & 1) * 256, mu_n, rs_n);
         }
       }
       if (HIST) mbar_wait(&bar[10], ph, status, c.abort_flag);   // P has been read
@@ -1126,21 +1145,21 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         tmem_ld16(ta + kYd + c0 + 16, y + 16);
         tmem_ld_wait();
         tc_fence_before();
-        named_bar_sync(1, kXaEpi);   // every thread has read P (the MMA is done) and Yd
-        if (threadIdx.x == 0) mbar_arrive(&bar[11]);
+        warp_arrive(&bar[11]);   // this warp has read its Yd columns (P: the MMA is done)
+        // the staging rows are the quadrant's own: P's rows, which Yd has read
 #pragma unroll
         for (int q = 0; q < 4; ++q) sw_st16(sA, kBlk, row, c0 + q * 8, pack8_f16(y + q * 8));
         fence_proxy_async_smem();
-        named_bar_sync(1, kXaEpi);
+        qbar();
         if (nv == kTile) {
-          if (threadIdx.x == 0) {
-            tma_store_2d(&tmY, sA, 0, r0);
-            tma_store_2d(&tmY, sA + kBlk, 64, r0);
+          if (qlead) {
+            tma_store_2d(&tmY, sA + quad * 4096, 0, r0 + 32 * quad);
+            tma_store_2d(&tmY, sA + kBlk + quad * 4096, 64, r0 + 32 * quad);
             bulk_commit();
           }
         } else {
-          for (int idx = (int)threadIdx.x; idx < 2048; idx += kXaEpi) {
-            const int r = idx >> 4, cc = idx & 15;
+          for (int idx = part * 32 + (threadIdx.x & 31); idx < 512; idx += 128) {
+            const int r = quad * 32 + (idx >> 4), cc = idx & 15;
             if (r < nv) reinterpret_cast<uint4*>(yd + (int64_t)(r0 + r) * kD)[cc] = sw_ld16(sA, kBlk, r, cc * 8);
           }
         }
@@ -1151,7 +1170,7 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         t += gridDim.x;
       }
     }
-    if (threadIdx.x == 0) bulk_wait<0>();
+    if (qlead) bulk_wait<0>();
   }
   cta_teardown(c);
 }
@@ -1507,124 +1526,136 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
 //                far too little work per query for a tensor-core tile)
 //   k_rows_proj  Yd = A Wo (fp16), which the GatedMLP kernel reads as usual.
 
-// out_w[r, :] = x_r W_w for w < NW, x_r = LN1(X[r, :]) (LN) or X[r, :] (X bf16,
-// or fp32 for IN_F32), with W_w^T's K-major image at ws + img[w].  x_r enters
-// the products split into bf16 hi + lo (two MMAs each), so the fp32 outputs
-// carry no bf16 rounding of the operand.  Persistent CTAs of 512 threads take
-// tiles of 128 rows (the weight images are loaded once per CTA): thread
-// (row, part) loads, normalises and splits its 32 columns, one thread issues
-// the products, and each output leaves through a [128 x 128] fp32 staging
-// buffer over the dead operands, a warp writing whole 512-byte rows (fp32, or
-// 256-byte fp16 rows for F16).
-struct RowsProjArgs {
+// out_w[r, :] = x_r W_w, x_r = LN1(X[r, :]) (LN) or X[r, :] (X bf16, or fp32
+// for IN_F32), with W_w^T's K-major image at ws + img[w].  x_r enters the
+// products split into bf16 hi + lo (two MMAs each), so the fp32 outputs carry
+// no bf16 rounding of the operand.  Two jobs share one persistent launch: job
+// 0 (n0 rows of x[0], outputs o[0 .. NW)) and job 1 (n1 rows of x[1], the
+// products with images 1 and 2 into o[3], o[4]; the link rows' K and V beside
+// the history rows' Q, K, V).  Persistent CTAs of 512 threads walk the 128-row
+// tiles of both jobs; the weight images are loaded once per CTA.  A tile's
+// rows arrive by TMA (the next tile's load is issued as soon as this one has
+// been read), thread (row, part) normalises and splits its 32 columns, one
+// thread issues the products, and each output leaves by TMA tensor stores from
+// a staging buffer over the dead operands (128-byte swizzled boxes: four
+// fp32 boxes of 32 columns, or two fp16 boxes of 64; rows past the end are
+// clipped by the stores and zero-filled by the loads).
+struct RowsMaps {
+  CUtensorMap x[2];
+  CUtensorMap o[5];
+};
+struct RowsImgs {
   uint32_t img[3];
-  void* out[3];
 };
 
 template <int NW, bool LN, bool IN_F32, bool F16>
 __global__ void __launch_bounds__(512, 1)
-    k_rows_proj(const void* __restrict__ Xv, int64_t n, const bf16* __restrict__ g,
-                const bf16* __restrict__ b, const uint8_t* __restrict__ ws, RowsProjArgs args,
-                unsigned* status) {
+    k_rows_proj(const __grid_constant__ RowsMaps tm, int64_t n0, int64_t n1,
+                const bf16* __restrict__ g, const bf16* __restrict__ b,
+                const uint8_t* __restrict__ ws, RowsImgs im, unsigned* status) {
   constexpr uint32_t kCols = NW == 1 ? 128 : (NW == 2 ? 256 : 512);
+  constexpr uint32_t kXBytes = IN_F32 ? 4 * kBlk : 2 * kBlk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1k(smem_raw);
   uint8_t* sAh = sm;
   uint8_t* sAl = sm + 2 * kBlk;
   uint8_t* stage = sm;   // 64 KB over sAh and sAl once a tile's products are done
   uint8_t* sW = sm + 4 * kBlk;
-  float* red = reinterpret_cast<float*>(sm + (4 + 2 * NW) * kBlk);
+  uint8_t* sX = sW + NW * 2 * kBlk;
+  float* red = reinterpret_cast<float*>(sX + kXBytes);
   Cta c;
-  cta_setup(sm + (4 + 2 * NW) * kBlk + kLnBytes, 2, c, kCols);
+  // bar: 0 weights, 1 products, 2 row tile
+  cta_setup(sX + kXBytes + kLnBytes, 3, c, kCols);
   if (LN) ln_stage(red + 1024, g, b);
-  uint32_t mph = 0;
+  const int64_t T0 = (n0 + kTile - 1) / kTile, T = T0 + (n1 + kTile - 1) / kTile;
+  auto load_x = [&](int64_t tile) {
+    const bool j1 = tile >= T0;
+    const int row0 = (int)((j1 ? tile - T0 : tile) * kTile);
+    mbar_arrive_expect_tx(&c.bar[2], kXBytes);
+#pragma unroll
+    for (int p = 0; p < (IN_F32 ? 4 : 2); ++p)
+      tma_load_2d(sX + p * kBlk, &tm.x[j1 ? 1 : 0], p * (IN_F32 ? 32 : 64), row0, &c.bar[2]);
+  };
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(&c.bar[0], NW * 2 * kBlk);
 #pragma unroll
-    for (int w = 0; w < NW; ++w) bulk_load(sW + w * 2 * kBlk, ws + args.img[w], 2 * kBlk, &c.bar[0]);
+    for (int w = 0; w < NW; ++w) bulk_load(sW + w * 2 * kBlk, ws + im.img[w], 2 * kBlk, &c.bar[0]);
+    if ((int64_t)blockIdx.x < T) load_x(blockIdx.x);
   }
   const int warp = threadIdx.x >> 5;
   const int part = warp >> 2;
   const int r = (warp & 3) * 32 + (threadIdx.x & 31);
   const int c0 = part * 32;
   const uint32_t ta = quad_addr(c);
-  const int64_t ntiles = (n + kTile - 1) / kTile;
-  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int64_t R = tile * kTile + r;
-    const bool valid = R < n;
-    {
-      float x[32];
-      if (valid) {
-        if constexpr (IN_F32) {
-          const float4* src =
-              reinterpret_cast<const float4*>(reinterpret_cast<const float*>(Xv) + R * kD + c0);
+  uint32_t mph = 0;
+  int k = 0;
+  for (int64_t tile = blockIdx.x; tile < T; tile += gridDim.x, ++k) {
+    const bool j1 = tile >= T0;
+    const int row0 = (int)((j1 ? tile - T0 : tile) * kTile);
+    mbar_wait(&c.bar[2], (uint32_t)k & 1u, status, c.abort_flag);
+    float x[32];
+    if constexpr (IN_F32) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 v = src[q];
-            x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
-          }
-        } else {
-          const uint4* src =
-              reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(Xv) + R * kD + c0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) unpack8(src[q], x + q * 8);
-        }
-      } else {
-#pragma unroll
-        for (int i2 = 0; i2 < 32; ++i2) x[i2] = 0.f;
+      for (int j = 0; j < 8; ++j) {
+        const float4 v = *reinterpret_cast<const float4*>(sX + part * kBlk + r * 128 + ((j ^ (r & 7)) << 4));
+        x[4 * j] = v.x; x[4 * j + 1] = v.y; x[4 * j + 2] = v.z; x[4 * j + 3] = v.w;
       }
-      if (LN) layer_norm_part(x, c0, red, part, r);
-      split_part_st(sAh, sAl, r, c0, x);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) unpack8(sw_ld16(sX, kBlk, r, c0 + q * 8), x + q * 8);
     }
+    if (LN) layer_norm_part(x, c0, red, part, r);
+    // the previous tile's stores have read the staging (= this tile's operands)
+    if (threadIdx.x == 0) bulk_wait_read<0>();
+    __syncthreads();   // every thread has read the row tile
+    if (threadIdx.x == 0 && tile + gridDim.x < T) load_x(tile + gridDim.x);
+    split_part_st(sAh, sAl, r, c0, x);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tile == blockIdx.x) mbar_wait(&c.bar[0], 0, status, c.abort_flag);
+    if (k == 0) mbar_wait(&c.bar[0], 0, status, c.abort_flag);
+    const int nout = j1 ? 2 : NW;
     if (threadIdx.x == 0) {
       tc_fence_after();
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        mma_tile(c.tmem + w * 128, smem_u32(sAh), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128,
-                 128, false);
-        mma_tile(c.tmem + w * 128, smem_u32(sAl), kBlk, smem_u32(sW + w * 2 * kBlk), kBlk, 128,
-                 128, true);
+      for (int w = 0; w < nout; ++w) {
+        const uint8_t* wimg = sW + (j1 ? w + 1 : w) * 2 * kBlk;
+        mma_tile(c.tmem + w * 128, smem_u32(sAh), kBlk, smem_u32(wimg), kBlk, 128, 128, false);
+        mma_tile(c.tmem + w * 128, smem_u32(sAl), kBlk, smem_u32(wimg), kBlk, 128, 128, true);
       }
     }
     cta_mma_wait(&c.bar[1], mph, status, c.abort_flag);
 #pragma unroll 1
-    for (int w = 0; w < NW; ++w) {
+    for (int w = 0; w < nout; ++w) {
       float v[32];
       tmem_ld16(ta + w * 128 + c0, v);
       tmem_ld16(ta + w * 128 + c0 + 16, v + 16);
       tmem_ld_wait();
+      if (w > 0) {
+        if (threadIdx.x == 0) bulk_wait_read<0>();   // the previous output's stores
+        __syncthreads();
+      }
+      if constexpr (F16) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        *f32_chunk(stage, r, c0 / 4 + q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        for (int q = 0; q < 4; ++q) sw_st16(stage, kBlk, r, c0 + q * 8, pack8_f16(v + q * 8));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<float4*>(stage + part * kBlk + r * 128 + ((j ^ (r & 7)) << 4)) =
+              make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      }
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
-      const int64_t row0 = tile * kTile;
-      if constexpr (F16) {
-        __half* out = reinterpret_cast<__half*>(args.out[w]);
+      if (threadIdx.x == 0) {
+        const CUtensorMap* om = &tm.o[j1 ? 3 + w : w];
 #pragma unroll
-        for (int t = threadIdx.x; t < kTile * 16; t += 512) {
-          const int rr = t >> 4, cp = t & 15;
-          if (row0 + rr < n) {
-            const float4 x0 = *f32_chunk(stage, rr, 2 * cp), x1 = *f32_chunk(stage, rr, 2 * cp + 1);
-            const float f8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-            reinterpret_cast<uint4*>(out + (row0 + rr) * kD)[cp] = pack8_f16(f8);
-          }
-        }
-      } else {
-        float* out = reinterpret_cast<float*>(args.out[w]);
-#pragma unroll
-        for (int t = threadIdx.x; t < kTile * 32; t += 512) {
-          const int rr = t >> 5, cc = t & 31;
-          if (row0 + rr < n) reinterpret_cast<float4*>(out + (row0 + rr) * kD)[cc] = *f32_chunk(stage, rr, cc);
-        }
+        for (int p = 0; p < (F16 ? 2 : 4); ++p)
+          tma_store_2d(om, stage + p * kBlk, p * (F16 ? 64 : 32), row0);
+        bulk_commit();
       }
-      __syncthreads();
     }
   }
+  if (threadIdx.x == 0) bulk_wait<0>();
   cta_teardown(c);
 }
 
@@ -2275,7 +2306,7 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
   if (nh > 0) {
     CUtensorMap tmE, tmY;
     if (!make_tmap_2d_bf16(&tmE, E_in, kD, (uint64_t)nh, kD * 2, 64, kTile) ||
-        !make_tmap_2d_f16(&tmY, ws + Lw.yd, kD, (uint64_t)nh, kD * 2, 64, kTile))
+        !make_tmap_2d_f16(&tmY, ws + Lw.yd, kD, (uint64_t)nh, kD * 2, 64, 32))   // a quadrant's rows
       return LIME_ERR_CUDA;
     tmE_ffn = tmE;
     const int64_t tiles_hi = Lw.max_tiles;
@@ -2294,27 +2325,26 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
       const bf16* g1 = (const bf16*)w.g1;
       const bf16* b1 = (const bf16*)w.b1;
       // LN1 and Q, K, V of the history rows; K, V of the link rows (fp32)
-      constexpr int smem3 = 1024 + 10 * kBlk + kLnBytes + kBarBytes;
-      constexpr int smem2 = 1024 + 8 * kBlk + kLnBytes + kBarBytes;
-      constexpr int smem1 = 1024 + 6 * kBlk + kLnBytes + kBarBytes;
+      constexpr int smem3 = 1024 + 12 * kBlk + kLnBytes + kBarBytes;
+      constexpr int smem1 = 1024 + 10 * kBlk + kLnBytes + kBarBytes;
       auto kq = k_rows_proj<3, true, false, false>;
-      auto kz = k_rows_proj<2, true, false, false>;
       auto ko = k_rows_proj<1, false, true, true>;
-      if (!set_smem(kq, smem3) || !set_smem(kz, smem2) || !set_smem(ko, smem1))
-        return LIME_ERR_CUDA;
-      RowsProjArgs a3{{(uint32_t)Lw.img_q, (uint32_t)Lw.img_k, (uint32_t)Lw.img_v},
-                      {ws + Lw.qe, ws + Lw.ke, ws + Lw.ve}};
-      auto pgrid = [&](int64_t rows) {
-        const int64_t t = (rows + kTile - 1) / kTile;
-        return dim3((unsigned)(t < sms ? t : sms));
+      if (!set_smem(kq, smem3) || !set_smem(ko, smem1)) return LIME_ERR_CUDA;
+      auto f32map = [](CUtensorMap* m, void* base, int64_t rows) {
+        return make_tmap_2d_f32(m, base, kD, (uint64_t)rows, kD * 4, 32, kTile);
       };
-      int rc = launch_pdl(kq, pgrid(nh), dim3(512), smem3, st, 1,
-                          (const void*)E_in, nh, g1, b1, (const uint8_t*)ws, a3, status);
-      if (rc) return rc;
-      RowsProjArgs a2{{(uint32_t)Lw.img_k, (uint32_t)Lw.img_v, 0u},
-                      {ws + Lw.kz, ws + Lw.vz, nullptr}};
-      rc = launch_pdl(kz, pgrid(nz), dim3(512), smem2, st, 1,
-                      (const void*)Z_in, nz, g1, b1, (const uint8_t*)ws, a2, status);
+      auto pgrid = [&](int64_t tiles) { return dim3((unsigned)(tiles < sms ? tiles : sms)); };
+      const int64_t th = (nh + kTile - 1) / kTile, tz = (nz + kTile - 1) / kTile;
+      RowsMaps m3{};
+      m3.x[0] = tmE;
+      if (!make_tmap_2d_bf16(&m3.x[1], Z_in, kD, (uint64_t)nz, kD * 2, 64, kTile) ||
+          !f32map(&m3.o[0], ws + Lw.qe, nh) || !f32map(&m3.o[1], ws + Lw.ke, nh) ||
+          !f32map(&m3.o[2], ws + Lw.ve, nh) || !f32map(&m3.o[3], ws + Lw.kz, nz) ||
+          !f32map(&m3.o[4], ws + Lw.vz, nz))
+        return LIME_ERR_CUDA;
+      const RowsImgs i3{{(uint32_t)Lw.img_q, (uint32_t)Lw.img_k, (uint32_t)Lw.img_v}};
+      int rc = launch_pdl(kq, pgrid(th + tz), dim3(512), smem3, st, 1, m3, nh, nz, g1, b1,
+                          (const uint8_t*)ws, i3, status);
       if (rc) return rc;
       if (!set_smem(k_win_attn, kWinSmem)) return LIME_ERR_CUDA;
       rc = launch_pdl(k_win_attn, dim3((unsigned)((nh + kWinRows - 1) / kWinRows)), dim3(256),
@@ -2325,9 +2355,13 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
                       (float*)(ws + Lw.att));
       if (rc) return rc;
       // Yd = A Wo (fp16), the attention delta the GatedMLP kernel adds to E
-      RowsProjArgs a1{{(uint32_t)Lw.img_o, 0u, 0u}, {ws + Lw.yd, nullptr, nullptr}};
-      rc = launch_pdl(ko, pgrid(nh), dim3(512), smem1, st, 1,
-                      (const void*)(ws + Lw.att), nh, g1, b1, (const uint8_t*)ws, a1, status);
+      RowsMaps m1{};
+      if (!f32map(&m1.x[0], ws + Lw.att, nh) ||
+          !make_tmap_2d_f16(&m1.o[0], ws + Lw.yd, kD, (uint64_t)nh, kD * 2, 64, kTile))
+        return LIME_ERR_CUDA;
+      const RowsImgs i1{{(uint32_t)Lw.img_o, 0u, 0u}};
+      rc = launch_pdl(ko, pgrid(th), dim3(512), smem1, st, 1, m1, nh, (int64_t)0, g1, b1,
+                      (const uint8_t*)ws, i1, status);
       if (rc) return rc;
     }
   }

@@ -267,7 +267,8 @@ def sample_users(counts, k, g):
     return sorted({nonempty[i] for i in pick} | {longest})
 
 
-FULL = ["standard", "long", "large_cand", "ragged16", "ragged32", "ragged64", "tiny"]
+FULL = ["standard", "long", "large_cand", "ragged16", "ragged32", "ragged64", "tiny",
+        "standard_window", "ragged32_window"]
 
 
 @pytest.mark.slow
@@ -279,8 +280,12 @@ def test_full_size_sampled(case):
     end (its own cache rows for those users' candidates and its own L^P) and
     isolated (the GPU's cache rows and L^P), plus 65,536 sampled cache rows."""
     base, over = case, {}
-    if case.startswith("ragged"):
-        base, over = "ragged", dict(l=int(case[6:]))
+    if case.endswith("_window"):
+        # LIME-XOR+Window at the pages' half-width l/2 (several row tiles per
+        # persistent CTA in the window kernels)
+        base, over = case[:-len("_window")], dict(window=16)
+    if base.startswith("ragged"):
+        base, over = "ragged", dict(over, l=int(base[6:]))
     w = synth.workload(base, **over)
     us = synth.user_side(w)
     cs = synth.candidate_side(w)
@@ -298,7 +303,8 @@ def test_full_size_sampled(case):
     offs = us.hist_offsets.numpy()
     layers = oracle_layer_weights(us)
     Z0 = oracle_Z0(w, us)
-    _, LP_ref = O.user_encode(f64(us.E), offs, Z0, layers, w.H, users=users)
+    _, LP_ref = O.user_encode(f64(us.E), offs, Z0, layers, w.H, users=users, phi=w.phi,
+                              window=w.window)
     LP_cpu = LP.cpu()
     chain = w.layers + (1 if w.c > 0 else 0)
     got_lp = torch.stack([LP_cpu[u] for u in users])

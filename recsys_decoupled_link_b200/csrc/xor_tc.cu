@@ -1202,7 +1202,7 @@ constexpr int kFfnGrp = 256;
 constexpr int kFfnTiles = 32;  // tile descriptors of a CTA kept in shared memory
 constexpr int kFfnSmem = 1024 + 14 * kBlk + 1024 + kFfnTiles * 16 + 256;
 
-__global__ void __launch_bounds__(kFfnEpi + 64, 1)
+__global__ void __launch_bounds__(kFfnEpi + 96, 1)
     k_hist_ffn(const __grid_constant__ CUtensorMap tmE, const bf16* __restrict__ g2,
                const bf16* __restrict__ b2, const uint8_t* __restrict__ ws, LayerWs Lw,
                bf16* __restrict__ E_out, unsigned* status) {
@@ -1268,16 +1268,11 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
   };
   const int n_chunks = my_tiles * (kF / 64);
 
-  if (warp == kFfnEpi / 32 + 1) {
-    // loader: the W1|W3 ring, the E tiles and W2.  It runs apart from the MMA
-    // issuer because tcgen05.mma issue stalls while the tensor pipe is busy,
-    // which would hold back the next loads.
+  if (warp == kFfnEpi / 32 + 2) {
+    // E-tile loader: E(0), E(1), then E(k+2) into buffer k%2 once the row
+    // group has read tile k's E' staging out of it.  Apart from the weight
+    // loader, so the W1|W3 ring never waits on the readout.
     if (lane == 0 && my_tiles > 0) {
-      auto load_w13 = [&](int g) {
-        const int s = g & 1, ch = g & 3;
-        mbar_arrive_expect_tx(&barWt[s], 2 * kBlk);
-        bulk_load(sW13 + s * 2 * kBlk, ws + Lw.img_13 + ch * 2 * kBlk, 2 * kBlk, &barWt[s]);
-      };
       auto load_e = [&](int k) {
         const int4 tl = tile_of(k);
         uint8_t* dst = sE0 + (k & 1) * 2 * kBlk;
@@ -1291,41 +1286,59 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
       prefetch_tmap(&tmE);
       load_e(0);
       if (my_tiles > 1) load_e(1);
+      for (int k = 0; k + 2 < my_tiles; ++k) {
+        // buffer k%2 held h2(k) and then tile k's E' staging
+        if (!mbar_wait(barSE, k & 1, status, abort_flag)) break;
+        load_e(k + 2);
+      }
+    }
+  } else if (warp == kFfnEpi / 32 + 1) {
+    // weight loader: the W1|W3 ring and W2.  It runs apart from the MMA
+    // issuer because tcgen05.mma issue stalls while the tensor pipe is busy,
+    // which would hold back the next loads.
+    if (lane == 0 && my_tiles > 0) {
+      auto load_w13 = [&](int g) {
+        const int s = g & 1, ch = g & 3;
+        mbar_arrive_expect_tx(&barWt[s], 2 * kBlk);
+        bulk_load(sW13 + s * 2 * kBlk, ws + Lw.img_13 + ch * 2 * kBlk, 2 * kBlk, &barWt[s]);
+      };
       load_w13(0);
       if (n_chunks > 1) load_w13(1);
       mbar_arrive_expect_tx(barW2in, 4 * kBlk);
       bulk_load(sW2, ws + Lw.img_2, 4 * kBlk, barW2in);
-      for (int g = 0; g < n_chunks; ++g) {
-        if (g >= 1) {
-          // G(g-1) done: its ring slot takes chunk g+1
-          if (!mbar_wait(&barG[(g - 1) & 1], (uint32_t)(((g - 1) >> 1) & 1), status, abort_flag))
-            break;
-          if (g + 1 < n_chunks) load_w13(g + 1);
-        }
-        const int k = g / (kF / 64);
-        if (g % (kF / 64) == kF / 64 - 1 && k + 2 < my_tiles) {
-          // E(k+2) goes to buffer k%2, which held h2(k) and then tile k's E'
-          // staging: wait until the row group has read the staging out
-          if (!mbar_wait(barSE, k & 1, status, abort_flag)) break;
-          load_e(k + 2);
-        }
+      for (int g = 1; g + 1 < n_chunks; ++g) {
+        // G(g-1) done: its ring slot takes chunk g+1
+        if (!mbar_wait(&barG[(g - 1) & 1], (uint32_t)(((g - 1) >> 1) & 1), status, abort_flag))
+          break;
+        load_w13(g + 1);
       }
     }
   } else if (warp == kFfnEpi / 32) {
     // MMA issuer
     if (lane == 0 && my_tiles > 0) {
-      bool ok = mbar_wait(barW2in, 0, status, abort_flag);
-      for (int k = 0; k < my_tiles && ok; ++k) {
-        if (!(ok = mbar_wait(barH2, k & 1, status, abort_flag))) break;
+      // G(k, c) = h2(k) [W1c | W3c] into gate buffer g%2 (g = 4k + c)
+      auto gate = [&](int k, int c) {
+        const int g = k * (kF / 64) + c, s = g & 1;
+        if (!mbar_wait(&barWt[s], (uint32_t)((g >> 1) & 1), status, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t a_h2 = smem_u32(sE0 + (k & 1) * 2 * kBlk);
+        mma_tile(tmem + s * 128, smem_u32(sE0 + (k & 1) * 2 * kBlk), kBlk,
+                 smem_u32(sW13 + s * 2 * kBlk), kBlk, 128, 128, false);
+        mma_commit(&barG[s]);
+        return true;
+      };
+      bool ok = mbar_wait(barW2in, 0, status, abort_flag);
+      bool g0 = false;   // G(k, 0) already issued (ahead of tile k-1's last W2 product)
+      for (int k = 0; k < my_tiles && ok; ++k) {
         const uint32_t t_out = tmem + T_OUT + (k & 1) * 128;
-        for (int c = 0; c < kF / 64; ++c) {
-          const int g = k * (kF / 64) + c, s = g & 1;
-          if (!(ok = mbar_wait(&barWt[s], (uint32_t)((g >> 1) & 1), status, abort_flag))) break;
+        if (!g0) {
+          if (!(ok = mbar_wait(barH2, k & 1, status, abort_flag))) break;
           tc_fence_after();
-          mma_tile(tmem + s * 128, a_h2, kBlk, smem_u32(sW13 + s * 2 * kBlk), kBlk, 128, 128, false);
-          mma_commit(&barG[s]);
+          if (!(ok = gate(k, 0))) break;
+        }
+        g0 = false;
+        for (int c = 0; c < kF / 64; ++c) {
+          const int g = k * (kF / 64) + c;
+          if (c >= 1 && !(ok = gate(k, c))) break;
           if (c >= 1) {
             const int pg = g - 1, pb = pg & 1;
             if (!(ok = mbar_wait(&barHid[pb], (uint32_t)((pg >> 1) & 1), status, abort_flag))) break;
@@ -1337,6 +1350,28 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
         }
         if (!ok) break;
         const int lg = k * (kF / 64) + kF / 64 - 1, lb = lg & 1;
+        // Whichever is ready first: the next tile's first gate product (its
+        // gate buffer is the other one) or this tile's last W2 product.
+        if (k + 1 < my_tiles) {
+          const uint64_t t0 = global_ns();
+          for (;;) {
+            if (mbar_try_wait_ns(barH2, (k + 1) & 1, 20)) {
+              tc_fence_after();
+              if (!(ok = gate(k + 1, 0))) break;
+              g0 = true;
+              break;
+            }
+            if (mbar_try_wait_ns(&barHid[lb], (uint32_t)((lg >> 1) & 1), 20)) break;
+            if (*abort_flag) { ok = false; break; }
+            if (global_ns() - t0 > 2000000000ull) {
+              raise_flag(status, LIME_FLAG_TIMEOUT);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+          }
+          if (!ok) break;
+        }
         if (!(ok = mbar_wait(&barHid[lb], (uint32_t)((lg >> 1) & 1), status, abort_flag))) break;
         tc_fence_after();
         mma_tile(t_out, smem_u32(sH0 + lb * kBlk), kBlk, smem_u32(sW2 + (kF / 64 - 1) * kBlk), kBlk,
@@ -1377,6 +1412,12 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
       uint8_t* sE = sE0 + (j & 1) * 2 * kBlk;
       const uint32_t t_out = ta + T_OUT + (j & 1) * 128;
       mbar_wait(&barE[j & 1], (uint32_t)((j >> 1) & 1), status, abort_flag);
+      // LN2 statistics per half of the row: shifted sums (shift = the half's
+      // first value) of 64 values, accumulated in column order.  This half's
+      // come from the registers that form Y; the other half's are read back
+      // from TMEM below, in the same order, so both threads of a row compute
+      // bitwise the same two halves and the same merge.
+      float K = 0.f, s1 = 0.f, s2 = 0.f;
 #pragma unroll
       for (int p2 = 0; p2 < 2; ++p2) {
         float y[32];
@@ -1388,6 +1429,13 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
 #pragma unroll
           for (int i = 0; i < 8; ++i) y[q * 8 + i] += e[i];
         }
+        if (p2 == 0) K = y[0];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float t = y[i] - K;
+          s1 += t;
+          s2 = fmaf(t, t, s2);
+        }
         tmem_st16(t_out + c0 + p2 * 32, y);
         tmem_st16(t_out + c0 + p2 * 32 + 16, y + 16);
       }
@@ -1395,25 +1443,29 @@ __global__ void __launch_bounds__(kFfnEpi + 64, 1)
       tc_fence_before();
       named_bar_sync(1, kFfnGrp);   // both halves of every row are in OUT (and E is read)
       tc_fence_after();
-      // statistics over all 128 columns, read back from TMEM in column order
-      float K = 0.f, s1 = 0.f, s2 = 0.f;
+      float Ko = 0.f, o1 = 0.f, o2 = 0.f;
 #pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 2; ++q) {
         float o[32];
-        tmem_ld16(t_out + q * 32, o);
-        tmem_ld16(t_out + q * 32 + 16, o + 16);
+        tmem_ld16(t_out + (c0 ^ 64) + q * 32, o);
+        tmem_ld16(t_out + (c0 ^ 64) + q * 32 + 16, o + 16);
         tmem_ld_wait();
-        if (q == 0) K = o[0];
+        if (q == 0) Ko = o[0];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float t = o[i] - K;
-          s1 += t;
-          s2 = fmaf(t, t, s2);
+          const float t = o[i] - Ko;
+          o1 += t;
+          o2 = fmaf(t, t, o2);
         }
       }
-      const float ms = s1 * (1.0f / kD);
-      const float mu = K + ms;
-      const float rstd = rsqrtf(fmaxf(s2 * (1.0f / kD) - ms * ms, 0.f) + kLnEps);
+      // each half's mean and centred sum of squares, merged for equal counts
+      // (M2 = M2a + M2b + 128 ((ma - mb) / 2)^2; symmetric in the halves)
+      const float ma = K + s1 * (1.0f / 64), mb = Ko + o1 * (1.0f / 64);
+      const float qa = fmaxf(s2 - s1 * s1 * (1.0f / 64), 0.f);
+      const float qb = fmaxf(o2 - o1 * o1 * (1.0f / 64), 0.f);
+      const float mu = 0.5f * (ma + mb);
+      const float dh = 0.5f * (ma - mb);
+      const float rstd = rsqrtf((qa + qb + 128.0f * dh * dh) * (1.0f / kD) + kLnEps);
       // h2 of this thread's 64 columns, 16 at a time from TMEM
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
@@ -2387,7 +2439,7 @@ int run_layer(const lime_dims& D, int64_t B, const int64_t* off, int64_t nh, con
   const int64_t tiles_hi = Lw.max_tiles;
   const int grid = (int)(tiles_hi < sms ? tiles_hi : sms);
   auto ffn = [&]() {
-    return launch_pdl(k_hist_ffn, dim3(grid), dim3(kFfnEpi + 64), kFfnSmem, st, 1, tmE_ffn,
+    return launch_pdl(k_hist_ffn, dim3(grid), dim3(kFfnEpi + 96), kFfnSmem, st, 1, tmE_ffn,
                       (const bf16*)w.g2, (const bf16*)w.b2, (const uint8_t*)ws, Lw,
                       (bf16*)E_out, status);
   };

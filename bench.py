@@ -45,10 +45,13 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# the committed ncu captures under profiles/, keyed by what the roofline
-# reports; an entry is removed when its kernel changes.
-NCU_TRAFFIC = {}
+# DRAM traffic per launch in bytes (dram__bytes_read.sum +
+# dram__bytes_write.sum, summed over the launch's kernels) from the committed
+# ncu captures under profiles/, keyed by what the roofline reports and by
+# workload; an entry is removed when its kernels change.
+#   layer: the first lime_xor_layer call of the ragged workload at l = 32
+#          (profiles/layer_traffic_ragged.md)
+NCU_TRAFFIC = {("layer", "ragged_l32"): 885_460_000}
 
 METRIC = "user-candidate pairs scored/s (online LIME step: context links, LIME-XOR layers, cached scoring)"
 
@@ -706,7 +709,7 @@ def main():
         roof = {"bound": "tensor", "achieved": r4(lf / (layer_ms * 1e-3) / 1e12),
                 "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": r4(lf / (layer_ms * 1e-3) / 1e12 / pk["bf16_tflops"]),
-                "traffic": NCU_TRAFFIC.get("layer"),
+                "traffic": NCU_TRAFFIC.get(("layer", args.workload)),
                 "kernel": "lime_xor_layer (one non-final layer, all its kernels)",
                 "launch_ms": r4(layer_ms), "algorithmic_flops_per_launch": lf,
                 "peak_source": pk["source"] + " bf16 burst"}

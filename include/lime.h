@@ -227,6 +227,9 @@ int lime_context_links(const lime_dims* dims, int64_t B, const void* L,
  *   workspace, workspace_bytes: at least lime_workspace_bytes(dims, B,
  *          total_hist) bytes (ERR_ARG when smaller).
  * No output may overlap an input or the other output (ERR_ALIAS).
+ * E_in, E_out, Z_in, Z_out and every weight pointer must be 16-byte aligned
+ * and hist_offsets 8-byte aligned (ERR_ARG otherwise): the tensor-core path
+ * moves them by TMA and 16-byte vector accesses.
  * A user with no history gets a zero link-branch attention output.
  * Streams: on the bf16 tensor-core path a non-final layer runs its link-row
  * tail on a library-owned side stream (the device's highest priority),

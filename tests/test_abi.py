@@ -80,6 +80,10 @@ def test_host_validation_of_layer_calls(lime):
     assert _call_layer(lime, dims, weights=0x60008) == lime.LIME_ERR_ARG       # unaligned
     assert _call_layer(lime, dims, ws=0x100010) == lime.LIME_ERR_ARG           # ws unaligned
     assert _call_layer(lime, dims, ws_bytes=512) == lime.LIME_ERR_ARG          # ws too small
+    assert _call_layer(lime, dims, E_in=0x10008) == lime.LIME_ERR_ARG          # E_in unaligned
+    assert _call_layer(lime, dims, E_out=0x30008) == lime.LIME_ERR_ARG         # E_out unaligned
+    assert _call_layer(lime, dims, Z_out=0x40008) == lime.LIME_ERR_ARG         # Z_out unaligned
+    assert _call_layer(lime, dims, offs=0x50004) == lime.LIME_ERR_ARG          # offsets unaligned
     assert _call_layer(lime, dims, E_out=0x10000) == lime.LIME_ERR_ALIAS       # E_out == E_in
     assert _call_layer(lime, dims, Z_out=0x20000 + 64) == lime.LIME_ERR_ALIAS  # overlap
     bad = lime.make_dims(128, 4, 129, 256, 64, "bf16")

@@ -369,6 +369,7 @@ WINDOW = {
     "standard": dict(B=3, n_items=50_000, window=16),
     "standard_silu": dict(B=3, n_items=50_000, window=16, phi="silu"),
     "ragged16": dict(B=4, l=16, n_items=50_000, window=8),
+    "ragged64": dict(B=3, l=64, n_items=50_000, window=32),
 }
 
 

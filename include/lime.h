@@ -192,13 +192,22 @@ int lime_score_candidates_uncached(const lime_dims* dims, int64_t B, const void*
  *   - The scratch a call needs is lime_workspace_bytes(dims, 0, 0); when that
  *     exceeds LIME_NOALLOC_SCRATCH_BYTES the call returns LIME_ERR_SCRATCH
  *     (use lime_build_qk_cache with a workspace instead).
- *   - Device-side status flags of these calls are not reported.
+ *   - Device-side status flags of these calls (LIME_FLAG_TIMEOUT when a
+ *     bounded wait gave up and the cache may be partly written) are kept in
+ *     the array's status word and read by lime_noalloc_get_status.
  * Calls no cudaMalloc, cudaFree or allocating library routine.            */
 #define LIME_NOALLOC_SCRATCH_BYTES (1u << 20)
 enum { LIME_ERR_SCRATCH = -5 /* scratch need above LIME_NOALLOC_SCRATCH_BYTES */ };
 int lime_build_qk_cache_noalloc(const lime_dims* dims, const void* T, int64_t n_items,
                                 const void* L, const void* Wq_c, const void* Wk_c,
                                 void* cache_out, cudaStream_t stream);
+
+/* The status word of lime_build_qk_cache_noalloc's static array on the
+ * current device: synchronises `stream`, copies the sticky LIME_FLAG_* word
+ * to *flags and clears it (as lime_get_status does for a workspace).
+ * Allocation-free.  ERR_ARG for a null `flags` or while `stream` is being
+ * captured.                                                               */
+int lime_noalloc_get_status(cudaStream_t stream, int* flags);
 
 /* Context links: LC[u, k, :] = SiLU([L_k ; ctx_u] Wc1 + bc1) Wc2 + bc2.
  * LIME note 整体框架 (L^C = MLP(L ⊕ E^C)) and 一个完整示例 step 2.

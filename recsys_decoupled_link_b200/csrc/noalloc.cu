@@ -89,3 +89,18 @@ extern "C" int lime_build_qk_cache_noalloc(const lime_dims* dims, const void* T,
   return lime_build_qk_cache(dims, T, n_items, L, Wq_c, Wk_c, cache_out, scratch,
                              LIME_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+// The status word of the static array (device-side flags of the last
+// lime_build_qk_cache_noalloc call on this device: LIME_FLAG_TIMEOUT when a
+// bounded wait gave up and the cache may be partly written), read and cleared
+// like lime_get_status reads a workspace's.  Allocation-free; not callable
+// while `stream` is capturing (the read synchronises).
+extern "C" int lime_noalloc_get_status(cudaStream_t stream, int* flags) {
+  if (!flags) return LIME_ERR_ARG;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return LIME_ERR_CUDA;
+  if (cs != cudaStreamCaptureStatusNone) return LIME_ERR_ARG;
+  void* scratch = scratch_address(stream);
+  if (!scratch) return LIME_ERR_CUDA;
+  return lime_get_status(scratch, stream, flags);
+}

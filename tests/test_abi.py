@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
         "lime_workspace_bytes", "lime_workspace_init", "lime_build_qk_cache",
         "lime_context_links", "lime_xor_layer", "lime_score_candidates", "lime_get_status",
-        "lime_launch_count", "lime_build_qk_cache_noalloc", "lime_build_qk_cache_u8",
+        "lime_launch_count", "lime_build_qk_cache_noalloc", "lime_noalloc_get_status",
+        "lime_build_qk_cache_u8",
         "lime_score_candidates_u8", "lime_qk_image_bytes", "lime_fold_qk",
         "lime_build_qk_cache_folded", "lime_score_candidates_uncached"])
 
@@ -169,6 +170,10 @@ def test_phi_validation(lime):
     g = lime._lib.lime_build_qk_cache_u8
     assert g(ctypes.byref(d), 0x100000, 10, 0x200000, 0x300000, 0x400000, 0x500000,
              0x1000000, nws, None) == lime.LIME_ERR_SHAPE
+
+
+def test_noalloc_status_reader_checks_its_argument(lime):
+    assert lime._lib.lime_noalloc_get_status(None, None) == lime.LIME_ERR_ARG
 
 
 def test_noalloc_checks_arguments_like_the_workspace_call(lime):

@@ -50,6 +50,7 @@ def test_noalloc_cache_matches_workspace_entry_point(case):
         assert rc == lime.LIME_OK
         torch.cuda.synchronize()
         assert lime.lime_get_status(ws) == 0
+        assert lime.lime_noalloc_get_status() == 0   # the array's status word: no timeout
         assert torch.equal(got, ref), f"no-alloc cache, call {call + 1}"
 
 

@@ -812,6 +812,13 @@ __global__ void __launch_bounds__(kXaThreads, 1)
         if (tn < n_tiles) {
           load_e(sB, tiles[tn].y);
           if (HIST) load(&bar[3], sG, uimg(un, hn));
+          // the E tile after that into L2: its load is issued only once this
+          // slot frees again, and would otherwise come from DRAM
+          const int tp = tn + (int)gridDim.x;
+          if (hf + 1 == NH && tp < n_tiles) {
+            tma_prefetch_2d(&tmE, 0, tiles[tp].y);
+            tma_prefetch_2d(&tmE, 64, tiles[tp].y);
+          }
         }
         if (HIST) {
           mbar_wait(&bar[13], ph, status, c.abort_flag);
@@ -1290,6 +1297,12 @@ __global__ void __launch_bounds__(kFfnEpi + 96, 1)
         // buffer k%2 held h2(k) and then tile k's E' staging
         if (!mbar_wait(barSE, k & 1, status, abort_flag)) break;
         load_e(k + 2);
+        // E(k+3) into L2: its load waits for the next readout
+        if (k + 3 < my_tiles) {
+          const int4 tp = tile_of(k + 3);
+          tma_prefetch_2d(&tmE, 0, tp.y);
+          tma_prefetch_2d(&tmE, 64, tp.y);
+        }
       }
     }
   } else if (warp == kFfnEpi / 32 + 1) {

@@ -5,7 +5,9 @@
 Phases: ``cache`` (QK-cache build over the catalogue), ``score`` (cached
 scoring; the cache is built once first), ``score_scale`` (cached scoring of
 16 users x 65,536 candidate IDs drawn uniformly from the whole catalogue, so
-the gathered rows far exceed L2), ``layer`` (one LIME-XOR layer, the
+the gathered rows far exceed L2), ``uncached_scale`` (the same candidates
+scored without the cache: weights computed per candidate from the item rows
+and the folded image), ``layer`` (one LIME-XOR layer, the
 first of the stack, with history outputs), ``last`` (the last-layer variant
 without history outputs), ``step`` (the whole pass), ``online`` (the online
 step: context links, the layer stack and cached scoring against a cache built
@@ -23,7 +25,9 @@ from . import lime, pipeline, synth
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--phase", default="cache", choices=["cache", "score", "score_scale", "layer", "last", "step", "online"])
+    ap.add_argument("--phase", default="cache", choices=["cache", "score", "score_scale",
+                                                          "uncached_scale", "layer", "last",
+                                                          "step", "online"])
     ap.add_argument("--workload", default="standard")
     ap.add_argument("--items", type=int, default=None)
     ap.add_argument("--users", type=int, default=None)
@@ -51,7 +55,9 @@ def main():
         Z = x.Z0
     if a.phase in ("score", "score_scale", "online"):
         pipeline.build_cache(x, buf)
-    if a.phase == "score_scale":
+    if a.phase == "uncached_scale":
+        lime.lime_fold_qk(x.dims, x.L, x.Wq_c, x.Wk_c, buf.image)
+    if a.phase in ("score_scale", "uncached_scale"):
         users, per = 16, 65536
         g = torch.Generator().manual_seed(4242)
         sc_ids = torch.randint(0, w.n_items, (users * per,), generator=g).to(torch.int32).cuda()
@@ -66,6 +72,9 @@ def main():
         elif a.phase == "score_scale":
             lime.lime_score_candidates(x.dims, buf.cache, sc_ids, sc_off, users * per, sc_LP,
                                        sc_O, buf.ws)
+        elif a.phase == "uncached_scale":
+            lime.lime_score_candidates_uncached(x.dims, x.T, buf.image, sc_ids, sc_off,
+                                                users * per, sc_LP, sc_O, buf.ws)
         elif a.phase == "layer":
             lime.lime_xor_layer(x.dims, x.hist_offsets, x.total_hist, x.E, Z, x.layers[0],
                                 buf.E_bufs[0], buf.Z_bufs[0], buf.ws)

@@ -296,6 +296,13 @@ int lime_score_candidates_u8(const lime_dims* dims, int64_t B, const uint8_t* ca
                              const void* LP, void* O_out, void* workspace,
                              size_t workspace_bytes, cudaStream_t stream);
 
+/* Test hook for the failure detection: runs one kernel whose bounded
+ * device-side wait nothing completes.  After the wait's time limit (about
+ * two seconds) it sets LIME_FLAG_TIMEOUT in the workspace's status word and
+ * returns; the context stays usable.  workspace: initialised, 256-byte
+ * aligned (ERR_ARG otherwise).                                            */
+int lime_debug_wait_timeout(void* workspace, cudaStream_t stream);
+
 /* Synchronises stream, copies the sticky LIME_FLAG_* word to *flags and
  * clears it. */
 int lime_get_status(void* workspace, cudaStream_t stream, int* flags);

@@ -68,6 +68,7 @@ def _load() -> ctypes.CDLL:
         "lime_launch_count": (ctypes.c_uint64, []),
         "lime_build_qk_cache_noalloc": (I32, [D, P, I64, P, P, P, P, P]),
         "lime_noalloc_get_status": (I32, [P, P]),
+        "lime_debug_wait_timeout": (I32, [P, P]),
         "lime_build_qk_cache_u8": (I32, [D, P, I64, P, P, P, P, P, SZ, P]),
         "lime_score_candidates_u8": (I32, [D, I64, P, I64, P, P, I64, P, P, P, SZ, P]),
         "lime_qk_image_bytes": (SZ, [D]),
@@ -85,7 +86,7 @@ _lib = _load()
 EXPORTED = ("lime_workspace_bytes", "lime_workspace_init", "lime_build_qk_cache",
             "lime_context_links", "lime_xor_layer", "lime_score_candidates",
             "lime_get_status", "lime_launch_count", "lime_build_qk_cache_noalloc",
-            "lime_noalloc_get_status",
+            "lime_noalloc_get_status", "lime_debug_wait_timeout",
             "lime_build_qk_cache_u8", "lime_score_candidates_u8", "lime_qk_image_bytes",
             "lime_fold_qk", "lime_build_qk_cache_folded", "lime_score_candidates_uncached")
 
@@ -205,6 +206,11 @@ def lime_build_qk_cache_noalloc(dims, T, L, Wq_c, Wk_c, cache_out, stream=None):
     _check("lime_build_qk_cache_noalloc", _lib.lime_build_qk_cache_noalloc(
         ctypes.byref(dims), _ptr(T), n_items, _ptr(L), _ptr(Wq_c), _ptr(Wk_c),
         _ptr(cache_out), _stream(stream)))
+
+
+def lime_debug_wait_timeout(ws: Workspace, stream=None):
+    """Runs a kernel whose bounded wait runs out (a failure-detection test hook)."""
+    _check("lime_debug_wait_timeout", _lib.lime_debug_wait_timeout(ws.ptr, _stream(stream)))
 
 
 def lime_noalloc_get_status(stream=None) -> int:

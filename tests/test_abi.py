@@ -31,6 +31,7 @@ def test_header_declares_the_boundary():
         "lime_workspace_bytes", "lime_workspace_init", "lime_build_qk_cache",
         "lime_context_links", "lime_xor_layer", "lime_score_candidates", "lime_get_status",
         "lime_launch_count", "lime_build_qk_cache_noalloc", "lime_noalloc_get_status",
+        "lime_debug_wait_timeout",
         "lime_build_qk_cache_u8",
         "lime_score_candidates_u8", "lime_qk_image_bytes", "lime_fold_qk",
         "lime_build_qk_cache_folded", "lime_score_candidates_uncached"])
@@ -174,6 +175,11 @@ def test_phi_validation(lime):
 
 def test_noalloc_status_reader_checks_its_argument(lime):
     assert lime._lib.lime_noalloc_get_status(None, None) == lime.LIME_ERR_ARG
+
+
+def test_wait_timeout_hook_checks_its_argument(lime):
+    assert lime._lib.lime_debug_wait_timeout(None, None) == lime.LIME_ERR_ARG
+    assert lime._lib.lime_debug_wait_timeout(0x100010, None) == lime.LIME_ERR_ARG
 
 
 def test_noalloc_checks_arguments_like_the_workspace_call(lime):
